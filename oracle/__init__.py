@@ -1,0 +1,187 @@
+"""fp64 CPU oracle of the Vision Mamba / VMamba selective scan.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The CUDA library never
+calls it, and it never calls the CUDA library.
+
+Every function converts its inputs to contiguous float64 arrays (bf16 and fp32
+values are represented exactly), runs the plain sequential recurrence of
+``oracle.c`` and returns float64 numpy arrays.  The equations followed are those of
+the page "Vision Mamba Guide: Efficient Bidirectional SSM & VMamba": sections
+"Discretization via Zero-Order Hold (ZOH)", "The Selective State Space (S6)
+Mechanism", "2. The Bidirectional Mamba Block", "1. Cross-Scan Traversal
+(CS-Traverse)" and "3. Cross-Merge Reversal (CS-Merge)".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I64 = ctypes.POINTER(ctypes.c_int64)
+
+
+def _f64(x):
+    """Contiguous float64 copy of a numpy array or a (CPU or CUDA) torch tensor."""
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor
+        import torch
+
+        x = x.detach().to("cpu", torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(_D)
+
+
+class Oracle:
+    """ctypes view of one build of ``oracle.c``.
+
+    The module-level functions use the default build next to this file; the test
+    suite also loads deliberately broken copies (built in a temporary directory)
+    to show that the pins catch a planted mistake.
+    """
+
+    def __init__(self, path: str):
+        lib = ctypes.CDLL(path)
+        lib.oracle_s6_direction.argtypes = [_D, _D, _D, _D, _D, _D, _D, _I64, _D] + [ctypes.c_int] * 6
+        lib.oracle_vim_bidir.argtypes = [_D, _D, _D, _D, _D, ctypes.c_int64, _D, _D, _D, _D] + [ctypes.c_int] * 5
+        lib.oracle_cross_scan4.argtypes = [_D] * 9 + [ctypes.c_int] * 6
+        lib.oracle_cross_merge4.argtypes = [_D, _D, _D] + [ctypes.c_int] * 4
+        lib.oracle_cross_order.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _I64]
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_max_threads.restype = ctypes.c_int
+        self.lib = lib
+        self.path = path
+
+    def set_threads(self, n: int) -> None:
+        """Number of OpenMP threads (parallel over independent sequences only)."""
+        self.lib.oracle_set_threads(int(n))
+
+    def max_threads(self) -> int:
+        return int(self.lib.oracle_max_threads())
+
+    def cross_order(self, k: int, H: int, W: int) -> np.ndarray:
+        """Grid position (p = h*W + w) visited at each step of CS-Traverse scan k+1."""
+        out = np.zeros(H * W, dtype=np.int64)
+        if self.lib.oracle_cross_order(int(k), int(H), int(W), out.ctypes.data_as(_I64)):
+            raise ValueError("bad direction index")
+        return out
+
+    def s6_direction(self, u, delta, B, C, A, D, bias, order, *, delta_is_raw=True):
+        """One S6 direction (no gate) over tokens visited in ``order``.
+
+        u, delta: [batch, L, Di]; B, C: [batch, L, N] (by position); A: [Di, N];
+        D, bias: [Di]; order: [L] permutation.  Returns y [batch, L, Di] with
+        y[b, order[t], d] = C_t . h_t + D u_t.
+        """
+        u, delta, B, C, A, D, bias = map(_f64, (u, delta, B, C, A, D, bias))
+        batch, L, Di = u.shape
+        N = B.shape[-1]
+        order = np.ascontiguousarray(np.asarray(order, dtype=np.int64))
+        assert sorted(order.tolist()) == list(range(L)), "order must be a permutation"
+        if bias is None:
+            bias = np.zeros(Di)
+        y = np.zeros((batch, L, Di))
+        rc = self.lib.oracle_s6_direction(_p(u), _p(delta), _p(B), _p(C), _p(A), _p(D), _p(bias),
+                                          order.ctypes.data_as(_I64), _p(y),
+                                          batch, L, Di, N, int(bool(delta_is_raw)), 0)
+        if rc:
+            raise ValueError("oracle_s6_direction: bad sizes")
+        return y
+
+    def vim_bidir(self, u, delta, z, B, C, A, D, bias, *, bc_dir_stride=0, delta_is_raw=True):
+        """Vim bidirectional scan: (y^f + y^b) * silu(z); z=None gives the ungated sum.
+
+        u, delta, z: [batch, L, Di]; B, C: [batch, L, N] shared by both directions,
+        or a larger buffer whose backward copy starts ``bc_dir_stride`` elements in;
+        A: [2, Di, N]; D, bias: [2, Di].
+        """
+        u, delta, z, B, C, A, D, bias = map(_f64, (u, delta, z, B, C, A, D, bias))
+        batch, L, Di = u.shape
+        N = B.shape[-1]
+        if bias is None:
+            bias = np.zeros((2, Di))
+        y = np.zeros((batch, L, Di))
+        rc = self.lib.oracle_vim_bidir(_p(u), _p(delta), _p(z), _p(B), _p(C), int(bc_dir_stride),
+                                       _p(A), _p(D), _p(bias), _p(y), batch, L, Di, N,
+                                       int(bool(delta_is_raw)))
+        if rc:
+            raise ValueError("oracle_vim_bidir: bad sizes")
+        return y
+
+    def cross_scan4(self, u, delta, z, B, C, A, D, bias, *, delta_is_raw=True):
+        """VMamba four-direction scan with CS-Merge: (sum_k y_k) * silu(z).
+
+        u, delta, z: [batch, H, W, Ci]; B, C: [4, batch, H*W, N] in grid order;
+        A: [4, Ci, N]; D, bias: [4, Ci].
+        """
+        u, delta, z, B, C, A, D, bias = map(_f64, (u, delta, z, B, C, A, D, bias))
+        batch, H, W, Ci = u.shape
+        N = B.shape[-1]
+        if bias is None:
+            bias = np.zeros((4, Ci))
+        y = np.zeros((batch, H, W, Ci))
+        rc = self.lib.oracle_cross_scan4(_p(u), _p(delta), _p(z), _p(B), _p(C), _p(A), _p(D),
+                                         _p(bias), _p(y), batch, H, W, Ci, N, int(bool(delta_is_raw)))
+        if rc:
+            raise ValueError("oracle_cross_scan4: bad sizes")
+        return y
+
+    def cross_merge4(self, ys, z, H, W):
+        """CS-Merge alone: ys [4, batch, H*W, Ci] in scan order -> [batch, H, W, Ci]."""
+        ys, z = _f64(ys), _f64(z)
+        _, batch, L, Ci = ys.shape
+        assert L == H * W
+        y = np.zeros((batch, H, W, Ci))
+        rc = self.lib.oracle_cross_merge4(_p(ys), _p(z), _p(y), batch, H, W, Ci)
+        if rc:
+            raise ValueError("oracle_cross_merge4: bad sizes")
+        return y
+
+
+_default = None
+
+
+def default() -> Oracle:
+    """The oracle built from ``oracle.c`` next to this file (built on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle(_build.build())
+    return _default
+
+
+def set_threads(n):
+    default().set_threads(n)
+
+
+def max_threads():
+    return default().max_threads()
+
+
+def cross_order(k, H, W):
+    return default().cross_order(k, H, W)
+
+
+def s6_direction(*a, **k):
+    return default().s6_direction(*a, **k)
+
+
+def vim_bidir(*a, **k):
+    return default().vim_bidir(*a, **k)
+
+
+def cross_scan4(*a, **k):
+    return default().cross_scan4(*a, **k)
+
+
+def cross_merge4(*a, **k):
+    return default().cross_merge4(*a, **k)

@@ -1,0 +1,235 @@
+/*
+ * oracle.c -- plain sequential fp64 reference of the selective scan (S6) used by
+ * Vision Mamba (bidirectional scan) and VMamba (four-direction cross-scan).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or call
+ * this file; only the test suite, the smoke check and the CPU-baseline leg of the
+ * benchmark do.  It shares no code with the CUDA library.
+ *
+ * What it computes is written straight from the equations of the page
+ * "Vision Mamba Guide: Efficient Bidirectional SSM & VMamba" (aifetchly-blog):
+ *   - ZOH discretisation, section "Discretization via Zero-Order Hold (ZOH)":
+ *       Abar = exp(Delta*A),  Bbar ~= Delta*B  (the approximate form is used);
+ *   - recurrence and readout, same section and section "Continuous-Time State
+ *     Space Equations":  h_t = Abar h_{t-1} + Bbar x_t,  y_t = C h_t + D x_t;
+ *   - selectivity, section "The Selective State Space (S6) Mechanism":
+ *       Delta_t = softplus(...) (here softplus(delta_raw + delta_bias));
+ *   - bidirectional pathways and the gated fusion, section "2. The Bidirectional
+ *     Mamba Block": forward pass over tokens 1..N+1, backward pass from N+1 down to
+ *     1, Y = y^f * silu(z) + y^b * silu(z) (the output projection is not part of it);
+ *   - the four traversal orders and the merge, sections "1. Cross-Scan Traversal
+ *     (CS-Traverse)" and "3. Cross-Merge Reversal (CS-Merge)".
+ *
+ * Readings where the page is silent (the same list is kept with the design notes):
+ *   softplus(x) = log1p(exp(x)), taken as x itself for x > 20;  h starts at 0 for
+ *   every direction;  the D*u skip is added once per direction;  per-direction B/C
+ *   of the cross-scan are stored in grid order (direction k reads them at the grid
+ *   position it visits);  silu(z) = z / (1 + exp(-z)).
+ *
+ * Everything is double precision and strictly sequential along each scan; the
+ * only parallelism is over independent (batch, channel) pairs.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_MAX_STATE 256
+
+/* "Delta_t = Softplus(Linear_Delta(x_t))" -- S6 mechanism section. */
+static double softplus(double x) { return x > 20.0 ? x : log1p(exp(x)); }
+
+/* sigma(z) in the gated fusion is the SiLU activation (Bidirectional Mamba Block). */
+static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+void oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * The four CS-Traverse orders on an H x W grid whose positions are numbered
+ * p = h*W + w (row-major, "Top-Left (0,0)" first).  Writes order[t] = grid
+ * position visited at scan step t, for t = 0..H*W-1.
+ *   k = 0  Scan 1, rows from (0,0) to (H-1,W-1)
+ *   k = 1  Scan 2, the reverse of scan 1
+ *   k = 2  Scan 3, columns from (0,0) down to (H-1,W-1): step t = w*H + h
+ *   k = 3  Scan 4, the reverse of scan 3
+ * Returns 0, or -1 for a bad direction index.
+ */
+int oracle_cross_order(int k, int H, int W, int64_t *order)
+{
+    int64_t L = (int64_t)H * W;
+    for (int64_t t = 0; t < L; ++t) {
+        int64_t s = (k == 1 || k == 3) ? (L - 1 - t) : t;
+        int64_t p;
+        if (k == 0 || k == 1) {
+            p = s;
+        } else if (k == 2 || k == 3) {
+            int64_t h = s % H, w = s / H;
+            p = h * W + w;
+        } else {
+            return -1;
+        }
+        order[t] = p;
+    }
+    return 0;
+}
+
+/*
+ * One S6 direction over every (batch, channel) sequence.
+ *   u, delta : [batch, L, Di]          input and Delta (raw or final, see below)
+ *   B, C     : [batch, L, N]           indexed by token position
+ *   A        : [Di, N], D, bias : [Di]
+ *   order    : [L] positions in visiting order (a permutation of 0..L-1)
+ *   y        : [batch, L, Di]          y[b, order[t], d] receives the readout of step t;
+ *                                      added to the existing value if accumulate != 0
+ *   delta_is_raw != 0 : Delta = softplus(delta + bias[d]); otherwise Delta = delta
+ *                       as given and bias is ignored.
+ * Returns 0, or -1 on bad sizes.
+ */
+int oracle_s6_direction(const double *u, const double *delta, const double *B, const double *C,
+                        const double *A, const double *D, const double *bias,
+                        const int64_t *order, double *y,
+                        int batch, int L, int Di, int N, int delta_is_raw, int accumulate)
+{
+    if (batch < 0 || L < 0 || Di < 0 || N < 1 || N > ORACLE_MAX_STATE) return -1;
+    int64_t pairs = (int64_t)batch * Di;
+    #pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t bd = 0; bd < pairs; ++bd) {
+        int64_t b = bd / Di, d = bd % Di;
+        double h[ORACLE_MAX_STATE];
+        for (int n = 0; n < N; ++n) h[n] = 0.0;                 /* h_0 = 0 */
+        for (int64_t t = 0; t < L; ++t) {
+            int64_t p = order[t];
+            int64_t ix = (b * L + p) * Di + d;                    /* [b, p, d] */
+            const double *Bt = B + (b * L + p) * N;               /* [b, p, :] */
+            const double *Ct = C + (b * L + p) * N;
+            double dt = delta_is_raw ? softplus(delta[ix] + bias[d]) : delta[ix];
+            double x = u[ix];
+            double yt = 0.0;
+            for (int n = 0; n < N; ++n) {
+                double Abar = exp(dt * A[d * N + n]);             /* Abar = exp(Delta A) */
+                double Bbar = dt * Bt[n];                         /* Bbar ~= Delta B     */
+                h[n] = Abar * h[n] + Bbar * x;                    /* h_t = Abar h + Bbar x */
+                yt += Ct[n] * h[n];                               /* C h_t               */
+            }
+            yt += D[d] * x;                                       /* + D x_t             */
+            if (accumulate) y[ix] += yt; else y[ix] = yt;
+        }
+    }
+    return 0;
+}
+
+/* y <- y * silu(z), elementwise over n values (skipped when z is NULL). */
+static void apply_gate(double *y, const double *z, int64_t n)
+{
+    if (!z) return;
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) y[i] *= silu(z[i]);
+}
+
+/*
+ * Vim bidirectional S6 with gated fusion.
+ *   u, delta, z : [batch, L, Di];  z may be NULL (no gate)
+ *   B, C        : [batch, L, N]; the backward direction reads B + bc_dir_stride and
+ *                 C + bc_dir_stride (0 = both directions share B and C)
+ *   A [2, Di, N], D [2, Di], bias [2, Di]: index 0 = forward, 1 = backward
+ *   y           : [batch, L, Di] = (y^f + y^b) * silu(z)
+ */
+int oracle_vim_bidir(const double *u, const double *delta, const double *z,
+                     const double *B, const double *C, int64_t bc_dir_stride,
+                     const double *A, const double *D, const double *bias,
+                     double *y, int batch, int L, int Di, int N, int delta_is_raw)
+{
+    if (L < 0) return -1;
+    int64_t *order = (int64_t *)calloc((size_t)(L > 0 ? L : 1), sizeof(int64_t));
+    if (!order) return -1;
+    int rc = 0;
+    for (int64_t t = 0; t < L; ++t) order[t] = t;                 /* forward: 1 .. N+1 */
+    rc |= oracle_s6_direction(u, delta, B, C, A, D, bias, order, y,
+                              batch, L, Di, N, delta_is_raw, 0);
+    for (int64_t t = 0; t < L; ++t) order[t] = L - 1 - t;         /* backward: N+1 .. 1 */
+    rc |= oracle_s6_direction(u, delta, B + bc_dir_stride, C + bc_dir_stride,
+                              A + (int64_t)Di * N, D + Di, bias + Di, order, y,
+                              batch, L, Di, N, delta_is_raw, 1);
+    free(order);
+    if (rc) return -1;
+    apply_gate(y, z, (int64_t)batch * L * Di);
+    return 0;
+}
+
+/*
+ * VMamba SS2D: four independent S6 over the CS-Traverse orders, CS-Merge by sum.
+ *   u, delta, z : [batch, H, W, Ci] (grid positions p = h*W + w);  z may be NULL
+ *   B, C        : [4, batch, H*W, N], grid order (direction k reads B[k, b, p, :])
+ *   A [4, Ci, N], D [4, Ci], bias [4, Ci]
+ *   y           : [batch, H, W, Ci] = (y_1 + y_2 + y_3 + y_4) * silu(z)
+ */
+int oracle_cross_scan4(const double *u, const double *delta, const double *z,
+                       const double *B, const double *C,
+                       const double *A, const double *D, const double *bias,
+                       double *y, int batch, int H, int W, int Ci, int N, int delta_is_raw)
+{
+    if (H < 0 || W < 0) return -1;
+    int64_t L = (int64_t)H * W;
+    int64_t *order = (int64_t *)calloc((size_t)(L > 0 ? L : 1), sizeof(int64_t));
+    if (!order) return -1;
+    int rc = 0;
+    int64_t bc = (int64_t)batch * L * N;
+    for (int k = 0; k < 4; ++k) {
+        rc |= oracle_cross_order(k, H, W, order);
+        rc |= oracle_s6_direction(u, delta, B + k * bc, C + k * bc,
+                                  A + (int64_t)k * Ci * N, D + (int64_t)k * Ci,
+                                  bias + (int64_t)k * Ci, order, y,
+                                  batch, (int)L, Ci, N, delta_is_raw, k > 0);
+    }
+    free(order);
+    if (rc) return -1;
+    apply_gate(y, z, (int64_t)batch * L * Ci);
+    return 0;
+}
+
+/*
+ * CS-Merge alone: ys [4, batch, H*W, Ci], each direction's outputs in its own
+ * scan order (row t of direction k belongs to grid position order_k[t]).
+ *   y [batch, H, W, Ci] = (sum_k ys_k mapped back to (h, w)) * silu(z)
+ */
+int oracle_cross_merge4(const double *ys, const double *z, double *y,
+                        int batch, int H, int W, int Ci)
+{
+    if (H < 0 || W < 0 || batch < 0 || Ci < 0) return -1;
+    int64_t L = (int64_t)H * W;
+    int64_t *order = (int64_t *)calloc((size_t)(L > 0 ? L : 1), sizeof(int64_t));
+    if (!order) return -1;
+    int64_t total = (int64_t)batch * L * Ci;
+    for (int64_t i = 0; i < total; ++i) y[i] = 0.0;
+    for (int k = 0; k < 4; ++k) {
+        if (oracle_cross_order(k, H, W, order)) { free(order); return -1; }
+        const double *yk = ys + (int64_t)k * total;
+        for (int64_t b = 0; b < batch; ++b)
+            for (int64_t t = 0; t < L; ++t) {
+                int64_t p = order[t];
+                for (int64_t c = 0; c < Ci; ++c)
+                    y[(b * L + p) * Ci + c] += yk[(b * L + t) * Ci + c];
+            }
+    }
+    free(order);
+    apply_gate(y, z, total);
+    return 0;
+}

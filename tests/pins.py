@@ -1,0 +1,328 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Each ``pin_*`` function takes an oracle object (``oracle.Oracle``) and raises
+AssertionError when the oracle disagrees.  ``test_oracle_pins.py`` runs them on the
+oracle as built; ``test_oracle_mutants.py`` runs them on copies of the oracle with a
+planted mistake and requires every copy to fail at least one of them.
+
+The equations cited are those of the page "Vision Mamba Guide: Efficient
+Bidirectional SSM & VMamba" (aifetchly-blog); section names are given per pin.
+"""
+import math
+import os
+
+import numpy as np
+
+import brute
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _vim_case(rng, batch=2, L=7, Di=3, N=4, separate_bc=True):
+    """Random Vim inputs with every parameter different per direction and channel."""
+    u = rng.normal(size=(batch, L, Di))
+    delta = rng.uniform(0.01, 0.6, size=(batch, L, Di))          # post-softplus Delta
+    z = rng.normal(size=(batch, L, Di))
+    nb = 2 if separate_bc else 1
+    B = rng.normal(size=(nb, batch, L, N))
+    C = rng.normal(size=(nb, batch, L, N))
+    A = -rng.uniform(0.2, 3.0, size=(2, Di, N))
+    D = rng.normal(size=(2, Di))
+    bias = rng.normal(size=(2, Di))
+    stride = batch * L * N if separate_bc else 0
+    return dict(u=u, delta=delta, z=z, B=B, C=C, A=A, D=D, bias=bias, stride=stride)
+
+
+def _vim(orc, c, *, gate=True, raw=False, **over):
+    c = {**c, **over}
+    return orc.vim_bidir(c["u"], c["delta"], c["z"] if gate else None, c["B"], c["C"], c["A"], c["D"],
+                         c["bias"], bc_dir_stride=c["stride"], delta_is_raw=raw)
+
+
+def pin_delta_zero(orc):
+    """Delta = 0 gives Abar = 1 and Bbar = 0: h stays at 0, so y = (D_f + D_b) u.
+
+    Sections "Discretization via Zero-Order Hold (ZOH)" and "Continuous-Time State
+    Space Equations" (the D x skip).
+    """
+    c = _vim_case(_rng(1))
+    y = _vim(orc, c, gate=False, delta=np.zeros_like(c["delta"]))
+    expect = (c["D"][0] + c["D"][1])[None, None, :] * c["u"]
+    np.testing.assert_allclose(y, expect, rtol=1e-14, atol=1e-14)
+
+
+def pin_constant_input_geometric(orc):
+    """Constant Delta, u, B and C: h after k steps is the geometric series
+    Delta B u (1 - Abar^k) / (1 - Abar); the forward pass has taken t+1 steps at
+    token t and the backward pass L-t steps.
+
+    Sections "Discretization via Zero-Order Hold (ZOH)" and "2. The Bidirectional
+    Mamba Block" (forward over 1..N+1, backward from N+1 down to 1).
+    """
+    rng = _rng(2)
+    batch, L, Di, N = 1, 23, 3, 5
+    dlt, uu = 0.37, -1.3
+    B = np.broadcast_to(rng.normal(size=(2, 1, 1, N)), (2, batch, L, N)).copy()
+    C = np.broadcast_to(rng.normal(size=(2, 1, 1, N)), (2, batch, L, N)).copy()
+    A = -rng.uniform(0.1, 2.0, size=(2, Di, N))
+    D = rng.normal(size=(2, Di))
+    u = np.full((batch, L, Di), uu)
+    delta = np.full((batch, L, Di), dlt)
+    y = orc.vim_bidir(u, delta, None, B, C, A, D, None, bc_dir_stride=batch * L * N,
+                      delta_is_raw=False)
+    t = np.arange(L)[:, None, None]
+    steps = (t + 1, L - t)
+    expect = np.zeros((L, Di))
+    for k in range(2):
+        abar = np.exp(dlt * A[k])[None]                      # [1, Di, N]
+        geo = -np.expm1(steps[k] * np.log(abar)) / -np.expm1(np.log(abar))
+        h = dlt * B[k, 0, 0][None, None, :] * uu * geo        # [L, Di, N]
+        expect += (h * C[k, 0, 0][None, None, :]).sum(-1) + D[k][None, :] * uu
+    np.testing.assert_allclose(y[0], expect, rtol=1e-12, atol=1e-12)
+
+
+def pin_reverse_symmetry(orc):
+    """Reversing the token sequence and swapping the forward/backward parameters
+    reverses the output: the backward pathway is the forward pathway run on the
+    reversed sequence with its output flipped back (section "2. The Bidirectional
+    Mamba Block").  Checked both for one direction alone and for the gated pair.
+    """
+    rng = _rng(3)
+    c = _vim_case(rng, L=9)
+    # one direction: the reversed order on x equals flip(forward(flip(x)))
+    u, dl, B, C = c["u"], c["delta"], c["B"][0], c["C"][0]
+    L = u.shape[1]
+    rev = np.arange(L)[::-1]
+    yb = orc.s6_direction(u, dl, B, C, c["A"][1], c["D"][1], c["bias"][1], rev, delta_is_raw=True)
+    yf = orc.s6_direction(u[:, ::-1], dl[:, ::-1], B[:, ::-1], C[:, ::-1], c["A"][1], c["D"][1],
+                          c["bias"][1], np.arange(L), delta_is_raw=True)
+    np.testing.assert_allclose(yb, yf[:, ::-1], rtol=1e-13, atol=1e-13)
+    # the whole gated block, raw Delta through the bias
+    y = _vim(orc, c, raw=True)
+    flip = lambda a: a[..., ::-1, :]
+    swapped = dict(u=flip(c["u"]), delta=flip(c["delta"]), z=flip(c["z"]),
+                   B=flip(c["B"][::-1]), C=flip(c["C"][::-1]), A=c["A"][::-1], D=c["D"][::-1],
+                   bias=c["bias"][::-1])
+    y2 = _vim(orc, c, raw=True, **{k: np.ascontiguousarray(v) for k, v in swapped.items()})
+    np.testing.assert_allclose(y, flip(y2), rtol=1e-12, atol=1e-12)
+
+
+def pin_brute_force(orc):
+    """Explicit unrolled sums (tests/brute.py) agree on tiny inputs, L = 1..8."""
+    rng = _rng(4)
+    for L in (1, 2, 3, 5, 8):
+        c = _vim_case(rng, batch=1, L=L, Di=2, N=3)
+        y = _vim(orc, c, gate=False)
+        Bf, Bb = c["B"][0, 0].tolist(), c["B"][1, 0].tolist()
+        Cf, Cb = c["C"][0, 0].tolist(), c["C"][1, 0].tolist()
+        ref = brute.bidir_ungated(c["u"][0].tolist(), c["delta"][0].tolist(), Bf, Cf,
+                                  c["A"].tolist(), c["D"].tolist(), Bb, Cb)
+        np.testing.assert_allclose(y[0], np.array(ref), rtol=1e-12, atol=1e-12)
+
+
+def pin_prefix_sum(orc):
+    """A = 0, N = 1, B = C = 1, D = 0: Abar = 1, so the forward output is the prefix
+    sum of Delta u and the backward output the suffix sum (math.fsum)."""
+    rng = _rng(5)
+    L = 57
+    u = rng.normal(size=(1, L, 1))
+    delta = rng.uniform(0, 1, size=(1, L, 1))
+    ones = np.ones((1, L, 1))
+    y = orc.vim_bidir(u, delta, None, ones, ones, np.zeros((2, 1, 1)), np.zeros((2, 1)), None,
+                      delta_is_raw=False)
+    du = (u * delta)[0, :, 0].tolist()
+    expect = [math.fsum(du[: t + 1]) + math.fsum(du[t:]) for t in range(L)]
+    np.testing.assert_allclose(y[0, :, 0], expect, rtol=1e-13, atol=1e-13)
+
+
+def pin_linearity(orc):
+    """At fixed Delta, B and C the recurrence and readout are linear in u."""
+    rng = _rng(6)
+    c = _vim_case(rng, L=11)
+    u2 = rng.normal(size=c["u"].shape)
+    a, b = 0.7, -1.9
+    y1 = _vim(orc, c, gate=False)
+    y2 = _vim(orc, c, gate=False, u=u2)
+    y12 = _vim(orc, c, gate=False, u=a * c["u"] + b * u2)
+    np.testing.assert_allclose(y12, a * y1 + b * y2, rtol=1e-11, atol=1e-11)
+
+
+def pin_softplus(orc):
+    """Delta = softplus(delta_raw + bias) (section "The Selective State Space (S6)
+    Mechanism").  With L = 1, N = 1, A = 0, B = C = u = 1 and D = 0 each direction
+    outputs its Delta, so one pass reads softplus off.  Checked against properties
+    that fix it: softplus(0) = ln 2, softplus(x) - softplus(-x) = x, softplus(x) ->
+    e^x - e^{2x}/2 for x -> -inf, and softplus(x) = x above the cut at 20.
+    """
+    def sp1(x):
+        ones = np.ones((1, 1, 1))
+        bias = np.array([[x], [-40.0]])                 # backward direction: Delta ~ e^-40
+        y = orc.vim_bidir(ones, ones * 0.0, None, ones, ones, np.zeros((2, 1, 1)),
+                          np.zeros((2, 1)), bias, delta_is_raw=True)
+        return float(y[0, 0, 0]) - math.exp(-40.0)
+
+    assert abs(sp1(0.0) - math.log(2.0)) < 1e-15
+    for x in (0.5, 3.0, 7.25, 15.0):
+        assert abs((sp1(x) - sp1(-x)) - x) < 1e-13 * max(1.0, x)
+    for x in (-12.0, -25.0, -30.0):
+        e = math.exp(x)
+        assert abs(sp1(x) - (e - e * e / 2 + e * e * e / 3)) <= 1e-13 * e
+    assert sp1(25.0) == 25.0 and sp1(21.0) == 21.0
+
+
+def pin_gate_is_silu(orc):
+    """The fused output is multiplied by silu(z) = z * sigmoid(z) (section "2. The
+    Bidirectional Mamba Block").  Pinned by silu(z) - silu(-z) = z: the gated
+    outputs for z and -z differ by z times the ungated output, and silu(0) = 0."""
+    c = _vim_case(_rng(7))
+    y0 = _vim(orc, c, gate=False)
+    yp = _vim(orc, c, gate=True)
+    ym = orc.vim_bidir(c["u"], c["delta"], -c["z"], c["B"], c["C"], c["A"], c["D"], c["bias"],
+                       bc_dir_stride=c["stride"], delta_is_raw=False)
+    np.testing.assert_allclose(yp - ym, c["z"] * y0, rtol=1e-12, atol=1e-12)
+    yz = orc.vim_bidir(c["u"], c["delta"], np.zeros_like(c["z"]), c["B"], c["C"], c["A"], c["D"],
+                       c["bias"], bc_dir_stride=c["stride"], delta_is_raw=False)
+    assert np.all(yz == 0.0)
+    # large |z|: silu(z) -> z, silu(-z) -> 0
+    big = np.full_like(c["z"], 40.0)
+    yb = orc.vim_bidir(c["u"], c["delta"], big, c["B"], c["C"], c["A"], c["D"], c["bias"],
+                       bc_dir_stride=c["stride"], delta_is_raw=False)
+    np.testing.assert_allclose(yb, 40.0 * y0, rtol=1e-15, atol=1e-15)
+
+
+def _golden_orders():
+    rows = []
+    with open(os.path.join(GOLDEN, "cross_scan_orders.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                v = [int(x) for x in line.split()]
+                rows.append((v[0], v[1], v[2], v[3:]))
+    return rows
+
+
+def pin_cross_orders_golden(orc):
+    """The four traversal orders match the hand-written fixture (section "1.
+    Cross-Scan Traversal (CS-Traverse)")."""
+    rows = _golden_orders()
+    assert len(rows) >= 12
+    for H, W, k, order in rows:
+        assert orc.cross_order(k - 1, H, W).tolist() == order, (H, W, k)
+
+
+def _traverse(x):
+    """Explicit CS-Traverse of a channels-last grid x [B, H, W, C] into the four
+    sequences [4, B, H*W, C]: row-major, its reverse, column-major (transpose, then
+    flatten), its reverse."""
+    b, H, W, c = x.shape
+    s1 = x.reshape(b, H * W, c)
+    s3 = x.transpose(0, 2, 1, 3).reshape(b, W * H, c)
+    return np.stack([s1, s1[:, ::-1], s3, s3[:, ::-1]])
+
+
+def _untraverse(ys, H, W):
+    """Inverse of _traverse for one direction each: [4, B, H*W, C] -> 4 grids."""
+    _, b, L, c = ys.shape
+    g1 = ys[0].reshape(b, H, W, c)
+    g2 = ys[1][:, ::-1].reshape(b, H, W, c)
+    g3 = ys[2].reshape(b, W, H, c).transpose(0, 2, 1, 3)
+    g4 = ys[3][:, ::-1].reshape(b, W, H, c).transpose(0, 2, 1, 3)
+    return [g1, g2, g3, g4]
+
+
+def pin_cross_scan_is_transpose_and_flip(orc):
+    """The four-direction scan equals: explicit transpose/flip of the grid into four
+    sequences, four plain forward scans (each with its own parameters and its own
+    B/C, gathered the same way), the inverse maps, the sum and the gate (sections
+    "1. Cross-Scan Traversal", "2. Parallel S6 State Space Processing",
+    "3. Cross-Merge Reversal").  H != W so a transposed index cannot pass."""
+    rng = _rng(8)
+    b, H, W, c, N = 2, 3, 5, 4, 3
+    u = rng.normal(size=(b, H, W, c))
+    dr = rng.normal(size=(b, H, W, c)) * 0.5
+    z = rng.normal(size=(b, H, W, c))
+    B = rng.normal(size=(4, b, H * W, N))
+    C = rng.normal(size=(4, b, H * W, N))
+    A = -rng.uniform(0.1, 2.0, size=(4, c, N))
+    D = rng.normal(size=(4, c))
+    bias = rng.normal(size=(4, c))
+    y = orc.cross_scan4(u, dr, z, B, C, A, D, bias, delta_is_raw=True)
+    seq_u, seq_d = _traverse(u), _traverse(dr)
+    outs = []
+    for k in range(4):
+        Bk = _traverse(B[k].reshape(b, H, W, N))[k]
+        Ck = _traverse(C[k].reshape(b, H, W, N))[k]
+        outs.append(orc.s6_direction(np.ascontiguousarray(seq_u[k]), np.ascontiguousarray(seq_d[k]),
+                                     np.ascontiguousarray(Bk), np.ascontiguousarray(Ck),
+                                     A[k], D[k], bias[k], np.arange(H * W), delta_is_raw=True))
+    grids = _untraverse(np.stack(outs), H, W)
+    gate = orc.cross_scan4(u, dr, None, B, C, A, D, bias, delta_is_raw=True)
+    np.testing.assert_allclose(gate, sum(grids), rtol=1e-12, atol=1e-12)
+    # the gate, through the silu(z) - silu(-z) = z identity
+    ym = orc.cross_scan4(u, dr, -z, B, C, A, D, bias, delta_is_raw=True)
+    np.testing.assert_allclose(y - ym, z * gate, rtol=1e-12, atol=1e-12)
+
+
+def pin_cross_merge(orc):
+    """CS-Merge maps each scan back to (h, w) and sums (section "3. Cross-Merge
+    Reversal"): merging the explicit traversal of a grid gives 4x the grid, and
+    one-hot scans land where the inverse maps say.  Shapes follow the page's
+    verification block: a (2, 64, 16, 16) map traverses to (4, 2, 256, 64) and
+    merges back to (2, 64, 16, 16) (channels last here)."""
+    rng = _rng(9)
+    shapes = {}
+    with open(os.path.join(GOLDEN, "page_shapes.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                k, *v = line.split()
+                shapes[k] = tuple(int(x) for x in v)
+    b, c, H, W = shapes["cross_in_bchw"]
+    x = rng.normal(size=(b, H, W, c))
+    scans = _traverse(x)
+    assert scans.shape == shapes["cross_scans"]
+    merged = orc.cross_merge4(np.ascontiguousarray(scans), None, H, W)
+    assert merged.transpose(0, 3, 1, 2).shape == shapes["cross_merged_bchw"]
+    np.testing.assert_allclose(merged, 4 * x, rtol=1e-14, atol=1e-14)
+    # non-square, per-direction distinct inputs
+    H, W = 2, 3
+    ys = rng.normal(size=(4, 1, H * W, 2))
+    got = orc.cross_merge4(ys, None, H, W)
+    want = sum(_untraverse(ys, H, W))
+    np.testing.assert_allclose(got, want, rtol=1e-14, atol=1e-14)
+    z = rng.normal(size=(1, H, W, 2))
+    gz = orc.cross_merge4(ys, z, H, W)
+    gm = orc.cross_merge4(ys, -z, H, W)
+    np.testing.assert_allclose(gz - gm, z * want, rtol=1e-13, atol=1e-13)
+
+
+def pin_separate_bc(orc):
+    """With bc_dir_stride the backward direction reads its own B and C: running the
+    pair with swapped copies equals the brute force with swapped copies."""
+    rng = _rng(10)
+    c = _vim_case(rng, batch=1, L=4, Di=2, N=2)
+    y = _vim(orc, c, gate=False)
+    ref = brute.bidir_ungated(c["u"][0].tolist(), c["delta"][0].tolist(), c["B"][0, 0].tolist(),
+                              c["C"][0, 0].tolist(), c["A"].tolist(), c["D"].tolist(),
+                              c["B"][1, 0].tolist(), c["C"][1, 0].tolist())
+    np.testing.assert_allclose(y[0], np.array(ref), rtol=1e-12, atol=1e-12)
+
+
+ALL_PINS = [
+    pin_delta_zero,
+    pin_constant_input_geometric,
+    pin_reverse_symmetry,
+    pin_brute_force,
+    pin_prefix_sum,
+    pin_linearity,
+    pin_softplus,
+    pin_gate_is_silu,
+    pin_cross_orders_golden,
+    pin_cross_scan_is_transpose_and_flip,
+    pin_cross_merge,
+    pin_separate_bc,
+]

@@ -1,0 +1,59 @@
+"""Plant a mistake in a copy of the oracle and check that some pin catches it.
+
+Each mutant is oracle.c with one plausible slip (a dropped term, a wrong sign, a
+wrong index, a transposed operand), compiled into a temporary directory.  The test
+passes when every mutant fails at least one pin, which shows that the pins do not
+merely re-run the oracle's own formula.  CPU only; nothing here touches a GPU.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+MUTANTS = {
+    "drop_D_skip": ("yt += D[d] * x;", "yt += 0.0 * x;"),
+    "decay_sign": ("exp(dt * A[d * N + n])", "exp(-dt * A[d * N + n])"),
+    "bbar_without_delta": ("double Bbar = dt * Bt[n];", "double Bbar = Bt[n];"),
+    "readout_uses_B": ("yt += Ct[n] * h[n];", "yt += Bt[n] * h[n];"),
+    "A_transposed": ("exp(dt * A[d * N + n])", "exp(dt * A[n * Di + d])"),
+    "readout_before_update": (
+        "h[n] = Abar * h[n] + Bbar * x;                    /* h_t = Abar h + Bbar x */\n"
+        "                yt += Ct[n] * h[n];",
+        "yt += Ct[n] * h[n];\n                h[n] = Abar * h[n] + Bbar * x;"),
+    "backward_not_reversed": ("order[t] = L - 1 - t;", "order[t] = t;"),
+    "backward_uses_forward_bias": ("D + Di, bias + Di, order", "D + Di, bias, order"),
+    "backward_uses_forward_bc": ("B + bc_dir_stride, C + bc_dir_stride", "B, C"),
+    "softplus_wrong": ("log1p(exp(x))", "log(exp(x) + 0.5)"),
+    "gate_is_sigmoid": ("return z / (1.0 + exp(-z));", "return 1.0 / (1.0 + exp(-z));"),
+    "column_scan_is_row_scan": ("int64_t h = s % H, w = s / H;", "int64_t h = s / W, w = s % W;"),
+    "column_scan_transposed": ("p = h * W + w;", "p = w * H + h;"),
+    "cross_bc_not_per_direction": ("B + k * bc, C + k * bc", "B, C"),
+    "merge_ignores_order": ("int64_t p = order[t];\n                for (int64_t c = 0",
+                            "int64_t p = t;\n                for (int64_t c = 0"),
+    "delta_bias_ignored": ("softplus(delta[ix] + bias[d])", "softplus(delta[ix])"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation site for {name} not found"
+    path_c = tmp_path / "oracle_mut.c"
+    path_c.write_text(src.replace(old, new))
+    path_so = tmp_path / "liboracle_mut.so"
+    subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", str(path_so), str(path_c), "-lm"],
+                   check=True)
+    mutant = oracle.Oracle(str(path_so))
+    caught = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(mutant)
+        except (AssertionError, ValueError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches mutant {name}"
