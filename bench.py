@@ -1,0 +1,390 @@
+#!/usr/bin/env python
+"""Throughput of the bidirectional selective scan (S6) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one pass of the whole scan -- softplus Delta, the forward and backward
+recurrences, readout, D skip, the merge of the directions and the silu(z) gate --
+over one batch of the workload, through the library's C ABI.  The default workload
+is the 1024 px Vim-Tiny scan (batch 8, L = 4097, d_inner 384, d_state 16, bf16 I/O,
+fp32 state).  Inputs are seeded synthetic tensors shaped like the pages' workloads.
+
+Multi-GPU (torchrun, one process per GPU): the batch items are independent, so every
+rank runs the same workload on its own inputs with no collective on the data path
+(weak scaling); NCCL is used only for the barrier and the max over ranks of the time.
+
+--impl reference times the fp64 CPU oracle (the correctness reference, not tuned) on
+the host cores, on a bounded sample of the same workload; under torchrun only rank 0
+runs it.
+
+Rank 0 prints one JSON line.
+"""
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 2**20
+MEASURED = os.path.join(ROOT, "MEASURED_PEAKS.json")
+# FP32 lanes per SM on B200 (an FMA counts as one lane-op); 148 SMs.
+FP32_LANES_PER_SM = 128
+SMS = 148
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="vim_tiny_1024px_bf16")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(MEASURED) as f:
+            m = json.load(f)
+        return dict(hbm_gbs=float(m["hbm_gbs"]), sm_max_mhz=float(m.get("sm_max_mhz", 1965.0)),
+                    source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, sm_max_mhz=1965.0, source="fallback")
+
+
+def algorithmic(w):
+    """Algorithmic bytes and FP32 lane-ops of one step.
+
+    Bytes: one read of u, delta_raw, z and one write of y per token-channel, one read
+    of B and C per token (per direction when they are separate), the fp32 parameters
+    once.  Ops: the recurrence core, 4 FP32 lane-ops per state per direction per
+    token-channel (decay, Delta*B*u, the state update, the readout).
+    """
+    el = 4 if w.dtype == "f32" else 2
+    n_bc_sets = 1 if w.kind == "vim" else w.directions
+    bc = 2 * w.batch * w.tokens * w.d_state * el * n_bc_sets
+    params = w.directions * w.channels * (w.d_state + 2) * 4
+    nbytes = 4 * w.tok_ch * el + bc + params
+    ops = 4 * w.d_state * w.directions * w.tok_ch
+    return nbytes, ops
+
+
+class ClockSampler:
+    """NVML samples of the SM clock and the clock-event reasons, in a thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index, period=0.002):
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover
+            self.err = repr(e)
+        self.period = period
+        self.samples, self.reasons = [], 0
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+def run_oracle(w, x, threads):
+    import oracle
+
+    oracle.set_threads(threads)
+    t = time.perf_counter()
+    if w.kind == "vim":
+        oracle.vim_bidir(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"])
+    else:
+        oracle.cross_scan4(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"])
+    return time.perf_counter() - t
+
+
+def oracle_sample(w, target_s):
+    """A bounded sample of the workload for the oracle: its first batch items and
+    first channels at the full sequence length, sized for about ``target_s`` seconds
+    of fp64 work on the host cores (calibrated on a small run)."""
+    from vision_mamba_selective_b200 import workloads as wl
+
+    cores = cpu_cores()
+    full = wl.make_inputs(w)
+    step = 8
+
+    def cut(b, c):
+        x = {}
+        for k, v in full.items():
+            if k in ("u", "delta", "z"):
+                x[k] = v[:b, ..., :c].contiguous()
+            elif k in ("B", "C"):
+                x[k] = (v[:b] if w.kind == "vim" else v[:, :b]).contiguous()
+            else:
+                x[k] = v[..., :c, :].contiguous() if k == "A" else v[..., :c].contiguous()
+        return w.scaled(batch=b, channels=c), x
+
+    cal_c = min(w.channels, 64)
+    s, x = cut(1, cal_c)
+    t = max(run_oracle(s, x, cores), 1e-4)
+    per = t / s.tok_ch
+    want = max(1, int(target_s / per))                      # token-channels to process
+    per_item = w.tokens * w.channels
+    if want >= per_item:
+        b, c = min(w.batch, want // per_item), w.channels
+    else:
+        b, c = 1, max(step, min(w.channels, (want // w.tokens) // step * step))
+    return cut(b, c) + (cores,)
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def reference_arm(args, w):
+    """The oracle, as it stands, on the host cores: K timed steps of a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    per_step = min(2.0, 150.0 / max(1, args.steps + args.warmup))
+    s, x, cores = oracle_sample(w, per_step)
+    for _ in range(args.warmup):
+        run_oracle(s, x, cores)
+    times = [run_oracle(s, x, cores) for _ in range(args.steps)]
+    sec = sum(times) / len(times)
+    value = s.tok_ch / sec
+    sample = (f"{s.batch} of {w.batch} batch items x {s.channels} of {w.channels} channels at the full "
+              f"{w.tokens} tokens ({s.tok_ch} token-channels) per step, fp64")
+    line = {
+        "impl": "reference", "metric": "bidirectional S6 scan token-channels/s at L=4097; achieved HBM GB/s vs peak",
+        "value": value, "unit": "tok*ch/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch_per_gpu": w.batch, "tokens": w.tokens,
+                   "channels": w.channels, "d_state": w.d_state, "io_dtype": w.dtype},
+        "cpu_baseline": {"value": value, "unit": "tok*ch/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tok*ch/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    from vision_mamba_selective_b200 import workloads as wl
+
+    w = wl.BY_NAME[args.workload]
+    if args.impl == "reference":
+        reference_arm(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    from vision_mamba_selective_b200 import vimscan as vs
+
+    # ---- inputs: rank-specific seed; enough rotating copies to exceed L2 ---------
+    host = wl.make_inputs(w, seed=w.seed + 7919 * rank)
+    act_keys = ["u", "delta", "z", "B", "C"]
+    set_bytes = sum(host[k].numel() * host[k].element_size() for k in act_keys) + \
+        w.tok_ch * (4 if w.dtype == "f32" else 2)
+    nsets = max(2, math.ceil(2.2 * L2_BYTES / set_bytes))
+    params = {k: host[k].to(dev) for k in ("A", "D", "delta_bias")}
+    sets = []
+    for _ in range(nsets):
+        s = {k: host[k].to(dev) for k in act_keys}
+        s["y"] = torch.empty_like(s["u"])
+        sets.append(s)
+    if w.kind == "vim":
+        ws_bytes = vs.vim_scan_workspace_bytes(0, w.batch, w.L, 0, w.channels, w.d_state)
+    else:
+        ws_bytes = vs.vim_scan_workspace_bytes(1, w.batch, w.H, w.W, w.channels, w.d_state)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    fn = vs.vim_scan_bidir if w.kind == "vim" else vs.vmamba_cross_scan4
+
+    def step(i, events=None):
+        s = sets[i % nsets]
+        fn(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"], params["delta_bias"],
+           y=s["y"], workspace=ws, events=events)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # ---- timed region -----------------------------------------------------------
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record()
+        for i in range(args.steps):
+            step(i)
+        end.record()
+        torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(start.elapsed_time(end))
+    ms_step = ms / args.steps
+    value = world * w.tok_ch * args.steps / (ms * 1e-3)
+
+    # ---- per-kernel times (same launches plus event records), after the timed region
+    kernels_per_pair = 3
+    pairs = 1 if w.kind == "vim" else 2
+    nev = 1 + kernels_per_pair * pairs
+    prof_steps = min(args.steps, 200)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(prof_steps)]
+    for i in range(prof_steps):
+        step(i, events=evs[i])
+    torch.cuda.synchronize()
+    names = ["pair_carry", "pair_combine", "pair_main"]
+    per_kernel = {}
+    for p in range(pairs):
+        for k in range(kernels_per_pair):
+            a = 1 + 3 * p + k
+            t = [evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(prof_steps)]
+            per_kernel[f"{names[k]}[{p}]" if pairs > 1 else names[k]] = sum(t) / len(t)
+    G = math.ceil(w.tokens / 128) if w.tokens > 256 else 1
+    launches_per_step = pairs * (3 if G > 1 else 1)
+
+    # ---- end to end: pinned host inputs -> device -> scan -> host result ---------
+    pinned = {k: host[k].pin_memory() for k in act_keys}
+    y_host = torch.empty(sets[0]["y"].shape, dtype=sets[0]["y"].dtype).pin_memory()
+    h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in act_keys)
+    d2h = y_host.numel() * y_host.element_size()
+    e2e_steps = min(args.steps, 50)
+    for _ in range(2):
+        for k in act_keys:
+            sets[0][k].copy_(pinned[k], non_blocking=True)
+        step(0)
+        y_host.copy_(sets[0]["y"], non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        for k in act_keys:
+            sets[0][k].copy_(pinned[k], non_blocking=True)
+        step(0)
+        y_host.copy_(sets[0]["y"], non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = world * w.tok_ch * e2e_steps / (e2e_ms * 1e-3)
+
+    # ---- roofline of the dominant kernel -----------------------------------------
+    pk = peaks()
+    nbytes, ops = algorithmic(w)
+    main_ms = sum(v for k, v in per_kernel.items() if k.startswith("pair_main"))
+    clocks = clk.summary()
+    peak_ops = SMS * FP32_LANES_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e12
+    achieved_ops = ops / (main_ms * 1e-3) / 1e12
+    roofline = {
+        "bound": "alu", "kernel": "pair_main", "achieved": achieved_ops, "peak": peak_ops,
+        "unit": "Tops/s", "frac": achieved_ops / peak_ops, "traffic": None,
+        "ops_per_launch": ops, "ms_per_launch": main_ms,
+        "peak_basis": f"{SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x {pk['sm_max_mhz']:.0f} MHz",
+        "hbm_gbs_whole_step": nbytes / (ms_step * 1e-3) / 1e9,
+        "hbm_frac_whole_step": nbytes / (ms_step * 1e-3) / 1e9 / pk["hbm_gbs"],
+        "hbm_peak_gbs": pk["hbm_gbs"], "peak_source": pk["source"],
+    }
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        s, x, cores = oracle_sample(w, 5.0)
+        sec = run_oracle(s, x, cores)
+        cpu = {"value": s.tok_ch / sec, "unit": "tok*ch/s", "cores": cores, "kind": "oracle",
+               "sample": f"{s.batch} of {w.batch} batch items x {s.channels} of {w.channels} channels "
+                         f"at the full {w.tokens} tokens ({s.tok_ch} token-channels), fp64, {sec:.2f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": "bidirectional S6 scan token-channels/s at L=4097; achieved HBM GB/s vs peak",
+            "value": value, "unit": "tok*ch/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded, shaped like the pages' workloads)",
+            "config": {"workload": w.name, "batch_per_gpu": w.batch, "tokens": w.tokens,
+                       "channels": w.channels, "d_state": w.d_state, "io_dtype": w.dtype,
+                       "parallelism": f"replicas x{world} (batch shards, no collective)",
+                       "l2": f"{nsets} rotating input sets of {set_bytes / 1e6:.0f} MB (> 126 MB L2)"},
+            "hbm_gbs": roofline["hbm_gbs_whole_step"], "hbm_frac": roofline["hbm_frac_whole_step"],
+            "kernel_ms": per_kernel,
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tok*ch/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,165 @@
+/*
+ * vimscan.h -- C ABI of the B200 (sm_100a) selective-scan library libvimscan.so.
+ *
+ * The operations are those of the page "Vision Mamba Guide: Efficient Bidirectional
+ * SSM & VMamba" (aifetchly-blog):
+ *   - the S6 recurrence with input-dependent Delta, B, C (sections "Discretization
+ *     via Zero-Order Hold (ZOH)" and "The Selective State Space (S6) Mechanism"):
+ *         Delta_t = softplus(delta_raw_t + delta_bias)      (softplus(x) = x for x > 20)
+ *         h_t     = exp(Delta_t * A) * h_{t-1} + Delta_t * B_t * u_t     (h starts at 0)
+ *         y_t     = C_t . h_t + D * u_t
+ *   - the Vim bidirectional block (section "2. The Bidirectional Mamba Block"): a
+ *     forward pass over the tokens and a backward pass from the last token to the
+ *     first, fused as (y^f + y^b) * silu(z), silu(z) = z / (1 + exp(-z));
+ *   - the VMamba cross-scan (sections "1. Cross-Scan Traversal (CS-Traverse)",
+ *     "2. Parallel S6 State Space Processing", "3. Cross-Merge Reversal
+ *     (CS-Merge)"): four scans of an H x W grid (row-major, its reverse,
+ *     column-major, its reverse), each mapped back to (h, w) and summed.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous and
+ *     row-major, 16-byte aligned.  The library allocates no device memory and keeps
+ *     no state between calls; scratch memory is the caller's workspace.
+ *   - `dt` is the element type of u, delta, z, B, C, ys and y (fp32 or bf16).  A, D
+ *     and delta_bias are always fp32.  Arithmetic is fp32 with the state h held in
+ *     fp32 registers; bf16 outputs are rounded once, to nearest even.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream) and
+ *     return before the kernels finish.  Inputs must stay valid and unmodified, and
+ *     outputs and workspace untouched, until the stream reaches that point.
+ *   - Arguments are checked on the host before anything is launched.  A failed
+ *     check returns VIM_ERR_INVALID_ARG, VIM_ERR_UNSUPPORTED or VIM_ERR_WORKSPACE and
+ *     launches nothing.  A launch failure returns VIM_ERR_CUDA.  No call aborts,
+ *     throws or prints.
+ *   - Sizes of 0 (batch, tokens or channels) are valid and do nothing.
+ *   - Supported: d_state in {2, 4, 8, 16}; channels a multiple of 8 (bf16) or of 4
+ *     (fp32).  Anything else returns VIM_ERR_UNSUPPORTED.
+ *   - Outputs must not overlap inputs or the workspace.
+ */
+#ifndef VIMSCAN_H
+#define VIMSCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    VIM_OK = 0,
+    VIM_ERR_INVALID_ARG = 1,   /* null or misaligned pointer, negative size        */
+    VIM_ERR_UNSUPPORTED = 2,   /* d_state or channel count outside the supported set */
+    VIM_ERR_WORKSPACE = 3,     /* workspace missing, misaligned or too small        */
+    VIM_ERR_CUDA = 4,          /* a CUDA launch failed                              */
+    VIM_ERR_TIMEOUT = 5        /* reserved: a bounded device-side wait ran out      */
+} vim_status;
+
+typedef enum { VIM_F32 = 0, VIM_BF16 = 1 } vim_dtype;
+
+/*
+ * Vim bidirectional selective scan with gated fusion (section "2. The Bidirectional
+ * Mamba Block"; its output projection is not part of this call):
+ *
+ *   y[b,t,d] = ( y^f[b,t,d] + y^b[b,t,d] ) * silu(z[b,t,d])
+ *   y^f : forward S6 over t = 0 .. L-1 with A[0], D[0], delta_bias[0], B, C
+ *   y^b : backward S6 over t = L-1 .. 0 with A[1], D[1], delta_bias[1],
+ *         B + bc_dir_stride, C + bc_dir_stride; y^b is indexed by original position.
+ *
+ *   u, delta, z : [batch, L, d_inner] (dt).  delta holds the raw value; the call
+ *                 applies softplus(delta + delta_bias[k][d]).  z may be NULL: no gate.
+ *   B, C        : [batch, L, d_state] (dt), shared by all channels of a token.
+ *   bc_dir_stride: element offset of the backward direction's B and C from B and C
+ *                 (0 = both directions read the same B and C).  Must be >= 0.
+ *   A           : [2, d_inner, d_state] fp32 (index 0 = forward, 1 = backward);
+ *                 fastest when A[k][d][n] == (n+1) * A[k][d][0] (the S4D-real form).
+ *   D, delta_bias : [2, d_inner] fp32.
+ *   y           : [batch, L, d_inner] (dt), written once.
+ *   workspace   : caller-owned device scratch of at least
+ *                 vim_scan_workspace_bytes(0, batch, L, 0, d_inner, d_state) bytes,
+ *                 256-byte aligned (may be NULL when that size is 0).
+ */
+vim_status vim_scan_bidir(const void *u, const void *delta, const void *z,
+                          const void *B, const void *C, int64_t bc_dir_stride,
+                          const float *A, const float *D, const float *delta_bias,
+                          void *y, int batch, int L, int d_inner, int d_state, vim_dtype dt,
+                          void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * VMamba four-direction cross-scan with CS-Merge (sections "1. Cross-Scan
+ * Traversal", "2. Parallel S6 State Space Processing", "3. Cross-Merge Reversal"):
+ *
+ *   y[b,h,w,c] = ( sum_{k=1..4} y_k[b,h,w,c] ) * silu(z[b,h,w,c])
+ *   scan 1 visits p = h*W + w in increasing order, scan 2 in decreasing order,
+ *   scan 3 visits the grid column by column (step t = w*H + h), scan 4 the reverse
+ *   of scan 3; each y_k is written back at the grid position its step visited.
+ *
+ *   u, delta, z : [batch, H, W, channels] (dt), channels last.  z may be NULL.
+ *   B, C        : [4, batch, H*W, d_state] (dt), per direction, stored by GRID
+ *                 position: scan k reads B[k, b, p, :] when it visits position p.
+ *   A           : [4, channels, d_state] fp32; D, delta_bias : [4, channels] fp32.
+ *   y           : [batch, H, W, channels] (dt).
+ *   workspace   : at least vim_scan_workspace_bytes(1, batch, H, W, channels,
+ *                 d_state) bytes, 256-byte aligned.
+ */
+vim_status vmamba_cross_scan4(const void *u, const void *delta, const void *z,
+                              const void *B, const void *C,
+                              const float *A, const float *D, const float *delta_bias,
+                              void *y, int batch, int H, int W, int channels, int d_state,
+                              vim_dtype dt, void *workspace, size_t workspace_bytes,
+                              cudaStream_t stream);
+
+/*
+ * CS-Merge alone (section "3. Cross-Merge Reversal (CS-Merge)"): maps each of four
+ * scan-order outputs back to its grid position and sums them.
+ *
+ *   ys : [4, batch, H*W, channels] (dt); row t of ys[k] belongs to the grid position
+ *        that scan k+1 visits at step t (orders as in vmamba_cross_scan4).
+ *   z  : [batch, H, W, channels] (dt) or NULL; the sum is multiplied by silu(z).
+ *   y  : [batch, H, W, channels] (dt).  Sums are formed in fp32.
+ */
+vim_status cross_merge4(const void *ys, const void *z, void *y, int batch, int H, int W,
+                        int channels, vim_dtype dt, cudaStream_t stream);
+
+/*
+ * Instrumented variants for benchmarks: the same checks and the same launches as
+ * vim_scan_bidir / vmamba_cross_scan4, plus cudaEventRecord(events[i], stream) at
+ * each kernel boundary.  A scan runs, per pair of directions, up to three kernels:
+ * chunk summaries, their fold, and the main pass (the first two only when the
+ * sequence spans more than one chunk; a skipped kernel's two events are recorded back
+ * to back).  events[0] is recorded before the first kernel and events[3*k+i+1] after
+ * kernel i of pair k, so vim_scan_bidir_events needs 4 events and
+ * vmamba_cross_scan4_events 7.  Events are created by the caller; a NULL `events`
+ * behaves exactly like the plain entry point.
+ */
+vim_status vim_scan_bidir_events(const void *u, const void *delta, const void *z,
+                                 const void *B, const void *C, int64_t bc_dir_stride,
+                                 const float *A, const float *D, const float *delta_bias,
+                                 void *y, int batch, int L, int d_inner, int d_state,
+                                 vim_dtype dt, void *workspace, size_t workspace_bytes,
+                                 cudaStream_t stream, cudaEvent_t *events);
+
+vim_status vmamba_cross_scan4_events(const void *u, const void *delta, const void *z,
+                                     const void *B, const void *C,
+                                     const float *A, const float *D, const float *delta_bias,
+                                     void *y, int batch, int H, int W, int channels,
+                                     int d_state, vim_dtype dt, void *workspace,
+                                     size_t workspace_bytes, cudaStream_t stream,
+                                     cudaEvent_t *events);
+
+/*
+ * Workspace bytes the scan entry points need (0 when none).  which = 0 for
+ * vim_scan_bidir (L_or_H = L, W ignored), 1 for vmamba_cross_scan4 (L_or_H = H).
+ * Returns 0 for invalid arguments as well; the entry point then reports them.
+ */
+size_t vim_scan_workspace_bytes(int which, int batch, int L_or_H, int W, int channels,
+                                int d_state);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+const char *vim_status_string(vim_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VIMSCAN_H */

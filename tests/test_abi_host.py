@@ -1,0 +1,149 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol, and
+rejects bad arguments on the host before anything is launched.
+
+Every call below fails a host-side check (or is a size-0 no-op), so none of them
+reaches a kernel launch; that keeps these tests safe on a machine with a GPU too.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vimscan.h")
+
+
+@pytest.fixture(scope="module")
+def vs():
+    from vision_mamba_selective_b200 import build
+
+    build.build()
+    from vision_mamba_selective_b200 import vimscan
+
+    return vimscan
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:vim_status|size_t|const char \*)\s*\*?\s*(\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    assert set(names) == {"vim_scan_bidir", "vmamba_cross_scan4", "cross_merge4",
+                          "vim_scan_bidir_events", "vmamba_cross_scan4_events",
+                          "vim_scan_workspace_bytes", "vim_status_string"}, names
+
+
+def test_header_compiles_as_c():
+    subprocess.run(["gcc", "-fsyntax-only", "-x", "c", "-std=c99", "-I/usr/local/cuda/include", HEADER],
+                   check=True)
+
+
+def test_exports_every_symbol(vs):
+    out = subprocess.run(["nm", "-D", "--defined-only", vs.LIB_PATH], check=True,
+                         capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(vs.lib, name)
+
+
+def test_status_strings(vs):
+    for code in range(6):
+        s = vs.status_string(code)
+        assert isinstance(s, str) and s
+    assert vs.status_string(0) == "ok"
+    assert "unknown" in vs.status_string(99)
+
+
+def test_workspace_bytes(vs):
+    assert vs.vim_scan_workspace_bytes(0, 64, 197, 0, 768, 16) == 0          # one chunk
+    n = vs.vim_scan_workspace_bytes(0, 8, 4097, 0, 384, 16)
+    G = (4097 + 127) // 128
+    assert n >= 8 * G * 2 * 384 * 17 * 4 and n % 256 == 0
+    m = vs.vim_scan_workspace_bytes(1, 16, 64, 64, 192, 16)
+    assert m >= 16 * 4096 * 192 * 4 + 16 * 32 * 2 * 192 * 17 * 4
+    assert vs.vim_scan_workspace_bytes(0, 1, 100, 0, 8, 3) == 0               # unsupported N
+    assert vs.vim_scan_workspace_bytes(7, 1, 100, 0, 8, 16) == 0              # unknown kind
+
+
+FAKE = 0x7f0000000000   # 256-byte aligned, never dereferenced: every call fails a check first
+
+
+def bidir(vs, **kw):
+    a = dict(u=FAKE, delta=FAKE, z=FAKE, B=FAKE, C=FAKE, stride=0, A=FAKE, D=FAKE, bias=FAKE, y=FAKE,
+             batch=2, L=33, Di=64, N=16, dt=vs.VIM_BF16, ws=None, ws_bytes=0)
+    a.update(kw)
+    return vs.lib.vim_scan_bidir(a["u"], a["delta"], a["z"], a["B"], a["C"], a["stride"], a["A"],
+                                 a["D"], a["bias"], a["y"], a["batch"], a["L"], a["Di"], a["N"],
+                                 a["dt"], a["ws"], a["ws_bytes"], None)
+
+
+def test_bidir_rejects(vs):
+    assert bidir(vs, u=None) == vs.VIM_ERR_INVALID_ARG
+    assert bidir(vs, y=None) == vs.VIM_ERR_INVALID_ARG
+    assert bidir(vs, A=None) == vs.VIM_ERR_INVALID_ARG
+    assert bidir(vs, u=FAKE + 8) == vs.VIM_ERR_INVALID_ARG            # not 16-byte aligned
+    assert bidir(vs, z=FAKE + 2) == vs.VIM_ERR_INVALID_ARG
+    assert bidir(vs, B=FAKE + 1) == vs.VIM_ERR_INVALID_ARG            # not element aligned
+    assert bidir(vs, D=FAKE + 2) == vs.VIM_ERR_INVALID_ARG
+    assert bidir(vs, batch=-1) == vs.VIM_ERR_INVALID_ARG
+    assert bidir(vs, L=-5) == vs.VIM_ERR_INVALID_ARG
+    assert bidir(vs, stride=-1) == vs.VIM_ERR_INVALID_ARG
+    assert bidir(vs, dt=7) == vs.VIM_ERR_INVALID_ARG
+    assert bidir(vs, N=3) == vs.VIM_ERR_UNSUPPORTED
+    assert bidir(vs, N=32) == vs.VIM_ERR_UNSUPPORTED
+    assert bidir(vs, Di=12) == vs.VIM_ERR_UNSUPPORTED                 # bf16 needs multiples of 8
+    assert bidir(vs, Di=6, dt=vs.VIM_F32) == vs.VIM_ERR_UNSUPPORTED   # fp32 needs multiples of 4
+    # long sequences need the caller's workspace
+    assert bidir(vs, L=4097, ws=None) == vs.VIM_ERR_WORKSPACE
+    assert bidir(vs, L=4097, ws=FAKE, ws_bytes=16) == vs.VIM_ERR_WORKSPACE
+    assert bidir(vs, L=4097, ws=FAKE + 16, ws_bytes=1 << 40) == vs.VIM_ERR_WORKSPACE
+
+
+def test_size_zero_is_a_noop(vs):
+    # nothing is read or launched, so even null pointers are fine
+    assert bidir(vs, batch=0, u=None, y=None) == vs.VIM_OK
+    assert bidir(vs, L=0, u=None) == vs.VIM_OK
+    assert bidir(vs, Di=0, u=None) == vs.VIM_OK
+    assert vs.lib.cross_merge4(None, None, None, 0, 4, 4, 8, vs.VIM_BF16, None) == vs.VIM_OK
+
+
+def test_cross4_rejects(vs):
+    f = vs.lib.vmamba_cross_scan4
+
+    def call(**kw):
+        a = dict(u=FAKE, delta=FAKE, z=None, B=FAKE, C=FAKE, A=FAKE, D=FAKE, bias=FAKE, y=FAKE,
+                 batch=2, H=8, W=8, ch=64, N=16, dt=vs.VIM_BF16, ws=None, ws_bytes=0)
+        a.update(kw)
+        return f(a["u"], a["delta"], a["z"], a["B"], a["C"], a["A"], a["D"], a["bias"], a["y"],
+                 a["batch"], a["H"], a["W"], a["ch"], a["N"], a["dt"], a["ws"], a["ws_bytes"], None)
+
+    assert call(u=None) == vs.VIM_ERR_INVALID_ARG
+    assert call(H=-1) == vs.VIM_ERR_INVALID_ARG
+    assert call(N=5) == vs.VIM_ERR_UNSUPPORTED
+    assert call() == vs.VIM_ERR_WORKSPACE            # the merge always needs the fp32 partial
+    assert call(ws=FAKE + 128, ws_bytes=1 << 40) == vs.VIM_ERR_WORKSPACE
+    assert call(H=0) == vs.VIM_OK
+
+
+def test_merge_rejects(vs):
+    f = vs.lib.cross_merge4
+    assert f(None, None, FAKE, 1, 4, 4, 8, vs.VIM_BF16, None) == vs.VIM_ERR_INVALID_ARG
+    assert f(FAKE, None, None, 1, 4, 4, 8, vs.VIM_BF16, None) == vs.VIM_ERR_INVALID_ARG
+    assert f(FAKE + 4, None, FAKE, 1, 4, 4, 8, vs.VIM_BF16, None) == vs.VIM_ERR_INVALID_ARG
+    assert f(FAKE, None, FAKE, 1, 4, 4, 6, vs.VIM_BF16, None) == vs.VIM_ERR_UNSUPPORTED
+    assert f(FAKE, None, FAKE, -1, 4, 4, 8, vs.VIM_BF16, None) == vs.VIM_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors(vs):
+    import torch
+
+    x = torch.zeros(1, 4, 8)
+    with pytest.raises(TypeError):
+        vs.vim_scan_bidir(x, x, x, torch.zeros(1, 4, 2), torch.zeros(1, 4, 2), torch.zeros(2, 8, 2),
+                          torch.zeros(2, 8), torch.zeros(2, 8), y=torch.zeros(1, 4, 8))

@@ -1,0 +1,251 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Both sides get the same seeded input bits (bf16 or fp32; the oracle reads them
+exactly in fp64).  The error measure is normwise:  max_i |y_i - r_i| / max_i |r_i|,
+with the tolerances of the target: 1e-5 for fp32 I/O and 2e-2 for bf16 I/O (fp32
+state in both).  Shapes cover several chunks and tiles with ragged tails, channel
+counts that leave a partial block of 64, d_state 2..16, general (not S4D-real) A,
+the softplus cut at 20, large |z|, empty inputs, and the five full-size workloads
+in the launch configuration the benchmark times.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from vision_mamba_selective_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.float32: 1e-5, torch.bfloat16: 2e-2}
+REPORT = os.environ.get("VIMSCAN_PARITY_REPORT")
+
+
+@pytest.fixture(scope="module")
+def vs():
+    from vision_mamba_selective_b200 import vimscan
+
+    return vimscan
+
+
+def normwise(y, ref):
+    y = y.detach().to("cpu", torch.float64).numpy()
+    den = np.max(np.abs(ref))
+    return float(np.max(np.abs(y - ref)) / den) if den > 0 else float(np.max(np.abs(y - ref)))
+
+
+def check(name, y, ref, dtype):
+    err = normwise(y, ref)
+    if REPORT:
+        with open(REPORT, "a") as f:
+            f.write(json.dumps({"case": name, "dtype": str(dtype), "normwise": err}) + "\n")
+    assert np.all(np.isfinite(y.float().cpu().numpy()))
+    assert err <= TOL[dtype], f"{name}: normwise error {err:.3e} > {TOL[dtype]:.0e}"
+    return err
+
+
+def vim_inputs(batch, L, Di, N, dtype, seed, *, generic_A=False, separate_bc=False, delta_scale=0.5):
+    g = torch.Generator().manual_seed(seed)
+    r = lambda *s, std=1.0: (torch.randn(s, generator=g) * std)
+    u, dr, z = r(batch, L, Di), r(batch, L, Di, std=delta_scale), r(batch, L, Di)
+    nb = 2 if separate_bc else 1
+    B, C = r(nb, batch, L, N), r(nb, batch, L, N)
+    if generic_A:
+        A = -(0.05 + 3 * torch.rand((2, Di, N), generator=g))
+    else:
+        A = -torch.arange(1, N + 1, dtype=torch.float32).repeat(2, Di, 1)
+    D = r(2, Di)
+    s = torch.exp(np.log(1e-3) + (np.log(1e-1) - np.log(1e-3)) * torch.rand((2, Di), generator=g, dtype=torch.float64))
+    bias = torch.log(torch.expm1(s)).float()
+    t = lambda x: x.to(dtype).contiguous()
+    return dict(u=t(u), delta=t(dr), z=t(z), B=t(B), C=t(C), A=A.contiguous(), D=D.contiguous(),
+                bias=bias.contiguous(), stride=batch * L * N if separate_bc else 0)
+
+
+def run_vim(vs, x, gate=True):
+    dev = lambda t: t.cuda()
+    y = vs.vim_scan_bidir(dev(x["u"]), dev(x["delta"]), dev(x["z"]) if gate else None,
+                          dev(x["B"]), dev(x["C"]), dev(x["A"]), dev(x["D"]), dev(x["bias"]),
+                          bc_dir_stride=x["stride"])
+    torch.cuda.synchronize()
+    return y
+
+
+def ref_vim(x, gate=True):
+    return oracle.vim_bidir(x["u"], x["delta"], x["z"] if gate else None, x["B"], x["C"], x["A"],
+                            x["D"], x["bias"], bc_dir_stride=x["stride"])
+
+
+VIM_CASES = [
+    # batch, L, Di, N, dtype, generic_A, separate_bc, gate
+    (1, 1, 8, 16, torch.float32, False, False, True),
+    (2, 2, 64, 16, torch.float32, False, False, True),
+    (1, 7, 72, 16, torch.bfloat16, False, False, True),
+    (3, 16, 64, 8, torch.float32, True, True, True),
+    (2, 17, 136, 16, torch.bfloat16, False, True, False),
+    (1, 33, 64, 4, torch.float32, False, False, True),
+    (2, 197, 200, 16, torch.float32, False, False, True),
+    (1, 197, 64, 2, torch.bfloat16, True, False, True),
+    (1, 256, 64, 16, torch.float32, False, False, True),      # longest single chunk
+    (2, 257, 72, 16, torch.float32, False, False, True),      # 3 chunks, last one 1 token
+    (1, 300, 64, 16, torch.float32, True, True, True),        # chunks with general A
+    (1, 1000, 128, 16, torch.bfloat16, False, False, True),
+    (2, 1111, 64, 8, torch.float32, False, True, True),
+    (2, 50, 12, 16, torch.float32, False, False, True),       # fp32: channels a multiple of 4 only
+    (1, 400, 36, 16, torch.float32, True, False, True),
+]
+
+
+@pytest.mark.parametrize("case", VIM_CASES, ids=lambda c: f"b{c[0]}_L{c[1]}_D{c[2]}_N{c[3]}_{str(c[4])[6:]}"
+                         f"{'_genA' if c[5] else ''}{'_sepBC' if c[6] else ''}{'' if c[7] else '_nogate'}")
+def test_vim_small(vs, case):
+    batch, L, Di, N, dtype, gen, sep, gate = case
+    x = vim_inputs(batch, L, Di, N, dtype, seed=L * 7 + Di, generic_A=gen, separate_bc=sep)
+    check(f"vim_{case}", run_vim(vs, x, gate), ref_vim(x, gate), dtype)
+
+
+def test_vim_softplus_cut_and_large_gate(vs):
+    x = vim_inputs(2, 40, 64, 16, torch.float32, seed=5)
+    x["delta"] = (x["delta"] * 0 + torch.linspace(-30, 30, 40)[None, :, None]).contiguous()
+    x["z"] = (x["z"] * 40).contiguous()
+    check("vim_extreme", run_vim(vs, x), ref_vim(x), torch.float32)
+
+
+def test_vim_empty(vs):
+    x = vim_inputs(1, 5, 64, 16, torch.float32, seed=1)
+    for k in ("u", "delta", "z"):
+        x[k] = x[k][:0]
+    y = run_vim(vs, x)
+    assert y.shape == (0, 5, 64)
+    x = vim_inputs(1, 0, 64, 16, torch.bfloat16, seed=1)
+    assert run_vim(vs, x).shape == (1, 0, 64)
+
+
+def test_vim_output_written_once_and_inputs_untouched(vs):
+    x = vim_inputs(2, 300, 72, 16, torch.bfloat16, seed=9)
+    dev = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
+    before = {k: v.clone() for k, v in dev.items() if torch.is_tensor(v)}
+    y = torch.full_like(dev["u"], float("nan"))
+    vs.vim_scan_bidir(dev["u"], dev["delta"], dev["z"], dev["B"], dev["C"], dev["A"], dev["D"],
+                      dev["bias"], y=y)
+    torch.cuda.synchronize()
+    assert torch.isfinite(y.float()).all()
+    for k, v in before.items():
+        assert torch.equal(v, dev[k]), k
+    check("vim_prefilled", y, ref_vim(x), torch.bfloat16)
+
+
+def test_vim_deterministic(vs):
+    x = vim_inputs(2, 600, 64, 16, torch.float32, seed=3)
+    y1, y2 = run_vim(vs, x), run_vim(vs, x)
+    assert torch.equal(y1, y2)
+
+
+def cross_inputs(batch, H, W, Ch, N, dtype, seed, generic_A=False):
+    g = torch.Generator().manual_seed(seed)
+    r = lambda *s, std=1.0: (torch.randn(s, generator=g) * std)
+    u, dr, z = r(batch, H, W, Ch), r(batch, H, W, Ch, std=0.5), r(batch, H, W, Ch)
+    B, C = r(4, batch, H * W, N), r(4, batch, H * W, N)
+    if generic_A:
+        A = -(0.05 + 3 * torch.rand((4, Ch, N), generator=g))
+    else:
+        A = -torch.arange(1, N + 1, dtype=torch.float32).repeat(4, Ch, 1)
+    D = r(4, Ch)
+    s = torch.exp(np.log(1e-3) + (np.log(1e-1) - np.log(1e-3)) * torch.rand((4, Ch), generator=g, dtype=torch.float64))
+    bias = torch.log(torch.expm1(s)).float()
+    t = lambda x: x.to(dtype).contiguous()
+    return dict(u=t(u), delta=t(dr), z=t(z), B=t(B), C=t(C), A=A, D=D.contiguous(), bias=bias)
+
+
+def run_cross(vs, x, gate=True):
+    c = lambda t: t.cuda()
+    y = vs.vmamba_cross_scan4(c(x["u"]), c(x["delta"]), c(x["z"]) if gate else None, c(x["B"]),
+                              c(x["C"]), c(x["A"]), c(x["D"]), c(x["bias"]))
+    torch.cuda.synchronize()
+    return y
+
+
+def ref_cross(x, gate=True):
+    return oracle.cross_scan4(x["u"], x["delta"], x["z"] if gate else None, x["B"], x["C"], x["A"],
+                              x["D"], x["bias"])
+
+
+CROSS_CASES = [
+    # batch, H, W, C, N, dtype, generic_A, gate
+    (1, 1, 1, 8, 16, torch.float32, False, True),
+    (2, 3, 5, 64, 16, torch.float32, False, True),
+    (1, 5, 3, 72, 8, torch.bfloat16, True, True),
+    (2, 16, 16, 64, 16, torch.bfloat16, False, False),
+    (1, 7, 40, 64, 16, torch.float32, False, True),     # 280 tokens: several chunks
+    (1, 40, 7, 64, 4, torch.float32, True, True),
+    (2, 32, 48, 72, 16, torch.bfloat16, False, True),
+]
+
+
+@pytest.mark.parametrize("case", CROSS_CASES, ids=lambda c: f"b{c[0]}_{c[1]}x{c[2]}_C{c[3]}_N{c[4]}_{str(c[5])[6:]}"
+                         f"{'_genA' if c[6] else ''}{'' if c[7] else '_nogate'}")
+def test_cross_small(vs, case):
+    batch, H, W, Ch, N, dtype, gen, gate = case
+    x = cross_inputs(batch, H, W, Ch, N, dtype, seed=H * 100 + W, generic_A=gen)
+    check(f"cross_{case}", run_cross(vs, x, gate), ref_cross(x, gate), dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("hw", [(1, 1), (3, 5), (16, 16), (9, 33)])
+def test_merge(vs, dtype, hw):
+    H, W = hw
+    g = torch.Generator().manual_seed(H * W)
+    ys = torch.randn((4, 2, H * W, 24), generator=g).to(dtype)
+    z = torch.randn((2, H, W, 24), generator=g).to(dtype)
+    for zz in (None, z):
+        y = vs.cross_merge4(ys.cuda(), None if zz is None else zz.cuda(), H, W)
+        torch.cuda.synchronize()
+        check(f"merge_{hw}_{zz is not None}", y, oracle.cross_merge4(ys, zz, H, W), dtype)
+
+
+def test_merge_then_is_cross_scan(vs):
+    """The unfused path: four single-direction scans (each run as a pair's forward
+    half on its traversal) merged by cross_merge4 equal the fused cross-scan."""
+    x = cross_inputs(1, 6, 10, 64, 16, torch.float32, seed=77)
+    yfused = run_cross(vs, x)
+    H, W = 6, 10
+    ys = []
+    for k in range(4):
+        order = oracle.cross_order(k, H, W)
+        seq = lambda t: t.reshape(1, H * W, -1)[:, order].contiguous()
+        Bk, Ck = x["B"][k][:, order].contiguous(), x["C"][k][:, order].contiguous()
+        # a pair whose backward half sees B = C = 0 and D = 0 contributes nothing
+        Bp = torch.stack([Bk, torch.zeros_like(Bk)]).contiguous()
+        Cp = torch.stack([Ck, torch.zeros_like(Ck)]).contiguous()
+        A = torch.stack([x["A"][k], x["A"][k]]).contiguous()
+        D = torch.stack([x["D"][k], torch.zeros_like(x["D"][k])]).contiguous()
+        bias = torch.stack([x["bias"][k], x["bias"][k]]).contiguous()
+        yk = vs.vim_scan_bidir(seq(x["u"]).cuda(), seq(x["delta"]).cuda(), None, Bp.cuda(), Cp.cuda(),
+                               A.cuda(), D.cuda(), bias.cuda(), bc_dir_stride=Bk.numel())
+        ys.append(yk)
+    ym = vs.cross_merge4(torch.stack(ys).contiguous(), x["z"].cuda(), H, W)
+    torch.cuda.synchronize()
+    err = normwise(ym, yfused.double().cpu().numpy())
+    assert err < 1e-5, err
+
+
+@pytest.mark.parametrize("w", wl.WORKLOADS, ids=lambda w: w.name)
+def test_full_size(vs, w):
+    """Every workload at full size, in the launch configuration the benchmark
+    times, against the oracle on every output."""
+    x = wl.make_inputs(w)
+    oracle.set_threads(max(1, len(os.sched_getaffinity(0))))
+    dev = {k: v.cuda() for k, v in x.items()}
+    if w.kind == "vim":
+        y = vs.vim_scan_bidir(dev["u"], dev["delta"], dev["z"], dev["B"], dev["C"], dev["A"], dev["D"],
+                              dev["delta_bias"])
+        ref = oracle.vim_bidir(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"])
+    else:
+        y = vs.vmamba_cross_scan4(dev["u"], dev["delta"], dev["z"], dev["B"], dev["C"], dev["A"], dev["D"],
+                                  dev["delta_bias"])
+        ref = oracle.cross_scan4(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"])
+    torch.cuda.synchronize()
+    check(f"full_{w.name}", y, ref, w.torch_dtype())

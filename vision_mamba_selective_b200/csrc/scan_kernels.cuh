@@ -1,0 +1,643 @@
+// scan_kernels.cuh -- sm_100a kernels of the bidirectional selective scan (S6).
+//
+// The work unit is a "pair": two S6 directions that visit the same L positions in
+// opposite orders.  The Vim block (page "Vision Mamba Guide: Efficient Bidirectional
+// SSM & VMamba", section "2. The Bidirectional Mamba Block") is one pair over the
+// token order; the VMamba cross-scan (sections "1. Cross-Scan Traversal" to "3.
+// Cross-Merge Reversal") is two pairs, one over the row-major order and one over the
+// column-major order of the grid.
+//
+// A sequence of L tokens is cut into G chunks of up to `chunk` tokens.  One CTA owns
+// one chunk of 64 channels of one batch item and runs both directions of the pair
+// over it: warps 0-1 the forward direction (ascending), warps 2-3 the backward
+// direction (descending), one thread per (channel, direction) with all d_state
+// states of h in fp32 registers.  The chunk's inputs stream through shared memory in
+// tiles of 16 tokens (cp.async for u/delta, register prefetch + fp32 conversion for
+// B/C), double buffered.  The two directions meet in a per-chunk fp32 buffer of
+// partial outputs, and the summed, gated result is written once with 16-byte stores.
+//
+// For G > 1 the state entering each chunk comes from two small kernels: `pair_carry`
+// reduces every chunk to its end state from h = 0 plus its total Delta, and
+// `pair_combine` folds those summaries along each direction.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace vimscan {
+
+constexpr int kDC = 64;            // channels per CTA
+constexpr int kThreads = 2 * kDC;  // one thread per (channel, direction)
+constexpr int kTile = 16;          // tokens per staged tile
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ----------------------------------------------------------------------------
+// element types
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> struct Vec;           // 16-byte vector of T
+template <> struct Vec<float> { static constexpr int n = 4; };
+template <> struct Vec<__nv_bfloat16> { static constexpr int n = 8; };
+
+// 16 bytes of T -> 8 or 4 floats
+__device__ __forceinline__ void unpack16(const uint4 &v, float (&f)[4]) {
+    f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+}
+__device__ __forceinline__ void unpack16(const uint4 &v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ uint4 pack16(const float (&f)[4]) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                      __float_as_uint(f[3]));
+}
+__device__ __forceinline__ uint4 pack16(const float (&f)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 p = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t *>(&p);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// ----------------------------------------------------------------------------
+// math
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// softplus(x) = max(x, 0) + log1p(exp(-|x|)), and x itself above 20.  log1p(e) for
+// e in (0, 1] is evaluated as 2 atanh(s) with s = e / (2 + e) in (0, 1/3], through
+// the Taylor series of atanh up to s^13 (truncation error below 2e-8 relative).
+__device__ __forceinline__ float softplus(float x) {
+    const float e = ex2(-fabsf(x) * kLog2e);
+    const float s = e * rcp(2.0f + e);
+    const float s2 = s * s;
+    float p = fmaf(s2, 2.0f / 13.0f, 2.0f / 11.0f);
+    p = fmaf(s2, p, 2.0f / 9.0f);
+    p = fmaf(s2, p, 2.0f / 7.0f);
+    p = fmaf(s2, p, 2.0f / 5.0f);
+    p = fmaf(s2, p, 2.0f / 3.0f);
+    p = fmaf(s2, p, 2.0f);
+    const float r = fmaf(s, p, fmaxf(x, 0.0f));
+    return x > 20.0f ? x : r;
+}
+
+// silu(z) = z / (1 + exp(-z))
+__device__ __forceinline__ float silu(float z) { return z * rcp(1.0f + ex2(-z * kLog2e)); }
+
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+// a[k] = (q^(2k+1), q^(2k+2)), k < NP, by doubling blocks: depth log2(2 NP).
+template <int NP>
+__device__ __forceinline__ void powers2(float q, float2 (&a)[NP]) {
+    a[0] = f2(q, q * q);
+#pragma unroll
+    for (int m = 1; m < NP; m *= 2) {
+        const float2 step = f2(a[m - 1].y, a[m - 1].y);   // q^(2m)
+#pragma unroll
+        for (int j = 0; j < m && m + j < NP; ++j) a[m + j] = mul2(a[j], step);
+    }
+}
+
+// Reads of the fp32 B/C rows staged in shared memory, as pairs of states.
+template <int NP>
+__device__ __forceinline__ void load_row(const float *row, float2 (&v)[NP]) {
+    if constexpr (NP >= 2) {
+        const float4 *r4 = reinterpret_cast<const float4 *>(row);
+#pragma unroll
+        for (int k = 0; k < NP / 2; ++k) {
+            const float4 t = r4[k];
+            v[2 * k] = f2(t.x, t.y);
+            v[2 * k + 1] = f2(t.z, t.w);
+        }
+    } else {
+        v[0] = *reinterpret_cast<const float2 *>(row);
+    }
+}
+
+// ----------------------------------------------------------------------------
+// arguments
+// ----------------------------------------------------------------------------
+struct PairArgs {
+    const void *u, *delta, *z;      // [batch, L, Di] by position
+    const void *B[2], *C[2];        // per direction of the pair: [batch, L, N] by position
+    const float *A;                 // [2][Di][N]: forward, backward
+    const float *D;                 // [2][Di]
+    const float *bias;              // [2][Di]
+    void *y;                        // final output [batch, L, Di] (element type), or null
+    float *partial_out;             // fp32 [batch, L, Di] (ungated pair sum), or null
+    const float *partial_in;        // fp32 [batch, L, Di] added before the gate, or null
+    float *hloc;                    // [batch][G][2][Di][N] chunk summaries / carries
+    float *ssum;                    // [batch][G][2][Di]    chunk Delta sums
+    int batch, L, Di, H, W;
+    int order;                      // 0: position = step; 1: column-major on H x W
+    int chunk, G;                   // tokens per chunk (multiple of kTile), chunks
+};
+
+// position visited at step t of the forward direction
+__device__ __forceinline__ int position(const PairArgs &p, int t) {
+    if (p.order == 0) return t;
+    const int h = t % p.H, w = t / p.H;
+    return h * p.W + w;
+}
+
+// ----------------------------------------------------------------------------
+// shared-memory staging of one step: the forward tile and the backward tile
+// ----------------------------------------------------------------------------
+template <typename T, int N>
+struct Stage {
+    static constexpr int kUV = kTile * kDC;                  // elements per u or delta tile
+    static constexpr int kBC = kTile * N;                    // elements per B or C tile
+    // one slot: [dir][u|delta][kUV] T, then [dir][B|C][kBC] float
+    static constexpr int kSlotBytes = 2 * 2 * kUV * (int)sizeof(T) + 2 * 2 * kBC * 4;
+    static constexpr int kBCPerThread = (4 * kBC + kThreads - 1) / kThreads;
+
+    __device__ static T *uv(char *slot, int dir, int which) {
+        return reinterpret_cast<T *>(slot) + (dir * 2 + which) * kUV;
+    }
+    __device__ static float *bc(char *slot, int dir, int which) {
+        return reinterpret_cast<float *>(slot + 2 * 2 * kUV * sizeof(T)) + (dir * 2 + which) * kBC;
+    }
+};
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool valid) {
+    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    const int n = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::); }
+
+// Tile j of the chunk holds chunk tokens [j*kTile, j*kTile + rows).
+struct TileRef {
+    int j, rows;
+};
+
+template <typename T, int N>
+struct Stager {
+    using S = Stage<T, N>;
+    const PairArgs &p;
+    int b, t0, tc, d0;
+    float pre[S::kBCPerThread];   // B/C prefetch registers
+
+    __device__ Stager(const PairArgs &pa, int b_, int t0_, int tc_, int d0_)
+        : p(pa), b(b_), t0(t0_), tc(tc_), d0(d0_) {}
+
+    __device__ TileRef tile(int j) const {
+        const int rows = min(kTile, tc - j * kTile);
+        return {j, rows};
+    }
+
+    // u/delta of both tiles -> slot, asynchronously (zero-filled outside the data)
+    __device__ void issue_uv(char *slot, TileRef tf, TileRef tb) const {
+        constexpr int V = Vec<T>::n;
+        constexpr int per_row = kDC / V;
+        constexpr int pieces = 2 * 2 * kTile * per_row;
+        const T *src[2] = {static_cast<const T *>(p.u), static_cast<const T *>(p.delta)};
+        for (int i = threadIdx.x; i < pieces; i += kThreads) {
+            const int v = i % per_row;
+            const int r = (i / per_row) % kTile;
+            const int which = (i / (per_row * kTile)) % 2;
+            const int dir = i / (per_row * kTile * 2);
+            const TileRef t = dir ? tb : tf;
+            const int ch = d0 + v * V;
+            const bool ok = r < t.rows && ch < p.Di;
+            const T *g = src[which];
+            size_t off = 0;
+            if (ok) {
+                const int pos = position(p, t0 + t.j * kTile + r);
+                off = ((size_t)b * p.L + pos) * p.Di + ch;
+            }
+            T *dst = S::uv(slot, dir, which) + r * kDC + v * V;
+            cp_async16(dst, g + off, ok);
+        }
+        cp_async_commit();
+    }
+
+    // B/C of both tiles -> registers
+    __device__ void load_bc(TileRef tf, TileRef tb) {
+#pragma unroll
+        for (int k = 0; k < S::kBCPerThread; ++k) {
+            const int i = threadIdx.x + k * kThreads;
+            float v = 0.0f;
+            if (i < 4 * S::kBC) {
+                const int n = i % N;
+                const int r = (i / N) % kTile;
+                const int which = (i / (N * kTile)) % 2;
+                const int dir = i / (N * kTile * 2);
+                const TileRef t = dir ? tb : tf;
+                if (r < t.rows) {
+                    const int pos = position(p, t0 + t.j * kTile + r);
+                    const T *g = static_cast<const T *>(which ? p.C[dir] : p.B[dir]);
+                    v = to_f32(g[((size_t)b * p.L + pos) * N + n]);
+                }
+            }
+            pre[k] = v;
+        }
+    }
+
+    __device__ void store_bc(char *slot) const {
+#pragma unroll
+        for (int k = 0; k < S::kBCPerThread; ++k) {
+            const int i = threadIdx.x + k * kThreads;
+            if (i < 4 * S::kBC) {
+                const int n = i % N;
+                const int r = (i / N) % kTile;
+                const int which = (i / (N * kTile)) % 2;
+                const int dir = i / (N * kTile * 2);
+                S::bc(slot, dir, which)[r * N + n] = pre[k];
+            }
+        }
+    }
+};
+
+// ----------------------------------------------------------------------------
+// per-thread parameters of one (channel, direction)
+// ----------------------------------------------------------------------------
+template <int N>
+struct ChannelParams {
+    float A2[N];        // A[d][n] * log2(e)
+    float D, bias;
+    bool structured;    // A[d][n] == (n+1) A[d][0] for every n
+    bool valid;
+
+    __device__ void load(const PairArgs &p, int dir, int d) {
+        valid = d < p.Di;
+        structured = true;
+        D = 0.0f;
+        bias = 0.0f;
+#pragma unroll
+        for (int n = 0; n < N; ++n) A2[n] = 0.0f;
+        if (!valid) return;
+        const float *a = p.A + ((size_t)dir * p.Di + d) * N;
+        const float a0 = a[0];
+#pragma unroll
+        for (int n = 0; n < N; ++n) {
+            const float an = a[n];
+            structured = structured && (an == (float)(n + 1) * a0);
+            A2[n] = an * kLog2e;
+        }
+        D = p.D[(size_t)dir * p.Di + d];
+        bias = p.bias[(size_t)dir * p.Di + d];
+    }
+};
+
+// ----------------------------------------------------------------------------
+// kernel 1: chunk summaries (end state from h = 0, and the total Delta)
+// ----------------------------------------------------------------------------
+// Each direction walks its chunk in the reverse of its own visiting order and
+// accumulates H_n = sum_s exp(A_n * S_s) * Delta_s * u_s * B_sn, where S_s is the
+// Delta summed over the tokens the direction visits after s inside the chunk.  With
+// A_n = (n+1) A_0 the weights are powers of w = exp(A_0 S_s), built by one multiply
+// per state.
+template <typename T, int N>
+__global__ void __launch_bounds__(kThreads, 3) pair_carry(PairArgs p) {
+    using S = Stage<T, N>;
+    constexpr int NP = N / 2;
+    extern __shared__ __align__(16) char smem[];
+    char *slots[2] = {smem, smem + S::kSlotBytes};
+
+    const int b = blockIdx.z, c = blockIdx.y, d0 = blockIdx.x * kDC;
+    const int dir = threadIdx.x / kDC, dl = threadIdx.x % kDC, d = d0 + dl;
+    const int t0 = c * p.chunk, tc = min(p.chunk, p.L - t0);
+    const int nT = (tc + kTile - 1) / kTile;
+    // the forward summary of the last chunk and the backward one of the first are unused
+    const bool active = dir == 0 ? (c < p.G - 1) : (c > 0);
+
+    ChannelParams<N> prm;
+    prm.load(p, dir, d);
+    const bool fast = __all_sync(0xffffffffu, prm.structured);
+
+    Stager<T, N> st(p, b, t0, tc, d0);
+    // forward walks tiles nT-1 .. 0, backward walks 0 .. nT-1
+    auto tiles = [&](int s, TileRef &tf, TileRef &tb) {
+        tf = st.tile(nT - 1 - s);
+        tb = st.tile(s);
+    };
+    TileRef tf, tb;
+    tiles(0, tf, tb);
+    st.issue_uv(slots[0], tf, tb);
+    st.load_bc(tf, tb);
+    st.store_bc(slots[0]);
+    cp_async_wait_all();
+    __syncthreads();
+
+    float2 Hs[NP];
+#pragma unroll
+    for (int k = 0; k < NP; ++k) Hs[k] = f2(0.f, 0.f);
+    float Ssum = 0.0f;
+
+    for (int s = 0; s < nT; ++s) {
+        char *cur = slots[s & 1], *nxt = slots[(s + 1) & 1];
+        TileRef nf, nb;
+        if (s + 1 < nT) {
+            tiles(s + 1, nf, nb);
+            st.issue_uv(nxt, nf, nb);
+            st.load_bc(nf, nb);
+        }
+        tiles(s, tf, tb);
+        const TileRef me = dir ? tb : tf;
+        if (active && prm.valid) {
+            const T *su = S::uv(cur, dir, 0);
+            const T *sd = S::uv(cur, dir, 1);
+            const float *sB = S::bc(cur, dir, 0);
+            for (int i = 0; i < me.rows; ++i) {
+                const int r = dir ? i : me.rows - 1 - i;   // reverse of the visiting order
+                const float uu = to_f32(su[r * kDC + dl]);
+                const float dt = softplus(to_f32(sd[r * kDC + dl]) + prm.bias);
+                const float du = dt * uu;
+                float2 Bv[NP];
+                load_row<NP>(sB + r * N, Bv);
+                if (fast) {
+                    const float w = ex2(prm.A2[0] * Ssum);
+                    const float x0 = w * du;
+                    float2 x = f2(x0, x0 * w);
+                    const float2 w2 = f2(w * w, w * w);
+#pragma unroll
+                    for (int k = 0; k < NP; ++k) {
+                        Hs[k] = fma2(x, Bv[k], Hs[k]);
+                        x = mul2(x, w2);
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < NP; ++k) {
+                        const float2 wk = f2(ex2(prm.A2[2 * k] * Ssum), ex2(prm.A2[2 * k + 1] * Ssum));
+                        Hs[k] = fma2(mul2(wk, f2(du, du)), Bv[k], Hs[k]);
+                    }
+                }
+                Ssum += dt;
+            }
+        }
+        if (s + 1 < nT) {
+            st.store_bc(nxt);
+            cp_async_wait_all();
+        }
+        __syncthreads();
+    }
+
+    if (active && prm.valid) {
+        const size_t base = (((size_t)b * p.G + c) * 2 + dir) * p.Di + d;
+        float2 *out = reinterpret_cast<float2 *>(p.hloc + base * N);
+#pragma unroll
+        for (int k = 0; k < NP; ++k) out[k] = Hs[k];
+        p.ssum[base] = Ssum;
+    }
+}
+
+// ----------------------------------------------------------------------------
+// kernel 2: fold the chunk summaries along each direction
+// ----------------------------------------------------------------------------
+// hloc[b][c][dir][d][:] is replaced by the state entering chunk c in that
+// direction's visiting order: H_in(next) = exp(A_n * Ssum(c)) * H_in(c) + H_loc(c).
+template <int N>
+__global__ void __launch_bounds__(128) pair_combine(PairArgs p) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t total = (int64_t)p.batch * 2 * p.Di;
+    if (idx >= total) return;
+    const int d = (int)(idx % p.Di);
+    const int dir = (int)((idx / p.Di) % 2);
+    const int b = (int)(idx / (2 * p.Di));
+    ChannelParams<N> prm;
+    prm.load(p, dir, d);
+    float h[N];
+#pragma unroll
+    for (int n = 0; n < N; ++n) h[n] = 0.0f;
+    for (int i = 0; i < p.G; ++i) {
+        const int c = dir ? p.G - 1 - i : i;
+        const size_t base = (((size_t)b * p.G + c) * 2 + dir) * p.Di + d;
+        float *hl = p.hloc + base * N;
+        const float S = p.ssum[base];
+        float loc[N];
+#pragma unroll
+        for (int n = 0; n < N; ++n) loc[n] = hl[n];
+#pragma unroll
+        for (int n = 0; n < N; ++n) hl[n] = h[n];
+        if (i == p.G - 1) break;   // the last chunk's summary is never formed
+#pragma unroll
+        for (int n = 0; n < N; ++n) h[n] = fmaf(ex2(prm.A2[n] * S), h[n], loc[n]);
+    }
+}
+
+// acc (+)= V consecutive floats (16-byte aligned), V a multiple of 4
+template <int V, bool ADD>
+__device__ __forceinline__ void add_f32(float (&acc)[V], const float *src) {
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+    for (int q = 0; q < V / 4; ++q) {
+        const float4 a = s4[q];
+        if (ADD) {
+            acc[4 * q] += a.x; acc[4 * q + 1] += a.y; acc[4 * q + 2] += a.z; acc[4 * q + 3] += a.w;
+        } else {
+            acc[4 * q] = a.x; acc[4 * q + 1] = a.y; acc[4 * q + 2] = a.z; acc[4 * q + 3] = a.w;
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------
+// kernel 3: both directions over one chunk, merge, gate, store
+// ----------------------------------------------------------------------------
+template <typename T, int N>
+__global__ void __launch_bounds__(kThreads, 3) pair_main(PairArgs p) {
+    using S = Stage<T, N>;
+    constexpr int NP = N / 2;
+    extern __shared__ __align__(16) char smem[];
+    char *slots[2] = {smem, smem + S::kSlotBytes};
+    float *ybuf = reinterpret_cast<float *>(smem + 2 * S::kSlotBytes);   // [chunk][kDC]
+    float *ymid = ybuf + (size_t)p.chunk * kDC;                          // [kTile][kDC]
+
+    const int b = blockIdx.z, c = blockIdx.y, d0 = blockIdx.x * kDC;
+    const int dir = threadIdx.x / kDC, dl = threadIdx.x % kDC, d = d0 + dl;
+    const int t0 = c * p.chunk, tc = min(p.chunk, p.L - t0);
+    const int nT = (tc + kTile - 1) / kTile;
+
+    ChannelParams<N> prm;
+    prm.load(p, dir, d);
+    const bool fast = __all_sync(0xffffffffu, prm.structured);
+
+    // state entering this chunk
+    float2 h[NP];
+    const bool has_carry = p.G > 1 && (dir == 0 ? c > 0 : c < p.G - 1);
+    if (has_carry && prm.valid) {
+        const size_t base = (((size_t)b * p.G + c) * 2 + dir) * p.Di + d;
+        const float2 *hin = reinterpret_cast<const float2 *>(p.hloc + base * N);
+#pragma unroll
+        for (int k = 0; k < NP; ++k) h[k] = hin[k];
+    } else {
+#pragma unroll
+        for (int k = 0; k < NP; ++k) h[k] = f2(0.f, 0.f);
+    }
+
+    Stager<T, N> st(p, b, t0, tc, d0);
+    TileRef tf = st.tile(0), tb = st.tile(nT - 1);
+    st.issue_uv(slots[0], tf, tb);
+    st.load_bc(tf, tb);
+    st.store_bc(slots[0]);
+    cp_async_wait_all();
+    __syncthreads();
+
+    for (int s = 0; s < nT; ++s) {
+        char *cur = slots[s & 1], *nxt = slots[(s + 1) & 1];
+        if (s + 1 < nT) {
+            const TileRef nf = st.tile(s + 1), nb = st.tile(nT - 2 - s);
+            st.issue_uv(nxt, nf, nb);
+            st.load_bc(nf, nb);
+        }
+        const TileRef me = dir ? st.tile(nT - 1 - s) : st.tile(s);
+        // the forward direction visits tile j at step j, the backward one at nT-1-j
+        const int twice = 2 * s - (nT - 1);   // < 0 first visit, 0 both at once, > 0 second
+        if (prm.valid) {
+            const T *su = S::uv(cur, dir, 0);
+            const T *sd = S::uv(cur, dir, 1);
+            const float *sB = S::bc(cur, dir, 0);
+            const float *sC = S::bc(cur, dir, 1);
+            for (int i = 0; i < me.rows; ++i) {
+                const int r = dir ? me.rows - 1 - i : i;
+                const float uu = to_f32(su[r * kDC + dl]);
+                const float dt = softplus(to_f32(sd[r * kDC + dl]) + prm.bias);
+                const float du = dt * uu;
+                float2 a[NP];
+                if (fast) {
+                    powers2<NP>(ex2(dt * prm.A2[0]), a);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < NP; ++k)
+                        a[k] = f2(ex2(dt * prm.A2[2 * k]), ex2(dt * prm.A2[2 * k + 1]));
+                }
+                float2 Bv[NP], Cv[NP];
+                load_row<NP>(sB + r * N, Bv);
+                load_row<NP>(sC + r * N, Cv);
+                const float2 du2 = f2(du, du);
+                float2 y0 = f2(0.f, 0.f), y1 = f2(0.f, 0.f);
+#pragma unroll
+                for (int k = 0; k < NP; ++k) {
+                    h[k] = fma2(a[k], h[k], mul2(du2, Bv[k]));
+                    if (k & 1) y1 = fma2(Cv[k], h[k], y1);
+                    else y0 = fma2(Cv[k], h[k], y0);
+                }
+                const float yv = fmaf(prm.D, uu, (y0.x + y0.y) + (y1.x + y1.y));
+                const int tl = me.j * kTile + r;
+                if (twice < 0) {
+                    ybuf[tl * kDC + dl] = yv;
+                } else if (twice == 0) {
+                    if (dir == 0) ybuf[tl * kDC + dl] = yv;
+                    else ymid[r * kDC + dl] = yv;
+                } else {
+                    ybuf[tl * kDC + dl] += yv;
+                }
+            }
+        }
+        if (s + 1 < nT) {
+            st.store_bc(nxt);
+            cp_async_wait_all();
+        }
+        __syncthreads();
+    }
+
+    // merge the middle tile (both directions wrote it in the same step), gate, store:
+    // one item = one 16-byte vector of output channels
+    constexpr int V = Vec<T>::n;
+    constexpr int per_row = kDC / V;
+    const int mid_tile = (nT & 1) ? (nT - 1) / 2 : -1;
+    for (int i = threadIdx.x; i < tc * per_row; i += kThreads) {
+        const int v = i % per_row, tl = i / per_row;
+        const int ch = d0 + v * V;
+        if (ch >= p.Di) continue;   // Di is a multiple of V: the vector is whole or absent
+        float acc[V];
+        add_f32<V, false>(acc, ybuf + tl * kDC + v * V);
+        if (tl / kTile == mid_tile) add_f32<V, true>(acc, ymid + (tl % kTile) * kDC + v * V);
+        const int pos = position(p, t0 + tl);
+        const size_t off = ((size_t)b * p.L + pos) * p.Di + ch;
+        if (p.partial_in) add_f32<V, true>(acc, p.partial_in + off);
+        if (p.partial_out) {
+            float4 *po = reinterpret_cast<float4 *>(p.partial_out + off);
+#pragma unroll
+            for (int q = 0; q < V / 4; ++q)
+                po[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+            continue;
+        }
+        if (p.z) {
+            float zf[V];
+            unpack16(*reinterpret_cast<const uint4 *>(static_cast<const T *>(p.z) + off), zf);
+#pragma unroll
+            for (int e = 0; e < V; ++e) acc[e] *= silu(zf[e]);
+        }
+        *reinterpret_cast<uint4 *>(static_cast<T *>(p.y) + off) = pack16(acc);
+    }
+}
+
+// ----------------------------------------------------------------------------
+// CS-Merge alone
+// ----------------------------------------------------------------------------
+struct MergeArgs {
+    const void *ys;   // [4][batch][L][C] in scan order
+    const void *z;    // [batch][L][C] or null
+    void *y;          // [batch][L][C]
+    int batch, H, W, C;
+};
+
+// scan step at which direction k visits grid position pos
+__device__ __forceinline__ int merge_step(int k, int pos, int H, int W) {
+    const int L = H * W;
+    if (k < 2) return k == 0 ? pos : L - 1 - pos;
+    const int h = pos / W, w = pos % W;
+    const int t = w * H + h;
+    return k == 2 ? t : L - 1 - t;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) merge4(MergeArgs a) {
+    constexpr int V = Vec<T>::n;
+    const int per_row = a.C / V;
+    const int L = a.H * a.W;
+    const int64_t items = (int64_t)a.batch * L * per_row;
+    const T *ys = static_cast<const T *>(a.ys);
+    const size_t dir_stride = (size_t)a.batch * L * a.C;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < items;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int v = (int)(i % per_row);
+        const int64_t bp = i / per_row;
+        const int pos = (int)(bp % L);
+        const int b = (int)(bp / L);
+        float acc[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int t = merge_step(k, pos, a.H, a.W);
+            float f[V];
+            unpack16(*reinterpret_cast<const uint4 *>(ys + k * dir_stride + ((size_t)b * L + t) * a.C + v * V), f);
+#pragma unroll
+            for (int e = 0; e < V; ++e) acc[e] += f[e];
+        }
+        const size_t off = ((size_t)b * L + pos) * a.C + v * V;
+        if (a.z) {
+            float zf[V];
+            unpack16(*reinterpret_cast<const uint4 *>(static_cast<const T *>(a.z) + off), zf);
+#pragma unroll
+            for (int e = 0; e < V; ++e) acc[e] *= silu(zf[e]);
+        }
+        *reinterpret_cast<uint4 *>(static_cast<T *>(a.y) + off) = pack16(acc);
+    }
+}
+
+}  // namespace vimscan

@@ -1,0 +1,295 @@
+// vimscan.cu -- host side of libvimscan.so: argument checks, planning, launches.
+//
+// Entry points are declared (with their contracts) in include/vimscan.h.  Every
+// check runs on the host before the first launch; nothing here allocates memory or
+// synchronises the stream.
+#include "vimscan.h"
+
+#include <cstdint>
+#include <cstring>
+
+#include "scan_kernels.cuh"
+
+namespace vimscan {
+namespace {
+
+constexpr int kSingleChunkMax = 256;   // sequences up to this length run as one chunk
+constexpr int kLongChunk = 128;        // chunk length otherwise (a multiple of kTile)
+constexpr size_t kAlign = 256;
+
+struct Plan {
+    int chunk;  // tokens per chunk (multiple of kTile)
+    int G;      // chunks
+};
+
+Plan plan_for(int L) {
+    Plan pl;
+    if (L <= kSingleChunkMax) {
+        pl.chunk = ((L + kTile - 1) / kTile) * kTile;
+        if (pl.chunk == 0) pl.chunk = kTile;
+        pl.G = 1;
+    } else {
+        pl.chunk = kLongChunk;
+        pl.G = (L + kLongChunk - 1) / kLongChunk;
+    }
+    return pl;
+}
+
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// summaries for one pair: hloc [batch][G][2][Di][N] + ssum [batch][G][2][Di]
+size_t summary_bytes(int batch, int L, int Di, int N) {
+    const Plan pl = plan_for(L);
+    if (pl.G <= 1) return 0;
+    const size_t units = (size_t)batch * pl.G * 2 * Di;
+    return round_up(units * N * sizeof(float)) + round_up(units * sizeof(float));
+}
+
+bool supported_state(int N) { return N == 2 || N == 4 || N == 8 || N == 16; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t elem_size(vim_dtype dt) { return dt == VIM_F32 ? 4 : 2; }
+
+vim_status check_common(int batch, int L, int Di, int N, vim_dtype dt) {
+    if (batch < 0 || L < 0 || Di < 0 || N < 0) return VIM_ERR_INVALID_ARG;
+    if (dt != VIM_F32 && dt != VIM_BF16) return VIM_ERR_INVALID_ARG;
+    if (!supported_state(N)) return VIM_ERR_UNSUPPORTED;
+    if (Di % (dt == VIM_F32 ? 4 : 8) != 0) return VIM_ERR_UNSUPPORTED;
+    if ((int64_t)batch * L * Di > INT32_MAX || (int64_t)batch * L * N > INT32_MAX)
+        return VIM_ERR_UNSUPPORTED;
+    return VIM_OK;
+}
+
+template <typename T, int N>
+size_t main_smem(int chunk) {
+    return 2 * (size_t)Stage<T, N>::kSlotBytes + (size_t)chunk * kDC * 4 + (size_t)kTile * kDC * 4;
+}
+template <typename T, int N>
+size_t carry_smem() {
+    return 2 * (size_t)Stage<T, N>::kSlotBytes;
+}
+
+// events: null, or 3 events recorded after the carry, combine and main kernels
+inline vim_status mark(cudaEvent_t *events, int i, cudaStream_t stream) {
+    if (!events) return VIM_OK;
+    return cudaEventRecord(events[i], stream) == cudaSuccess ? VIM_OK : VIM_ERR_CUDA;
+}
+
+template <typename T, int N>
+vim_status launch_pair_t(PairArgs a, cudaStream_t stream, cudaEvent_t *ev) {
+    const dim3 grid((a.Di + kDC - 1) / kDC, a.G, a.batch);
+    if (a.G > 1) {
+        const size_t sc = carry_smem<T, N>();
+        if (cudaFuncSetAttribute(pair_carry<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sc) != cudaSuccess)
+            return VIM_ERR_CUDA;
+        pair_carry<T, N><<<grid, kThreads, sc, stream>>>(a);
+        if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+        const int64_t units = (int64_t)a.batch * 2 * a.Di;
+        if (mark(ev, 0, stream) != VIM_OK) return VIM_ERR_CUDA;
+        pair_combine<N><<<(unsigned)((units + 127) / 128), 128, 0, stream>>>(a);
+        if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+        if (mark(ev, 1, stream) != VIM_OK) return VIM_ERR_CUDA;
+    } else if (ev) {
+        if (mark(ev, 0, stream) != VIM_OK || mark(ev, 1, stream) != VIM_OK) return VIM_ERR_CUDA;
+    }
+    const size_t sm = main_smem<T, N>(a.chunk);
+    if (cudaFuncSetAttribute(pair_main<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
+        cudaSuccess)
+        return VIM_ERR_CUDA;
+    pair_main<T, N><<<grid, kThreads, sm, stream>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+    return mark(ev, 2, stream);
+}
+
+template <typename T>
+vim_status launch_pair_n(PairArgs a, int N, cudaStream_t stream, cudaEvent_t *ev) {
+    switch (N) {
+        case 2: return launch_pair_t<T, 2>(a, stream, ev);
+        case 4: return launch_pair_t<T, 4>(a, stream, ev);
+        case 8: return launch_pair_t<T, 8>(a, stream, ev);
+        case 16: return launch_pair_t<T, 16>(a, stream, ev);
+        default: return VIM_ERR_UNSUPPORTED;
+    }
+}
+
+vim_status launch_pair(PairArgs a, int N, vim_dtype dt, cudaStream_t stream, cudaEvent_t *ev) {
+    return dt == VIM_F32 ? launch_pair_n<float>(a, N, stream, ev)
+                         : launch_pair_n<__nv_bfloat16>(a, N, stream, ev);
+}
+
+}  // namespace
+}  // namespace vimscan
+
+using namespace vimscan;
+
+extern "C" {
+
+const char *vim_status_string(vim_status s) {
+    switch (s) {
+        case VIM_OK: return "ok";
+        case VIM_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, or negative size)";
+        case VIM_ERR_UNSUPPORTED: return "unsupported size (d_state or channel count)";
+        case VIM_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case VIM_ERR_CUDA: return "CUDA launch failed";
+        case VIM_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+        default: return "unknown status";
+    }
+}
+
+size_t vim_scan_workspace_bytes(int which, int batch, int L_or_H, int W, int channels, int d_state) {
+    if (batch < 0 || L_or_H < 0 || channels < 0 || !supported_state(d_state)) return 0;
+    if (which == 0) return summary_bytes(batch, L_or_H, channels, d_state);
+    if (which == 1) {
+        if (W < 0) return 0;
+        const int L = L_or_H * W;
+        const size_t partial = round_up((size_t)batch * L * channels * sizeof(float));
+        return summary_bytes(batch, L, channels, d_state) + partial;
+    }
+    return 0;
+}
+
+vim_status vim_scan_bidir_events(const void *u, const void *delta, const void *z, const void *B,
+                                 const void *C, int64_t bc_dir_stride, const float *A,
+                                 const float *D, const float *delta_bias, void *y, int batch, int L,
+                                 int d_inner, int d_state, vim_dtype dt, void *workspace,
+                                 size_t workspace_bytes, cudaStream_t stream, cudaEvent_t *events) {
+    vim_status st = check_common(batch, L, d_inner, d_state, dt);
+    if (st != VIM_OK) return st;
+    if (bc_dir_stride < 0) return VIM_ERR_INVALID_ARG;
+    if (batch == 0 || L == 0 || d_inner == 0) return VIM_OK;
+    if (!u || !delta || !B || !C || !A || !D || !delta_bias || !y) return VIM_ERR_INVALID_ARG;
+    if (!aligned16(u) || !aligned16(delta) || !aligned16(y) || (z && !aligned16(z)))
+        return VIM_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(B) | reinterpret_cast<uintptr_t>(C)) % elem_size(dt))
+        return VIM_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(D) |
+         reinterpret_cast<uintptr_t>(delta_bias)) % 4)
+        return VIM_ERR_INVALID_ARG;
+    const size_t need = summary_bytes(batch, L, d_inner, d_state);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need) return VIM_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return VIM_ERR_WORKSPACE;
+    }
+    const Plan pl = plan_for(L);
+    PairArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.u = u; a.delta = delta; a.z = z;
+    const char *Bc = static_cast<const char *>(B), *Cc = static_cast<const char *>(C);
+    a.B[0] = B; a.C[0] = C;
+    a.B[1] = Bc + bc_dir_stride * (int64_t)elem_size(dt);
+    a.C[1] = Cc + bc_dir_stride * (int64_t)elem_size(dt);
+    a.A = A; a.D = D; a.bias = delta_bias;
+    a.y = y;
+    a.batch = batch; a.L = L; a.Di = d_inner; a.H = 1; a.W = L; a.order = 0;
+    a.chunk = pl.chunk; a.G = pl.G;
+    if (pl.G > 1) {
+        const size_t units = (size_t)batch * pl.G * 2 * d_inner;
+        a.hloc = static_cast<float *>(workspace);
+        a.ssum = reinterpret_cast<float *>(static_cast<char *>(workspace) + round_up(units * d_state * 4));
+    }
+    if (mark(events, 0, stream) != VIM_OK) return VIM_ERR_CUDA;
+    return launch_pair(a, d_state, dt, stream, events ? events + 1 : nullptr);
+}
+
+vim_status vim_scan_bidir(const void *u, const void *delta, const void *z, const void *B,
+                          const void *C, int64_t bc_dir_stride, const float *A, const float *D,
+                          const float *delta_bias, void *y, int batch, int L, int d_inner,
+                          int d_state, vim_dtype dt, void *workspace, size_t workspace_bytes,
+                          cudaStream_t stream) {
+    return vim_scan_bidir_events(u, delta, z, B, C, bc_dir_stride, A, D, delta_bias, y, batch, L,
+                                 d_inner, d_state, dt, workspace, workspace_bytes, stream, nullptr);
+}
+
+vim_status vmamba_cross_scan4_events(const void *u, const void *delta, const void *z,
+                                     const void *B, const void *C, const float *A, const float *D,
+                                     const float *delta_bias, void *y, int batch, int H, int W,
+                                     int channels, int d_state, vim_dtype dt, void *workspace,
+                                     size_t workspace_bytes, cudaStream_t stream,
+                                     cudaEvent_t *events) {
+    if (H < 0 || W < 0) return VIM_ERR_INVALID_ARG;
+    if ((int64_t)H * W > INT32_MAX) return VIM_ERR_UNSUPPORTED;
+    const int L = H * W;
+    vim_status st = check_common(batch, L, channels, d_state, dt);
+    if (st != VIM_OK) return st;
+    if (batch == 0 || L == 0 || channels == 0) return VIM_OK;
+    if (!u || !delta || !B || !C || !A || !D || !delta_bias || !y) return VIM_ERR_INVALID_ARG;
+    if (!aligned16(u) || !aligned16(delta) || !aligned16(y) || (z && !aligned16(z)))
+        return VIM_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(B) | reinterpret_cast<uintptr_t>(C)) % elem_size(dt))
+        return VIM_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(D) |
+         reinterpret_cast<uintptr_t>(delta_bias)) % 4)
+        return VIM_ERR_INVALID_ARG;
+    const size_t sum_b = summary_bytes(batch, L, channels, d_state);
+    const size_t need = sum_b + round_up((size_t)batch * L * channels * sizeof(float));
+    if (!workspace || workspace_bytes < need) return VIM_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return VIM_ERR_WORKSPACE;
+
+    const Plan pl = plan_for(L);
+    float *partial = reinterpret_cast<float *>(static_cast<char *>(workspace) + sum_b);
+    const size_t el = elem_size(dt);
+    const size_t bc_dir = (size_t)batch * L * d_state * el;   // bytes between directions
+    if (mark(events, 0, stream) != VIM_OK) return VIM_ERR_CUDA;
+    vim_status rc = VIM_OK;
+    for (int pair = 0; pair < 2 && rc == VIM_OK; ++pair) {
+        PairArgs a;
+        std::memset(&a, 0, sizeof(a));
+        a.u = u; a.delta = delta; a.z = z;
+        for (int k = 0; k < 2; ++k) {
+            a.B[k] = static_cast<const char *>(B) + (2 * pair + k) * bc_dir;
+            a.C[k] = static_cast<const char *>(C) + (2 * pair + k) * bc_dir;
+        }
+        a.A = A + (size_t)2 * pair * channels * d_state;
+        a.D = D + (size_t)2 * pair * channels;
+        a.bias = delta_bias + (size_t)2 * pair * channels;
+        a.batch = batch; a.L = L; a.Di = channels; a.H = H; a.W = W;
+        a.order = pair;               // pair 0: scans 1/2 (rows), pair 1: scans 3/4 (columns)
+        a.chunk = pl.chunk; a.G = pl.G;
+        if (pl.G > 1) {
+            const size_t units = (size_t)batch * pl.G * 2 * channels;
+            a.hloc = static_cast<float *>(workspace);
+            a.ssum = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                               round_up(units * d_state * 4));
+        }
+        if (pair == 0) {
+            a.partial_out = partial;
+        } else {
+            a.partial_in = partial;
+            a.y = y;
+        }
+        rc = launch_pair(a, d_state, dt, stream, events ? events + 1 + 3 * pair : nullptr);
+    }
+    return rc;
+}
+
+vim_status vmamba_cross_scan4(const void *u, const void *delta, const void *z, const void *B,
+                              const void *C, const float *A, const float *D,
+                              const float *delta_bias, void *y, int batch, int H, int W,
+                              int channels, int d_state, vim_dtype dt, void *workspace,
+                              size_t workspace_bytes, cudaStream_t stream) {
+    return vmamba_cross_scan4_events(u, delta, z, B, C, A, D, delta_bias, y, batch, H, W, channels,
+                                     d_state, dt, workspace, workspace_bytes, stream, nullptr);
+}
+
+vim_status cross_merge4(const void *ys, const void *z, void *y, int batch, int H, int W, int channels,
+                        vim_dtype dt, cudaStream_t stream) {
+    if (batch < 0 || H < 0 || W < 0 || channels < 0) return VIM_ERR_INVALID_ARG;
+    if (dt != VIM_F32 && dt != VIM_BF16) return VIM_ERR_INVALID_ARG;
+    if (channels % (dt == VIM_F32 ? 4 : 8) != 0) return VIM_ERR_UNSUPPORTED;
+    if ((int64_t)H * W > INT32_MAX || (int64_t)batch * H * W * channels * 4 > INT32_MAX * (int64_t)4)
+        return VIM_ERR_UNSUPPORTED;
+    if (batch == 0 || H == 0 || W == 0 || channels == 0) return VIM_OK;
+    if (!ys || !y) return VIM_ERR_INVALID_ARG;
+    if (!aligned16(ys) || !aligned16(y) || (z && !aligned16(z))) return VIM_ERR_INVALID_ARG;
+    MergeArgs a{ys, z, y, batch, H, W, channels};
+    const int64_t items = (int64_t)batch * H * W * (channels / (dt == VIM_F32 ? 4 : 8));
+    int blocks = (int)((items + 255) / 256);
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (dt == VIM_F32)
+        merge4<float><<<blocks, 256, 0, stream>>>(a);
+    else
+        merge4<__nv_bfloat16><<<blocks, 256, 0, stream>>>(a);
+    return cudaGetLastError() == cudaSuccess ? VIM_OK : VIM_ERR_CUDA;
+}
+
+}  // extern "C"

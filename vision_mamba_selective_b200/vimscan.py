@@ -1,0 +1,172 @@
+"""Thin ctypes binding of libvimscan.so (declared in include/vimscan.h).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, turned into raw device pointers and handed to the C ABI together with
+the current torch CUDA stream.  Every step of the scan runs in the library's sm_100a
+kernels; there is no fallback of any kind, and a missing library is an ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libvimscan.so")
+
+VIM_OK, VIM_ERR_INVALID_ARG, VIM_ERR_UNSUPPORTED, VIM_ERR_WORKSPACE, VIM_ERR_CUDA, VIM_ERR_TIMEOUT = range(6)
+VIM_F32, VIM_BF16 = 0, 1
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m vision_mamba_selective_b200.build` "
+        "(nvcc, sm_100a); the selective scan has no other implementation")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _i, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+lib.vim_scan_bidir.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
+                               _i, _i, _i, _i, _i, _vp, _sz, _vp]
+lib.vim_scan_bidir.restype = _i
+lib.vmamba_cross_scan4.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                   _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
+lib.vmamba_cross_scan4.restype = _i
+lib.vim_scan_bidir_events.argtypes = lib.vim_scan_bidir.argtypes + [_vp]
+lib.vim_scan_bidir_events.restype = _i
+lib.vmamba_cross_scan4_events.argtypes = lib.vmamba_cross_scan4.argtypes + [_vp]
+lib.vmamba_cross_scan4_events.restype = _i
+lib.cross_merge4.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
+lib.cross_merge4.restype = _i
+lib.vim_scan_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
+lib.vim_scan_workspace_bytes.restype = _sz
+lib.vim_status_string.argtypes = [_i]
+lib.vim_status_string.restype = ctypes.c_char_p
+
+
+class VimScanError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+def status_string(status: int) -> str:
+    return lib.vim_status_string(int(status)).decode()
+
+
+def vim_scan_workspace_bytes(which: int, batch: int, L_or_H: int, W: int, channels: int, d_state: int) -> int:
+    return int(lib.vim_scan_workspace_bytes(which, batch, L_or_H, W, channels, d_state))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return VIM_F32
+    if t.dtype == torch.bfloat16:
+        return VIM_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}: fp32 or bf16")
+
+
+def _ptr(t, *, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _workspace(nbytes, workspace, device):
+    if nbytes == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    if workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace too small: need {nbytes} bytes")
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def _events(events):
+    """Raw cudaEvent_t handles of torch CUDA events (created by recording them once)."""
+    handles = []
+    for e in events:
+        if e.cuda_event == 0:
+            e.record()
+        handles.append(e.cuda_event)
+    return (ctypes.c_void_p * len(handles))(*handles)
+
+
+def vim_scan_bidir(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride=0,
+                   workspace=None, stream=None, events=None):
+    """Vim bidirectional selective scan, (y^f + y^b) * silu(z); see include/vimscan.h.
+
+    u, delta, z: [batch, L, d_inner]; B, C: [batch, L, d_state] (or a larger buffer
+    whose backward copy starts ``bc_dir_stride`` elements in); A: [2, d_inner,
+    d_state] fp32; D, delta_bias: [2, d_inner] fp32.  Returns y [batch, L, d_inner].
+    """
+    batch, L, Di = u.shape
+    N = B.shape[-1]
+    dt = _dtype_code(u)
+    if y is None:
+        y = torch.empty_like(u)
+    ws, ws_bytes = _workspace(vim_scan_workspace_bytes(0, batch, L, 0, Di, N), workspace, u.device)
+    extra = () if events is None else (_events(events),)
+    fn = lib.vim_scan_bidir if events is None else lib.vim_scan_bidir_events
+    st = fn(
+        _ptr(u, name="u"), _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
+        _ptr(B, dtype=u.dtype, name="B"), _ptr(C, dtype=u.dtype, name="C"), int(bc_dir_stride),
+        _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
+        _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(y, dtype=u.dtype, name="y"),
+        batch, L, Di, N, dt, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream), *extra)
+    if st != VIM_OK:
+        raise VimScanError(st, "vim_scan_bidir")
+    return y
+
+
+def vmamba_cross_scan4(u, delta, z, B, C, A, D, delta_bias, *, y=None, workspace=None, stream=None,
+                       events=None):
+    """VMamba four-direction cross-scan with CS-Merge; see include/vimscan.h.
+
+    u, delta, z: [batch, H, W, C]; B, C: [4, batch, H*W, d_state] by grid position;
+    A: [4, C, d_state] fp32; D, delta_bias: [4, C] fp32.  Returns y [batch, H, W, C].
+    """
+    batch, H, W, Ch = u.shape
+    N = B.shape[-1]
+    dt = _dtype_code(u)
+    if y is None:
+        y = torch.empty_like(u)
+    ws, ws_bytes = _workspace(vim_scan_workspace_bytes(1, batch, H, W, Ch, N), workspace, u.device)
+    extra = () if events is None else (_events(events),)
+    fn = lib.vmamba_cross_scan4 if events is None else lib.vmamba_cross_scan4_events
+    st = fn(
+        _ptr(u, name="u"), _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
+        _ptr(B, dtype=u.dtype, name="B"), _ptr(C, dtype=u.dtype, name="C"),
+        _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
+        _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(y, dtype=u.dtype, name="y"),
+        batch, H, W, Ch, N, dt, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream), *extra)
+    if st != VIM_OK:
+        raise VimScanError(st, "vmamba_cross_scan4")
+    return y
+
+
+def cross_merge4(ys, z, H, W, *, y=None, stream=None):
+    """CS-Merge alone: ys [4, batch, H*W, C] in scan order -> y [batch, H, W, C]."""
+    _, batch, L, Ch = ys.shape
+    if L != H * W:
+        raise ValueError("ys.shape[2] must be H*W")
+    dt = _dtype_code(ys)
+    if y is None:
+        y = torch.empty((batch, H, W, Ch), dtype=ys.dtype, device=ys.device)
+    st = lib.cross_merge4(_ptr(ys, name="ys"), _ptr(z, dtype=ys.dtype, name="z"),
+                          _ptr(y, dtype=ys.dtype, name="y"), batch, H, W, Ch, dt, _stream(stream))
+    if st != VIM_OK:
+        raise VimScanError(st, "cross_merge4")
+    return y
