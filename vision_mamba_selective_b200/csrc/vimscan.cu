@@ -74,35 +74,46 @@ inline vim_status mark(cudaEvent_t *events, int i, cudaStream_t stream) {
     return cudaEventRecord(events[i], stream) == cudaSuccess ? VIM_OK : VIM_ERR_CUDA;
 }
 
-template <typename T, int N>
-vim_status launch_pair_t(PairArgs a, cudaStream_t stream, cudaEvent_t *ev) {
+template <typename T, int N, bool VEC_BC>
+vim_status launch_pair_v(const PairArgs &a, cudaStream_t stream, cudaEvent_t *ev) {
     const dim3 grid((a.Di + kDC - 1) / kDC, a.G, a.batch);
     if (a.G > 1) {
         const size_t sc = carry_smem<T, N>();
-        if (cudaFuncSetAttribute(pair_carry<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(pair_carry<T, N, VEC_BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sc) != cudaSuccess)
             return VIM_ERR_CUDA;
-        pair_carry<T, N><<<grid, kThreads, sc, stream>>>(a);
+        pair_carry<T, N, VEC_BC><<<grid, kThreads, sc, stream>>>(a);
         if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
-        const int64_t units = (int64_t)a.batch * 2 * a.Di;
         if (mark(ev, 0, stream) != VIM_OK) return VIM_ERR_CUDA;
-        pair_combine<N><<<(unsigned)((units + 127) / 128), 128, 0, stream>>>(a);
+        const int64_t units = (int64_t)a.batch * 2 * a.Di * N;
+        pair_combine<N><<<(unsigned)((units + 255) / 256), 256, 0, stream>>>(a);
         if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
         if (mark(ev, 1, stream) != VIM_OK) return VIM_ERR_CUDA;
     } else if (ev) {
         if (mark(ev, 0, stream) != VIM_OK || mark(ev, 1, stream) != VIM_OK) return VIM_ERR_CUDA;
     }
     const size_t sm = main_smem<T, N>(a.chunk);
-    if (cudaFuncSetAttribute(pair_main<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(pair_main<T, N, VEC_BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sm) != cudaSuccess)
         return VIM_ERR_CUDA;
-    pair_main<T, N><<<grid, kThreads, sm, stream>>>(a);
+    pair_main<T, N, VEC_BC><<<grid, kThreads, sm, stream>>>(a);
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     return mark(ev, 2, stream);
 }
 
+// B/C move as 16-byte vectors when their rows allow it and every base is aligned
+template <typename T, int N>
+vim_status launch_pair_t(const PairArgs &a, cudaStream_t stream, cudaEvent_t *ev) {
+    if constexpr (bc_vectorizable<T, N>()) {
+        const bool aligned = aligned16(a.B[0]) && aligned16(a.B[1]) && aligned16(a.C[0]) &&
+                             aligned16(a.C[1]);
+        if (aligned) return launch_pair_v<T, N, true>(a, stream, ev);
+    }
+    return launch_pair_v<T, N, false>(a, stream, ev);
+}
+
 template <typename T>
-vim_status launch_pair_n(PairArgs a, int N, cudaStream_t stream, cudaEvent_t *ev) {
+vim_status launch_pair_n(const PairArgs &a, int N, cudaStream_t stream, cudaEvent_t *ev) {
     switch (N) {
         case 2: return launch_pair_t<T, 2>(a, stream, ev);
         case 4: return launch_pair_t<T, 4>(a, stream, ev);
@@ -112,7 +123,7 @@ vim_status launch_pair_n(PairArgs a, int N, cudaStream_t stream, cudaEvent_t *ev
     }
 }
 
-vim_status launch_pair(PairArgs a, int N, vim_dtype dt, cudaStream_t stream, cudaEvent_t *ev) {
+vim_status launch_pair(const PairArgs &a, int N, vim_dtype dt, cudaStream_t stream, cudaEvent_t *ev) {
     return dt == VIM_F32 ? launch_pair_n<float>(a, N, stream, ev)
                          : launch_pair_n<__nv_bfloat16>(a, N, stream, ev);
 }
