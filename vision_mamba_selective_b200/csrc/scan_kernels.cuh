@@ -12,9 +12,12 @@
 // over it: warps 0-1 the forward direction (ascending), warps 2-3 the backward
 // direction (descending), one thread per (channel, direction) with all d_state
 // states of h in fp32 registers.  The chunk's inputs stream through shared memory in
-// tiles of 16 tokens (cp.async for u/delta, register prefetch + fp32 conversion for
-// B/C), double buffered.  The two directions meet in a per-chunk fp32 buffer of
-// partial outputs, and the summed, gated result is written once with 16-byte stores.
+// tiles of 16 tokens (cp.async for u/delta/z, register prefetch + fp32 conversion for
+// B/C), double buffered.  The forward direction visits tile j at step j and the
+// backward one at step nT-1-j: the first visitor leaves its partial output in a
+// per-chunk fp32 buffer, the second adds its own, applies the silu(z) gate and
+// writes the result, so every output is written once and no separate output pass
+// is needed.
 //
 // For G > 1 the state entering each chunk comes from two small kernels: `pair_carry`
 // reduces every chunk to its end state from h = 0 plus its total Delta, and
@@ -27,9 +30,10 @@
 
 namespace vimscan {
 
-constexpr int kDC = 64;            // channels per CTA
-constexpr int kThreads = 2 * kDC;  // one thread per (channel, direction)
-constexpr int kTile = 16;          // tokens per staged tile
+constexpr int kDC = 64;              // channels per CTA
+constexpr int kThreads = 2 * kDC;    // one thread per (channel, direction)
+constexpr int kTile = 16;            // tokens per staged tile
+constexpr int kSub = 4;              // tokens whose independent work is formed ahead of the recurrence
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ----------------------------------------------------------------------------
@@ -69,6 +73,15 @@ __device__ __forceinline__ uint4 pack16(const float (&f)[8]) {
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// 16 bytes of T, every element equal to x
+template <typename T>
+__device__ __forceinline__ uint4 pad16(float x) {
+    float f[Vec<T>::n];
+#pragma unroll
+    for (int i = 0; i < Vec<T>::n; ++i) f[i] = x;
+    return pack16(f);
+}
+
 // ----------------------------------------------------------------------------
 // math
 // ----------------------------------------------------------------------------
@@ -98,6 +111,25 @@ __device__ __forceinline__ float softplus(float x) {
     p = fmaf(s2, p, 2.0f);
     const float r = fmaf(s, p, fmaxf(x, 0.0f));
     return x > 20.0f ? x : r;
+}
+
+// softplus from the MUFU exp2/log2 approximations: log2(1 + 2^(x log2 e)) ln 2, and x
+// above 20.  Its absolute error is about 1e-7 (the log2 approximation near 1), far
+// below the resolution of bf16 inputs; the fp32-I/O kernels use softplus() instead.
+__device__ __forceinline__ float lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float softplus_fast(float x) {
+    const float r = lg2(1.0f + ex2(x * kLog2e)) * 0.69314718055994531f;
+    return x > 20.0f ? x : r;
+}
+
+template <typename T>
+__device__ __forceinline__ float softplus_io(float x) {
+    if constexpr (sizeof(T) == 4) return softplus(x);
+    else return softplus_fast(x);
 }
 
 // silu(z) = z / (1 + exp(-z))
@@ -164,18 +196,31 @@ __device__ __forceinline__ int position(const PairArgs &p, int t) {
 // ----------------------------------------------------------------------------
 // shared-memory staging of one step: the forward tile and the backward tile
 // ----------------------------------------------------------------------------
+// One slot: [dir][u|delta][kTile][kDC] T | [dir][B|C][kTile][N] fp32 |
+//           [dir][kTile][kDC] T (z)     | [dir][kTile][kDC] fp32 (partial_in, optional)
 template <typename T, int N>
 struct Stage {
-    static constexpr int kUV = kTile * kDC;                  // elements per u or delta tile
+    static constexpr int kUV = kTile * kDC;                  // elements per u, delta or z tile
     static constexpr int kBC = kTile * N;                    // elements per B or C tile
-    // one slot: [dir][u|delta][kUV] T, then [dir][B|C][kBC] float
-    static constexpr int kSlotBytes = 2 * 2 * kUV * (int)sizeof(T) + 2 * 2 * kBC * 4;
+    static constexpr int kUVBytes = 2 * 2 * kUV * (int)sizeof(T);
+    static constexpr int kBCBytes = 2 * 2 * kBC * 4;
+    static constexpr int kZBytes = 2 * kUV * (int)sizeof(T);
+    static constexpr int kPinBytes = 2 * kUV * 4;
 
+    __host__ __device__ static constexpr int slot_bytes(bool pin) {
+        return kUVBytes + kBCBytes + kZBytes + (pin ? kPinBytes : 0);
+    }
     __device__ static T *uv(char *slot, int dir, int which) {
         return reinterpret_cast<T *>(slot) + (dir * 2 + which) * kUV;
     }
     __device__ static float *bc(char *slot, int dir, int which) {
-        return reinterpret_cast<float *>(slot + 2 * 2 * kUV * sizeof(T)) + (dir * 2 + which) * kBC;
+        return reinterpret_cast<float *>(slot + kUVBytes) + (dir * 2 + which) * kBC;
+    }
+    __device__ static T *zt(char *slot, int dir) {
+        return reinterpret_cast<T *>(slot + kUVBytes + kBCBytes) + dir * kUV;
+    }
+    __device__ static float *pin(char *slot, int dir) {
+        return reinterpret_cast<float *>(slot + kUVBytes + kBCBytes + kZBytes) + dir * kUV;
     }
 };
 
@@ -192,15 +237,18 @@ template <typename T, int N>
 constexpr bool bc_vectorizable() { return (N * sizeof(T)) % 16 == 0; }
 
 // Loads of one step (tile jf of the forward direction, jb of the backward one):
-// u/delta by cp.async straight into the slot, B/C into registers first and then,
-// converted to fp32, into the slot.  Rows past the end of the chunk and channels
-// past d_inner are zero-filled, so that they act as no-op tokens.
+// u/delta (and z, partial_in on the steps that complete a tile) by cp.async straight
+// into the slot, B/C into registers first and then, converted to fp32, into the slot.
+// Rows past the end of the chunk and channels past d_inner are zero-filled, so that
+// they act as no-op tokens.
 template <typename T, int N, bool VEC_BC>
 struct Stager {
     using S = Stage<T, N>;
     static constexpr int V = Vec<T>::n;                 // elements per 16-byte piece
     static constexpr int kRowPieces = kDC / V;          // pieces per u/delta row
     static constexpr int kUVRep = kTile * kRowPieces / kThreads;   // pieces per thread per tensor
+    static constexpr int kPinRowPieces = kDC / 4;
+    static constexpr int kPinRep = kTile * kPinRowPieces / kThreads;
     static constexpr int kBCRow = VEC_BC ? (int)(N * sizeof(T) / 16) : N;   // units per B/C row
     static constexpr int kBCUnits = 4 * kTile * kBCRow;
     static constexpr int kBCPer = (kBCUnits + kThreads - 1) / kThreads;
@@ -216,9 +264,17 @@ struct Stager {
 
     __device__ int rows_of(int j) const { return min(kTile, tc - j * kTile); }
 
-    __device__ void issue_uv(char *slot, int jf, int jb) const {
+    // element offset of row r of tile j, channel ch (valid rows only)
+    __device__ size_t row_off(int j, int r, int ch) const {
+        return ((size_t)b * p.L + position(p, t0 + j * kTile + r)) * p.Di + ch;
+    }
+
+    // u and delta; with `aux`, also z (if gated) and partial_in (if present)
+    __device__ void issue(char *slot, int jf, int jb, bool aux) const {
         const T *gu = static_cast<const T *>(p.u);
         const T *gd = static_cast<const T *>(p.delta);
+        const T *gz = static_cast<const T *>(p.z);
+        const bool with_z = aux && gz != nullptr;
 #pragma unroll
         for (int dir = 0; dir < 2; ++dir) {
             const int j = dir ? jb : jf;
@@ -229,11 +285,30 @@ struct Stager {
                 const int v = li % kRowPieces, r = li / kRowPieces;
                 const int ch = d0 + v * V;
                 const bool ok = r < rows && ch < p.Di;
-                size_t off = 0;
-                if (ok) off = ((size_t)b * p.L + position(p, t0 + j * kTile + r)) * p.Di + ch;
                 const int so = r * kDC + v * V;
-                cp_async16(S::uv(slot, dir, 0) + so, gu + off, ok);
-                cp_async16(S::uv(slot, dir, 1) + so, gd + off, ok);
+                if (ok) {
+                    const size_t off = row_off(j, r, ch);
+                    cp_async16(S::uv(slot, dir, 0) + so, gu + off, true);
+                    cp_async16(S::uv(slot, dir, 1) + so, gd + off, true);
+                    if (with_z) cp_async16(S::zt(slot, dir) + so, gz + off, true);
+                } else {
+                    // outside the data: u = 0 and delta_raw = -1e4, so that Delta =
+                    // softplus(-1e4 + bias) = 0 exactly (Abar = 1, Bbar u = 0): a no-op token
+                    *reinterpret_cast<uint4 *>(S::uv(slot, dir, 0) + so) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(S::uv(slot, dir, 1) + so) = pad16<T>(-1.0e4f);
+                    if (with_z) *reinterpret_cast<uint4 *>(S::zt(slot, dir) + so) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            if (aux && p.partial_in) {
+#pragma unroll
+                for (int m = 0; m < kPinRep; ++m) {
+                    const int li = threadIdx.x + m * kThreads;
+                    const int v = li % kPinRowPieces, r = li / kPinRowPieces;
+                    const int ch = d0 + v * 4;
+                    const bool ok = r < rows && ch < p.Di;
+                    const size_t off = ok ? row_off(j, r, ch) : 0;
+                    cp_async16(S::pin(slot, dir) + r * kDC + v * 4, p.partial_in + off, ok);
+                }
             }
         }
         cp_async_commit();
@@ -291,7 +366,8 @@ struct Stager {
 // ----------------------------------------------------------------------------
 template <int N>
 struct ChannelParams {
-    float A2[N];        // A[d][n] * log2(e)
+    const float *A;     // A[dir][d][:] (general-A path)
+    float A0;           // A[d][0] * log2(e)
     float D, bias;
     bool structured;    // A[d][n] == (n+1) A[d][0] for every n
     bool valid;
@@ -299,28 +375,28 @@ struct ChannelParams {
     __device__ void load(const PairArgs &p, int dir, int d) {
         valid = d < p.Di;
         structured = true;
-        D = 0.0f;
-        bias = 0.0f;
-#pragma unroll
-        for (int n = 0; n < N; ++n) A2[n] = 0.0f;
+        A0 = D = bias = 0.0f;
+        A = p.A;
         if (!valid) return;
-        const float *a = p.A + ((size_t)dir * p.Di + d) * N;
-        const float a0 = a[0];
+        A = p.A + ((size_t)dir * p.Di + d) * N;
+        const float a0 = A[0];
 #pragma unroll
-        for (int n = 0; n < N; ++n) {
-            const float an = a[n];
-            structured = structured && (an == (float)(n + 1) * a0);
-            A2[n] = an * kLog2e;
-        }
+        for (int n = 0; n < N; ++n) structured = structured && (A[n] == (float)(n + 1) * a0);
+        A0 = a0 * kLog2e;
         D = p.D[(size_t)dir * p.Di + d];
         bias = p.bias[(size_t)dir * p.Di + d];
     }
 };
 
-constexpr int kSub = 8;   // tokens whose independent work is formed ahead of the recurrence
-
 // row of the tile that step i of a walk over it visits (ascending or descending)
-__device__ __forceinline__ int walk_row(bool descending, int i) { return descending ? kTile - 1 - i : i; }
+template <bool DESC>
+__device__ __forceinline__ int walk_row(int i) { return DESC ? kTile - 1 - i : i; }
+
+// Delta of one staged row (rows past the tile end hold delta_raw = -1e4: Delta = 0)
+template <typename T>
+__device__ __forceinline__ float delta_of(const T *sd, int r, int dl, float bias) {
+    return softplus_io<T>(to_f32(sd[r * kDC + dl]) + bias);
+}
 
 // ----------------------------------------------------------------------------
 // kernel 1: chunk summaries (end state from h = 0, and the total Delta)
@@ -330,30 +406,28 @@ __device__ __forceinline__ int walk_row(bool descending, int i) { return descend
 // Delta summed over the tokens the direction visits after s inside the chunk.  With
 // A_n = (n+1) A_0 the weights are powers of w = exp(A_0 S_s), built by one multiply
 // per state.
-template <typename T, int N, bool FAST>
+template <typename T, int N, bool FAST, bool DESC>
 __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, const ChannelParams<N> &prm,
-                                           bool descending, int dl, int rows, const T *su, const T *sd,
-                                           const float *sB) {
+                                           int dl, const T *su, const T *sd, const float *sB) {
     constexpr int NP = N / 2;
-#pragma unroll
-    for (int half = 0; half < kTile / kSub; ++half) {
+#pragma unroll 1
+    for (int sub = 0; sub < kTile / kSub; ++sub) {
         float Sv[kSub], duv[kSub];
 #pragma unroll
         for (int k = 0; k < kSub; ++k) {
-            const int r = walk_row(descending, half * kSub + k);
-            const float uu = to_f32(su[r * kDC + dl]);
-            const float dt = r < rows ? softplus(to_f32(sd[r * kDC + dl]) + prm.bias) : 0.0f;
-            duv[k] = dt * uu;
+            const int r = walk_row<DESC>(sub * kSub + k);
+            const float dt = delta_of<T>(sd, r, dl, prm.bias);
+            duv[k] = dt * to_f32(su[r * kDC + dl]);
             Sv[k] = Ssum;          // Delta of the tokens walked before this one
             Ssum += dt;
         }
 #pragma unroll
         for (int k = 0; k < kSub; ++k) {
-            const int r = walk_row(descending, half * kSub + k);
+            const int r = walk_row<DESC>(sub * kSub + k);
             float2 Bv[NP];
             load_row<NP>(sB + r * N, Bv);
             if constexpr (FAST) {
-                const float w = ex2(prm.A2[0] * Sv[k]);
+                const float w = ex2(prm.A0 * Sv[k]);
                 const float x0 = w * duv[k];
                 float2 x = f2(x0, x0 * w);
                 const float2 w2 = f2(w * w, w * w);
@@ -366,7 +440,8 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
                 const float2 du2 = f2(duv[k], duv[k]);
 #pragma unroll
                 for (int q = 0; q < NP; ++q) {
-                    const float2 wq = f2(ex2(prm.A2[2 * q] * Sv[k]), ex2(prm.A2[2 * q + 1] * Sv[k]));
+                    const float2 wq = f2(ex2(__ldg(prm.A + 2 * q) * kLog2e * Sv[k]),
+                                         ex2(__ldg(prm.A + 2 * q + 1) * kLog2e * Sv[k]));
                     H[q] = fma2(mul2(wq, du2), Bv[q], H[q]);
                 }
             }
@@ -375,9 +450,10 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
 }
 
 template <typename T, int N, bool VEC_BC>
-__global__ void __launch_bounds__(kThreads, 3) pair_carry(PairArgs p) {
+__global__ void __launch_bounds__(kThreads, 4) pair_carry(PairArgs p) {
     using S = Stage<T, N>;
     constexpr int NP = N / 2;
+    constexpr int kSlot = S::slot_bytes(false);
     extern __shared__ __align__(16) char smem[];
 
     const int b = blockIdx.z, c = blockIdx.y, d0 = blockIdx.x * kDC;
@@ -393,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 3) pair_carry(PairArgs p) {
 
     // the forward direction walks tiles nT-1 .. 0, the backward one 0 .. nT-1
     Stager<T, N, VEC_BC> st(p, b, t0, tc, d0);
-    st.issue_uv(smem, nT - 1, 0);
+    st.issue(smem, nT - 1, 0, false);
     st.load_bc(nT - 1, 0);
     st.store_bc(smem);
     cp_async_wait_all();
@@ -405,20 +481,22 @@ __global__ void __launch_bounds__(kThreads, 3) pair_carry(PairArgs p) {
     float Ssum = 0.0f;
 
     for (int s = 0; s < nT; ++s) {
-        char *cur = smem + (s & 1) * S::kSlotBytes;
-        char *nxt = smem + ((s + 1) & 1) * S::kSlotBytes;
+        char *cur = smem + (s & 1) * kSlot;
+        char *nxt = smem + ((s + 1) & 1) * kSlot;
         if (s + 1 < nT) {
-            st.issue_uv(nxt, nT - 2 - s, s + 1);
+            st.issue(nxt, nT - 2 - s, s + 1, false);
             st.load_bc(nT - 2 - s, s + 1);
         }
-        const int j = dir ? s : nT - 1 - s;
         if (active) {
             const T *su = S::uv(cur, dir, 0), *sd = S::uv(cur, dir, 1);
             const float *sB = S::bc(cur, dir, 0);
-            if (fast)
-                carry_tile<T, N, true>(H, Ssum, prm, dir == 0, dl, st.rows_of(j), su, sd, sB);
-            else
-                carry_tile<T, N, false>(H, Ssum, prm, dir == 0, dl, st.rows_of(j), su, sd, sB);
+            if (dir == 0) {
+                if (fast) carry_tile<T, N, true, true>(H, Ssum, prm, dl, su, sd, sB);
+                else carry_tile<T, N, false, true>(H, Ssum, prm, dl, su, sd, sB);
+            } else {
+                if (fast) carry_tile<T, N, true, false>(H, Ssum, prm, dl, su, sd, sB);
+                else carry_tile<T, N, false, false>(H, Ssum, prm, dl, su, sd, sB);
+            }
         }
         if (s + 1 < nT) {
             st.store_bc(nxt);
@@ -480,55 +558,73 @@ __global__ void __launch_bounds__(256) pair_combine(PairArgs p) {
     }
 }
 
-// acc (+)= V consecutive floats (16-byte aligned), V a multiple of 4
-template <int V, bool ADD>
-__device__ __forceinline__ void add_f32(float (&acc)[V], const float *src) {
-    const float4 *s4 = reinterpret_cast<const float4 *>(src);
-#pragma unroll
-    for (int q = 0; q < V / 4; ++q) {
-        const float4 a = s4[q];
-        if (ADD) {
-            acc[4 * q] += a.x; acc[4 * q + 1] += a.y; acc[4 * q + 2] += a.z; acc[4 * q + 3] += a.w;
-        } else {
-            acc[4 * q] = a.x; acc[4 * q + 1] = a.y; acc[4 * q + 2] = a.z; acc[4 * q + 3] = a.w;
-        }
-    }
-}
-
 // ----------------------------------------------------------------------------
 // kernel 3: both directions over one chunk, merge, gate, store
 // ----------------------------------------------------------------------------
+// Where one thread's outputs go: rows of a tile lie at base + r * rstride elements
+// unless the tile wraps into the next grid column (column-major order only).
+template <typename T>
+struct OutRows {
+    size_t base, rstride;
+    bool linear;
+    int j, d;         // tile index and channel (for the exact fallback)
+};
+
+template <typename T, int N, bool VEC_BC>
+__device__ __forceinline__ OutRows<T> out_rows(const Stager<T, N, VEC_BC> &st, const PairArgs &p, int j,
+                                               int rows, int d) {
+    OutRows<T> o;
+    const int t = st.t0 + j * kTile;
+    o.j = j;
+    o.d = d;
+    if (p.order == 0) {
+        o.linear = true;
+        o.base = ((size_t)st.b * p.L + t) * p.Di + d;
+        o.rstride = (size_t)p.Di;
+    } else {
+        o.linear = (t % p.H) + rows <= p.H;
+        o.base = ((size_t)st.b * p.L + position(p, t)) * p.Di + d;
+        o.rstride = (size_t)p.W * p.Di;
+    }
+    return o;
+}
+
 // One direction's pass over one staged tile: the softplus, Delta*u and decay base of
 // kSub tokens are formed first (independent of h), then the recurrence runs through
-// them.  Rows past the tile's end are no-op tokens (Delta = 0: Abar = 1, Bbar u = 0).
-template <typename T, int N, bool FAST>
-__device__ __forceinline__ void main_tile(float2 (&h)[N / 2], const ChannelParams<N> &prm,
-                                          bool descending, int dl, int rows, const T *su,
-                                          const T *sd, const float *sB, const float *sC, float *ydst,
-                                          bool yadd) {
+// them.  Rows past the tile's end are no-op tokens and store nothing.  First visit:
+// the partial output goes to ypart.  Second visit: it is added to the partial left
+// there, the gate applied and the result stored (or, for the first pair of the
+// cross-scan, the ungated fp32 sum).
+template <typename T, int N, bool VEC_BC, bool FAST, bool DESC>
+__device__ __forceinline__ void main_tile(bool second, int rows, float2 (&h)[N / 2],
+                                          const ChannelParams<N> &prm, int dl, const T *su,
+                                          const T *sd, const float *sB, const float *sC,
+                                          float *ypart, const T *sz, const float *spin,
+                                          const Stager<T, N, VEC_BC> &st, const PairArgs &p,
+                                          const OutRows<T> &o) {
     constexpr int NP = N / 2;
-#pragma unroll
-    for (int half = 0; half < kTile / kSub; ++half) {
+#pragma unroll 1
+    for (int sub = 0; sub < kTile / kSub; ++sub) {
         float qv[kSub], duv[kSub], uv[kSub];
 #pragma unroll
         for (int k = 0; k < kSub; ++k) {
-            const int r = walk_row(descending, half * kSub + k);
-            const float uu = to_f32(su[r * kDC + dl]);
-            const float dt = r < rows ? softplus(to_f32(sd[r * kDC + dl]) + prm.bias) : 0.0f;
-            uv[k] = uu;
-            duv[k] = dt * uu;
-            qv[k] = FAST ? ex2(dt * prm.A2[0]) : dt;
+            const int r = walk_row<DESC>(sub * kSub + k);
+            const float dt = delta_of<T>(sd, r, dl, prm.bias);
+            uv[k] = to_f32(su[r * kDC + dl]);
+            duv[k] = dt * uv[k];
+            qv[k] = FAST ? ex2(dt * prm.A0) : dt;
         }
 #pragma unroll
         for (int k = 0; k < kSub; ++k) {
-            const int r = walk_row(descending, half * kSub + k);
+            const int r = walk_row<DESC>(sub * kSub + k);
             float2 a[NP];
             if constexpr (FAST) {
                 powers2<NP>(qv[k], a);
             } else {
 #pragma unroll
                 for (int q = 0; q < NP; ++q)
-                    a[q] = f2(ex2(qv[k] * prm.A2[2 * q]), ex2(qv[k] * prm.A2[2 * q + 1]));
+                    a[q] = f2(ex2(qv[k] * __ldg(prm.A + 2 * q) * kLog2e),
+                              ex2(qv[k] * __ldg(prm.A + 2 * q + 1) * kLog2e));
             }
             float2 Bv[NP], Cv[NP];
             load_row<NP>(sB + r * N, Bv);
@@ -541,22 +637,33 @@ __device__ __forceinline__ void main_tile(float2 (&h)[N / 2], const ChannelParam
                 if (q & 1) y1 = fma2(Cv[q], h[q], y1);
                 else y0 = fma2(Cv[q], h[q], y0);
             }
-            const float yv = fmaf(prm.D, uv[k], (y0.x + y0.y) + (y1.x + y1.y));
-            if (r < rows) {
-                float *py = ydst + r * kDC;
-                *py = yadd ? *py + yv : yv;
+            const float2 ys = __fadd2_rn(y0, y1);
+            const float yv = fmaf(prm.D, uv[k], ys.x + ys.y);
+            if (!second) {
+                ypart[r * kDC] = yv;   // rows past the end land inside the chunk buffer, unread
+            } else if (r < rows) {
+                float tot = ypart[r * kDC] + yv;
+                if (spin) tot += spin[r * kDC + dl];
+                const size_t off = o.linear ? o.base + (size_t)r * o.rstride : st.row_off(o.j, r, o.d);
+                if (p.partial_out) {
+                    p.partial_out[off] = tot;
+                } else {
+                    if (sz) tot *= silu(to_f32(sz[r * kDC + dl]));
+                    static_cast<T *>(p.y)[off] = T(tot);
+                }
             }
         }
     }
 }
 
 template <typename T, int N, bool VEC_BC>
-__global__ void __launch_bounds__(kThreads, 3) pair_main(PairArgs p) {
+__global__ void __launch_bounds__(kThreads, 4) pair_main(PairArgs p) {
     using S = Stage<T, N>;
     constexpr int NP = N / 2;
     extern __shared__ __align__(16) char smem[];
-    float *ybuf = reinterpret_cast<float *>(smem + 2 * S::kSlotBytes);   // [chunk][kDC]
-    float *ymid = ybuf + (size_t)p.chunk * kDC;                          // [kTile][kDC]
+    const int slot_bytes = S::slot_bytes(p.partial_in != nullptr);
+    float *ybuf = reinterpret_cast<float *>(smem + 2 * slot_bytes);   // [chunk][kDC]
+    float *ymid = ybuf + (size_t)p.chunk * kDC;                        // [kTile][kDC]
 
     const int b = blockIdx.z, c = blockIdx.y, d0 = blockIdx.x * kDC;
     const int dir = threadIdx.x / kDC, dl = threadIdx.x % kDC, d = d0 + dl;
@@ -569,81 +676,78 @@ __global__ void __launch_bounds__(kThreads, 3) pair_main(PairArgs p) {
 
     // state entering this chunk
     float2 h[NP];
-    const bool has_carry = p.G > 1 && (dir == 0 ? c > 0 : c < p.G - 1);
-    if (has_carry && prm.valid) {
+#pragma unroll
+    for (int k = 0; k < NP; ++k) h[k] = f2(0.f, 0.f);
+    if (p.G > 1 && (dir == 0 ? c > 0 : c < p.G - 1) && prm.valid) {
         const size_t base = (((size_t)b * p.G + c) * 2 + dir) * p.Di + d;
         const float2 *hin = reinterpret_cast<const float2 *>(p.hloc + base * N);
 #pragma unroll
         for (int k = 0; k < NP; ++k) h[k] = hin[k];
-    } else {
-#pragma unroll
-        for (int k = 0; k < NP; ++k) h[k] = f2(0.f, 0.f);
     }
 
+    // step s completes the tiles it visits when 2s >= nT-1 (z/partial_in needed then)
+    auto completes = [&](int s) { return 2 * s >= nT - 1; };
     Stager<T, N, VEC_BC> st(p, b, t0, tc, d0);
-    st.issue_uv(smem, 0, nT - 1);
+    st.issue(smem, 0, nT - 1, completes(0));
     st.load_bc(0, nT - 1);
     st.store_bc(smem);
     cp_async_wait_all();
     __syncthreads();
 
     for (int s = 0; s < nT; ++s) {
-        char *cur = smem + (s & 1) * S::kSlotBytes;
-        char *nxt = smem + ((s + 1) & 1) * S::kSlotBytes;
+        char *cur = smem + (s & 1) * slot_bytes;
+        char *nxt = smem + ((s + 1) & 1) * slot_bytes;
         if (s + 1 < nT) {
-            st.issue_uv(nxt, s + 1, nT - 2 - s);
+            st.issue(nxt, s + 1, nT - 2 - s, completes(s + 1));
             st.load_bc(s + 1, nT - 2 - s);
         }
         const int j = dir ? nT - 1 - s : s;
+        const int rows = st.rows_of(j);
         // the forward direction visits tile j at step j, the backward one at nT-1-j:
-        // the first visitor stores its partial, the second adds to it; when both come
-        // in the same step (the middle tile) the backward one writes aside to ymid
+        // the first visitor stores its partial, the second completes the output; when
+        // both come in the same step (the middle tile) the backward one writes aside
+        // to ymid and the tile is finished after the step
         const int twice = 2 * s - (nT - 1);
-        float *ydst = (twice == 0 && dir == 1) ? ymid + dl : ybuf + (size_t)j * kTile * kDC + dl;
-        const bool yadd = twice > 0;
+        float *ypart = (twice == 0 && dir == 1) ? ymid + dl : ybuf + (size_t)j * kTile * kDC + dl;
         if (prm.valid) {
             const T *su = S::uv(cur, dir, 0), *sd = S::uv(cur, dir, 1);
             const float *sB = S::bc(cur, dir, 0), *sC = S::bc(cur, dir, 1);
-            if (fast)
-                main_tile<T, N, true>(h, prm, dir == 1, dl, st.rows_of(j), su, sd, sB, sC, ydst, yadd);
-            else
-                main_tile<T, N, false>(h, prm, dir == 1, dl, st.rows_of(j), su, sd, sB, sC, ydst, yadd);
+            const T *sz = p.z ? S::zt(cur, dir) : nullptr;
+            const float *spin = p.partial_in ? S::pin(cur, dir) : nullptr;
+            const OutRows<T> o = out_rows(st, p, j, rows, d);
+            const bool second = twice > 0;
+            if (dir == 0) {
+                if (fast) main_tile<T, N, VEC_BC, true, false>(second, rows, h, prm, dl, su, sd, sB, sC, ypart, sz, spin, st, p, o);
+                else main_tile<T, N, VEC_BC, false, false>(second, rows, h, prm, dl, su, sd, sB, sC, ypart, sz, spin, st, p, o);
+            } else {
+                if (fast) main_tile<T, N, VEC_BC, true, true>(second, rows, h, prm, dl, su, sd, sB, sC, ypart, sz, spin, st, p, o);
+                else main_tile<T, N, VEC_BC, false, true>(second, rows, h, prm, dl, su, sd, sB, sC, ypart, sz, spin, st, p, o);
+            }
         }
         if (s + 1 < nT) {
             st.store_bc(nxt);
             cp_async_wait_all();
         }
         __syncthreads();
-    }
-
-    // merge the middle tile, gate, store: one item = one 16-byte vector of channels
-    constexpr int V = Vec<T>::n;
-    constexpr int per_row = kDC / V;
-    const int mid_tile = (nT & 1) ? (nT - 1) / 2 : -1;
-    for (int i = threadIdx.x; i < tc * per_row; i += kThreads) {
-        const int v = i % per_row, tl = i / per_row;
-        const int ch = d0 + v * V;
-        if (ch >= p.Di) continue;   // Di is a multiple of V: the vector is whole or absent
-        float acc[V];
-        add_f32<V, false>(acc, ybuf + tl * kDC + v * V);
-        if (tl / kTile == mid_tile) add_f32<V, true>(acc, ymid + (tl % kTile) * kDC + v * V);
-        const int pos = position(p, t0 + tl);
-        const size_t off = ((size_t)b * p.L + pos) * p.Di + ch;
-        if (p.partial_in) add_f32<V, true>(acc, p.partial_in + off);
-        if (p.partial_out) {
-            float4 *po = reinterpret_cast<float4 *>(p.partial_out + off);
-#pragma unroll
-            for (int q = 0; q < V / 4; ++q)
-                po[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
-            continue;
+        if (twice == 0) {
+            // the middle tile: both partials are in shared memory; z and partial_in were
+            // staged for it in this step's slot (the two directions' tiles coincide)
+            const int jm = s, rm = st.rows_of(jm);
+            for (int i = threadIdx.x; i < rm * kDC; i += kThreads) {
+                const int r = i / kDC, cl = i % kDC, ch = d0 + cl;
+                if (ch >= p.Di) continue;
+                float tot = ybuf[((size_t)jm * kTile + r) * kDC + cl] + ymid[r * kDC + cl];
+                if (p.partial_in) tot += S::pin(cur, 0)[r * kDC + cl];
+                const size_t off = st.row_off(jm, r, ch);
+                if (p.partial_out) {
+                    p.partial_out[off] = tot;
+                } else {
+                    if (p.z) tot *= silu(to_f32(S::zt(cur, 0)[r * kDC + cl]));
+                    static_cast<T *>(p.y)[off] = T(tot);
+                }
+            }
+            __syncthreads();   // slot `cur` is refilled by the next step's loads
         }
-        if (p.z) {
-            float zf[V];
-            unpack16(*reinterpret_cast<const uint4 *>(static_cast<const T *>(p.z) + off), zf);
-#pragma unroll
-            for (int e = 0; e < V; ++e) acc[e] *= silu(zf[e]);
-        }
-        *reinterpret_cast<uint4 *>(static_cast<T *>(p.y) + off) = pack16(acc);
     }
 }
 

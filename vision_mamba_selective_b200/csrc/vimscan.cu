@@ -13,8 +13,18 @@
 namespace vimscan {
 namespace {
 
-constexpr int kSingleChunkMax = 256;   // sequences up to this length run as one chunk
-constexpr int kLongChunk = 128;        // chunk length otherwise (a multiple of kTile)
+#ifndef VIMSCAN_SINGLE_CHUNK_MAX
+#define VIMSCAN_SINGLE_CHUNK_MAX 256
+#endif
+#ifndef VIMSCAN_LONG_CHUNK
+#define VIMSCAN_LONG_CHUNK 64
+#endif
+// sequences up to kSingleChunkMax tokens run as one chunk; longer ones in chunks of
+// kLongChunk tokens (a multiple of kTile), sized so that four CTAs of the main kernel
+// fit in one SM's shared memory
+constexpr int kSingleChunkMax = VIMSCAN_SINGLE_CHUNK_MAX;
+constexpr int kLongChunk = VIMSCAN_LONG_CHUNK;
+static_assert(kLongChunk % kTile == 0, "chunks are whole tiles");
 constexpr size_t kAlign = 256;
 
 struct Plan {
@@ -60,12 +70,12 @@ vim_status check_common(int batch, int L, int Di, int N, vim_dtype dt) {
 }
 
 template <typename T, int N>
-size_t main_smem(int chunk) {
-    return 2 * (size_t)Stage<T, N>::kSlotBytes + (size_t)chunk * kDC * 4 + (size_t)kTile * kDC * 4;
+size_t main_smem(int chunk, bool pin) {
+    return 2 * (size_t)Stage<T, N>::slot_bytes(pin) + (size_t)chunk * kDC * 4 + (size_t)kTile * kDC * 4;
 }
 template <typename T, int N>
 size_t carry_smem() {
-    return 2 * (size_t)Stage<T, N>::kSlotBytes;
+    return 2 * (size_t)Stage<T, N>::slot_bytes(false);
 }
 
 // events: null, or 3 events recorded after the carry, combine and main kernels
@@ -92,7 +102,7 @@ vim_status launch_pair_v(const PairArgs &a, cudaStream_t stream, cudaEvent_t *ev
     } else if (ev) {
         if (mark(ev, 0, stream) != VIM_OK || mark(ev, 1, stream) != VIM_OK) return VIM_ERR_CUDA;
     }
-    const size_t sm = main_smem<T, N>(a.chunk);
+    const size_t sm = main_smem<T, N>(a.chunk, a.partial_in != nullptr);
     if (cudaFuncSetAttribute(pair_main<T, N, VEC_BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sm) != cudaSuccess)
         return VIM_ERR_CUDA;
