@@ -33,7 +33,14 @@ namespace vimscan {
 constexpr int kDC = 64;              // channels per CTA
 constexpr int kThreads = 2 * kDC;    // one thread per (channel, direction)
 constexpr int kTile = 16;            // tokens per staged tile
-constexpr int kSub = 4;              // tokens whose independent work is formed ahead of the recurrence
+#ifndef VIMSCAN_KSUB
+#define VIMSCAN_KSUB 4
+#endif
+#ifndef VIMSCAN_MIN_BLOCKS
+#define VIMSCAN_MIN_BLOCKS 4
+#endif
+constexpr int kSub = VIMSCAN_KSUB;   // tokens whose independent work is formed ahead of the recurrence
+constexpr int kMinBlocks = VIMSCAN_MIN_BLOCKS;   // resident CTAs per SM the register budget targets
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ----------------------------------------------------------------------------
@@ -450,7 +457,7 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
 }
 
 template <typename T, int N, bool VEC_BC>
-__global__ void __launch_bounds__(kThreads, 4) pair_carry(PairArgs p) {
+__global__ void __launch_bounds__(kThreads, kMinBlocks) pair_carry(PairArgs p) {
     using S = Stage<T, N>;
     constexpr int NP = N / 2;
     constexpr int kSlot = S::slot_bytes(false);
@@ -520,41 +527,44 @@ __global__ void __launch_bounds__(kThreads, 4) pair_carry(PairArgs p) {
 // One thread per (batch, direction, channel, state).  hloc[b][c][dir][d][n] is
 // replaced by the state entering chunk c in that direction's visiting order:
 // H_in(next) = exp(A_n * Ssum(c)) * H_in(c) + H_loc(c).  Loads run 16 chunks ahead.
+// The last chunk's summary in each direction was never formed: it is read and fed
+// into h after the last carry has been stored, which is harmless.
 template <int N>
 __global__ void __launch_bounds__(256) pair_combine(PairArgs p) {
     constexpr int kAhead = 16;
-    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t total = (int64_t)p.batch * 2 * p.Di * N;
-    if (idx >= total) return;
-    const int n = (int)(idx % N);
-    const int d = (int)((idx / N) % p.Di);
-    const int dir = (int)((idx / ((int64_t)N * p.Di)) % 2);
-    const int b = (int)(idx / ((int64_t)2 * N * p.Di));
-    const float A2n = p.A[((size_t)dir * p.Di + d) * N + n] * kLog2e;
+    const int idx = blockIdx.x * blockDim.x + threadIdx.x;   // (b, dir, d, n), n fastest
+    const int per_b = 2 * p.Di * N;
+    if (idx >= p.batch * per_b) return;
+    const int b = idx / per_b, rem = idx % per_b;            // rem = (dir * Di + d) * N + n
+    const int dir = rem / (p.Di * N);
+    const float A2n = p.A[rem] * kLog2e;                     // A is [2][Di][N]: same index
+    // hloc[b][c][dir][d][n] and ssum[b][c][dir][d]: chunk c+1 lies per_b (per_b / N) further
+    const int step = dir ? -1 : 1;
+    const int c0 = dir ? p.G - 1 : 0;
+    float *hl = p.hloc + ((size_t)b * p.G + c0) * per_b + rem;
+    const float *ss = p.ssum + ((size_t)b * p.G + c0) * (per_b / N) + rem / N;
+    const ptrdiff_t hstride = (ptrdiff_t)step * per_b, sstride = (ptrdiff_t)step * (per_b / N);
     float h = 0.0f;
     for (int i0 = 0; i0 < p.G; i0 += kAhead) {
-        float loc[kAhead], S[kAhead];
+        float loc[kAhead], P[kAhead];
 #pragma unroll
         for (int k = 0; k < kAhead; ++k) {
-            const int i = i0 + k;
-            if (i < p.G) {
-                const int c = dir ? p.G - 1 - i : i;
-                const size_t base = (((size_t)b * p.G + c) * 2 + dir) * p.Di + d;
-                loc[k] = p.hloc[base * N + n];
-                S[k] = p.ssum[base];
+            if (i0 + k < p.G) {
+                loc[k] = hl[k * hstride];
+                P[k] = ss[k * sstride];
             }
         }
 #pragma unroll
+        for (int k = 0; k < kAhead; ++k) P[k] = ex2(A2n * P[k]);   // exp(A_n * Ssum(c))
+#pragma unroll
         for (int k = 0; k < kAhead; ++k) {
-            const int i = i0 + k;
-            if (i < p.G) {
-                const int c = dir ? p.G - 1 - i : i;
-                const size_t base = (((size_t)b * p.G + c) * 2 + dir) * p.Di + d;
-                p.hloc[base * N + n] = h;
-                // the last chunk's summary (never formed) is not needed
-                if (i < p.G - 1) h = fmaf(ex2(A2n * S[k]), h, loc[k]);
+            if (i0 + k < p.G) {
+                hl[k * hstride] = h;                 // the state entering this chunk
+                h = fmaf(P[k], h, loc[k]);           // (unused after the last chunk)
             }
         }
+        hl += kAhead * hstride;
+        ss += kAhead * sstride;
     }
 }
 
@@ -617,25 +627,40 @@ __device__ __forceinline__ void main_tile(bool second, int rows, float2 (&h)[N /
 #pragma unroll
         for (int k = 0; k < kSub; ++k) {
             const int r = walk_row<DESC>(sub * kSub + k);
-            float2 a[NP];
-            if constexpr (FAST) {
-                powers2<NP>(qv[k], a);
-            } else {
-#pragma unroll
-                for (int q = 0; q < NP; ++q)
-                    a[q] = f2(ex2(qv[k] * __ldg(prm.A + 2 * q) * kLog2e),
-                              ex2(qv[k] * __ldg(prm.A + 2 * q + 1) * kLog2e));
-            }
-            float2 Bv[NP], Cv[NP];
-            load_row<NP>(sB + r * N, Bv);
-            load_row<NP>(sC + r * N, Cv);
+            const float4 *B4 = reinterpret_cast<const float4 *>(sB + r * N);
+            const float4 *C4 = reinterpret_cast<const float4 *>(sC + r * N);
             const float2 du2 = f2(duv[k], duv[k]);
             float2 y0 = f2(0.f, 0.f), y1 = f2(0.f, 0.f);
+            // decays a = (Abar_2q, Abar_2q+1): with A_n = (n+1) A_0 they are the powers
+            // q^(2q+1), q^(2q+2) of q = exp(Delta A_0), one multiply per state
+            const float q = qv[k];
+            float2 a = FAST ? f2(q, q * q) : f2(0.f, 0.f);
+            const float2 step = FAST ? f2(a.y, a.y) : f2(0.f, 0.f);
 #pragma unroll
-            for (int q = 0; q < NP; ++q) {
-                h[q] = fma2(a[q], h[q], mul2(du2, Bv[q]));
-                if (q & 1) y1 = fma2(Cv[q], h[q], y1);
-                else y0 = fma2(Cv[q], h[q], y0);
+            for (int qq = 0; qq < NP; qq += 2) {
+                float2 Bp[2], Cp[2];
+                if constexpr (NP >= 2) {
+                    const float4 b4 = B4[qq / 2], c4 = C4[qq / 2];
+                    Bp[0] = f2(b4.x, b4.y); Bp[1] = f2(b4.z, b4.w);
+                    Cp[0] = f2(c4.x, c4.y); Cp[1] = f2(c4.z, c4.w);
+                } else {
+                    Bp[0] = *reinterpret_cast<const float2 *>(sB + r * N);
+                    Cp[0] = *reinterpret_cast<const float2 *>(sC + r * N);
+                }
+#pragma unroll
+                for (int e = 0; e < 2 && qq + e < NP; ++e) {
+                    const int qi = qq + e;
+                    float2 aq;
+                    if constexpr (FAST) {
+                        aq = a;
+                        a = mul2(a, step);
+                    } else {
+                        aq = f2(ex2(q * __ldg(prm.A + 2 * qi) * kLog2e), ex2(q * __ldg(prm.A + 2 * qi + 1) * kLog2e));
+                    }
+                    h[qi] = fma2(aq, h[qi], mul2(du2, Bp[e]));
+                    if (qi & 1) y1 = fma2(Cp[e], h[qi], y1);
+                    else y0 = fma2(Cp[e], h[qi], y0);
+                }
             }
             const float2 ys = __fadd2_rn(y0, y1);
             const float yv = fmaf(prm.D, uv[k], ys.x + ys.y);
@@ -657,7 +682,7 @@ __device__ __forceinline__ void main_tile(bool second, int rows, float2 (&h)[N /
 }
 
 template <typename T, int N, bool VEC_BC>
-__global__ void __launch_bounds__(kThreads, 4) pair_main(PairArgs p) {
+__global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
     using S = Stage<T, N>;
     constexpr int NP = N / 2;
     extern __shared__ __align__(16) char smem[];
