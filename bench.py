@@ -20,7 +20,6 @@ runs it.
 Rank 0 prints one JSON line.
 """
 import argparse
-import datetime
 import json
 import math
 import os
@@ -58,6 +57,26 @@ def peaks():
                     source="measured")
     except Exception:
         return dict(hbm_gbs=6650.0, sm_max_mhz=1965.0, source="fallback")
+
+
+def profiled_traffic(w):
+    """DRAM bytes per launch of pair_main from the committed ncu summary of this workload,
+    or None when there is none or the kernel source changed since it was captured."""
+    import hashlib
+    import re
+
+    path = os.path.join(ROOT, "profiles", f"ncu_scan_kernels_{w.name}.md")
+    src = os.path.join(ROOT, "vision_mamba_selective_b200", "csrc", "scan_kernels.cuh")
+    try:
+        text = open(path).read()
+        fp = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch pair_main: (\d+)", text)
+    f = re.search(r"kernel source fingerprint \(sha256 of scan_kernels.cuh, first 16 hex\): ([0-9a-f]+)", text)
+    if not m or not f or f.group(1) != fp:
+        return None
+    return int(m.group(1))
 
 
 def algorithmic(w):
@@ -227,18 +246,18 @@ def main():
     import torch
     import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from vision_mamba_selective_b200 import replicas
+
+    rank, local, world = replicas.env_rank_world()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        replicas.init("nccl", device=dev)
 
     from vision_mamba_selective_b200 import vimscan as vs
 
     # ---- inputs: rank-specific seed; enough rotating copies to exceed L2 ---------
-    host = wl.make_inputs(w, seed=w.seed + 7919 * rank)
+    host = wl.make_inputs(w, seed=replicas.rank_seed(w.seed, rank))
     act_keys = ["u", "delta", "z", "B", "C"]
     set_bytes = sum(host[k].numel() * host[k].element_size() for k in act_keys) + \
         w.tok_ch * (4 if w.dtype == "f32" else 2)
@@ -261,16 +280,10 @@ def main():
         fn(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"], params["delta_bias"],
            y=s["y"], workspace=ws, events=events)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    barrier = replicas.barrier
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(v, device=dev)
 
     for i in range(args.warmup):
         step(i)
@@ -344,7 +357,8 @@ def main():
     achieved_ops = ops / (main_ms * 1e-3) / 1e12
     roofline = {
         "bound": "alu", "kernel": "pair_main", "achieved": achieved_ops, "peak": peak_ops,
-        "unit": "Tops/s", "frac": achieved_ops / peak_ops, "traffic": None,
+        "unit": "Tops/s", "frac": achieved_ops / peak_ops, "traffic": profiled_traffic(w),
+        "algorithmic_bytes": nbytes,
         "ops_per_launch": ops, "ms_per_launch": main_ms,
         "peak_basis": f"{SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x {pk['sm_max_mhz']:.0f} MHz",
         "hbm_gbs_whole_step": nbytes / (ms_step * 1e-3) / 1e9,
