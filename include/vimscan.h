@@ -148,6 +148,38 @@ vim_status vmamba_cross_scan4_events(const void *u, const void *delta, const voi
                                      cudaEvent_t *events);
 
 /*
+ * vim_scan_bidir for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this call; it is a packaging variant.  Some
+ * callers cannot hand the scan a workspace: code running where cudaMalloc is not
+ * allowed or not wanted (inside a stream capture that must not allocate, under an
+ * allocator that owns all device memory, or from a plugin with no allocator of its
+ * own).  This entry point takes the same inputs and output as vim_scan_bidir, without
+ * a workspace, and keeps the chunk carries in a buffer built into the library: a
+ * file-scope device array of VIM_NOALLOC_SCRATCH_BYTES bytes, which every GPU that
+ * loads the library holds until the process exits.  The call allocates nothing.
+ *
+ *   - Limit: the problem must need at most VIM_NOALLOC_SCRATCH_BYTES of scratch, that
+ *     is vim_scan_workspace_bytes(0, batch, L, 0, d_inner, d_state) <= that size
+ *     (sequences of up to 256 tokens need none).  Larger problems return
+ *     VIM_ERR_WORKSPACE and launch nothing.
+ *   - The first call on each device looks up the buffer's device address (with that
+ *     device current) and remembers it; make that first call before any stream
+ *     capture.  A failed lookup returns VIM_ERR_CUDA.
+ *   - All calls share the one buffer, and it keeps whatever the last call left in it.
+ *     Nothing in it needs to start at zero: every value a call reads was written
+ *     earlier by the same call.  Calls whose work overlaps on the GPU (two streams,
+ *     or two threads with the same device) race on the buffer and corrupt each
+ *     other's results: serialise them.
+ */
+#define VIM_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+vim_status vim_scan_bidir_noalloc(const void *u, const void *delta, const void *z,
+                                  const void *B, const void *C, int64_t bc_dir_stride,
+                                  const float *A, const float *D, const float *delta_bias,
+                                  void *y, int batch, int L, int d_inner, int d_state,
+                                  vim_dtype dt, cudaStream_t stream);
+
+/*
  * Workspace bytes the scan entry points need (0 when none).  which = 0 for
  * vim_scan_bidir (L_or_H = L, W ignored), 1 for vmamba_cross_scan4 (L_or_H = H).
  * Returns 0 for invalid arguments as well; the entry point then reports them.

@@ -7,6 +7,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "scan_kernels.cuh"
 
@@ -311,6 +312,50 @@ vim_status cross_merge4(const void *ys, const void *z, void *y, int batch, int H
     else
         merge4<__nv_bfloat16><<<blocks, 256, 0, stream>>>(a);
     return cudaGetLastError() == cudaSuccess ? VIM_OK : VIM_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------------------
+// the no-allocation variant of vim_scan_bidir (declared in vimscan.h)
+// ----------------------------------------------------------------------------
+// The built-in scratch buffer.  In host code its name only stands in for the symbol:
+// the device address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char vim_noalloc_scratch[VIM_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_addr[kMaxDevices] = {};
+
+// device address of the scratch buffer on the current device (looked up on first use)
+vim_status noalloc_scratch(void **addr) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return VIM_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, vim_noalloc_scratch) != cudaSuccess || !p) return VIM_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *addr = g_noalloc_addr[dev];
+    return VIM_OK;
+}
+}  // namespace
+
+vim_status vim_scan_bidir_noalloc(const void *u, const void *delta, const void *z, const void *B,
+                                  const void *C, int64_t bc_dir_stride, const float *A,
+                                  const float *D, const float *delta_bias, void *y, int batch,
+                                  int L, int d_inner, int d_state, vim_dtype dt,
+                                  cudaStream_t stream) {
+    vim_status st = check_common(batch, L, d_inner, d_state, dt);
+    if (st != VIM_OK) return st;
+    if (summary_bytes(batch, L, d_inner, d_state) > VIM_NOALLOC_SCRATCH_BYTES) return VIM_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    if (batch > 0 && L > 0 && d_inner > 0) {
+        st = noalloc_scratch(&scratch);
+        if (st != VIM_OK) return st;
+    }
+    return vim_scan_bidir(u, delta, z, B, C, bc_dir_stride, A, D, delta_bias, y, batch, L, d_inner,
+                          d_state, dt, scratch, VIM_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"

@@ -36,6 +36,10 @@ lib.vim_scan_bidir_events.argtypes = lib.vim_scan_bidir.argtypes + [_vp]
 lib.vim_scan_bidir_events.restype = _i
 lib.vmamba_cross_scan4_events.argtypes = lib.vmamba_cross_scan4.argtypes + [_vp]
 lib.vmamba_cross_scan4_events.restype = _i
+lib.vim_scan_bidir_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
+                                       _i, _i, _i, _i, _i, _vp]
+lib.vim_scan_bidir_noalloc.restype = _i
+VIM_NOALLOC_SCRATCH_BYTES = 8 << 20
 lib.cross_merge4.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
 lib.cross_merge4.restype = _i
 lib.vim_scan_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
@@ -128,6 +132,30 @@ def vim_scan_bidir(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride
         batch, L, Di, N, dt, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream), *extra)
     if st != VIM_OK:
         raise VimScanError(st, "vim_scan_bidir")
+    return y
+
+
+def vim_scan_bidir_noalloc(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride=0, stream=None):
+    """vim_scan_bidir without a workspace, for callers that cannot allocate device memory.
+
+    The chunk carries live in a fixed buffer inside the library
+    (VIM_NOALLOC_SCRATCH_BYTES), shared by every call: calls must not overlap on the GPU.
+    Problems needing more scratch than that raise VimScanError (VIM_ERR_WORKSPACE).
+    ``y`` must be given by callers that cannot allocate; otherwise it is allocated here.
+    """
+    batch, L, Di = u.shape
+    N = B.shape[-1]
+    dt = _dtype_code(u)
+    if y is None:
+        y = torch.empty_like(u)
+    st = lib.vim_scan_bidir_noalloc(
+        _ptr(u, name="u"), _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
+        _ptr(B, dtype=u.dtype, name="B"), _ptr(C, dtype=u.dtype, name="C"), int(bc_dir_stride),
+        _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
+        _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(y, dtype=u.dtype, name="y"),
+        batch, L, Di, N, dt, _stream(stream))
+    if st != VIM_OK:
+        raise VimScanError(st, "vim_scan_bidir_noalloc")
     return y
 
 
