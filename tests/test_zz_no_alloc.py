@@ -71,10 +71,12 @@ def test_single_chunk_needs_no_scratch(vs):
 
 
 def test_too_large_is_refused(vs):
-    # 16385 tokens x 256 channels needs more carry scratch than the built-in buffer
-    need = vs.vim_scan_workspace_bytes(0, 1, 16385, 0, 256, 16)
-    assert need > vs.VIM_NOALLOC_SCRATCH_BYTES
-    x = make(1, 16385, 256, 16, torch.bfloat16, 7)
+    # the smallest batch of 16385-token, 256-channel sequences whose carries do not fit
+    L, Di, N = 16385, 256, 16
+    batch = 1
+    while vs.vim_scan_workspace_bytes(0, batch, L, 0, Di, N) <= vs.VIM_NOALLOC_SCRATCH_BYTES:
+        batch += 1
+    x = make(batch, L, Di, N, torch.bfloat16, 7)
     y = torch.full_like(x["u"], float("nan"))
     with pytest.raises(vs.VimScanError) as e:
         vs.vim_scan_bidir_noalloc(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["bias"], y=y)

@@ -203,31 +203,20 @@ __device__ __forceinline__ int position(const PairArgs &p, int t) {
 // ----------------------------------------------------------------------------
 // shared-memory staging of one step: the forward tile and the backward tile
 // ----------------------------------------------------------------------------
-// One slot: [dir][u|delta][kTile][kDC] T | [dir][B|C][kTile][N] fp32 |
-//           [dir][kTile][kDC] T (z)     | [dir][kTile][kDC] fp32 (partial_in, optional)
+// One slot: [dir][u|delta][kTile][kDC] T | [dir][B|C][kTile][N] fp32
 template <typename T, int N>
 struct Stage {
-    static constexpr int kUV = kTile * kDC;                  // elements per u, delta or z tile
+    static constexpr int kUV = kTile * kDC;                  // elements per u or delta tile
     static constexpr int kBC = kTile * N;                    // elements per B or C tile
     static constexpr int kUVBytes = 2 * 2 * kUV * (int)sizeof(T);
     static constexpr int kBCBytes = 2 * 2 * kBC * 4;
-    static constexpr int kZBytes = 2 * kUV * (int)sizeof(T);
-    static constexpr int kPinBytes = 2 * kUV * 4;
+    static constexpr int kSlotBytes = kUVBytes + kBCBytes;
 
-    __host__ __device__ static constexpr int slot_bytes(bool pin) {
-        return kUVBytes + kBCBytes + kZBytes + (pin ? kPinBytes : 0);
-    }
     __device__ static T *uv(char *slot, int dir, int which) {
         return reinterpret_cast<T *>(slot) + (dir * 2 + which) * kUV;
     }
     __device__ static float *bc(char *slot, int dir, int which) {
         return reinterpret_cast<float *>(slot + kUVBytes) + (dir * 2 + which) * kBC;
-    }
-    __device__ static T *zt(char *slot, int dir) {
-        return reinterpret_cast<T *>(slot + kUVBytes + kBCBytes) + dir * kUV;
-    }
-    __device__ static float *pin(char *slot, int dir) {
-        return reinterpret_cast<float *>(slot + kUVBytes + kBCBytes + kZBytes) + dir * kUV;
     }
 };
 
@@ -244,8 +233,8 @@ template <typename T, int N>
 constexpr bool bc_vectorizable() { return (N * sizeof(T)) % 16 == 0; }
 
 // Loads of one step (tile jf of the forward direction, jb of the backward one):
-// u/delta (and z, partial_in on the steps that complete a tile) by cp.async straight
-// into the slot, B/C into registers first and then, converted to fp32, into the slot.
+// u/delta by cp.async straight into the slot, B/C into registers first and then,
+// converted to fp32, into the slot.
 // Rows past the end of the chunk and channels past d_inner are zero-filled, so that
 // they act as no-op tokens.
 template <typename T, int N, bool VEC_BC>
@@ -254,8 +243,6 @@ struct Stager {
     static constexpr int V = Vec<T>::n;                 // elements per 16-byte piece
     static constexpr int kRowPieces = kDC / V;          // pieces per u/delta row
     static constexpr int kUVRep = kTile * kRowPieces / kThreads;   // pieces per thread per tensor
-    static constexpr int kPinRowPieces = kDC / 4;
-    static constexpr int kPinRep = kTile * kPinRowPieces / kThreads;
     static constexpr int kBCRow = VEC_BC ? (int)(N * sizeof(T) / 16) : N;   // units per B/C row
     static constexpr int kBCUnits = 4 * kTile * kBCRow;
     static constexpr int kBCPer = (kBCUnits + kThreads - 1) / kThreads;
@@ -276,12 +263,10 @@ struct Stager {
         return ((size_t)b * p.L + position(p, t0 + j * kTile + r)) * p.Di + ch;
     }
 
-    // u and delta; with `aux`, also z (if gated) and partial_in (if present)
-    __device__ void issue(char *slot, int jf, int jb, bool aux) const {
+    // u and delta of both tiles
+    __device__ void issue(char *slot, int jf, int jb) const {
         const T *gu = static_cast<const T *>(p.u);
         const T *gd = static_cast<const T *>(p.delta);
-        const T *gz = static_cast<const T *>(p.z);
-        const bool with_z = aux && gz != nullptr;
 #pragma unroll
         for (int dir = 0; dir < 2; ++dir) {
             const int j = dir ? jb : jf;
@@ -297,24 +282,11 @@ struct Stager {
                     const size_t off = row_off(j, r, ch);
                     cp_async16(S::uv(slot, dir, 0) + so, gu + off, true);
                     cp_async16(S::uv(slot, dir, 1) + so, gd + off, true);
-                    if (with_z) cp_async16(S::zt(slot, dir) + so, gz + off, true);
                 } else {
                     // outside the data: u = 0 and delta_raw = -1e4, so that Delta =
                     // softplus(-1e4 + bias) = 0 exactly (Abar = 1, Bbar u = 0): a no-op token
                     *reinterpret_cast<uint4 *>(S::uv(slot, dir, 0) + so) = make_uint4(0, 0, 0, 0);
                     *reinterpret_cast<uint4 *>(S::uv(slot, dir, 1) + so) = pad16<T>(-1.0e4f);
-                    if (with_z) *reinterpret_cast<uint4 *>(S::zt(slot, dir) + so) = make_uint4(0, 0, 0, 0);
-                }
-            }
-            if (aux && p.partial_in) {
-#pragma unroll
-                for (int m = 0; m < kPinRep; ++m) {
-                    const int li = threadIdx.x + m * kThreads;
-                    const int v = li % kPinRowPieces, r = li / kPinRowPieces;
-                    const int ch = d0 + v * 4;
-                    const bool ok = r < rows && ch < p.Di;
-                    const size_t off = ok ? row_off(j, r, ch) : 0;
-                    cp_async16(S::pin(slot, dir) + r * kDC + v * 4, p.partial_in + off, ok);
                 }
             }
         }
@@ -460,7 +432,7 @@ template <typename T, int N, bool VEC_BC>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_carry(PairArgs p) {
     using S = Stage<T, N>;
     constexpr int NP = N / 2;
-    constexpr int kSlot = S::slot_bytes(false);
+    constexpr int kSlot = S::kSlotBytes;
     extern __shared__ __align__(16) char smem[];
 
     const int b = blockIdx.z, c = blockIdx.y, d0 = blockIdx.x * kDC;
@@ -476,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_carry(PairArgs p) {
 
     // the forward direction walks tiles nT-1 .. 0, the backward one 0 .. nT-1
     Stager<T, N, VEC_BC> st(p, b, t0, tc, d0);
-    st.issue(smem, nT - 1, 0, false);
+    st.issue(smem, nT - 1, 0);
     st.load_bc(nT - 1, 0);
     st.store_bc(smem);
     cp_async_wait_all();
@@ -491,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_carry(PairArgs p) {
         char *cur = smem + (s & 1) * kSlot;
         char *nxt = smem + ((s + 1) & 1) * kSlot;
         if (s + 1 < nT) {
-            st.issue(nxt, nT - 2 - s, s + 1, false);
+            st.issue(nxt, nT - 2 - s, s + 1);
             st.load_bc(nT - 2 - s, s + 1);
         }
         if (active) {
@@ -568,50 +540,33 @@ __global__ void __launch_bounds__(256) pair_combine(PairArgs p) {
     }
 }
 
+// acc (+)= V consecutive floats (16-byte aligned), V a multiple of 4
+template <int V, bool ADD>
+__device__ __forceinline__ void add_f32(float (&acc)[V], const float *src) {
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+    for (int q = 0; q < V / 4; ++q) {
+        const float4 a = s4[q];
+        if (ADD) {
+            acc[4 * q] += a.x; acc[4 * q + 1] += a.y; acc[4 * q + 2] += a.z; acc[4 * q + 3] += a.w;
+        } else {
+            acc[4 * q] = a.x; acc[4 * q + 1] = a.y; acc[4 * q + 2] = a.z; acc[4 * q + 3] = a.w;
+        }
+    }
+}
+
 // ----------------------------------------------------------------------------
 // kernel 3: both directions over one chunk, merge, gate, store
 // ----------------------------------------------------------------------------
-// Where one thread's outputs go: rows of a tile lie at base + r * rstride elements
-// unless the tile wraps into the next grid column (column-major order only).
-template <typename T>
-struct OutRows {
-    size_t base, rstride;
-    bool linear;
-    int j, d;         // tile index and channel (for the exact fallback)
-};
-
-template <typename T, int N, bool VEC_BC>
-__device__ __forceinline__ OutRows<T> out_rows(const Stager<T, N, VEC_BC> &st, const PairArgs &p, int j,
-                                               int rows, int d) {
-    OutRows<T> o;
-    const int t = st.t0 + j * kTile;
-    o.j = j;
-    o.d = d;
-    if (p.order == 0) {
-        o.linear = true;
-        o.base = ((size_t)st.b * p.L + t) * p.Di + d;
-        o.rstride = (size_t)p.Di;
-    } else {
-        o.linear = (t % p.H) + rows <= p.H;
-        o.base = ((size_t)st.b * p.L + position(p, t)) * p.Di + d;
-        o.rstride = (size_t)p.W * p.Di;
-    }
-    return o;
-}
-
 // One direction's pass over one staged tile: the softplus, Delta*u and decay base of
 // kSub tokens are formed first (independent of h), then the recurrence runs through
-// them.  Rows past the tile's end are no-op tokens and store nothing.  First visit:
-// the partial output goes to ypart.  Second visit: it is added to the partial left
-// there, the gate applied and the result stored (or, for the first pair of the
-// cross-scan, the ungated fp32 sum).
-template <typename T, int N, bool VEC_BC, bool FAST, bool DESC>
-__device__ __forceinline__ void main_tile(bool second, int rows, float2 (&h)[N / 2],
-                                          const ChannelParams<N> &prm, int dl, const T *su,
-                                          const T *sd, const float *sB, const float *sC,
-                                          float *ypart, const T *sz, const float *spin,
-                                          const Stager<T, N, VEC_BC> &st, const PairArgs &p,
-                                          const OutRows<T> &o) {
+// them.  Rows past the tile's end are no-op tokens.  The output of each token goes
+// to the chunk's fp32 partial buffer: stored on the tile's first visit, added on the
+// second (rows past the end only touch unread rows of the buffer).
+template <typename T, int N, bool FAST, bool DESC>
+__device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], const ChannelParams<N> &prm,
+                                          int dl, const T *su, const T *sd, const float *sB,
+                                          const float *sC, float *ypart) {
     constexpr int NP = N / 2;
 #pragma unroll 1
     for (int sub = 0; sub < kTile / kSub; ++sub) {
@@ -664,31 +619,120 @@ __device__ __forceinline__ void main_tile(bool second, int rows, float2 (&h)[N /
             }
             const float2 ys = __fadd2_rn(y0, y1);
             const float yv = fmaf(prm.D, uv[k], ys.x + ys.y);
-            if (!second) {
-                ypart[r * kDC] = yv;   // rows past the end land inside the chunk buffer, unread
-            } else if (r < rows) {
-                float tot = ypart[r * kDC] + yv;
-                if (spin) tot += spin[r * kDC + dl];
-                const size_t off = o.linear ? o.base + (size_t)r * o.rstride : st.row_off(o.j, r, o.d);
-                if (p.partial_out) {
-                    p.partial_out[off] = tot;
-                } else {
-                    if (sz) tot *= silu(to_f32(sz[r * kDC + dl]));
-                    static_cast<T *>(p.y)[off] = T(tot);
-                }
-            }
+            float *py = ypart + r * kDC;
+            *py = second ? *py + yv : yv;
         }
     }
 }
 
-template <typename T, int N, bool VEC_BC>
+// Completion of the tiles a step finishes.  A tile is complete once both directions
+// have visited it; its sums sit in the chunk buffer (the middle tile of an odd tile
+// count keeps the backward half in ymid).  Each thread finishes one 8-channel vector
+// of one row per completed tile: it adds partial_in (the first pair's sum, for the
+// second pair of the cross-scan), applies silu(z) and stores 16 or 32 bytes; the first
+// pair of the cross-scan stores its ungated fp32 sum instead.  z and partial_in are
+// loaded into registers at the start of the step, so their latency hides behind it.
+template <typename T, bool PIN>
+struct Finisher {
+    static constexpr int kG = 8;                                    // channels per vector
+    static constexpr int kZ = kG * (int)sizeof(T) / 16;             // uint4 of z per vector
+    uint4 z[2][kZ];
+    float4 pin[2][PIN ? 2 : 1];
+    int ntiles, tile[2];
+
+    __device__ int row() const { return threadIdx.x / (kDC / kG); }
+    __device__ int group() const { return threadIdx.x % (kDC / kG); }
+
+    // the tiles completed by step s (none before the middle of the chunk)
+    __device__ void plan(int s, int nT) {
+        ntiles = 0;
+        if (2 * s < nT - 1) return;
+        tile[0] = s;
+        tile[1] = nT - 1 - s;
+        ntiles = tile[0] == tile[1] ? 1 : 2;
+    }
+
+    template <int N, bool VEC_BC>
+    __device__ void prefetch(const Stager<T, N, VEC_BC> &st, const PairArgs &p) {
+        const int r = row(), ch = st.d0 + group() * kG;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            if (i >= ntiles) break;
+            const int j = tile[i];
+            if (r >= st.rows_of(j) || ch >= p.Di) continue;
+            const size_t off = st.row_off(j, r, ch);
+            if (p.z) {
+                const uint4 *zs = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.z) + off);
+#pragma unroll
+                for (int q = 0; q < kZ; ++q)
+                    if (sizeof(T) == 2 || ch + 4 * q < p.Di) z[i][q] = zs[q];
+            }
+            if constexpr (PIN) {
+                const float4 *ps = reinterpret_cast<const float4 *>(p.partial_in + off);
+                pin[i][0] = ps[0];
+                if (ch + 4 < p.Di) pin[i][1] = ps[1];
+            }
+        }
+    }
+
+    template <int N, bool VEC_BC>
+    __device__ void finish(const Stager<T, N, VEC_BC> &st, const PairArgs &p, const float *ybuf,
+                           const float *ymid) const {
+        const int r = row(), cl = group() * kG, ch = st.d0 + cl;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            if (i >= ntiles) break;
+            const int j = tile[i];
+            if (r >= st.rows_of(j) || ch >= p.Di) continue;
+            float acc[kG];
+            add_f32<kG, false>(acc, ybuf + (size_t)(j * kTile + r) * kDC + cl);
+            if (ntiles == 1) add_f32<kG, true>(acc, ymid + r * kDC + cl);
+            if constexpr (PIN) {
+                acc[0] += pin[i][0].x; acc[1] += pin[i][0].y; acc[2] += pin[i][0].z; acc[3] += pin[i][0].w;
+                acc[4] += pin[i][1].x; acc[5] += pin[i][1].y; acc[6] += pin[i][1].z; acc[7] += pin[i][1].w;
+            }
+            const size_t off = st.row_off(j, r, ch);
+            const bool whole = ch + kG <= p.Di;   // fp32 channel counts may end half-way
+            if (p.partial_out) {
+                float4 *po = reinterpret_cast<float4 *>(p.partial_out + off);
+                po[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                if (whole) po[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+                continue;
+            }
+            if (p.z) {
+                float zf[kG];
+                if constexpr (sizeof(T) == 2) {
+                    unpack16(z[i][0], zf);
+                } else {
+                    float a4[4], b4[4];
+                    unpack16(z[i][0], a4);
+                    unpack16(z[i][kZ - 1], b4);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) { zf[e] = a4[e]; zf[4 + e] = b4[e]; }
+                }
+#pragma unroll
+                for (int e = 0; e < kG; ++e) acc[e] *= silu(zf[e]);
+            }
+            uint4 *yo = reinterpret_cast<uint4 *>(static_cast<T *>(p.y) + off);
+            if constexpr (sizeof(T) == 2) {
+                yo[0] = pack16(acc);
+            } else {
+                float a4[4] = {acc[0], acc[1], acc[2], acc[3]}, b4[4] = {acc[4], acc[5], acc[6], acc[7]};
+                yo[0] = pack16(a4);
+                if (whole) yo[1] = pack16(b4);
+            }
+        }
+    }
+};
+
+template <typename T, int N, bool VEC_BC, bool PIN>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
     using S = Stage<T, N>;
     constexpr int NP = N / 2;
+    constexpr int kSlot = S::kSlotBytes;
     extern __shared__ __align__(16) char smem[];
-    const int slot_bytes = S::slot_bytes(p.partial_in != nullptr);
-    float *ybuf = reinterpret_cast<float *>(smem + 2 * slot_bytes);   // [chunk][kDC]
-    float *ymid = ybuf + (size_t)p.chunk * kDC;                        // [kTile][kDC]
+    float *ybuf = reinterpret_cast<float *>(smem + 2 * kSlot);   // [chunk][kDC]
+    float *ymid = ybuf + (size_t)p.chunk * kDC;                   // [kTile][kDC]
 
     const int b = blockIdx.z, c = blockIdx.y, d0 = blockIdx.x * kDC;
     const int dir = threadIdx.x / kDC, dl = threadIdx.x % kDC, d = d0 + dl;
@@ -710,43 +754,39 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
         for (int k = 0; k < NP; ++k) h[k] = hin[k];
     }
 
-    // step s completes the tiles it visits when 2s >= nT-1 (z/partial_in needed then)
-    auto completes = [&](int s) { return 2 * s >= nT - 1; };
     Stager<T, N, VEC_BC> st(p, b, t0, tc, d0);
-    st.issue(smem, 0, nT - 1, completes(0));
+    st.issue(smem, 0, nT - 1);
     st.load_bc(0, nT - 1);
     st.store_bc(smem);
     cp_async_wait_all();
     __syncthreads();
 
+    Finisher<T, PIN> fin;
     for (int s = 0; s < nT; ++s) {
-        char *cur = smem + (s & 1) * slot_bytes;
-        char *nxt = smem + ((s + 1) & 1) * slot_bytes;
+        char *cur = smem + (s & 1) * kSlot;
+        char *nxt = smem + ((s + 1) & 1) * kSlot;
         if (s + 1 < nT) {
-            st.issue(nxt, s + 1, nT - 2 - s, completes(s + 1));
+            st.issue(nxt, s + 1, nT - 2 - s);
             st.load_bc(s + 1, nT - 2 - s);
         }
-        const int j = dir ? nT - 1 - s : s;
-        const int rows = st.rows_of(j);
+        fin.plan(s, nT);
+        fin.prefetch(st, p);
         // the forward direction visits tile j at step j, the backward one at nT-1-j:
-        // the first visitor stores its partial, the second completes the output; when
-        // both come in the same step (the middle tile) the backward one writes aside
-        // to ymid and the tile is finished after the step
+        // the first visitor stores its partial, the second adds to it; when both come
+        // in the same step (the middle tile) the backward one writes to ymid instead
+        const int j = dir ? nT - 1 - s : s;
         const int twice = 2 * s - (nT - 1);
         float *ypart = (twice == 0 && dir == 1) ? ymid + dl : ybuf + (size_t)j * kTile * kDC + dl;
         if (prm.valid) {
             const T *su = S::uv(cur, dir, 0), *sd = S::uv(cur, dir, 1);
             const float *sB = S::bc(cur, dir, 0), *sC = S::bc(cur, dir, 1);
-            const T *sz = p.z ? S::zt(cur, dir) : nullptr;
-            const float *spin = p.partial_in ? S::pin(cur, dir) : nullptr;
-            const OutRows<T> o = out_rows(st, p, j, rows, d);
             const bool second = twice > 0;
             if (dir == 0) {
-                if (fast) main_tile<T, N, VEC_BC, true, false>(second, rows, h, prm, dl, su, sd, sB, sC, ypart, sz, spin, st, p, o);
-                else main_tile<T, N, VEC_BC, false, false>(second, rows, h, prm, dl, su, sd, sB, sC, ypart, sz, spin, st, p, o);
+                if (fast) main_tile<T, N, true, false>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                else main_tile<T, N, false, false>(second, h, prm, dl, su, sd, sB, sC, ypart);
             } else {
-                if (fast) main_tile<T, N, VEC_BC, true, true>(second, rows, h, prm, dl, su, sd, sB, sC, ypart, sz, spin, st, p, o);
-                else main_tile<T, N, VEC_BC, false, true>(second, rows, h, prm, dl, su, sd, sB, sC, ypart, sz, spin, st, p, o);
+                if (fast) main_tile<T, N, true, true>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                else main_tile<T, N, false, true>(second, h, prm, dl, su, sd, sB, sC, ypart);
             }
         }
         if (s + 1 < nT) {
@@ -754,25 +794,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
             cp_async_wait_all();
         }
         __syncthreads();
-        if (twice == 0) {
-            // the middle tile: both partials are in shared memory; z and partial_in were
-            // staged for it in this step's slot (the two directions' tiles coincide)
-            const int jm = s, rm = st.rows_of(jm);
-            for (int i = threadIdx.x; i < rm * kDC; i += kThreads) {
-                const int r = i / kDC, cl = i % kDC, ch = d0 + cl;
-                if (ch >= p.Di) continue;
-                float tot = ybuf[((size_t)jm * kTile + r) * kDC + cl] + ymid[r * kDC + cl];
-                if (p.partial_in) tot += S::pin(cur, 0)[r * kDC + cl];
-                const size_t off = st.row_off(jm, r, ch);
-                if (p.partial_out) {
-                    p.partial_out[off] = tot;
-                } else {
-                    if (p.z) tot *= silu(to_f32(S::zt(cur, 0)[r * kDC + cl]));
-                    static_cast<T *>(p.y)[off] = T(tot);
-                }
-            }
-            __syncthreads();   // slot `cur` is refilled by the next step's loads
-        }
+        // the tiles this step completed are read by no later step of this chunk, so
+        // they can be finished while the next step runs without another barrier
+        fin.finish(st, p, ybuf, ymid);
     }
 }
 

@@ -18,7 +18,7 @@ namespace {
 #define VIMSCAN_SINGLE_CHUNK_MAX 256
 #endif
 #ifndef VIMSCAN_LONG_CHUNK
-#define VIMSCAN_LONG_CHUNK 64
+#define VIMSCAN_LONG_CHUNK 96
 #endif
 // sequences up to kSingleChunkMax tokens run as one chunk; longer ones in chunks of
 // kLongChunk tokens (a multiple of kTile), sized so that four CTAs of the main kernel
@@ -71,12 +71,12 @@ vim_status check_common(int batch, int L, int Di, int N, vim_dtype dt) {
 }
 
 template <typename T, int N>
-size_t main_smem(int chunk, bool pin) {
-    return 2 * (size_t)Stage<T, N>::slot_bytes(pin) + (size_t)chunk * kDC * 4 + (size_t)kTile * kDC * 4;
+size_t main_smem(int chunk) {
+    return 2 * (size_t)Stage<T, N>::kSlotBytes + (size_t)chunk * kDC * 4 + (size_t)kTile * kDC * 4;
 }
 template <typename T, int N>
 size_t carry_smem() {
-    return 2 * (size_t)Stage<T, N>::slot_bytes(false);
+    return 2 * (size_t)Stage<T, N>::kSlotBytes;
 }
 
 // events: null, or 3 events recorded after the carry, combine and main kernels
@@ -103,11 +103,18 @@ vim_status launch_pair_v(const PairArgs &a, cudaStream_t stream, cudaEvent_t *ev
     } else if (ev) {
         if (mark(ev, 0, stream) != VIM_OK || mark(ev, 1, stream) != VIM_OK) return VIM_ERR_CUDA;
     }
-    const size_t sm = main_smem<T, N>(a.chunk, a.partial_in != nullptr);
-    if (cudaFuncSetAttribute(pair_main<T, N, VEC_BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sm) != cudaSuccess)
-        return VIM_ERR_CUDA;
-    pair_main<T, N, VEC_BC><<<grid, kThreads, sm, stream>>>(a);
+    const size_t sm = main_smem<T, N>(a.chunk);
+    if (a.partial_in) {
+        if (cudaFuncSetAttribute(pair_main<T, N, VEC_BC, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sm) != cudaSuccess)
+            return VIM_ERR_CUDA;
+        pair_main<T, N, VEC_BC, true><<<grid, kThreads, sm, stream>>>(a);
+    } else {
+        if (cudaFuncSetAttribute(pair_main<T, N, VEC_BC, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sm) != cudaSuccess)
+            return VIM_ERR_CUDA;
+        pair_main<T, N, VEC_BC, false><<<grid, kThreads, sm, stream>>>(a);
+    }
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     return mark(ev, 2, stream);
 }
