@@ -39,8 +39,16 @@ constexpr int kTile = 16;            // tokens per staged tile
 #ifndef VIMSCAN_MIN_BLOCKS
 #define VIMSCAN_MIN_BLOCKS 4
 #endif
+#ifndef VIMSCAN_CARRY_KSUB
+#define VIMSCAN_CARRY_KSUB 8
+#endif
+#ifndef VIMSCAN_CARRY_MIN_BLOCKS
+#define VIMSCAN_CARRY_MIN_BLOCKS 6
+#endif
 constexpr int kSub = VIMSCAN_KSUB;   // tokens whose independent work is formed ahead of the recurrence
 constexpr int kMinBlocks = VIMSCAN_MIN_BLOCKS;   // resident CTAs per SM the register budget targets
+constexpr int kCarrySub = VIMSCAN_CARRY_KSUB;          // the same for the chunk-summary kernel
+constexpr int kCarryMinBlocks = VIMSCAN_CARRY_MIN_BLOCKS;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ----------------------------------------------------------------------------
@@ -390,19 +398,19 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
                                            int dl, const T *su, const T *sd, const float *sB) {
     constexpr int NP = N / 2;
 #pragma unroll 1
-    for (int sub = 0; sub < kTile / kSub; ++sub) {
-        float Sv[kSub], duv[kSub];
+    for (int sub = 0; sub < kTile / kCarrySub; ++sub) {
+        float Sv[kCarrySub], duv[kCarrySub];
 #pragma unroll
-        for (int k = 0; k < kSub; ++k) {
-            const int r = walk_row<DESC>(sub * kSub + k);
+        for (int k = 0; k < kCarrySub; ++k) {
+            const int r = walk_row<DESC>(sub * kCarrySub + k);
             const float dt = delta_of<T>(sd, r, dl, prm.bias);
             duv[k] = dt * to_f32(su[r * kDC + dl]);
             Sv[k] = Ssum;          // Delta of the tokens walked before this one
             Ssum += dt;
         }
 #pragma unroll
-        for (int k = 0; k < kSub; ++k) {
-            const int r = walk_row<DESC>(sub * kSub + k);
+        for (int k = 0; k < kCarrySub; ++k) {
+            const int r = walk_row<DESC>(sub * kCarrySub + k);
             float2 Bv[NP];
             load_row<NP>(sB + r * N, Bv);
             if constexpr (FAST) {
@@ -429,7 +437,7 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
 }
 
 template <typename T, int N, bool VEC_BC>
-__global__ void __launch_bounds__(kThreads, kMinBlocks) pair_carry(PairArgs p) {
+__global__ void __launch_bounds__(kThreads, kCarryMinBlocks) pair_carry(PairArgs p) {
     using S = Stage<T, N>;
     constexpr int NP = N / 2;
     constexpr int kSlot = S::kSlotBytes;
@@ -504,6 +512,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_carry(PairArgs p) {
 template <int N>
 __global__ void __launch_bounds__(256) pair_combine(PairArgs p) {
     constexpr int kAhead = 16;
+    // launched as a programmatic dependent of pair_carry: wait for its summaries
+    cudaGridDependencySynchronize();
     const int idx = blockIdx.x * blockDim.x + threadIdx.x;   // (b, dir, d, n), n fastest
     const int per_b = 2 * p.Di * N;
     if (idx >= p.batch * per_b) return;
@@ -511,32 +521,32 @@ __global__ void __launch_bounds__(256) pair_combine(PairArgs p) {
     const int dir = rem / (p.Di * N);
     const float A2n = p.A[rem] * kLog2e;                     // A is [2][Di][N]: same index
     // hloc[b][c][dir][d][n] and ssum[b][c][dir][d]: chunk c+1 lies per_b (per_b / N) further
-    const int step = dir ? -1 : 1;
     const int c0 = dir ? p.G - 1 : 0;
     float *hl = p.hloc + ((size_t)b * p.G + c0) * per_b + rem;
     const float *ss = p.ssum + ((size_t)b * p.G + c0) * (per_b / N) + rem / N;
-    const ptrdiff_t hstride = (ptrdiff_t)step * per_b, sstride = (ptrdiff_t)step * (per_b / N);
+    const int hs = dir ? -per_b : per_b, sstep = dir ? -(per_b / N) : per_b / N;
     float h = 0.0f;
     for (int i0 = 0; i0 < p.G; i0 += kAhead) {
+        const int cnt = min(kAhead, p.G - i0);
         float loc[kAhead], P[kAhead];
 #pragma unroll
         for (int k = 0; k < kAhead; ++k) {
-            if (i0 + k < p.G) {
-                loc[k] = hl[k * hstride];
-                P[k] = ss[k * sstride];
+            if (k < cnt) {
+                loc[k] = hl[k * hs];
+                P[k] = ss[k * sstep];
             }
         }
 #pragma unroll
         for (int k = 0; k < kAhead; ++k) P[k] = ex2(A2n * P[k]);   // exp(A_n * Ssum(c))
 #pragma unroll
         for (int k = 0; k < kAhead; ++k) {
-            if (i0 + k < p.G) {
-                hl[k * hstride] = h;                 // the state entering this chunk
-                h = fmaf(P[k], h, loc[k]);           // (unused after the last chunk)
+            if (k < cnt) {
+                hl[k * hs] = h;                 // the state entering this chunk
+                h = fmaf(P[k], h, loc[k]);      // (unused after the last chunk)
             }
         }
-        hl += kAhead * hstride;
-        ss += kAhead * sstride;
+        hl += kAhead * hs;
+        ss += kAhead * sstep;
     }
 }
 
@@ -743,10 +753,18 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
     prm.load(p, dir, d);
     const bool fast = __all_sync(0xffffffffu, prm.structured);
 
-    // state entering this chunk
+    Stager<T, N, VEC_BC> st(p, b, t0, tc, d0);
+    st.issue(smem, 0, nT - 1);
+    st.load_bc(0, nT - 1);
+
+    // state entering this chunk.  With several chunks this kernel is launched as a
+    // programmatic dependent of pair_combine (whose own predecessor, pair_carry, was an
+    // ordinary launch, so the inputs were complete before the chain began): everything
+    // above only reads the inputs; the carries are read after the wait.
     float2 h[NP];
 #pragma unroll
     for (int k = 0; k < NP; ++k) h[k] = f2(0.f, 0.f);
+    if (p.G > 1) cudaGridDependencySynchronize();
     if (p.G > 1 && (dir == 0 ? c > 0 : c < p.G - 1) && prm.valid) {
         const size_t base = (((size_t)b * p.G + c) * 2 + dir) * p.Di + d;
         const float2 *hin = reinterpret_cast<const float2 *>(p.hloc + base * N);
@@ -754,9 +772,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
         for (int k = 0; k < NP; ++k) h[k] = hin[k];
     }
 
-    Stager<T, N, VEC_BC> st(p, b, t0, tc, d0);
-    st.issue(smem, 0, nT - 1);
-    st.load_bc(0, nT - 1);
     st.store_bc(smem);
     cp_async_wait_all();
     __syncthreads();

@@ -79,6 +79,32 @@ size_t carry_smem() {
     return 2 * (size_t)Stage<T, N>::kSlotBytes;
 }
 
+// Launch of a kernel that may start while the previous kernel on the stream drains
+// (programmatic dependent launch); the kernel itself waits, with
+// cudaGridDependencySynchronize, before it reads anything that kernel writes.
+#ifndef VIMSCAN_PDL
+#define VIMSCAN_PDL 1
+#endif
+template <typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Args...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, Args... args) {
+    if (!VIMSCAN_PDL) {
+        kernel<<<grid, block, smem, stream>>>(args...);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // events: null, or 3 events recorded after the carry, combine and main kernels
 inline vim_status mark(cudaEvent_t *events, int i, cudaStream_t stream) {
     if (!events) return VIM_OK;
@@ -97,8 +123,9 @@ vim_status launch_pair_v(const PairArgs &a, cudaStream_t stream, cudaEvent_t *ev
         if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
         if (mark(ev, 0, stream) != VIM_OK) return VIM_ERR_CUDA;
         const int64_t units = (int64_t)a.batch * 2 * a.Di * N;
-        pair_combine<N><<<(unsigned)((units + 255) / 256), 256, 0, stream>>>(a);
-        if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+        if (launch_dependent(pair_combine<N>, dim3((unsigned)((units + 255) / 256)), dim3(256), 0, stream,
+                             a) != cudaSuccess)
+            return VIM_ERR_CUDA;
         if (mark(ev, 1, stream) != VIM_OK) return VIM_ERR_CUDA;
     } else if (ev) {
         if (mark(ev, 0, stream) != VIM_OK || mark(ev, 1, stream) != VIM_OK) return VIM_ERR_CUDA;
@@ -108,12 +135,24 @@ vim_status launch_pair_v(const PairArgs &a, cudaStream_t stream, cudaEvent_t *ev
         if (cudaFuncSetAttribute(pair_main<T, N, VEC_BC, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sm) != cudaSuccess)
             return VIM_ERR_CUDA;
-        pair_main<T, N, VEC_BC, true><<<grid, kThreads, sm, stream>>>(a);
+        if (a.G > 1) {
+            if (launch_dependent(pair_main<T, N, VEC_BC, true>, grid, dim3(kThreads), sm, stream, a) !=
+                cudaSuccess)
+                return VIM_ERR_CUDA;
+        } else {
+            pair_main<T, N, VEC_BC, true><<<grid, kThreads, sm, stream>>>(a);
+        }
     } else {
         if (cudaFuncSetAttribute(pair_main<T, N, VEC_BC, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sm) != cudaSuccess)
             return VIM_ERR_CUDA;
-        pair_main<T, N, VEC_BC, false><<<grid, kThreads, sm, stream>>>(a);
+        if (a.G > 1) {
+            if (launch_dependent(pair_main<T, N, VEC_BC, false>, grid, dim3(kThreads), sm, stream, a) !=
+                cudaSuccess)
+                return VIM_ERR_CUDA;
+        } else {
+            pair_main<T, N, VEC_BC, false><<<grid, kThreads, sm, stream>>>(a);
+        }
     }
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     return mark(ev, 2, stream);
