@@ -57,6 +57,8 @@ class Oracle:
         lib.oracle_cross_scan4.argtypes = [_D] * 9 + [ctypes.c_int] * 6
         lib.oracle_cross_merge4.argtypes = [_D, _D, _D] + [ctypes.c_int] * 4
         lib.oracle_cross_order.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _I64]
+        lib.oracle_conv_silu.argtypes = [_D, _D, _D, _D] + [ctypes.c_int] * 4
+        lib.oracle_vim_bidir_conv.argtypes = [_D, _D, _D, _D, _D, _D, _D, ctypes.c_int64, _D, _D, _D, _D] + [ctypes.c_int] * 5
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
         self.lib = lib
@@ -116,6 +118,41 @@ class Oracle:
                                        int(bool(delta_is_raw)))
         if rc:
             raise ValueError("oracle_vim_bidir: bad sizes")
+        return y
+
+    def conv_silu(self, x, w, cb, *, reversed=False):
+        """silu of the kernel-3 depthwise convolution (zero padding 1) in front of a
+        pathway; reversed=True for the backward pathway (taps x[t+1], x[t], x[t-1]).
+
+        x: [batch, L, Di]; w: [Di, 3]; cb: [Di].  Returns u [batch, L, Di].
+        """
+        x, w, cb = map(_f64, (x, w, cb))
+        batch, L, Di = x.shape
+        u = np.zeros((batch, L, Di))
+        if self.lib.oracle_conv_silu(_p(x), _p(w), _p(cb), _p(u), batch, L, Di, int(bool(reversed))):
+            raise ValueError("oracle_conv_silu: bad sizes")
+        return u
+
+    def vim_bidir_conv(self, x, conv_w, conv_b, delta, z, B, C, A, D, bias, *, bc_dir_stride=0,
+                       delta_is_raw=True):
+        """Vim scan with its convolution front: u_f = silu(conv_f(x)), u_b = silu of
+        conv_b on the reversed sequence; then (y^f + y^b) * silu(z).
+
+        x, delta, z: [batch, L, Di]; conv_w: [2, Di, 3]; conv_b: [2, Di]; the rest as
+        in vim_bidir.
+        """
+        x, conv_w, conv_b, delta, z, B, C, A, D, bias = map(
+            _f64, (x, conv_w, conv_b, delta, z, B, C, A, D, bias))
+        batch, L, Di = x.shape
+        N = B.shape[-1]
+        if bias is None:
+            bias = np.zeros((2, Di))
+        y = np.zeros((batch, L, Di))
+        rc = self.lib.oracle_vim_bidir_conv(_p(x), _p(conv_w), _p(conv_b), _p(delta), _p(z), _p(B), _p(C),
+                                            int(bc_dir_stride), _p(A), _p(D), _p(bias), _p(y), batch, L, Di,
+                                            N, int(bool(delta_is_raw)))
+        if rc:
+            raise ValueError("oracle_vim_bidir_conv: bad sizes")
         return y
 
     def cross_scan4(self, u, delta, z, B, C, A, D, bias, *, delta_is_raw=True):
@@ -181,6 +218,14 @@ def vim_bidir(*a, **k):
 
 def cross_scan4(*a, **k):
     return default().cross_scan4(*a, **k)
+
+
+def conv_silu(*a, **k):
+    return default().conv_silu(*a, **k)
+
+
+def vim_bidir_conv(*a, **k):
+    return default().vim_bidir_conv(*a, **k)
 
 
 def cross_merge4(*a, **k):

@@ -136,6 +136,33 @@ int oracle_s6_direction(const double *u, const double *delta, const double *B, c
     return 0;
 }
 
+/*
+ * The smoothing in front of each pathway of the Vim block (page "Vision Mamba Guide",
+ * section "2. The Bidirectional Mamba Block" figure: "Linear Projection -> 1D Conv ->
+ * SiLU"; its PyTorch block: a depthwise Conv1d with kernel 3 and padding 1 per
+ * pathway, the backward one applied to the reversed sequence):
+ *   u_f[t] = silu(cb_f + w_f[0] x[t-1] + w_f[1] x[t] + w_f[2] x[t+1])
+ *   u_b[t] = silu(cb_b + w_b[0] x[t+1] + w_b[1] x[t] + w_b[2] x[t-1])
+ * with x = 0 outside 0..L-1 (u_b is the convolution of the reversed sequence, read
+ * back at original positions).  x, u: [batch, L, Di]; w: [Di][3]; cb: [Di].
+ */
+int oracle_conv_silu(const double *x, const double *w, const double *cb, double *u,
+                     int batch, int L, int Di, int reversed)
+{
+    if (batch < 0 || L < 0 || Di < 0) return -1;
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t t = 0; t < L; ++t)
+            for (int64_t d = 0; d < Di; ++d) {
+                double acc = cb[d];
+                for (int k = 0; k < 3; ++k) {
+                    int64_t s = reversed ? t + 1 - k : t + k - 1;   /* tap k reads x[s] */
+                    if (s >= 0 && s < L) acc += w[d * 3 + k] * x[(b * L + s) * Di + d];
+                }
+                u[(b * L + t) * Di + d] = silu(acc);
+            }
+    return 0;
+}
+
 /* y <- y * silu(z), elementwise over n values (skipped when z is NULL). */
 static void apply_gate(double *y, const double *z, int64_t n)
 {
@@ -169,6 +196,39 @@ int oracle_vim_bidir(const double *u, const double *delta, const double *z,
                               A + (int64_t)Di * N, D + Di, bias + Di, order, y,
                               batch, L, Di, N, delta_is_raw, 1);
     free(order);
+    if (rc) return -1;
+    apply_gate(y, z, (int64_t)batch * L * Di);
+    return 0;
+}
+
+/*
+ * The Vim block's scan with its convolution front: each pathway runs on its own
+ * smoothed input, u_f = oracle_conv_silu(x, w[0], cb[0], forward) and u_b =
+ * oracle_conv_silu(x, w[1], cb[1], reversed); the rest is oracle_vim_bidir.
+ *   conv_w [2][Di][3], conv_b [2][Di]; other arguments as in oracle_vim_bidir.
+ */
+int oracle_vim_bidir_conv(const double *x, const double *conv_w, const double *conv_b,
+                          const double *delta, const double *z,
+                          const double *B, const double *C, int64_t bc_dir_stride,
+                          const double *A, const double *D, const double *bias,
+                          double *y, int batch, int L, int Di, int N, int delta_is_raw)
+{
+    if (batch < 0 || L < 0 || Di < 0) return -1;
+    size_t n = (size_t)batch * (size_t)L * (size_t)Di;
+    double *uf = (double *)calloc(n > 0 ? n : 1, sizeof(double));
+    double *ub = (double *)calloc(n > 0 ? n : 1, sizeof(double));
+    int64_t *order = (int64_t *)calloc((size_t)(L > 0 ? L : 1), sizeof(int64_t));
+    int rc = (!uf || !ub || !order) ? -1 : 0;
+    if (!rc) rc |= oracle_conv_silu(x, conv_w, conv_b, uf, batch, L, Di, 0);
+    if (!rc) rc |= oracle_conv_silu(x, conv_w + (int64_t)Di * 3, conv_b + Di, ub, batch, L, Di, 1);
+    if (!rc) {
+        for (int64_t t = 0; t < L; ++t) order[t] = t;
+        rc |= oracle_s6_direction(uf, delta, B, C, A, D, bias, order, y, batch, L, Di, N, delta_is_raw, 0);
+        for (int64_t t = 0; t < L; ++t) order[t] = L - 1 - t;
+        rc |= oracle_s6_direction(ub, delta, B + bc_dir_stride, C + bc_dir_stride, A + (int64_t)Di * N,
+                                  D + Di, bias + Di, order, y, batch, L, Di, N, delta_is_raw, 1);
+    }
+    free(uf); free(ub); free(order);
     if (rc) return -1;
     apply_gate(y, z, (int64_t)batch * L * Di);
     return 0;

@@ -312,6 +312,62 @@ def pin_separate_bc(orc):
     np.testing.assert_allclose(y[0], np.array(ref), rtol=1e-12, atol=1e-12)
 
 
+def pin_conv_front_is_correlation(orc):
+    """The convolution in front of each pathway (section "2. The Bidirectional Mamba
+    Block": "1D Conv -> SiLU"; a depthwise kernel-3 convolution with padding 1, the
+    backward one on the reversed sequence).  With a large bias the SiLU is the
+    identity to within e^-40, so the pre-activation is read off and compared with
+    numpy's 'same'-mode correlation: directly for the forward pathway, and on the
+    reversed sequence, flipped back, for the backward one."""
+    rng = _rng(11)
+    b, L, Di = 2, 13, 3
+    x = rng.normal(size=(b, L, Di))
+    w = rng.normal(size=(Di, 3))
+    big = 60.0
+    cb = np.full(Di, big)
+    uf = orc.conv_silu(x, w, cb) - big
+    ub = orc.conv_silu(x, w, cb, reversed=True) - big
+    for bi in range(b):
+        for d in range(Di):
+            ref_f = np.correlate(x[bi, :, d], w[d], mode="same")
+            ref_b = np.correlate(x[bi, ::-1, d], w[d], mode="same")[::-1]
+            np.testing.assert_allclose(uf[bi, :, d], ref_f, rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(ub[bi, :, d], ref_b, rtol=1e-12, atol=1e-12)
+    # the activation is silu: the identity silu(v) - silu(-v) = v with w = (0, 1, 0)
+    e = np.zeros((Di, 3)); e[:, 1] = 1.0
+    np.testing.assert_allclose(orc.conv_silu(x, e, np.zeros(Di)) - orc.conv_silu(-x, e, np.zeros(Di)), x,
+                               rtol=1e-12, atol=1e-12)
+
+
+def pin_conv_scan_composition(orc):
+    """The scan with the convolution front is the plain bidirectional scan with each
+    direction fed its own smoothed input; and reversing the sequence while swapping
+    every per-direction parameter (weights, biases, B/C copies) reverses the output."""
+    rng = _rng(12)
+    c = _vim_case(rng, L=10)
+    x = rng.normal(size=c["u"].shape)
+    cw = rng.normal(size=(2, 3, 3))
+    cbias = rng.normal(size=(2, 3))
+    y = orc.vim_bidir_conv(x, cw, cbias, c["delta"], c["z"], c["B"], c["C"], c["A"], c["D"], c["bias"],
+                           bc_dir_stride=c["stride"], delta_is_raw=True)
+    uf = orc.conv_silu(x, cw[0], cbias[0])
+    ub = orc.conv_silu(x, cw[1], cbias[1], reversed=True)
+    L = x.shape[1]
+    yf = orc.s6_direction(uf, c["delta"], c["B"][0], c["C"][0], c["A"][0], c["D"][0], c["bias"][0],
+                          np.arange(L), delta_is_raw=True)
+    yb = orc.s6_direction(ub, c["delta"], c["B"][1], c["C"][1], c["A"][1], c["D"][1], c["bias"][1],
+                          np.arange(L)[::-1], delta_is_raw=True)
+    gate_ref = orc.vim_bidir(np.ones_like(x), np.zeros_like(x), c["z"], c["B"], c["C"], c["A"],
+                             np.stack([np.ones(3), np.zeros(3)]), c["bias"], bc_dir_stride=c["stride"],
+                             delta_is_raw=False)   # = silu(z): Delta = 0, D_f = 1, u = 1
+    np.testing.assert_allclose(y, (yf + yb) * gate_ref, rtol=1e-12, atol=1e-12)
+    flip = lambda a: np.ascontiguousarray(a[..., ::-1, :])
+    y2 = orc.vim_bidir_conv(flip(x), cw[::-1].copy(), cbias[::-1].copy(), flip(c["delta"]), flip(c["z"]),
+                            flip(c["B"][::-1]), flip(c["C"][::-1]), c["A"][::-1].copy(), c["D"][::-1].copy(),
+                            c["bias"][::-1].copy(), bc_dir_stride=c["stride"], delta_is_raw=True)
+    np.testing.assert_allclose(y, flip(y2), rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [
     pin_delta_zero,
     pin_constant_input_geometric,
@@ -325,4 +381,6 @@ ALL_PINS = [
     pin_cross_scan_is_transpose_and_flip,
     pin_cross_merge,
     pin_separate_bc,
+    pin_conv_front_is_correlation,
+    pin_conv_scan_composition,
 ]

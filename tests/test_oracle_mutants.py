@@ -36,6 +36,12 @@ MUTANTS = {
     "merge_ignores_order": ("int64_t p = order[t];\n                for (int64_t c = 0",
                             "int64_t p = t;\n                for (int64_t c = 0"),
     "delta_bias_ignored": ("softplus(delta[ix] + bias[d])", "softplus(delta[ix])"),
+    "conv_backward_taps_forward": ("int64_t s = reversed ? t + 1 - k : t + k - 1;",
+                                   "int64_t s = t + k - 1;"),
+    "conv_bias_dropped": ("double acc = cb[d];", "double acc = 0.0;"),
+    "conv_no_silu": ("u[(b * L + t) * Di + d] = silu(acc);", "u[(b * L + t) * Di + d] = acc;"),
+    "conv_backward_uses_forward_weights": ("oracle_conv_silu(x, conv_w + (int64_t)Di * 3, conv_b + Di, ub",
+                                           "oracle_conv_silu(x, conv_w, conv_b, ub"),
 }
 
 
