@@ -2,12 +2,15 @@
 """Throughput of the bidirectional selective scan (S6) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--conv]
 
 One step is one pass of the whole scan -- softplus Delta, the forward and backward
 recurrences, readout, D skip, the merge of the directions and the silu(z) gate --
 over one batch of the workload, through the library's C ABI.  The default workload
 is the 1024 px Vim-Tiny scan (batch 8, L = 4097, d_inner 384, d_state 16, bf16 I/O,
 fp32 state).  Inputs are seeded synthetic tensors shaped like the pages' workloads.
+--conv times the same scan with the pathways' kernel-3 convolution + SiLU fused in
+front (the input tensor is then x, the convolutions' input).
 
 Multi-GPU (torchrun, one process per GPU): the batch items are independent, so every
 rank runs the same workload on its own inputs with no collective on the data path
@@ -46,6 +49,8 @@ def parse():
     ap.add_argument("--workload", default="vim_tiny_1024px_bf16")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--conv", action="store_true",
+                    help="Vim workloads: time the scan with the fused kernel-3 convolution + SiLU front")
     return ap.parse_args()
 
 
@@ -79,7 +84,7 @@ def profiled_traffic(w):
     return int(m.group(1))
 
 
-def algorithmic(w):
+def algorithmic(w, conv=False):
     """Algorithmic bytes and FP32 lane-ops of one step.
 
     Bytes: one read of u, delta_raw, z and one write of y per token-channel, one read
@@ -90,7 +95,7 @@ def algorithmic(w):
     el = 4 if w.dtype == "f32" else 2
     n_bc_sets = 1 if w.kind == "vim" else w.directions
     bc = 2 * w.batch * w.tokens * w.d_state * el * n_bc_sets
-    params = w.directions * w.channels * (w.d_state + 2) * 4
+    params = w.directions * w.channels * (w.d_state + 2 + (4 if conv else 0)) * 4
     nbytes = 4 * w.tok_ch * el + bc + params
     ops = 4 * w.d_state * w.directions * w.tok_ch
     return nbytes, ops
@@ -153,19 +158,34 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+def conv_params(w, seed):
+    """Depthwise kernel-3 weights [2, channels, 3] and biases [2, channels] of the two
+    pathways' convolution front, uniform in +-1/sqrt(3) (a default Conv1d init)."""
+    import torch
+
+    g = torch.Generator().manual_seed(seed)
+    k = 3 ** -0.5
+    cw = (torch.rand((2, w.channels, 3), generator=g) * 2 - 1) * k
+    cb = (torch.rand((2, w.channels), generator=g) * 2 - 1) * k
+    return cw.contiguous(), cb.contiguous()
+
+
 def run_oracle(w, x, threads):
     import oracle
 
     oracle.set_threads(threads)
     t = time.perf_counter()
-    if w.kind == "vim":
+    if "conv_w" in x:
+        oracle.vim_bidir_conv(x["u"], x["conv_w"], x["conv_b"], x["delta"], x["z"], x["B"], x["C"], x["A"],
+                              x["D"], x["delta_bias"])
+    elif w.kind == "vim":
         oracle.vim_bidir(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"])
     else:
         oracle.cross_scan4(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"])
     return time.perf_counter() - t
 
 
-def oracle_sample(w, target_s):
+def oracle_sample(w, target_s, conv=False):
     """A bounded sample of the workload for the oracle: its first batch items and
     first channels at the full sequence length, sized for about ``target_s`` seconds
     of fp64 work on the host cores (calibrated on a small run)."""
@@ -173,6 +193,8 @@ def oracle_sample(w, target_s):
 
     cores = cpu_cores()
     full = wl.make_inputs(w)
+    if conv:
+        full["conv_w"], full["conv_b"] = conv_params(w, w.seed + 1)
     step = 8
 
     def cut(b, c):
@@ -183,7 +205,7 @@ def oracle_sample(w, target_s):
             elif k in ("B", "C"):
                 x[k] = (v[:b] if w.kind == "vim" else v[:, :b]).contiguous()
             else:
-                x[k] = v[..., :c, :].contiguous() if k == "A" else v[..., :c].contiguous()
+                x[k] = v[..., :c, :].contiguous() if k in ("A", "conv_w") else v[..., :c].contiguous()
         return w.scaled(batch=b, channels=c), x
 
     cal_c = min(w.channels, 64)
@@ -212,7 +234,7 @@ def reference_arm(args, w):
     if rank != 0:
         return
     per_step = min(2.0, 150.0 / max(1, args.steps + args.warmup))
-    s, x, cores = oracle_sample(w, per_step)
+    s, x, cores = oracle_sample(w, per_step, conv=args.conv)
     for _ in range(args.warmup):
         run_oracle(s, x, cores)
     times = [run_oracle(s, x, cores) for _ in range(args.steps)]
@@ -225,7 +247,7 @@ def reference_arm(args, w):
         "value": value, "unit": "tok*ch/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "batch_per_gpu": w.batch, "tokens": w.tokens,
+        "config": {"workload": workload_name(w, args), "batch_per_gpu": w.batch, "tokens": w.tokens,
                    "channels": w.channels, "d_state": w.d_state, "io_dtype": w.dtype},
         "cpu_baseline": {"value": value, "unit": "tok*ch/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
@@ -234,11 +256,17 @@ def reference_arm(args, w):
     print(json.dumps(line), flush=True)
 
 
+def workload_name(w, args):
+    return w.name + ("+conv_front" if args.conv else "")
+
+
 def main():
     args = parse()
     from vision_mamba_selective_b200 import workloads as wl
 
     w = wl.BY_NAME[args.workload]
+    if args.conv and w.kind != "vim":
+        raise SystemExit("--conv applies to the Vim workloads only")
     if args.impl == "reference":
         reference_arm(args, w)
         return
@@ -274,9 +302,18 @@ def main():
         ws_bytes = vs.vim_scan_workspace_bytes(1, w.batch, w.H, w.W, w.channels, w.d_state)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     fn = vs.vim_scan_bidir if w.kind == "vim" else vs.vmamba_cross_scan4
+    if args.conv:
+        cw, cb = conv_params(w, w.seed + 1)
+        params["conv_w"], params["conv_b"] = cw.to(dev), cb.to(dev)
 
     def step(i, events=None):
         s = sets[i % nsets]
+        if args.conv:
+            # u holds x, the pathways' common input in front of the convolutions
+            vs.vim_scan_bidir_conv(s["u"], params["conv_w"], params["conv_b"], s["delta"], s["z"], s["B"],
+                                   s["C"], params["A"], params["D"], params["delta_bias"], y=s["y"],
+                                   workspace=ws, events=events)
+            return
         fn(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"], params["delta_bias"],
            y=s["y"], workspace=ws, events=events)
 
@@ -320,8 +357,8 @@ def main():
             a = 1 + 3 * p + k
             t = [evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(prof_steps)]
             per_kernel[f"{names[k]}[{p}]" if pairs > 1 else names[k]] = sum(t) / len(t)
-    G = math.ceil(w.tokens / 128) if w.tokens > 256 else 1
-    launches_per_step = pairs * (3 if G > 1 else 1)
+    # sequences longer than one chunk (256 tokens) take carry, combine and main
+    launches_per_step = pairs * (3 if w.tokens > 256 else 1)
 
     # ---- end to end: pinned host inputs -> device -> scan -> host result ---------
     pinned = {k: host[k].pin_memory() for k in act_keys}
@@ -350,7 +387,7 @@ def main():
 
     # ---- roofline of the dominant kernel -----------------------------------------
     pk = peaks()
-    nbytes, ops = algorithmic(w)
+    nbytes, ops = algorithmic(w, args.conv)
     main_ms = sum(v for k, v in per_kernel.items() if k.startswith("pair_main"))
     clocks = clk.summary()
     peak_ops = SMS * FP32_LANES_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e12
@@ -368,7 +405,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        s, x, cores = oracle_sample(w, 5.0)
+        s, x, cores = oracle_sample(w, 5.0, conv=args.conv)
         sec = run_oracle(s, x, cores)
         cpu = {"value": s.tok_ch / sec, "unit": "tok*ch/s", "cores": cores, "kind": "oracle",
                "sample": f"{s.batch} of {w.batch} batch items x {s.channels} of {w.channels} channels "
@@ -381,7 +418,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded, shaped like the pages' workloads)",
-            "config": {"workload": w.name, "batch_per_gpu": w.batch, "tokens": w.tokens,
+            "config": {"workload": workload_name(w, args), "batch_per_gpu": w.batch, "tokens": w.tokens,
                        "channels": w.channels, "d_state": w.d_state, "io_dtype": w.dtype,
                        "parallelism": f"replicas x{world} (batch shards, no collective)",
                        "l2": f"{nsets} rotating input sets of {set_bytes / 1e6:.0f} MB (> 126 MB L2)"},

@@ -86,6 +86,39 @@ vim_status vim_scan_bidir(const void *u, const void *delta, const void *z,
                           void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * vim_scan_bidir with the pathways' convolution front fused in (section "2. The
+ * Bidirectional Mamba Block": each pathway runs "1D Conv -> SiLU" before its S6; the
+ * page's block uses a depthwise Conv1d of kernel 3 and padding 1, the backward one on
+ * the reversed sequence):
+ *
+ *   u_f[b,t,d] = silu(conv_b[0][d] + w[0][d][0] x[t-1] + w[0][d][1] x[t] + w[0][d][2] x[t+1])
+ *   u_b[b,t,d] = silu(conv_b[1][d] + w[1][d][0] x[t+1] + w[1][d][1] x[t] + w[1][d][2] x[t-1])
+ *   (x = 0 outside 0..L-1; silu(v) = v / (1 + exp(-v)))
+ *
+ * and then exactly vim_scan_bidir with the forward direction fed u_f and the backward
+ * one u_b (each direction's D skip uses its own u).  The smoothed inputs are formed in
+ * registers from the staged x and never written to memory.
+ *
+ *   x       : [batch, L, d_inner] (dt), the pathways' common input.
+ *   conv_w  : [2, d_inner, 3] fp32 (index 0 = forward); conv_b : [2, d_inner] fp32.
+ *   all other arguments and the workspace as in vim_scan_bidir.
+ */
+vim_status vim_scan_bidir_conv(const void *x, const float *conv_w, const float *conv_b,
+                               const void *delta, const void *z, const void *B, const void *C,
+                               int64_t bc_dir_stride, const float *A, const float *D,
+                               const float *delta_bias, void *y, int batch, int L, int d_inner,
+                               int d_state, vim_dtype dt, void *workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+
+/* vim_scan_bidir_conv with the per-kernel events of vim_scan_bidir_events. */
+vim_status vim_scan_bidir_conv_events(const void *x, const float *conv_w, const float *conv_b,
+                                      const void *delta, const void *z, const void *B, const void *C,
+                                      int64_t bc_dir_stride, const float *A, const float *D,
+                                      const float *delta_bias, void *y, int batch, int L, int d_inner,
+                                      int d_state, vim_dtype dt, void *workspace, size_t workspace_bytes,
+                                      cudaStream_t stream, cudaEvent_t *events);
+
+/*
  * VMamba four-direction cross-scan with CS-Merge (sections "1. Cross-Scan
  * Traversal", "2. Parallel S6 State Space Processing", "3. Cross-Merge Reversal"):
  *

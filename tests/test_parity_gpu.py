@@ -6,7 +6,8 @@ with the tolerances of the target: 1e-5 for fp32 I/O and 2e-2 for bf16 I/O (fp32
 state in both).  Shapes cover several chunks and tiles with ragged tails, channel
 counts that leave a partial block of 64, d_state 2..16, general (not S4D-real) A,
 the softplus cut at 20, large |z|, empty inputs, and the five full-size workloads
-in the launch configuration the benchmark times.
+in the launch configuration the benchmark times, and the same over the fused
+convolution front.
 """
 import json
 import os
@@ -144,6 +145,81 @@ def test_vim_deterministic(vs):
     assert torch.equal(y1, y2)
 
 
+def conv_params(Di, seed):
+    """Depthwise kernel-3 weights and biases of the two pathways, drawn like a
+    default-initialised Conv1d (uniform in +-1/sqrt(3), fan-in 3)."""
+    g = torch.Generator().manual_seed(seed)
+    k = 1 / np.sqrt(3)
+    w = (torch.rand((2, Di, 3), generator=g) * 2 - 1) * k
+    b = (torch.rand((2, Di), generator=g) * 2 - 1) * k
+    return w.contiguous(), b.contiguous()
+
+
+def run_vim_conv(vs, x, w, b, gate=True):
+    dev = lambda t: t.cuda()
+    y = vs.vim_scan_bidir_conv(dev(x["u"]), dev(w), dev(b), dev(x["delta"]), dev(x["z"]) if gate else None,
+                               dev(x["B"]), dev(x["C"]), dev(x["A"]), dev(x["D"]), dev(x["bias"]),
+                               bc_dir_stride=x["stride"])
+    torch.cuda.synchronize()
+    return y
+
+
+def ref_vim_conv(x, w, b, gate=True):
+    return oracle.vim_bidir_conv(x["u"], w, b, x["delta"], x["z"] if gate else None, x["B"], x["C"], x["A"],
+                                 x["D"], x["bias"], bc_dir_stride=x["stride"])
+
+
+CONV_CASES = [
+    # batch, L, Di, N, dtype, generic_A, separate_bc, gate
+    (1, 1, 8, 16, torch.float32, False, False, True),        # both taps fall in the padding
+    (1, 2, 64, 16, torch.float32, False, False, True),
+    (2, 17, 72, 16, torch.bfloat16, False, True, True),      # tile edge + 1 token
+    (1, 32, 64, 8, torch.float32, True, False, False),       # two whole tiles
+    (2, 197, 200, 16, torch.float32, False, False, True),
+    (1, 256, 64, 16, torch.bfloat16, False, False, True),    # longest single chunk
+    (2, 257, 72, 16, torch.float32, False, True, True),      # chunk edges with 1-token tail
+    (1, 300, 64, 4, torch.float32, True, False, True),
+    (1, 1000, 136, 16, torch.bfloat16, False, False, True),
+    (2, 1111, 64, 16, torch.float32, False, False, True),
+    (1, 400, 36, 16, torch.float32, True, True, True),
+]
+
+
+@pytest.mark.parametrize("case", CONV_CASES, ids=lambda c: f"b{c[0]}_L{c[1]}_D{c[2]}_N{c[3]}_{str(c[4])[6:]}"
+                         f"{'_genA' if c[5] else ''}{'_sepBC' if c[6] else ''}{'' if c[7] else '_nogate'}")
+def test_vim_conv(vs, case):
+    """The convolution front fused into the scan: every output against the oracle's
+    conv + SiLU followed by the two-direction scan, over chunk and tile edges (the
+    taps read one token across each)."""
+    batch, L, Di, N, dtype, gen, sep, gate = case
+    x = vim_inputs(batch, L, Di, N, dtype, seed=L * 11 + Di, generic_A=gen, separate_bc=sep)
+    w, b = conv_params(Di, seed=L + Di)
+    check(f"vim_conv_{case}", run_vim_conv(vs, x, w, b, gate), ref_vim_conv(x, w, b, gate), dtype)
+
+
+def test_vim_conv_identity_taps_is_plain_scan(vs):
+    """Taps (0, 1, 0) with a bias that makes SiLU the identity on the inputs' range are
+    the plain scan of x + bias: the fused path and vim_scan_bidir on x + bias agree."""
+    x = vim_inputs(2, 300, 64, 16, torch.float32, seed=21)
+    w = torch.zeros(2, 64, 3)
+    w[:, :, 1] = 1
+    b = torch.full((2, 64), 40.0)
+    y_conv = run_vim_conv(vs, x, w, b)
+    x2 = dict(x, u=(x["u"] + 40.0).contiguous())
+    y_plain = run_vim(vs, x2)
+    err = normwise(y_conv, y_plain.double().cpu().numpy())
+    assert err < 1e-6, err
+
+
+def test_vim_conv_rejects_missing_weights(vs):
+    x = vim_inputs(1, 20, 64, 16, torch.float32, seed=2)
+    w, b = conv_params(64, seed=2)
+    d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
+    with pytest.raises(vs.VimScanError):
+        vs.vim_scan_bidir_conv(d["u"], w.cuda(), None, d["delta"], d["z"], d["B"], d["C"], d["A"], d["D"],
+                               d["bias"])
+
+
 def cross_inputs(batch, H, W, Ch, N, dtype, seed, generic_A=False):
     g = torch.Generator().manual_seed(seed)
     r = lambda *s, std=1.0: (torch.randn(s, generator=g) * std)
@@ -249,3 +325,19 @@ def test_full_size(vs, w):
         ref = oracle.cross_scan4(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"])
     torch.cuda.synchronize()
     check(f"full_{w.name}", y, ref, w.torch_dtype())
+
+
+def test_full_size_conv(vs):
+    """The fused convolution front at the full size of the 1024 px Vim-Ti workload
+    (bf16), against the oracle on every output."""
+    w = wl.BY_NAME["vim_tiny_1024px_bf16"]
+    x = wl.make_inputs(w)
+    cw, cb = conv_params(w.channels, seed=4242)
+    oracle.set_threads(max(1, len(os.sched_getaffinity(0))))
+    dev = {k: v.cuda() for k, v in x.items()}
+    y = vs.vim_scan_bidir_conv(dev["u"], cw.cuda(), cb.cuda(), dev["delta"], dev["z"], dev["B"], dev["C"],
+                               dev["A"], dev["D"], dev["delta_bias"])
+    torch.cuda.synchronize()
+    ref = oracle.vim_bidir_conv(x["u"], cw, cb, x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"],
+                                x["delta_bias"])
+    check("full_conv_vim_tiny_1024px_bf16", y, ref, w.torch_dtype())

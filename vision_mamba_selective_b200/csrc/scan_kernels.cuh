@@ -191,6 +191,8 @@ struct PairArgs {
     const float *A;                 // [2][Di][N]: forward, backward
     const float *D;                 // [2][Di]
     const float *bias;              // [2][Di]
+    const float *conv_w;            // [2][Di][3] convolution front of the pathways, or null
+    const float *conv_b;            // [2][Di]
     void *y;                        // final output [batch, L, Di] (element type), or null
     float *partial_out;             // fp32 [batch, L, Di] (ungated pair sum), or null
     const float *partial_in;        // fp32 [batch, L, Di] added before the gate, or null
@@ -211,17 +213,20 @@ __device__ __forceinline__ int position(const PairArgs &p, int t) {
 // ----------------------------------------------------------------------------
 // shared-memory staging of one step: the forward tile and the backward tile
 // ----------------------------------------------------------------------------
-// One slot: [dir][u|delta][kTile][kDC] T | [dir][B|C][kTile][N] fp32
-template <typename T, int N>
+// One slot: per direction [u rows][kDC] T then [delta rows][kDC] T, then
+// [dir][B|C][kTile][N] fp32.  With the convolution front (CONV) the u area holds the
+// raw input x with one halo row on each side: row rr is token row rr - 1.
+template <typename T, int N, bool CONV = false>
 struct Stage {
-    static constexpr int kUV = kTile * kDC;                  // elements per u or delta tile
+    static constexpr int kURows = CONV ? kTile + 2 : kTile;
+    static constexpr int kDirUV = (kURows + kTile) * kDC;   // elements per direction
     static constexpr int kBC = kTile * N;                    // elements per B or C tile
-    static constexpr int kUVBytes = 2 * 2 * kUV * (int)sizeof(T);
+    static constexpr int kUVBytes = 2 * kDirUV * (int)sizeof(T);
     static constexpr int kBCBytes = 2 * 2 * kBC * 4;
     static constexpr int kSlotBytes = kUVBytes + kBCBytes;
 
     __device__ static T *uv(char *slot, int dir, int which) {
-        return reinterpret_cast<T *>(slot) + (dir * 2 + which) * kUV;
+        return reinterpret_cast<T *>(slot) + dir * kDirUV + (which ? kURows * kDC : 0);
     }
     __device__ static float *bc(char *slot, int dir, int which) {
         return reinterpret_cast<float *>(slot + kUVBytes) + (dir * 2 + which) * kBC;
@@ -245,9 +250,9 @@ constexpr bool bc_vectorizable() { return (N * sizeof(T)) % 16 == 0; }
 // converted to fp32, into the slot.
 // Rows past the end of the chunk and channels past d_inner are zero-filled, so that
 // they act as no-op tokens.
-template <typename T, int N, bool VEC_BC>
+template <typename T, int N, bool VEC_BC, bool CONV = false>
 struct Stager {
-    using S = Stage<T, N>;
+    using S = Stage<T, N, CONV>;
     static constexpr int V = Vec<T>::n;                 // elements per 16-byte piece
     static constexpr int kRowPieces = kDC / V;          // pieces per u/delta row
     static constexpr int kUVRep = kTile * kRowPieces / kThreads;   // pieces per thread per tensor
@@ -271,7 +276,7 @@ struct Stager {
         return ((size_t)b * p.L + position(p, t0 + j * kTile + r)) * p.Di + ch;
     }
 
-    // u and delta of both tiles
+    // u and delta of both tiles (with CONV: x and its halo rows instead of u)
     __device__ void issue(char *slot, int jf, int jb) const {
         const T *gu = static_cast<const T *>(p.u);
         const T *gd = static_cast<const T *>(p.delta);
@@ -288,13 +293,27 @@ struct Stager {
                 const int so = r * kDC + v * V;
                 if (ok) {
                     const size_t off = row_off(j, r, ch);
-                    cp_async16(S::uv(slot, dir, 0) + so, gu + off, true);
+                    if (!CONV) cp_async16(S::uv(slot, dir, 0) + so, gu + off, true);
                     cp_async16(S::uv(slot, dir, 1) + so, gd + off, true);
                 } else {
                     // outside the data: u = 0 and delta_raw = -1e4, so that Delta =
                     // softplus(-1e4 + bias) = 0 exactly (Abar = 1, Bbar u = 0): a no-op token
-                    *reinterpret_cast<uint4 *>(S::uv(slot, dir, 0) + so) = make_uint4(0, 0, 0, 0);
+                    if (!CONV) *reinterpret_cast<uint4 *>(S::uv(slot, dir, 0) + so) = make_uint4(0, 0, 0, 0);
                     *reinterpret_cast<uint4 *>(S::uv(slot, dir, 1) + so) = pad16<T>(-1.0e4f);
+                }
+            }
+            if constexpr (CONV) {
+                // x rows -1 .. kTile of the tile (the convolution's neighbours), zero
+                // outside the sequence (the convolution's zero padding)
+                for (int li = threadIdx.x; li < S::kURows * kRowPieces; li += kThreads) {
+                    const int v = li % kRowPieces, rr = li / kRowPieces;
+                    const int ch = d0 + v * V;
+                    const int t = t0 + j * kTile + rr - 1;
+                    T *dst = S::uv(slot, dir, 0) + rr * kDC + v * V;
+                    if (t >= 0 && t < p.L && ch < p.Di)
+                        cp_async16(dst, gu + ((size_t)b * p.L + t) * p.Di + ch, true);
+                    else
+                        *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
                 }
             }
         }
@@ -356,6 +375,7 @@ struct ChannelParams {
     const float *A;     // A[dir][d][:] (general-A path)
     float A0;           // A[d][0] * log2(e)
     float D, bias;
+    float cw_prev, cw_cur, cw_next, cbias;   // convolution front: taps on x[t-1], x[t], x[t+1]
     bool structured;    // A[d][n] == (n+1) A[d][0] for every n
     bool valid;
 
@@ -363,8 +383,18 @@ struct ChannelParams {
         valid = d < p.Di;
         structured = true;
         A0 = D = bias = 0.0f;
+        cw_prev = cw_cur = cw_next = cbias = 0.0f;
         A = p.A;
         if (!valid) return;
+        if (p.conv_w) {
+            // forward: w[0] x[t-1] + w[1] x[t] + w[2] x[t+1]; the backward pathway
+            // convolves the reversed sequence: w[0] x[t+1] + w[1] x[t] + w[2] x[t-1]
+            const float *w = p.conv_w + ((size_t)dir * p.Di + d) * 3;
+            cw_prev = dir ? w[2] : w[0];
+            cw_cur = w[1];
+            cw_next = dir ? w[0] : w[2];
+            cbias = p.conv_b[(size_t)dir * p.Di + d];
+        }
         A = p.A + ((size_t)dir * p.Di + d) * N;
         const float a0 = A[0];
 #pragma unroll
@@ -378,6 +408,21 @@ struct ChannelParams {
 // row of the tile that step i of a walk over it visits (ascending or descending)
 template <bool DESC>
 __device__ __forceinline__ int walk_row(int i) { return DESC ? kTile - 1 - i : i; }
+
+// u of one staged row: the input itself, or, with the convolution front, silu of the
+// kernel-3 convolution of the staged x rows around it (section "2. The Bidirectional
+// Mamba Block": "1D Conv -> SiLU" on each pathway)
+template <typename T, int N, bool CONV>
+__device__ __forceinline__ float u_of(const T *su, int r, int dl, const ChannelParams<N> &prm) {
+    if constexpr (!CONV) {
+        return to_f32(su[r * kDC + dl]);
+    } else {
+        const float v = fmaf(prm.cw_prev, to_f32(su[r * kDC + dl]),
+                             fmaf(prm.cw_cur, to_f32(su[(r + 1) * kDC + dl]),
+                                  fmaf(prm.cw_next, to_f32(su[(r + 2) * kDC + dl]), prm.cbias)));
+        return silu(v);
+    }
+}
 
 // Delta of one staged row (rows past the tile end hold delta_raw = -1e4: Delta = 0)
 template <typename T>
@@ -393,7 +438,7 @@ __device__ __forceinline__ float delta_of(const T *sd, int r, int dl, float bias
 // Delta summed over the tokens the direction visits after s inside the chunk.  With
 // A_n = (n+1) A_0 the weights are powers of w = exp(A_0 S_s), built by one multiply
 // per state.
-template <typename T, int N, bool FAST, bool DESC>
+template <typename T, int N, bool FAST, bool DESC, bool CONV>
 __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, const ChannelParams<N> &prm,
                                            int dl, const T *su, const T *sd, const float *sB) {
     constexpr int NP = N / 2;
@@ -404,7 +449,7 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
         for (int k = 0; k < kCarrySub; ++k) {
             const int r = walk_row<DESC>(sub * kCarrySub + k);
             const float dt = delta_of<T>(sd, r, dl, prm.bias);
-            duv[k] = dt * to_f32(su[r * kDC + dl]);
+            duv[k] = dt * u_of<T, N, CONV>(su, r, dl, prm);
             Sv[k] = Ssum;          // Delta of the tokens walked before this one
             Ssum += dt;
         }
@@ -436,9 +481,9 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
     }
 }
 
-template <typename T, int N, bool VEC_BC>
+template <typename T, int N, bool VEC_BC, bool CONV>
 __global__ void __launch_bounds__(kThreads, kCarryMinBlocks) pair_carry(PairArgs p) {
-    using S = Stage<T, N>;
+    using S = Stage<T, N, CONV>;
     constexpr int NP = N / 2;
     constexpr int kSlot = S::kSlotBytes;
     extern __shared__ __align__(16) char smem[];
@@ -455,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, kCarryMinBlocks) pair_carry(PairArgs
     const bool fast = __all_sync(0xffffffffu, prm.structured);
 
     // the forward direction walks tiles nT-1 .. 0, the backward one 0 .. nT-1
-    Stager<T, N, VEC_BC> st(p, b, t0, tc, d0);
+    Stager<T, N, VEC_BC, CONV> st(p, b, t0, tc, d0);
     st.issue(smem, nT - 1, 0);
     st.load_bc(nT - 1, 0);
     st.store_bc(smem);
@@ -478,11 +523,11 @@ __global__ void __launch_bounds__(kThreads, kCarryMinBlocks) pair_carry(PairArgs
             const T *su = S::uv(cur, dir, 0), *sd = S::uv(cur, dir, 1);
             const float *sB = S::bc(cur, dir, 0);
             if (dir == 0) {
-                if (fast) carry_tile<T, N, true, true>(H, Ssum, prm, dl, su, sd, sB);
-                else carry_tile<T, N, false, true>(H, Ssum, prm, dl, su, sd, sB);
+                if (fast) carry_tile<T, N, true, true, CONV>(H, Ssum, prm, dl, su, sd, sB);
+                else carry_tile<T, N, false, true, CONV>(H, Ssum, prm, dl, su, sd, sB);
             } else {
-                if (fast) carry_tile<T, N, true, false>(H, Ssum, prm, dl, su, sd, sB);
-                else carry_tile<T, N, false, false>(H, Ssum, prm, dl, su, sd, sB);
+                if (fast) carry_tile<T, N, true, false, CONV>(H, Ssum, prm, dl, su, sd, sB);
+                else carry_tile<T, N, false, false, CONV>(H, Ssum, prm, dl, su, sd, sB);
             }
         }
         if (s + 1 < nT) {
@@ -573,7 +618,7 @@ __device__ __forceinline__ void add_f32(float (&acc)[V], const float *src) {
 // them.  Rows past the tile's end are no-op tokens.  The output of each token goes
 // to the chunk's fp32 partial buffer: stored on the tile's first visit, added on the
 // second (rows past the end only touch unread rows of the buffer).
-template <typename T, int N, bool FAST, bool DESC>
+template <typename T, int N, bool FAST, bool DESC, bool CONV>
 __device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], const ChannelParams<N> &prm,
                                           int dl, const T *su, const T *sd, const float *sB,
                                           const float *sC, float *ypart) {
@@ -585,7 +630,7 @@ __device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], const
         for (int k = 0; k < kSub; ++k) {
             const int r = walk_row<DESC>(sub * kSub + k);
             const float dt = delta_of<T>(sd, r, dl, prm.bias);
-            uv[k] = to_f32(su[r * kDC + dl]);
+            uv[k] = u_of<T, N, CONV>(su, r, dl, prm);
             duv[k] = dt * uv[k];
             qv[k] = FAST ? ex2(dt * prm.A0) : dt;
         }
@@ -662,8 +707,8 @@ struct Finisher {
         ntiles = tile[0] == tile[1] ? 1 : 2;
     }
 
-    template <int N, bool VEC_BC>
-    __device__ void prefetch(const Stager<T, N, VEC_BC> &st, const PairArgs &p) {
+    template <class ST>
+    __device__ void prefetch(const ST &st, const PairArgs &p) {
         const int r = row(), ch = st.d0 + group() * kG;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
@@ -685,8 +730,8 @@ struct Finisher {
         }
     }
 
-    template <int N, bool VEC_BC>
-    __device__ void finish(const Stager<T, N, VEC_BC> &st, const PairArgs &p, const float *ybuf,
+    template <class ST>
+    __device__ void finish(const ST &st, const PairArgs &p, const float *ybuf,
                            const float *ymid) const {
         const int r = row(), cl = group() * kG, ch = st.d0 + cl;
 #pragma unroll
@@ -735,9 +780,9 @@ struct Finisher {
     }
 };
 
-template <typename T, int N, bool VEC_BC, bool PIN>
+template <typename T, int N, bool VEC_BC, bool PIN, bool CONV>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
-    using S = Stage<T, N>;
+    using S = Stage<T, N, CONV>;
     constexpr int NP = N / 2;
     constexpr int kSlot = S::kSlotBytes;
     extern __shared__ __align__(16) char smem[];
@@ -753,7 +798,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
     prm.load(p, dir, d);
     const bool fast = __all_sync(0xffffffffu, prm.structured);
 
-    Stager<T, N, VEC_BC> st(p, b, t0, tc, d0);
+    Stager<T, N, VEC_BC, CONV> st(p, b, t0, tc, d0);
     st.issue(smem, 0, nT - 1);
     st.load_bc(0, nT - 1);
 
@@ -797,11 +842,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
             const float *sB = S::bc(cur, dir, 0), *sC = S::bc(cur, dir, 1);
             const bool second = twice > 0;
             if (dir == 0) {
-                if (fast) main_tile<T, N, true, false>(second, h, prm, dl, su, sd, sB, sC, ypart);
-                else main_tile<T, N, false, false>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                if (fast) main_tile<T, N, true, false, CONV>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                else main_tile<T, N, false, false, CONV>(second, h, prm, dl, su, sd, sB, sC, ypart);
             } else {
-                if (fast) main_tile<T, N, true, true>(second, h, prm, dl, su, sd, sB, sC, ypart);
-                else main_tile<T, N, false, true>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                if (fast) main_tile<T, N, true, true, CONV>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                else main_tile<T, N, false, true, CONV>(second, h, prm, dl, su, sd, sB, sC, ypart);
             }
         }
         if (s + 1 < nT) {

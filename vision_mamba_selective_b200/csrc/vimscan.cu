@@ -70,13 +70,13 @@ vim_status check_common(int batch, int L, int Di, int N, vim_dtype dt) {
     return VIM_OK;
 }
 
-template <typename T, int N>
+template <typename T, int N, bool CONV>
 size_t main_smem(int chunk) {
-    return 2 * (size_t)Stage<T, N>::kSlotBytes + (size_t)chunk * kDC * 4 + (size_t)kTile * kDC * 4;
+    return 2 * (size_t)Stage<T, N, CONV>::kSlotBytes + (size_t)chunk * kDC * 4 + (size_t)kTile * kDC * 4;
 }
-template <typename T, int N>
+template <typename T, int N, bool CONV>
 size_t carry_smem() {
-    return 2 * (size_t)Stage<T, N>::kSlotBytes;
+    return 2 * (size_t)Stage<T, N, CONV>::kSlotBytes;
 }
 
 // Launch of a kernel that may start while the previous kernel on the stream drains
@@ -111,15 +111,15 @@ inline vim_status mark(cudaEvent_t *events, int i, cudaStream_t stream) {
     return cudaEventRecord(events[i], stream) == cudaSuccess ? VIM_OK : VIM_ERR_CUDA;
 }
 
-template <typename T, int N, bool VEC_BC>
+template <typename T, int N, bool VEC_BC, bool PIN, bool CONV>
 vim_status launch_pair_v(const PairArgs &a, cudaStream_t stream, cudaEvent_t *ev) {
     const dim3 grid((a.Di + kDC - 1) / kDC, a.G, a.batch);
     if (a.G > 1) {
-        const size_t sc = carry_smem<T, N>();
-        if (cudaFuncSetAttribute(pair_carry<T, N, VEC_BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        const size_t sc = carry_smem<T, N, CONV>();
+        if (cudaFuncSetAttribute(pair_carry<T, N, VEC_BC, CONV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sc) != cudaSuccess)
             return VIM_ERR_CUDA;
-        pair_carry<T, N, VEC_BC><<<grid, kThreads, sc, stream>>>(a);
+        pair_carry<T, N, VEC_BC, CONV><<<grid, kThreads, sc, stream>>>(a);
         if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
         if (mark(ev, 0, stream) != VIM_OK) return VIM_ERR_CUDA;
         const int64_t units = (int64_t)a.batch * 2 * a.Di * N;
@@ -130,32 +130,26 @@ vim_status launch_pair_v(const PairArgs &a, cudaStream_t stream, cudaEvent_t *ev
     } else if (ev) {
         if (mark(ev, 0, stream) != VIM_OK || mark(ev, 1, stream) != VIM_OK) return VIM_ERR_CUDA;
     }
-    const size_t sm = main_smem<T, N>(a.chunk);
-    if (a.partial_in) {
-        if (cudaFuncSetAttribute(pair_main<T, N, VEC_BC, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sm) != cudaSuccess)
-            return VIM_ERR_CUDA;
-        if (a.G > 1) {
-            if (launch_dependent(pair_main<T, N, VEC_BC, true>, grid, dim3(kThreads), sm, stream, a) !=
-                cudaSuccess)
-                return VIM_ERR_CUDA;
-        } else {
-            pair_main<T, N, VEC_BC, true><<<grid, kThreads, sm, stream>>>(a);
-        }
+    const size_t sm = main_smem<T, N, CONV>(a.chunk);
+    auto kernel = pair_main<T, N, VEC_BC, PIN, CONV>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
+        return VIM_ERR_CUDA;
+    if (a.G > 1) {
+        if (launch_dependent(kernel, grid, dim3(kThreads), sm, stream, a) != cudaSuccess) return VIM_ERR_CUDA;
     } else {
-        if (cudaFuncSetAttribute(pair_main<T, N, VEC_BC, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sm) != cudaSuccess)
-            return VIM_ERR_CUDA;
-        if (a.G > 1) {
-            if (launch_dependent(pair_main<T, N, VEC_BC, false>, grid, dim3(kThreads), sm, stream, a) !=
-                cudaSuccess)
-                return VIM_ERR_CUDA;
-        } else {
-            pair_main<T, N, VEC_BC, false><<<grid, kThreads, sm, stream>>>(a);
-        }
+        kernel<<<grid, kThreads, sm, stream>>>(a);
     }
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     return mark(ev, 2, stream);
+}
+
+// the kernel variants a pair needs: fp32 partial_in (second pair of the cross-scan)
+// and the convolution front (Vim with x as input) are never combined
+template <typename T, int N, bool VEC_BC>
+vim_status launch_pair_v(const PairArgs &a, cudaStream_t stream, cudaEvent_t *ev) {
+    if (a.conv_w) return launch_pair_v<T, N, VEC_BC, false, true>(a, stream, ev);
+    if (a.partial_in) return launch_pair_v<T, N, VEC_BC, true, false>(a, stream, ev);
+    return launch_pair_v<T, N, VEC_BC, false, false>(a, stream, ev);
 }
 
 // B/C move as 16-byte vectors when their rows allow it and every base is aligned
@@ -216,11 +210,15 @@ size_t vim_scan_workspace_bytes(int which, int batch, int L_or_H, int W, int cha
     return 0;
 }
 
-vim_status vim_scan_bidir_events(const void *u, const void *delta, const void *z, const void *B,
-                                 const void *C, int64_t bc_dir_stride, const float *A,
-                                 const float *D, const float *delta_bias, void *y, int batch, int L,
-                                 int d_inner, int d_state, vim_dtype dt, void *workspace,
-                                 size_t workspace_bytes, cudaStream_t stream, cudaEvent_t *events) {
+}  // extern "C"
+
+namespace {
+// vim_scan_bidir with an optional convolution front (conv_w/conv_b non-null: u holds x)
+vim_status bidir_impl(const void *u, const float *conv_w, const float *conv_b, const void *delta,
+                      const void *z, const void *B, const void *C, int64_t bc_dir_stride, const float *A,
+                      const float *D, const float *delta_bias, void *y, int batch, int L, int d_inner,
+                      int d_state, vim_dtype dt, void *workspace, size_t workspace_bytes,
+                      cudaStream_t stream, cudaEvent_t *events) {
     vim_status st = check_common(batch, L, d_inner, d_state, dt);
     if (st != VIM_OK) return st;
     if (bc_dir_stride < 0) return VIM_ERR_INVALID_ARG;
@@ -247,6 +245,7 @@ vim_status vim_scan_bidir_events(const void *u, const void *delta, const void *z
     a.B[1] = Bc + bc_dir_stride * (int64_t)elem_size(dt);
     a.C[1] = Cc + bc_dir_stride * (int64_t)elem_size(dt);
     a.A = A; a.D = D; a.bias = delta_bias;
+    a.conv_w = conv_w; a.conv_b = conv_b;
     a.y = y;
     a.batch = batch; a.L = L; a.Di = d_inner; a.H = 1; a.W = L; a.order = 0;
     a.chunk = pl.chunk; a.G = pl.G;
@@ -257,6 +256,45 @@ vim_status vim_scan_bidir_events(const void *u, const void *delta, const void *z
     }
     if (mark(events, 0, stream) != VIM_OK) return VIM_ERR_CUDA;
     return launch_pair(a, d_state, dt, stream, events ? events + 1 : nullptr);
+}
+
+}  // namespace
+
+extern "C" {
+
+vim_status vim_scan_bidir_events(const void *u, const void *delta, const void *z, const void *B,
+                                 const void *C, int64_t bc_dir_stride, const float *A,
+                                 const float *D, const float *delta_bias, void *y, int batch, int L,
+                                 int d_inner, int d_state, vim_dtype dt, void *workspace,
+                                 size_t workspace_bytes, cudaStream_t stream, cudaEvent_t *events) {
+    return bidir_impl(u, nullptr, nullptr, delta, z, B, C, bc_dir_stride, A, D, delta_bias, y, batch, L,
+                      d_inner, d_state, dt, workspace, workspace_bytes, stream, events);
+}
+
+vim_status vim_scan_bidir_conv_events(const void *x, const float *conv_w, const float *conv_b,
+                                      const void *delta, const void *z, const void *B, const void *C,
+                                      int64_t bc_dir_stride, const float *A, const float *D,
+                                      const float *delta_bias, void *y, int batch, int L, int d_inner,
+                                      int d_state, vim_dtype dt, void *workspace, size_t workspace_bytes,
+                                      cudaStream_t stream, cudaEvent_t *events) {
+    if (batch > 0 && L > 0 && d_inner > 0) {
+        if (!conv_w || !conv_b) return VIM_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(conv_w) | reinterpret_cast<uintptr_t>(conv_b)) % 4)
+            return VIM_ERR_INVALID_ARG;
+    }
+    return bidir_impl(x, conv_w, conv_b, delta, z, B, C, bc_dir_stride, A, D, delta_bias, y, batch, L,
+                      d_inner, d_state, dt, workspace, workspace_bytes, stream, events);
+}
+
+vim_status vim_scan_bidir_conv(const void *x, const float *conv_w, const float *conv_b,
+                               const void *delta, const void *z, const void *B, const void *C,
+                               int64_t bc_dir_stride, const float *A, const float *D,
+                               const float *delta_bias, void *y, int batch, int L, int d_inner,
+                               int d_state, vim_dtype dt, void *workspace, size_t workspace_bytes,
+                               cudaStream_t stream) {
+    return vim_scan_bidir_conv_events(x, conv_w, conv_b, delta, z, B, C, bc_dir_stride, A, D, delta_bias,
+                                      y, batch, L, d_inner, d_state, dt, workspace, workspace_bytes,
+                                      stream, nullptr);
 }
 
 vim_status vim_scan_bidir(const void *u, const void *delta, const void *z, const void *B,

@@ -36,6 +36,11 @@ lib.vim_scan_bidir_events.argtypes = lib.vim_scan_bidir.argtypes + [_vp]
 lib.vim_scan_bidir_events.restype = _i
 lib.vmamba_cross_scan4_events.argtypes = lib.vmamba_cross_scan4.argtypes + [_vp]
 lib.vmamba_cross_scan4_events.restype = _i
+lib.vim_scan_bidir_conv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
+                                    _i, _i, _i, _i, _i, _vp, _sz, _vp]
+lib.vim_scan_bidir_conv.restype = _i
+lib.vim_scan_bidir_conv_events.argtypes = lib.vim_scan_bidir_conv.argtypes + [_vp]
+lib.vim_scan_bidir_conv_events.restype = _i
 lib.vim_scan_bidir_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
                                        _i, _i, _i, _i, _i, _vp]
 lib.vim_scan_bidir_noalloc.restype = _i
@@ -132,6 +137,33 @@ def vim_scan_bidir(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride
         batch, L, Di, N, dt, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream), *extra)
     if st != VIM_OK:
         raise VimScanError(st, "vim_scan_bidir")
+    return y
+
+
+def vim_scan_bidir_conv(x, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride=0,
+                        workspace=None, stream=None, events=None):
+    """vim_scan_bidir with the pathways' kernel-3 convolution + SiLU front fused in.
+
+    x, delta, z: [batch, L, d_inner]; conv_w: [2, d_inner, 3] fp32; conv_b: [2, d_inner]
+    fp32; the rest as in vim_scan_bidir.  Returns y [batch, L, d_inner].
+    """
+    batch, L, Di = x.shape
+    N = B.shape[-1]
+    dt = _dtype_code(x)
+    if y is None:
+        y = torch.empty_like(x)
+    ws, ws_bytes = _workspace(vim_scan_workspace_bytes(0, batch, L, 0, Di, N), workspace, x.device)
+    extra = () if events is None else (_events(events),)
+    fn = lib.vim_scan_bidir_conv if events is None else lib.vim_scan_bidir_conv_events
+    st = fn(
+        _ptr(x, name="x"), _ptr(conv_w, dtype=torch.float32, name="conv_w"),
+        _ptr(conv_b, dtype=torch.float32, name="conv_b"), _ptr(delta, dtype=x.dtype, name="delta"),
+        _ptr(z, dtype=x.dtype, name="z"), _ptr(B, dtype=x.dtype, name="B"), _ptr(C, dtype=x.dtype, name="C"),
+        int(bc_dir_stride), _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
+        _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(y, dtype=x.dtype, name="y"),
+        batch, L, Di, N, dt, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream), *extra)
+    if st != VIM_OK:
+        raise VimScanError(st, "vim_scan_bidir_conv")
     return y
 
 
