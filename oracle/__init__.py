@@ -52,13 +52,13 @@ class Oracle:
 
     def __init__(self, path: str):
         lib = ctypes.CDLL(path)
-        lib.oracle_s6_direction.argtypes = [_D, _D, _D, _D, _D, _D, _D, _I64, _D] + [ctypes.c_int] * 6
-        lib.oracle_vim_bidir.argtypes = [_D, _D, _D, _D, _D, ctypes.c_int64, _D, _D, _D, _D] + [ctypes.c_int] * 5
-        lib.oracle_cross_scan4.argtypes = [_D] * 9 + [ctypes.c_int] * 6
+        lib.oracle_s6_direction.argtypes = [_D, _D, _D, _D, _D, _D, _D, _I64, _D] + [ctypes.c_int] * 7
+        lib.oracle_vim_bidir.argtypes = [_D, _D, _D, _D, _D, ctypes.c_int64, _D, _D, _D, _D] + [ctypes.c_int] * 6
+        lib.oracle_cross_scan4.argtypes = [_D] * 9 + [ctypes.c_int] * 7
         lib.oracle_cross_merge4.argtypes = [_D, _D, _D] + [ctypes.c_int] * 4
         lib.oracle_cross_order.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _I64]
         lib.oracle_conv_silu.argtypes = [_D, _D, _D, _D] + [ctypes.c_int] * 4
-        lib.oracle_vim_bidir_conv.argtypes = [_D, _D, _D, _D, _D, _D, _D, ctypes.c_int64, _D, _D, _D, _D] + [ctypes.c_int] * 5
+        lib.oracle_vim_bidir_conv.argtypes = [_D, _D, _D, _D, _D, _D, _D, ctypes.c_int64, _D, _D, _D, _D] + [ctypes.c_int] * 6
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
         self.lib = lib
@@ -78,12 +78,13 @@ class Oracle:
             raise ValueError("bad direction index")
         return out
 
-    def s6_direction(self, u, delta, B, C, A, D, bias, order, *, delta_is_raw=True):
+    def s6_direction(self, u, delta, B, C, A, D, bias, order, *, delta_is_raw=True, zoh=False):
         """One S6 direction (no gate) over tokens visited in ``order``.
 
         u, delta: [batch, L, Di]; B, C: [batch, L, N] (by position); A: [Di, N];
         D, bias: [Di]; order: [L] permutation.  Returns y [batch, L, Di] with
-        y[b, order[t], d] = C_t . h_t + D u_t.
+        y[b, order[t], d] = C_t . h_t + D u_t.  zoh=True takes the exact zero-order-hold
+        Bbar = expm1(Delta A) / A * B instead of Delta B.
         """
         u, delta, B, C, A, D, bias = map(_f64, (u, delta, B, C, A, D, bias))
         batch, L, Di = u.shape
@@ -95,12 +96,12 @@ class Oracle:
         y = np.zeros((batch, L, Di))
         rc = self.lib.oracle_s6_direction(_p(u), _p(delta), _p(B), _p(C), _p(A), _p(D), _p(bias),
                                           order.ctypes.data_as(_I64), _p(y),
-                                          batch, L, Di, N, int(bool(delta_is_raw)), 0)
+                                          batch, L, Di, N, int(bool(delta_is_raw)), 0, int(bool(zoh)))
         if rc:
             raise ValueError("oracle_s6_direction: bad sizes")
         return y
 
-    def vim_bidir(self, u, delta, z, B, C, A, D, bias, *, bc_dir_stride=0, delta_is_raw=True):
+    def vim_bidir(self, u, delta, z, B, C, A, D, bias, *, bc_dir_stride=0, delta_is_raw=True, zoh=False):
         """Vim bidirectional scan: (y^f + y^b) * silu(z); z=None gives the ungated sum.
 
         u, delta, z: [batch, L, Di]; B, C: [batch, L, N] shared by both directions,
@@ -115,7 +116,7 @@ class Oracle:
         y = np.zeros((batch, L, Di))
         rc = self.lib.oracle_vim_bidir(_p(u), _p(delta), _p(z), _p(B), _p(C), int(bc_dir_stride),
                                        _p(A), _p(D), _p(bias), _p(y), batch, L, Di, N,
-                                       int(bool(delta_is_raw)))
+                                       int(bool(delta_is_raw)), int(bool(zoh)))
         if rc:
             raise ValueError("oracle_vim_bidir: bad sizes")
         return y
@@ -134,7 +135,7 @@ class Oracle:
         return u
 
     def vim_bidir_conv(self, x, conv_w, conv_b, delta, z, B, C, A, D, bias, *, bc_dir_stride=0,
-                       delta_is_raw=True):
+                       delta_is_raw=True, zoh=False):
         """Vim scan with its convolution front: u_f = silu(conv_f(x)), u_b = silu of
         conv_b on the reversed sequence; then (y^f + y^b) * silu(z).
 
@@ -150,12 +151,12 @@ class Oracle:
         y = np.zeros((batch, L, Di))
         rc = self.lib.oracle_vim_bidir_conv(_p(x), _p(conv_w), _p(conv_b), _p(delta), _p(z), _p(B), _p(C),
                                             int(bc_dir_stride), _p(A), _p(D), _p(bias), _p(y), batch, L, Di,
-                                            N, int(bool(delta_is_raw)))
+                                            N, int(bool(delta_is_raw)), int(bool(zoh)))
         if rc:
             raise ValueError("oracle_vim_bidir_conv: bad sizes")
         return y
 
-    def cross_scan4(self, u, delta, z, B, C, A, D, bias, *, delta_is_raw=True):
+    def cross_scan4(self, u, delta, z, B, C, A, D, bias, *, delta_is_raw=True, zoh=False):
         """VMamba four-direction scan with CS-Merge: (sum_k y_k) * silu(z).
 
         u, delta, z: [batch, H, W, Ci]; B, C: [4, batch, H*W, N] in grid order;
@@ -168,7 +169,8 @@ class Oracle:
             bias = np.zeros((4, Ci))
         y = np.zeros((batch, H, W, Ci))
         rc = self.lib.oracle_cross_scan4(_p(u), _p(delta), _p(z), _p(B), _p(C), _p(A), _p(D),
-                                         _p(bias), _p(y), batch, H, W, Ci, N, int(bool(delta_is_raw)))
+                                         _p(bias), _p(y), batch, H, W, Ci, N, int(bool(delta_is_raw)),
+                                         int(bool(zoh)))
         if rc:
             raise ValueError("oracle_cross_scan4: bad sizes")
         return y

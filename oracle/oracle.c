@@ -9,7 +9,9 @@
  * What it computes is written straight from the equations of the page
  * "Vision Mamba Guide: Efficient Bidirectional SSM & VMamba" (aifetchly-blog):
  *   - ZOH discretisation, section "Discretization via Zero-Order Hold (ZOH)":
- *       Abar = exp(Delta*A),  Bbar ~= Delta*B  (the approximate form is used);
+ *       Abar = exp(Delta*A),  Bbar ~= Delta*B  (the approximate form, the default),
+ *       or on request the exact form Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B,
+ *       which for a diagonal A is expm1(Delta A_n) / A_n * B_n per state;
  *   - recurrence and readout, same section and section "Continuous-Time State
  *     Space Equations":  h_t = Abar h_{t-1} + Bbar x_t,  y_t = C h_t + D x_t;
  *   - selectivity, section "The Selective State Space (S6) Mechanism":
@@ -101,12 +103,26 @@ int oracle_cross_order(int k, int H, int W, int64_t *order)
  *                                      added to the existing value if accumulate != 0
  *   delta_is_raw != 0 : Delta = softplus(delta + bias[d]); otherwise Delta = delta
  *                       as given and bias is ignored.
+ *   zoh != 0 : exact zero-order-hold Bbar (see bbar below); otherwise Bbar = Delta B.
  * Returns 0, or -1 on bad sizes.
  */
+/*
+ * Bbar of one state.  Section "Discretization via Zero-Order Hold (ZOH)" gives
+ * Bbar = (Delta A)^-1 (exp(Delta A) - I) . Delta B and its first-order form Delta B.
+ * With A diagonal the matrix inverse is a division per state, so the exact form is
+ * (exp(Delta A_n) - 1) / A_n * B_n, evaluated with expm1 so that small Delta A_n
+ * loses nothing to cancellation; at A_n = 0 it is its limit Delta B_n.
+ */
+static double bbar(double dt, double An, double Bn, int zoh)
+{
+    if (!zoh || An == 0.0) return dt * Bn;
+    return expm1(dt * An) / An * Bn;
+}
+
 int oracle_s6_direction(const double *u, const double *delta, const double *B, const double *C,
                         const double *A, const double *D, const double *bias,
                         const int64_t *order, double *y,
-                        int batch, int L, int Di, int N, int delta_is_raw, int accumulate)
+                        int batch, int L, int Di, int N, int delta_is_raw, int accumulate, int zoh)
 {
     if (batch < 0 || L < 0 || Di < 0 || N < 1 || N > ORACLE_MAX_STATE) return -1;
     int64_t pairs = (int64_t)batch * Di;
@@ -125,7 +141,7 @@ int oracle_s6_direction(const double *u, const double *delta, const double *B, c
             double yt = 0.0;
             for (int n = 0; n < N; ++n) {
                 double Abar = exp(dt * A[d * N + n]);             /* Abar = exp(Delta A) */
-                double Bbar = dt * Bt[n];                         /* Bbar ~= Delta B     */
+                double Bbar = bbar(dt, A[d * N + n], Bt[n], zoh); /* Bbar (~= Delta B)   */
                 h[n] = Abar * h[n] + Bbar * x;                    /* h_t = Abar h + Bbar x */
                 yt += Ct[n] * h[n];                               /* C h_t               */
             }
@@ -178,11 +194,12 @@ static void apply_gate(double *y, const double *z, int64_t n)
  *                 C + bc_dir_stride (0 = both directions share B and C)
  *   A [2, Di, N], D [2, Di], bias [2, Di]: index 0 = forward, 1 = backward
  *   y           : [batch, L, Di] = (y^f + y^b) * silu(z)
+ *   delta_is_raw, zoh: as in oracle_s6_direction
  */
 int oracle_vim_bidir(const double *u, const double *delta, const double *z,
                      const double *B, const double *C, int64_t bc_dir_stride,
                      const double *A, const double *D, const double *bias,
-                     double *y, int batch, int L, int Di, int N, int delta_is_raw)
+                     double *y, int batch, int L, int Di, int N, int delta_is_raw, int zoh)
 {
     if (L < 0) return -1;
     int64_t *order = (int64_t *)calloc((size_t)(L > 0 ? L : 1), sizeof(int64_t));
@@ -190,11 +207,11 @@ int oracle_vim_bidir(const double *u, const double *delta, const double *z,
     int rc = 0;
     for (int64_t t = 0; t < L; ++t) order[t] = t;                 /* forward: 1 .. N+1 */
     rc |= oracle_s6_direction(u, delta, B, C, A, D, bias, order, y,
-                              batch, L, Di, N, delta_is_raw, 0);
+                              batch, L, Di, N, delta_is_raw, 0, zoh);
     for (int64_t t = 0; t < L; ++t) order[t] = L - 1 - t;         /* backward: N+1 .. 1 */
     rc |= oracle_s6_direction(u, delta, B + bc_dir_stride, C + bc_dir_stride,
                               A + (int64_t)Di * N, D + Di, bias + Di, order, y,
-                              batch, L, Di, N, delta_is_raw, 1);
+                              batch, L, Di, N, delta_is_raw, 1, zoh);
     free(order);
     if (rc) return -1;
     apply_gate(y, z, (int64_t)batch * L * Di);
@@ -211,7 +228,7 @@ int oracle_vim_bidir_conv(const double *x, const double *conv_w, const double *c
                           const double *delta, const double *z,
                           const double *B, const double *C, int64_t bc_dir_stride,
                           const double *A, const double *D, const double *bias,
-                          double *y, int batch, int L, int Di, int N, int delta_is_raw)
+                          double *y, int batch, int L, int Di, int N, int delta_is_raw, int zoh)
 {
     if (batch < 0 || L < 0 || Di < 0) return -1;
     size_t n = (size_t)batch * (size_t)L * (size_t)Di;
@@ -223,10 +240,10 @@ int oracle_vim_bidir_conv(const double *x, const double *conv_w, const double *c
     if (!rc) rc |= oracle_conv_silu(x, conv_w + (int64_t)Di * 3, conv_b + Di, ub, batch, L, Di, 1);
     if (!rc) {
         for (int64_t t = 0; t < L; ++t) order[t] = t;
-        rc |= oracle_s6_direction(uf, delta, B, C, A, D, bias, order, y, batch, L, Di, N, delta_is_raw, 0);
+        rc |= oracle_s6_direction(uf, delta, B, C, A, D, bias, order, y, batch, L, Di, N, delta_is_raw, 0, zoh);
         for (int64_t t = 0; t < L; ++t) order[t] = L - 1 - t;
         rc |= oracle_s6_direction(ub, delta, B + bc_dir_stride, C + bc_dir_stride, A + (int64_t)Di * N,
-                                  D + Di, bias + Di, order, y, batch, L, Di, N, delta_is_raw, 1);
+                                  D + Di, bias + Di, order, y, batch, L, Di, N, delta_is_raw, 1, zoh);
     }
     free(uf); free(ub); free(order);
     if (rc) return -1;
@@ -244,7 +261,7 @@ int oracle_vim_bidir_conv(const double *x, const double *conv_w, const double *c
 int oracle_cross_scan4(const double *u, const double *delta, const double *z,
                        const double *B, const double *C,
                        const double *A, const double *D, const double *bias,
-                       double *y, int batch, int H, int W, int Ci, int N, int delta_is_raw)
+                       double *y, int batch, int H, int W, int Ci, int N, int delta_is_raw, int zoh)
 {
     if (H < 0 || W < 0) return -1;
     int64_t L = (int64_t)H * W;
@@ -257,7 +274,7 @@ int oracle_cross_scan4(const double *u, const double *delta, const double *z,
         rc |= oracle_s6_direction(u, delta, B + k * bc, C + k * bc,
                                   A + (int64_t)k * Ci * N, D + (int64_t)k * Ci,
                                   bias + (int64_t)k * Ci, order, y,
-                                  batch, (int)L, Ci, N, delta_is_raw, k > 0);
+                                  batch, (int)L, Ci, N, delta_is_raw, k > 0, zoh);
     }
     free(order);
     if (rc) return -1;

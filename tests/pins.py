@@ -368,6 +368,131 @@ def pin_conv_scan_composition(orc):
     np.testing.assert_allclose(y, flip(y2), rtol=1e-12, atol=1e-12)
 
 
+def pin_zoh_matches_ode(orc):
+    """The exact zero-order hold is exact for inputs held over each step: with
+    Delta_t, u_t and B_t constant on a step of length Delta_t, integrating the
+    continuous system h' = A h + B x (section "Continuous-Time State Space
+    Equations") over that step gives h_t = Abar h_{t-1} + Bbar x_t with Abar =
+    exp(Delta A) and Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B (section
+    "Discretization via Zero-Order Hold (ZOH)").  The reference here is a numerical
+    ODE solver (scipy's DOP853 at rtol 1e-12), independent of the closed form; the
+    first-order form Delta B must differ from it by far more than the tolerance.
+    """
+    from scipy.integrate import solve_ivp
+
+    rng = _rng(91)
+    batch, L, Di, N = 1, 6, 2, 4
+    u = rng.normal(size=(batch, L, Di))
+    delta = rng.uniform(0.05, 0.9, size=(batch, L, Di))
+    B = rng.normal(size=(batch, L, N))
+    C = rng.normal(size=(batch, L, N))
+    A = -rng.uniform(0.2, 3.0, size=(Di, N))
+    D = rng.normal(size=Di)
+    order = np.arange(L)
+    expect = np.zeros((batch, L, Di))
+    for b in range(batch):
+        for d in range(Di):
+            h = np.zeros(N)
+            for t in range(L):
+                drive = B[b, t] * u[b, t, d]
+                sol = solve_ivp(lambda _s, hh: A[d] * hh + drive, (0.0, delta[b, t, d]), h,
+                                method="DOP853", rtol=1e-12, atol=1e-14)
+                h = sol.y[:, -1]
+                expect[b, t, d] = C[b, t] @ h + D[d] * u[b, t, d]
+    got = orc.s6_direction(u, delta, B, C, A, D, None, order, delta_is_raw=False, zoh=True)
+    np.testing.assert_allclose(got, expect, rtol=1e-9, atol=1e-11)
+    euler = orc.s6_direction(u, delta, B, C, A, D, None, order, delta_is_raw=False, zoh=False)
+    assert np.max(np.abs(euler - expect)) > 1e-3
+
+
+def pin_zoh_fixed_point_and_limits(orc):
+    """Three consequences of the exact form, each checked through the two-direction
+    scan (section "Discretization via Zero-Order Hold (ZOH)"):
+    - constant input: h tends to the continuous system's rest point -B u / A,
+      whatever Delta is, so both directions end at y = sum_k (C (-B u / A_k) + D_k u);
+    - A = 0: Bbar is its limit Delta B, so the exact and first-order forms agree;
+    - small Delta: the two forms differ by O(Delta^2) per step, so halving Delta
+      quarters the gap (ratio within 3.5 .. 4.5).
+    """
+    rng = _rng(92)
+    batch, L, Di, N = 1, 400, 3, 4
+    u0 = rng.normal(size=Di)
+    Bc, Cc = rng.normal(size=N), rng.normal(size=N)
+    A = -rng.uniform(0.3, 2.0, size=(2, Di, N))
+    D = rng.normal(size=(2, Di))
+    u = np.broadcast_to(u0, (batch, L, Di)).copy()
+    B = np.broadcast_to(Bc, (batch, L, N)).copy()
+    Cm = np.broadcast_to(Cc, (batch, L, N)).copy()
+    delta = np.full((batch, L, Di), 0.7)
+    y = orc.vim_bidir(u, delta, None, B, Cm, A, D, None, delta_is_raw=False, zoh=True)
+    rest = sum(((-Bc[None, :] / A[k]) @ Cc) * u0 + D[k] * u0 for k in range(2))
+    # forward has taken L steps at the last token, backward L steps at the first;
+    # only the sum at the middle has both near rest, so check y at L/2 against it
+    np.testing.assert_allclose(y[0, L // 2], rest, rtol=1e-12, atol=1e-12)
+
+    c = _vim_case(_rng(93))
+    A0 = np.zeros_like(c["A"])
+    ye = _vim(orc, c, gate=False, A=A0)
+    yz = orc.vim_bidir(c["u"], c["delta"], None, c["B"], c["C"], A0, c["D"], c["bias"],
+                       bc_dir_stride=c["stride"], delta_is_raw=False, zoh=True)
+    np.testing.assert_allclose(yz, ye, rtol=1e-14, atol=1e-14)
+
+    gaps = []
+    for scale in (1e-3, 5e-4):
+        dl = np.full_like(c["delta"], scale)
+        y1 = _vim(orc, c, gate=False, delta=dl)
+        y2 = orc.vim_bidir(c["u"], dl, None, c["B"], c["C"], c["A"], c["D"], c["bias"],
+                           bc_dir_stride=c["stride"], delta_is_raw=False, zoh=True)
+        gaps.append(np.max(np.abs(y2 - y1)))
+    assert 3.5 < gaps[0] / gaps[1] < 4.5, gaps
+
+
+def pin_zoh_reaches_every_entry(orc):
+    """The exact-ZOH choice reaches every direction of every entry: the
+    two-direction scan (with and without the convolution front) and the
+    four-direction scan each equal their explicit composition from single exact-ZOH
+    directions (the single direction itself is pinned by pin_zoh_matches_ode)."""
+    rng = _rng(94)
+    c = _vim_case(rng, L=9)
+    L = c["u"].shape[1]
+    yf = orc.s6_direction(c["u"], c["delta"], c["B"][0], c["C"][0], c["A"][0], c["D"][0], None,
+                          np.arange(L), delta_is_raw=False, zoh=True)
+    yb = orc.s6_direction(c["u"], c["delta"], c["B"][1], c["C"][1], c["A"][1], c["D"][1], None,
+                          np.arange(L)[::-1], delta_is_raw=False, zoh=True)
+    y = orc.vim_bidir(c["u"], c["delta"], None, c["B"], c["C"], c["A"], c["D"], None,
+                      bc_dir_stride=c["stride"], delta_is_raw=False, zoh=True)
+    np.testing.assert_allclose(y, yf + yb, rtol=1e-12, atol=1e-12)
+
+    x = rng.normal(size=c["u"].shape)
+    cw, cbias = rng.normal(size=(2, 3, 3)), rng.normal(size=(2, 3))
+    uf, ub = orc.conv_silu(x, cw[0], cbias[0]), orc.conv_silu(x, cw[1], cbias[1], reversed=True)
+    yf = orc.s6_direction(uf, c["delta"], c["B"][0], c["C"][0], c["A"][0], c["D"][0], None,
+                          np.arange(L), delta_is_raw=False, zoh=True)
+    yb = orc.s6_direction(ub, c["delta"], c["B"][1], c["C"][1], c["A"][1], c["D"][1], None,
+                          np.arange(L)[::-1], delta_is_raw=False, zoh=True)
+    y = orc.vim_bidir_conv(x, cw, cbias, c["delta"], None, c["B"], c["C"], c["A"], c["D"], None,
+                           bc_dir_stride=c["stride"], delta_is_raw=False, zoh=True)
+    np.testing.assert_allclose(y, yf + yb, rtol=1e-12, atol=1e-12)
+
+    b, H, W, ch, N = 1, 3, 4, 2, 3
+    u = rng.normal(size=(b, H, W, ch))
+    dl = rng.uniform(0.05, 0.8, size=(b, H, W, ch))
+    B = rng.normal(size=(4, b, H * W, N))
+    C = rng.normal(size=(4, b, H * W, N))
+    A = -rng.uniform(0.1, 2.0, size=(4, ch, N))
+    D = rng.normal(size=(4, ch))
+    y = orc.cross_scan4(u, dl, None, B, C, A, D, None, delta_is_raw=False, zoh=True)
+    seq_u, seq_d = _traverse(u), _traverse(dl)
+    outs = []
+    for k in range(4):
+        Bk = _traverse(B[k].reshape(b, H, W, N))[k]
+        Ck = _traverse(C[k].reshape(b, H, W, N))[k]
+        outs.append(orc.s6_direction(np.ascontiguousarray(seq_u[k]), np.ascontiguousarray(seq_d[k]),
+                                     np.ascontiguousarray(Bk), np.ascontiguousarray(Ck), A[k], D[k], None,
+                                     np.arange(H * W), delta_is_raw=False, zoh=True))
+    np.testing.assert_allclose(y, sum(_untraverse(np.stack(outs), H, W)), rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [
     pin_delta_zero,
     pin_constant_input_geometric,
@@ -383,4 +508,7 @@ ALL_PINS = [
     pin_separate_bc,
     pin_conv_front_is_correlation,
     pin_conv_scan_composition,
+    pin_zoh_matches_ode,
+    pin_zoh_fixed_point_and_limits,
+    pin_zoh_reaches_every_entry,
 ]

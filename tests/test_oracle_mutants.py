@@ -18,7 +18,7 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
 MUTANTS = {
     "drop_D_skip": ("yt += D[d] * x;", "yt += 0.0 * x;"),
     "decay_sign": ("exp(dt * A[d * N + n])", "exp(-dt * A[d * N + n])"),
-    "bbar_without_delta": ("double Bbar = dt * Bt[n];", "double Bbar = Bt[n];"),
+    "bbar_without_delta": ("if (!zoh || An == 0.0) return dt * Bn;", "if (!zoh || An == 0.0) return Bn;"),
     "readout_uses_B": ("yt += Ct[n] * h[n];", "yt += Bt[n] * h[n];"),
     "A_transposed": ("exp(dt * A[d * N + n])", "exp(dt * A[n * Di + d])"),
     "readout_before_update": (
@@ -42,6 +42,13 @@ MUTANTS = {
     "conv_no_silu": ("u[(b * L + t) * Di + d] = silu(acc);", "u[(b * L + t) * Di + d] = acc;"),
     "conv_backward_uses_forward_weights": ("oracle_conv_silu(x, conv_w + (int64_t)Di * 3, conv_b + Di, ub",
                                            "oracle_conv_silu(x, conv_w, conv_b, ub"),
+    "zoh_ignored": ("return expm1(dt * An) / An * Bn;", "return dt * Bn;"),
+    "zoh_no_division_by_A": ("return expm1(dt * An) / An * Bn;", "return expm1(dt * An) * Bn;"),
+    "zoh_exp_for_expm1": ("return expm1(dt * An) / An * Bn;", "return exp(dt * An) / An * Bn;"),
+    "zoh_delta_twice": ("return expm1(dt * An) / An * Bn;", "return dt * expm1(dt * An) / An * Bn;"),
+    "zoh_dropped_in_bidir": ("delta_is_raw, 0, zoh);", "delta_is_raw, 0, 0);"),
+    "zoh_dropped_in_cross": ("delta_is_raw, k > 0, zoh);", "delta_is_raw, k > 0, 0);"),
+    "zoh_sign": ("return expm1(dt * An) / An * Bn;", "return expm1(-dt * An) / An * Bn;"),
 }
 
 
