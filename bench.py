@@ -2,7 +2,7 @@
 """Throughput of the bidirectional selective scan (S6) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
-                    [--conv]
+                    [--conv] [--zoh]
 
 One step is one pass of the whole scan -- softplus Delta, the forward and backward
 recurrences, readout, D skip, the merge of the directions and the silu(z) gate --
@@ -10,7 +10,8 @@ over one batch of the workload, through the library's C ABI.  The default worklo
 is the 1024 px Vim-Tiny scan (batch 8, L = 4097, d_inner 384, d_state 16, bf16 I/O,
 fp32 state).  Inputs are seeded synthetic tensors shaped like the pages' workloads.
 --conv times the same scan with the pathways' kernel-3 convolution + SiLU fused in
-front (the input tensor is then x, the convolutions' input).
+front (the input tensor is then x, the convolutions' input); --zoh times it with the
+exact zero-order-hold Bbar = (exp(Delta A) - 1) / A * B in place of Delta B.
 
 Multi-GPU (torchrun, one process per GPU): the batch items are independent, so every
 rank runs the same workload on its own inputs with no collective on the data path
@@ -51,6 +52,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--conv", action="store_true",
                     help="Vim workloads: time the scan with the fused kernel-3 convolution + SiLU front")
+    ap.add_argument("--zoh", action="store_true",
+                    help="time the scan with the exact zero-order-hold Bbar instead of Delta B")
     return ap.parse_args()
 
 
@@ -170,18 +173,19 @@ def conv_params(w, seed):
     return cw.contiguous(), cb.contiguous()
 
 
-def run_oracle(w, x, threads):
+def run_oracle(w, x, threads, zoh=False):
     import oracle
 
     oracle.set_threads(threads)
     t = time.perf_counter()
     if "conv_w" in x:
         oracle.vim_bidir_conv(x["u"], x["conv_w"], x["conv_b"], x["delta"], x["z"], x["B"], x["C"], x["A"],
-                              x["D"], x["delta_bias"])
+                              x["D"], x["delta_bias"], zoh=zoh)
     elif w.kind == "vim":
-        oracle.vim_bidir(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"])
+        oracle.vim_bidir(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], zoh=zoh)
     else:
-        oracle.cross_scan4(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"])
+        oracle.cross_scan4(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"],
+                           zoh=zoh)
     return time.perf_counter() - t
 
 
@@ -236,8 +240,8 @@ def reference_arm(args, w):
     per_step = min(2.0, 150.0 / max(1, args.steps + args.warmup))
     s, x, cores = oracle_sample(w, per_step, conv=args.conv)
     for _ in range(args.warmup):
-        run_oracle(s, x, cores)
-    times = [run_oracle(s, x, cores) for _ in range(args.steps)]
+        run_oracle(s, x, cores, args.zoh)
+    times = [run_oracle(s, x, cores, args.zoh) for _ in range(args.steps)]
     sec = sum(times) / len(times)
     value = s.tok_ch / sec
     sample = (f"{s.batch} of {w.batch} batch items x {s.channels} of {w.channels} channels at the full "
@@ -257,7 +261,7 @@ def reference_arm(args, w):
 
 
 def workload_name(w, args):
-    return w.name + ("+conv_front" if args.conv else "")
+    return w.name + ("+conv_front" if args.conv else "") + ("+zoh_exact" if args.zoh else "")
 
 
 def main():
@@ -312,10 +316,10 @@ def main():
             # u holds x, the pathways' common input in front of the convolutions
             vs.vim_scan_bidir_conv(s["u"], params["conv_w"], params["conv_b"], s["delta"], s["z"], s["B"],
                                    s["C"], params["A"], params["D"], params["delta_bias"], y=s["y"],
-                                   workspace=ws, events=events)
+                                   workspace=ws, events=events, zoh=args.zoh)
             return
         fn(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"], params["delta_bias"],
-           y=s["y"], workspace=ws, events=events)
+           y=s["y"], workspace=ws, events=events, zoh=args.zoh)
 
     barrier = replicas.barrier
 
@@ -406,7 +410,7 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         s, x, cores = oracle_sample(w, 5.0, conv=args.conv)
-        sec = run_oracle(s, x, cores)
+        sec = run_oracle(s, x, cores, args.zoh)
         cpu = {"value": s.tok_ch / sec, "unit": "tok*ch/s", "cores": cores, "kind": "oracle",
                "sample": f"{s.batch} of {w.batch} batch items x {s.channels} of {w.channels} channels "
                          f"at the full {w.tokens} tokens ({s.tok_ch} token-channels), fp64, {sec:.2f} s"}

@@ -6,8 +6,10 @@
  *   - the S6 recurrence with input-dependent Delta, B, C (sections "Discretization
  *     via Zero-Order Hold (ZOH)" and "The Selective State Space (S6) Mechanism"):
  *         Delta_t = softplus(delta_raw_t + delta_bias)      (softplus(x) = x for x > 20)
- *         h_t     = exp(Delta_t * A) * h_{t-1} + Delta_t * B_t * u_t     (h starts at 0)
+ *         h_t     = exp(Delta_t * A) * h_{t-1} + Bbar_t * u_t            (h starts at 0)
  *         y_t     = C_t . h_t + D * u_t
+ *     with the first-order Bbar_t = Delta_t * B_t, or on request (VIM_FLAG_ZOH_EXACT)
+ *     the exact zero-order-hold form;
  *   - the Vim bidirectional block (section "2. The Bidirectional Mamba Block"): a
  *     forward pass over the tokens and a backward pass from the last token to the
  *     first, fused as (y^f + y^b) * silu(z), silu(z) = z / (1 + exp(-z));
@@ -179,6 +181,42 @@ vim_status vmamba_cross_scan4_events(const void *u, const void *delta, const voi
                                      int d_state, vim_dtype dt, void *workspace,
                                      size_t workspace_bytes, cudaStream_t stream,
                                      cudaEvent_t *events);
+
+/*
+ * Options of the _ex entry points, or-ed into `flags` (unknown bits return
+ * VIM_ERR_INVALID_ARG).
+ *
+ * VIM_FLAG_ZOH_EXACT: the exact zero-order-hold input matrix of section
+ * "Discretization via Zero-Order Hold (ZOH)", Bbar = (Delta A)^-1 (exp(Delta A) - I)
+ * Delta B, which for the diagonal A is, per state,
+ *     Bbar_n = (exp(Delta A_n) - 1) / A_n * B_n      (Delta B_n where A_n = 0),
+ * in place of its first-order form Bbar = Delta B used otherwise.  exp(Delta A_n) - 1
+ * is formed without cancellation for small Delta A_n.
+ */
+#define VIM_FLAG_ZOH_EXACT 1u
+
+/*
+ * vim_scan_bidir with every option: the convolution front when conv_w and conv_b are
+ * both non-NULL (then u holds x, as in vim_scan_bidir_conv; one NULL and the other
+ * not is VIM_ERR_INVALID_ARG), the options in `flags`, and the events of
+ * vim_scan_bidir_events when `events` is non-NULL.  Other arguments as in
+ * vim_scan_bidir.
+ */
+vim_status vim_scan_bidir_ex(const void *u, const float *conv_w, const float *conv_b,
+                             const void *delta, const void *z, const void *B, const void *C,
+                             int64_t bc_dir_stride, const float *A, const float *D,
+                             const float *delta_bias, void *y, int batch, int L, int d_inner,
+                             int d_state, vim_dtype dt, unsigned flags, void *workspace,
+                             size_t workspace_bytes, cudaStream_t stream, cudaEvent_t *events);
+
+/* vmamba_cross_scan4 with the options in `flags` and the events of
+ * vmamba_cross_scan4_events when `events` is non-NULL. */
+vim_status vmamba_cross_scan4_ex(const void *u, const void *delta, const void *z,
+                                 const void *B, const void *C,
+                                 const float *A, const float *D, const float *delta_bias,
+                                 void *y, int batch, int H, int W, int channels, int d_state,
+                                 vim_dtype dt, unsigned flags, void *workspace,
+                                 size_t workspace_bytes, cudaStream_t stream, cudaEvent_t *events);
 
 /*
  * vim_scan_bidir for callers that cannot allocate device memory.

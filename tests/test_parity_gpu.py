@@ -66,18 +66,18 @@ def vim_inputs(batch, L, Di, N, dtype, seed, *, generic_A=False, separate_bc=Fal
                 bias=bias.contiguous(), stride=batch * L * N if separate_bc else 0)
 
 
-def run_vim(vs, x, gate=True):
+def run_vim(vs, x, gate=True, zoh=False):
     dev = lambda t: t.cuda()
     y = vs.vim_scan_bidir(dev(x["u"]), dev(x["delta"]), dev(x["z"]) if gate else None,
                           dev(x["B"]), dev(x["C"]), dev(x["A"]), dev(x["D"]), dev(x["bias"]),
-                          bc_dir_stride=x["stride"])
+                          bc_dir_stride=x["stride"], zoh=zoh)
     torch.cuda.synchronize()
     return y
 
 
-def ref_vim(x, gate=True):
+def ref_vim(x, gate=True, zoh=False):
     return oracle.vim_bidir(x["u"], x["delta"], x["z"] if gate else None, x["B"], x["C"], x["A"],
-                            x["D"], x["bias"], bc_dir_stride=x["stride"])
+                            x["D"], x["bias"], bc_dir_stride=x["stride"], zoh=zoh)
 
 
 VIM_CASES = [
@@ -155,18 +155,18 @@ def conv_params(Di, seed):
     return w.contiguous(), b.contiguous()
 
 
-def run_vim_conv(vs, x, w, b, gate=True):
+def run_vim_conv(vs, x, w, b, gate=True, zoh=False):
     dev = lambda t: t.cuda()
     y = vs.vim_scan_bidir_conv(dev(x["u"]), dev(w), dev(b), dev(x["delta"]), dev(x["z"]) if gate else None,
                                dev(x["B"]), dev(x["C"]), dev(x["A"]), dev(x["D"]), dev(x["bias"]),
-                               bc_dir_stride=x["stride"])
+                               bc_dir_stride=x["stride"], zoh=zoh)
     torch.cuda.synchronize()
     return y
 
 
-def ref_vim_conv(x, w, b, gate=True):
+def ref_vim_conv(x, w, b, gate=True, zoh=False):
     return oracle.vim_bidir_conv(x["u"], w, b, x["delta"], x["z"] if gate else None, x["B"], x["C"], x["A"],
-                                 x["D"], x["bias"], bc_dir_stride=x["stride"])
+                                 x["D"], x["bias"], bc_dir_stride=x["stride"], zoh=zoh)
 
 
 CONV_CASES = [
@@ -236,17 +236,17 @@ def cross_inputs(batch, H, W, Ch, N, dtype, seed, generic_A=False):
     return dict(u=t(u), delta=t(dr), z=t(z), B=t(B), C=t(C), A=A, D=D.contiguous(), bias=bias)
 
 
-def run_cross(vs, x, gate=True):
+def run_cross(vs, x, gate=True, zoh=False):
     c = lambda t: t.cuda()
     y = vs.vmamba_cross_scan4(c(x["u"]), c(x["delta"]), c(x["z"]) if gate else None, c(x["B"]),
-                              c(x["C"]), c(x["A"]), c(x["D"]), c(x["bias"]))
+                              c(x["C"]), c(x["A"]), c(x["D"]), c(x["bias"]), zoh=zoh)
     torch.cuda.synchronize()
     return y
 
 
-def ref_cross(x, gate=True):
+def ref_cross(x, gate=True, zoh=False):
     return oracle.cross_scan4(x["u"], x["delta"], x["z"] if gate else None, x["B"], x["C"], x["A"],
-                              x["D"], x["bias"])
+                              x["D"], x["bias"], zoh=zoh)
 
 
 CROSS_CASES = [
@@ -341,3 +341,95 @@ def test_full_size_conv(vs):
     ref = oracle.vim_bidir_conv(x["u"], cw, cb, x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"],
                                 x["delta_bias"])
     check("full_conv_vim_tiny_1024px_bf16", y, ref, w.torch_dtype())
+
+
+# ---------------------------------------------------------------------------
+# exact zero-order hold (VIM_FLAG_ZOH_EXACT)
+# ---------------------------------------------------------------------------
+ZOH_VIM_CASES = [
+    # batch, L, Di, N, dtype, generic_A, separate_bc, delta_scale
+    (1, 1, 8, 16, torch.float32, False, False, 0.5),
+    (2, 17, 64, 16, torch.float32, False, True, 0.5),
+    (1, 33, 72, 8, torch.bfloat16, False, False, 0.5),
+    (2, 197, 200, 16, torch.float32, False, False, 3.0),    # Delta A_0 on both sides of -1/2
+    (1, 197, 64, 2, torch.bfloat16, True, False, 0.5),
+    (2, 257, 72, 16, torch.float32, False, True, 0.5),      # 3 chunks
+    (1, 300, 64, 4, torch.float32, True, True, 3.0),        # chunks with general A
+    (1, 1000, 128, 16, torch.bfloat16, False, False, 0.5),
+    (2, 1111, 64, 8, torch.float32, False, False, 3.0),
+    (1, 400, 36, 16, torch.float32, True, False, 0.5),
+]
+
+
+@pytest.mark.parametrize("case", ZOH_VIM_CASES, ids=lambda c: f"b{c[0]}_L{c[1]}_D{c[2]}_N{c[3]}_{str(c[4])[6:]}"
+                         f"{'_genA' if c[5] else ''}{'_sepBC' if c[6] else ''}_ds{c[7]}")
+def test_vim_zoh(vs, case):
+    """The exact zero-order-hold Bbar through the two-direction scan, against the
+    oracle's expm1(Delta A) / A * B; delta scale 3 puts Delta A_0 on both sides of the
+    kernel's switch between its series and exp - 1."""
+    batch, L, Di, N, dtype, gen, sep, ds = case
+    x = vim_inputs(batch, L, Di, N, dtype, seed=L * 13 + Di, generic_A=gen, separate_bc=sep, delta_scale=ds)
+    check(f"vim_zoh_{case}", run_vim(vs, x, zoh=True), ref_vim(x, zoh=True), dtype)
+
+
+def test_vim_zoh_differs_from_first_order(vs):
+    """The flag reaches the kernels: at Delta near 1 the two forms differ by far more
+    than the tolerance, and each side matches its own oracle."""
+    x = vim_inputs(1, 300, 64, 16, torch.float32, seed=44, delta_scale=3.0)
+    x["delta"] = (x["delta"].abs() + 4.0).contiguous()        # Delta about 4 .. 10
+    y_e, y_z = run_vim(vs, x), run_vim(vs, x, zoh=True)
+    r_e, r_z = ref_vim(x), ref_vim(x, zoh=True)
+    check("vim_zoh_big_delta", y_z, r_z, torch.float32)
+    check("vim_euler_big_delta", y_e, r_e, torch.float32)
+    assert normwise(y_z, r_e) > 1e-2
+
+
+def test_vim_zoh_zero_A(vs):
+    """A = 0 in one direction (structured, A_0 = 0): Bbar is its limit Delta B there."""
+    x = vim_inputs(2, 300, 64, 16, torch.float32, seed=45)
+    x["A"] = x["A"].clone()
+    x["A"][1] = 0.0
+    check("vim_zoh_zero_A", run_vim(vs, x, zoh=True), ref_vim(x, zoh=True), torch.float32)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_vim_conv_zoh(vs, dtype):
+    x = vim_inputs(2, 300, 72, 16, dtype, seed=46, separate_bc=True)
+    w, b = conv_params(72, seed=46)
+    check(f"vim_conv_zoh_{dtype}", run_vim_conv(vs, x, w, b, zoh=True), ref_vim_conv(x, w, b, zoh=True), dtype)
+
+
+ZOH_CROSS_CASES = [
+    # batch, H, W, C, N, dtype, generic_A
+    (1, 3, 5, 64, 16, torch.float32, False),
+    (1, 5, 3, 72, 8, torch.bfloat16, True),
+    (1, 7, 40, 64, 16, torch.float32, False),
+    (2, 32, 48, 72, 16, torch.bfloat16, False),
+]
+
+
+@pytest.mark.parametrize("case", ZOH_CROSS_CASES, ids=lambda c: f"b{c[0]}_{c[1]}x{c[2]}_C{c[3]}_N{c[4]}_"
+                         f"{str(c[5])[6:]}{'_genA' if c[6] else ''}")
+def test_cross_zoh(vs, case):
+    batch, H, W, Ch, N, dtype, gen = case
+    x = cross_inputs(batch, H, W, Ch, N, dtype, seed=H * 31 + W, generic_A=gen)
+    check(f"cross_zoh_{case}", run_cross(vs, x, zoh=True), ref_cross(x, zoh=True), dtype)
+
+
+@pytest.mark.parametrize("name", ["vim_tiny_1024px_bf16", "vmamba_64x64_bf16"])
+def test_full_size_zoh(vs, name):
+    """The exact hold at full size, in the benchmark's launch configuration."""
+    w = wl.BY_NAME[name]
+    x = wl.make_inputs(w)
+    oracle.set_threads(max(1, len(os.sched_getaffinity(0))))
+    dev = {k: v.cuda() for k, v in x.items()}
+    args = [dev[k] for k in ("u", "delta", "z", "B", "C", "A", "D", "delta_bias")]
+    refargs = [x[k] for k in ("u", "delta", "z", "B", "C", "A", "D", "delta_bias")]
+    if w.kind == "vim":
+        y = vs.vim_scan_bidir(*args, zoh=True)
+        ref = oracle.vim_bidir(*refargs, zoh=True)
+    else:
+        y = vs.vmamba_cross_scan4(*args, zoh=True)
+        ref = oracle.cross_scan4(*refargs, zoh=True)
+    torch.cuda.synchronize()
+    check(f"full_zoh_{name}", y, ref, w.torch_dtype())

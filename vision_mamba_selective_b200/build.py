@@ -9,6 +9,7 @@ import glob
 import os
 import subprocess
 import sys
+import tempfile
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -27,16 +28,25 @@ def deps():
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every csrc/*.cu to an object in parallel (the kernel variants are
+    spread over several units for that), then link the shared library."""
     if not force and os.path.exists(LIB):
         t = os.path.getmtime(LIB)
         if all(os.path.getmtime(f) <= t for f in deps()):
             return LIB
-    cmd = [NVCC, *ARCH, "-O3", "-lineinfo", "-std=c++17", "--cudart", "static",
-           "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"),
-           "-o", LIB, *sources()]
+    flags = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include")]
     if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
+        flags.insert(0, "-Xptxas=-v")
+    with tempfile.TemporaryDirectory(prefix="vimscan_build_") as tmp:
+        objs, procs = [], []
+        for src in sources():
+            obj = os.path.join(tmp, os.path.basename(src) + ".o")
+            objs.append(obj)
+            procs.append((src, subprocess.Popen([NVCC, *flags, "-c", "-o", obj, src])))
+        failed = [src for src, p in procs if p.wait() != 0]
+        if failed:
+            raise subprocess.CalledProcessError(1, f"nvcc ({', '.join(map(os.path.basename, failed))})")
+        subprocess.run([NVCC, *ARCH, "--cudart", "static", "-shared", "-o", LIB, *objs], check=True)
     return LIB
 
 

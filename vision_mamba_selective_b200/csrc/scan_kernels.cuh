@@ -147,6 +147,28 @@ __device__ __forceinline__ float softplus_io(float x) {
     else return softplus_fast(x);
 }
 
+// expm1(x) = exp(x) - 1 without the cancellation of exp(x) - 1 near 0: for |x| < 1/2
+// the Taylor series x + x^2/2! + ... + x^8/8! (Horner), whose first omitted term is
+// below 1.1e-8 of the result; elsewhere e - 1 with e = exp(x) given (from ex2), where
+// |result| > 0.39 keeps the relative error of the difference within a few 1e-7.
+__device__ __forceinline__ float expm1_acc(float x, float e) {
+    float p = fmaf(x, 1.0f / 40320.0f, 1.0f / 5040.0f);
+    p = fmaf(x, p, 1.0f / 720.0f);
+    p = fmaf(x, p, 1.0f / 120.0f);
+    p = fmaf(x, p, 1.0f / 24.0f);
+    p = fmaf(x, p, 1.0f / 6.0f);
+    p = fmaf(x, p, 0.5f);
+    p = fmaf(x, p, 1.0f);
+    return fabsf(x) < 0.5f ? x * p : e - 1.0f;
+}
+__device__ __forceinline__ float expm1_acc(float x) { return expm1_acc(x, ex2(x * kLog2e)); }
+
+// Bbar_n / B_n of the exact zero-order hold for one state, (exp(Delta A_n) - 1) / A_n,
+// and its limit Delta at A_n = 0
+__device__ __forceinline__ float zoh_gain(float dt, float An) {
+    return An != 0.0f ? expm1_acc(dt * An) / An : dt;
+}
+
 // silu(z) = z / (1 + exp(-z))
 __device__ __forceinline__ float silu(float z) { return z * rcp(1.0f + ex2(-z * kLog2e)); }
 
@@ -201,6 +223,7 @@ struct PairArgs {
     int batch, L, Di, H, W;
     int order;                      // 0: position = step; 1: column-major on H x W
     int chunk, G;                   // tokens per chunk (multiple of kTile), chunks
+    int zoh;                        // exact zero-order-hold Bbar instead of Delta B
 };
 
 // position visited at step t of the forward direction
@@ -209,6 +232,11 @@ __device__ __forceinline__ int position(const PairArgs &p, int t) {
     const int h = t % p.H, w = t / p.H;
     return h * p.W + w;
 }
+
+// Everything below is internal to each translation unit that includes this file:
+// the kernel variants are split over several units, which compile in parallel, and
+// each unit launches only the kernels it instantiates itself.
+namespace {
 
 // ----------------------------------------------------------------------------
 // shared-memory staging of one step: the forward tile and the backward tile
@@ -250,7 +278,7 @@ constexpr bool bc_vectorizable() { return (N * sizeof(T)) % 16 == 0; }
 // converted to fp32, into the slot.
 // Rows past the end of the chunk and channels past d_inner are zero-filled, so that
 // they act as no-op tokens.
-template <typename T, int N, bool VEC_BC, bool CONV = false>
+template <typename T, int N, bool VEC_BC, bool CONV = false, bool ZOH = false>
 struct Stager {
     using S = Stage<T, N, CONV>;
     static constexpr int V = Vec<T>::n;                 // elements per 16-byte piece
@@ -343,6 +371,8 @@ struct Stager {
         }
     }
 
+    // With the exact zero-order hold, B is staged as B_n / (n + 1) (the kernels' form
+    // of Bbar divides by A_n = (n + 1) A_0; see main_tile).
     __device__ void store_bc(char *slot) const {
 #pragma unroll
         for (int k = 0; k < kBCPer; ++k) {
@@ -356,12 +386,16 @@ struct Stager {
             if constexpr (VEC_BC) {
                 float f[V];
                 unpack16(pre_v[k], f);
+                if (ZOH && which == 0) {
+#pragma unroll
+                    for (int e = 0; e < V; ++e) f[e] *= __frcp_rn((float)(part * V + e + 1));
+                }
                 float4 *d4 = reinterpret_cast<float4 *>(dst + part * V);
 #pragma unroll
                 for (int q = 0; q < V / 4; ++q)
                     d4[q] = make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
             } else {
-                dst[part] = pre_s[k];
+                dst[part] = (ZOH && which == 0) ? pre_s[k] * __frcp_rn((float)(part + 1)) : pre_s[k];
             }
         }
     }
@@ -374,6 +408,7 @@ template <int N>
 struct ChannelParams {
     const float *A;     // A[dir][d][:] (general-A path)
     float A0;           // A[d][0] * log2(e)
+    float a0, inv_a0;   // A[d][0] and its reciprocal (0 when A[d][0] = 0)
     float D, bias;
     float cw_prev, cw_cur, cw_next, cbias;   // convolution front: taps on x[t-1], x[t], x[t+1]
     bool structured;    // A[d][n] == (n+1) A[d][0] for every n
@@ -382,7 +417,7 @@ struct ChannelParams {
     __device__ void load(const PairArgs &p, int dir, int d) {
         valid = d < p.Di;
         structured = true;
-        A0 = D = bias = 0.0f;
+        A0 = D = bias = a0 = inv_a0 = 0.0f;
         cw_prev = cw_cur = cw_next = cbias = 0.0f;
         A = p.A;
         if (!valid) return;
@@ -396,10 +431,11 @@ struct ChannelParams {
             cbias = p.conv_b[(size_t)dir * p.Di + d];
         }
         A = p.A + ((size_t)dir * p.Di + d) * N;
-        const float a0 = A[0];
+        a0 = A[0];
 #pragma unroll
         for (int n = 0; n < N; ++n) structured = structured && (A[n] == (float)(n + 1) * a0);
         A0 = a0 * kLog2e;
+        inv_a0 = a0 != 0.0f ? 1.0f / a0 : 0.0f;
         D = p.D[(size_t)dir * p.Di + d];
         bias = p.bias[(size_t)dir * p.Di + d];
     }
@@ -438,18 +474,32 @@ __device__ __forceinline__ float delta_of(const T *sd, int r, int dl, float bias
 // Delta summed over the tokens the direction visits after s inside the chunk.  With
 // A_n = (n+1) A_0 the weights are powers of w = exp(A_0 S_s), built by one multiply
 // per state.
-template <typename T, int N, bool FAST, bool DESC, bool CONV>
+template <typename T, int N, bool FAST, bool DESC, bool CONV, bool ZOH>
 __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, const ChannelParams<N> &prm,
                                            int dl, const T *su, const T *sd, const float *sB) {
     constexpr int NP = N / 2;
 #pragma unroll 1
     for (int sub = 0; sub < kTile / kCarrySub; ++sub) {
-        float Sv[kCarrySub], duv[kCarrySub];
+        // duv: Delta u (first-order Bbar); with the exact hold, the structured path
+        // keeps kappa u with kappa = expm1(Delta A_0) / A_0 and q = exp(Delta A_0), the
+        // general path u and Delta
+        float Sv[kCarrySub], duv[kCarrySub], qv[ZOH ? kCarrySub : 1];
 #pragma unroll
         for (int k = 0; k < kCarrySub; ++k) {
             const int r = walk_row<DESC>(sub * kCarrySub + k);
             const float dt = delta_of<T>(sd, r, dl, prm.bias);
-            duv[k] = dt * u_of<T, N, CONV>(su, r, dl, prm);
+            const float u = u_of<T, N, CONV>(su, r, dl, prm);
+            if constexpr (!ZOH) {
+                duv[k] = dt * u;
+            } else if constexpr (FAST) {
+                const float q = ex2(dt * prm.A0);
+                const float em1 = expm1_acc(dt * prm.a0, q);
+                duv[k] = u * (prm.a0 != 0.0f ? em1 * prm.inv_a0 : dt);
+                qv[k] = q;
+            } else {
+                duv[k] = u;
+                qv[k] = dt;
+            }
             Sv[k] = Ssum;          // Delta of the tokens walked before this one
             Ssum += dt;
         }
@@ -458,7 +508,7 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
             const int r = walk_row<DESC>(sub * kCarrySub + k);
             float2 Bv[NP];
             load_row<NP>(sB + r * N, Bv);
-            if constexpr (FAST) {
+            if constexpr (FAST && !ZOH) {
                 const float w = ex2(prm.A0 * Sv[k]);
                 const float x0 = w * duv[k];
                 float2 x = f2(x0, x0 * w);
@@ -468,12 +518,33 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
                     H[q] = fma2(x, Bv[q], H[q]);
                     x = mul2(x, w2);
                 }
+            } else if constexpr (FAST) {
+                // exact hold: state n gets w^(n+1) kappa u S_n B_n / (n+1) (B is staged
+                // divided by n+1), S_n = 1 + q + ... + q^n.  T_n = w^(n+1) kappa u S_n
+                // runs two states at a time: T_(n+2) = w^2 T_n + Q_n with
+                // Q_n = w^2 kappa u (1+q) (wq)^(n+1).
+                const float w = ex2(prm.A0 * Sv[k]);
+                const float q = qv[k], ku = duv[k];
+                const float c = ku * (1.0f + q);
+                const float ww = w * w, wq = w * q, wqwq = wq * wq;
+                float2 T = f2(ku * w, c * ww);
+                float2 Q = f2(ww * c * wq, ww * c * wqwq);
+                const float2 w2 = f2(ww, ww), wq2 = f2(wqwq, wqwq);
+#pragma unroll
+                for (int j = 0; j < NP; ++j) {
+                    H[j] = fma2(T, Bv[j], H[j]);
+                    T = fma2(w2, T, Q);
+                    Q = mul2(Q, wq2);
+                }
             } else {
                 const float2 du2 = f2(duv[k], duv[k]);
 #pragma unroll
                 for (int q = 0; q < NP; ++q) {
-                    const float2 wq = f2(ex2(__ldg(prm.A + 2 * q) * kLog2e * Sv[k]),
-                                         ex2(__ldg(prm.A + 2 * q + 1) * kLog2e * Sv[k]));
+                    const float A0n = __ldg(prm.A + 2 * q), A1n = __ldg(prm.A + 2 * q + 1);
+                    float2 wq = f2(ex2(A0n * kLog2e * Sv[k]), ex2(A1n * kLog2e * Sv[k]));
+                    if constexpr (ZOH)   // gain per state, times n+1 against the staged B / (n+1)
+                        wq = mul2(wq, f2(zoh_gain(qv[k], A0n) * (float)(2 * q + 1),
+                                         zoh_gain(qv[k], A1n) * (float)(2 * q + 2)));
                     H[q] = fma2(mul2(wq, du2), Bv[q], H[q]);
                 }
             }
@@ -481,8 +552,9 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
     }
 }
 
-template <typename T, int N, bool VEC_BC, bool CONV>
-__global__ void __launch_bounds__(kThreads, kCarryMinBlocks) pair_carry(PairArgs p) {
+// (the exact hold needs more registers than 6 CTAs per SM leave: 4 CTAs per SM)
+template <typename T, int N, bool VEC_BC, bool CONV, bool ZOH>
+__global__ void __launch_bounds__(kThreads, ZOH ? kMinBlocks : kCarryMinBlocks) pair_carry(PairArgs p) {
     using S = Stage<T, N, CONV>;
     constexpr int NP = N / 2;
     constexpr int kSlot = S::kSlotBytes;
@@ -500,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, kCarryMinBlocks) pair_carry(PairArgs
     const bool fast = __all_sync(0xffffffffu, prm.structured);
 
     // the forward direction walks tiles nT-1 .. 0, the backward one 0 .. nT-1
-    Stager<T, N, VEC_BC, CONV> st(p, b, t0, tc, d0);
+    Stager<T, N, VEC_BC, CONV, ZOH> st(p, b, t0, tc, d0);
     st.issue(smem, nT - 1, 0);
     st.load_bc(nT - 1, 0);
     st.store_bc(smem);
@@ -523,11 +595,11 @@ __global__ void __launch_bounds__(kThreads, kCarryMinBlocks) pair_carry(PairArgs
             const T *su = S::uv(cur, dir, 0), *sd = S::uv(cur, dir, 1);
             const float *sB = S::bc(cur, dir, 0);
             if (dir == 0) {
-                if (fast) carry_tile<T, N, true, true, CONV>(H, Ssum, prm, dl, su, sd, sB);
-                else carry_tile<T, N, false, true, CONV>(H, Ssum, prm, dl, su, sd, sB);
+                if (fast) carry_tile<T, N, true, true, CONV, ZOH>(H, Ssum, prm, dl, su, sd, sB);
+                else carry_tile<T, N, false, true, CONV, ZOH>(H, Ssum, prm, dl, su, sd, sB);
             } else {
-                if (fast) carry_tile<T, N, true, false, CONV>(H, Ssum, prm, dl, su, sd, sB);
-                else carry_tile<T, N, false, false, CONV>(H, Ssum, prm, dl, su, sd, sB);
+                if (fast) carry_tile<T, N, true, false, CONV, ZOH>(H, Ssum, prm, dl, su, sd, sB);
+                else carry_tile<T, N, false, false, CONV, ZOH>(H, Ssum, prm, dl, su, sd, sB);
             }
         }
         if (s + 1 < nT) {
@@ -618,21 +690,26 @@ __device__ __forceinline__ void add_f32(float (&acc)[V], const float *src) {
 // them.  Rows past the tile's end are no-op tokens.  The output of each token goes
 // to the chunk's fp32 partial buffer: stored on the tile's first visit, added on the
 // second (rows past the end only touch unread rows of the buffer).
-template <typename T, int N, bool FAST, bool DESC, bool CONV>
+template <typename T, int N, bool FAST, bool DESC, bool CONV, bool ZOH>
 __device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], const ChannelParams<N> &prm,
                                           int dl, const T *su, const T *sd, const float *sB,
                                           const float *sC, float *ypart) {
     constexpr int NP = N / 2;
 #pragma unroll 1
     for (int sub = 0; sub < kTile / kSub; ++sub) {
+        // qv: q = exp(Delta A_0) (structured A) or Delta (general A); duv: Delta u, or
+        // with the exact hold kappa u, kappa = expm1(Delta A_0) / A_0 (structured A)
         float qv[kSub], duv[kSub], uv[kSub];
 #pragma unroll
         for (int k = 0; k < kSub; ++k) {
             const int r = walk_row<DESC>(sub * kSub + k);
             const float dt = delta_of<T>(sd, r, dl, prm.bias);
             uv[k] = u_of<T, N, CONV>(su, r, dl, prm);
-            duv[k] = dt * uv[k];
             qv[k] = FAST ? ex2(dt * prm.A0) : dt;
+            if constexpr (ZOH && FAST)
+                duv[k] = uv[k] * (prm.a0 != 0.0f ? expm1_acc(dt * prm.a0, qv[k]) * prm.inv_a0 : dt);
+            else
+                duv[k] = dt * uv[k];
         }
 #pragma unroll
         for (int k = 0; k < kSub; ++k) {
@@ -646,6 +723,12 @@ __device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], const
             const float q = qv[k];
             float2 a = FAST ? f2(q, q * q) : f2(0.f, 0.f);
             const float2 step = FAST ? f2(a.y, a.y) : f2(0.f, 0.f);
+            // exact hold, structured A: Bbar_n u = kappa u S_n B_n / (n+1) with
+            // S_n = 1 + q + ... + q^n and B staged divided by n+1; KS = kappa u S for two
+            // states at a time, KS_(n+2) = KS_n + kappa u (1+q) q^(n+1)
+            const float cz = (ZOH && FAST) ? duv[k] * (1.0f + q) : 0.0f;
+            float2 KS = f2(duv[k], cz);
+            const float2 cz2 = f2(cz, cz);
 #pragma unroll
             for (int qq = 0; qq < NP; qq += 2) {
                 float2 Bp[2], Cp[2];
@@ -660,14 +743,28 @@ __device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], const
 #pragma unroll
                 for (int e = 0; e < 2 && qq + e < NP; ++e) {
                     const int qi = qq + e;
-                    float2 aq;
+                    float2 aq, drive;
                     if constexpr (FAST) {
                         aq = a;
                         a = mul2(a, step);
+                        if constexpr (ZOH) {
+                            drive = mul2(KS, Bp[e]);
+                            KS = fma2(aq, cz2, KS);
+                        } else {
+                            drive = mul2(du2, Bp[e]);
+                        }
                     } else {
-                        aq = f2(ex2(q * __ldg(prm.A + 2 * qi) * kLog2e), ex2(q * __ldg(prm.A + 2 * qi + 1) * kLog2e));
+                        const float A0n = __ldg(prm.A + 2 * qi), A1n = __ldg(prm.A + 2 * qi + 1);
+                        aq = f2(ex2(q * A0n * kLog2e), ex2(q * A1n * kLog2e));
+                        if constexpr (ZOH)   // gain per state, times n+1 against the staged B / (n+1)
+                            drive = mul2(mul2(f2(zoh_gain(q, A0n) * (float)(2 * qi + 1),
+                                                 zoh_gain(q, A1n) * (float)(2 * qi + 2)),
+                                              f2(uv[k], uv[k])),
+                                         Bp[e]);
+                        else
+                            drive = mul2(du2, Bp[e]);
                     }
-                    h[qi] = fma2(aq, h[qi], mul2(du2, Bp[e]));
+                    h[qi] = fma2(aq, h[qi], drive);
                     if (qi & 1) y1 = fma2(Cp[e], h[qi], y1);
                     else y0 = fma2(Cp[e], h[qi], y0);
                 }
@@ -780,7 +877,7 @@ struct Finisher {
     }
 };
 
-template <typename T, int N, bool VEC_BC, bool PIN, bool CONV>
+template <typename T, int N, bool VEC_BC, bool PIN, bool CONV, bool ZOH>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
     using S = Stage<T, N, CONV>;
     constexpr int NP = N / 2;
@@ -798,7 +895,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
     prm.load(p, dir, d);
     const bool fast = __all_sync(0xffffffffu, prm.structured);
 
-    Stager<T, N, VEC_BC, CONV> st(p, b, t0, tc, d0);
+    Stager<T, N, VEC_BC, CONV, ZOH> st(p, b, t0, tc, d0);
     st.issue(smem, 0, nT - 1);
     st.load_bc(0, nT - 1);
 
@@ -842,11 +939,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
             const float *sB = S::bc(cur, dir, 0), *sC = S::bc(cur, dir, 1);
             const bool second = twice > 0;
             if (dir == 0) {
-                if (fast) main_tile<T, N, true, false, CONV>(second, h, prm, dl, su, sd, sB, sC, ypart);
-                else main_tile<T, N, false, false, CONV>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                if (fast) main_tile<T, N, true, false, CONV, ZOH>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                else main_tile<T, N, false, false, CONV, ZOH>(second, h, prm, dl, su, sd, sB, sC, ypart);
             } else {
-                if (fast) main_tile<T, N, true, true, CONV>(second, h, prm, dl, su, sd, sB, sC, ypart);
-                else main_tile<T, N, false, true, CONV>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                if (fast) main_tile<T, N, true, true, CONV, ZOH>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                else main_tile<T, N, false, true, CONV, ZOH>(second, h, prm, dl, su, sd, sB, sC, ypart);
             }
         }
         if (s + 1 < nT) {
@@ -915,4 +1012,5 @@ __global__ void __launch_bounds__(256) merge4(MergeArgs a) {
     }
 }
 
+}  // namespace
 }  // namespace vimscan

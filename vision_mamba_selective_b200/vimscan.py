@@ -41,6 +41,14 @@ lib.vim_scan_bidir_conv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp
 lib.vim_scan_bidir_conv.restype = _i
 lib.vim_scan_bidir_conv_events.argtypes = lib.vim_scan_bidir_conv.argtypes + [_vp]
 lib.vim_scan_bidir_conv_events.restype = _i
+_u = ctypes.c_uint
+lib.vim_scan_bidir_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
+                                  _i, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp]
+lib.vim_scan_bidir_ex.restype = _i
+lib.vmamba_cross_scan4_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                      _i, _i, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp]
+lib.vmamba_cross_scan4_ex.restype = _i
+VIM_FLAG_ZOH_EXACT = 1
 lib.vim_scan_bidir_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
                                        _i, _i, _i, _i, _i, _vp]
 lib.vim_scan_bidir_noalloc.restype = _i
@@ -113,58 +121,61 @@ def _events(events):
     return (ctypes.c_void_p * len(handles))(*handles)
 
 
-def vim_scan_bidir(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride=0,
-                   workspace=None, stream=None, events=None):
-    """Vim bidirectional selective scan, (y^f + y^b) * silu(z); see include/vimscan.h.
-
-    u, delta, z: [batch, L, d_inner]; B, C: [batch, L, d_state] (or a larger buffer
-    whose backward copy starts ``bc_dir_stride`` elements in); A: [2, d_inner,
-    d_state] fp32; D, delta_bias: [2, d_inner] fp32.  Returns y [batch, L, d_inner].
-    """
+def _bidir(name, u, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, y, bc_dir_stride, workspace, stream,
+           events, zoh):
     batch, L, Di = u.shape
     N = B.shape[-1]
     dt = _dtype_code(u)
     if y is None:
         y = torch.empty_like(u)
     ws, ws_bytes = _workspace(vim_scan_workspace_bytes(0, batch, L, 0, Di, N), workspace, u.device)
-    extra = () if events is None else (_events(events),)
-    fn = lib.vim_scan_bidir if events is None else lib.vim_scan_bidir_events
-    st = fn(
-        _ptr(u, name="u"), _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
+    conv = conv_w is not None or conv_b is not None
+    pre = (_ptr(u, name="x" if conv else "u"),)
+    if conv or zoh:
+        pre += (_ptr(conv_w, dtype=torch.float32, name="conv_w"), _ptr(conv_b, dtype=torch.float32, name="conv_b"))
+    args = pre + (
+        _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
         _ptr(B, dtype=u.dtype, name="B"), _ptr(C, dtype=u.dtype, name="C"), int(bc_dir_stride),
         _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
         _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(y, dtype=u.dtype, name="y"),
-        batch, L, Di, N, dt, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream), *extra)
+        batch, L, Di, N, dt)
+    tail = (None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
+    ev = None if events is None else _events(events)
+    if zoh:
+        st = lib.vim_scan_bidir_ex(*args, VIM_FLAG_ZOH_EXACT, *tail, ev)
+    elif conv:
+        st = (lib.vim_scan_bidir_conv(*args, *tail) if ev is None
+              else lib.vim_scan_bidir_conv_events(*args, *tail, ev))
+    else:
+        st = lib.vim_scan_bidir(*args, *tail) if ev is None else lib.vim_scan_bidir_events(*args, *tail, ev)
     if st != VIM_OK:
-        raise VimScanError(st, "vim_scan_bidir")
+        raise VimScanError(st, name)
     return y
+
+
+def vim_scan_bidir(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride=0,
+                   workspace=None, stream=None, events=None, zoh=False):
+    """Vim bidirectional selective scan, (y^f + y^b) * silu(z); see include/vimscan.h.
+
+    u, delta, z: [batch, L, d_inner]; B, C: [batch, L, d_state] (or a larger buffer
+    whose backward copy starts ``bc_dir_stride`` elements in); A: [2, d_inner,
+    d_state] fp32; D, delta_bias: [2, d_inner] fp32.  Returns y [batch, L, d_inner].
+    zoh=True takes the exact zero-order-hold Bbar (VIM_FLAG_ZOH_EXACT).
+    """
+    return _bidir("vim_scan_bidir", u, None, None, delta, z, B, C, A, D, delta_bias, y, bc_dir_stride,
+                  workspace, stream, events, zoh)
 
 
 def vim_scan_bidir_conv(x, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride=0,
-                        workspace=None, stream=None, events=None):
+                        workspace=None, stream=None, events=None, zoh=False):
     """vim_scan_bidir with the pathways' kernel-3 convolution + SiLU front fused in.
 
     x, delta, z: [batch, L, d_inner]; conv_w: [2, d_inner, 3] fp32; conv_b: [2, d_inner]
-    fp32; the rest as in vim_scan_bidir.  Returns y [batch, L, d_inner].
+    fp32; the rest as in vim_scan_bidir.  Returns y [batch, L, d_inner].  A missing
+    half of the front (conv_w or conv_b None) is rejected by the library.
     """
-    batch, L, Di = x.shape
-    N = B.shape[-1]
-    dt = _dtype_code(x)
-    if y is None:
-        y = torch.empty_like(x)
-    ws, ws_bytes = _workspace(vim_scan_workspace_bytes(0, batch, L, 0, Di, N), workspace, x.device)
-    extra = () if events is None else (_events(events),)
-    fn = lib.vim_scan_bidir_conv if events is None else lib.vim_scan_bidir_conv_events
-    st = fn(
-        _ptr(x, name="x"), _ptr(conv_w, dtype=torch.float32, name="conv_w"),
-        _ptr(conv_b, dtype=torch.float32, name="conv_b"), _ptr(delta, dtype=x.dtype, name="delta"),
-        _ptr(z, dtype=x.dtype, name="z"), _ptr(B, dtype=x.dtype, name="B"), _ptr(C, dtype=x.dtype, name="C"),
-        int(bc_dir_stride), _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
-        _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(y, dtype=x.dtype, name="y"),
-        batch, L, Di, N, dt, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream), *extra)
-    if st != VIM_OK:
-        raise VimScanError(st, "vim_scan_bidir_conv")
-    return y
+    return _bidir("vim_scan_bidir_conv", x, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, y,
+                  bc_dir_stride, workspace, stream, events, zoh)
 
 
 def vim_scan_bidir_noalloc(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride=0, stream=None):
@@ -192,11 +203,12 @@ def vim_scan_bidir_noalloc(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_di
 
 
 def vmamba_cross_scan4(u, delta, z, B, C, A, D, delta_bias, *, y=None, workspace=None, stream=None,
-                       events=None):
+                       events=None, zoh=False):
     """VMamba four-direction cross-scan with CS-Merge; see include/vimscan.h.
 
     u, delta, z: [batch, H, W, C]; B, C: [4, batch, H*W, d_state] by grid position;
     A: [4, C, d_state] fp32; D, delta_bias: [4, C] fp32.  Returns y [batch, H, W, C].
+    zoh=True takes the exact zero-order-hold Bbar (VIM_FLAG_ZOH_EXACT).
     """
     batch, H, W, Ch = u.shape
     N = B.shape[-1]
@@ -204,14 +216,20 @@ def vmamba_cross_scan4(u, delta, z, B, C, A, D, delta_bias, *, y=None, workspace
     if y is None:
         y = torch.empty_like(u)
     ws, ws_bytes = _workspace(vim_scan_workspace_bytes(1, batch, H, W, Ch, N), workspace, u.device)
-    extra = () if events is None else (_events(events),)
-    fn = lib.vmamba_cross_scan4 if events is None else lib.vmamba_cross_scan4_events
-    st = fn(
+    args = (
         _ptr(u, name="u"), _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
         _ptr(B, dtype=u.dtype, name="B"), _ptr(C, dtype=u.dtype, name="C"),
         _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
         _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(y, dtype=u.dtype, name="y"),
-        batch, H, W, Ch, N, dt, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream), *extra)
+        batch, H, W, Ch, N, dt)
+    tail = (None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
+    ev = None if events is None else _events(events)
+    if zoh:
+        st = lib.vmamba_cross_scan4_ex(*args, VIM_FLAG_ZOH_EXACT, *tail, ev)
+    elif ev is None:
+        st = lib.vmamba_cross_scan4(*args, *tail)
+    else:
+        st = lib.vmamba_cross_scan4_events(*args, *tail, ev)
     if st != VIM_OK:
         raise VimScanError(st, "vmamba_cross_scan4")
     return y
