@@ -59,6 +59,8 @@ class Oracle:
         lib.oracle_cross_order.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _I64]
         lib.oracle_conv_silu.argtypes = [_D, _D, _D, _D] + [ctypes.c_int] * 4
         lib.oracle_vim_bidir_conv.argtypes = [_D, _D, _D, _D, _D, _D, _D, ctypes.c_int64, _D, _D, _D, _D] + [ctypes.c_int] * 6
+        lib.oracle_s6_direction_bwd.argtypes = [_D] * 7 + [_I64] + [_D] * 8 + [ctypes.c_int] * 5
+        lib.oracle_vim_bidir_bwd.argtypes = [_D, _D, _D, _D, _D, ctypes.c_int64] + [_D] * 12 + [ctypes.c_int] * 5
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
         self.lib = lib
@@ -120,6 +122,31 @@ class Oracle:
         if rc:
             raise ValueError("oracle_vim_bidir: bad sizes")
         return y
+
+    def vim_bidir_bwd(self, u, delta, z, B, C, A, D, bias, dout, *, bc_dir_stride=0, delta_is_raw=True):
+        """Derivatives of vim_bidir (first-order Bbar) for the loss sum(dout * y).
+
+        Returns a dict of fp64 arrays: du, ddelta (w.r.t. the raw delta when
+        delta_is_raw), dz (None without a gate), dB and dC shaped like B and C, dA
+        [2, Di, N], dD and dbias [2, Di] (dbias zero when not delta_is_raw).
+        """
+        u, delta, z, B, C, A, D, bias, dout = map(_f64, (u, delta, z, B, C, A, D, bias, dout))
+        batch, L, Di = u.shape
+        N = B.shape[-1]
+        if bias is None:
+            bias = np.zeros((2, Di))
+        out = dict(du=np.zeros((batch, L, Di)), ddelta=np.zeros((batch, L, Di)),
+                   dz=np.zeros((batch, L, Di)) if z is not None else None,
+                   dB=np.zeros(B.shape), dC=np.zeros(C.shape), dA=np.zeros((2, Di, N)),
+                   dD=np.zeros((2, Di)), dbias=np.zeros((2, Di)))
+        rc = self.lib.oracle_vim_bidir_bwd(_p(u), _p(delta), _p(z), _p(B), _p(C), int(bc_dir_stride),
+                                           _p(A), _p(D), _p(bias), _p(dout), _p(out["du"]),
+                                           _p(out["ddelta"]), _p(out["dz"]), _p(out["dB"]), _p(out["dC"]),
+                                           _p(out["dA"]), _p(out["dD"]), _p(out["dbias"]),
+                                           batch, L, Di, N, int(bool(delta_is_raw)))
+        if rc:
+            raise ValueError("oracle_vim_bidir_bwd: bad sizes")
+        return out
 
     def conv_silu(self, x, w, cb, *, reversed=False):
         """silu of the kernel-3 depthwise convolution (zero padding 1) in front of a
@@ -224,6 +251,10 @@ def cross_scan4(*a, **k):
 
 def conv_silu(*a, **k):
     return default().conv_silu(*a, **k)
+
+
+def vim_bidir_bwd(*a, **k):
+    return default().vim_bidir_bwd(*a, **k)
 
 
 def vim_bidir_conv(*a, **k):

@@ -310,3 +310,179 @@ int oracle_cross_merge4(const double *ys, const double *z, double *y,
     apply_gate(y, z, total);
     return 0;
 }
+
+/* ------------------------------------------------------------------------------
+ * Reverse-mode derivatives (training through the scan).  The pages motivate the
+ * scan by efficient training on GPUs; the derivative of the forward map above is
+ * taken here by the chain rule, step by step in reverse visiting order, for a
+ * scalar loss  ell = sum dy[b,t,d] * y[b,t,d].  Only the first-order Bbar = Delta B
+ * is covered.
+ * ------------------------------------------------------------------------------ */
+
+/* d softplus(x) / dx with the same cut as softplus(): 1/(1 + e^-x), and 1 above 20. */
+static double softplus_grad(double x) { return x > 20.0 ? 1.0 : 1.0 / (1.0 + exp(-x)); }
+
+/* d silu(z) / dz = s (1 + z (1 - s)), s = 1/(1 + e^-z). */
+static double silu_grad(double z)
+{
+    double s = 1.0 / (1.0 + exp(-z));
+    return s * (1.0 + z * (1.0 - s));
+}
+
+/*
+ * Derivative of one S6 direction (oracle_s6_direction, first-order Bbar).
+ *   dy       : [batch, L, Di], the loss's derivative with respect to y
+ *   du, ddelta : [batch, L, Di]   (ddelta is w.r.t. the raw delta when delta_is_raw,
+ *                                  else w.r.t. Delta itself)
+ *   dB, dC   : [batch, L, N];  dA : [Di, N];  dD, dbias : [Di]  (dbias only when raw)
+ * Every output is ADDED to (so that directions sharing an input accumulate).
+ * For each (b, d) the forward pass is run first, keeping h_t for every step; then
+ * the adjoint g of h runs backwards: g <- g + C_t dy_t is dl/dh_t, from which
+ *   dl/dC_t = dy_t h_t,  dl/dD += dy_t u_t,  dl/du_t += D dy_t + sum_n g_n Delta_t B_tn,
+ *   dl/dAbar_n = g_n h_{t-1,n}  ->  dl/dDelta += that * Abar_n * A_n,
+ *                                   dl/dA_n   += that * Abar_n * Delta_t,
+ *   dl/dDelta += sum_n g_n B_tn u_t,  dl/dB_tn += g_n Delta_t u_t,
+ * and g <- g * Abar is dl/dh_{t-1}.
+ */
+int oracle_s6_direction_bwd(const double *u, const double *delta, const double *B, const double *C,
+                            const double *A, const double *D, const double *bias,
+                            const int64_t *order, const double *dy,
+                            double *du, double *ddelta, double *dB, double *dC,
+                            double *dA, double *dD, double *dbias,
+                            int batch, int L, int Di, int N, int delta_is_raw)
+{
+    if (batch < 0 || L < 0 || Di < 0 || N < 1 || N > ORACLE_MAX_STATE) return -1;
+    int rc = 0;
+    #pragma omp parallel
+    {
+        double *hs = (double *)malloc(((size_t)(L > 0 ? L : 1)) * (size_t)N * sizeof(double));
+        double *dts = (double *)malloc(((size_t)(L > 0 ? L : 1)) * sizeof(double));
+        double *dA_loc = (double *)calloc((size_t)Di * N, sizeof(double));
+        double *dD_loc = (double *)calloc((size_t)(Di > 0 ? Di : 1), sizeof(double));
+        double *db_loc = (double *)calloc((size_t)(Di > 0 ? Di : 1), sizeof(double));
+        int ok = hs && dts && dA_loc && dD_loc && db_loc;
+        if (!ok) {
+            #pragma omp atomic write
+            rc = -1;
+        }
+        /* batch items in parallel: dB and dC rows belong to one batch item */
+        #pragma omp for schedule(dynamic, 1)
+        for (int64_t b = 0; b < batch; ++b) {
+            if (!ok) continue;
+            for (int64_t d = 0; d < Di; ++d) {
+                const double *Ad = A + d * N;
+                double h[ORACLE_MAX_STATE], g[ORACLE_MAX_STATE];
+                for (int n = 0; n < N; ++n) h[n] = 0.0;
+                for (int64_t t = 0; t < L; ++t) {                 /* forward, keeping h_t */
+                    int64_t p = order[t];
+                    int64_t ix = (b * L + p) * Di + d;
+                    const double *Bt = B + (b * L + p) * N;
+                    double dt = delta_is_raw ? softplus(delta[ix] + bias[d]) : delta[ix];
+                    dts[t] = dt;
+                    for (int n = 0; n < N; ++n) {
+                        h[n] = exp(dt * Ad[n]) * h[n] + dt * Bt[n] * u[ix];
+                        hs[t * N + n] = h[n];
+                    }
+                }
+                for (int n = 0; n < N; ++n) g[n] = 0.0;
+                for (int64_t t = L - 1; t >= 0; --t) {            /* adjoint, in reverse */
+                    int64_t p = order[t];
+                    int64_t ix = (b * L + p) * Di + d;
+                    const double *Bt = B + (b * L + p) * N, *Ct = C + (b * L + p) * N;
+                    double *dBt = dB + (b * L + p) * N, *dCt = dC + (b * L + p) * N;
+                    double dt = dts[t], x = u[ix], e = dy[ix];
+                    double dDelta = 0.0, dx = D[d] * e;
+                    dD_loc[d] += e * x;
+                    for (int n = 0; n < N; ++n) {
+                        g[n] += Ct[n] * e;                        /* dl/dh_t            */
+                        dCt[n] += e * hs[t * N + n];
+                        double Abar = exp(dt * Ad[n]);
+                        double hprev = t > 0 ? hs[(t - 1) * N + n] : 0.0;
+                        double dAbar = g[n] * hprev;
+                        dDelta += dAbar * Abar * Ad[n] + g[n] * Bt[n] * x;
+                        dA_loc[d * N + n] += dAbar * Abar * dt;
+                        dBt[n] += g[n] * dt * x;
+                        dx += g[n] * dt * Bt[n];
+                        g[n] *= Abar;                             /* dl/dh_{t-1} part   */
+                    }
+                    du[ix] += dx;
+                    if (delta_is_raw) {
+                        double s = softplus_grad(delta[ix] + bias[d]);
+                        ddelta[ix] += dDelta * s;
+                        db_loc[d] += dDelta * s;
+                    } else {
+                        ddelta[ix] += dDelta;
+                    }
+                }
+            }
+        }
+        #pragma omp critical
+        {
+            if (ok) {
+                for (int64_t i = 0; i < (int64_t)Di * N; ++i) dA[i] += dA_loc[i];
+                for (int64_t d = 0; d < Di; ++d) {
+                    dD[d] += dD_loc[d];
+                    if (delta_is_raw) dbias[d] += db_loc[d];
+                }
+            }
+        }
+        free(hs); free(dts); free(dA_loc); free(dD_loc); free(db_loc);
+    }
+    return rc;
+}
+
+/*
+ * Derivative of oracle_vim_bidir (first-order Bbar) for ell = sum dout * y.
+ *   dout : [batch, L, Di].  Outputs (overwritten):
+ *   du, ddelta, dz : [batch, L, Di]  (dz untouched when z is NULL; ddelta w.r.t. the
+ *                    raw delta when delta_is_raw)
+ *   dB, dC : shaped like B and C (with bc_dir_stride > 0 the backward direction's part
+ *            starts bc_dir_stride elements in; with 0 both directions add into one)
+ *   dA [2, Di, N], dD [2, Di], dbias [2, Di]
+ * With y = (y^f + y^b) silu(z):  dl/dz = dout (y^f + y^b) silu'(z) and each direction
+ * sees dl/dy^k = dout silu(z).
+ */
+int oracle_vim_bidir_bwd(const double *u, const double *delta, const double *z,
+                         const double *B, const double *C, int64_t bc_dir_stride,
+                         const double *A, const double *D, const double *bias, const double *dout,
+                         double *du, double *ddelta, double *dz, double *dB, double *dC,
+                         double *dA, double *dD, double *dbias,
+                         int batch, int L, int Di, int N, int delta_is_raw)
+{
+    if (batch < 0 || L < 0 || Di < 0 || N < 1 || bc_dir_stride < 0) return -1;
+    int64_t n_act = (int64_t)batch * L * Di, n_bc = (int64_t)batch * L * N;
+    int64_t n_bc_all = bc_dir_stride > 0 ? bc_dir_stride + n_bc : n_bc;
+    double *dy = (double *)malloc((size_t)(n_act > 0 ? n_act : 1) * sizeof(double));
+    int64_t *order = (int64_t *)malloc((size_t)(L > 0 ? L : 1) * sizeof(int64_t));
+    if (!dy || !order) { free(dy); free(order); return -1; }
+    for (int64_t i = 0; i < n_act; ++i) { du[i] = 0.0; ddelta[i] = 0.0; }
+    for (int64_t i = 0; i < n_bc_all; ++i) { dB[i] = 0.0; dC[i] = 0.0; }
+    for (int64_t i = 0; i < 2 * (int64_t)Di * N; ++i) dA[i] = 0.0;
+    for (int64_t i = 0; i < 2 * (int64_t)Di; ++i) { dD[i] = 0.0; dbias[i] = 0.0; }
+    int rc = 0;
+    if (z) {
+        /* the ungated sum y^f + y^b, for dl/dz */
+        double *ys = (double *)malloc((size_t)(n_act > 0 ? n_act : 1) * sizeof(double));
+        if (!ys) { free(dy); free(order); return -1; }
+        rc |= oracle_vim_bidir(u, delta, NULL, B, C, bc_dir_stride, A, D, bias, ys,
+                               batch, L, Di, N, delta_is_raw, 0);
+        for (int64_t i = 0; i < n_act; ++i) {
+            dz[i] = dout[i] * ys[i] * silu_grad(z[i]);
+            dy[i] = dout[i] * silu(z[i]);
+        }
+        free(ys);
+    } else {
+        for (int64_t i = 0; i < n_act; ++i) dy[i] = dout[i];
+    }
+    for (int64_t t = 0; t < L; ++t) order[t] = t;
+    rc |= oracle_s6_direction_bwd(u, delta, B, C, A, D, bias, order, dy, du, ddelta, dB, dC,
+                                  dA, dD, dbias, batch, L, Di, N, delta_is_raw);
+    for (int64_t t = 0; t < L; ++t) order[t] = L - 1 - t;
+    rc |= oracle_s6_direction_bwd(u, delta, B + bc_dir_stride, C + bc_dir_stride,
+                                  A + (int64_t)Di * N, D + Di, bias + Di, order, dy, du, ddelta,
+                                  dB + bc_dir_stride, dC + bc_dir_stride,
+                                  dA + (int64_t)Di * N, dD + Di, dbias + Di,
+                                  batch, L, Di, N, delta_is_raw);
+    free(dy); free(order);
+    return rc ? -1 : 0;
+}

@@ -493,6 +493,61 @@ def pin_zoh_reaches_every_entry(orc):
     np.testing.assert_allclose(y, sum(_untraverse(np.stack(outs), H, W)), rtol=1e-12, atol=1e-12)
 
 
+def _bwd_case(rng, batch=1, L=5, Di=2, N=3, separate_bc=True):
+    c = _vim_case(rng, batch=batch, L=L, Di=Di, N=N, separate_bc=separate_bc)
+    c["delta"] = rng.normal(size=c["u"].shape) * 0.8          # raw delta
+    c["dout"] = rng.normal(size=c["u"].shape)
+    return c
+
+
+def _loss(orc, c, **over):
+    c = {**c, **over}
+    y = orc.vim_bidir(c["u"], c["delta"], c["z"], c["B"], c["C"], c["A"], c["D"], c["bias"],
+                      bc_dir_stride=c["stride"], delta_is_raw=True)
+    return float(np.sum(c["dout"] * y))
+
+
+def pin_bwd_finite_differences(orc):
+    """Every derivative of the two-direction scan (u, raw delta, z, per-direction B
+    and C, A, D, delta bias) against central finite differences of the loss
+    sum(dout * y) computed with the forward oracle alone (sections "Discretization
+    via Zero-Order Hold (ZOH)", "The Selective State Space (S6) Mechanism", "2. The
+    Bidirectional Mamba Block").  Step 1e-6 in fp64: truncation and rounding stay
+    near 1e-9 of the gradient's size."""
+    c = _bwd_case(_rng(101))
+    g = orc.vim_bidir_bwd(c["u"], c["delta"], c["z"], c["B"], c["C"], c["A"], c["D"], c["bias"], c["dout"],
+                          bc_dir_stride=c["stride"])
+    for name, key in (("u", "du"), ("delta", "ddelta"), ("z", "dz"), ("B", "dB"), ("C", "dC"),
+                      ("A", "dA"), ("D", "dD"), ("bias", "dbias")):
+        arr, eps = c[name], 1e-6
+        fd = np.zeros_like(arr)
+        for i in np.ndindex(arr.shape):
+            up, dn = arr.copy(), arr.copy()
+            up[i] += eps
+            dn[i] -= eps
+            fd[i] = (_loss(orc, c, **{name: up}) - _loss(orc, c, **{name: dn})) / (2 * eps)
+        err = np.max(np.abs(fd - g[key])) / np.max(np.abs(fd))
+        assert err < 1e-7, (name, err)
+
+
+def pin_bwd_homogeneity(orc):
+    """Identities of the loss's derivative at a larger size, with B and C shared by
+    the directions: the output is linear in u, in B and in C (Delta fixed), so by
+    Euler's theorem sum(du*u) = ell, sum(dB*B) = sum(dC*C) = ell minus the D u part,
+    and sum(dD*D) = the D u part (each direction's D enters linearly)."""
+    rng = _rng(102)
+    c = _bwd_case(rng, batch=2, L=40, Di=5, N=4, separate_bc=False)
+    g = orc.vim_bidir_bwd(c["u"], c["delta"], c["z"], c["B"], c["C"], c["A"], c["D"], c["bias"], c["dout"],
+                          bc_dir_stride=0)
+    ell = _loss(orc, c)
+    silu = c["z"] / (1 + np.exp(-c["z"]))
+    ell_D = float(np.sum(c["dout"] * silu * (c["D"][0] + c["D"][1])[None, None, :] * c["u"]))
+    np.testing.assert_allclose(np.sum(g["du"] * c["u"]), ell, rtol=1e-11)
+    np.testing.assert_allclose(np.sum(g["dB"] * c["B"]), ell - ell_D, rtol=1e-11)
+    np.testing.assert_allclose(np.sum(g["dC"] * c["C"]), ell - ell_D, rtol=1e-11)
+    np.testing.assert_allclose(np.sum(g["dD"] * c["D"]), ell_D, rtol=1e-11)
+
+
 ALL_PINS = [
     pin_delta_zero,
     pin_constant_input_geometric,
@@ -511,4 +566,6 @@ ALL_PINS = [
     pin_zoh_matches_ode,
     pin_zoh_fixed_point_and_limits,
     pin_zoh_reaches_every_entry,
+    pin_bwd_finite_differences,
+    pin_bwd_homogeneity,
 ]

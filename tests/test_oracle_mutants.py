@@ -48,6 +48,17 @@ MUTANTS = {
     "zoh_delta_twice": ("return expm1(dt * An) / An * Bn;", "return dt * expm1(dt * An) / An * Bn;"),
     "zoh_dropped_in_bidir": ("delta_is_raw, 0, zoh);", "delta_is_raw, 0, 0);"),
     "zoh_dropped_in_cross": ("delta_is_raw, k > 0, zoh);", "delta_is_raw, k > 0, 0);"),
+    "bwd_adjoint_not_decayed": ("g[n] *= Abar;", "g[n] *= 1.0;"),
+    "bwd_hprev_is_h": ("double hprev = t > 0 ? hs[(t - 1) * N + n] : 0.0;", "double hprev = hs[t * N + n];"),
+    "bwd_dA_without_delta": ("dA_loc[d * N + n] += dAbar * Abar * dt;", "dA_loc[d * N + n] += dAbar * Abar;"),
+    "bwd_dB_without_u": ("dBt[n] += g[n] * dt * x;", "dBt[n] += g[n] * dt;"),
+    "bwd_softplus_grad_sign": ("return x > 20.0 ? 1.0 : 1.0 / (1.0 + exp(-x));",
+                               "return x > 20.0 ? 1.0 : 1.0 / (1.0 + exp(x));"),
+    "bwd_gate_grad_is_sigmoid": ("return s * (1.0 + z * (1.0 - s));", "return s;"),
+    "bwd_D_skip_dropped": ("double dDelta = 0.0, dx = D[d] * e;", "double dDelta = 0.0, dx = 0.0;"),
+    "bwd_backward_dir_forward_params": ("A + (int64_t)Di * N, D + Di, bias + Di, order, dy,",
+                                        "A, D, bias, order, dy,"),
+    "bwd_dy_ungated": ("dy[i] = dout[i] * silu(z[i]);", "dy[i] = dout[i];"),
     "zoh_sign": ("return expm1(dt * An) / An * Bn;", "return expm1(-dt * An) / An * Bn;"),
 }
 

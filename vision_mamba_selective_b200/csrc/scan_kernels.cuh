@@ -45,10 +45,18 @@ constexpr int kTile = 16;            // tokens per staged tile
 #ifndef VIMSCAN_CARRY_MIN_BLOCKS
 #define VIMSCAN_CARRY_MIN_BLOCKS 6
 #endif
+#ifndef VIMSCAN_CARRY_ZOH_KSUB
+#define VIMSCAN_CARRY_ZOH_KSUB 8
+#endif
+#ifndef VIMSCAN_CARRY_ZOH_MIN_BLOCKS
+#define VIMSCAN_CARRY_ZOH_MIN_BLOCKS 4
+#endif
 constexpr int kSub = VIMSCAN_KSUB;   // tokens whose independent work is formed ahead of the recurrence
 constexpr int kMinBlocks = VIMSCAN_MIN_BLOCKS;   // resident CTAs per SM the register budget targets
 constexpr int kCarrySub = VIMSCAN_CARRY_KSUB;          // the same for the chunk-summary kernel
 constexpr int kCarryMinBlocks = VIMSCAN_CARRY_MIN_BLOCKS;
+constexpr int kCarryZohSub = VIMSCAN_CARRY_ZOH_KSUB;   // the same two with the exact hold
+constexpr int kCarryZohMinBlocks = VIMSCAN_CARRY_ZOH_MIN_BLOCKS;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ----------------------------------------------------------------------------
@@ -478,6 +486,7 @@ template <typename T, int N, bool FAST, bool DESC, bool CONV, bool ZOH>
 __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, const ChannelParams<N> &prm,
                                            int dl, const T *su, const T *sd, const float *sB) {
     constexpr int NP = N / 2;
+    constexpr int kCarrySub = ZOH ? kCarryZohSub : vimscan::kCarrySub;
 #pragma unroll 1
     for (int sub = 0; sub < kTile / kCarrySub; ++sub) {
         // duv: Delta u (first-order Bbar); with the exact hold, the structured path
@@ -552,9 +561,9 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
     }
 }
 
-// (the exact hold needs more registers than 6 CTAs per SM leave: 4 CTAs per SM)
+// (the exact hold needs more registers per thread, so fewer CTAs per SM)
 template <typename T, int N, bool VEC_BC, bool CONV, bool ZOH>
-__global__ void __launch_bounds__(kThreads, ZOH ? kMinBlocks : kCarryMinBlocks) pair_carry(PairArgs p) {
+__global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMinBlocks) pair_carry(PairArgs p) {
     using S = Stage<T, N, CONV>;
     constexpr int NP = N / 2;
     constexpr int kSlot = S::kSlotBytes;
