@@ -183,6 +183,36 @@ vim_status vmamba_cross_scan4_events(const void *u, const void *delta, const voi
                                      cudaEvent_t *events);
 
 /*
+ * Derivative of vim_scan_bidir (first-order Bbar) for a loss with derivative `dout`
+ * with respect to y: the chain rule through the gate and each direction's recurrence
+ * in reverse visiting order (the adjoint g of h obeys g_t = C_t dy_t + Abar_(t+1)
+ * g_(t+1), dy = dout * silu(z)); training through the scan is what the pages'
+ * "efficient training" of the selective scan refers to.
+ *
+ *   u, delta, z, B, C, bc_dir_stride, A, D, delta_bias : the forward call's inputs.
+ *   dout   : [batch, L, d_inner] (dt).
+ *   du, ddelta, dz : [batch, L, d_inner] (dt), written.  ddelta is with respect to the
+ *            raw delta (through softplus).  dz must be NULL exactly when z is NULL.
+ *   dB, dC : fp32, shaped like B and C: [batch, L, d_state], and with bc_dir_stride > 0
+ *            the backward direction's part bc_dir_stride elements further on (at least
+ *            bc_dir_stride + batch*L*d_state floats); with 0 both directions' terms
+ *            are summed into one.
+ *   dA [2, d_inner, d_state], dD [2, d_inner], ddelta_bias [2, d_inner] : fp32, written.
+ *   workspace : vim_scan_bwd_workspace_bytes(batch, L, d_inner, d_state,
+ *            bc_dir_stride > 0) bytes, 256-byte aligned.
+ * The same size limits as vim_scan_bidir.  Results are deterministic (no floating
+ * point atomics in global memory).
+ */
+vim_status vim_scan_bidir_bwd(const void *u, const void *delta, const void *z,
+                              const void *B, const void *C, int64_t bc_dir_stride,
+                              const float *A, const float *D, const float *delta_bias,
+                              const void *dout, void *du, void *ddelta, void *dz,
+                              float *dB, float *dC, float *dA, float *dD, float *ddelta_bias,
+                              int batch, int L, int d_inner, int d_state, vim_dtype dt,
+                              void *workspace, size_t workspace_bytes, cudaStream_t stream);
+size_t vim_scan_bwd_workspace_bytes(int batch, int L, int d_inner, int d_state, int separate_bc);
+
+/*
  * Options of the _ex entry points, or-ed into `flags` (unknown bits return
  * VIM_ERR_INVALID_ARG).
  *

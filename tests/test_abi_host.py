@@ -36,6 +36,7 @@ def test_header_declares_the_boundary():
     assert set(names) == {"vim_scan_bidir", "vmamba_cross_scan4", "cross_merge4",
                           "vim_scan_bidir_events", "vmamba_cross_scan4_events", "vim_scan_bidir_noalloc", "vim_scan_bidir_conv", "vim_scan_bidir_conv_events",
                           "vim_scan_bidir_ex", "vmamba_cross_scan4_ex",
+                          "vim_scan_bidir_bwd", "vim_scan_bwd_workspace_bytes",
                           "vim_scan_workspace_bytes", "vim_status_string"}, names
 
 
@@ -104,6 +105,39 @@ def test_bidir_rejects(vs):
     assert bidir(vs, L=4097, ws=None) == vs.VIM_ERR_WORKSPACE
     assert bidir(vs, L=4097, ws=FAKE, ws_bytes=16) == vs.VIM_ERR_WORKSPACE
     assert bidir(vs, L=4097, ws=FAKE + 16, ws_bytes=1 << 40) == vs.VIM_ERR_WORKSPACE
+
+
+def bwd(vs, **kw):
+    """vim_scan_bidir_bwd on fake device addresses; every case below fails a host check."""
+    a = dict(u=FAKE, delta=FAKE, z=FAKE, B=FAKE, C=FAKE, stride=0, A=FAKE, D=FAKE, bias=FAKE, dout=FAKE,
+             du=FAKE, ddelta=FAKE, dz=FAKE, dB=FAKE, dC=FAKE, dA=FAKE, dD=FAKE, dbias=FAKE,
+             batch=2, L=100, Di=64, N=16, dt=vs.VIM_BF16, ws=FAKE, ws_bytes=1 << 40)
+    a.update(kw)
+    return vs.lib.vim_scan_bidir_bwd(a["u"], a["delta"], a["z"], a["B"], a["C"], a["stride"], a["A"], a["D"],
+                                     a["bias"], a["dout"], a["du"], a["ddelta"], a["dz"], a["dB"], a["dC"],
+                                     a["dA"], a["dD"], a["dbias"], a["batch"], a["L"], a["Di"], a["N"],
+                                     a["dt"], a["ws"], a["ws_bytes"], None)
+
+
+def test_bwd_rejects(vs):
+    assert bwd(vs, dz=None) == vs.VIM_ERR_INVALID_ARG              # z given, dz missing
+    assert bwd(vs, z=None) == vs.VIM_ERR_INVALID_ARG               # dz given, z missing
+    assert bwd(vs, A=None) == vs.VIM_ERR_INVALID_ARG
+    assert bwd(vs, dA=FAKE + 2) == vs.VIM_ERR_INVALID_ARG
+    assert bwd(vs, u=FAKE + 8) == vs.VIM_ERR_INVALID_ARG
+    assert bwd(vs, dout=None) == vs.VIM_ERR_INVALID_ARG
+    assert bwd(vs, dB=FAKE + 2) == vs.VIM_ERR_INVALID_ARG
+    assert bwd(vs, stride=-3) == vs.VIM_ERR_INVALID_ARG
+    assert bwd(vs, N=3) == vs.VIM_ERR_UNSUPPORTED
+    assert bwd(vs, Di=12) == vs.VIM_ERR_UNSUPPORTED
+    assert bwd(vs, ws=None) == vs.VIM_ERR_WORKSPACE
+    assert bwd(vs, ws_bytes=64) == vs.VIM_ERR_WORKSPACE
+    assert bwd(vs, ws=FAKE + 16) == vs.VIM_ERR_WORKSPACE
+    # the workspace grows with the sequence and with separate B/C
+    small = vs.vim_scan_bwd_workspace_bytes(2, 100, 64, 16, False)
+    assert 0 < small < vs.vim_scan_bwd_workspace_bytes(2, 1000, 64, 16, False)
+    assert small < vs.vim_scan_bwd_workspace_bytes(2, 100, 64, 16, True)
+    assert vs.vim_scan_bwd_workspace_bytes(0, 100, 64, 16, False) == 0
 
 
 def test_size_zero_is_a_noop(vs):

@@ -1,0 +1,132 @@
+"""Parity of the scan's derivative (vim_scan_bidir_bwd, through the C ABI) with the
+fp64 oracle's reverse-mode derivative (itself pinned against finite differences).
+
+Error measure: normwise, max|g - r| / max|r|, per derivative.  Tolerances: the
+per-element derivatives du, d delta_raw and dz take the forward's (1e-5 for fp32
+I/O, 2e-2 for bf16 I/O, whose outputs are rounded to bf16); the fp32 sums over
+channels (dB, dC) and over tokens (dA, dD, d delta_bias) take 1e-4 on the small
+cases and 1e-3 at full size: they add up to batch*L terms of both signs in fp32, and
+a cancelling sum's rounding error is relative to its terms, not to the result.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from vision_mamba_selective_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+ELEM_TOL = {torch.float32: 1e-5, torch.bfloat16: 2e-2}
+SUM_TOL = 1e-4
+KEYS = [("du", "du"), ("ddelta", "ddelta"), ("dz", "dz"), ("dB", "dB"), ("dC", "dC"), ("dA", "dA"),
+        ("dD", "dD"), ("ddelta_bias", "dbias")]
+
+
+@pytest.fixture(scope="module")
+def vs():
+    from vision_mamba_selective_b200 import vimscan
+
+    return vimscan
+
+
+def normwise(y, ref):
+    y = y.detach().to("cpu", torch.float64).numpy()
+    den = np.max(np.abs(ref))
+    return float(np.max(np.abs(y - ref)) / den) if den > 0 else float(np.max(np.abs(y - ref)))
+
+
+def inputs(batch, L, Di, N, dtype, seed, *, separate_bc=False, generic_A=False):
+    g = torch.Generator().manual_seed(seed)
+    r = lambda *s, std=1.0: torch.randn(s, generator=g) * std
+    u, dr, z, dout = r(batch, L, Di), r(batch, L, Di, std=0.5), r(batch, L, Di), r(batch, L, Di)
+    nb = 2 if separate_bc else 1
+    B, C = r(nb, batch, L, N), r(nb, batch, L, N)
+    if not separate_bc:
+        B, C = B[0], C[0]
+    if generic_A:
+        A = -(0.05 + 3 * torch.rand((2, Di, N), generator=g))
+    else:
+        A = -torch.arange(1, N + 1, dtype=torch.float32).repeat(2, Di, 1)
+    D = r(2, Di)
+    s = torch.exp(np.log(1e-3) + (np.log(1e-1) - np.log(1e-3)) * torch.rand((2, Di), generator=g, dtype=torch.float64))
+    bias = torch.log(torch.expm1(s)).float()
+    t = lambda x: x.to(dtype).contiguous()
+    return dict(u=t(u), delta=t(dr), z=t(z), dout=t(dout), B=t(B), C=t(C), A=A.contiguous(), D=D.contiguous(),
+                bias=bias.contiguous(), stride=batch * L * N if separate_bc else 0)
+
+
+def run(vs, x, gate=True):
+    c = lambda k: x[k].cuda()
+    out = vs.vim_scan_bidir_bwd(c("u"), c("delta"), c("z") if gate else None, c("B"), c("C"), c("A"), c("D"),
+                                c("bias"), c("dout"), bc_dir_stride=x["stride"])
+    torch.cuda.synchronize()
+    return out
+
+
+def ref(x, gate=True):
+    return oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"] if gate else None, x["B"], x["C"], x["A"], x["D"],
+                                x["bias"], x["dout"], bc_dir_stride=x["stride"])
+
+
+def check_all(name, got, want, dtype, sum_tol=SUM_TOL):
+    errs = {}
+    for k_got, k_ref in KEYS:
+        if want[k_ref] is None:
+            assert got[k_got] is None
+            continue
+        g = got[k_got]
+        assert torch.isfinite(g.float()).all(), (name, k_got)
+        errs[k_got] = normwise(g, want[k_ref])
+        tol = ELEM_TOL[dtype] if k_got in ("du", "ddelta", "dz") else sum_tol
+        assert errs[k_got] <= tol, f"{name}: {k_got} normwise error {errs[k_got]:.3e} > {tol:.0e} ({errs})"
+    return errs
+
+
+CASES = [
+    # batch, L, Di, N, dtype, separate_bc, generic_A, gate
+    (1, 1, 16, 16, torch.float32, False, False, True),
+    (1, 5, 16, 4, torch.float32, True, False, True),
+    (2, 31, 24, 16, torch.float32, False, False, True),      # partial channel block
+    (1, 32, 16, 8, torch.float32, False, True, True),        # one whole chunk
+    (2, 33, 64, 16, torch.float32, True, False, True),       # 2 chunks, the last 1 token
+    (1, 100, 40, 2, torch.float32, False, False, False),
+    (2, 197, 64, 16, torch.bfloat16, False, False, True),
+    (1, 300, 72, 8, torch.bfloat16, True, True, True),
+    (2, 300, 200, 16, torch.float32, False, False, True),
+    (1, 1000, 64, 16, torch.float32, True, False, True),
+    (1, 777, 48, 4, torch.bfloat16, False, True, False),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"b{c[0]}_L{c[1]}_D{c[2]}_N{c[3]}_{str(c[4])[6:]}"
+                         f"{'_sepBC' if c[5] else ''}{'_genA' if c[6] else ''}{'' if c[7] else '_nogate'}")
+def test_bwd_small(vs, case):
+    batch, L, Di, N, dtype, sep, gen, gate = case
+    x = inputs(batch, L, Di, N, dtype, seed=L * 3 + Di, separate_bc=sep, generic_A=gen)
+    check_all(f"bwd_{case}", run(vs, x, gate), ref(x, gate), dtype)
+
+
+def test_bwd_deterministic(vs):
+    x = inputs(2, 500, 64, 16, torch.float32, seed=8)
+    a, b = run(vs, x), run(vs, x)
+    for k, _ in KEYS:
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_bwd_full_size(vs):
+    """The 1024 px Vim-Ti workload (bf16, batch 8, L 4097, d_inner 384) against the
+    oracle on every output, with dout drawn like the inputs."""
+    w = wl.BY_NAME["vim_tiny_1024px_bf16"]
+    x = wl.make_inputs(w)
+    g = torch.Generator().manual_seed(777)
+    dout = torch.randn(x["u"].shape, generator=g).to(x["u"].dtype)
+    oracle.set_threads(max(1, len(os.sched_getaffinity(0))))
+    d = {k: v.cuda() for k, v in x.items()}
+    got = vs.vim_scan_bidir_bwd(d["u"], d["delta"], d["z"], d["B"], d["C"], d["A"], d["D"], d["delta_bias"],
+                                dout.cuda())
+    torch.cuda.synchronize()
+    want = oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], dout)
+    check_all("bwd_full", got, want, torch.bfloat16, sum_tol=1e-3)

@@ -1,0 +1,191 @@
+// bwd.cu -- host side of the derivative of the Vim two-direction scan:
+// vim_scan_bidir_bwd and its workspace query (declared in include/vimscan.h).
+#include "vimscan.h"
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "bwd_kernels.cuh"
+#include "launch.cuh"
+
+namespace vimscan {
+namespace {
+
+struct BwdPlan {
+    int G, nblk, nsets;
+    size_t off_hloc, off_ssum, off_gloc, off_gsum, off_dA, off_dD, off_db, off_dBp, off_dCp, off_tmp, total;
+};
+
+BwdPlan bwd_plan(int batch, int L, int Di, int N, int separate_bc) {
+    BwdPlan pl;
+    pl.G = (L + kBwdChunk - 1) / kBwdChunk;
+    pl.nblk = (Di + kBwdCh - 1) / kBwdCh;
+    pl.nsets = separate_bc ? 2 : 1;
+    const size_t units = (size_t)batch * pl.G * 2 * Di;      // (b, chunk, dir, channel)
+    const size_t cols = std::max((size_t)2 * Di * N, (size_t)2 * Di);
+    size_t o = 0;
+    auto take = [&](size_t bytes) { const size_t at = o; o += round_up(bytes); return at; };
+    pl.off_hloc = take(units * N * 4);
+    pl.off_ssum = take(units * 4);
+    pl.off_gloc = take(units * N * 4);
+    pl.off_gsum = take(units * 4);
+    pl.off_dA = take(units * N * 4);
+    pl.off_dD = take(units * 4);
+    pl.off_db = take(units * 4);
+    pl.off_dBp = take((size_t)pl.nsets * batch * L * pl.nblk * N * 4);
+    pl.off_dCp = take((size_t)pl.nsets * batch * L * pl.nblk * N * 4);
+    pl.off_tmp = take((size_t)kReduceParts * cols * 4);
+    pl.total = o;
+    return pl;
+}
+
+// column sums of rows x cols fp32 into out (two passes through tmp)
+vim_status reduce_cols(const float *src, float *tmp, float *out, int rows, int cols, cudaStream_t stream) {
+    const dim3 g1((cols + 255) / 256, kReduceParts);
+    bwd_reduce_cols1<<<g1, 256, 0, stream>>>(src, tmp, rows, cols);
+    if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+    bwd_reduce_cols2<<<(cols + 255) / 256, 256, 0, stream>>>(tmp, out, cols);
+    return cudaGetLastError() == cudaSuccess ? VIM_OK : VIM_ERR_CUDA;
+}
+
+template <typename T, int N>
+vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], float *dC_out[2], float *dA,
+                      float *dD, float *dbias, float *tmp, cudaStream_t stream) {
+    if (a.G > 1) {
+        // h entering each chunk: the forward scan's own summary kernels
+        const dim3 gf((a.Di + kDC - 1) / kDC, a.G, a.batch);
+        const size_t sc = 2 * (size_t)Stage<T, N, false>::kSlotBytes;
+        auto carry = pair_carry<T, N, false, false, false>;
+        if (cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sc) != cudaSuccess)
+            return VIM_ERR_CUDA;
+        carry<<<gf, kThreads, sc, stream>>>(fwd);
+        if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+        const int64_t units = (int64_t)a.batch * 2 * a.Di * N;
+        const dim3 gc((unsigned)((units + 255) / 256));
+        pair_combine<N><<<gc, 256, 0, stream>>>(fwd);
+        if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+        // adjoint entering each chunk from the side its direction visits later
+        adj_carry<T, N><<<dim3((a.Di + kAdjCh - 1) / kAdjCh, a.G, a.batch), 2 * kAdjCh, 0, stream>>>(a);
+        if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+        PairArgs adj = fwd;
+        adj.hloc = a.gloc;
+        adj.ssum = a.gsum;
+        adj.fold_reverse = 1;
+        pair_combine<N><<<gc, 256, 0, stream>>>(adj);
+        if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+    }
+    bwd_main<T, N><<<dim3(a.nblk, a.G, a.batch), BwdShape<N>::kThr, 0, stream>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+    const int sets = a.separate_bc ? 2 : 1;
+    const int rows = a.batch * a.L;
+    for (int k = 0; k < sets; ++k) {
+        const unsigned blocks = (unsigned)(((int64_t)rows * N + 255) / 256);
+        bwd_reduce_bc<N><<<blocks, 256, 0, stream>>>(a.dB_part[k], dB_out[k], rows, a.nblk);
+        bwd_reduce_bc<N><<<blocks, 256, 0, stream>>>(a.dC_part[k], dC_out[k], rows, a.nblk);
+        if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+    }
+    const int prow = a.batch * a.G;
+    if (reduce_cols(a.dA_part, tmp, dA, prow, 2 * a.Di * N, stream) != VIM_OK) return VIM_ERR_CUDA;
+    if (reduce_cols(a.dD_part, tmp, dD, prow, 2 * a.Di, stream) != VIM_OK) return VIM_ERR_CUDA;
+    return reduce_cols(a.dbias_part, tmp, dbias, prow, 2 * a.Di, stream);
+}
+
+template <typename T>
+vim_status launch_bwd_n(int N, const BwdArgs &a, const PairArgs &fwd, float *dB[2], float *dC[2], float *dA,
+                        float *dD, float *dbias, float *tmp, cudaStream_t stream) {
+    switch (N) {
+        case 2: return launch_bwd<T, 2>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream);
+        case 4: return launch_bwd<T, 4>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream);
+        case 8: return launch_bwd<T, 8>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream);
+        case 16: return launch_bwd<T, 16>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream);
+        default: return VIM_ERR_UNSUPPORTED;
+    }
+}
+
+bool aligned_to(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+}  // namespace vimscan
+
+using namespace vimscan;
+
+extern "C" {
+
+size_t vim_scan_bwd_workspace_bytes(int batch, int L, int d_inner, int d_state, int separate_bc) {
+    if (batch <= 0 || L <= 0 || d_inner <= 0 || d_state <= 0) return 0;
+    return bwd_plan(batch, L, d_inner, d_state, separate_bc).total;
+}
+
+vim_status vim_scan_bidir_bwd(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                              int64_t bc_dir_stride, const float *A, const float *D, const float *delta_bias,
+                              const void *dout, void *du, void *ddelta, void *dz, float *dB, float *dC,
+                              float *dA, float *dD, float *ddelta_bias, int batch, int L, int d_inner,
+                              int d_state, vim_dtype dt, void *workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
+    vim_status st = check_common(batch, L, d_inner, d_state, dt);
+    if (st != VIM_OK) return st;
+    if (bc_dir_stride < 0) return VIM_ERR_INVALID_ARG;
+    if ((z == nullptr) != (dz == nullptr)) return VIM_ERR_INVALID_ARG;
+    if (!A || !D || !delta_bias || !dA || !dD || !ddelta_bias) return VIM_ERR_INVALID_ARG;
+    if (!aligned_to(A, 4) || !aligned_to(D, 4) || !aligned_to(delta_bias, 4) || !aligned_to(dA, 4) ||
+        !aligned_to(dD, 4) || !aligned_to(ddelta_bias, 4))
+        return VIM_ERR_INVALID_ARG;
+    const size_t es = elem_size(dt);
+    if (batch == 0 || L == 0 || d_inner == 0) {
+        // no tokens: the parameter derivatives are zero
+        if (cudaMemsetAsync(dA, 0, sizeof(float) * 2 * (size_t)d_inner * d_state, stream) != cudaSuccess ||
+            cudaMemsetAsync(dD, 0, sizeof(float) * 2 * (size_t)d_inner, stream) != cudaSuccess ||
+            cudaMemsetAsync(ddelta_bias, 0, sizeof(float) * 2 * (size_t)d_inner, stream) != cudaSuccess)
+            return VIM_ERR_CUDA;
+        return VIM_OK;
+    }
+    if (!u || !delta || !B || !C || !dout || !du || !ddelta || !dB || !dC) return VIM_ERR_INVALID_ARG;
+    if (!aligned16(u) || !aligned16(delta) || !aligned_to(B, es) || !aligned_to(C, es) || !aligned_to(dout, es) ||
+        !aligned_to(du, es) || !aligned_to(ddelta, es) || (z && !aligned_to(z, es)) || (dz && !aligned_to(dz, es)) ||
+        !aligned_to(dB, 4) || !aligned_to(dC, 4))
+        return VIM_ERR_INVALID_ARG;
+    const int separate = bc_dir_stride > 0 ? 1 : 0;
+    const BwdPlan pl = bwd_plan(batch, L, d_inner, d_state, separate);
+    if (!workspace || workspace_bytes < pl.total || !aligned_to(workspace, kAlign)) return VIM_ERR_WORKSPACE;
+    char *ws = static_cast<char *>(workspace);
+
+    BwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.u = u; a.delta = delta; a.z = z; a.dout = dout;
+    a.B[0] = B; a.C[0] = C;
+    a.B[1] = static_cast<const char *>(B) + bc_dir_stride * (int64_t)es;
+    a.C[1] = static_cast<const char *>(C) + bc_dir_stride * (int64_t)es;
+    a.A = A; a.D = D; a.bias = delta_bias;
+    a.du = du; a.ddelta = ddelta; a.dz = dz;
+    const size_t set_elems = (size_t)batch * L * pl.nblk * d_state;
+    a.dB_part[0] = reinterpret_cast<float *>(ws + pl.off_dBp);
+    a.dC_part[0] = reinterpret_cast<float *>(ws + pl.off_dCp);
+    a.dB_part[1] = separate ? a.dB_part[0] + set_elems : a.dB_part[0];
+    a.dC_part[1] = separate ? a.dC_part[0] + set_elems : a.dC_part[0];
+    a.dA_part = reinterpret_cast<float *>(ws + pl.off_dA);
+    a.dD_part = reinterpret_cast<float *>(ws + pl.off_dD);
+    a.dbias_part = reinterpret_cast<float *>(ws + pl.off_db);
+    a.hin = reinterpret_cast<const float *>(ws + pl.off_hloc);
+    a.gloc = reinterpret_cast<float *>(ws + pl.off_gloc);
+    a.gsum = reinterpret_cast<float *>(ws + pl.off_gsum);
+    a.batch = batch; a.L = L; a.Di = d_inner; a.G = pl.G; a.nblk = pl.nblk;
+    a.separate_bc = separate;
+
+    PairArgs f;
+    std::memset(&f, 0, sizeof(f));
+    f.u = u; f.delta = delta;
+    f.B[0] = a.B[0]; f.B[1] = a.B[1]; f.C[0] = a.C[0]; f.C[1] = a.C[1];
+    f.A = A; f.D = D; f.bias = delta_bias;
+    f.hloc = reinterpret_cast<float *>(ws + pl.off_hloc);
+    f.ssum = reinterpret_cast<float *>(ws + pl.off_ssum);
+    f.batch = batch; f.L = L; f.Di = d_inner; f.H = 1; f.W = L; f.order = 0;
+    f.chunk = kBwdChunk; f.G = pl.G;
+
+    float *dBo[2] = {dB, dB + bc_dir_stride}, *dCo[2] = {dC, dC + bc_dir_stride};
+    float *tmp = reinterpret_cast<float *>(ws + pl.off_tmp);
+    return dt == VIM_F32 ? launch_bwd_n<float>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream)
+                         : launch_bwd_n<__nv_bfloat16>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream);
+}
+
+}  // extern "C"

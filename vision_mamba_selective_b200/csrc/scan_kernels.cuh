@@ -232,6 +232,7 @@ struct PairArgs {
     int order;                      // 0: position = step; 1: column-major on H x W
     int chunk, G;                   // tokens per chunk (multiple of kTile), chunks
     int zoh;                        // exact zero-order-hold Bbar instead of Delta B
+    int fold_reverse;               // pair_combine folds each direction against its order
 };
 
 // position visited at step t of the forward direction
@@ -529,20 +530,20 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
                 }
             } else if constexpr (FAST) {
                 // exact hold: state n gets w^(n+1) kappa u S_n B_n / (n+1) (B is staged
-                // divided by n+1), S_n = 1 + q + ... + q^n.  T_n = w^(n+1) kappa u S_n
-                // runs two states at a time: T_(n+2) = w^2 T_n + Q_n with
+                // divided by n+1), S_n = 1 + q + ... + q^n.  W_n = w^(n+1) kappa u S_n
+                // runs two states at a time: W_(n+2) = w^2 W_n + Q_n with
                 // Q_n = w^2 kappa u (1+q) (wq)^(n+1).
                 const float w = ex2(prm.A0 * Sv[k]);
                 const float q = qv[k], ku = duv[k];
                 const float c = ku * (1.0f + q);
                 const float ww = w * w, wq = w * q, wqwq = wq * wq;
-                float2 T = f2(ku * w, c * ww);
+                float2 Wn = f2(ku * w, c * ww);
                 float2 Q = f2(ww * c * wq, ww * c * wqwq);
                 const float2 w2 = f2(ww, ww), wq2 = f2(wqwq, wqwq);
 #pragma unroll
                 for (int j = 0; j < NP; ++j) {
-                    H[j] = fma2(T, Bv[j], H[j]);
-                    T = fma2(w2, T, Q);
+                    H[j] = fma2(Wn, Bv[j], H[j]);
+                    Wn = fma2(w2, Wn, Q);
                     Q = mul2(Q, wq2);
                 }
             } else {
@@ -634,7 +635,9 @@ __global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMin
 // replaced by the state entering chunk c in that direction's visiting order:
 // H_in(next) = exp(A_n * Ssum(c)) * H_in(c) + H_loc(c).  Loads run 16 chunks ahead.
 // The last chunk's summary in each direction was never formed: it is read and fed
-// into h after the last carry has been stored, which is harmless.
+// into h after the last carry has been stored, which is harmless.  With fold_reverse
+// each direction is folded from its last chunk to its first (the adjoint of the
+// scan, whose summaries come from adj_carry).
 template <int N>
 __global__ void __launch_bounds__(256) pair_combine(PairArgs p) {
     constexpr int kAhead = 16;
@@ -647,10 +650,11 @@ __global__ void __launch_bounds__(256) pair_combine(PairArgs p) {
     const int dir = rem / (p.Di * N);
     const float A2n = p.A[rem] * kLog2e;                     // A is [2][Di][N]: same index
     // hloc[b][c][dir][d][n] and ssum[b][c][dir][d]: chunk c+1 lies per_b (per_b / N) further
-    const int c0 = dir ? p.G - 1 : 0;
+    const bool desc = (dir != 0) != (p.fold_reverse != 0);
+    const int c0 = desc ? p.G - 1 : 0;
     float *hl = p.hloc + ((size_t)b * p.G + c0) * per_b + rem;
     const float *ss = p.ssum + ((size_t)b * p.G + c0) * (per_b / N) + rem / N;
-    const int hs = dir ? -per_b : per_b, sstep = dir ? -(per_b / N) : per_b / N;
+    const int hs = desc ? -per_b : per_b, sstep = desc ? -(per_b / N) : per_b / N;
     float h = 0.0f;
     for (int i0 = 0; i0 < p.G; i0 += kAhead) {
         const int cnt = min(kAhead, p.G - i0);

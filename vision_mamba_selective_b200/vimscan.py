@@ -49,6 +49,11 @@ lib.vmamba_cross_scan4_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _v
                                       _i, _i, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp]
 lib.vmamba_cross_scan4_ex.restype = _i
 VIM_FLAG_ZOH_EXACT = 1
+lib.vim_scan_bidir_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                   _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _vp]
+lib.vim_scan_bidir_bwd.restype = _i
+lib.vim_scan_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+lib.vim_scan_bwd_workspace_bytes.restype = _sz
 lib.vim_scan_bidir_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
                                        _i, _i, _i, _i, _i, _vp]
 lib.vim_scan_bidir_noalloc.restype = _i
@@ -176,6 +181,44 @@ def vim_scan_bidir_conv(x, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, *, 
     """
     return _bidir("vim_scan_bidir_conv", x, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, y,
                   bc_dir_stride, workspace, stream, events, zoh)
+
+
+def vim_scan_bwd_workspace_bytes(batch, L, d_inner, d_state, separate_bc):
+    return int(lib.vim_scan_bwd_workspace_bytes(batch, L, d_inner, d_state, int(bool(separate_bc))))
+
+
+def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stride=0, workspace=None,
+                       stream=None):
+    """Derivatives of vim_scan_bidir (first-order Bbar) for a loss whose derivative
+    with respect to y is ``dout``; see include/vimscan.h.
+
+    Returns a dict: du, ddelta (w.r.t. the raw delta), dz (None without z), in the
+    input dtype; dB and dC (fp32, shaped like B and C); dA [2, d_inner, d_state], dD
+    and ddelta_bias [2, d_inner] (fp32).
+    """
+    batch, L, Di = u.shape
+    N = B.shape[-1]
+    dt = _dtype_code(u)
+    dev = u.device
+    out = dict(du=torch.empty_like(u), ddelta=torch.empty_like(u),
+               dz=torch.empty_like(u) if z is not None else None,
+               dB=torch.zeros(B.shape, dtype=torch.float32, device=dev),
+               dC=torch.zeros(C.shape, dtype=torch.float32, device=dev),
+               dA=torch.empty((2, Di, N), dtype=torch.float32, device=dev),
+               dD=torch.empty((2, Di), dtype=torch.float32, device=dev),
+               ddelta_bias=torch.empty((2, Di), dtype=torch.float32, device=dev))
+    ws, ws_bytes = _workspace(vim_scan_bwd_workspace_bytes(batch, L, Di, N, bc_dir_stride > 0), workspace, dev)
+    st = lib.vim_scan_bidir_bwd(
+        _ptr(u, name="u"), _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
+        _ptr(B, dtype=u.dtype, name="B"), _ptr(C, dtype=u.dtype, name="C"), int(bc_dir_stride),
+        _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
+        _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(dout, dtype=u.dtype, name="dout"),
+        _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dz"]), _ptr(out["dB"]), _ptr(out["dC"]),
+        _ptr(out["dA"]), _ptr(out["dD"]), _ptr(out["ddelta_bias"]),
+        batch, L, Di, N, dt, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
+    if st != VIM_OK:
+        raise VimScanError(st, "vim_scan_bidir_bwd")
+    return out
 
 
 def vim_scan_bidir_noalloc(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride=0, stream=None):
