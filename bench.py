@@ -2,7 +2,7 @@
 """Throughput of the bidirectional selective scan (S6) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
-                    [--conv] [--zoh]
+                    [--conv] [--zoh] [--bwd]
 
 One step is one pass of the whole scan -- softplus Delta, the forward and backward
 recurrences, readout, D skip, the merge of the directions and the silu(z) gate --
@@ -11,7 +11,8 @@ is the 1024 px Vim-Tiny scan (batch 8, L = 4097, d_inner 384, d_state 16, bf16 I
 fp32 state).  Inputs are seeded synthetic tensors shaped like the pages' workloads.
 --conv times the same scan with the pathways' kernel-3 convolution + SiLU fused in
 front (the input tensor is then x, the convolutions' input); --zoh times it with the
-exact zero-order-hold Bbar = (exp(Delta A) - 1) / A * B in place of Delta B.
+exact zero-order-hold Bbar = (exp(Delta A) - 1) / A * B in place of Delta B; --bwd
+times the derivative of the scan (every input's gradient from a seeded dout).
 
 Multi-GPU (torchrun, one process per GPU): the batch items are independent, so every
 rank runs the same workload on its own inputs with no collective on the data path
@@ -54,6 +55,8 @@ def parse():
                     help="Vim workloads: time the scan with the fused kernel-3 convolution + SiLU front")
     ap.add_argument("--zoh", action="store_true",
                     help="time the scan with the exact zero-order-hold Bbar instead of Delta B")
+    ap.add_argument("--bwd", action="store_true",
+                    help="Vim workloads: time the scan's derivative (vim_scan_bidir_bwd) instead")
     return ap.parse_args()
 
 
@@ -85,6 +88,24 @@ def profiled_traffic(w):
     if not m or not f or f.group(1) != fp:
         return None
     return int(m.group(1))
+
+
+def algorithmic_bwd(w):
+    """Algorithmic bytes and FP32 lane-ops of one derivative step (Vim, shared B/C).
+
+    Bytes: reads of u, delta_raw, z, dout and writes of du, d delta_raw, dz per
+    token-channel; B, C read and dB, dC (fp32) written per token; parameters and
+    their derivatives once.  Ops: 11 FP32 lane-ops per state per direction per
+    token-channel -- the forward state update (decay multiply, Delta*B*u, FMA), the
+    readout for dz, the dC term, and in the adjoint sweep the C*dy update, the decay
+    multiply, the h_(t-1) product, the dA, A- and B-weighted sums and the dB term.
+    """
+    el = 4 if w.dtype == "f32" else 2
+    bc = 2 * w.batch * w.tokens * w.d_state * (el + 4)
+    params = 2 * w.directions * w.channels * (w.d_state + 2) * 4
+    nbytes = 7 * w.tok_ch * el + bc + params
+    ops = 11 * w.d_state * w.directions * w.tok_ch
+    return nbytes, ops
 
 
 def algorithmic(w, conv=False):
@@ -178,7 +199,9 @@ def run_oracle(w, x, threads, zoh=False):
 
     oracle.set_threads(threads)
     t = time.perf_counter()
-    if "conv_w" in x:
+    if "dout" in x:
+        oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], x["dout"])
+    elif "conv_w" in x:
         oracle.vim_bidir_conv(x["u"], x["conv_w"], x["conv_b"], x["delta"], x["z"], x["B"], x["C"], x["A"],
                               x["D"], x["delta_bias"], zoh=zoh)
     elif w.kind == "vim":
@@ -189,7 +212,15 @@ def run_oracle(w, x, threads, zoh=False):
     return time.perf_counter() - t
 
 
-def oracle_sample(w, target_s, conv=False):
+def bwd_dout(w, seed):
+    """dout for the derivative runs: drawn like z, in the workload's dtype."""
+    import torch
+
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn((w.batch, w.tokens, w.channels), generator=g).to(w.torch_dtype()).contiguous()
+
+
+def oracle_sample(w, target_s, conv=False, bwd=False):
     """A bounded sample of the workload for the oracle: its first batch items and
     first channels at the full sequence length, sized for about ``target_s`` seconds
     of fp64 work on the host cores (calibrated on a small run)."""
@@ -197,6 +228,8 @@ def oracle_sample(w, target_s, conv=False):
 
     cores = cpu_cores()
     full = wl.make_inputs(w)
+    if bwd:
+        full["dout"] = bwd_dout(w, w.seed + 2)
     if conv:
         full["conv_w"], full["conv_b"] = conv_params(w, w.seed + 1)
     step = 8
@@ -204,7 +237,7 @@ def oracle_sample(w, target_s, conv=False):
     def cut(b, c):
         x = {}
         for k, v in full.items():
-            if k in ("u", "delta", "z"):
+            if k in ("u", "delta", "z", "dout"):
                 x[k] = v[:b, ..., :c].contiguous()
             elif k in ("B", "C"):
                 x[k] = (v[:b] if w.kind == "vim" else v[:, :b]).contiguous()
@@ -238,7 +271,7 @@ def reference_arm(args, w):
     if rank != 0:
         return
     per_step = min(2.0, 150.0 / max(1, args.steps + args.warmup))
-    s, x, cores = oracle_sample(w, per_step, conv=args.conv)
+    s, x, cores = oracle_sample(w, per_step, conv=args.conv, bwd=args.bwd)
     for _ in range(args.warmup):
         run_oracle(s, x, cores, args.zoh)
     times = [run_oracle(s, x, cores, args.zoh) for _ in range(args.steps)]
@@ -261,7 +294,8 @@ def reference_arm(args, w):
 
 
 def workload_name(w, args):
-    return w.name + ("+conv_front" if args.conv else "") + ("+zoh_exact" if args.zoh else "")
+    return (w.name + ("+conv_front" if args.conv else "") + ("+zoh_exact" if args.zoh else "")
+            + ("+derivative" if args.bwd else ""))
 
 
 def main():
@@ -269,8 +303,10 @@ def main():
     from vision_mamba_selective_b200 import workloads as wl
 
     w = wl.BY_NAME[args.workload]
-    if args.conv and w.kind != "vim":
-        raise SystemExit("--conv applies to the Vim workloads only")
+    if (args.conv or args.bwd) and w.kind != "vim":
+        raise SystemExit("--conv and --bwd apply to the Vim workloads only")
+    if args.bwd and (args.conv or args.zoh):
+        raise SystemExit("--bwd covers the plain scan (no --conv, no --zoh)")
     if args.impl == "reference":
         reference_arm(args, w)
         return
@@ -291,19 +327,31 @@ def main():
     # ---- inputs: rank-specific seed; enough rotating copies to exceed L2 ---------
     host = wl.make_inputs(w, seed=replicas.rank_seed(w.seed, rank))
     act_keys = ["u", "delta", "z", "B", "C"]
-    set_bytes = sum(host[k].numel() * host[k].element_size() for k in act_keys) + \
-        w.tok_ch * (4 if w.dtype == "f32" else 2)
+    el = 4 if w.dtype == "f32" else 2
+    out_bytes = w.tok_ch * el
+    if args.bwd:
+        host["dout"] = bwd_dout(w, replicas.rank_seed(w.seed + 2, rank))
+        act_keys.append("dout")
+        out_bytes = 3 * w.tok_ch * el + 2 * w.batch * w.tokens * w.d_state * 4
+    set_bytes = sum(host[k].numel() * host[k].element_size() for k in act_keys) + out_bytes
     nsets = max(2, math.ceil(2.2 * L2_BYTES / set_bytes))
     params = {k: host[k].to(dev) for k in ("A", "D", "delta_bias")}
     sets = []
     for _ in range(nsets):
         s = {k: host[k].to(dev) for k in act_keys}
         s["y"] = torch.empty_like(s["u"])
+        if args.bwd:
+            f32 = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
+            s["out"] = dict(du=torch.empty_like(s["u"]), ddelta=torch.empty_like(s["u"]), dz=torch.empty_like(s["u"]),
+                            dB=f32(*s["B"].shape), dC=f32(*s["C"].shape), dA=f32(2, w.channels, w.d_state),
+                            dD=f32(2, w.channels), ddelta_bias=f32(2, w.channels))
         sets.append(s)
     if w.kind == "vim":
         ws_bytes = vs.vim_scan_workspace_bytes(0, w.batch, w.L, 0, w.channels, w.d_state)
     else:
         ws_bytes = vs.vim_scan_workspace_bytes(1, w.batch, w.H, w.W, w.channels, w.d_state)
+    if args.bwd:
+        ws_bytes = vs.vim_scan_bwd_workspace_bytes(w.batch, w.L, w.channels, w.d_state, False)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     fn = vs.vim_scan_bidir if w.kind == "vim" else vs.vmamba_cross_scan4
     if args.conv:
@@ -312,6 +360,10 @@ def main():
 
     def step(i, events=None):
         s = sets[i % nsets]
+        if args.bwd:
+            vs.vim_scan_bidir_bwd(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"],
+                                  params["delta_bias"], s["dout"], workspace=ws, out=s["out"], events=events)
+            return
         if args.conv:
             # u holds x, the pathways' common input in front of the convolutions
             vs.vim_scan_bidir_conv(s["u"], params["conv_w"], params["conv_b"], s["delta"], s["z"], s["B"],
@@ -348,33 +400,49 @@ def main():
     # ---- per-kernel times (same launches plus event records), after the timed region
     kernels_per_pair = 3
     pairs = 1 if w.kind == "vim" else 2
-    nev = 1 + kernels_per_pair * pairs
+    nev = 4 if args.bwd else 1 + kernels_per_pair * pairs
     prof_steps = min(args.steps, 200)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(prof_steps)]
     for i in range(prof_steps):
         step(i, events=evs[i])
     torch.cuda.synchronize()
-    names = ["pair_carry", "pair_combine", "pair_main"]
     per_kernel = {}
-    for p in range(pairs):
-        for k in range(kernels_per_pair):
-            a = 1 + 3 * p + k
+    if args.bwd:
+        for a, name in enumerate(["summaries", "bwd_main", "reductions"], start=1):
             t = [evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(prof_steps)]
-            per_kernel[f"{names[k]}[{p}]" if pairs > 1 else names[k]] = sum(t) / len(t)
-    # sequences longer than one chunk (256 tokens) take carry, combine and main
-    launches_per_step = pairs * (3 if w.tokens > 256 else 1)
+            per_kernel[name] = sum(t) / len(t)
+        # pair_carry, pair_combine, adj_carry, pair_combine (more than one chunk of
+        # 32 tokens), bwd_main, two dB/dC reductions, three two-pass column sums
+        launches_per_step = (4 if w.tokens > 32 else 0) + 1 + 2 + 6
+    else:
+        names = ["pair_carry", "pair_combine", "pair_main"]
+        for p in range(pairs):
+            for k in range(kernels_per_pair):
+                a = 1 + 3 * p + k
+                t = [evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(prof_steps)]
+                per_kernel[f"{names[k]}[{p}]" if pairs > 1 else names[k]] = sum(t) / len(t)
+        # sequences longer than one chunk (256 tokens) take carry, combine and main
+        launches_per_step = pairs * (3 if w.tokens > 256 else 1)
 
     # ---- end to end: pinned host inputs -> device -> scan -> host result ---------
     pinned = {k: host[k].pin_memory() for k in act_keys}
-    y_host = torch.empty(sets[0]["y"].shape, dtype=sets[0]["y"].dtype).pin_memory()
+    if args.bwd:
+        res_dev = [sets[0]["out"][k] for k in ("du", "ddelta", "dz", "dB", "dC")]
+    else:
+        res_dev = [sets[0]["y"]]
+    res_host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in res_dev]
     h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in act_keys)
-    d2h = y_host.numel() * y_host.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in res_host)
+
+    def fetch():
+        for hst, dv in zip(res_host, res_dev):
+            hst.copy_(dv, non_blocking=True)
     e2e_steps = min(args.steps, 50)
     for _ in range(2):
         for k in act_keys:
             sets[0][k].copy_(pinned[k], non_blocking=True)
         step(0)
-        y_host.copy_(sets[0]["y"], non_blocking=True)
+        fetch()
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -383,7 +451,7 @@ def main():
         for k in act_keys:
             sets[0][k].copy_(pinned[k], non_blocking=True)
         step(0)
-        y_host.copy_(sets[0]["y"], non_blocking=True)
+        fetch()
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
@@ -391,14 +459,16 @@ def main():
 
     # ---- roofline of the dominant kernel -----------------------------------------
     pk = peaks()
-    nbytes, ops = algorithmic(w, args.conv)
-    main_ms = sum(v for k, v in per_kernel.items() if k.startswith("pair_main"))
+    nbytes, ops = algorithmic_bwd(w) if args.bwd else algorithmic(w, args.conv)
+    main_name = "bwd_main" if args.bwd else "pair_main"
+    main_ms = sum(v for k, v in per_kernel.items() if k.startswith(main_name))
     clocks = clk.summary()
     peak_ops = SMS * FP32_LANES_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e12
     achieved_ops = ops / (main_ms * 1e-3) / 1e12
     roofline = {
-        "bound": "alu", "kernel": "pair_main", "achieved": achieved_ops, "peak": peak_ops,
-        "unit": "Tops/s", "frac": achieved_ops / peak_ops, "traffic": profiled_traffic(w),
+        "bound": "alu", "kernel": main_name, "achieved": achieved_ops, "peak": peak_ops,
+        "unit": "Tops/s", "frac": achieved_ops / peak_ops,
+        "traffic": None if (args.bwd or args.conv or args.zoh) else profiled_traffic(w),
         "algorithmic_bytes": nbytes,
         "ops_per_launch": ops, "ms_per_launch": main_ms,
         "peak_basis": f"{SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x {pk['sm_max_mhz']:.0f} MHz",
@@ -409,7 +479,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        s, x, cores = oracle_sample(w, 5.0, conv=args.conv)
+        s, x, cores = oracle_sample(w, 5.0, conv=args.conv, bwd=args.bwd)
         sec = run_oracle(s, x, cores, args.zoh)
         cpu = {"value": s.tok_ch / sec, "unit": "tok*ch/s", "cores": cores, "kind": "oracle",
                "sample": f"{s.batch} of {w.batch} batch items x {s.channels} of {w.channels} channels "

@@ -211,6 +211,17 @@ vim_status vim_scan_bidir_bwd(const void *u, const void *delta, const void *z,
                               int batch, int L, int d_inner, int d_state, vim_dtype dt,
                               void *workspace, size_t workspace_bytes, cudaStream_t stream);
 size_t vim_scan_bwd_workspace_bytes(int batch, int L, int d_inner, int d_state, int separate_bc);
+/* vim_scan_bidir_bwd plus 4 CUDA events (caller-created, or NULL for none) recorded
+ * before the chunk summaries, after them, after the main derivative kernel and at
+ * the end, for per-phase times. */
+vim_status vim_scan_bidir_bwd_events(const void *u, const void *delta, const void *z,
+                                     const void *B, const void *C, int64_t bc_dir_stride,
+                                     const float *A, const float *D, const float *delta_bias,
+                                     const void *dout, void *du, void *ddelta, void *dz,
+                                     float *dB, float *dC, float *dA, float *dD, float *ddelta_bias,
+                                     int batch, int L, int d_inner, int d_state, vim_dtype dt,
+                                     void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                                     cudaEvent_t *events);
 
 /*
  * Options of the _ex entry points, or-ed into `flags` (unknown bits return

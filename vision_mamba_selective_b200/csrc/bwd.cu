@@ -20,7 +20,8 @@ struct BwdPlan {
 BwdPlan bwd_plan(int batch, int L, int Di, int N, int separate_bc) {
     BwdPlan pl;
     pl.G = (L + kBwdChunk - 1) / kBwdChunk;
-    pl.nblk = (Di + kBwdCh - 1) / kBwdCh;
+    const int ch = N >= 8 ? BwdShape<16>::CH : BwdShape<4>::CH;   // channels per bwd_main CTA
+    pl.nblk = (Di + ch - 1) / ch;
     pl.nsets = separate_bc ? 2 : 1;
     const size_t units = (size_t)batch * pl.G * 2 * Di;      // (b, chunk, dir, channel)
     const size_t cols = std::max((size_t)2 * Di * N, (size_t)2 * Di);
@@ -49,14 +50,26 @@ vim_status reduce_cols(const float *src, float *tmp, float *out, int rows, int c
     return cudaGetLastError() == cudaSuccess ? VIM_OK : VIM_ERR_CUDA;
 }
 
+// events: null, or 4 events recorded before the summaries, after them, after bwd_main
+// and after the reductions
+inline bool rec(cudaEvent_t *ev, int i, cudaStream_t stream) {
+    return !ev || cudaEventRecord(ev[i], stream) == cudaSuccess;
+}
+
 template <typename T, int N>
 vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], float *dC_out[2], float *dA,
-                      float *dD, float *dbias, float *tmp, cudaStream_t stream) {
+                      float *dD, float *dbias, float *tmp, cudaStream_t stream, cudaEvent_t *ev) {
+    if (!rec(ev, 0, stream)) return VIM_ERR_CUDA;
     if (a.G > 1) {
         // h entering each chunk: the forward scan's own summary kernels
         const dim3 gf((a.Di + kDC - 1) / kDC, a.G, a.batch);
         const size_t sc = 2 * (size_t)Stage<T, N, false>::kSlotBytes;
         auto carry = pair_carry<T, N, false, false, false>;
+        if constexpr (bc_vectorizable<T, N>()) {
+            // B and C rows as 16-byte vectors when every base allows it
+            if (aligned16(fwd.B[0]) && aligned16(fwd.B[1]) && aligned16(fwd.C[0]) && aligned16(fwd.C[1]))
+                carry = pair_carry<T, N, true, false, false>;
+        }
         if (cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sc) != cudaSuccess)
             return VIM_ERR_CUDA;
         carry<<<gf, kThreads, sc, stream>>>(fwd);
@@ -75,8 +88,13 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
         pair_combine<N><<<gc, 256, 0, stream>>>(adj);
         if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     }
-    bwd_main<T, N><<<dim3(a.nblk, a.G, a.batch), BwdShape<N>::kThr, 0, stream>>>(a);
+    if (!rec(ev, 1, stream)) return VIM_ERR_CUDA;
+    constexpr size_t sm = BwdShape<N>::kSmemBytes;
+    if (cudaFuncSetAttribute(bwd_main<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
+        return VIM_ERR_CUDA;
+    bwd_main<T, N><<<dim3(a.nblk, a.G, a.batch), BwdShape<N>::kThr, sm, stream>>>(a);
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+    if (!rec(ev, 2, stream)) return VIM_ERR_CUDA;
     const int sets = a.separate_bc ? 2 : 1;
     const int rows = a.batch * a.L;
     for (int k = 0; k < sets; ++k) {
@@ -88,17 +106,18 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
     const int prow = a.batch * a.G;
     if (reduce_cols(a.dA_part, tmp, dA, prow, 2 * a.Di * N, stream) != VIM_OK) return VIM_ERR_CUDA;
     if (reduce_cols(a.dD_part, tmp, dD, prow, 2 * a.Di, stream) != VIM_OK) return VIM_ERR_CUDA;
-    return reduce_cols(a.dbias_part, tmp, dbias, prow, 2 * a.Di, stream);
+    if (reduce_cols(a.dbias_part, tmp, dbias, prow, 2 * a.Di, stream) != VIM_OK) return VIM_ERR_CUDA;
+    return rec(ev, 3, stream) ? VIM_OK : VIM_ERR_CUDA;
 }
 
 template <typename T>
 vim_status launch_bwd_n(int N, const BwdArgs &a, const PairArgs &fwd, float *dB[2], float *dC[2], float *dA,
-                        float *dD, float *dbias, float *tmp, cudaStream_t stream) {
+                        float *dD, float *dbias, float *tmp, cudaStream_t stream, cudaEvent_t *ev) {
     switch (N) {
-        case 2: return launch_bwd<T, 2>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream);
-        case 4: return launch_bwd<T, 4>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream);
-        case 8: return launch_bwd<T, 8>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream);
-        case 16: return launch_bwd<T, 16>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream);
+        case 2: return launch_bwd<T, 2>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
+        case 4: return launch_bwd<T, 4>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
+        case 8: return launch_bwd<T, 8>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
+        case 16: return launch_bwd<T, 16>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
         default: return VIM_ERR_UNSUPPORTED;
     }
 }
@@ -117,12 +136,12 @@ size_t vim_scan_bwd_workspace_bytes(int batch, int L, int d_inner, int d_state, 
     return bwd_plan(batch, L, d_inner, d_state, separate_bc).total;
 }
 
-vim_status vim_scan_bidir_bwd(const void *u, const void *delta, const void *z, const void *B, const void *C,
-                              int64_t bc_dir_stride, const float *A, const float *D, const float *delta_bias,
-                              const void *dout, void *du, void *ddelta, void *dz, float *dB, float *dC,
-                              float *dA, float *dD, float *ddelta_bias, int batch, int L, int d_inner,
-                              int d_state, vim_dtype dt, void *workspace, size_t workspace_bytes,
-                              cudaStream_t stream) {
+vim_status vim_scan_bidir_bwd_events(const void *u, const void *delta, const void *z, const void *B,
+                                     const void *C, int64_t bc_dir_stride, const float *A, const float *D,
+                                     const float *delta_bias, const void *dout, void *du, void *ddelta, void *dz,
+                                     float *dB, float *dC, float *dA, float *dD, float *ddelta_bias, int batch,
+                                     int L, int d_inner, int d_state, vim_dtype dt, void *workspace,
+                                     size_t workspace_bytes, cudaStream_t stream, cudaEvent_t *events) {
     vim_status st = check_common(batch, L, d_inner, d_state, dt);
     if (st != VIM_OK) return st;
     if (bc_dir_stride < 0) return VIM_ERR_INVALID_ARG;
@@ -184,8 +203,20 @@ vim_status vim_scan_bidir_bwd(const void *u, const void *delta, const void *z, c
 
     float *dBo[2] = {dB, dB + bc_dir_stride}, *dCo[2] = {dC, dC + bc_dir_stride};
     float *tmp = reinterpret_cast<float *>(ws + pl.off_tmp);
-    return dt == VIM_F32 ? launch_bwd_n<float>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream)
-                         : launch_bwd_n<__nv_bfloat16>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream);
+    return dt == VIM_F32
+               ? launch_bwd_n<float>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream, events)
+               : launch_bwd_n<__nv_bfloat16>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream, events);
+}
+
+vim_status vim_scan_bidir_bwd(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                              int64_t bc_dir_stride, const float *A, const float *D, const float *delta_bias,
+                              const void *dout, void *du, void *ddelta, void *dz, float *dB, float *dC,
+                              float *dA, float *dD, float *ddelta_bias, int batch, int L, int d_inner,
+                              int d_state, vim_dtype dt, void *workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
+    return vim_scan_bidir_bwd_events(u, delta, z, B, C, bc_dir_stride, A, D, delta_bias, dout, du, ddelta, dz,
+                                     dB, dC, dA, dD, ddelta_bias, batch, L, d_inner, d_state, dt, workspace,
+                                     workspace_bytes, stream, nullptr);
 }
 
 }  // extern "C"

@@ -14,11 +14,13 @@
 // chunk comes from the forward scan's own summary kernels (pair_carry, pair_combine);
 // the adjoint g entering each chunk from the later side comes from adj_carry plus
 // pair_combine folding against the direction.  bwd_main then runs one chunk of 16
-// channels, both directions: a forward sweep that keeps h every kBwdSeg tokens (in
+// or 32 channels, both directions: a forward sweep that keeps h every kBwdSeg tokens (in
 // registers) and forms y (for dz) and the dC terms, then segment by segment in
 // reverse a re-run of h over the segment followed by the adjoint sweep.  A thread
-// holds NT <= 4 states of one (channel, direction), so the checkpoints and the
-// segment's h fit in registers; Q = N / NT threads share a channel.
+// holds NT <= 4 states of one (channel, direction), so the segment's h and decays fit
+// in registers (the checkpoints go to shared memory); Q = N / NT threads share a
+// channel.  Each warp serves one direction, whose code is compiled separately so that
+// its token addresses are constants.
 // Sums over channels (dB, dC) are reduced across the warp by shuffles, then across
 // the CTA's warps and directions in shared memory, and written per CTA; sums over
 // tokens (dA, dD, dbias) are written per chunk.  Small reduction kernels finish both.
@@ -33,7 +35,6 @@ namespace vimscan {
 constexpr int kBwdChunk = 32;                 // tokens per chunk
 constexpr int kBwdSeg = 4;                    // tokens between checkpoints of h
 constexpr int kBwdNSeg = kBwdChunk / kBwdSeg;
-constexpr int kBwdCh = 16;                    // channels per bwd_main CTA
 constexpr int kAdjCh = 64;                    // channels per adj_carry CTA
 constexpr int kReduceParts = 32;              // row groups of the first parameter-reduction pass
 #ifndef VIMSCAN_BWD_MIN_WARPS
@@ -80,12 +81,13 @@ __device__ __forceinline__ float silu_grad(float z) {
 // adjoint summaries: per chunk and direction, the adjoint a chunk passes to the one
 // its direction visits before it, from zero entering the chunk:
 //   G_n = sum_s exp(A_n S_s) C_sn dy_s,  S_s = Delta summed over the chunk's tokens
-// visited up to and including s.  One thread per (channel, direction), all N states.
+// visited up to and including s.  One thread per (channel, direction), all N states;
+// with A_n = (n+1) A_0 (checked per warp) the weights are powers of one exp.
 // ----------------------------------------------------------------------------
 template <typename T, int N>
 __global__ void __launch_bounds__(2 * kAdjCh) adj_carry(BwdArgs p) {
     __shared__ float sDr[kBwdChunk][kAdjCh], sDy[kBwdChunk][kAdjCh];
-    __shared__ float sC[2][kBwdChunk][N];
+    __shared__ __align__(16) float sC[2][kBwdChunk][N];
     const int b = blockIdx.z, c = blockIdx.y, d0 = blockIdx.x * kAdjCh;
     const int t0 = c * kBwdChunk, tc = min(kBwdChunk, p.L - t0);
     for (int li = threadIdx.x; li < kBwdChunk * kAdjCh; li += 2 * kAdjCh) {
@@ -107,25 +109,46 @@ __global__ void __launch_bounds__(2 * kAdjCh) adj_carry(BwdArgs p) {
     __syncthreads();
 
     const int dir = threadIdx.x / kAdjCh, dl = threadIdx.x % kAdjCh, d = d0 + dl;
-    if (d >= p.Di) return;
-    float A2[N], G[N];
+    const bool valid = d < p.Di;
+    constexpr int NP = N / 2;
+    const float *Ad = p.A + ((size_t)dir * p.Di + (valid ? d : 0)) * N;
+    bool structured = true;
 #pragma unroll
-    for (int n = 0; n < N; ++n) {
-        A2[n] = p.A[((size_t)dir * p.Di + d) * N + n] * kLog2e;
-        G[n] = 0.0f;
-    }
+    for (int n = 0; n < N; ++n) structured = structured && (Ad[n] == (float)(n + 1) * Ad[0]);
+    const bool fast = __all_sync(0xffffffffu, structured);
+    if (!valid) return;
+    const float A0 = Ad[0] * kLog2e;
     const float bias = p.bias[(size_t)dir * p.Di + d];
+    float2 G[NP];
+#pragma unroll
+    for (int k = 0; k < NP; ++k) G[k] = f2(0.f, 0.f);
     float S = 0.0f;
     for (int i = 0; i < tc; ++i) {
         const int r = dir ? tc - 1 - i : i;
         S += softplus(sDr[r][dl] + bias);
         const float e = sDy[r][dl];
+        float2 Cv[NP];
+        load_row<NP>(&sC[dir][r][0], Cv);
+        if (fast) {
+            // weights exp(A_n S) = w^(n+1), w = exp(A_0 S), two states at a time
+            const float w = ex2(A0 * S);
+            float2 x = f2(w * e, w * w * e);
+            const float2 w2 = f2(w * w, w * w);
 #pragma unroll
-        for (int n = 0; n < N; ++n) G[n] = fmaf(ex2(A2[n] * S) * sC[dir][r][n], e, G[n]);
+            for (int k = 0; k < NP; ++k) {
+                G[k] = fma2(x, Cv[k], G[k]);
+                x = mul2(x, w2);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < NP; ++k)
+                G[k] = fma2(f2(ex2(Ad[2 * k] * kLog2e * S) * e, ex2(Ad[2 * k + 1] * kLog2e * S) * e), Cv[k], G[k]);
+        }
     }
     const size_t base = (((size_t)b * p.G + c) * 2 + dir) * p.Di + d;
+    float2 *out = reinterpret_cast<float2 *>(p.gloc + base * N);
 #pragma unroll
-    for (int n = 0; n < N; ++n) p.gloc[base * N + n] = G[n];
+    for (int k = 0; k < NP; ++k) out[k] = G[k];
     p.gsum[base] = S;
 }
 
@@ -165,217 +188,302 @@ __device__ __forceinline__ void reduce_channels(float (&v)[NT], int lane, int *o
 // ----------------------------------------------------------------------------
 // the derivative over one chunk of 16 channels, both directions
 // ----------------------------------------------------------------------------
+// ----------------------------------------------------------------------------
+// the derivative over one chunk of CH channels, both directions
+// ----------------------------------------------------------------------------
+template <int N> struct BwdShape {
+    static constexpr int NT = N < 4 ? N : 4;                 // states per thread
+    static constexpr int Q = N / NT;                         // threads per (channel, direction)
+    static constexpr int CH = 32 / Q > 16 ? 32 / Q : 16;     // channels per CTA (whole warps per direction)
+    static constexpr int kThr = 2 * CH * Q;
+    static constexpr int WPD = CH * Q / 32;                  // warps per direction
+    static constexpr int CW = 32 / Q;                        // channels per warp
+    static constexpr int kMinBlocks = VIMSCAN_BWD_MIN_WARPS * 32 / kThr;
+    static constexpr int TC = kBwdChunk;
+    // shared memory, in floats (every row of the chunk):
+    //   tok[2][TC][CH] float4 {Delta, u, dy, sigmoid(delta_raw + bias)} per direction
+    //   yb[2][TC][CH]  y^k in the forward sweep, then du^k in the adjoint sweep
+    //   dd[2][TC][CH]  d delta_raw from direction k
+    //   B[2][TC][N], C[2][TC][N]
+    //   red[2][WPD][TC][N]  per direction and warp: the dC terms, then the dB terms
+    //   ck[kBwdNSeg][kThr] float4  h at every kBwdSeg-th token, per thread
+    static constexpr int oTok = 0;
+    static constexpr int oYb = oTok + 2 * TC * CH * 4;
+    static constexpr int oDd = oYb + 2 * TC * CH;
+    static constexpr int oB = oDd + 2 * TC * CH;
+    static constexpr int oC = oB + 2 * TC * N;
+    static constexpr int oRed = oC + 2 * TC * N;
+    static constexpr int oCk = oRed + 2 * WPD * TC * N;
+    static constexpr int kFloats = oCk + kBwdNSeg * kThr * 4;
+    static constexpr size_t kSmemBytes = (size_t)kFloats * 4;
+    static_assert(oCk % 4 == 0 && oTok % 4 == 0, "float4 areas must be 16-byte aligned");
+};
+
+template <int N>
+struct BwdSmem {
+    using SH = BwdShape<N>;
+    float4 *tok;
+    float *yb, *dd, *B, *C, *red;
+    float4 *ck;
+    __device__ explicit BwdSmem(float *base)
+        : tok(reinterpret_cast<float4 *>(base + SH::oTok)), yb(base + SH::oYb), dd(base + SH::oDd),
+          B(base + SH::oB), C(base + SH::oC), red(base + SH::oRed), ck(reinterpret_cast<float4 *>(base + SH::oCk)) {}
+};
+
+// per-thread identity and parameters of one (channel, direction, state group)
+template <int N>
+struct BwdThread {
+    using SH = BwdShape<N>;
+    int tid, lane, q, cl, dir, wid, j0, d;
+    bool valid;
+    float A2[SH::NT], Araw[SH::NT];
+    float Dk;
+    size_t cbase;   // [b][c][dir][d]
+};
+
+template <int NT>
+__device__ __forceinline__ void load_states(const float *row, float (&v)[NT]) {
+    if constexpr (NT == 4) {
+        const float4 t = *reinterpret_cast<const float4 *>(row);
+        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    } else {
+#pragma unroll
+        for (int j = 0; j < NT; ++j) v[j] = row[j];
+    }
+}
+
+// forward sweep of direction DIR: checkpoints, y^DIR (ungated) and the dC terms
+template <int N, int DIR>
+__device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
+    using SH = BwdShape<N>;
+    constexpr int NT = SH::NT, Q = SH::Q, CH = SH::CH, TC = SH::TC;
+    float h[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) h[j] = (p.G > 1 && th.valid) ? p.hin[th.cbase * N + th.j0 + j] : 0.0f;
+#pragma unroll 1
+    for (int sg = 0; sg < kBwdNSeg; ++sg) {
+        sm.ck[sg * SH::kThr + th.tid] = make_float4(h[0], NT > 1 ? h[NT > 1 ? 1 : 0] : 0.0f,
+                                                    NT > 2 ? h[NT > 2 ? 2 : 0] : 0.0f, NT > 3 ? h[NT > 3 ? 3 : 0] : 0.0f);
+#pragma unroll
+        for (int m = 0; m < kBwdSeg; ++m) {
+            const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
+            const float4 tk = sm.tok[(DIR * TC + r) * CH + th.cl];   // Delta, u, dy, sigmoid
+            float Bv[NT], Cv[NT], v[NT];
+            load_states<NT>(sm.B + (DIR * TC + r) * N + th.j0, Bv);
+            load_states<NT>(sm.C + (DIR * TC + r) * N + th.j0, Cv);
+            const float du = tk.x * tk.y;
+            float yp = th.q == 0 ? th.Dk * tk.y : 0.0f;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                h[j] = fmaf(ex2(tk.x * th.A2[j]), h[j], du * Bv[j]);
+                yp = fmaf(Cv[j], h[j], yp);
+                v[j] = tk.z * h[j];
+            }
+#pragma unroll
+            for (int s = 1; s < Q; s <<= 1) yp += __shfl_xor_sync(0xffffffffu, yp, s);
+            if (th.q == 0) sm.yb[(DIR * TC + r) * CH + th.cl] = yp;
+            int off;
+            bool wr;
+            reduce_channels<NT, Q, SH::CW>(v, th.lane, &off, &wr);
+            if (wr) sm.red[((DIR * SH::WPD + th.wid) * TC + r) * N + th.j0 + off] = v[0];
+        }
+    }
+}
+
+// adjoint sweep of direction DIR, segment by segment from the last: h re-run over
+// the segment from its checkpoint (keeping h and the decays), then g backwards
+template <int N, int DIR>
+__device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
+    using SH = BwdShape<N>;
+    constexpr int NT = SH::NT, Q = SH::Q, CH = SH::CH, TC = SH::TC;
+    // with Q > 1 lane q = 0 gathers du and lane q = 1 d delta_raw of the channel
+    constexpr int kDdLane = Q > 1 ? 1 : 0;
+    float g[NT], dA[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        g[j] = (p.G > 1 && th.valid) ? p.gloc[th.cbase * N + th.j0 + j] : 0.0f;
+        dA[j] = 0.0f;
+    }
+    float dD = 0.0f, dbias = 0.0f;
+#pragma unroll 1
+    for (int sg = kBwdNSeg - 1; sg >= 0; --sg) {
+        const float4 c4 = sm.ck[sg * SH::kThr + th.tid];
+        const float h0[4] = {c4.x, c4.y, c4.z, c4.w};
+        float hh[kBwdSeg][NT], aa[kBwdSeg][NT];
+#pragma unroll
+        for (int m = 0; m < kBwdSeg; ++m) {
+            const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
+            const float4 tk = sm.tok[(DIR * TC + r) * CH + th.cl];
+            float Bv[NT];
+            load_states<NT>(sm.B + (DIR * TC + r) * N + th.j0, Bv);
+            const float du = tk.x * tk.y;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                aa[m][j] = ex2(tk.x * th.A2[j]);
+                hh[m][j] = fmaf(aa[m][j], m > 0 ? hh[m > 0 ? m - 1 : 0][j] : h0[j], du * Bv[j]);
+            }
+        }
+#pragma unroll
+        for (int m = kBwdSeg - 1; m >= 0; --m) {
+            const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
+            const float4 tk = sm.tok[(DIR * TC + r) * CH + th.cl];   // Delta, u, dy, sigmoid
+            float Bv[NT], Cv[NT], v[NT];
+            load_states<NT>(sm.B + (DIR * TC + r) * N + th.j0, Bv);
+            load_states<NT>(sm.C + (DIR * TC + r) * N + th.j0, Cv);
+            const float du = tk.x * tk.y;
+            float sA = 0.0f, sBg = 0.0f;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                g[j] = fmaf(Cv[j], tk.z, g[j]);                           // dl/dh_t
+                const float hp = m > 0 ? hh[m > 0 ? m - 1 : 0][j] : h0[j];  // h_(t-1)
+                const float ga = aa[m][j] * g[j];
+                const float w = ga * hp;
+                dA[j] = fmaf(tk.x, w, dA[j]);
+                sA = fmaf(th.Araw[j], w, sA);
+                sBg = fmaf(g[j], Bv[j], sBg);
+                v[j] = g[j] * du;
+                g[j] = ga;                                                // dl/dh_(t-1) part
+            }
+            // this thread's share of du and d delta_raw, gathered over the Q lanes of
+            // the channel: lane q = 0 ends with du, lane q = 1 with d delta_raw
+            float x0 = tk.x * sBg, x1 = fmaf(tk.y, sBg, sA) * tk.w;
+            if constexpr (Q > 1) {
+                const bool odd = (th.q & 1) != 0;
+                const float send = odd ? x0 : x1;
+                float keep = odd ? x1 : x0;
+                keep += __shfl_xor_sync(0xffffffffu, send, 1);
+#pragma unroll
+                for (int s = 2; s < Q; s <<= 1) keep += __shfl_xor_sync(0xffffffffu, keep, s);
+                x0 = keep;
+                x1 = keep;
+            }
+            if (th.q == 0) {
+                sm.yb[(DIR * TC + r) * CH + th.cl] = fmaf(th.Dk, tk.z, x0);
+                dD = fmaf(tk.z, tk.y, dD);
+            }
+            if (th.q == kDdLane) {
+                sm.dd[(DIR * TC + r) * CH + th.cl] = x1;
+                dbias += x1;
+            }
+            int off;
+            bool wr;
+            reduce_channels<NT, Q, SH::CW>(v, th.lane, &off, &wr);
+            if (wr) sm.red[((DIR * SH::WPD + th.wid) * TC + r) * N + th.j0 + off] = v[0];
+        }
+    }
+    if (th.valid) {
+#pragma unroll
+        for (int j = 0; j < NT; ++j) p.dA_part[th.cbase * N + th.j0 + j] = dA[j];
+        if (th.q == 0) p.dD_part[th.cbase] = dD;
+        if (th.q == kDdLane) p.dbias_part[th.cbase] = dbias;
+    }
+}
+
 // The CTA's per-token sums over its channels of the dB (or dC) terms, from the
 // per-direction, per-warp slots, into part[set][b][t][blk][n]: the two directions
 // add into one set when B and C are shared.
-template <int N, int WPD>
-__device__ __forceinline__ void store_bc_part(const BwdArgs &p, const float (&red)[2][WPD][kBwdChunk][N],
-                                              float *const (&part)[2], int b, int t0, int tc, int blk) {
+template <int N>
+__device__ __forceinline__ void store_bc_part(const BwdArgs &p, const float *red, float *const (&part)[2], int b,
+                                              int t0, int tc, int blk) {
+    using SH = BwdShape<N>;
+    constexpr int TC = SH::TC;
     const int nsets = p.separate_bc ? 2 : 1;
-    for (int li = threadIdx.x; li < nsets * kBwdChunk * N; li += blockDim.x) {
-        const int k = li / (kBwdChunk * N), r = (li / N) % kBwdChunk, n = li % N;
+    for (int li = threadIdx.x; li < nsets * TC * N; li += SH::kThr) {
+        const int k = li / (TC * N), r = (li / N) % TC, n = li % N;
         if (r >= tc) continue;
         float acc = 0.0f;
 #pragma unroll
         for (int dir = 0; dir < 2; ++dir) {
             if (p.separate_bc && dir != k) continue;
 #pragma unroll
-            for (int w = 0; w < WPD; ++w) acc += red[dir][w][r][n];
+            for (int w = 0; w < SH::WPD; ++w) acc += red[((dir * SH::WPD + w) * TC + r) * N + n];
         }
         part[k][(((size_t)b * p.L + t0 + r) * p.nblk + blk) * N + n] = acc;
     }
 }
 
-template <int N> struct BwdShape {
-    static constexpr int NT = N < 4 ? N : 4;           // states per thread
-    static constexpr int Q = N / NT;                   // threads per (channel, direction)
-    static constexpr int kThr = 2 * kBwdCh * Q;
-    static constexpr int CW = (32 / Q < kBwdCh) ? 32 / Q : kBwdCh;   // channels per warp
-    static constexpr int WPD = (kBwdCh * Q + 31) / 32;                // warps per direction
-    static constexpr int kMinBlocks = VIMSCAN_BWD_MIN_WARPS * 32 / kThr;   // resident CTAs per SM aimed at
-};
-
 template <typename T, int N>
 __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bwd_main(BwdArgs p) {
     using SH = BwdShape<N>;
-    constexpr int NT = SH::NT, Q = SH::Q, CH = kBwdCh, TC = kBwdChunk;
-    constexpr int WPD = SH::WPD;
-    __shared__ float sU[TC][CH], sDy[TC][CH], sDzf[TC][CH];
-    __shared__ float sY[2][TC][CH], sDu[2][TC][CH], sDd[2][TC][CH];   // per direction
-    __shared__ float sDelta[2][TC][CH], sSig[2][TC][CH];
-    __shared__ __align__(16) float sB[2][TC][N], sC[2][TC][N];
-    __shared__ float sRed[2][WPD][TC][N];   // per direction and warp: dC terms, then dB terms
+    constexpr int NT = SH::NT, Q = SH::Q, CH = SH::CH, TC = SH::TC;
+    extern __shared__ __align__(16) float smem_f[];
+    const BwdSmem<N> sm(smem_f);
 
     const int b = blockIdx.z, c = blockIdx.y, blk = blockIdx.x, d0 = blk * CH;
     const int t0 = c * TC, tc = min(TC, p.L - t0);
 
-    // ---- stage the chunk: u, dy = dout silu(z), dout silu'(z), Delta and
-    // sigmoid(delta_raw + bias) per direction, B and C per direction ----------------
+    // ---- stage the chunk: {Delta, u, dy, sigmoid} per direction, B and C ------------
     for (int li = threadIdx.x; li < TC * CH; li += SH::kThr) {
         const int r = li / CH, cl = li % CH, ch = d0 + cl;
-        float u = 0.0f, e = 0.0f, ezf = 0.0f, dl0 = 0.0f, dl1 = 0.0f, sg0 = 0.0f, sg1 = 0.0f;
+        float u = 0.0f, e = 0.0f, dl0 = 0.0f, dl1 = 0.0f, sg0 = 0.0f, sg1 = 0.0f;
         if (r < tc && ch < p.Di) {
             const size_t i = ((size_t)b * p.L + t0 + r) * p.Di + ch;
             u = ld<T>(p.u, i);
-            const float dr = ld<T>(p.delta, i), o = ld<T>(p.dout, i);
-            if (p.z) {
-                const float z = ld<T>(p.z, i);
-                e = o * silu(z);
-                ezf = o * silu_grad(z);
-            } else {
-                e = o;
-            }
+            const float dr = ld<T>(p.delta, i);
+            e = ld<T>(p.dout, i);
+            if (p.z) e *= silu(ld<T>(p.z, i));
             const float x0 = dr + p.bias[ch], x1 = dr + p.bias[p.Di + ch];
             dl0 = softplus(x0); sg0 = softplus_grad(x0);
             dl1 = softplus(x1); sg1 = softplus_grad(x1);
         }
-        sU[r][cl] = u; sDy[r][cl] = e; sDzf[r][cl] = ezf;
-        sDelta[0][r][cl] = dl0; sDelta[1][r][cl] = dl1;
-        sSig[0][r][cl] = sg0; sSig[1][r][cl] = sg1;
+        sm.tok[r * CH + cl] = make_float4(dl0, u, e, sg0);
+        sm.tok[(TC + r) * CH + cl] = make_float4(dl1, u, e, sg1);
     }
     for (int li = threadIdx.x; li < 2 * TC * N; li += SH::kThr) {
         const int k = li / (TC * N), r = (li / N) % TC, n = li % N;
         const size_t i = ((size_t)b * p.L + t0 + r) * N + n;
-        sB[k][r][n] = r < tc ? ld<T>(p.B[k], i) : 0.0f;
-        sC[k][r][n] = r < tc ? ld<T>(p.C[k], i) : 0.0f;
+        sm.B[li] = r < tc ? ld<T>(p.B[k], i) : 0.0f;
+        sm.C[li] = r < tc ? ld<T>(p.C[k], i) : 0.0f;
     }
+
+    BwdThread<N> th;
+    th.tid = threadIdx.x;
+    th.lane = th.tid & 31;
+    th.q = th.tid % Q;
+    th.cl = (th.tid / Q) % CH;
+    th.dir = th.tid / (Q * CH);
+    th.wid = (th.tid / 32) % SH::WPD;
+    th.j0 = th.q * NT;
+    th.d = d0 + th.cl;
+    th.valid = th.d < p.Di;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        th.Araw[j] = th.valid ? p.A[((size_t)th.dir * p.Di + th.d) * N + th.j0 + j] : 0.0f;
+        th.A2[j] = th.Araw[j] * kLog2e;
+    }
+    th.Dk = th.valid ? p.D[(size_t)th.dir * p.Di + th.d] : 0.0f;
+    th.cbase = (((size_t)b * p.G + c) * 2 + th.dir) * p.Di + th.d;
     __syncthreads();
 
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int q = tid % Q, cl = (tid / Q) % CH, dir = tid / (Q * CH), d = d0 + cl;
-    const bool valid = d < p.Di;
-    const int j0 = q * NT;                       // first state of this thread
-    const int wid = (tid / 32) % WPD;            // warp within the direction
-    float A2[NT], Araw[NT];
-    float Dk = 0.0f;
-#pragma unroll
-    for (int j = 0; j < NT; ++j) Araw[j] = valid ? p.A[((size_t)dir * p.Di + d) * N + j0 + j] : 0.0f;
-#pragma unroll
-    for (int j = 0; j < NT; ++j) A2[j] = Araw[j] * kLog2e;
-    if (valid) Dk = p.D[(size_t)dir * p.Di + d];
-    const size_t cbase = (((size_t)b * p.G + c) * 2 + dir) * p.Di + d;   // [b][c][dir][d]
-
-    // ---- forward sweep: checkpoints, y (ungated) and the dC terms -------------------
-    float h[NT], ck[kBwdNSeg][NT];
-#pragma unroll
-    for (int j = 0; j < NT; ++j) h[j] = (p.G > 1 && valid) ? p.hin[cbase * N + j0 + j] : 0.0f;
-#pragma unroll
-    for (int i = 0; i < TC; ++i) {
-        const int r = dir ? TC - 1 - i : i;
-        if (i % kBwdSeg == 0) {
-#pragma unroll
-            for (int j = 0; j < NT; ++j) ck[i / kBwdSeg][j] = h[j];
-        }
-        const float dt = sDelta[dir][r][cl], x = sU[r][cl], e = sDy[r][cl];
-        const float du = dt * x;
-        float yp = q == 0 ? Dk * x : 0.0f;
-        float v[NT];
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-            h[j] = fmaf(ex2(dt * A2[j]), h[j], du * sB[dir][r][j0 + j]);
-            yp = fmaf(sC[dir][r][j0 + j], h[j], yp);
-            v[j] = e * h[j];
-        }
-#pragma unroll
-        for (int s = 1; s < Q; s <<= 1) yp += __shfl_xor_sync(0xffffffffu, yp, s);
-        if (q == 0) sY[dir][r][cl] = yp;
-        int off;
-        bool wr;
-        reduce_channels<NT, Q, SH::CW>(v, lane, &off, &wr);
-        if (wr) sRed[dir][wid][r][j0 + off] = v[0];
-    }
+    if (th.dir == 0) bwd_forward<N, 0>(p, sm, th);
+    else bwd_forward<N, 1>(p, sm, th);
     __syncthreads();
     // dz = dout silu'(z) (y^f + y^b), and the CTA's dC terms
     if (p.dz) {
         for (int li = threadIdx.x; li < TC * CH; li += SH::kThr) {
             const int r = li / CH, c2 = li % CH, ch = d0 + c2;
-            if (r < tc && ch < p.Di)
-                static_cast<T *>(p.dz)[((size_t)b * p.L + t0 + r) * p.Di + ch] =
-                    from_f32<T>(sDzf[r][c2] * (sY[0][r][c2] + sY[1][r][c2]));
+            if (r < tc && ch < p.Di) {
+                const size_t i = ((size_t)b * p.L + t0 + r) * p.Di + ch;
+                const float y = sm.yb[r * CH + c2] + sm.yb[(TC + r) * CH + c2];
+                static_cast<T *>(p.dz)[i] = from_f32<T>(ld<T>(p.dout, i) * silu_grad(ld<T>(p.z, i)) * y);
+            }
         }
     }
-    store_bc_part<N, WPD>(p, sRed, p.dC_part, b, t0, tc, blk);
+    store_bc_part<N>(p, sm.red, p.dC_part, b, t0, tc, blk);
     __syncthreads();
 
-    // ---- reverse: per segment, re-run h over it, then the adjoint sweep -------------
-    float g[NT], dA[NT];
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-        g[j] = (p.G > 1 && valid) ? p.gloc[cbase * N + j0 + j] : 0.0f;
-        dA[j] = 0.0f;
-    }
-    float dD = 0.0f, dbias = 0.0f;
-#pragma unroll
-    for (int sg = kBwdNSeg - 1; sg >= 0; --sg) {
-        float hist[kBwdSeg][NT];
-#pragma unroll
-        for (int j = 0; j < NT; ++j) h[j] = ck[sg][j];
-#pragma unroll
-        for (int m = 0; m < kBwdSeg; ++m) {
-            const int i = sg * kBwdSeg + m, r = dir ? TC - 1 - i : i;
-            const float dt = sDelta[dir][r][cl], du = dt * sU[r][cl];
-#pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                h[j] = fmaf(ex2(dt * A2[j]), h[j], du * sB[dir][r][j0 + j]);
-                hist[m][j] = h[j];
-            }
-        }
-#pragma unroll
-        for (int m = kBwdSeg - 1; m >= 0; --m) {
-            const int i = sg * kBwdSeg + m, r = dir ? TC - 1 - i : i;
-            const float dt = sDelta[dir][r][cl], x = sU[r][cl], e = sDy[r][cl];
-            float sA = 0.0f, sBg = 0.0f, v[NT];
-#pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                g[j] = fmaf(sC[dir][r][j0 + j], e, g[j]);                 // dl/dh_t
-                const float hp = m > 0 ? hist[m - 1][j] : ck[sg][j];     // h_(t-1)
-                const float ga = ex2(dt * A2[j]) * g[j];
-                const float w = ga * hp;
-                dA[j] = fmaf(dt, w, dA[j]);
-                sA = fmaf(Araw[j], w, sA);
-                sBg = fmaf(g[j], sB[dir][r][j0 + j], sBg);
-                v[j] = g[j] * (dt * x);
-                g[j] = ga;                                               // dl/dh_(t-1) part
-            }
-            float dup = dt * sBg;
-            float ddp = fmaf(x, sBg, sA) * sSig[dir][r][cl];
-#pragma unroll
-            for (int s = 1; s < Q; s <<= 1) {
-                dup += __shfl_xor_sync(0xffffffffu, dup, s);
-                ddp += __shfl_xor_sync(0xffffffffu, ddp, s);
-            }
-            if (q == 0) {
-                sDu[dir][r][cl] = fmaf(Dk, e, dup);
-                sDd[dir][r][cl] = ddp;
-                dD = fmaf(e, x, dD);
-                dbias += ddp;
-            }
-            int off;
-            bool wr;
-            reduce_channels<NT, Q, SH::CW>(v, lane, &off, &wr);
-            if (wr) sRed[dir][wid][r][j0 + off] = v[0];
-        }
-    }
-
-    // ---- per-chunk sums over tokens ------------------------------------------------
-    if (valid) {
-#pragma unroll
-        for (int j = 0; j < NT; ++j) p.dA_part[cbase * N + j0 + j] = dA[j];
-        if (q == 0) {
-            p.dD_part[cbase] = dD;
-            p.dbias_part[cbase] = dbias;
-        }
-    }
+    if (th.dir == 0) bwd_adjoint<N, 0>(p, sm, th);
+    else bwd_adjoint<N, 1>(p, sm, th);
     __syncthreads();
     for (int li = threadIdx.x; li < TC * CH; li += SH::kThr) {
         const int r = li / CH, c2 = li % CH, ch = d0 + c2;
         if (r < tc && ch < p.Di) {
             const size_t i = ((size_t)b * p.L + t0 + r) * p.Di + ch;
-            static_cast<T *>(p.du)[i] = from_f32<T>(sDu[0][r][c2] + sDu[1][r][c2]);
-            static_cast<T *>(p.ddelta)[i] = from_f32<T>(sDd[0][r][c2] + sDd[1][r][c2]);
+            static_cast<T *>(p.du)[i] = from_f32<T>(sm.yb[r * CH + c2] + sm.yb[(TC + r) * CH + c2]);
+            static_cast<T *>(p.ddelta)[i] = from_f32<T>(sm.dd[r * CH + c2] + sm.dd[(TC + r) * CH + c2]);
         }
     }
-    store_bc_part<N, WPD>(p, sRed, p.dB_part, b, t0, tc, blk);
+    store_bc_part<N>(p, sm.red, p.dB_part, b, t0, tc, blk);
 }
 
 // dB / dC: sum of the per-CTA partials, [batch][L][nblk][N] -> [batch][L][N]

@@ -52,6 +52,8 @@ VIM_FLAG_ZOH_EXACT = 1
 lib.vim_scan_bidir_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                    _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _vp]
 lib.vim_scan_bidir_bwd.restype = _i
+lib.vim_scan_bidir_bwd_events.argtypes = lib.vim_scan_bidir_bwd.argtypes + [_vp]
+lib.vim_scan_bidir_bwd_events.restype = _i
 lib.vim_scan_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
 lib.vim_scan_bwd_workspace_bytes.restype = _sz
 lib.vim_scan_bidir_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
@@ -188,19 +190,21 @@ def vim_scan_bwd_workspace_bytes(batch, L, d_inner, d_state, separate_bc):
 
 
 def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stride=0, workspace=None,
-                       stream=None):
+                       stream=None, out=None, events=None):
     """Derivatives of vim_scan_bidir (first-order Bbar) for a loss whose derivative
     with respect to y is ``dout``; see include/vimscan.h.
 
     Returns a dict: du, ddelta (w.r.t. the raw delta), dz (None without z), in the
     input dtype; dB and dC (fp32, shaped like B and C); dA [2, d_inner, d_state], dD
-    and ddelta_bias [2, d_inner] (fp32).
+    and ddelta_bias [2, d_inner] (fp32).  ``out`` may hold those tensors from an
+    earlier call to be written again; ``events`` 4 CUDA events (see
+    vim_scan_bidir_bwd_events).
     """
     batch, L, Di = u.shape
     N = B.shape[-1]
     dt = _dtype_code(u)
     dev = u.device
-    out = dict(du=torch.empty_like(u), ddelta=torch.empty_like(u),
+    out = out if out is not None else dict(du=torch.empty_like(u), ddelta=torch.empty_like(u),
                dz=torch.empty_like(u) if z is not None else None,
                dB=torch.zeros(B.shape, dtype=torch.float32, device=dev),
                dC=torch.zeros(C.shape, dtype=torch.float32, device=dev),
@@ -208,14 +212,16 @@ def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stri
                dD=torch.empty((2, Di), dtype=torch.float32, device=dev),
                ddelta_bias=torch.empty((2, Di), dtype=torch.float32, device=dev))
     ws, ws_bytes = _workspace(vim_scan_bwd_workspace_bytes(batch, L, Di, N, bc_dir_stride > 0), workspace, dev)
-    st = lib.vim_scan_bidir_bwd(
+    fn = lib.vim_scan_bidir_bwd if events is None else lib.vim_scan_bidir_bwd_events
+    extra = () if events is None else (_events(events),)
+    st = fn(
         _ptr(u, name="u"), _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
         _ptr(B, dtype=u.dtype, name="B"), _ptr(C, dtype=u.dtype, name="C"), int(bc_dir_stride),
         _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
         _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(dout, dtype=u.dtype, name="dout"),
         _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dz"]), _ptr(out["dB"]), _ptr(out["dC"]),
         _ptr(out["dA"]), _ptr(out["dD"]), _ptr(out["ddelta_bias"]),
-        batch, L, Di, N, dt, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
+        batch, L, Di, N, dt, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream), *extra)
     if st != VIM_OK:
         raise VimScanError(st, "vim_scan_bidir_bwd")
     return out
