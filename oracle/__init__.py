@@ -61,6 +61,7 @@ class Oracle:
         lib.oracle_vim_bidir_conv.argtypes = [_D, _D, _D, _D, _D, _D, _D, ctypes.c_int64, _D, _D, _D, _D] + [ctypes.c_int] * 6
         lib.oracle_s6_direction_bwd.argtypes = [_D] * 7 + [_I64] + [_D] * 8 + [ctypes.c_int] * 5
         lib.oracle_vim_bidir_bwd.argtypes = [_D, _D, _D, _D, _D, ctypes.c_int64] + [_D] * 12 + [ctypes.c_int] * 5
+        lib.oracle_xproj.argtypes = [_D, _D, _D, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
         self.lib = lib
@@ -147,6 +148,46 @@ class Oracle:
         if rc:
             raise ValueError("oracle_vim_bidir_bwd: bad sizes")
         return out
+
+    def xproj(self, u, Wx):
+        """x_proj of the S6 module: P = u @ Wx, u [..., Di], Wx [Di, NO] -> P [..., NO]."""
+        u, Wx = _f64(u), _f64(Wx)
+        Di, NO = Wx.shape
+        lead = u.shape[:-1]
+        M = int(np.prod(lead)) if lead else 1
+        P = np.zeros(lead + (NO,))
+        if self.lib.oracle_xproj(_p(np.ascontiguousarray(u)), _p(Wx), _p(P), M, Di, NO):
+            raise ValueError("oracle_xproj: bad sizes")
+        return P
+
+    def vim_block_scan(self, x, Wx, Wdt, A, D, bias, z, *, conv_w=None, conv_b=None):
+        """The Vim block's two S6 modules from their common input, each with its own
+        projections (page "Vision Mamba Guide": the block runs "1D Conv -> SiLU -> SSM"
+        per pathway, the backward one on the reversed sequence; each SSM derives B, C
+        and Delta from its own input by x_proj and dt_proj):
+          u_k   = silu(conv_k(x)) (conv_w given) or x
+          P_k   = u_k @ Wx[k];  B_k = P_k[..., :N], C_k = P_k[..., N:2N], s_k = P_k[..., 2N]
+          delta_raw_k[t, d] = s_k[t] * Wdt[k, d]   (dt_proj; its bias is `bias`, inside softplus)
+          y = (S6_f(u_f) + S6_b(u_b)) * silu(z)
+        x, z: [batch, L, Di]; Wx [2, Di, 2N+1]; Wdt, bias, D [2, Di]; A [2, Di, N].
+        """
+        x, Wx, Wdt, A, D, bias, z = map(_f64, (x, Wx, Wdt, A, D, bias, z))
+        batch, L, Di = x.shape
+        N = A.shape[-1]
+        y = np.zeros((batch, L, Di))
+        for k in range(2):
+            if conv_w is not None:
+                u = self.conv_silu(x, _f64(conv_w)[k], _f64(conv_b)[k], reversed=bool(k))
+            else:
+                u = x
+            P = self.xproj(u, Wx[k])
+            Bk, Ck = np.ascontiguousarray(P[..., :N]), np.ascontiguousarray(P[..., N:2 * N])
+            draw = P[..., 2 * N][..., None] * Wdt[k][None, None, :]
+            order = np.arange(L) if k == 0 else np.arange(L)[::-1].copy()
+            y += self.s6_direction(u, draw, Bk, Ck, A[k], D[k], bias[k], order, delta_is_raw=True)
+        if z is not None:
+            y *= z / (1.0 + np.exp(-z))
+        return y
 
     def conv_silu(self, x, w, cb, *, reversed=False):
         """silu of the kernel-3 depthwise convolution (zero padding 1) in front of a
@@ -255,6 +296,14 @@ def conv_silu(*a, **k):
 
 def vim_bidir_bwd(*a, **k):
     return default().vim_bidir_bwd(*a, **k)
+
+
+def xproj(*a, **k):
+    return default().xproj(*a, **k)
+
+
+def vim_block_scan(*a, **k):
+    return default().vim_block_scan(*a, **k)
 
 
 def vim_bidir_conv(*a, **k):

@@ -486,3 +486,25 @@ int oracle_vim_bidir_bwd(const double *u, const double *delta, const double *z,
     free(dy); free(order);
     return rc ? -1 : 0;
 }
+
+/*
+ * The input projections of the S6 module (page "Vision Mamba Guide", the PyTorch
+ * SimpleSelectiveSSM under "The Selective State Space (S6) Mechanism": x_proj is a
+ * linear map without bias from d_model to 2N + 1 columns, read as B (columns 0..N-1),
+ * C (columns N..2N-1) and the one-column step input (column 2N); dt_proj maps that
+ * column back to d_model with a bias, and softplus gives Delta):
+ *   P[m, j] = sum_d u[m, d] Wx[d, j]          m < M, j < NO
+ * u: [M, Di], Wx: [Di, NO], P: [M, NO].
+ */
+int oracle_xproj(const double *u, const double *Wx, double *P, int64_t M, int Di, int NO)
+{
+    if (M < 0 || Di < 0 || NO < 1) return -1;
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int j = 0; j < NO; ++j) {
+            double acc = 0.0;
+            for (int d = 0; d < Di; ++d) acc += u[m * Di + d] * Wx[(int64_t)d * NO + j];
+            P[m * NO + j] = acc;
+        }
+    return 0;
+}

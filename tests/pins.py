@@ -548,6 +548,61 @@ def pin_bwd_homogeneity(orc):
     np.testing.assert_allclose(np.sum(g["dD"] * c["D"]), ell_D, rtol=1e-11)
 
 
+def pin_xproj_is_matmul(orc):
+    """x_proj is a plain matrix product (the PyTorch SimpleSelectiveSSM's
+    nn.Linear without bias, page "Vision Mamba Guide"): checked against numpy's
+    matmul on a non-square weight, so a transposed index cannot pass."""
+    rng = _rng(111)
+    u = rng.normal(size=(2, 7, 6))
+    Wx = rng.normal(size=(6, 9))
+    np.testing.assert_allclose(orc.xproj(u, Wx), np.matmul(u, Wx), rtol=1e-13, atol=1e-13)
+
+
+def pin_block_scan_composition(orc):
+    """The Vim block scan with its projections equals its steps done separately:
+    each pathway's smoothed input by numpy correlation (the conv pin's method), its
+    projection by numpy matmul split as the page's module splits it (B = columns
+    0..N-1, C = N..2N-1, the step input = column 2N), dt_proj as the outer product of
+    that column with the pathway's weights, the two directions by single-direction
+    scans (pinned separately), then the gate."""
+    rng = _rng(112)
+    batch, L, Di, N = 2, 9, 3, 4
+    x = rng.normal(size=(batch, L, Di))
+    z = rng.normal(size=(batch, L, Di))
+    Wx = rng.normal(size=(2, Di, 2 * N + 1)) * 0.5
+    Wdt = rng.normal(size=(2, Di))
+    bias = rng.normal(size=(2, Di))
+    A = -rng.uniform(0.2, 2.0, size=(2, Di, N))
+    D = rng.normal(size=(2, Di))
+    cw = rng.normal(size=(2, Di, 3))
+    cb = rng.normal(size=(2, Di))
+    y = orc.vim_block_scan(x, Wx, Wdt, A, D, bias, z, conv_w=cw, conv_b=cb)
+    silu = lambda v: v / (1 + np.exp(-v))
+    total = np.zeros_like(x)
+    for k in range(2):
+        u = np.zeros_like(x)
+        for b in range(batch):
+            for d in range(Di):
+                seq = x[b, :, d] if k == 0 else x[b, ::-1, d]
+                sm = np.correlate(np.pad(seq, 1), cw[k, d], mode="valid") + cb[k, d]
+                u[b, :, d] = silu(sm) if k == 0 else silu(sm)[::-1]
+        P = np.matmul(u, Wx[k])
+        Bk, Ck, s = P[..., :N], P[..., N:2 * N], P[..., 2 * N]
+        draw = s[..., None] * Wdt[k][None, None, :]
+        order = np.arange(L) if k == 0 else np.arange(L)[::-1]
+        total += orc.s6_direction(u, draw, np.ascontiguousarray(Bk), np.ascontiguousarray(Ck), A[k], D[k],
+                                  bias[k], order, delta_is_raw=True)
+    np.testing.assert_allclose(y, total * silu(z), rtol=1e-11, atol=1e-11)
+    # without the convolution the pathways see x itself
+    y0 = orc.vim_block_scan(x, Wx, Wdt, A, D, bias, None)
+    P0 = [np.matmul(x, Wx[k]) for k in range(2)]
+    ref0 = sum(orc.s6_direction(x, P0[k][..., 2 * N][..., None] * Wdt[k][None, None, :],
+                                np.ascontiguousarray(P0[k][..., :N]), np.ascontiguousarray(P0[k][..., N:2 * N]),
+                                A[k], D[k], bias[k], np.arange(L) if k == 0 else np.arange(L)[::-1],
+                                delta_is_raw=True) for k in range(2))
+    np.testing.assert_allclose(y0, ref0, rtol=1e-11, atol=1e-11)
+
+
 ALL_PINS = [
     pin_delta_zero,
     pin_constant_input_geometric,
@@ -568,4 +623,6 @@ ALL_PINS = [
     pin_zoh_reaches_every_entry,
     pin_bwd_finite_differences,
     pin_bwd_homogeneity,
+    pin_xproj_is_matmul,
+    pin_block_scan_composition,
 ]

@@ -8,6 +8,7 @@ channels (dB, dC) and over tokens (dA, dD, d delta_bias) take 1e-4 on the small
 cases and 1e-3 at full size: they add up to batch*L terms of both signs in fp32, and
 a cancelling sum's rounding error is relative to its terms, not to the result.
 """
+import json
 import os
 
 import numpy as np
@@ -21,6 +22,7 @@ pytestmark = pytest.mark.gpu
 
 ELEM_TOL = {torch.float32: 1e-5, torch.bfloat16: 2e-2}
 SUM_TOL = 1e-4
+REPORT = os.environ.get("VIMSCAN_PARITY_REPORT")
 KEYS = [("du", "du"), ("ddelta", "ddelta"), ("dz", "dz"), ("dB", "dB"), ("dC", "dC"), ("dA", "dA"),
         ("dD", "dD"), ("ddelta_bias", "dbias")]
 
@@ -82,6 +84,9 @@ def check_all(name, got, want, dtype, sum_tol=SUM_TOL):
         errs[k_got] = normwise(g, want[k_ref])
         tol = ELEM_TOL[dtype] if k_got in ("du", "ddelta", "dz") else sum_tol
         assert errs[k_got] <= tol, f"{name}: {k_got} normwise error {errs[k_got]:.3e} > {tol:.0e} ({errs})"
+    if REPORT:
+        with open(REPORT, "a") as f:
+            f.write(json.dumps({"case": name, "dtype": str(dtype), "normwise": errs}) + "\n")
     return errs
 
 

@@ -59,6 +59,8 @@ MUTANTS = {
     "bwd_backward_dir_forward_params": ("A + (int64_t)Di * N, D + Di, bias + Di, order, dy,",
                                         "A, D, bias, order, dy,"),
     "bwd_dy_ungated": ("dy[i] = dout[i] * silu(z[i]);", "dy[i] = dout[i];"),
+    "xproj_weight_transposed": ("acc += u[m * Di + d] * Wx[(int64_t)d * NO + j];",
+                                "acc += u[m * Di + d] * Wx[(int64_t)j * Di + d];"),
     "zoh_sign": ("return expm1(dt * An) / An * Bn;", "return expm1(-dt * An) / An * Bn;"),
 }
 
