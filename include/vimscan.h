@@ -224,6 +224,38 @@ vim_status vim_scan_bidir_bwd_events(const void *u, const void *delta, const voi
                                      cudaEvent_t *events);
 
 /*
+ * The Vim block's two S6 modules from their common input x, projections included
+ * (page "Vision Mamba Guide": section "2. The Bidirectional Mamba Block" runs
+ * "1D Conv -> SiLU -> SSM" per pathway; its SSM module, under "The Selective State
+ * Space (S6) Mechanism", derives B, C and Delta from its own input):
+ *
+ *   u_k   = silu(conv_k(x)) as in vim_scan_bidir_conv (conv_w, conv_b non-NULL), else x
+ *   P_k   = u_k Wx[k]   (x_proj, no bias; [batch*L, 2N+1])
+ *   B_k   = P_k[:, 0:N],  C_k = P_k[:, N:2N],  s_k = P_k[:, 2N]
+ *   delta_raw_k[t, d] = s_k[t] * Wdt[k][d]      (dt_proj; its bias is dt_bias, in softplus)
+ *   y = (S6_f(u_f; B_f, C_f, delta_f) + S6_b(u_b; B_b, C_b, delta_b)) * silu(z)
+ *
+ *   x, z, y : [batch, L, d_inner] bf16 (z may be NULL).
+ *   Wx      : [2, d_inner, 2*d_state + 1] bf16 (index 0 = forward pathway).
+ *   Wdt, dt_bias, D : [2, d_inner] fp32;  A : [2, d_inner, d_state] fp32.
+ *   conv_w [2, d_inner, 3], conv_b [2, d_inner] fp32, both or neither.
+ *   events  : NULL, or 5 CUDA events: start, after the projection, then those of
+ *             vim_scan_bidir_events.
+ *   workspace : vim_block_workspace_bytes(...) bytes, 256-byte aligned; it holds B, C
+ *             (bf16) and s (fp32) of both pathways between the two kernels.
+ * x_proj runs on the tensor cores with u_k rounded to bf16 and fp32 accumulation; B and
+ * C are rounded to bf16, s stays fp32; Delta is never written to memory.  Only bf16 I/O
+ * (VIM_F32 returns VIM_ERR_UNSUPPORTED), the first-order Bbar, and d_inner up to 2776
+ * (one pathway's Wx, transposed, is held in one CTA's shared memory).
+ */
+vim_status vim_block_scan(const void *x, const float *conv_w, const float *conv_b, const void *Wx,
+                          const float *Wdt, const float *dt_bias, const float *A, const float *D,
+                          const void *z, void *y, int batch, int L, int d_inner, int d_state,
+                          vim_dtype dt, void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                          cudaEvent_t *events);
+size_t vim_block_workspace_bytes(int batch, int L, int d_inner, int d_state);
+
+/*
  * Options of the _ex entry points, or-ed into `flags` (unknown bits return
  * VIM_ERR_INVALID_ARG).
  *

@@ -37,6 +37,7 @@ def test_header_declares_the_boundary():
                           "vim_scan_bidir_events", "vmamba_cross_scan4_events", "vim_scan_bidir_noalloc", "vim_scan_bidir_conv", "vim_scan_bidir_conv_events",
                           "vim_scan_bidir_ex", "vmamba_cross_scan4_ex",
                           "vim_scan_bidir_bwd", "vim_scan_bwd_workspace_bytes", "vim_scan_bidir_bwd_events",
+                          "vim_block_scan", "vim_block_workspace_bytes",
                           "vim_scan_workspace_bytes", "vim_status_string"}, names
 
 

@@ -111,15 +111,15 @@ inline vim_status mark(cudaEvent_t *events, int i, cudaStream_t stream) {
     return cudaEventRecord(events[i], stream) == cudaSuccess ? VIM_OK : VIM_ERR_CUDA;
 }
 
-template <typename T, int N, bool VEC_BC, bool PIN, bool CONV, bool ZOH>
+template <typename T, int N, bool VEC_BC, bool PIN, bool CONV, bool ZOH, bool DT>
 vim_status launch_pair_v(const PairArgs &a, cudaStream_t stream, cudaEvent_t *ev) {
     const dim3 grid((a.Di + kDC - 1) / kDC, a.G, a.batch);
     if (a.G > 1) {
         const size_t sc = carry_smem<T, N, CONV>();
-        if (cudaFuncSetAttribute(pair_carry<T, N, VEC_BC, CONV, ZOH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(pair_carry<T, N, VEC_BC, CONV, ZOH, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sc) != cudaSuccess)
             return VIM_ERR_CUDA;
-        pair_carry<T, N, VEC_BC, CONV, ZOH><<<grid, kThreads, sc, stream>>>(a);
+        pair_carry<T, N, VEC_BC, CONV, ZOH, DT><<<grid, kThreads, sc, stream>>>(a);
         if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
         if (mark(ev, 0, stream) != VIM_OK) return VIM_ERR_CUDA;
         const int64_t units = (int64_t)a.batch * 2 * a.Di * N;
@@ -131,7 +131,7 @@ vim_status launch_pair_v(const PairArgs &a, cudaStream_t stream, cudaEvent_t *ev
         if (mark(ev, 0, stream) != VIM_OK || mark(ev, 1, stream) != VIM_OK) return VIM_ERR_CUDA;
     }
     const size_t sm = main_smem<T, N, CONV>(a.chunk);
-    auto kernel = pair_main<T, N, VEC_BC, PIN, CONV, ZOH>;
+    auto kernel = pair_main<T, N, VEC_BC, PIN, CONV, ZOH, DT>;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
         return VIM_ERR_CUDA;
     if (a.G > 1) {
@@ -144,12 +144,22 @@ vim_status launch_pair_v(const PairArgs &a, cudaStream_t stream, cudaEvent_t *ev
 }
 
 // the kernel variants a pair needs: fp32 partial_in (second pair of the cross-scan)
-// and the convolution front (Vim with x as input) are never combined
+// and the convolution front (Vim with x as input) are never combined; the step-input
+// mode (delta from the x_proj column, bf16 I/O, first-order Bbar) comes with or
+// without the convolution front
 template <typename T, int N, bool VEC_BC, bool ZOH>
 vim_status launch_pair_v(const PairArgs &a, cudaStream_t stream, cudaEvent_t *ev) {
-    if (a.conv_w) return launch_pair_v<T, N, VEC_BC, false, true, ZOH>(a, stream, ev);
-    if (a.partial_in) return launch_pair_v<T, N, VEC_BC, true, false, ZOH>(a, stream, ev);
-    return launch_pair_v<T, N, VEC_BC, false, false, ZOH>(a, stream, ev);
+    if (a.dt_in) {
+        if constexpr (sizeof(T) == 2 && !ZOH) {
+            if (a.conv_w) return launch_pair_v<T, N, VEC_BC, false, true, false, true>(a, stream, ev);
+            return launch_pair_v<T, N, VEC_BC, false, false, false, true>(a, stream, ev);
+        } else {
+            return VIM_ERR_UNSUPPORTED;
+        }
+    }
+    if (a.conv_w) return launch_pair_v<T, N, VEC_BC, false, true, ZOH, false>(a, stream, ev);
+    if (a.partial_in) return launch_pair_v<T, N, VEC_BC, true, false, ZOH, false>(a, stream, ev);
+    return launch_pair_v<T, N, VEC_BC, false, false, ZOH, false>(a, stream, ev);
 }
 
 // B/C move as 16-byte vectors when their rows allow it and every base is aligned

@@ -231,6 +231,8 @@ struct PairArgs {
     int batch, L, Di, H, W;
     int order;                      // 0: position = step; 1: column-major on H x W
     int chunk, G;                   // tokens per chunk (multiple of kTile), chunks
+    const float *dt_in;             // [2][batch*L] step input per direction and position, or null
+    const float *dt_w;              // [2][Di] its dt_proj weights: delta_raw = dt_in * dt_w
     int zoh;                        // exact zero-order-hold Bbar instead of Delta B
     int fold_reverse;               // pair_combine folds each direction against its order
 };
@@ -287,7 +289,7 @@ constexpr bool bc_vectorizable() { return (N * sizeof(T)) % 16 == 0; }
 // converted to fp32, into the slot.
 // Rows past the end of the chunk and channels past d_inner are zero-filled, so that
 // they act as no-op tokens.
-template <typename T, int N, bool VEC_BC, bool CONV = false, bool ZOH = false>
+template <typename T, int N, bool VEC_BC, bool CONV = false, bool ZOH = false, bool DT = false>
 struct Stager {
     using S = Stage<T, N, CONV>;
     static constexpr int V = Vec<T>::n;                 // elements per 16-byte piece
@@ -331,12 +333,22 @@ struct Stager {
                 if (ok) {
                     const size_t off = row_off(j, r, ch);
                     if (!CONV) cp_async16(S::uv(slot, dir, 0) + so, gu + off, true);
-                    cp_async16(S::uv(slot, dir, 1) + so, gd + off, true);
+                    if (!DT) cp_async16(S::uv(slot, dir, 1) + so, gd + off, true);
                 } else {
                     // outside the data: u = 0 and delta_raw = -1e4, so that Delta =
                     // softplus(-1e4 + bias) = 0 exactly (Abar = 1, Bbar u = 0): a no-op token
                     if (!CONV) *reinterpret_cast<uint4 *>(S::uv(slot, dir, 0) + so) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(S::uv(slot, dir, 1) + so) = pad16<T>(-1.0e4f);
+                    if (!DT) *reinterpret_cast<uint4 *>(S::uv(slot, dir, 1) + so) = pad16<T>(-1.0e4f);
+                }
+            }
+            if constexpr (DT) {
+                // the step input of each row (one value per token; the delta area holds
+                // them as floats), NaN past the data: delta_at turns it into Delta = 0
+                if (threadIdx.x < kTile) {
+                    const int r = threadIdx.x;
+                    float v = __int_as_float(0x7fc00000);
+                    if (r < rows) v = p.dt_in[(size_t)dir * p.batch * p.L + (size_t)b * p.L + position(p, t0 + j * kTile + r)];
+                    reinterpret_cast<float *>(S::uv(slot, dir, 1))[r] = v;
                 }
             }
             if constexpr (CONV) {
@@ -420,6 +432,7 @@ struct ChannelParams {
     float a0, inv_a0;   // A[d][0] and its reciprocal (0 when A[d][0] = 0)
     float D, bias;
     float cw_prev, cw_cur, cw_next, cbias;   // convolution front: taps on x[t-1], x[t], x[t+1]
+    float dtw;          // dt_proj weight of the channel (step input mode)
     bool structured;    // A[d][n] == (n+1) A[d][0] for every n
     bool valid;
 
@@ -427,7 +440,7 @@ struct ChannelParams {
         valid = d < p.Di;
         structured = true;
         A0 = D = bias = a0 = inv_a0 = 0.0f;
-        cw_prev = cw_cur = cw_next = cbias = 0.0f;
+        cw_prev = cw_cur = cw_next = cbias = dtw = 0.0f;
         A = p.A;
         if (!valid) return;
         if (p.conv_w) {
@@ -439,6 +452,7 @@ struct ChannelParams {
             cw_next = dir ? w[0] : w[2];
             cbias = p.conv_b[(size_t)dir * p.Di + d];
         }
+        if (p.dt_w) dtw = p.dt_w[(size_t)dir * p.Di + d];
         A = p.A + ((size_t)dir * p.Di + d) * N;
         a0 = A[0];
 #pragma unroll
@@ -469,10 +483,17 @@ __device__ __forceinline__ float u_of(const T *su, int r, int dl, const ChannelP
     }
 }
 
-// Delta of one staged row (rows past the tile end hold delta_raw = -1e4: Delta = 0)
-template <typename T>
-__device__ __forceinline__ float delta_of(const T *sd, int r, int dl, float bias) {
-    return softplus_io<T>(to_f32(sd[r * kDC + dl]) + bias);
+// Delta of one staged row (rows past the tile end hold delta_raw = -1e4: Delta = 0).
+// In the step-input mode (DT) the row holds the token's x_proj step input s, and
+// delta_raw = s * dt_w[d] (dt_proj); rows past the data hold NaN and give Delta = 0.
+template <typename T, bool DT>
+__device__ __forceinline__ float delta_at(const void *sd, int r, int dl, float bias, float dtw) {
+    if constexpr (DT) {
+        const float s = static_cast<const float *>(sd)[r];
+        return s == s ? softplus_io<T>(fmaf(s, dtw, bias)) : 0.0f;
+    } else {
+        return softplus_io<T>(to_f32(static_cast<const T *>(sd)[r * kDC + dl]) + bias);
+    }
 }
 
 // ----------------------------------------------------------------------------
@@ -483,9 +504,9 @@ __device__ __forceinline__ float delta_of(const T *sd, int r, int dl, float bias
 // Delta summed over the tokens the direction visits after s inside the chunk.  With
 // A_n = (n+1) A_0 the weights are powers of w = exp(A_0 S_s), built by one multiply
 // per state.
-template <typename T, int N, bool FAST, bool DESC, bool CONV, bool ZOH>
+template <typename T, int N, bool FAST, bool DESC, bool CONV, bool ZOH, bool DT>
 __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, const ChannelParams<N> &prm,
-                                           int dl, const T *su, const T *sd, const float *sB) {
+                                           int dl, const T *su, const void *sd, const float *sB) {
     constexpr int NP = N / 2;
     constexpr int kCarrySub = ZOH ? kCarryZohSub : vimscan::kCarrySub;
 #pragma unroll 1
@@ -497,7 +518,7 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
 #pragma unroll
         for (int k = 0; k < kCarrySub; ++k) {
             const int r = walk_row<DESC>(sub * kCarrySub + k);
-            const float dt = delta_of<T>(sd, r, dl, prm.bias);
+            const float dt = delta_at<T, DT>(sd, r, dl, prm.bias, prm.dtw);
             const float u = u_of<T, N, CONV>(su, r, dl, prm);
             if constexpr (!ZOH) {
                 duv[k] = dt * u;
@@ -563,7 +584,7 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
 }
 
 // (the exact hold needs more registers per thread, so fewer CTAs per SM)
-template <typename T, int N, bool VEC_BC, bool CONV, bool ZOH>
+template <typename T, int N, bool VEC_BC, bool CONV, bool ZOH, bool DT = false>
 __global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMinBlocks) pair_carry(PairArgs p) {
     using S = Stage<T, N, CONV>;
     constexpr int NP = N / 2;
@@ -582,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMin
     const bool fast = __all_sync(0xffffffffu, prm.structured);
 
     // the forward direction walks tiles nT-1 .. 0, the backward one 0 .. nT-1
-    Stager<T, N, VEC_BC, CONV, ZOH> st(p, b, t0, tc, d0);
+    Stager<T, N, VEC_BC, CONV, ZOH, DT> st(p, b, t0, tc, d0);
     st.issue(smem, nT - 1, 0);
     st.load_bc(nT - 1, 0);
     st.store_bc(smem);
@@ -605,11 +626,11 @@ __global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMin
             const T *su = S::uv(cur, dir, 0), *sd = S::uv(cur, dir, 1);
             const float *sB = S::bc(cur, dir, 0);
             if (dir == 0) {
-                if (fast) carry_tile<T, N, true, true, CONV, ZOH>(H, Ssum, prm, dl, su, sd, sB);
-                else carry_tile<T, N, false, true, CONV, ZOH>(H, Ssum, prm, dl, su, sd, sB);
+                if (fast) carry_tile<T, N, true, true, CONV, ZOH, DT>(H, Ssum, prm, dl, su, sd, sB);
+                else carry_tile<T, N, false, true, CONV, ZOH, DT>(H, Ssum, prm, dl, su, sd, sB);
             } else {
-                if (fast) carry_tile<T, N, true, false, CONV, ZOH>(H, Ssum, prm, dl, su, sd, sB);
-                else carry_tile<T, N, false, false, CONV, ZOH>(H, Ssum, prm, dl, su, sd, sB);
+                if (fast) carry_tile<T, N, true, false, CONV, ZOH, DT>(H, Ssum, prm, dl, su, sd, sB);
+                else carry_tile<T, N, false, false, CONV, ZOH, DT>(H, Ssum, prm, dl, su, sd, sB);
             }
         }
         if (s + 1 < nT) {
@@ -703,9 +724,9 @@ __device__ __forceinline__ void add_f32(float (&acc)[V], const float *src) {
 // them.  Rows past the tile's end are no-op tokens.  The output of each token goes
 // to the chunk's fp32 partial buffer: stored on the tile's first visit, added on the
 // second (rows past the end only touch unread rows of the buffer).
-template <typename T, int N, bool FAST, bool DESC, bool CONV, bool ZOH>
+template <typename T, int N, bool FAST, bool DESC, bool CONV, bool ZOH, bool DT>
 __device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], const ChannelParams<N> &prm,
-                                          int dl, const T *su, const T *sd, const float *sB,
+                                          int dl, const T *su, const void *sd, const float *sB,
                                           const float *sC, float *ypart) {
     constexpr int NP = N / 2;
 #pragma unroll 1
@@ -716,7 +737,7 @@ __device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], const
 #pragma unroll
         for (int k = 0; k < kSub; ++k) {
             const int r = walk_row<DESC>(sub * kSub + k);
-            const float dt = delta_of<T>(sd, r, dl, prm.bias);
+            const float dt = delta_at<T, DT>(sd, r, dl, prm.bias, prm.dtw);
             uv[k] = u_of<T, N, CONV>(su, r, dl, prm);
             qv[k] = FAST ? ex2(dt * prm.A0) : dt;
             if constexpr (ZOH && FAST)
@@ -890,7 +911,7 @@ struct Finisher {
     }
 };
 
-template <typename T, int N, bool VEC_BC, bool PIN, bool CONV, bool ZOH>
+template <typename T, int N, bool VEC_BC, bool PIN, bool CONV, bool ZOH, bool DT = false>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
     using S = Stage<T, N, CONV>;
     constexpr int NP = N / 2;
@@ -908,7 +929,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
     prm.load(p, dir, d);
     const bool fast = __all_sync(0xffffffffu, prm.structured);
 
-    Stager<T, N, VEC_BC, CONV, ZOH> st(p, b, t0, tc, d0);
+    Stager<T, N, VEC_BC, CONV, ZOH, DT> st(p, b, t0, tc, d0);
     st.issue(smem, 0, nT - 1);
     st.load_bc(0, nT - 1);
 
@@ -952,11 +973,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
             const float *sB = S::bc(cur, dir, 0), *sC = S::bc(cur, dir, 1);
             const bool second = twice > 0;
             if (dir == 0) {
-                if (fast) main_tile<T, N, true, false, CONV, ZOH>(second, h, prm, dl, su, sd, sB, sC, ypart);
-                else main_tile<T, N, false, false, CONV, ZOH>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                if (fast) main_tile<T, N, true, false, CONV, ZOH, DT>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                else main_tile<T, N, false, false, CONV, ZOH, DT>(second, h, prm, dl, su, sd, sB, sC, ypart);
             } else {
-                if (fast) main_tile<T, N, true, true, CONV, ZOH>(second, h, prm, dl, su, sd, sB, sC, ypart);
-                else main_tile<T, N, false, true, CONV, ZOH>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                if (fast) main_tile<T, N, true, true, CONV, ZOH, DT>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                else main_tile<T, N, false, true, CONV, ZOH, DT>(second, h, prm, dl, su, sd, sB, sC, ypart);
             }
         }
         if (s + 1 < nT) {

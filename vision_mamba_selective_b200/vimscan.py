@@ -56,6 +56,11 @@ lib.vim_scan_bidir_bwd_events.argtypes = lib.vim_scan_bidir_bwd.argtypes + [_vp]
 lib.vim_scan_bidir_bwd_events.restype = _i
 lib.vim_scan_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
 lib.vim_scan_bwd_workspace_bytes.restype = _sz
+lib.vim_block_scan.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                               _vp, _sz, _vp, _vp]
+lib.vim_block_scan.restype = _i
+lib.vim_block_workspace_bytes.argtypes = [_i, _i, _i, _i]
+lib.vim_block_workspace_bytes.restype = _sz
 lib.vim_scan_bidir_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
                                        _i, _i, _i, _i, _i, _vp]
 lib.vim_scan_bidir_noalloc.restype = _i
@@ -225,6 +230,35 @@ def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stri
     if st != VIM_OK:
         raise VimScanError(st, "vim_scan_bidir_bwd")
     return out
+
+
+def vim_block_workspace_bytes(batch, L, d_inner, d_state):
+    return int(lib.vim_block_workspace_bytes(batch, L, d_inner, d_state))
+
+
+def vim_block_scan(x, Wx, Wdt, dt_bias, A, D, z, *, conv_w=None, conv_b=None, y=None, workspace=None,
+                   stream=None, events=None):
+    """The Vim block's two S6 modules from their common input x with their own
+    projections (x_proj on the tensor cores, dt_proj inside the scan) and optionally
+    the convolution front; see include/vimscan.h.  bf16 x, z, Wx [2, d_inner, 2N+1];
+    fp32 Wdt, dt_bias, D [2, d_inner], A [2, d_inner, N].  Returns y [batch, L, d_inner].
+    """
+    batch, L, Di = x.shape
+    N = A.shape[-1]
+    if y is None:
+        y = torch.empty_like(x)
+    ws, ws_bytes = _workspace(vim_block_workspace_bytes(batch, L, Di, N), workspace, x.device)
+    st = lib.vim_block_scan(
+        _ptr(x, name="x"), _ptr(conv_w, dtype=torch.float32, name="conv_w"),
+        _ptr(conv_b, dtype=torch.float32, name="conv_b"), _ptr(Wx, dtype=x.dtype, name="Wx"),
+        _ptr(Wdt, dtype=torch.float32, name="Wdt"), _ptr(dt_bias, dtype=torch.float32, name="dt_bias"),
+        _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
+        _ptr(z, dtype=x.dtype, name="z"), _ptr(y, dtype=x.dtype, name="y"),
+        batch, L, Di, N, _dtype_code(x), None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream),
+        None if events is None else _events(events))
+    if st != VIM_OK:
+        raise VimScanError(st, "vim_block_scan")
+    return y
 
 
 def vim_scan_bidir_noalloc(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride=0, stream=None):
