@@ -55,6 +55,8 @@ def parse():
                     help="Vim workloads: time the scan with the fused kernel-3 convolution + SiLU front")
     ap.add_argument("--zoh", action="store_true",
                     help="time the scan with the exact zero-order-hold Bbar instead of Delta B")
+    ap.add_argument("--block", action="store_true",
+                    help="Vim workloads: time vim_block_scan (x_proj + dt_proj + the convolution front + scan)")
     ap.add_argument("--bwd", action="store_true",
                     help="Vim workloads: time the scan's derivative (vim_scan_bidir_bwd) instead")
     return ap.parse_args()
@@ -88,6 +90,26 @@ def profiled_traffic(w):
     if not m or not f or f.group(1) != fp:
         return None
     return int(m.group(1))
+
+
+def block_params(w, seed):
+    """Weights of the block's projections, drawn as the block parity tests draw them:
+    Wx ~ N(0, 1/d_inner) (bf16) [2, d_inner, 2N+1]; dt_proj weights ~ N(0, 0.5) and
+    biases log(expm1(s)), s log-uniform in [1e-3, 1e-1]; the convolution front uniform
+    in +-1/sqrt(3)."""
+    import torch
+
+    g = torch.Generator().manual_seed(seed)
+    Di, N = w.channels, w.d_state
+    Wx = (torch.randn((2, Di, 2 * N + 1), generator=g) / math.sqrt(Di)).to(torch.bfloat16).contiguous()
+    Wdt = (torch.randn((2, Di), generator=g) * 0.5).contiguous()
+    s = torch.exp(math.log(1e-3) + (math.log(1e-1) - math.log(1e-3)) * torch.rand((2, Di), generator=g,
+                                                                                   dtype=torch.float64))
+    dt_bias = torch.log(torch.expm1(s)).float().contiguous()
+    k = 3 ** -0.5
+    cw = ((torch.rand((2, Di, 3), generator=g) * 2 - 1) * k).contiguous()
+    cb = ((torch.rand((2, Di), generator=g) * 2 - 1) * k).contiguous()
+    return dict(Wx=Wx, Wdt=Wdt, dt_bias=dt_bias, conv_w=cw, conv_b=cb)
 
 
 def algorithmic_bwd(w):
@@ -199,7 +221,10 @@ def run_oracle(w, x, threads, zoh=False):
 
     oracle.set_threads(threads)
     t = time.perf_counter()
-    if "dout" in x:
+    if "Wx" in x:
+        oracle.vim_block_scan(x["u"], x["Wx"], x["Wdt"], x["A"], x["D"], x["dt_bias"], x["z"],
+                              conv_w=x["conv_w"], conv_b=x["conv_b"])
+    elif "dout" in x:
         oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], x["dout"])
     elif "conv_w" in x:
         oracle.vim_bidir_conv(x["u"], x["conv_w"], x["conv_b"], x["delta"], x["z"], x["B"], x["C"], x["A"],
@@ -220,7 +245,7 @@ def bwd_dout(w, seed):
     return torch.randn((w.batch, w.tokens, w.channels), generator=g).to(w.torch_dtype()).contiguous()
 
 
-def oracle_sample(w, target_s, conv=False, bwd=False):
+def oracle_sample(w, target_s, conv=False, bwd=False, block=False):
     """A bounded sample of the workload for the oracle: its first batch items and
     first channels at the full sequence length, sized for about ``target_s`` seconds
     of fp64 work on the host cores (calibrated on a small run)."""
@@ -230,6 +255,8 @@ def oracle_sample(w, target_s, conv=False, bwd=False):
     full = wl.make_inputs(w)
     if bwd:
         full["dout"] = bwd_dout(w, w.seed + 2)
+    if block:
+        full.update(block_params(w, w.seed + 3))
     if conv:
         full["conv_w"], full["conv_b"] = conv_params(w, w.seed + 1)
     step = 8
@@ -241,6 +268,8 @@ def oracle_sample(w, target_s, conv=False, bwd=False):
                 x[k] = v[:b, ..., :c].contiguous()
             elif k in ("B", "C"):
                 x[k] = (v[:b] if w.kind == "vim" else v[:, :b]).contiguous()
+            elif k == "Wx":
+                x[k] = v[:, :c, :].contiguous()
             else:
                 x[k] = v[..., :c, :].contiguous() if k in ("A", "conv_w") else v[..., :c].contiguous()
         return w.scaled(batch=b, channels=c), x
@@ -271,7 +300,7 @@ def reference_arm(args, w):
     if rank != 0:
         return
     per_step = min(2.0, 150.0 / max(1, args.steps + args.warmup))
-    s, x, cores = oracle_sample(w, per_step, conv=args.conv, bwd=args.bwd)
+    s, x, cores = oracle_sample(w, per_step, conv=args.conv, bwd=args.bwd, block=args.block)
     for _ in range(args.warmup):
         run_oracle(s, x, cores, args.zoh)
     times = [run_oracle(s, x, cores, args.zoh) for _ in range(args.steps)]
@@ -295,7 +324,7 @@ def reference_arm(args, w):
 
 def workload_name(w, args):
     return (w.name + ("+conv_front" if args.conv else "") + ("+zoh_exact" if args.zoh else "")
-            + ("+derivative" if args.bwd else ""))
+            + ("+derivative" if args.bwd else "") + ("+projections+conv_front" if args.block else ""))
 
 
 def main():
@@ -303,8 +332,10 @@ def main():
     from vision_mamba_selective_b200 import workloads as wl
 
     w = wl.BY_NAME[args.workload]
-    if (args.conv or args.bwd) and w.kind != "vim":
-        raise SystemExit("--conv and --bwd apply to the Vim workloads only")
+    if (args.conv or args.bwd or args.block) and w.kind != "vim":
+        raise SystemExit("--conv, --bwd and --block apply to the Vim workloads only")
+    if args.block and (args.conv or args.zoh or args.bwd or w.dtype != "bf16"):
+        raise SystemExit("--block runs alone, on a bf16 workload")
     if args.bwd and (args.conv or args.zoh):
         raise SystemExit("--bwd covers the plain scan (no --conv, no --zoh)")
     if args.impl == "reference":
@@ -352,6 +383,10 @@ def main():
         ws_bytes = vs.vim_scan_workspace_bytes(1, w.batch, w.H, w.W, w.channels, w.d_state)
     if args.bwd:
         ws_bytes = vs.vim_scan_bwd_workspace_bytes(w.batch, w.L, w.channels, w.d_state, False)
+    if args.block:
+        ws_bytes = vs.vim_block_workspace_bytes(w.batch, w.L, w.channels, w.d_state)
+        blk = block_params(w, w.seed + 3)
+        params.update({k: v.to(dev) for k, v in blk.items()})
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     fn = vs.vim_scan_bidir if w.kind == "vim" else vs.vmamba_cross_scan4
     if args.conv:
@@ -360,6 +395,12 @@ def main():
 
     def step(i, events=None):
         s = sets[i % nsets]
+        if args.block:
+            # u holds x, the block's input; B, C and delta come from the projections
+            vs.vim_block_scan(s["u"], params["Wx"], params["Wdt"], params["dt_bias"], params["A"], params["D"],
+                              s["z"], conv_w=params["conv_w"], conv_b=params["conv_b"], y=s["y"], workspace=ws,
+                              events=events)
+            return
         if args.bwd:
             vs.vim_scan_bidir_bwd(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"],
                                   params["delta_bias"], s["dout"], workspace=ws, out=s["out"], events=events)
@@ -400,14 +441,19 @@ def main():
     # ---- per-kernel times (same launches plus event records), after the timed region
     kernels_per_pair = 3
     pairs = 1 if w.kind == "vim" else 2
-    nev = 4 if args.bwd else 1 + kernels_per_pair * pairs
+    nev = 4 if args.bwd else (5 if args.block else 1 + kernels_per_pair * pairs)
     prof_steps = min(args.steps, 200)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(prof_steps)]
     for i in range(prof_steps):
         step(i, events=evs[i])
     torch.cuda.synchronize()
     per_kernel = {}
-    if args.bwd:
+    if args.block:
+        for a, name in enumerate(["xproj", "pair_carry", "pair_combine", "pair_main"], start=1):
+            t = [evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(prof_steps)]
+            per_kernel[name] = sum(t) / len(t)
+        launches_per_step = 1 + (3 if w.tokens > 256 else 1)
+    elif args.bwd:
         for a, name in enumerate(["summaries", "bwd_main", "reductions"], start=1):
             t = [evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(prof_steps)]
             per_kernel[name] = sum(t) / len(t)
@@ -468,7 +514,7 @@ def main():
     roofline = {
         "bound": "alu", "kernel": main_name, "achieved": achieved_ops, "peak": peak_ops,
         "unit": "Tops/s", "frac": achieved_ops / peak_ops,
-        "traffic": None if (args.bwd or args.conv or args.zoh) else profiled_traffic(w),
+        "traffic": None if (args.bwd or args.conv or args.zoh or args.block) else profiled_traffic(w),
         "algorithmic_bytes": nbytes,
         "ops_per_launch": ops, "ms_per_launch": main_ms,
         "peak_basis": f"{SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x {pk['sm_max_mhz']:.0f} MHz",
@@ -477,9 +523,19 @@ def main():
         "hbm_peak_gbs": pk["hbm_gbs"], "peak_source": pk["source"],
     }
 
+    projection = None
+    if args.block:
+        # x_proj: x read once, B and C (bf16) and the step input (fp32) written per pathway
+        M = w.batch * w.tokens
+        pb = M * w.channels * 2 + 2 * (2 * M * w.d_state * 2 + M * 4) + 2 * w.channels * (2 * w.d_state + 1) * 2
+        pms = per_kernel["xproj"]
+        projection = {"kernel": "xproj_kernel", "bound": "hbm", "ms_per_launch": pms, "algorithmic_bytes": pb,
+                      "achieved_gbs": pb / (pms * 1e-3) / 1e9, "peak_gbs": pk["hbm_gbs"],
+                      "frac": pb / (pms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        s, x, cores = oracle_sample(w, 5.0, conv=args.conv, bwd=args.bwd)
+        s, x, cores = oracle_sample(w, 5.0, conv=args.conv, bwd=args.bwd, block=args.block)
         sec = run_oracle(s, x, cores, args.zoh)
         cpu = {"value": s.tok_ch / sec, "unit": "tok*ch/s", "cores": cores, "kind": "oracle",
                "sample": f"{s.batch} of {w.batch} batch items x {s.channels} of {w.channels} channels "
@@ -499,6 +555,7 @@ def main():
             "hbm_gbs": roofline["hbm_gbs_whole_step"], "hbm_frac": roofline["hbm_frac_whole_step"],
             "kernel_ms": per_kernel,
             "roofline": roofline,
+            "projection": projection,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tok*ch/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
