@@ -458,8 +458,8 @@ def main():
             t = [evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(prof_steps)]
             per_kernel[name] = sum(t) / len(t)
         # pair_carry, pair_combine, adj_carry, pair_combine (more than one chunk of
-        # 32 tokens), bwd_main, two dB/dC reductions, three two-pass column sums
-        launches_per_step = (4 if w.tokens > 32 else 0) + 1 + 2 + 6
+        # 32 tokens), bwd_main, two dB/dC reductions, one two-pass column sum
+        launches_per_step = (4 if w.tokens > 32 else 0) + 1 + 2 + 2
     else:
         names = ["pair_carry", "pair_combine", "pair_main"]
         for p in range(pairs):

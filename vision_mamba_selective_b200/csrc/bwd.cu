@@ -14,7 +14,7 @@ namespace {
 
 struct BwdPlan {
     int G, nblk, nsets;
-    size_t off_hloc, off_ssum, off_gloc, off_gsum, off_dA, off_dD, off_db, off_dBp, off_dCp, off_tmp, total;
+    size_t off_hloc, off_ssum, off_gloc, off_gsum, off_par, off_dBp, off_dCp, off_tmp, total;
 };
 
 BwdPlan bwd_plan(int batch, int L, int Di, int N, int separate_bc) {
@@ -24,16 +24,14 @@ BwdPlan bwd_plan(int batch, int L, int Di, int N, int separate_bc) {
     pl.nblk = (Di + ch - 1) / ch;
     pl.nsets = separate_bc ? 2 : 1;
     const size_t units = (size_t)batch * pl.G * 2 * Di;      // (b, chunk, dir, channel)
-    const size_t cols = std::max((size_t)2 * Di * N, (size_t)2 * Di);
+    const size_t cols = (size_t)2 * Di * (N + 2);        // [dA | dD | d delta_bias]
     size_t o = 0;
     auto take = [&](size_t bytes) { const size_t at = o; o += round_up(bytes); return at; };
     pl.off_hloc = take(units * N * 4);
     pl.off_ssum = take(units * 4);
     pl.off_gloc = take(units * N * 4);
     pl.off_gsum = take(units * 4);
-    pl.off_dA = take(units * N * 4);
-    pl.off_dD = take(units * 4);
-    pl.off_db = take(units * 4);
+    pl.off_par = take(units * (N + 2) * 4);
     pl.off_dBp = take((size_t)pl.nsets * batch * L * pl.nblk * N * 4);
     pl.off_dCp = take((size_t)pl.nsets * batch * L * pl.nblk * N * 4);
     pl.off_tmp = take((size_t)kReduceParts * cols * 4);
@@ -41,12 +39,14 @@ BwdPlan bwd_plan(int batch, int L, int Di, int N, int separate_bc) {
     return pl;
 }
 
-// column sums of rows x cols fp32 into out (two passes through tmp)
-vim_status reduce_cols(const float *src, float *tmp, float *out, int rows, int cols, cudaStream_t stream) {
+// column sums of the per-chunk rows [dA | dD | d delta_bias] (two passes through tmp)
+vim_status reduce_params(const float *par, float *tmp, float *dA, float *dD, float *dbias, int rows, int Di, int N,
+                         cudaStream_t stream) {
+    const int nA = 2 * Di * N, nD = 2 * Di, cols = nA + 2 * nD;
     const dim3 g1((cols + 255) / 256, kReduceParts);
-    bwd_reduce_cols1<<<g1, 256, 0, stream>>>(src, tmp, rows, cols);
+    bwd_reduce_cols1<<<g1, 256, 0, stream>>>(par, tmp, rows, cols);
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
-    bwd_reduce_cols2<<<(cols + 255) / 256, 256, 0, stream>>>(tmp, out, cols);
+    bwd_reduce_cols2<<<(cols + 255) / 256, 256, 0, stream>>>(tmp, dA, dD, dbias, nA, nD);
     return cudaGetLastError() == cudaSuccess ? VIM_OK : VIM_ERR_CUDA;
 }
 
@@ -104,9 +104,7 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
         if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     }
     const int prow = a.batch * a.G;
-    if (reduce_cols(a.dA_part, tmp, dA, prow, 2 * a.Di * N, stream) != VIM_OK) return VIM_ERR_CUDA;
-    if (reduce_cols(a.dD_part, tmp, dD, prow, 2 * a.Di, stream) != VIM_OK) return VIM_ERR_CUDA;
-    if (reduce_cols(a.dbias_part, tmp, dbias, prow, 2 * a.Di, stream) != VIM_OK) return VIM_ERR_CUDA;
+    if (reduce_params(a.par, tmp, dA, dD, dbias, prow, a.Di, N, stream) != VIM_OK) return VIM_ERR_CUDA;
     return rec(ev, 3, stream) ? VIM_OK : VIM_ERR_CUDA;
 }
 
@@ -182,9 +180,7 @@ vim_status vim_scan_bidir_bwd_events(const void *u, const void *delta, const voi
     a.dC_part[0] = reinterpret_cast<float *>(ws + pl.off_dCp);
     a.dB_part[1] = separate ? a.dB_part[0] + set_elems : a.dB_part[0];
     a.dC_part[1] = separate ? a.dC_part[0] + set_elems : a.dC_part[0];
-    a.dA_part = reinterpret_cast<float *>(ws + pl.off_dA);
-    a.dD_part = reinterpret_cast<float *>(ws + pl.off_dD);
-    a.dbias_part = reinterpret_cast<float *>(ws + pl.off_db);
+    a.par = reinterpret_cast<float *>(ws + pl.off_par);
     a.hin = reinterpret_cast<const float *>(ws + pl.off_hloc);
     a.gloc = reinterpret_cast<float *>(ws + pl.off_gloc);
     a.gsum = reinterpret_cast<float *>(ws + pl.off_gsum);

@@ -47,8 +47,8 @@ struct BwdArgs {
     const float *A, *D, *bias;          // [2][Di][N], [2][Di], [2][Di]
     void *du, *ddelta, *dz;             // [batch, L, Di] (dz null when z is)
     float *dB_part[2], *dC_part[2];     // [batch][L][nblk][N] per B/C set ([1] = [0] when shared)
-    float *dA_part;                     // [batch][G][2][Di][N]
-    float *dD_part, *dbias_part;        // [batch][G][2][Di]
+    float *par;                         // per-chunk sums over tokens, one row per (batch, chunk):
+                                        // [dA: 2*Di*N | dD: 2*Di | d delta_bias: 2*Di]
     const float *hin;                   // [batch][G][2][Di][N] h entering each chunk (direction order)
     float *gloc;                        // [batch][G][2][Di][N] adjoint summaries, then adjoint entering
     float *gsum;                        // [batch][G][2][Di] chunk Delta sums
@@ -373,9 +373,12 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
     }
     if (th.valid) {
 #pragma unroll
-        for (int j = 0; j < NT; ++j) p.dA_part[th.cbase * N + th.j0 + j] = dA[j];
-        if (th.q == 0) p.dD_part[th.cbase] = dD;
-        if (th.q == kDdLane) p.dbias_part[th.cbase] = dbias;
+        // row (b, c) of par; cbase = (row * 2 + dir) * Di + d
+        const size_t row = th.cbase / ((size_t)2 * p.Di), col = th.cbase % ((size_t)2 * p.Di);
+        float *pr = p.par + row * ((size_t)2 * p.Di * (N + 2));
+        for (int j = 0; j < NT; ++j) pr[col * N + th.j0 + j] = dA[j];
+        if (th.q == 0) pr[(size_t)2 * p.Di * N + col] = dD;
+        if (th.q == kDdLane) pr[(size_t)2 * p.Di * (N + 1) + col] = dbias;
     }
 }
 
@@ -517,12 +520,17 @@ __global__ void __launch_bounds__(256) bwd_reduce_cols1(const float *src, float 
     for (; r < r1; ++r) a0 += src[(int64_t)r * cols + col];
     tmp[(int64_t)part * cols + col] = (a0 + a1) + (a2 + a3);
 }
-__global__ void __launch_bounds__(256) bwd_reduce_cols2(const float *tmp, float *out, int cols) {
+// second pass; the columns are [dA: 2*Di*N | dD: 2*Di | d delta_bias: 2*Di]
+__global__ void __launch_bounds__(256) bwd_reduce_cols2(const float *tmp, float *dA, float *dD, float *dbias,
+                                                        int nA, int nD) {
+    const int cols = nA + 2 * nD;
     const int col = blockIdx.x * blockDim.x + threadIdx.x;
     if (col >= cols) return;
     float acc = 0.0f;
     for (int part = 0; part < kReduceParts; ++part) acc += tmp[(int64_t)part * cols + col];
-    out[col] = acc;
+    if (col < nA) dA[col] = acc;
+    else if (col < nA + nD) dD[col - nA] = acc;
+    else dbias[col - nA - nD] = acc;
 }
 
 }  // namespace
