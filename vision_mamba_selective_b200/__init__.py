@@ -8,7 +8,9 @@ GPU; the first use of a scan entry point loads the library and fails loudly if i
 missing.
 """
 
-__all__ = ["vim_scan_bidir", "vmamba_cross_scan4", "cross_merge4", "vim_scan_workspace_bytes"]
+__all__ = ["vim_scan_bidir", "vmamba_cross_scan4", "cross_merge4", "vim_scan_workspace_bytes",
+           "vim_scan_bidir_conv", "vim_scan_bidir_bwd", "vim_scan_bwd_workspace_bytes", "vim_block_scan",
+           "vim_block_workspace_bytes", "vim_scan_bidir_noalloc"]
 
 
 def __getattr__(name):
