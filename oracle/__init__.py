@@ -61,6 +61,7 @@ class Oracle:
         lib.oracle_vim_bidir_conv.argtypes = [_D, _D, _D, _D, _D, _D, _D, ctypes.c_int64, _D, _D, _D, _D] + [ctypes.c_int] * 6
         lib.oracle_s6_direction_bwd.argtypes = [_D] * 7 + [_I64] + [_D] * 8 + [ctypes.c_int] * 5
         lib.oracle_vim_bidir_bwd.argtypes = [_D, _D, _D, _D, _D, ctypes.c_int64] + [_D] * 12 + [ctypes.c_int] * 5
+        lib.oracle_cross_scan4_bwd.argtypes = [_D] * 17 + [ctypes.c_int] * 6
         lib.oracle_xproj.argtypes = [_D, _D, _D, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
@@ -147,6 +148,29 @@ class Oracle:
                                            batch, L, Di, N, int(bool(delta_is_raw)))
         if rc:
             raise ValueError("oracle_vim_bidir_bwd: bad sizes")
+        return out
+
+    def cross_scan4_bwd(self, u, delta, z, B, C, A, D, bias, dout, *, delta_is_raw=True):
+        """Derivatives of cross_scan4 (first-order Bbar) for the loss sum(dout * y).
+
+        u, delta, z, dout: [batch, H, W, Ci]; B, C: [4, batch, H*W, N]; A [4, Ci, N];
+        D, bias [4, Ci].  Returns a dict of fp64 arrays shaped like the inputs: du,
+        ddelta, dz (None without a gate), dB, dC, dA, dD, dbias.
+        """
+        u, delta, z, B, C, A, D, bias, dout = map(_f64, (u, delta, z, B, C, A, D, bias, dout))
+        batch, H, W, Ci = u.shape
+        N = B.shape[-1]
+        if bias is None:
+            bias = np.zeros((4, Ci))
+        out = dict(du=np.zeros(u.shape), ddelta=np.zeros(u.shape), dz=np.zeros(u.shape) if z is not None else None,
+                   dB=np.zeros(B.shape), dC=np.zeros(C.shape), dA=np.zeros((4, Ci, N)), dD=np.zeros((4, Ci)),
+                   dbias=np.zeros((4, Ci)))
+        rc = self.lib.oracle_cross_scan4_bwd(_p(u), _p(delta), _p(z), _p(B), _p(C), _p(A), _p(D), _p(bias), _p(dout),
+                                             _p(out["du"]), _p(out["ddelta"]), _p(out["dz"]), _p(out["dB"]),
+                                             _p(out["dC"]), _p(out["dA"]), _p(out["dD"]), _p(out["dbias"]),
+                                             batch, H, W, Ci, N, int(bool(delta_is_raw)))
+        if rc:
+            raise ValueError("oracle_cross_scan4_bwd: bad sizes")
         return out
 
     def xproj(self, u, Wx):
@@ -300,6 +324,10 @@ def vim_bidir_bwd(*a, **k):
 
 def xproj(*a, **k):
     return default().xproj(*a, **k)
+
+
+def cross_scan4_bwd(*a, **k):
+    return default().cross_scan4_bwd(*a, **k)
 
 
 def vim_block_scan(*a, **k):

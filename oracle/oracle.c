@@ -508,3 +508,52 @@ int oracle_xproj(const double *u, const double *Wx, double *P, int64_t M, int Di
         }
     return 0;
 }
+
+/*
+ * Derivative of oracle_cross_scan4 (first-order Bbar) for ell = sum dout * y, with
+ * y = (sum_k y_k) * silu(z): dl/dz = dout (sum_k y_k) silu'(z), and each of the four
+ * CS-Traverse directions sees dl/dy_k = dout silu(z) at the grid positions it visits.
+ *   dout : [batch, H*W, Ci].  Outputs (overwritten): du, ddelta, dz [batch, H*W, Ci]
+ *   (dz untouched when z is NULL); dB, dC [4, batch, H*W, N] (grid order, per
+ *   direction); dA [4, Ci, N]; dD, dbias [4, Ci].
+ */
+int oracle_cross_scan4_bwd(const double *u, const double *delta, const double *z,
+                           const double *B, const double *C,
+                           const double *A, const double *D, const double *bias, const double *dout,
+                           double *du, double *ddelta, double *dz, double *dB, double *dC,
+                           double *dA, double *dD, double *dbias,
+                           int batch, int H, int W, int Ci, int N, int delta_is_raw)
+{
+    if (H < 0 || W < 0 || batch < 0 || Ci < 0 || N < 1) return -1;
+    int64_t L = (int64_t)H * W;
+    int64_t n_act = (int64_t)batch * L * Ci, bc = (int64_t)batch * L * N;
+    double *dy = (double *)malloc((size_t)(n_act > 0 ? n_act : 1) * sizeof(double));
+    int64_t *order = (int64_t *)malloc((size_t)(L > 0 ? L : 1) * sizeof(int64_t));
+    if (!dy || !order) { free(dy); free(order); return -1; }
+    for (int64_t i = 0; i < n_act; ++i) { du[i] = 0.0; ddelta[i] = 0.0; }
+    for (int64_t i = 0; i < 4 * bc; ++i) { dB[i] = 0.0; dC[i] = 0.0; }
+    for (int64_t i = 0; i < 4 * (int64_t)Ci * N; ++i) dA[i] = 0.0;
+    for (int64_t i = 0; i < 4 * (int64_t)Ci; ++i) { dD[i] = 0.0; dbias[i] = 0.0; }
+    int rc = 0;
+    if (z) {
+        double *ys = (double *)malloc((size_t)(n_act > 0 ? n_act : 1) * sizeof(double));
+        if (!ys) { free(dy); free(order); return -1; }
+        rc |= oracle_cross_scan4(u, delta, NULL, B, C, A, D, bias, ys, batch, H, W, Ci, N, delta_is_raw, 0);
+        for (int64_t i = 0; i < n_act; ++i) {
+            dz[i] = dout[i] * ys[i] * silu_grad(z[i]);
+            dy[i] = dout[i] * silu(z[i]);
+        }
+        free(ys);
+    } else {
+        for (int64_t i = 0; i < n_act; ++i) dy[i] = dout[i];
+    }
+    for (int k = 0; k < 4; ++k) {
+        rc |= oracle_cross_order(k, H, W, order);
+        rc |= oracle_s6_direction_bwd(u, delta, B + k * bc, C + k * bc, A + (int64_t)k * Ci * N,
+                                      D + (int64_t)k * Ci, bias + (int64_t)k * Ci, order, dy, du, ddelta,
+                                      dB + k * bc, dC + k * bc, dA + (int64_t)k * Ci * N, dD + (int64_t)k * Ci,
+                                      dbias + (int64_t)k * Ci, batch, (int)L, Ci, N, delta_is_raw);
+    }
+    free(dy); free(order);
+    return rc ? -1 : 0;
+}

@@ -603,6 +603,34 @@ def pin_block_scan_composition(orc):
     np.testing.assert_allclose(y0, ref0, rtol=1e-11, atol=1e-11)
 
 
+def pin_cross_bwd_finite_differences(orc):
+    """Every derivative of the four-direction scan against central finite differences
+    of the forward oracle's loss sum(dout * y) on a 2 x 3 grid (H != W, so a transposed
+    traversal cannot pass), with per-direction B, C, A, D and bias (sections "1.
+    Cross-Scan Traversal" to "3. Cross-Merge Reversal")."""
+    rng = _rng(121)
+    b, H, W, c, N = 1, 2, 3, 2, 2
+    x = dict(u=rng.normal(size=(b, H, W, c)), delta=rng.normal(size=(b, H, W, c)) * 0.8,
+             z=rng.normal(size=(b, H, W, c)), B=rng.normal(size=(4, b, H * W, N)),
+             C=rng.normal(size=(4, b, H * W, N)), A=-rng.uniform(0.2, 2.0, size=(4, c, N)),
+             D=rng.normal(size=(4, c)), bias=rng.normal(size=(4, c)))
+    dout = rng.normal(size=(b, H, W, c))
+    loss = lambda **o: float(np.sum(dout * orc.cross_scan4(*[{**x, **o}[k] for k in
+                                                               ("u", "delta", "z", "B", "C", "A", "D", "bias")])))
+    g = orc.cross_scan4_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["bias"], dout)
+    for name, key in (("u", "du"), ("delta", "ddelta"), ("z", "dz"), ("B", "dB"), ("C", "dC"), ("A", "dA"),
+                      ("D", "dD"), ("bias", "dbias")):
+        arr, eps = x[name], 1e-6
+        fd = np.zeros_like(arr)
+        for i in np.ndindex(arr.shape):
+            up, dn = arr.copy(), arr.copy()
+            up[i] += eps
+            dn[i] -= eps
+            fd[i] = (loss(**{name: up}) - loss(**{name: dn})) / (2 * eps)
+        err = np.max(np.abs(fd - g[key])) / np.max(np.abs(fd))
+        assert err < 1e-7, (name, err)
+
+
 ALL_PINS = [
     pin_delta_zero,
     pin_constant_input_geometric,
@@ -624,5 +652,6 @@ ALL_PINS = [
     pin_bwd_finite_differences,
     pin_bwd_homogeneity,
     pin_xproj_is_matmul,
+    pin_cross_bwd_finite_differences,
     pin_block_scan_composition,
 ]

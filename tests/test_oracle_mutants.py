@@ -61,6 +61,8 @@ MUTANTS = {
     "bwd_dy_ungated": ("dy[i] = dout[i] * silu(z[i]);", "dy[i] = dout[i];"),
     "xproj_weight_transposed": ("acc += u[m * Di + d] * Wx[(int64_t)d * NO + j];",
                                 "acc += u[m * Di + d] * Wx[(int64_t)j * Di + d];"),
+    "cross_bwd_same_order": ("rc |= oracle_cross_order(k, H, W, order);\n        rc |= oracle_s6_direction_bwd",
+                             "rc |= oracle_cross_order(0, H, W, order);\n        rc |= oracle_s6_direction_bwd"),
     "zoh_sign": ("return expm1(dt * An) / An * Bn;", "return expm1(-dt * An) / An * Bn;"),
 }
 
