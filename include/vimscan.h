@@ -211,6 +211,28 @@ vim_status vim_scan_bidir_bwd(const void *u, const void *delta, const void *z,
                               int batch, int L, int d_inner, int d_state, vim_dtype dt,
                               void *workspace, size_t workspace_bytes, cudaStream_t stream);
 size_t vim_scan_bwd_workspace_bytes(int batch, int L, int d_inner, int d_state, int separate_bc);
+/*
+ * Derivative of vmamba_cross_scan4 (first-order Bbar) for a loss with derivative `dout`
+ * with respect to y: dl/dz = dout (sum_k y_k) silu'(z), and each CS-Traverse direction
+ * runs the chain rule of its recurrence with dl/dy_k = dout silu(z) at the grid
+ * positions it visits (sections "1. Cross-Scan Traversal" to "3. Cross-Merge
+ * Reversal").
+ *
+ *   u, delta, z, B, C, A, D, delta_bias : the forward call's inputs and layouts.
+ *   dout, du, ddelta, dz : [batch, H, W, channels] (dt); dz NULL exactly when z is.
+ *   dB, dC : fp32 [4, batch, H*W, d_state], grid order like B and C.
+ *   dA [4, channels, d_state], dD [4, channels], ddelta_bias [4, channels] : fp32.
+ *   workspace : vmamba_cross_scan4_bwd_workspace_bytes(...) bytes, 256-byte aligned.
+ */
+vim_status vmamba_cross_scan4_bwd(const void *u, const void *delta, const void *z,
+                                  const void *B, const void *C,
+                                  const float *A, const float *D, const float *delta_bias,
+                                  const void *dout, void *du, void *ddelta, void *dz,
+                                  float *dB, float *dC, float *dA, float *dD, float *ddelta_bias,
+                                  int batch, int H, int W, int channels, int d_state, vim_dtype dt,
+                                  void *workspace, size_t workspace_bytes, cudaStream_t stream);
+size_t vmamba_cross_scan4_bwd_workspace_bytes(int batch, int H, int W, int channels, int d_state);
+
 /* vim_scan_bidir_bwd plus 4 CUDA events (caller-created, or NULL for none) recorded
  * before the chunk summaries, after them, after the main derivative kernel and at
  * the end, for per-phase times. */

@@ -38,6 +38,7 @@ def test_header_declares_the_boundary():
                           "vim_scan_bidir_ex", "vmamba_cross_scan4_ex",
                           "vim_scan_bidir_bwd", "vim_scan_bwd_workspace_bytes", "vim_scan_bidir_bwd_events",
                           "vim_block_scan", "vim_block_workspace_bytes",
+                          "vmamba_cross_scan4_bwd", "vmamba_cross_scan4_bwd_workspace_bytes",
                           "vim_scan_workspace_bytes", "vim_status_string"}, names
 
 

@@ -135,3 +135,63 @@ def test_bwd_full_size(vs):
     torch.cuda.synchronize()
     want = oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], dout)
     check_all("bwd_full", got, want, torch.bfloat16, sum_tol=1e-3)
+
+
+# ---------------------------------------------------------------------------
+# the four-direction cross-scan
+# ---------------------------------------------------------------------------
+def cross_inputs(batch, H, W, Ch, N, dtype, seed, generic_A=False):
+    g = torch.Generator().manual_seed(seed)
+    r = lambda *s, std=1.0: torch.randn(s, generator=g) * std
+    u, dr, z, dout = r(batch, H, W, Ch), r(batch, H, W, Ch, std=0.5), r(batch, H, W, Ch), r(batch, H, W, Ch)
+    B, C = r(4, batch, H * W, N), r(4, batch, H * W, N)
+    if generic_A:
+        A = -(0.05 + 3 * torch.rand((4, Ch, N), generator=g))
+    else:
+        A = -torch.arange(1, N + 1, dtype=torch.float32).repeat(4, Ch, 1)
+    D = r(4, Ch)
+    s = torch.exp(np.log(1e-3) + (np.log(1e-1) - np.log(1e-3)) * torch.rand((4, Ch), generator=g, dtype=torch.float64))
+    bias = torch.log(torch.expm1(s)).float()
+    t = lambda x: x.to(dtype).contiguous()
+    return dict(u=t(u), delta=t(dr), z=t(z), dout=t(dout), B=t(B), C=t(C), A=A.contiguous(), D=D.contiguous(),
+                bias=bias.contiguous())
+
+
+CROSS_CASES = [
+    # batch, H, W, C, N, dtype, generic_A, gate
+    (1, 1, 1, 16, 16, torch.float32, False, True),
+    (1, 3, 5, 16, 16, torch.float32, False, True),
+    (2, 5, 3, 24, 8, torch.float32, True, True),
+    (1, 7, 40, 64, 16, torch.float32, False, True),     # 280 tokens: several 32-token chunks
+    (1, 40, 7, 32, 4, torch.float32, True, False),
+    (2, 16, 16, 64, 16, torch.bfloat16, False, True),
+]
+
+
+@pytest.mark.parametrize("case", CROSS_CASES, ids=lambda c: f"b{c[0]}_{c[1]}x{c[2]}_C{c[3]}_N{c[4]}_"
+                         f"{str(c[5])[6:]}{'_genA' if c[6] else ''}{'' if c[7] else '_nogate'}")
+def test_cross_bwd_small(vs, case):
+    batch, H, W, Ch, N, dtype, gen, gate = case
+    x = cross_inputs(batch, H, W, Ch, N, dtype, seed=H * 17 + W, generic_A=gen)
+    c = lambda k: x[k].cuda()
+    got = vs.vmamba_cross_scan4_bwd(c("u"), c("delta"), c("z") if gate else None, c("B"), c("C"), c("A"), c("D"),
+                                    c("bias"), c("dout"))
+    torch.cuda.synchronize()
+    want = oracle.cross_scan4_bwd(x["u"], x["delta"], x["z"] if gate else None, x["B"], x["C"], x["A"], x["D"],
+                                  x["bias"], x["dout"])
+    check_all(f"cross_bwd_{case}", got, want, dtype)
+
+
+def test_cross_bwd_full_size(vs):
+    """The 64 x 64 VMamba workload (bf16, batch 16, 192 channels) against the oracle."""
+    w = wl.BY_NAME["vmamba_64x64_bf16"]
+    x = wl.make_inputs(w)
+    g = torch.Generator().manual_seed(778)
+    dout = torch.randn(x["u"].shape, generator=g).to(x["u"].dtype)
+    oracle.set_threads(max(1, len(os.sched_getaffinity(0))))
+    d = {k: v.cuda() for k, v in x.items()}
+    got = vs.vmamba_cross_scan4_bwd(d["u"], d["delta"], d["z"], d["B"], d["C"], d["A"], d["D"], d["delta_bias"],
+                                    dout.cuda())
+    torch.cuda.synchronize()
+    want = oracle.cross_scan4_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], dout)
+    check_all("cross_bwd_full", got, want, torch.bfloat16, sum_tol=1e-3)

@@ -215,4 +215,97 @@ vim_status vim_scan_bidir_bwd(const void *u, const void *delta, const void *z, c
                                      workspace_bytes, stream, nullptr);
 }
 
+size_t vmamba_cross_scan4_bwd_workspace_bytes(int batch, int H, int W, int channels, int d_state) {
+    if (batch <= 0 || H <= 0 || W <= 0 || channels <= 0 || d_state <= 0) return 0;
+    const int L = H * W;
+    return bwd_plan(batch, L, channels, d_state, 1).total + 3 * round_up((size_t)batch * L * channels * 4);
+}
+
+vim_status vmamba_cross_scan4_bwd(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                                  const float *A, const float *D, const float *delta_bias, const void *dout,
+                                  void *du, void *ddelta, void *dz, float *dB, float *dC, float *dA, float *dD,
+                                  float *ddelta_bias, int batch, int H, int W, int channels, int d_state,
+                                  vim_dtype dt, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (H < 0 || W < 0) return VIM_ERR_INVALID_ARG;
+    if ((int64_t)H * W > INT32_MAX) return VIM_ERR_UNSUPPORTED;
+    const int L = H * W;
+    vim_status st = check_common(batch, L, channels, d_state, dt);
+    if (st != VIM_OK) return st;
+    if ((z == nullptr) != (dz == nullptr)) return VIM_ERR_INVALID_ARG;
+    if (!A || !D || !delta_bias || !dA || !dD || !ddelta_bias) return VIM_ERR_INVALID_ARG;
+    if (!aligned_to(A, 4) || !aligned_to(D, 4) || !aligned_to(delta_bias, 4) || !aligned_to(dA, 4) ||
+        !aligned_to(dD, 4) || !aligned_to(ddelta_bias, 4))
+        return VIM_ERR_INVALID_ARG;
+    const size_t es = elem_size(dt);
+    if (batch == 0 || L == 0 || channels == 0) {
+        if (cudaMemsetAsync(dA, 0, sizeof(float) * 4 * (size_t)channels * d_state, stream) != cudaSuccess ||
+            cudaMemsetAsync(dD, 0, sizeof(float) * 4 * (size_t)channels, stream) != cudaSuccess ||
+            cudaMemsetAsync(ddelta_bias, 0, sizeof(float) * 4 * (size_t)channels, stream) != cudaSuccess)
+            return VIM_ERR_CUDA;
+        return VIM_OK;
+    }
+    if (!u || !delta || !B || !C || !dout || !du || !ddelta || !dB || !dC) return VIM_ERR_INVALID_ARG;
+    if (!aligned16(u) || !aligned16(delta) || !aligned_to(B, es) || !aligned_to(C, es) || !aligned_to(dout, es) ||
+        !aligned_to(du, es) || !aligned_to(ddelta, es) || (z && !aligned_to(z, es)) || (dz && !aligned_to(dz, es)) ||
+        !aligned_to(dB, 4) || !aligned_to(dC, 4))
+        return VIM_ERR_INVALID_ARG;
+    const BwdPlan pl = bwd_plan(batch, L, channels, d_state, 1);
+    const size_t acc_bytes = round_up((size_t)batch * L * channels * 4);
+    if (!workspace || workspace_bytes < pl.total + 3 * acc_bytes || !aligned_to(workspace, kAlign))
+        return VIM_ERR_WORKSPACE;
+    char *ws = static_cast<char *>(workspace);
+    float *acc = reinterpret_cast<float *>(ws + pl.total);
+    const size_t bc = (size_t)batch * L * d_state;               // elements per direction of B, C
+    const size_t set_elems = (size_t)batch * L * pl.nblk * d_state;
+
+    vim_status rc = VIM_OK;
+    for (int pair = 0; pair < 2 && rc == VIM_OK; ++pair) {
+        BwdArgs a;
+        std::memset(&a, 0, sizeof(a));
+        a.u = u; a.delta = delta; a.z = z; a.dout = dout;
+        for (int k = 0; k < 2; ++k) {
+            a.B[k] = static_cast<const char *>(B) + (2 * pair + k) * bc * es;
+            a.C[k] = static_cast<const char *>(C) + (2 * pair + k) * bc * es;
+        }
+        a.A = A + (size_t)2 * pair * channels * d_state;
+        a.D = D + (size_t)2 * pair * channels;
+        a.bias = delta_bias + (size_t)2 * pair * channels;
+        a.du = du; a.ddelta = ddelta; a.dz = dz;
+        a.dB_part[0] = reinterpret_cast<float *>(ws + pl.off_dBp);
+        a.dC_part[0] = reinterpret_cast<float *>(ws + pl.off_dCp);
+        a.dB_part[1] = a.dB_part[0] + set_elems;
+        a.dC_part[1] = a.dC_part[0] + set_elems;
+        a.par = reinterpret_cast<float *>(ws + pl.off_par);
+        a.hin = reinterpret_cast<const float *>(ws + pl.off_hloc);
+        a.gloc = reinterpret_cast<float *>(ws + pl.off_gloc);
+        a.gsum = reinterpret_cast<float *>(ws + pl.off_gsum);
+        a.batch = batch; a.L = L; a.Di = channels; a.G = pl.G; a.nblk = pl.nblk;
+        a.separate_bc = 1;
+        a.order = pair; a.H = H; a.W = W;
+        a.stage = pair + 1;                  // the row pair leaves partials, the column pair finishes
+        a.acc_y = acc;
+        a.acc_du = reinterpret_cast<float *>(ws + pl.total + acc_bytes);
+        a.acc_dd = reinterpret_cast<float *>(ws + pl.total + 2 * acc_bytes);
+
+        PairArgs f;
+        std::memset(&f, 0, sizeof(f));
+        f.u = u; f.delta = delta;
+        f.B[0] = a.B[0]; f.B[1] = a.B[1]; f.C[0] = a.C[0]; f.C[1] = a.C[1];
+        f.A = a.A; f.D = a.D; f.bias = a.bias;
+        f.hloc = reinterpret_cast<float *>(ws + pl.off_hloc);
+        f.ssum = reinterpret_cast<float *>(ws + pl.off_ssum);
+        f.batch = batch; f.L = L; f.Di = channels; f.H = H; f.W = W; f.order = pair;
+        f.chunk = kBwdChunk; f.G = pl.G;
+
+        float *dBo[2] = {dB + (2 * pair) * bc, dB + (2 * pair + 1) * bc};
+        float *dCo[2] = {dC + (2 * pair) * bc, dC + (2 * pair + 1) * bc};
+        float *tmp = reinterpret_cast<float *>(ws + pl.off_tmp);
+        float *dAp = dA + (size_t)2 * pair * channels * d_state;
+        float *dDp = dD + (size_t)2 * pair * channels, *dbp = ddelta_bias + (size_t)2 * pair * channels;
+        rc = dt == VIM_F32 ? launch_bwd_n<float>(d_state, a, f, dBo, dCo, dAp, dDp, dbp, tmp, stream, nullptr)
+                           : launch_bwd_n<__nv_bfloat16>(d_state, a, f, dBo, dCo, dAp, dDp, dbp, tmp, stream, nullptr);
+    }
+    return rc;
+}
+
 }  // extern "C"

@@ -54,9 +54,21 @@ struct BwdArgs {
     float *gsum;                        // [batch][G][2][Di] chunk Delta sums
     int batch, L, Di, G, nblk;
     int separate_bc;
+    int order, H, W;                    // visiting order of the pair (0: position = step;
+                                        // 1: column-major on H x W, the cross-scan's second pair)
+    int stage;                          // 0: one pair (Vim), final outputs; 1: first pair of the
+                                        // cross-scan, fp32 partials to acc_*; 2: second pair, adds them
+    float *acc_y, *acc_du, *acc_dd;     // [batch, L, Di] fp32 by position (stages 1 and 2)
 };
 
 namespace {
+
+// grid position visited at step t of the pair's forward direction
+__device__ __forceinline__ int bpos(const BwdArgs &p, int t) {
+    if (p.order == 0) return t;
+    const int h = t % p.H, w = t / p.H;
+    return h * p.W + w;
+}
 
 template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
@@ -94,7 +106,7 @@ __global__ void __launch_bounds__(2 * kAdjCh) adj_carry(BwdArgs p) {
         const int r = li / kAdjCh, cl = li % kAdjCh, ch = d0 + cl;
         float dr = 0.0f, e = 0.0f;
         if (r < tc && ch < p.Di) {
-            const size_t i = ((size_t)b * p.L + t0 + r) * p.Di + ch;
+            const size_t i = ((size_t)b * p.L + bpos(p, t0 + r)) * p.Di + ch;
             dr = ld<T>(p.delta, i);
             e = ld<T>(p.dout, i);
             if (p.z) e *= silu(ld<T>(p.z, i));
@@ -104,7 +116,7 @@ __global__ void __launch_bounds__(2 * kAdjCh) adj_carry(BwdArgs p) {
     }
     for (int li = threadIdx.x; li < 2 * kBwdChunk * N; li += 2 * kAdjCh) {
         const int k = li / (kBwdChunk * N), r = (li / N) % kBwdChunk, n = li % N;
-        sC[k][r][n] = r < tc ? ld<T>(p.C[k], ((size_t)b * p.L + t0 + r) * N + n) : 0.0f;
+        sC[k][r][n] = r < tc ? ld<T>(p.C[k], ((size_t)b * p.L + bpos(p, t0 + r)) * N + n) : 0.0f;
     }
     __syncthreads();
 
@@ -372,10 +384,10 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
         }
     }
     if (th.valid) {
-#pragma unroll
         // row (b, c) of par; cbase = (row * 2 + dir) * Di + d
         const size_t row = th.cbase / ((size_t)2 * p.Di), col = th.cbase % ((size_t)2 * p.Di);
         float *pr = p.par + row * ((size_t)2 * p.Di * (N + 2));
+#pragma unroll
         for (int j = 0; j < NT; ++j) pr[col * N + th.j0 + j] = dA[j];
         if (th.q == 0) pr[(size_t)2 * p.Di * N + col] = dD;
         if (th.q == kDdLane) pr[(size_t)2 * p.Di * (N + 1) + col] = dbias;
@@ -401,7 +413,7 @@ __device__ __forceinline__ void store_bc_part(const BwdArgs &p, const float *red
 #pragma unroll
             for (int w = 0; w < SH::WPD; ++w) acc += red[((dir * SH::WPD + w) * TC + r) * N + n];
         }
-        part[k][(((size_t)b * p.L + t0 + r) * p.nblk + blk) * N + n] = acc;
+        part[k][(((size_t)b * p.L + bpos(p, t0 + r)) * p.nblk + blk) * N + n] = acc;
     }
 }
 
@@ -420,7 +432,7 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
         const int r = li / CH, cl = li % CH, ch = d0 + cl;
         float u = 0.0f, e = 0.0f, dl0 = 0.0f, dl1 = 0.0f, sg0 = 0.0f, sg1 = 0.0f;
         if (r < tc && ch < p.Di) {
-            const size_t i = ((size_t)b * p.L + t0 + r) * p.Di + ch;
+            const size_t i = ((size_t)b * p.L + bpos(p, t0 + r)) * p.Di + ch;
             u = ld<T>(p.u, i);
             const float dr = ld<T>(p.delta, i);
             e = ld<T>(p.dout, i);
@@ -434,7 +446,7 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     }
     for (int li = threadIdx.x; li < 2 * TC * N; li += SH::kThr) {
         const int k = li / (TC * N), r = (li / N) % TC, n = li % N;
-        const size_t i = ((size_t)b * p.L + t0 + r) * N + n;
+        const size_t i = ((size_t)b * p.L + (r < tc ? bpos(p, t0 + r) : 0)) * N + n;
         sm.B[li] = r < tc ? ld<T>(p.B[k], i) : 0.0f;
         sm.C[li] = r < tc ? ld<T>(p.C[k], i) : 0.0f;
     }
@@ -461,14 +473,20 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     if (th.dir == 0) bwd_forward<N, 0>(p, sm, th);
     else bwd_forward<N, 1>(p, sm, th);
     __syncthreads();
-    // dz = dout silu'(z) (y^f + y^b), and the CTA's dC terms
-    if (p.dz) {
+    // dz = dout silu'(z) (sum of the directions' y), and the CTA's dC terms; the
+    // cross-scan's first pair leaves its y for the second
+    if (p.dz || p.stage == 1) {
         for (int li = threadIdx.x; li < TC * CH; li += SH::kThr) {
             const int r = li / CH, c2 = li % CH, ch = d0 + c2;
             if (r < tc && ch < p.Di) {
-                const size_t i = ((size_t)b * p.L + t0 + r) * p.Di + ch;
-                const float y = sm.yb[r * CH + c2] + sm.yb[(TC + r) * CH + c2];
-                static_cast<T *>(p.dz)[i] = from_f32<T>(ld<T>(p.dout, i) * silu_grad(ld<T>(p.z, i)) * y);
+                const size_t i = ((size_t)b * p.L + bpos(p, t0 + r)) * p.Di + ch;
+                float y = sm.yb[r * CH + c2] + sm.yb[(TC + r) * CH + c2];
+                if (p.stage == 1) {
+                    p.acc_y[i] = y;
+                } else {
+                    if (p.stage == 2) y += p.acc_y[i];
+                    static_cast<T *>(p.dz)[i] = from_f32<T>(ld<T>(p.dout, i) * silu_grad(ld<T>(p.z, i)) * y);
+                }
             }
         }
     }
@@ -481,9 +499,20 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     for (int li = threadIdx.x; li < TC * CH; li += SH::kThr) {
         const int r = li / CH, c2 = li % CH, ch = d0 + c2;
         if (r < tc && ch < p.Di) {
-            const size_t i = ((size_t)b * p.L + t0 + r) * p.Di + ch;
-            static_cast<T *>(p.du)[i] = from_f32<T>(sm.yb[r * CH + c2] + sm.yb[(TC + r) * CH + c2]);
-            static_cast<T *>(p.ddelta)[i] = from_f32<T>(sm.dd[r * CH + c2] + sm.dd[(TC + r) * CH + c2]);
+            const size_t i = ((size_t)b * p.L + bpos(p, t0 + r)) * p.Di + ch;
+            float du = sm.yb[r * CH + c2] + sm.yb[(TC + r) * CH + c2];
+            float dd = sm.dd[r * CH + c2] + sm.dd[(TC + r) * CH + c2];
+            if (p.stage == 1) {
+                p.acc_du[i] = du;
+                p.acc_dd[i] = dd;
+            } else {
+                if (p.stage == 2) {
+                    du += p.acc_du[i];
+                    dd += p.acc_dd[i];
+                }
+                static_cast<T *>(p.du)[i] = from_f32<T>(du);
+                static_cast<T *>(p.ddelta)[i] = from_f32<T>(dd);
+            }
         }
     }
     store_bc_part<N>(p, sm.red, p.dB_part, b, t0, tc, blk);
