@@ -113,7 +113,8 @@ def block_params(w, seed):
 
 
 def algorithmic_bwd(w):
-    """Algorithmic bytes and FP32 lane-ops of one derivative step (Vim, shared B/C).
+    """Algorithmic bytes and FP32 lane-ops of one derivative step (Vim with shared B/C,
+    or the cross-scan with B/C per direction).
 
     Bytes: reads of u, delta_raw, z, dout and writes of du, d delta_raw, dz per
     token-channel; B, C read and dB, dC (fp32) written per token; parameters and
@@ -123,7 +124,8 @@ def algorithmic_bwd(w):
     multiply, the h_(t-1) product, the dA, A- and B-weighted sums and the dB term.
     """
     el = 4 if w.dtype == "f32" else 2
-    bc = 2 * w.batch * w.tokens * w.d_state * (el + 4)
+    n_bc_sets = 1 if w.kind == "vim" else w.directions
+    bc = 2 * w.batch * w.tokens * w.d_state * (el + 4) * n_bc_sets
     params = 2 * w.directions * w.channels * (w.d_state + 2) * 4
     nbytes = 7 * w.tok_ch * el + bc + params
     ops = 11 * w.d_state * w.directions * w.tok_ch
@@ -224,8 +226,10 @@ def run_oracle(w, x, threads, zoh=False):
     if "Wx" in x:
         oracle.vim_block_scan(x["u"], x["Wx"], x["Wdt"], x["A"], x["D"], x["dt_bias"], x["z"],
                               conv_w=x["conv_w"], conv_b=x["conv_b"])
-    elif "dout" in x:
+    elif "dout" in x and w.kind == "vim":
         oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], x["dout"])
+    elif "dout" in x:
+        oracle.cross_scan4_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], x["dout"])
     elif "conv_w" in x:
         oracle.vim_bidir_conv(x["u"], x["conv_w"], x["conv_b"], x["delta"], x["z"], x["B"], x["C"], x["A"],
                               x["D"], x["delta_bias"], zoh=zoh)
@@ -254,7 +258,7 @@ def oracle_sample(w, target_s, conv=False, bwd=False, block=False):
     cores = cpu_cores()
     full = wl.make_inputs(w)
     if bwd:
-        full["dout"] = bwd_dout(w, w.seed + 2)
+        full["dout"] = bwd_dout(w, w.seed + 2).reshape(full["u"].shape).contiguous()
     if block:
         full.update(block_params(w, w.seed + 3))
     if conv:
@@ -332,8 +336,8 @@ def main():
     from vision_mamba_selective_b200 import workloads as wl
 
     w = wl.BY_NAME[args.workload]
-    if (args.conv or args.bwd or args.block) and w.kind != "vim":
-        raise SystemExit("--conv, --bwd and --block apply to the Vim workloads only")
+    if (args.conv or args.block) and w.kind != "vim":
+        raise SystemExit("--conv and --block apply to the Vim workloads only")
     if args.block and (args.conv or args.zoh or args.bwd or w.dtype != "bf16"):
         raise SystemExit("--block runs alone, on a bf16 workload")
     if args.bwd and (args.conv or args.zoh):
@@ -361,9 +365,9 @@ def main():
     el = 4 if w.dtype == "f32" else 2
     out_bytes = w.tok_ch * el
     if args.bwd:
-        host["dout"] = bwd_dout(w, replicas.rank_seed(w.seed + 2, rank))
+        host["dout"] = bwd_dout(w, replicas.rank_seed(w.seed + 2, rank)).reshape(host["u"].shape).contiguous()
         act_keys.append("dout")
-        out_bytes = 3 * w.tok_ch * el + 2 * w.batch * w.tokens * w.d_state * 4
+        out_bytes = 3 * w.tok_ch * el + 2 * w.batch * w.tokens * w.d_state * 4 * (1 if w.kind == "vim" else 4)
     set_bytes = sum(host[k].numel() * host[k].element_size() for k in act_keys) + out_bytes
     nsets = max(2, math.ceil(2.2 * L2_BYTES / set_bytes))
     params = {k: host[k].to(dev) for k in ("A", "D", "delta_bias")}
@@ -374,15 +378,17 @@ def main():
         if args.bwd:
             f32 = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
             s["out"] = dict(du=torch.empty_like(s["u"]), ddelta=torch.empty_like(s["u"]), dz=torch.empty_like(s["u"]),
-                            dB=f32(*s["B"].shape), dC=f32(*s["C"].shape), dA=f32(2, w.channels, w.d_state),
-                            dD=f32(2, w.channels), ddelta_bias=f32(2, w.channels))
+                            dB=f32(*s["B"].shape), dC=f32(*s["C"].shape), dA=f32(w.directions, w.channels, w.d_state),
+                            dD=f32(w.directions, w.channels), ddelta_bias=f32(w.directions, w.channels))
         sets.append(s)
     if w.kind == "vim":
         ws_bytes = vs.vim_scan_workspace_bytes(0, w.batch, w.L, 0, w.channels, w.d_state)
     else:
         ws_bytes = vs.vim_scan_workspace_bytes(1, w.batch, w.H, w.W, w.channels, w.d_state)
-    if args.bwd:
+    if args.bwd and w.kind == "vim":
         ws_bytes = vs.vim_scan_bwd_workspace_bytes(w.batch, w.L, w.channels, w.d_state, False)
+    elif args.bwd:
+        ws_bytes = int(vs.lib.vmamba_cross_scan4_bwd_workspace_bytes(w.batch, w.H, w.W, w.channels, w.d_state))
     if args.block:
         ws_bytes = vs.vim_block_workspace_bytes(w.batch, w.L, w.channels, w.d_state)
         blk = block_params(w, w.seed + 3)
@@ -401,9 +407,13 @@ def main():
                               s["z"], conv_w=params["conv_w"], conv_b=params["conv_b"], y=s["y"], workspace=ws,
                               events=events)
             return
-        if args.bwd:
+        if args.bwd and w.kind == "vim":
             vs.vim_scan_bidir_bwd(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"],
                                   params["delta_bias"], s["dout"], workspace=ws, out=s["out"], events=events)
+            return
+        if args.bwd:
+            vs.vmamba_cross_scan4_bwd(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"],
+                                      params["delta_bias"], s["dout"], workspace=ws, out=s["out"])
             return
         if args.conv:
             # u holds x, the pathways' common input in front of the convolutions
@@ -442,6 +452,8 @@ def main():
     kernels_per_pair = 3
     pairs = 1 if w.kind == "vim" else 2
     nev = 4 if args.bwd else (5 if args.block else 1 + kernels_per_pair * pairs)
+    if args.bwd and w.kind != "vim":
+        nev = 2       # the cross-scan derivative has no per-phase events: the whole call is timed
     prof_steps = min(args.steps, 200)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(prof_steps)]
     for i in range(prof_steps):
@@ -453,6 +465,19 @@ def main():
             t = [evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(prof_steps)]
             per_kernel[name] = sum(t) / len(t)
         launches_per_step = 1 + (3 if w.tokens > 256 else 1)
+    elif args.bwd and w.kind != "vim":
+        t = []
+        for i in range(prof_steps):
+            e0, e1 = evs[i]
+            e0.record()
+            step(i)
+            e1.record()
+        torch.cuda.synchronize()
+        t = [evs[i][0].elapsed_time(evs[i][1]) for i in range(prof_steps)]
+        per_kernel["vmamba_cross_scan4_bwd"] = sum(t) / len(t)
+        # per pair: pair_carry, pair_combine, adj_carry, pair_combine, bwd_main, four dB/dC
+        # reductions, one two-pass column sum
+        launches_per_step = 2 * ((4 if w.tokens > 32 else 0) + 1 + 4 + 2)
     elif args.bwd:
         for a, name in enumerate(["summaries", "bwd_main", "reductions"], start=1):
             t = [evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(prof_steps)]
@@ -507,6 +532,8 @@ def main():
     pk = peaks()
     nbytes, ops = algorithmic_bwd(w) if args.bwd else algorithmic(w, args.conv)
     main_name = "bwd_main" if args.bwd else "pair_main"
+    if args.bwd and w.kind != "vim":
+        main_name = "vmamba_cross_scan4_bwd"     # the whole call (all its kernels)
     main_ms = sum(v for k, v in per_kernel.items() if k.startswith(main_name))
     clocks = clk.summary()
     peak_ops = SMS * FP32_LANES_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e12

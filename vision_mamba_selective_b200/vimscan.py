@@ -236,18 +236,19 @@ def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stri
     return out
 
 
-def vmamba_cross_scan4_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, workspace=None, stream=None):
+def vmamba_cross_scan4_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, workspace=None, stream=None, out=None):
     """Derivatives of vmamba_cross_scan4 (first-order Bbar) for a loss whose derivative
     with respect to y is ``dout``; see include/vimscan.h.  Returns a dict: du, ddelta, dz
     (None without z) in the input dtype; dB, dC [4, batch, H*W, N], dA [4, C, N], dD and
-    ddelta_bias [4, C] in fp32.
+    ddelta_bias [4, C] in fp32.  ``out`` may hold those tensors from an earlier call.
     """
     batch, H, W, Ch = u.shape
     N = B.shape[-1]
     dev = u.device
     f32 = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
-    out = dict(du=torch.empty_like(u), ddelta=torch.empty_like(u), dz=torch.empty_like(u) if z is not None else None,
-               dB=f32(*B.shape), dC=f32(*C.shape), dA=f32(4, Ch, N), dD=f32(4, Ch), ddelta_bias=f32(4, Ch))
+    if out is None:
+        out = dict(du=torch.empty_like(u), ddelta=torch.empty_like(u), dz=torch.empty_like(u) if z is not None else None,
+                   dB=f32(*B.shape), dC=f32(*C.shape), dA=f32(4, Ch, N), dD=f32(4, Ch), ddelta_bias=f32(4, Ch))
     ws, ws_bytes = _workspace(int(lib.vmamba_cross_scan4_bwd_workspace_bytes(batch, H, W, Ch, N)), workspace, dev)
     st = lib.vmamba_cross_scan4_bwd(
         _ptr(u, name="u"), _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
