@@ -17,7 +17,7 @@
 // or 32 channels, both directions: a forward sweep that keeps h every kBwdSeg tokens (in
 // registers) and forms y (for dz) and the dC terms, then segment by segment in
 // reverse a re-run of h over the segment followed by the adjoint sweep.  A thread
-// holds NT <= 4 states of one (channel, direction), so the segment's h and decays fit
+// holds NT (4, or 8 when built so) states of one (channel, direction), so the segment's h and decays fit
 // in registers (the checkpoints go to shared memory); Q = N / NT threads share a
 // channel.  Each warp serves one direction, whose code is compiled separately so that
 // its token addresses are constants.
@@ -37,6 +37,9 @@ constexpr int kBwdSeg = 4;                    // tokens between checkpoints of h
 constexpr int kBwdNSeg = kBwdChunk / kBwdSeg;
 constexpr int kAdjCh = 64;                    // channels per adj_carry CTA
 constexpr int kReduceParts = 32;              // row groups of the first parameter-reduction pass
+#ifndef VIMSCAN_BWD_NT
+#define VIMSCAN_BWD_NT 4                         // states per thread of bwd_main (4 or 8)
+#endif
 #ifndef VIMSCAN_BWD_MIN_WARPS
 #define VIMSCAN_BWD_MIN_WARPS 16                 // resident warps per SM the register budget targets
 #endif
@@ -204,7 +207,8 @@ __device__ __forceinline__ void reduce_channels(float (&v)[NT], int lane, int *o
 // the derivative over one chunk of CH channels, both directions
 // ----------------------------------------------------------------------------
 template <int N> struct BwdShape {
-    static constexpr int NT = N < 4 ? N : 4;                 // states per thread
+    static constexpr int NT = N < VIMSCAN_BWD_NT ? N : VIMSCAN_BWD_NT;   // states per thread
+    static constexpr int CKW = (NT + 3) / 4;                 // float4 per checkpoint per thread
     static constexpr int Q = N / NT;                         // threads per (channel, direction)
     static constexpr int CH = 32 / Q > 16 ? 32 / Q : 16;     // channels per CTA (whole warps per direction)
     static constexpr int kThr = 2 * CH * Q;
@@ -218,7 +222,7 @@ template <int N> struct BwdShape {
     //   dd[2][TC][CH]  d delta_raw from direction k
     //   B[2][TC][N], C[2][TC][N]
     //   red[2][WPD][TC][N]  per direction and warp: the dC terms, then the dB terms
-    //   ck[kBwdNSeg][kThr] float4  h at every kBwdSeg-th token, per thread
+    //   ck[kBwdNSeg][CKW][kThr] float4  h at every kBwdSeg-th token, per thread
     static constexpr int oTok = 0;
     static constexpr int oYb = oTok + 2 * TC * CH * 4;
     static constexpr int oDd = oYb + 2 * TC * CH;
@@ -226,7 +230,7 @@ template <int N> struct BwdShape {
     static constexpr int oC = oB + 2 * TC * N;
     static constexpr int oRed = oC + 2 * TC * N;
     static constexpr int oCk = oRed + 2 * WPD * TC * N;
-    static constexpr int kFloats = oCk + kBwdNSeg * kThr * 4;
+    static constexpr int kFloats = oCk + kBwdNSeg * CKW * kThr * 4;
     static constexpr size_t kSmemBytes = (size_t)kFloats * 4;
     static_assert(oCk % 4 == 0 && oTok % 4 == 0, "float4 areas must be 16-byte aligned");
 };
@@ -255,9 +259,12 @@ struct BwdThread {
 
 template <int NT>
 __device__ __forceinline__ void load_states(const float *row, float (&v)[NT]) {
-    if constexpr (NT == 4) {
-        const float4 t = *reinterpret_cast<const float4 *>(row);
-        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    if constexpr (NT % 4 == 0) {
+#pragma unroll
+        for (int q = 0; q < NT / 4; ++q) {
+            const float4 t = *reinterpret_cast<const float4 *>(row + 4 * q);
+            v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
+        }
     } else {
 #pragma unroll
         for (int j = 0; j < NT; ++j) v[j] = row[j];
@@ -274,8 +281,13 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
     for (int j = 0; j < NT; ++j) h[j] = (p.G > 1 && th.valid) ? p.hin[th.cbase * N + th.j0 + j] : 0.0f;
 #pragma unroll 1
     for (int sg = 0; sg < kBwdNSeg; ++sg) {
-        sm.ck[sg * SH::kThr + th.tid] = make_float4(h[0], NT > 1 ? h[NT > 1 ? 1 : 0] : 0.0f,
-                                                    NT > 2 ? h[NT > 2 ? 2 : 0] : 0.0f, NT > 3 ? h[NT > 3 ? 3 : 0] : 0.0f);
+#pragma unroll
+        for (int w = 0; w < SH::CKW; ++w) {
+            float q4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) q4[e] = 4 * w + e < NT ? h[4 * w + e < NT ? 4 * w + e : 0] : 0.0f;
+            sm.ck[(sg * SH::CKW + w) * SH::kThr + th.tid] = make_float4(q4[0], q4[1], q4[2], q4[3]);
+        }
 #pragma unroll
         for (int m = 0; m < kBwdSeg; ++m) {
             const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
@@ -319,8 +331,12 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
     float dD = 0.0f, dbias = 0.0f;
 #pragma unroll 1
     for (int sg = kBwdNSeg - 1; sg >= 0; --sg) {
-        const float4 c4 = sm.ck[sg * SH::kThr + th.tid];
-        const float h0[4] = {c4.x, c4.y, c4.z, c4.w};
+        float h0[4 * SH::CKW];
+#pragma unroll
+        for (int w = 0; w < SH::CKW; ++w) {
+            const float4 c4 = sm.ck[(sg * SH::CKW + w) * SH::kThr + th.tid];
+            h0[4 * w] = c4.x; h0[4 * w + 1] = c4.y; h0[4 * w + 2] = c4.z; h0[4 * w + 3] = c4.w;
+        }
         float hh[kBwdSeg][NT], aa[kBwdSeg][NT];
 #pragma unroll
         for (int m = 0; m < kBwdSeg; ++m) {
