@@ -33,15 +33,22 @@ struct Plan {
     int G;      // chunks
 };
 
-Plan plan_for(int L) {
+// Chunking of a sequence.  Short sequences with few CTAs (fewer than a B200 has SMs)
+// are cut into kShortChunk-token chunks anyway, so that their walks run side by side
+// instead of one long walk per CTA (the latency-bound sizes).
+constexpr int kShortChunk = 32;
+constexpr int64_t kFewCtas = 148;
+
+Plan plan_for(int batch, int L, int Di) {
     Plan pl;
-    if (L <= kSingleChunkMax) {
+    const int64_t ctas = (int64_t)batch * ((Di + kDC - 1) / kDC);
+    if (L <= kSingleChunkMax && !(ctas < kFewCtas && L > 2 * kShortChunk)) {
         pl.chunk = ((L + kTile - 1) / kTile) * kTile;
         if (pl.chunk == 0) pl.chunk = kTile;
         pl.G = 1;
     } else {
-        pl.chunk = kLongChunk;
-        pl.G = (L + kLongChunk - 1) / kLongChunk;
+        pl.chunk = L <= kSingleChunkMax ? kShortChunk : kLongChunk;
+        pl.G = (L + pl.chunk - 1) / pl.chunk;
     }
     return pl;
 }
@@ -50,7 +57,7 @@ size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // summaries for one pair: hloc [batch][G][2][Di][N] + ssum [batch][G][2][Di]
 size_t summary_bytes(int batch, int L, int Di, int N) {
-    const Plan pl = plan_for(L);
+    const Plan pl = plan_for(batch, L, Di);
     if (pl.G <= 1) return 0;
     const size_t units = (size_t)batch * pl.G * 2 * Di;
     return round_up(units * N * sizeof(float)) + round_up(units * sizeof(float));

@@ -114,7 +114,7 @@ vim_status vim_block_scan(const void *x, const float *conv_w, const float *conv_
     if (st != VIM_OK) return st;
     if (events && cudaEventRecord(events[1], stream) != cudaSuccess) return VIM_ERR_CUDA;
 
-    const Plan sp = plan_for(L);
+    const Plan sp = plan_for(batch, L, d_inner);
     PairArgs a;
     std::memset(&a, 0, sizeof(a));
     a.u = x; a.z = z;

@@ -71,7 +71,7 @@ vim_status bidir_impl(const void *u, const float *conv_w, const float *conv_b, c
         if (!workspace || workspace_bytes < need) return VIM_ERR_WORKSPACE;
         if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return VIM_ERR_WORKSPACE;
     }
-    const Plan pl = plan_for(L);
+    const Plan pl = plan_for(batch, L, d_inner);
     PairArgs a;
     std::memset(&a, 0, sizeof(a));
     a.u = u; a.delta = delta; a.z = z;
@@ -171,7 +171,7 @@ vim_status vmamba_cross_scan4_ex(const void *u, const void *delta, const void *z
     if (!workspace || workspace_bytes < need) return VIM_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return VIM_ERR_WORKSPACE;
 
-    const Plan pl = plan_for(L);
+    const Plan pl = plan_for(batch, L, channels);
     float *partial = reinterpret_cast<float *>(static_cast<char *>(workspace) + sum_b);
     const size_t el = elem_size(dt);
     const size_t bc_dir = (size_t)batch * L * d_state * el;   // bytes between directions
