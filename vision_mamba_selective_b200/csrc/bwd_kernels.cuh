@@ -138,10 +138,14 @@ __global__ void __launch_bounds__(2 * kAdjCh) adj_carry(BwdArgs p) {
 #pragma unroll
     for (int k = 0; k < NP; ++k) G[k] = f2(0.f, 0.f);
     float S = 0.0f;
-    for (int i = 0; i < tc; ++i) {
-        const int r = dir ? tc - 1 - i : i;
-        S += softplus(sDr[r][dl] + bias);
-        const float e = sDy[r][dl];
+    // a fixed trip count (tokens past the chunk add Delta = 0 and dy = 0) lets the
+    // compiler overlap the independent softplus of later tokens with the chain
+#pragma unroll 4
+    for (int i = 0; i < kBwdChunk; ++i) {
+        const bool ok = i < tc;
+        const int r = ok ? (dir ? tc - 1 - i : i) : 0;
+        S += ok ? softplus_io<T>(sDr[r][dl] + bias) : 0.0f;
+        const float e = ok ? sDy[r][dl] : 0.0f;
         float2 Cv[NP];
         load_row<NP>(&sC[dir][r][0], Cv);
         if (fast) {
@@ -454,8 +458,8 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
             e = ld<T>(p.dout, i);
             if (p.z) e *= silu(ld<T>(p.z, i));
             const float x0 = dr + p.bias[ch], x1 = dr + p.bias[p.Di + ch];
-            dl0 = softplus(x0); sg0 = softplus_grad(x0);
-            dl1 = softplus(x1); sg1 = softplus_grad(x1);
+            dl0 = softplus_io<T>(x0); sg0 = softplus_grad(x0);
+            dl1 = softplus_io<T>(x1); sg1 = softplus_grad(x1);
         }
         sm.tok[r * CH + cl] = make_float4(dl0, u, e, sg0);
         sm.tok[(TC + r) * CH + cl] = make_float4(dl1, u, e, sg1);
