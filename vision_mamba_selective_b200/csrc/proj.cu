@@ -45,7 +45,7 @@ vim_status launch_proj_c(const ProjArgs &pa, cudaStream_t stream) {
         int dev = 0;
         if (cudaGetDevice(&dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 128, sm) != cudaSuccess)
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kProjThreads, sm) != cudaSuccess)
             return VIM_ERR_CUDA;
         cached_sms.store(sms);
         cached_per_sm.store(per_sm);
@@ -54,7 +54,7 @@ vim_status launch_proj_c(const ProjArgs &pa, cudaStream_t stream) {
     // each pathway's tiles spread over about half the resident CTAs; Wx is staged once per CTA
     const int64_t tiles = (pa.M + kProjRows - 1) / kProjRows;
     const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(tiles, (int64_t)sms * std::max(per_sm, 1) / 2));
-    kernel<<<dim3(2, (unsigned)ctas), 128, sm, stream>>>(pa);
+    kernel<<<dim3(2, (unsigned)ctas), kProjThreads, sm, stream>>>(pa);
     return cudaGetLastError() == cudaSuccess ? VIM_OK : VIM_ERR_CUDA;
 }
 

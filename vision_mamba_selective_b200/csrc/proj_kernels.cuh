@@ -9,7 +9,7 @@
 // A CTA serves one pathway: it stages Wx[k] transposed once, then for each of its
 // 64-token tiles (rows of the flattened [batch*L] sequence) forms u_k one 64-channel
 // slice at a time in shared memory (bf16) and multiplies on the tensor cores with
-// mma.sync m16n8k16 (bf16 in, fp32 accumulate), four warps of 16 rows each.  The
+// mma.sync m16n8k16 (bf16 in, fp32 accumulate), one warp per 16 rows.  The
 // product has only 2N + 1 <= 33 columns, so the kernel is bound by reading x, not by
 // the tensor pipe.
 #pragma once
@@ -28,7 +28,11 @@ struct ProjArgs {
     int L, Di;
 };
 
-constexpr int kProjRows = 64;       // tokens per CTA
+#ifndef VIMSCAN_PROJ_ROWS
+#define VIMSCAN_PROJ_ROWS 128
+#endif
+constexpr int kProjRows = VIMSCAN_PROJ_ROWS;   // tokens per tile: 16 per warp
+constexpr int kProjThreads = 2 * kProjRows;    // one warp per 16 rows
 constexpr int kProjK = 64;          // channels per K slice
 constexpr int kProjPad = 8;         // row padding (bf16 elements) of the shared tiles
 
@@ -58,9 +62,9 @@ template <int N> struct ProjShape {
 // ([output column][channel]).  The (tile, 64-channel slice) steps form one pipeline:
 // cp.async brings the next step's x rows (the tile plus one neighbour row on each side)
 // while the current step forms u -- thread (pair p, group q) takes channels 2p, 2p+1 of
-// rows 16q .. 16q+15 -- and the four warps run its tensor-core products.
+// rows 16q .. 16q+15 -- and the warps run its tensor-core products.
 template <int N, bool CONV>
-__global__ void __launch_bounds__(128) xproj_kernel(ProjArgs p) {
+__global__ void __launch_bounds__(kProjThreads) xproj_kernel(ProjArgs p) {
     using PS = ProjShape<N>;
     constexpr int NO = PS::NO, NT8 = PS::NT8, LDU = PS::LDU, XROWS = PS::XROWS;
     extern __shared__ __align__(16) __nv_bfloat16 psm[];
@@ -85,7 +89,7 @@ __global__ void __launch_bounds__(128) xproj_kernel(ProjArgs p) {
         const int tile = blockIdx.y + (st / nslice) * gridDim.y, kc = (st % nslice) * kProjK;
         const int m0 = tile * kProjRows;
         __nv_bfloat16 *dst = sX + buf * XROWS * LDU;
-        for (int li = tid; li < XROWS * (kProjK / 8); li += 128) {
+        for (int li = tid; li < XROWS * (kProjK / 8); li += kProjThreads) {
             const int r = li / (kProjK / 8), c8 = (li % (kProjK / 8)) * 8;
             const int m = m0 - 1 + r, d = kc + c8;
             const bool ok = m >= 0 && m < M && d < p.Di;
@@ -98,11 +102,11 @@ __global__ void __launch_bounds__(128) xproj_kernel(ProjArgs p) {
     // Wx[k] transposed: read in its own order (coalesced), eight loads in flight per thread
     const int nW = p.Di * NO;
 #pragma unroll 8
-    for (int li = tid; li < nW; li += 128) {
+    for (int li = tid; li < nW; li += kProjThreads) {
         const int d = li / NO, jcol = li % NO;
         sW[jcol * LDW + d] = W[li];
     }
-    for (int li = tid; li < (NT8 * 8 - NO) * p.Di; li += 128)
+    for (int li = tid; li < (NT8 * 8 - NO) * p.Di; li += kProjThreads)
         sW[(NO + li / p.Di) * LDW + li % p.Di] = __float2bfloat16_rn(0.0f);
 
     const int cp = lane, rg = warp;          // channel pair and row group of the u pass
