@@ -433,3 +433,29 @@ def test_full_size_zoh(vs, name):
         ref = oracle.cross_scan4(*refargs, zoh=True)
     torch.cuda.synchronize()
     check(f"full_zoh_{name}", y, ref, w.torch_dtype())
+
+
+def test_vim_cuda_graph(vs):
+    """The entry points only enqueue work on the given stream, so a call can be captured
+    into a CUDA graph and replayed; the replay matches the oracle on new inputs copied
+    into the captured buffers (here with PDL-chained kernels: L = 1111, several chunks)."""
+    x = vim_inputs(2, 1111, 64, 16, torch.bfloat16, seed=31)
+    d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
+    ws = torch.empty(vs.vim_scan_workspace_bytes(0, 2, 1111, 0, 64, 16), dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(d["u"])
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):      # first call outside capture (attribute set-up)
+        vs.vim_scan_bidir(d["u"], d["delta"], d["z"], d["B"], d["C"], d["A"], d["D"], d["bias"], y=y, workspace=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        vs.vim_scan_bidir(d["u"], d["delta"], d["z"], d["B"], d["C"], d["A"], d["D"], d["bias"], y=y, workspace=ws)
+    x2 = vim_inputs(2, 1111, 64, 16, torch.bfloat16, seed=32)
+    for k in ("u", "delta", "z", "B", "C"):
+        d[k].copy_(x2[k])
+    g.replay()
+    torch.cuda.synchronize()
+    ref_in = dict(x, **{k: x2[k] for k in ("u", "delta", "z", "B", "C")})   # captured parameters stay
+    check("vim_graph_replay", y, ref_vim(ref_in), torch.bfloat16)
