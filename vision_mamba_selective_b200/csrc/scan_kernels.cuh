@@ -12,12 +12,18 @@
 // over it: warps 0-1 the forward direction (ascending), warps 2-3 the backward
 // direction (descending), one thread per (channel, direction) with all d_state
 // states of h in fp32 registers.  The chunk's inputs stream through shared memory in
-// tiles of 16 tokens (cp.async for u/delta/z, register prefetch + fp32 conversion for
-// B/C), double buffered.  The forward direction visits tile j at step j and the
+// tiles of 16 tokens (cp.async for u and delta, register prefetch + fp32 conversion
+// for B/C), double buffered.  The forward direction visits tile j at step j and the
 // backward one at step nT-1-j: the first visitor leaves its partial output in a
-// per-chunk fp32 buffer, the second adds its own, applies the silu(z) gate and
-// writes the result, so every output is written once and no separate output pass
-// is needed.
+// per-chunk fp32 buffer, the second adds its own; after the step's barrier all
+// threads finish the completed tiles (z prefetched into registers, silu(z) gate,
+// 16-byte stores), so every output is written once and no separate output pass is
+// needed.
+//
+// Variants (template flags): CONV, the pathways' kernel-3 convolution + SiLU formed
+// from staged x; ZOH, the exact zero-order-hold Bbar; DT, delta from the x_proj step
+// input and the dt_proj weights; PIN, the cross-scan's second pair adding the first
+// pair's fp32 partial.
 //
 // For G > 1 the state entering each chunk comes from two small kernels: `pair_carry`
 // reduces every chunk to its end state from h = 0 plus its total Delta, and
@@ -183,18 +189,6 @@ __device__ __forceinline__ float silu(float z) { return z * rcp(1.0f + ex2(-z * 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-
-// a[k] = (q^(2k+1), q^(2k+2)), k < NP, by doubling blocks: depth log2(2 NP).
-template <int NP>
-__device__ __forceinline__ void powers2(float q, float2 (&a)[NP]) {
-    a[0] = f2(q, q * q);
-#pragma unroll
-    for (int m = 1; m < NP; m *= 2) {
-        const float2 step = f2(a[m - 1].y, a[m - 1].y);   // q^(2m)
-#pragma unroll
-        for (int j = 0; j < m && m + j < NP; ++j) a[m + j] = mul2(a[j], step);
-    }
-}
 
 // Reads of the fp32 B/C rows staged in shared memory, as pairs of states.
 template <int NP>
