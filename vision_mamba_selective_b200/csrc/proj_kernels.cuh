@@ -38,6 +38,15 @@ constexpr int kProjPad = 8;         // row padding (bf16 elements) of the shared
 
 namespace {
 
+#ifndef VIMSCAN_PROJ_TANH
+#define VIMSCAN_PROJ_TANH 1
+#endif
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -159,9 +168,16 @@ __global__ void __launch_bounds__(kProjThreads) xproj_kernel(ProjArgs p) {
                 // neighbours outside the sequence are the convolution's zero padding
                 const float2 mm = t > 0 ? wm : f2(0.f, 0.f), mp = t < p.L - 1 ? wp : f2(0.f, 0.f);
                 const float2 v = fma2(mm, xm, fma2(wc, x0, fma2(mp, xp, cbv)));
+#if VIMSCAN_PROJ_TANH
+                // silu(v) = v (1 + tanh(v/2)) / 2 with the MUFU tanh (relative error near
+                // 2^-11, below the bf16 rounding that u takes next)
+                const float2 hv = mul2(v, f2(0.5f, 0.5f));
+                u = fma2(hv, f2(tanh_approx(hv.x), tanh_approx(hv.y)), hv);
+#else
                 const float2 e = mul2(v, f2(-kLog2e, -kLog2e));
                 const float2 den = f2(1.0f + ex2(e.x), 1.0f + ex2(e.y));
                 u = mul2(v, f2(rcp(den.x), rcp(den.y)));          // silu(v) = v / (1 + e^-v)
+#endif
             }
             if (m >= M || !dvalid) u = f2(0.f, 0.f);
             *reinterpret_cast<__nv_bfloat162 *>(&sU[r0 + r][2 * cp]) = __floats2bfloat162_rn(u.x, u.y);
