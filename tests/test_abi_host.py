@@ -142,6 +142,38 @@ def test_bwd_rejects(vs):
     assert vs.vim_scan_bwd_workspace_bytes(0, 100, 64, 16, False) == 0
 
 
+def test_cross_bwd_and_block_reject(vs):
+    lib = vs.lib
+    F = FAKE
+    # cross-scan derivative: z without dz, unsupported d_state, missing workspace
+    args = [F] * 17 + [2, 8, 8, 64, 16, vs.VIM_BF16, F, 1 << 40, None]
+    def xb(**kw):
+        a = list(args)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return lib.vmamba_cross_scan4_bwd(*a)
+    assert xb(a11=None) == vs.VIM_ERR_INVALID_ARG             # dz missing while z is given
+    assert xb(a5=None) == vs.VIM_ERR_INVALID_ARG              # A
+    assert xb(a0=F + 8) == vs.VIM_ERR_INVALID_ARG             # u not 16-byte aligned
+    assert xb(a21=3) == vs.VIM_ERR_UNSUPPORTED                # d_state
+    assert xb(a23=None) == vs.VIM_ERR_WORKSPACE
+    assert xb(a23=F + 16) == vs.VIM_ERR_WORKSPACE
+    assert vs.lib.vmamba_cross_scan4_bwd_workspace_bytes(2, 8, 8, 64, 16) > 0
+    # block scan: fp32 unsupported, half a convolution front, missing weights
+    def blk(**kw):
+        a = dict(x=F, cw=F, cb=F, Wx=F, Wdt=F, db=F, A=F, D=F, z=F, y=F, b=2, L=100, Di=64, N=16,
+                 dt=vs.VIM_BF16, ws=F, wsb=1 << 40)
+        a.update(kw)
+        return lib.vim_block_scan(a["x"], a["cw"], a["cb"], a["Wx"], a["Wdt"], a["db"], a["A"], a["D"], a["z"],
+                                  a["y"], a["b"], a["L"], a["Di"], a["N"], a["dt"], a["ws"], a["wsb"], None, None)
+    assert blk(dt=vs.VIM_F32) == vs.VIM_ERR_UNSUPPORTED
+    assert blk(cb=None) == vs.VIM_ERR_INVALID_ARG
+    assert blk(Wx=None) == vs.VIM_ERR_INVALID_ARG
+    assert blk(x=F + 8) == vs.VIM_ERR_INVALID_ARG
+    assert blk(Di=3000) == vs.VIM_ERR_UNSUPPORTED             # Wx^T would not fit in shared memory
+    assert blk(ws=None) == vs.VIM_ERR_WORKSPACE
+
+
 def test_size_zero_is_a_noop(vs):
     # nothing is read or launched, so even null pointers are fine
     assert bidir(vs, batch=0, u=None, y=None) == vs.VIM_OK
