@@ -122,6 +122,17 @@ vim_status launch_bwd_n(int N, const BwdArgs &a, const PairArgs &fwd, float *dB[
 
 bool aligned_to(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// vector access of four channels (8 bytes of bf16, 16 of fp32) to every [.., Di]
+// tensor, and of whole 16-byte B/C vectors, when the pointers allow it
+void set_vector_flags(BwdArgs &a, vim_dtype dt, int N) {
+    const size_t va = dt == VIM_F32 ? 16 : 8;
+    a.vec_io = aligned_to(a.u, va) && aligned_to(a.delta, va) && aligned_to(a.dout, va) &&
+               (!a.z || aligned_to(a.z, va)) && aligned_to(a.du, va) && aligned_to(a.ddelta, va) &&
+               (!a.dz || aligned_to(a.dz, va));
+    a.vec_bc = (N * elem_size(dt)) % 16 == 0 && aligned16(a.B[0]) && aligned16(a.B[1]) && aligned16(a.C[0]) &&
+               aligned16(a.C[1]);
+}
+
 }  // namespace
 }  // namespace vimscan
 
@@ -186,6 +197,7 @@ vim_status vim_scan_bidir_bwd_events(const void *u, const void *delta, const voi
     a.gsum = reinterpret_cast<float *>(ws + pl.off_gsum);
     a.batch = batch; a.L = L; a.Di = d_inner; a.G = pl.G; a.nblk = pl.nblk;
     a.separate_bc = separate;
+    set_vector_flags(a, dt, d_state);
 
     PairArgs f;
     std::memset(&f, 0, sizeof(f));
@@ -281,6 +293,7 @@ vim_status vmamba_cross_scan4_bwd(const void *u, const void *delta, const void *
         a.gsum = reinterpret_cast<float *>(ws + pl.off_gsum);
         a.batch = batch; a.L = L; a.Di = channels; a.G = pl.G; a.nblk = pl.nblk;
         a.separate_bc = 1;
+        set_vector_flags(a, dt, d_state);
         a.order = pair; a.H = H; a.W = W;
         a.stage = pair + 1;                  // the row pair leaves partials, the column pair finishes
         a.acc_y = acc;

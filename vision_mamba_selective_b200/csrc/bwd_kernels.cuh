@@ -17,13 +17,15 @@
 // or 32 channels, both directions: a forward sweep that keeps h every kBwdSeg tokens (in
 // registers) and forms y (for dz) and the dC terms, then segment by segment in
 // reverse a re-run of h over the segment followed by the adjoint sweep.  A thread
-// holds NT (4, or 8 when built so) states of one (channel, direction), so the segment's h and decays fit
-// in registers (the checkpoints go to shared memory); Q = N / NT threads share a
-// channel.  Each warp serves one direction, whose code is compiled separately so that
-// its token addresses are constants.
-// Sums over channels (dB, dC) are reduced across the warp by shuffles, then across
-// the CTA's warps and directions in shared memory, and written per CTA; sums over
-// tokens (dA, dD, dbias) are written per chunk.  Small reduction kernels finish both.
+// holds NT (4, or 8 when built so) states of one (channel, direction), as pairs for
+// the f32x2 arithmetic, so the segment's h and decays fit in registers (the
+// checkpoints go to shared memory); Q = N / NT threads share a channel.  Each warp
+// serves one direction, whose code is compiled separately so that its token addresses
+// are constants.
+// Sums over channels (dB, dC) are taken across the warp (through a transposition in
+// shared memory when 4 lanes share a channel, else by shuffles), then across the CTA's
+// warps and directions in shared memory, and written per CTA; sums over tokens (dA,
+// dD, dbias) are written per chunk.  Small reduction kernels finish both.
 // Every sum is taken in a fixed order (no floating-point atomics), so results repeat
 // bit for bit.
 #pragma once
@@ -57,6 +59,8 @@ struct BwdArgs {
     float *gsum;                        // [batch][G][2][Di] chunk Delta sums
     int batch, L, Di, G, nblk;
     int separate_bc;
+    int vec_io;                         // u, delta, dout, z, du, d delta_raw, dz allow vector access
+    int vec_bc;                         // B and C rows move as 16-byte vectors
     int order, H, W;                    // visiting order of the pair (0: position = step;
                                         // 1: column-major on H x W, the cross-scan's second pair)
     int stage;                          // 0: one pair (Vim), final outputs; 1: first pair of the
@@ -205,13 +209,11 @@ __device__ __forceinline__ void reduce_channels(float (&v)[NT], int lane, int *o
 }
 
 // ----------------------------------------------------------------------------
-// the derivative over one chunk of 16 channels, both directions
-// ----------------------------------------------------------------------------
-// ----------------------------------------------------------------------------
 // the derivative over one chunk of CH channels, both directions
 // ----------------------------------------------------------------------------
 template <int N> struct BwdShape {
     static constexpr int NT = N < VIMSCAN_BWD_NT ? N : VIMSCAN_BWD_NT;   // states per thread
+    static constexpr int NP = NT / 2;                        // state pairs per thread (f32x2 arithmetic)
     static constexpr int CKW = (NT + 3) / 4;                 // float4 per checkpoint per thread
     static constexpr int Q = N / NT;                         // threads per (channel, direction)
     static constexpr int CH = 32 / Q > 16 ? 32 / Q : 16;     // channels per CTA (whole warps per direction)
@@ -220,34 +222,48 @@ template <int N> struct BwdShape {
     static constexpr int CW = 32 / Q;                        // channels per warp
     static constexpr int kMinBlocks = VIMSCAN_BWD_MIN_WARPS * 32 / kThr;
     static constexpr int TC = kBwdChunk;
+    // With 4 lanes of 4 states per channel the sums over a warp's channels of the dB/dC
+    // terms go through a transposition in shared memory (every lane stores its 4 terms,
+    // then each lane adds up one pair of outputs); otherwise through shuffles.
+    static constexpr bool XPOSE = Q == 4 && NT == 4;
+    static constexpr int kXT = 2;                            // tokens per transposition
     // shared memory, in floats (every row of the chunk):
-    //   tok[2][TC][CH] float4 {Delta, u, dy, sigmoid(delta_raw + bias)} per direction
-    //   yb[2][TC][CH]  y^k in the forward sweep, then du^k in the adjoint sweep
-    //   dd[2][TC][CH]  d delta_raw from direction k
-    //   B[2][TC][N], C[2][TC][N]
-    //   red[2][WPD][TC][N]  per direction and warp: the dC terms, then the dB terms
-    //   ck[kBwdNSeg][CKW][kThr] float4  h at every kBwdSeg-th token, per thread
+    //   tok [TC][CH] float4 {u, dy, Delta^0, Delta^1}
+    //   sig [TC][CH] float2 {sigmoid(delta_raw + bias^0), sigmoid(delta_raw + bias^1)}
+    //   yb  [2][TC][CH]  y^k in the forward sweep, then du^k in the adjoint sweep
+    //   dd  [2][TC][CH]  d delta_raw from direction k
+    //   B, C [2][TC][N]
+    //   red [2][WPD][TC][N]  per direction and warp: the dC terms, then the dB terms
+    //   xb  [kThr / 32][kXT][32] float4  (XPOSE) one warp's per-lane terms of kXT tokens
+    //   ck  [kBwdNSeg][CKW][kThr] float4  h at every kBwdSeg-th token, per thread
     static constexpr int oTok = 0;
-    static constexpr int oYb = oTok + 2 * TC * CH * 4;
+    static constexpr int oSig = oTok + TC * CH * 4;
+    static constexpr int oYb = oSig + TC * CH * 2;
     static constexpr int oDd = oYb + 2 * TC * CH;
     static constexpr int oB = oDd + 2 * TC * CH;
     static constexpr int oC = oB + 2 * TC * N;
     static constexpr int oRed = oC + 2 * TC * N;
-    static constexpr int oCk = oRed + 2 * WPD * TC * N;
+    static constexpr int oXb = oRed + 2 * WPD * TC * N;
+    static constexpr int oCk = oXb + (XPOSE ? (kThr / 32) * kXT * 32 * 4 : 0);
     static constexpr int kFloats = oCk + kBwdNSeg * CKW * kThr * 4;
     static constexpr size_t kSmemBytes = (size_t)kFloats * 4;
-    static_assert(oCk % 4 == 0 && oTok % 4 == 0, "float4 areas must be 16-byte aligned");
+    static_assert(oCk % 4 == 0 && oXb % 4 == 0 && oB % 4 == 0 && oC % 4 == 0 && oRed % 4 == 0,
+                  "float4 areas must be 16-byte aligned");
+    static_assert(oSig % 2 == 0, "float2 area must be 8-byte aligned");
+    static_assert(NT % 2 == 0, "states per thread come in pairs");
 };
 
 template <int N>
 struct BwdSmem {
     using SH = BwdShape<N>;
     float4 *tok;
+    float2 *sig;
     float *yb, *dd, *B, *C, *red;
-    float4 *ck;
+    float4 *xb, *ck;
     __device__ explicit BwdSmem(float *base)
-        : tok(reinterpret_cast<float4 *>(base + SH::oTok)), yb(base + SH::oYb), dd(base + SH::oDd),
-          B(base + SH::oB), C(base + SH::oC), red(base + SH::oRed), ck(reinterpret_cast<float4 *>(base + SH::oCk)) {}
+        : tok(reinterpret_cast<float4 *>(base + SH::oTok)), sig(reinterpret_cast<float2 *>(base + SH::oSig)),
+          yb(base + SH::oYb), dd(base + SH::oDd), B(base + SH::oB), C(base + SH::oC), red(base + SH::oRed),
+          xb(reinterpret_cast<float4 *>(base + SH::oXb)), ck(reinterpret_cast<float4 *>(base + SH::oCk)) {}
 };
 
 // per-thread identity and parameters of one (channel, direction, state group)
@@ -256,22 +272,77 @@ struct BwdThread {
     using SH = BwdShape<N>;
     int tid, lane, q, cl, dir, wid, j0, d;
     bool valid;
-    float A2[SH::NT], Araw[SH::NT];
+    float2 A2[SH::NP], Araw[SH::NP];   // A of the thread's states, times log2(e) and as given
     float Dk;
     size_t cbase;   // [b][c][dir][d]
 };
 
-template <int NT>
-__device__ __forceinline__ void load_states(const float *row, float (&v)[NT]) {
-    if constexpr (NT % 4 == 0) {
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+// h (or g) of the thread's states, from an fp32 row in global memory
+template <int NP>
+__device__ __forceinline__ void load_pairs(const float *row, float2 (&v)[NP]) {
+    const float2 *r2 = reinterpret_cast<const float2 *>(row);
 #pragma unroll
-        for (int q = 0; q < NT / 4; ++q) {
-            const float4 t = *reinterpret_cast<const float4 *>(row + 4 * q);
-            v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
-        }
+    for (int k = 0; k < NP; ++k) v[k] = r2[k];
+}
+
+// checkpoint of h for segment sg (float4 slots, unused lanes of the last slot zero)
+template <int N>
+__device__ __forceinline__ void store_ck(const BwdSmem<N> &sm, int tid, int sg, const float2 (&h)[BwdShape<N>::NP]) {
+    using SH = BwdShape<N>;
+#pragma unroll
+    for (int w = 0; w < SH::CKW; ++w) {
+        const float2 lo = h[2 * w], hi = 2 * w + 1 < SH::NP ? h[2 * w + 1 < SH::NP ? 2 * w + 1 : 0] : f2(0.f, 0.f);
+        sm.ck[(sg * SH::CKW + w) * SH::kThr + tid] = make_float4(lo.x, lo.y, hi.x, hi.y);
+    }
+}
+template <int N>
+__device__ __forceinline__ void load_ck(const BwdSmem<N> &sm, int tid, int sg, float2 (&h)[BwdShape<N>::NP]) {
+    using SH = BwdShape<N>;
+#pragma unroll
+    for (int w = 0; w < SH::CKW; ++w) {
+        const float4 c4 = sm.ck[(sg * SH::CKW + w) * SH::kThr + tid];
+        h[2 * w] = f2(c4.x, c4.y);
+        if (2 * w + 1 < SH::NP) h[2 * w + 1 < SH::NP ? 2 * w + 1 : 0] = f2(c4.z, c4.w);
+    }
+}
+
+// One token's dB (or dC) terms of this thread's states, summed over the warp's channels
+// into red_w[row][n] (red_w: this direction's and warp's slots).  With XPOSE the terms
+// are buffered for kXT tokens (slot = position among them; flush after the last, with
+// the rows of slots 0 and 1), otherwise reduced at once by shuffles.
+template <int N>
+__device__ __forceinline__ void channel_sum(const BwdSmem<N> &sm, const BwdThread<N> &th, float *red_w,
+                                            const float2 (&v)[BwdShape<N>::NP], int slot, bool flush, int r0,
+                                            int r1) {
+    using SH = BwdShape<N>;
+    if constexpr (SH::XPOSE) {
+        float4 *buf = sm.xb + (th.tid >> 5) * SH::kXT * 32;
+        buf[slot * 32 + th.lane] = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
+        if (!flush) return;
+        __syncwarp();
+        // lane o adds up half the channels (4 * half ..) of output pair e2 (states 2 e2,
+        // 2 e2 + 1) of token slot mm; the channel order is rotated by mm so that the two
+        // token slots read disjoint banks.  Lane (c, q) stored states 4q .. 4q+3 of
+        // channel c at float2 index c * 8 + 2q of its slot's 64.
+        const int o = th.lane, half = o >> 4, mm = (o >> 3) & 1, e2 = o & 7;
+        const float2 *b2 = reinterpret_cast<const float2 *>(buf) + mm * 64 + e2;
+        float2 s = b2[(half * 4 + (mm & 3)) * 8];
+#pragma unroll
+        for (int k = 1; k < 4; ++k) s = add2(s, b2[(half * 4 + ((k + mm) & 3)) * 8]);
+        s.x += __shfl_xor_sync(0xffffffffu, s.x, 16);
+        s.y += __shfl_xor_sync(0xffffffffu, s.y, 16);
+        __syncwarp();
+        if (half == 0) *reinterpret_cast<float2 *>(red_w + (mm ? r1 : r0) * N + 2 * e2) = s;
     } else {
+        float w[SH::NT];
 #pragma unroll
-        for (int j = 0; j < NT; ++j) v[j] = row[j];
+        for (int k = 0; k < SH::NP; ++k) { w[2 * k] = v[k].x; w[2 * k + 1] = v[k].y; }
+        int off;
+        bool wr;
+        reduce_channels<SH::NT, SH::Q, SH::CW>(w, th.lane, &off, &wr);
+        if (wr) red_w[r1 * N + th.j0 + off] = w[0];
     }
 }
 
@@ -279,41 +350,39 @@ __device__ __forceinline__ void load_states(const float *row, float (&v)[NT]) {
 template <int N, int DIR>
 __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
     using SH = BwdShape<N>;
-    constexpr int NT = SH::NT, Q = SH::Q, CH = SH::CH, TC = SH::TC;
-    float h[NT];
+    constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
+    float *red_w = sm.red + (DIR * SH::WPD + th.wid) * TC * N;
+    float2 h[NP];
 #pragma unroll
-    for (int j = 0; j < NT; ++j) h[j] = (p.G > 1 && th.valid) ? p.hin[th.cbase * N + th.j0 + j] : 0.0f;
+    for (int k = 0; k < NP; ++k) h[k] = f2(0.f, 0.f);
+    if (p.G > 1 && th.valid) load_pairs<NP>(p.hin + th.cbase * N + th.j0, h);
+    int rprev = 0;
 #pragma unroll 1
     for (int sg = 0; sg < kBwdNSeg; ++sg) {
-#pragma unroll
-        for (int w = 0; w < SH::CKW; ++w) {
-            float q4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) q4[e] = 4 * w + e < NT ? h[4 * w + e < NT ? 4 * w + e : 0] : 0.0f;
-            sm.ck[(sg * SH::CKW + w) * SH::kThr + th.tid] = make_float4(q4[0], q4[1], q4[2], q4[3]);
-        }
+        store_ck<N>(sm, th.tid, sg, h);
 #pragma unroll
         for (int m = 0; m < kBwdSeg; ++m) {
             const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
-            const float4 tk = sm.tok[(DIR * TC + r) * CH + th.cl];   // Delta, u, dy, sigmoid
-            float Bv[NT], Cv[NT], v[NT];
-            load_states<NT>(sm.B + (DIR * TC + r) * N + th.j0, Bv);
-            load_states<NT>(sm.C + (DIR * TC + r) * N + th.j0, Cv);
-            const float du = tk.x * tk.y;
-            float yp = th.q == 0 ? th.Dk * tk.y : 0.0f;
+            const float4 tk = sm.tok[r * CH + th.cl];   // u, dy, Delta^0, Delta^1
+            const float dl = DIR ? tk.w : tk.z, du = dl * tk.x;
+            float2 Bp[NP], Cp[NP], v[NP];
+            load_row<NP>(sm.B + (DIR * TC + r) * N + th.j0, Bp);
+            load_row<NP>(sm.C + (DIR * TC + r) * N + th.j0, Cp);
+            const float2 dl2 = f2(dl, dl), du2 = f2(du, du), dy2 = f2(tk.y, tk.y);
+            float2 yp = f2(th.q == 0 ? th.Dk * tk.x : 0.0f, 0.0f);
 #pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                h[j] = fmaf(ex2(tk.x * th.A2[j]), h[j], du * Bv[j]);
-                yp = fmaf(Cv[j], h[j], yp);
-                v[j] = tk.z * h[j];
+            for (int k = 0; k < NP; ++k) {
+                const float2 e = mul2(dl2, th.A2[k]);
+                h[k] = fma2(f2(ex2(e.x), ex2(e.y)), h[k], mul2(du2, Bp[k]));
+                yp = fma2(Cp[k], h[k], yp);
+                v[k] = mul2(dy2, h[k]);
             }
+            float y = yp.x + yp.y;
 #pragma unroll
-            for (int s = 1; s < Q; s <<= 1) yp += __shfl_xor_sync(0xffffffffu, yp, s);
-            if (th.q == 0) sm.yb[(DIR * TC + r) * CH + th.cl] = yp;
-            int off;
-            bool wr;
-            reduce_channels<NT, Q, SH::CW>(v, th.lane, &off, &wr);
-            if (wr) sm.red[((DIR * SH::WPD + th.wid) * TC + r) * N + th.j0 + off] = v[0];
+            for (int s = 1; s < Q; s <<= 1) y += __shfl_xor_sync(0xffffffffu, y, s);
+            if (th.q == 0) sm.yb[(DIR * TC + r) * CH + th.cl] = y;
+            channel_sum<N>(sm, th, red_w, v, m & 1, (m & 1) == 1, rprev, r);
+            rprev = r;
         }
     }
 }
@@ -323,62 +392,66 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
 template <int N, int DIR>
 __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
     using SH = BwdShape<N>;
-    constexpr int NT = SH::NT, Q = SH::Q, CH = SH::CH, TC = SH::TC;
+    constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
     // with Q > 1 lane q = 0 gathers du and lane q = 1 d delta_raw of the channel
     constexpr int kDdLane = Q > 1 ? 1 : 0;
-    float g[NT], dA[NT];
+    float *red_w = sm.red + (DIR * SH::WPD + th.wid) * TC * N;
+    float2 g[NP], dA[NP];
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-        g[j] = (p.G > 1 && th.valid) ? p.gloc[th.cbase * N + th.j0 + j] : 0.0f;
-        dA[j] = 0.0f;
+    for (int k = 0; k < NP; ++k) {
+        g[k] = f2(0.f, 0.f);
+        dA[k] = f2(0.f, 0.f);
     }
+    if (p.G > 1 && th.valid) load_pairs<NP>(p.gloc + th.cbase * N + th.j0, g);
     float dD = 0.0f, dbias = 0.0f;
+    int rprev = 0;
 #pragma unroll 1
     for (int sg = kBwdNSeg - 1; sg >= 0; --sg) {
-        float h0[4 * SH::CKW];
-#pragma unroll
-        for (int w = 0; w < SH::CKW; ++w) {
-            const float4 c4 = sm.ck[(sg * SH::CKW + w) * SH::kThr + th.tid];
-            h0[4 * w] = c4.x; h0[4 * w + 1] = c4.y; h0[4 * w + 2] = c4.z; h0[4 * w + 3] = c4.w;
-        }
-        float hh[kBwdSeg][NT], aa[kBwdSeg][NT];
+        float2 h0[NP];
+        load_ck<N>(sm, th.tid, sg, h0);
+        float2 hh[kBwdSeg][NP], aa[kBwdSeg][NP];
 #pragma unroll
         for (int m = 0; m < kBwdSeg; ++m) {
             const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
-            const float4 tk = sm.tok[(DIR * TC + r) * CH + th.cl];
-            float Bv[NT];
-            load_states<NT>(sm.B + (DIR * TC + r) * N + th.j0, Bv);
-            const float du = tk.x * tk.y;
+            const float4 tk = sm.tok[r * CH + th.cl];
+            const float dl = DIR ? tk.w : tk.z, du = dl * tk.x;
+            float2 Bp[NP];
+            load_row<NP>(sm.B + (DIR * TC + r) * N + th.j0, Bp);
+            const float2 dl2 = f2(dl, dl), du2 = f2(du, du);
 #pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                aa[m][j] = ex2(tk.x * th.A2[j]);
-                hh[m][j] = fmaf(aa[m][j], m > 0 ? hh[m > 0 ? m - 1 : 0][j] : h0[j], du * Bv[j]);
+            for (int k = 0; k < NP; ++k) {
+                const float2 e = mul2(dl2, th.A2[k]);
+                aa[m][k] = f2(ex2(e.x), ex2(e.y));
+                hh[m][k] = fma2(aa[m][k], m > 0 ? hh[m > 0 ? m - 1 : 0][k] : h0[k], mul2(du2, Bp[k]));
             }
         }
 #pragma unroll
         for (int m = kBwdSeg - 1; m >= 0; --m) {
             const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
-            const float4 tk = sm.tok[(DIR * TC + r) * CH + th.cl];   // Delta, u, dy, sigmoid
-            float Bv[NT], Cv[NT], v[NT];
-            load_states<NT>(sm.B + (DIR * TC + r) * N + th.j0, Bv);
-            load_states<NT>(sm.C + (DIR * TC + r) * N + th.j0, Cv);
-            const float du = tk.x * tk.y;
-            float sA = 0.0f, sBg = 0.0f;
+            const float4 tk = sm.tok[r * CH + th.cl];   // u, dy, Delta^0, Delta^1
+            const float2 sgm2 = sm.sig[r * CH + th.cl];
+            const float dl = DIR ? tk.w : tk.z, sgm = DIR ? sgm2.y : sgm2.x, du = dl * tk.x;
+            float2 Bp[NP], Cp[NP], v[NP];
+            load_row<NP>(sm.B + (DIR * TC + r) * N + th.j0, Bp);
+            load_row<NP>(sm.C + (DIR * TC + r) * N + th.j0, Cp);
+            const float2 dl2 = f2(dl, dl), du2 = f2(du, du), dy2 = f2(tk.y, tk.y);
+            float2 sA = f2(0.f, 0.f), sB = f2(0.f, 0.f);
 #pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                g[j] = fmaf(Cv[j], tk.z, g[j]);                           // dl/dh_t
-                const float hp = m > 0 ? hh[m > 0 ? m - 1 : 0][j] : h0[j];  // h_(t-1)
-                const float ga = aa[m][j] * g[j];
-                const float w = ga * hp;
-                dA[j] = fmaf(tk.x, w, dA[j]);
-                sA = fmaf(th.Araw[j], w, sA);
-                sBg = fmaf(g[j], Bv[j], sBg);
-                v[j] = g[j] * du;
-                g[j] = ga;                                                // dl/dh_(t-1) part
+            for (int k = 0; k < NP; ++k) {
+                g[k] = fma2(Cp[k], dy2, g[k]);                               // dl/dh_t
+                const float2 hp = m > 0 ? hh[m > 0 ? m - 1 : 0][k] : h0[k];  // h_(t-1)
+                const float2 ga = mul2(aa[m][k], g[k]);
+                const float2 w = mul2(ga, hp);
+                dA[k] = fma2(dl2, w, dA[k]);
+                sA = fma2(th.Araw[k], w, sA);
+                sB = fma2(g[k], Bp[k], sB);
+                v[k] = mul2(g[k], du2);
+                g[k] = ga;                                                   // dl/dh_(t-1) part
             }
+            const float sAs = sA.x + sA.y, sBg = sB.x + sB.y;
             // this thread's share of du and d delta_raw, gathered over the Q lanes of
             // the channel: lane q = 0 ends with du, lane q = 1 with d delta_raw
-            float x0 = tk.x * sBg, x1 = fmaf(tk.y, sBg, sA) * tk.w;
+            float x0 = dl * sBg, x1 = fmaf(tk.x, sBg, sAs) * sgm;
             if constexpr (Q > 1) {
                 const bool odd = (th.q & 1) != 0;
                 const float send = odd ? x0 : x1;
@@ -390,25 +463,25 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
                 x1 = keep;
             }
             if (th.q == 0) {
-                sm.yb[(DIR * TC + r) * CH + th.cl] = fmaf(th.Dk, tk.z, x0);
-                dD = fmaf(tk.z, tk.y, dD);
+                sm.yb[(DIR * TC + r) * CH + th.cl] = fmaf(th.Dk, tk.y, x0);
+                dD = fmaf(tk.y, tk.x, dD);
             }
             if (th.q == kDdLane) {
                 sm.dd[(DIR * TC + r) * CH + th.cl] = x1;
                 dbias += x1;
             }
-            int off;
-            bool wr;
-            reduce_channels<NT, Q, SH::CW>(v, th.lane, &off, &wr);
-            if (wr) sm.red[((DIR * SH::WPD + th.wid) * TC + r) * N + th.j0 + off] = v[0];
+            // token slots: the segment's tokens m = 3, 2 go to slots 0, 1 (then 1, 0)
+            channel_sum<N>(sm, th, red_w, v, (kBwdSeg - 1 - m) & 1, ((kBwdSeg - 1 - m) & 1) == 1, rprev, r);
+            rprev = r;
         }
     }
     if (th.valid) {
         // row (b, c) of par; cbase = (row * 2 + dir) * Di + d
         const size_t row = th.cbase / ((size_t)2 * p.Di), col = th.cbase % ((size_t)2 * p.Di);
         float *pr = p.par + row * ((size_t)2 * p.Di * (N + 2));
+        float2 *pa = reinterpret_cast<float2 *>(pr + col * N + th.j0);
 #pragma unroll
-        for (int j = 0; j < NT; ++j) pr[col * N + th.j0 + j] = dA[j];
+        for (int k = 0; k < NP; ++k) pa[k] = dA[k];
         if (th.q == 0) pr[(size_t)2 * p.Di * N + col] = dD;
         if (th.q == kDdLane) pr[(size_t)2 * p.Di * (N + 1) + col] = dbias;
     }
@@ -416,55 +489,139 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
 
 // The CTA's per-token sums over its channels of the dB (or dC) terms, from the
 // per-direction, per-warp slots, into part[set][b][t][blk][n]: the two directions
-// add into one set when B and C are shared.
+// add into one set when B and C are shared.  Four states at a time.
 template <int N>
 __device__ __forceinline__ void store_bc_part(const BwdArgs &p, const float *red, float *const (&part)[2], int b,
                                               int t0, int tc, int blk) {
     using SH = BwdShape<N>;
-    constexpr int TC = SH::TC;
+    constexpr int TC = SH::TC, V = N % 4 == 0 ? 4 : 2;
     const int nsets = p.separate_bc ? 2 : 1;
-    for (int li = threadIdx.x; li < nsets * TC * N; li += SH::kThr) {
-        const int k = li / (TC * N), r = (li / N) % TC, n = li % N;
+    for (int li = threadIdx.x; li < nsets * TC * (N / V); li += SH::kThr) {
+        const int k = li / (TC * (N / V)), r = (li / (N / V)) % TC, n = (li % (N / V)) * V;
         if (r >= tc) continue;
-        float acc = 0.0f;
+        float acc[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] = 0.0f;
 #pragma unroll
         for (int dir = 0; dir < 2; ++dir) {
             if (p.separate_bc && dir != k) continue;
 #pragma unroll
-            for (int w = 0; w < SH::WPD; ++w) acc += red[((dir * SH::WPD + w) * TC + r) * N + n];
+            for (int w = 0; w < SH::WPD; ++w) {
+                const float *src = red + ((dir * SH::WPD + w) * TC + r) * N + n;
+#pragma unroll
+                for (int e = 0; e < V; ++e) acc[e] += src[e];
+            }
         }
-        part[k][(((size_t)b * p.L + bpos(p, t0 + r)) * p.nblk + blk) * N + n] = acc;
+        float *dst = part[k] + (((size_t)b * p.L + bpos(p, t0 + r)) * p.nblk + blk) * N + n;
+        if constexpr (V == 4) *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        else *reinterpret_cast<float2 *>(dst) = f2(acc[0], acc[1]);
+    }
+}
+
+// four consecutive channels of an [.., Di] tensor of T (16-byte vector loads for fp32,
+// 8-byte for bf16; the channel index is a multiple of 4)
+template <typename T>
+__device__ __forceinline__ void load4(const void *base, size_t i, bool vec, float (&f)[4]) {
+    const T *s = static_cast<const T *>(base) + i;
+    if (vec) {
+        if constexpr (sizeof(T) == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(s);
+            f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+        } else {
+            const uint2 v = *reinterpret_cast<const uint2 *>(s);
+            f[0] = __uint_as_float(v.x << 16); f[1] = __uint_as_float(v.x & 0xffff0000u);
+            f[2] = __uint_as_float(v.y << 16); f[3] = __uint_as_float(v.y & 0xffff0000u);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) f[e] = to_f32(s[e]);
+    }
+}
+template <typename T>
+__device__ __forceinline__ void store4(void *base, size_t i, bool vec, const float (&f)[4]) {
+    T *d = static_cast<T *>(base) + i;
+    if (vec) {
+        if constexpr (sizeof(T) == 4) {
+            *reinterpret_cast<float4 *>(d) = make_float4(f[0], f[1], f[2], f[3]);
+        } else {
+            __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]), c = __floats2bfloat162_rn(f[2], f[3]);
+            *reinterpret_cast<uint2 *>(d) =
+                make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&c));
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) d[e] = from_f32<T>(f[e]);
     }
 }
 
 template <typename T, int N>
 __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bwd_main(BwdArgs p) {
     using SH = BwdShape<N>;
-    constexpr int NT = SH::NT, Q = SH::Q, CH = SH::CH, TC = SH::TC;
+    constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
+    constexpr int kG = 4;   // channels per staged or stored group (d_inner is a multiple of 4)
     extern __shared__ __align__(16) float smem_f[];
     const BwdSmem<N> sm(smem_f);
 
     const int b = blockIdx.z, c = blockIdx.y, blk = blockIdx.x, d0 = blk * CH;
     const int t0 = c * TC, tc = min(TC, p.L - t0);
+    const bool vio = p.vec_io != 0;
 
-    // ---- stage the chunk: {Delta, u, dy, sigmoid} per direction, B and C ------------
-    for (int li = threadIdx.x; li < TC * CH; li += SH::kThr) {
-        const int r = li / CH, cl = li % CH, ch = d0 + cl;
-        float u = 0.0f, e = 0.0f, dl0 = 0.0f, dl1 = 0.0f, sg0 = 0.0f, sg1 = 0.0f;
-        if (r < tc && ch < p.Di) {
+    // ---- stage the chunk: {u, dy, Delta^0, Delta^1} and the sigmoids per (token,
+    // channel), four channels per item; B and C rows ------------------------------------
+    for (int li = threadIdx.x; li < TC * (CH / kG); li += SH::kThr) {
+        const int r = li / (CH / kG), c0 = (li % (CH / kG)) * kG, ch = d0 + c0;
+        const bool ok = r < tc && ch < p.Di;
+        float u[kG], dr[kG], e[kG];
+#pragma unroll
+        for (int k = 0; k < kG; ++k) { u[k] = 0.0f; dr[k] = 0.0f; e[k] = 0.0f; }
+        if (ok) {
             const size_t i = ((size_t)b * p.L + bpos(p, t0 + r)) * p.Di + ch;
-            u = ld<T>(p.u, i);
-            const float dr = ld<T>(p.delta, i);
-            e = ld<T>(p.dout, i);
-            if (p.z) e *= silu(ld<T>(p.z, i));
-            const float x0 = dr + p.bias[ch], x1 = dr + p.bias[p.Di + ch];
-            dl0 = softplus_io<T>(x0); sg0 = softplus_grad(x0);
-            dl1 = softplus_io<T>(x1); sg1 = softplus_grad(x1);
+            load4<T>(p.u, i, vio, u);
+            load4<T>(p.delta, i, vio, dr);
+            load4<T>(p.dout, i, vio, e);
+            if (p.z) {
+                float zz[kG];
+                load4<T>(p.z, i, vio, zz);
+#pragma unroll
+                for (int k = 0; k < kG; ++k) e[k] *= silu(zz[k]);
+            }
         }
-        sm.tok[r * CH + cl] = make_float4(dl0, u, e, sg0);
-        sm.tok[(TC + r) * CH + cl] = make_float4(dl1, u, e, sg1);
+#pragma unroll
+        for (int k = 0; k < kG; ++k) {
+            float dl0 = 0.0f, dl1 = 0.0f, sg0 = 0.0f, sg1 = 0.0f;
+            if (ok) {
+                const float x0 = dr[k] + p.bias[ch + k], x1 = dr[k] + p.bias[p.Di + ch + k];
+                dl0 = softplus_io<T>(x0); sg0 = softplus_grad(x0);
+                dl1 = softplus_io<T>(x1); sg1 = softplus_grad(x1);
+            }
+            sm.tok[r * CH + c0 + k] = make_float4(u[k], e[k], dl0, dl1);
+            sm.sig[r * CH + c0 + k] = f2(sg0, sg1);
+        }
     }
-    for (int li = threadIdx.x; li < 2 * TC * N; li += SH::kThr) {
+    bool bc_done = false;
+    if constexpr ((N * sizeof(T)) % 16 == 0) {
+        if (p.vec_bc) {
+            constexpr int VB = 16 / (int)sizeof(T);   // states per 16-byte vector
+            constexpr int RV = N / VB;                 // vectors per row
+            for (int li = threadIdx.x; li < 2 * 2 * TC * RV; li += SH::kThr) {
+                const int which = li / (2 * TC * RV), k = (li / (TC * RV)) % 2, r = (li / RV) % TC, v = li % RV;
+                float f[VB];
+                if (r < tc) {
+                    const T *src = static_cast<const T *>(which ? p.C[k] : p.B[k]) +
+                                   ((size_t)b * p.L + bpos(p, t0 + r)) * N + v * VB;
+                    unpack16(*reinterpret_cast<const uint4 *>(src), f);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < VB; ++e) f[e] = 0.0f;
+                }
+                float4 *dst = reinterpret_cast<float4 *>((which ? sm.C : sm.B) + (k * TC + r) * N + v * VB);
+#pragma unroll
+                for (int e = 0; e < VB / 4; ++e) dst[e] = make_float4(f[4 * e], f[4 * e + 1], f[4 * e + 2], f[4 * e + 3]);
+            }
+            bc_done = true;
+        }
+    }
+    for (int li = threadIdx.x; !bc_done && li < 2 * TC * N; li += SH::kThr) {
         const int k = li / (TC * N), r = (li / N) % TC, n = li % N;
         const size_t i = ((size_t)b * p.L + (r < tc ? bpos(p, t0 + r) : 0)) * N + n;
         sm.B[li] = r < tc ? ld<T>(p.B[k], i) : 0.0f;
@@ -478,13 +635,15 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     th.cl = (th.tid / Q) % CH;
     th.dir = th.tid / (Q * CH);
     th.wid = (th.tid / 32) % SH::WPD;
-    th.j0 = th.q * NT;
+    th.j0 = th.q * SH::NT;
     th.d = d0 + th.cl;
     th.valid = th.d < p.Di;
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-        th.Araw[j] = th.valid ? p.A[((size_t)th.dir * p.Di + th.d) * N + th.j0 + j] : 0.0f;
-        th.A2[j] = th.Araw[j] * kLog2e;
+    for (int k = 0; k < NP; ++k) {
+        const float *Ar = p.A + ((size_t)th.dir * p.Di + (th.valid ? th.d : 0)) * N + th.j0 + 2 * k;
+        const float2 a = th.valid ? f2(Ar[0], Ar[1]) : f2(0.f, 0.f);
+        th.Araw[k] = a;
+        th.A2[k] = f2(a.x * kLog2e, a.y * kLog2e);
     }
     th.Dk = th.valid ? p.D[(size_t)th.dir * p.Di + th.d] : 0.0f;
     th.cbase = (((size_t)b * p.G + c) * 2 + th.dir) * p.Di + th.d;
@@ -496,16 +655,26 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     // dz = dout silu'(z) (sum of the directions' y), and the CTA's dC terms; the
     // cross-scan's first pair leaves its y for the second
     if (p.dz || p.stage == 1) {
-        for (int li = threadIdx.x; li < TC * CH; li += SH::kThr) {
-            const int r = li / CH, c2 = li % CH, ch = d0 + c2;
+        for (int li = threadIdx.x; li < TC * (CH / kG); li += SH::kThr) {
+            const int r = li / (CH / kG), c0 = (li % (CH / kG)) * kG, ch = d0 + c0;
             if (r < tc && ch < p.Di) {
                 const size_t i = ((size_t)b * p.L + bpos(p, t0 + r)) * p.Di + ch;
-                float y = sm.yb[r * CH + c2] + sm.yb[(TC + r) * CH + c2];
+                float y[kG];
+#pragma unroll
+                for (int k = 0; k < kG; ++k) y[k] = sm.yb[r * CH + c0 + k] + sm.yb[(TC + r) * CH + c0 + k];
                 if (p.stage == 1) {
-                    p.acc_y[i] = y;
+                    *reinterpret_cast<float4 *>(p.acc_y + i) = make_float4(y[0], y[1], y[2], y[3]);
                 } else {
-                    if (p.stage == 2) y += p.acc_y[i];
-                    static_cast<T *>(p.dz)[i] = from_f32<T>(ld<T>(p.dout, i) * silu_grad(ld<T>(p.z, i)) * y);
+                    if (p.stage == 2) {
+                        const float4 a = *reinterpret_cast<const float4 *>(p.acc_y + i);
+                        y[0] += a.x; y[1] += a.y; y[2] += a.z; y[3] += a.w;
+                    }
+                    float e[kG], zz[kG];
+                    load4<T>(p.dout, i, vio, e);
+                    load4<T>(p.z, i, vio, zz);
+#pragma unroll
+                    for (int k = 0; k < kG; ++k) y[k] *= e[k] * silu_grad(zz[k]);
+                    store4<T>(p.dz, i, vio, y);
                 }
             }
         }
@@ -516,22 +685,28 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     if (th.dir == 0) bwd_adjoint<N, 0>(p, sm, th);
     else bwd_adjoint<N, 1>(p, sm, th);
     __syncthreads();
-    for (int li = threadIdx.x; li < TC * CH; li += SH::kThr) {
-        const int r = li / CH, c2 = li % CH, ch = d0 + c2;
+    for (int li = threadIdx.x; li < TC * (CH / kG); li += SH::kThr) {
+        const int r = li / (CH / kG), c0 = (li % (CH / kG)) * kG, ch = d0 + c0;
         if (r < tc && ch < p.Di) {
             const size_t i = ((size_t)b * p.L + bpos(p, t0 + r)) * p.Di + ch;
-            float du = sm.yb[r * CH + c2] + sm.yb[(TC + r) * CH + c2];
-            float dd = sm.dd[r * CH + c2] + sm.dd[(TC + r) * CH + c2];
+            float du[kG], dd[kG];
+#pragma unroll
+            for (int k = 0; k < kG; ++k) {
+                du[k] = sm.yb[r * CH + c0 + k] + sm.yb[(TC + r) * CH + c0 + k];
+                dd[k] = sm.dd[r * CH + c0 + k] + sm.dd[(TC + r) * CH + c0 + k];
+            }
             if (p.stage == 1) {
-                p.acc_du[i] = du;
-                p.acc_dd[i] = dd;
+                *reinterpret_cast<float4 *>(p.acc_du + i) = make_float4(du[0], du[1], du[2], du[3]);
+                *reinterpret_cast<float4 *>(p.acc_dd + i) = make_float4(dd[0], dd[1], dd[2], dd[3]);
             } else {
                 if (p.stage == 2) {
-                    du += p.acc_du[i];
-                    dd += p.acc_dd[i];
+                    const float4 a = *reinterpret_cast<const float4 *>(p.acc_du + i);
+                    const float4 e = *reinterpret_cast<const float4 *>(p.acc_dd + i);
+                    du[0] += a.x; du[1] += a.y; du[2] += a.z; du[3] += a.w;
+                    dd[0] += e.x; dd[1] += e.y; dd[2] += e.z; dd[3] += e.w;
                 }
-                static_cast<T *>(p.du)[i] = from_f32<T>(du);
-                static_cast<T *>(p.ddelta)[i] = from_f32<T>(dd);
+                store4<T>(p.du, i, vio, du);
+                store4<T>(p.ddelta, i, vio, dd);
             }
         }
     }
