@@ -22,10 +22,9 @@
 // checkpoints go to shared memory); Q = N / NT threads share a channel.  Each warp
 // serves one direction, whose code is compiled separately so that its token addresses
 // are constants.
-// Sums over channels (dB, dC) are taken across the warp (through a transposition in
-// shared memory when 4 lanes share a channel, else by shuffles), then across the CTA's
-// warps and directions in shared memory, and written per CTA; sums over tokens (dA,
-// dD, dbias) are written per chunk.  Small reduction kernels finish both.
+// Sums over channels (dB, dC) are reduced across the warp by shuffles, then across
+// the CTA's warps and directions in shared memory, and written per CTA; sums over
+// tokens (dA, dD, dbias) are written per chunk.  Small reduction kernels finish both.
 // Every sum is taken in a fixed order (no floating-point atomics), so results repeat
 // bit for bit.
 #pragma once
@@ -86,6 +85,42 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 template <typename T>
 __device__ __forceinline__ float ld(const void *p, size_t i) { return to_f32(static_cast<const T *>(p)[i]); }
 
+// four consecutive channels of an [.., Di] tensor of T (16-byte vector loads for fp32,
+// 8-byte for bf16; the channel index is a multiple of 4)
+template <typename T>
+__device__ __forceinline__ void load4(const void *base, size_t i, bool vec, float (&f)[4]) {
+    const T *s = static_cast<const T *>(base) + i;
+    if (vec) {
+        if constexpr (sizeof(T) == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(s);
+            f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+        } else {
+            const uint2 v = *reinterpret_cast<const uint2 *>(s);
+            f[0] = __uint_as_float(v.x << 16); f[1] = __uint_as_float(v.x & 0xffff0000u);
+            f[2] = __uint_as_float(v.y << 16); f[3] = __uint_as_float(v.y & 0xffff0000u);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) f[e] = to_f32(s[e]);
+    }
+}
+template <typename T>
+__device__ __forceinline__ void store4(void *base, size_t i, bool vec, const float (&f)[4]) {
+    T *d = static_cast<T *>(base) + i;
+    if (vec) {
+        if constexpr (sizeof(T) == 4) {
+            *reinterpret_cast<float4 *>(d) = make_float4(f[0], f[1], f[2], f[3]);
+        } else {
+            __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]), c = __floats2bfloat162_rn(f[2], f[3]);
+            *reinterpret_cast<uint2 *>(d) =
+                make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&c));
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) d[e] = from_f32<T>(f[e]);
+    }
+}
+
 // d softplus / dx = 1 / (1 + e^-x), and 1 above the cut at 20
 __device__ __forceinline__ float softplus_grad(float x) {
     return x > 20.0f ? 1.0f : rcp(1.0f + ex2(-x * kLog2e));
@@ -105,23 +140,52 @@ __device__ __forceinline__ float silu_grad(float z) {
 // ----------------------------------------------------------------------------
 template <typename T, int N>
 __global__ void __launch_bounds__(2 * kAdjCh) adj_carry(BwdArgs p) {
-    __shared__ float sDr[kBwdChunk][kAdjCh], sDy[kBwdChunk][kAdjCh];
+    __shared__ __align__(16) float sDr[kBwdChunk][kAdjCh], sDy[kBwdChunk][kAdjCh];
     __shared__ __align__(16) float sC[2][kBwdChunk][N];
     const int b = blockIdx.z, c = blockIdx.y, d0 = blockIdx.x * kAdjCh;
     const int t0 = c * kBwdChunk, tc = min(kBwdChunk, p.L - t0);
-    for (int li = threadIdx.x; li < kBwdChunk * kAdjCh; li += 2 * kAdjCh) {
-        const int r = li / kAdjCh, cl = li % kAdjCh, ch = d0 + cl;
-        float dr = 0.0f, e = 0.0f;
+    // four channels per item (d_inner is a multiple of 4)
+    for (int li = threadIdx.x; li < kBwdChunk * (kAdjCh / 4); li += 2 * kAdjCh) {
+        const int r = li / (kAdjCh / 4), c0 = (li % (kAdjCh / 4)) * 4, ch = d0 + c0;
+        float dr[4] = {0.0f, 0.0f, 0.0f, 0.0f}, e[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         if (r < tc && ch < p.Di) {
             const size_t i = ((size_t)b * p.L + bpos(p, t0 + r)) * p.Di + ch;
-            dr = ld<T>(p.delta, i);
-            e = ld<T>(p.dout, i);
-            if (p.z) e *= silu(ld<T>(p.z, i));
+            load4<T>(p.delta, i, p.vec_io, dr);
+            load4<T>(p.dout, i, p.vec_io, e);
+            if (p.z) {
+                float zz[4];
+                load4<T>(p.z, i, p.vec_io, zz);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) e[k] *= silu(zz[k]);
+            }
         }
-        sDr[r][cl] = dr;
-        sDy[r][cl] = e;
+        *reinterpret_cast<float4 *>(&sDr[r][c0]) = make_float4(dr[0], dr[1], dr[2], dr[3]);
+        *reinterpret_cast<float4 *>(&sDy[r][c0]) = make_float4(e[0], e[1], e[2], e[3]);
     }
-    for (int li = threadIdx.x; li < 2 * kBwdChunk * N; li += 2 * kAdjCh) {
+    bool c_done = false;
+    if constexpr ((N * sizeof(T)) % 16 == 0) {
+        if (p.vec_bc) {
+            constexpr int VB = 16 / (int)sizeof(T), RV = N / VB;   // states per vector, vectors per row
+            for (int li = threadIdx.x; li < 2 * kBwdChunk * RV; li += 2 * kAdjCh) {
+                const int k = li / (kBwdChunk * RV), r = (li / RV) % kBwdChunk, v = li % RV;
+                float f[VB];
+                if (r < tc) {
+                    unpack16(*reinterpret_cast<const uint4 *>(static_cast<const T *>(p.C[k]) +
+                                                              ((size_t)b * p.L + bpos(p, t0 + r)) * N + v * VB),
+                             f);
+                } else {
+#pragma unroll
+                    for (int e2 = 0; e2 < VB; ++e2) f[e2] = 0.0f;
+                }
+                float4 *dst = reinterpret_cast<float4 *>(&sC[k][r][v * VB]);
+#pragma unroll
+                for (int e2 = 0; e2 < VB / 4; ++e2)
+                    dst[e2] = make_float4(f[4 * e2], f[4 * e2 + 1], f[4 * e2 + 2], f[4 * e2 + 3]);
+            }
+            c_done = true;
+        }
+    }
+    for (int li = threadIdx.x; !c_done && li < 2 * kBwdChunk * N; li += 2 * kAdjCh) {
         const int k = li / (kBwdChunk * N), r = (li / N) % kBwdChunk, n = li % N;
         sC[k][r][n] = r < tc ? ld<T>(p.C[k], ((size_t)b * p.L + bpos(p, t0 + r)) * N + n) : 0.0f;
     }
@@ -222,48 +286,40 @@ template <int N> struct BwdShape {
     static constexpr int CW = 32 / Q;                        // channels per warp
     static constexpr int kMinBlocks = VIMSCAN_BWD_MIN_WARPS * 32 / kThr;
     static constexpr int TC = kBwdChunk;
-    // With 4 lanes of 4 states per channel the sums over a warp's channels of the dB/dC
-    // terms go through a transposition in shared memory (every lane stores its 4 terms,
-    // then each lane adds up one pair of outputs); otherwise through shuffles.
-    static constexpr bool XPOSE = Q == 4 && NT == 4;
-    static constexpr int kXT = 2;                            // tokens per transposition
     // shared memory, in floats (every row of the chunk):
-    //   tok [TC][CH] float4 {u, dy, Delta^0, Delta^1}
-    //   sig [TC][CH] float2 {sigmoid(delta_raw + bias^0), sigmoid(delta_raw + bias^1)}
+    //   tok [TC][CH] float2 {u, dy}
+    //   dsg [2][TC][CH] float2 {Delta^k, sigmoid(delta_raw + bias^k)}
     //   yb  [2][TC][CH]  y^k in the forward sweep, then du^k in the adjoint sweep
     //   dd  [2][TC][CH]  d delta_raw from direction k
     //   B, C [2][TC][N]
     //   red [2][WPD][TC][N]  per direction and warp: the dC terms, then the dB terms
-    //   xb  [kThr / 32][kXT][32] float4  (XPOSE) one warp's per-lane terms of kXT tokens
     //   ck  [kBwdNSeg][CKW][kThr] float4  h at every kBwdSeg-th token, per thread
     static constexpr int oTok = 0;
-    static constexpr int oSig = oTok + TC * CH * 4;
-    static constexpr int oYb = oSig + TC * CH * 2;
+    static constexpr int oSig = oTok + TC * CH * 2;
+    static constexpr int oYb = oSig + 2 * TC * CH * 2;
     static constexpr int oDd = oYb + 2 * TC * CH;
     static constexpr int oB = oDd + 2 * TC * CH;
     static constexpr int oC = oB + 2 * TC * N;
     static constexpr int oRed = oC + 2 * TC * N;
-    static constexpr int oXb = oRed + 2 * WPD * TC * N;
-    static constexpr int oCk = oXb + (XPOSE ? (kThr / 32) * kXT * 32 * 4 : 0);
+    static constexpr int oCk = oRed + 2 * WPD * TC * N;
     static constexpr int kFloats = oCk + kBwdNSeg * CKW * kThr * 4;
     static constexpr size_t kSmemBytes = (size_t)kFloats * 4;
-    static_assert(oCk % 4 == 0 && oXb % 4 == 0 && oB % 4 == 0 && oC % 4 == 0 && oRed % 4 == 0,
+    static_assert(oCk % 4 == 0 && oB % 4 == 0 && oC % 4 == 0 && oRed % 4 == 0,
                   "float4 areas must be 16-byte aligned");
-    static_assert(oSig % 2 == 0, "float2 area must be 8-byte aligned");
+    static_assert(oSig % 2 == 0, "float2 areas must be 8-byte aligned");
     static_assert(NT % 2 == 0, "states per thread come in pairs");
 };
 
 template <int N>
 struct BwdSmem {
     using SH = BwdShape<N>;
-    float4 *tok;
-    float2 *sig;
+    float2 *tok, *dsg;
     float *yb, *dd, *B, *C, *red;
-    float4 *xb, *ck;
+    float4 *ck;
     __device__ explicit BwdSmem(float *base)
-        : tok(reinterpret_cast<float4 *>(base + SH::oTok)), sig(reinterpret_cast<float2 *>(base + SH::oSig)),
+        : tok(reinterpret_cast<float2 *>(base + SH::oTok)), dsg(reinterpret_cast<float2 *>(base + SH::oSig)),
           yb(base + SH::oYb), dd(base + SH::oDd), B(base + SH::oB), C(base + SH::oC), red(base + SH::oRed),
-          xb(reinterpret_cast<float4 *>(base + SH::oXb)), ck(reinterpret_cast<float4 *>(base + SH::oCk)) {}
+          ck(reinterpret_cast<float4 *>(base + SH::oCk)) {}
 };
 
 // per-thread identity and parameters of one (channel, direction, state group)
@@ -276,8 +332,6 @@ struct BwdThread {
     float Dk;
     size_t cbase;   // [b][c][dir][d]
 };
-
-__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
 // h (or g) of the thread's states, from an fp32 row in global memory
 template <int NP>
@@ -309,41 +363,18 @@ __device__ __forceinline__ void load_ck(const BwdSmem<N> &sm, int tid, int sg, f
 }
 
 // One token's dB (or dC) terms of this thread's states, summed over the warp's channels
-// into red_w[row][n] (red_w: this direction's and warp's slots).  With XPOSE the terms
-// are buffered for kXT tokens (slot = position among them; flush after the last, with
-// the rows of slots 0 and 1), otherwise reduced at once by shuffles.
+// by shuffles into red_w[r][n] (red_w: this direction's and warp's slots)
 template <int N>
-__device__ __forceinline__ void channel_sum(const BwdSmem<N> &sm, const BwdThread<N> &th, float *red_w,
-                                            const float2 (&v)[BwdShape<N>::NP], int slot, bool flush, int r0,
-                                            int r1) {
+__device__ __forceinline__ void channel_sum(const BwdThread<N> &th, float *red_w, const float2 (&v)[BwdShape<N>::NP],
+                                            int r) {
     using SH = BwdShape<N>;
-    if constexpr (SH::XPOSE) {
-        float4 *buf = sm.xb + (th.tid >> 5) * SH::kXT * 32;
-        buf[slot * 32 + th.lane] = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
-        if (!flush) return;
-        __syncwarp();
-        // lane o adds up half the channels (4 * half ..) of output pair e2 (states 2 e2,
-        // 2 e2 + 1) of token slot mm; the channel order is rotated by mm so that the two
-        // token slots read disjoint banks.  Lane (c, q) stored states 4q .. 4q+3 of
-        // channel c at float2 index c * 8 + 2q of its slot's 64.
-        const int o = th.lane, half = o >> 4, mm = (o >> 3) & 1, e2 = o & 7;
-        const float2 *b2 = reinterpret_cast<const float2 *>(buf) + mm * 64 + e2;
-        float2 s = b2[(half * 4 + (mm & 3)) * 8];
+    float w[SH::NT];
 #pragma unroll
-        for (int k = 1; k < 4; ++k) s = add2(s, b2[(half * 4 + ((k + mm) & 3)) * 8]);
-        s.x += __shfl_xor_sync(0xffffffffu, s.x, 16);
-        s.y += __shfl_xor_sync(0xffffffffu, s.y, 16);
-        __syncwarp();
-        if (half == 0) *reinterpret_cast<float2 *>(red_w + (mm ? r1 : r0) * N + 2 * e2) = s;
-    } else {
-        float w[SH::NT];
-#pragma unroll
-        for (int k = 0; k < SH::NP; ++k) { w[2 * k] = v[k].x; w[2 * k + 1] = v[k].y; }
-        int off;
-        bool wr;
-        reduce_channels<SH::NT, SH::Q, SH::CW>(w, th.lane, &off, &wr);
-        if (wr) red_w[r1 * N + th.j0 + off] = w[0];
-    }
+    for (int k = 0; k < SH::NP; ++k) { w[2 * k] = v[k].x; w[2 * k + 1] = v[k].y; }
+    int off;
+    bool wr;
+    reduce_channels<SH::NT, SH::Q, SH::CW>(w, th.lane, &off, &wr);
+    if (wr) red_w[r * N + th.j0 + off] = w[0];
 }
 
 // forward sweep of direction DIR: checkpoints, y^DIR (ungated) and the dC terms
@@ -356,15 +387,15 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
 #pragma unroll
     for (int k = 0; k < NP; ++k) h[k] = f2(0.f, 0.f);
     if (p.G > 1 && th.valid) load_pairs<NP>(p.hin + th.cbase * N + th.j0, h);
-    int rprev = 0;
 #pragma unroll 1
     for (int sg = 0; sg < kBwdNSeg; ++sg) {
         store_ck<N>(sm, th.tid, sg, h);
 #pragma unroll
         for (int m = 0; m < kBwdSeg; ++m) {
             const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
-            const float4 tk = sm.tok[r * CH + th.cl];   // u, dy, Delta^0, Delta^1
-            const float dl = DIR ? tk.w : tk.z, du = dl * tk.x;
+            const float2 tk = sm.tok[r * CH + th.cl];   // u, dy
+            const float dl = reinterpret_cast<const float *>(sm.dsg)[2 * ((DIR * TC + r) * CH + th.cl)];
+            const float du = dl * tk.x;
             float2 Bp[NP], Cp[NP], v[NP];
             load_row<NP>(sm.B + (DIR * TC + r) * N + th.j0, Bp);
             load_row<NP>(sm.C + (DIR * TC + r) * N + th.j0, Cp);
@@ -381,8 +412,7 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
 #pragma unroll
             for (int s = 1; s < Q; s <<= 1) y += __shfl_xor_sync(0xffffffffu, y, s);
             if (th.q == 0) sm.yb[(DIR * TC + r) * CH + th.cl] = y;
-            channel_sum<N>(sm, th, red_w, v, m & 1, (m & 1) == 1, rprev, r);
-            rprev = r;
+            channel_sum<N>(th, red_w, v, r);
         }
     }
 }
@@ -404,7 +434,6 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
     }
     if (p.G > 1 && th.valid) load_pairs<NP>(p.gloc + th.cbase * N + th.j0, g);
     float dD = 0.0f, dbias = 0.0f;
-    int rprev = 0;
 #pragma unroll 1
     for (int sg = kBwdNSeg - 1; sg >= 0; --sg) {
         float2 h0[NP];
@@ -413,8 +442,9 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
 #pragma unroll
         for (int m = 0; m < kBwdSeg; ++m) {
             const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
-            const float4 tk = sm.tok[r * CH + th.cl];
-            const float dl = DIR ? tk.w : tk.z, du = dl * tk.x;
+            const float u = reinterpret_cast<const float *>(sm.tok)[2 * (r * CH + th.cl)];
+            const float dl = reinterpret_cast<const float *>(sm.dsg)[2 * ((DIR * TC + r) * CH + th.cl)];
+            const float du = dl * u;
             float2 Bp[NP];
             load_row<NP>(sm.B + (DIR * TC + r) * N + th.j0, Bp);
             const float2 dl2 = f2(dl, dl), du2 = f2(du, du);
@@ -428,9 +458,9 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
 #pragma unroll
         for (int m = kBwdSeg - 1; m >= 0; --m) {
             const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
-            const float4 tk = sm.tok[r * CH + th.cl];   // u, dy, Delta^0, Delta^1
-            const float2 sgm2 = sm.sig[r * CH + th.cl];
-            const float dl = DIR ? tk.w : tk.z, sgm = DIR ? sgm2.y : sgm2.x, du = dl * tk.x;
+            const float2 tk = sm.tok[r * CH + th.cl];                   // u, dy
+            const float2 ds = sm.dsg[(DIR * TC + r) * CH + th.cl];      // Delta, sigmoid
+            const float dl = ds.x, sgm = ds.y, du = dl * tk.x;
             float2 Bp[NP], Cp[NP], v[NP];
             load_row<NP>(sm.B + (DIR * TC + r) * N + th.j0, Bp);
             load_row<NP>(sm.C + (DIR * TC + r) * N + th.j0, Cp);
@@ -470,9 +500,7 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
                 sm.dd[(DIR * TC + r) * CH + th.cl] = x1;
                 dbias += x1;
             }
-            // token slots: the segment's tokens m = 3, 2 go to slots 0, 1 (then 1, 0)
-            channel_sum<N>(sm, th, red_w, v, (kBwdSeg - 1 - m) & 1, ((kBwdSeg - 1 - m) & 1) == 1, rprev, r);
-            rprev = r;
+            channel_sum<N>(th, red_w, v, r);
         }
     }
     if (th.valid) {
@@ -518,42 +546,6 @@ __device__ __forceinline__ void store_bc_part(const BwdArgs &p, const float *red
     }
 }
 
-// four consecutive channels of an [.., Di] tensor of T (16-byte vector loads for fp32,
-// 8-byte for bf16; the channel index is a multiple of 4)
-template <typename T>
-__device__ __forceinline__ void load4(const void *base, size_t i, bool vec, float (&f)[4]) {
-    const T *s = static_cast<const T *>(base) + i;
-    if (vec) {
-        if constexpr (sizeof(T) == 4) {
-            const float4 v = *reinterpret_cast<const float4 *>(s);
-            f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
-        } else {
-            const uint2 v = *reinterpret_cast<const uint2 *>(s);
-            f[0] = __uint_as_float(v.x << 16); f[1] = __uint_as_float(v.x & 0xffff0000u);
-            f[2] = __uint_as_float(v.y << 16); f[3] = __uint_as_float(v.y & 0xffff0000u);
-        }
-    } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) f[e] = to_f32(s[e]);
-    }
-}
-template <typename T>
-__device__ __forceinline__ void store4(void *base, size_t i, bool vec, const float (&f)[4]) {
-    T *d = static_cast<T *>(base) + i;
-    if (vec) {
-        if constexpr (sizeof(T) == 4) {
-            *reinterpret_cast<float4 *>(d) = make_float4(f[0], f[1], f[2], f[3]);
-        } else {
-            __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]), c = __floats2bfloat162_rn(f[2], f[3]);
-            *reinterpret_cast<uint2 *>(d) =
-                make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&c));
-        }
-    } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) d[e] = from_f32<T>(f[e]);
-    }
-}
-
 template <typename T, int N>
 __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bwd_main(BwdArgs p) {
     using SH = BwdShape<N>;
@@ -566,7 +558,7 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     const int t0 = c * TC, tc = min(TC, p.L - t0);
     const bool vio = p.vec_io != 0;
 
-    // ---- stage the chunk: {u, dy, Delta^0, Delta^1} and the sigmoids per (token,
+    // ---- stage the chunk: {u, dy} and per direction {Delta, sigmoid} per (token,
     // channel), four channels per item; B and C rows ------------------------------------
     for (int li = threadIdx.x; li < TC * (CH / kG); li += SH::kThr) {
         const int r = li / (CH / kG), c0 = (li % (CH / kG)) * kG, ch = d0 + c0;
@@ -594,8 +586,9 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
                 dl0 = softplus_io<T>(x0); sg0 = softplus_grad(x0);
                 dl1 = softplus_io<T>(x1); sg1 = softplus_grad(x1);
             }
-            sm.tok[r * CH + c0 + k] = make_float4(u[k], e[k], dl0, dl1);
-            sm.sig[r * CH + c0 + k] = f2(sg0, sg1);
+            sm.tok[r * CH + c0 + k] = f2(u[k], e[k]);
+            sm.dsg[r * CH + c0 + k] = f2(dl0, sg0);
+            sm.dsg[(TC + r) * CH + c0 + k] = f2(dl1, sg1);
         }
     }
     bool bc_done = false;
