@@ -41,6 +41,9 @@ constexpr int kReduceParts = 32;              // row groups of the first paramet
 #ifndef VIMSCAN_BWD_NT
 #define VIMSCAN_BWD_NT 4                         // states per thread of bwd_main (4 or 8)
 #endif
+#ifndef VIMSCAN_BWD_BATCH
+#define VIMSCAN_BWD_BATCH 1                      // reductions batched over each segment's tokens
+#endif
 #ifndef VIMSCAN_BWD_MIN_WARPS
 #define VIMSCAN_BWD_MIN_WARPS 16                 // resident warps per SM the register budget targets
 #endif
@@ -272,6 +275,31 @@ __device__ __forceinline__ void reduce_channels(float (&v)[NT], int lane, int *o
     *writer = w && k == 1;
 }
 
+// Reduce-scatter of V values over the lanes whose index bits are S0, 2 S0, .. below S1:
+// at each bit the lane keeps the half of its values that the bit selects and adds
+// its partner's copy of that half.  On return v[0 ..) hold the sums of the values
+// that had indices off, off + 1, .. (off returned).
+template <int V, int S0, int S1>
+__device__ __forceinline__ int reduce_scatter(float (&v)[V], int lane) {
+    int k = V, off = 0;
+#pragma unroll
+    for (int s = S0; s < S1; s <<= 1) {
+        const bool hi = (lane & s) != 0;
+        const int half = k / 2;
+#pragma unroll
+        for (int i = 0; i < V / 2; ++i) {
+            if (i < half) {
+                const float send = hi ? v[i] : v[i + half];
+                const float keep = hi ? v[i + half] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+            }
+        }
+        off += hi ? half : 0;
+        k = half;
+    }
+    return off;
+}
+
 // ----------------------------------------------------------------------------
 // the derivative over one chunk of CH channels, both directions
 // ----------------------------------------------------------------------------
@@ -286,6 +314,9 @@ template <int N> struct BwdShape {
     static constexpr int CW = 32 / Q;                        // channels per warp
     static constexpr int kMinBlocks = VIMSCAN_BWD_MIN_WARPS * 32 / kThr;
     static constexpr int TC = kBwdChunk;
+    // with 4 lanes of 4 states per channel the shuffle reductions of a segment's tokens
+    // are taken together (reduce-scatter: independent shuffles, one store per lane)
+    static constexpr bool BATCH = Q == 4 && NT == 4 && VIMSCAN_BWD_BATCH;
     // shared memory, in floats (every row of the chunk):
     //   tok [TC][CH] float2 {u, dy}
     //   dsg [2][TC][CH] float2 {Delta^k, sigmoid(delta_raw + bias^k)}
@@ -390,6 +421,7 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
 #pragma unroll 1
     for (int sg = 0; sg < kBwdNSeg; ++sg) {
         store_ck<N>(sm, th.tid, sg, h);
+        float yv[kBwdSeg], vc[SH::BATCH ? kBwdSeg * SH::NT : 1];   // batched: y partials, dC terms
 #pragma unroll
         for (int m = 0; m < kBwdSeg; ++m) {
             const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
@@ -408,11 +440,26 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
                 yp = fma2(Cp[k], h[k], yp);
                 v[k] = mul2(dy2, h[k]);
             }
-            float y = yp.x + yp.y;
+            if constexpr (SH::BATCH) {
+                yv[m] = yp.x + yp.y;
 #pragma unroll
-            for (int s = 1; s < Q; s <<= 1) y += __shfl_xor_sync(0xffffffffu, y, s);
-            if (th.q == 0) sm.yb[(DIR * TC + r) * CH + th.cl] = y;
-            channel_sum<N>(th, red_w, v, r);
+                for (int k = 0; k < NP; ++k) { vc[m * SH::NT + 2 * k] = v[k].x; vc[m * SH::NT + 2 * k + 1] = v[k].y; }
+            } else {
+                float y = yp.x + yp.y;
+#pragma unroll
+                for (int s = 1; s < Q; s <<= 1) y += __shfl_xor_sync(0xffffffffu, y, s);
+                if (th.q == 0) sm.yb[(DIR * TC + r) * CH + th.cl] = y;
+                channel_sum<N>(th, red_w, v, r);
+            }
+        }
+        if constexpr (SH::BATCH) {
+            // y: one token of the segment per lane of the channel; dC: two terms per lane
+            const int oy = reduce_scatter<kBwdSeg, 1, Q>(yv, th.lane);
+            const int iy = sg * kBwdSeg + oy;
+            sm.yb[(DIR * TC + (DIR ? TC - 1 - iy : iy)) * CH + th.cl] = yv[0];
+            const int oc = reduce_scatter<kBwdSeg * SH::NT, Q, 32>(vc, th.lane);
+            const int ic = sg * kBwdSeg + oc / SH::NT;
+            *reinterpret_cast<float2 *>(red_w + (DIR ? TC - 1 - ic : ic) * N + th.j0 + oc % SH::NT) = f2(vc[0], vc[1]);
         }
     }
 }
@@ -439,6 +486,8 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
         float2 h0[NP];
         load_ck<N>(sm, th.tid, sg, h0);
         float2 hh[kBwdSeg][NP], aa[kBwdSeg][NP];
+        // batched: [slot][du, d delta_raw] partials and [slot][state] dB terms, slot = 3 - m
+        float xq[SH::BATCH ? 2 * kBwdSeg : 1], vb[SH::BATCH ? kBwdSeg * SH::NT : 1];
 #pragma unroll
         for (int m = 0; m < kBwdSeg; ++m) {
             const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
@@ -482,6 +531,14 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
             // this thread's share of du and d delta_raw, gathered over the Q lanes of
             // the channel: lane q = 0 ends with du, lane q = 1 with d delta_raw
             float x0 = dl * sBg, x1 = fmaf(tk.x, sBg, sAs) * sgm;
+            if constexpr (SH::BATCH) {
+                const int sl = kBwdSeg - 1 - m;
+                xq[2 * sl] = x0;
+                xq[2 * sl + 1] = x1;
+#pragma unroll
+                for (int k = 0; k < NP; ++k) { vb[sl * SH::NT + 2 * k] = v[k].x; vb[sl * SH::NT + 2 * k + 1] = v[k].y; }
+                continue;
+            }
             if constexpr (Q > 1) {
                 const bool odd = (th.q & 1) != 0;
                 const float send = odd ? x0 : x1;
@@ -501,6 +558,27 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
                 dbias += x1;
             }
             channel_sum<N>(th, red_w, v, r);
+        }
+        if constexpr (SH::BATCH) {
+            // du and d delta_raw of one token of the segment per lane of the channel
+            const int ox = reduce_scatter<2 * kBwdSeg, 1, Q>(xq, th.lane);
+            const int ix = sg * kBwdSeg + kBwdSeg - 1 - ox / 2, rx = DIR ? TC - 1 - ix : ix;
+            const float2 tk = sm.tok[rx * CH + th.cl];   // u, dy
+            sm.yb[(DIR * TC + rx) * CH + th.cl] = fmaf(th.Dk, tk.y, xq[0]);
+            sm.dd[(DIR * TC + rx) * CH + th.cl] = xq[1];
+            dD = fmaf(tk.y, tk.x, dD);
+            dbias += xq[1];
+            const int ob = reduce_scatter<kBwdSeg * SH::NT, Q, 32>(vb, th.lane);
+            const int ib = sg * kBwdSeg + kBwdSeg - 1 - ob / SH::NT;
+            *reinterpret_cast<float2 *>(red_w + (DIR ? TC - 1 - ib : ib) * N + th.j0 + ob % SH::NT) = f2(vb[0], vb[1]);
+        }
+    }
+    if constexpr (SH::BATCH) {
+        // every lane of the channel summed its own tokens
+#pragma unroll
+        for (int s = 1; s < Q; s <<= 1) {
+            dD += __shfl_xor_sync(0xffffffffu, dD, s);
+            dbias += __shfl_xor_sync(0xffffffffu, dbias, s);
         }
     }
     if (th.valid) {
