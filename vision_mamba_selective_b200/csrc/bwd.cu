@@ -92,7 +92,14 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
     constexpr size_t sm = BwdShape<N>::kSmemBytes;
     if (cudaFuncSetAttribute(bwd_main<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
         return VIM_ERR_CUDA;
-    bwd_main<T, N><<<dim3(a.nblk, a.G, a.batch), BwdShape<N>::kThr, sm, stream>>>(a);
+    const dim3 gm(a.nblk, a.G, a.batch);
+    if (a.G > 1) {
+        // staging overlaps the adjoint fold, which lets its dependents start early
+        if (launch_dependent(bwd_main<T, N>, gm, dim3(BwdShape<N>::kThr), sm, stream, a) != cudaSuccess)
+            return VIM_ERR_CUDA;
+    } else {
+        bwd_main<T, N><<<gm, BwdShape<N>::kThr, sm, stream>>>(a);
+    }
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     if (!rec(ev, 2, stream)) return VIM_ERR_CUDA;
     const int sets = a.separate_bc ? 2 : 1;

@@ -322,6 +322,7 @@ template <int N> struct BwdShape {
     //   dsg [2][TC][CH] float2 {Delta^k, sigmoid(delta_raw + bias^k)}
     //   yb  [2][TC][CH]  y^k in the forward sweep, then du^k in the adjoint sweep
     //   dd  [2][TC][CH]  d delta_raw from direction k
+    //   dzf [TC][CH]     dout silu'(z), dz's factor of y
     //   B, C [2][TC][N]
     //   red [2][WPD][TC][N]  per direction and warp: the dC terms, then the dB terms
     //   ck  [kBwdNSeg][CKW][kThr] float4  h at every kBwdSeg-th token, per thread
@@ -329,13 +330,15 @@ template <int N> struct BwdShape {
     static constexpr int oSig = oTok + TC * CH * 2;
     static constexpr int oYb = oSig + 2 * TC * CH * 2;
     static constexpr int oDd = oYb + 2 * TC * CH;
-    static constexpr int oB = oDd + 2 * TC * CH;
+    static constexpr int oDz = oDd + 2 * TC * CH;
+    static constexpr int oB = oDz + TC * CH;
     static constexpr int oC = oB + 2 * TC * N;
     static constexpr int oRed = oC + 2 * TC * N;
     static constexpr int oCk = oRed + 2 * WPD * TC * N;
     static constexpr int kFloats = oCk + kBwdNSeg * CKW * kThr * 4;
     static constexpr size_t kSmemBytes = (size_t)kFloats * 4;
-    static_assert(oCk % 4 == 0 && oB % 4 == 0 && oC % 4 == 0 && oRed % 4 == 0,
+    static_assert(oCk % 4 == 0 && oB % 4 == 0 && oC % 4 == 0 && oRed % 4 == 0 && oYb % 4 == 0 && oDd % 4 == 0 &&
+                      oDz % 4 == 0 && CH % 4 == 0,
                   "float4 areas must be 16-byte aligned");
     static_assert(oSig % 2 == 0, "float2 areas must be 8-byte aligned");
     static_assert(NT % 2 == 0, "states per thread come in pairs");
@@ -345,11 +348,11 @@ template <int N>
 struct BwdSmem {
     using SH = BwdShape<N>;
     float2 *tok, *dsg;
-    float *yb, *dd, *B, *C, *red;
+    float *yb, *dd, *dzf, *B, *C, *red;
     float4 *ck;
     __device__ explicit BwdSmem(float *base)
         : tok(reinterpret_cast<float2 *>(base + SH::oTok)), dsg(reinterpret_cast<float2 *>(base + SH::oSig)),
-          yb(base + SH::oYb), dd(base + SH::oDd), B(base + SH::oB), C(base + SH::oC), red(base + SH::oRed),
+          yb(base + SH::oYb), dd(base + SH::oDd), dzf(base + SH::oDz), B(base + SH::oB), C(base + SH::oC), red(base + SH::oRed),
           ck(reinterpret_cast<float4 *>(base + SH::oCk)) {}
 };
 
@@ -641,9 +644,9 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     for (int li = threadIdx.x; li < TC * (CH / kG); li += SH::kThr) {
         const int r = li / (CH / kG), c0 = (li % (CH / kG)) * kG, ch = d0 + c0;
         const bool ok = r < tc && ch < p.Di;
-        float u[kG], dr[kG], e[kG];
+        float u[kG], dr[kG], e[kG], zf[kG];
 #pragma unroll
-        for (int k = 0; k < kG; ++k) { u[k] = 0.0f; dr[k] = 0.0f; e[k] = 0.0f; }
+        for (int k = 0; k < kG; ++k) { u[k] = 0.0f; dr[k] = 0.0f; e[k] = 0.0f; zf[k] = 0.0f; }
         if (ok) {
             const size_t i = ((size_t)b * p.L + bpos(p, t0 + r)) * p.Di + ch;
             load4<T>(p.u, i, vio, u);
@@ -653,9 +656,13 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
                 float zz[kG];
                 load4<T>(p.z, i, vio, zz);
 #pragma unroll
-                for (int k = 0; k < kG; ++k) e[k] *= silu(zz[k]);
+                for (int k = 0; k < kG; ++k) {
+                    zf[k] = e[k] * silu_grad(zz[k]);
+                    e[k] *= silu(zz[k]);
+                }
             }
         }
+        float ds0[2 * kG], ds1[2 * kG];
 #pragma unroll
         for (int k = 0; k < kG; ++k) {
             float dl0 = 0.0f, dl1 = 0.0f, sg0 = 0.0f, sg1 = 0.0f;
@@ -664,10 +671,20 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
                 dl0 = softplus_io<T>(x0); sg0 = softplus_grad(x0);
                 dl1 = softplus_io<T>(x1); sg1 = softplus_grad(x1);
             }
-            sm.tok[r * CH + c0 + k] = f2(u[k], e[k]);
-            sm.dsg[r * CH + c0 + k] = f2(dl0, sg0);
-            sm.dsg[(TC + r) * CH + c0 + k] = f2(dl1, sg1);
+            ds0[2 * k] = dl0; ds0[2 * k + 1] = sg0;
+            ds1[2 * k] = dl1; ds1[2 * k + 1] = sg1;
         }
+        // 16-byte stores: two channels' pairs per float4
+        float4 *t4 = reinterpret_cast<float4 *>(sm.tok + r * CH + c0);
+        float4 *d4 = reinterpret_cast<float4 *>(sm.dsg + r * CH + c0);
+        float4 *e4 = reinterpret_cast<float4 *>(sm.dsg + (TC + r) * CH + c0);
+#pragma unroll
+        for (int h = 0; h < kG / 2; ++h) {
+            t4[h] = make_float4(u[2 * h], e[2 * h], u[2 * h + 1], e[2 * h + 1]);
+            d4[h] = make_float4(ds0[4 * h], ds0[4 * h + 1], ds0[4 * h + 2], ds0[4 * h + 3]);
+            e4[h] = make_float4(ds1[4 * h], ds1[4 * h + 1], ds1[4 * h + 2], ds1[4 * h + 3]);
+        }
+        *reinterpret_cast<float4 *>(sm.dzf + r * CH + c0) = make_float4(zf[0], zf[1], zf[2], zf[3]);
     }
     bool bc_done = false;
     if constexpr ((N * sizeof(T)) % 16 == 0) {
@@ -719,6 +736,11 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     th.Dk = th.valid ? p.D[(size_t)th.dir * p.Di + th.d] : 0.0f;
     th.cbase = (((size_t)b * p.G + c) * 2 + th.dir) * p.Di + th.d;
     __syncthreads();
+    // with several chunks this kernel is launched as a programmatic dependent of the
+    // adjoint fold (whose predecessors were ordinary launches, so the inputs were
+    // complete before the chain began): everything above reads only the inputs; the
+    // carries are read after the wait
+    if (p.G > 1) cudaGridDependencySynchronize();
 
     if (th.dir == 0) bwd_forward<N, 0>(p, sm, th);
     else bwd_forward<N, 1>(p, sm, th);
@@ -730,9 +752,9 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
             const int r = li / (CH / kG), c0 = (li % (CH / kG)) * kG, ch = d0 + c0;
             if (r < tc && ch < p.Di) {
                 const size_t i = ((size_t)b * p.L + bpos(p, t0 + r)) * p.Di + ch;
-                float y[kG];
-#pragma unroll
-                for (int k = 0; k < kG; ++k) y[k] = sm.yb[r * CH + c0 + k] + sm.yb[(TC + r) * CH + c0 + k];
+                const float4 y0 = *reinterpret_cast<const float4 *>(sm.yb + r * CH + c0);
+                const float4 y1 = *reinterpret_cast<const float4 *>(sm.yb + (TC + r) * CH + c0);
+                float y[kG] = {y0.x + y1.x, y0.y + y1.y, y0.z + y1.z, y0.w + y1.w};
                 if (p.stage == 1) {
                     *reinterpret_cast<float4 *>(p.acc_y + i) = make_float4(y[0], y[1], y[2], y[3]);
                 } else {
@@ -740,11 +762,8 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
                         const float4 a = *reinterpret_cast<const float4 *>(p.acc_y + i);
                         y[0] += a.x; y[1] += a.y; y[2] += a.z; y[3] += a.w;
                     }
-                    float e[kG], zz[kG];
-                    load4<T>(p.dout, i, vio, e);
-                    load4<T>(p.z, i, vio, zz);
-#pragma unroll
-                    for (int k = 0; k < kG; ++k) y[k] *= e[k] * silu_grad(zz[k]);
+                    const float4 f = *reinterpret_cast<const float4 *>(sm.dzf + r * CH + c0);
+                    y[0] *= f.x; y[1] *= f.y; y[2] *= f.z; y[3] *= f.w;
                     store4<T>(p.dz, i, vio, y);
                 }
             }
@@ -760,12 +779,12 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
         const int r = li / (CH / kG), c0 = (li % (CH / kG)) * kG, ch = d0 + c0;
         if (r < tc && ch < p.Di) {
             const size_t i = ((size_t)b * p.L + bpos(p, t0 + r)) * p.Di + ch;
-            float du[kG], dd[kG];
-#pragma unroll
-            for (int k = 0; k < kG; ++k) {
-                du[k] = sm.yb[r * CH + c0 + k] + sm.yb[(TC + r) * CH + c0 + k];
-                dd[k] = sm.dd[r * CH + c0 + k] + sm.dd[(TC + r) * CH + c0 + k];
-            }
+            const float4 a0 = *reinterpret_cast<const float4 *>(sm.yb + r * CH + c0);
+            const float4 a1 = *reinterpret_cast<const float4 *>(sm.yb + (TC + r) * CH + c0);
+            const float4 b0 = *reinterpret_cast<const float4 *>(sm.dd + r * CH + c0);
+            const float4 b1 = *reinterpret_cast<const float4 *>(sm.dd + (TC + r) * CH + c0);
+            float du[kG] = {a0.x + a1.x, a0.y + a1.y, a0.z + a1.z, a0.w + a1.w};
+            float dd[kG] = {b0.x + b1.x, b0.y + b1.y, b0.z + b1.z, b0.w + b1.w};
             if (p.stage == 1) {
                 *reinterpret_cast<float4 *>(p.acc_du + i) = make_float4(du[0], du[1], du[2], du[3]);
                 *reinterpret_cast<float4 *>(p.acc_dd + i) = make_float4(dd[0], dd[1], dd[2], dd[3]);
