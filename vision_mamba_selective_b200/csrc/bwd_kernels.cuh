@@ -15,14 +15,15 @@
 // the adjoint g entering each chunk from the later side comes from adj_carry plus
 // pair_combine folding against the direction.  bwd_main then runs one chunk of 16
 // or 32 channels, both directions: a forward sweep that keeps h every kBwdSeg tokens (in
-// registers) and forms y (for dz) and the dC terms, then segment by segment in
+// shared memory) and forms y (for dz) and the dC terms, then segment by segment in
 // reverse a re-run of h over the segment followed by the adjoint sweep.  A thread
 // holds NT (4, or 8 when built so) states of one (channel, direction), as pairs for
 // the f32x2 arithmetic, so the segment's h and decays fit in registers (the
 // checkpoints go to shared memory); Q = N / NT threads share a channel.  Each warp
 // serves one direction, whose code is compiled separately so that its token addresses
 // are constants.
-// Sums over channels (dB, dC) are reduced across the warp by shuffles, then across
+// Sums over channels (dB, dC) are reduced across the warp by shuffles, a segment's
+// tokens at a time (one reduce-scatter, so the shuffles are independent), then across
 // the CTA's warps and directions in shared memory, and written per CTA; sums over
 // tokens (dA, dD, dbias) are written per chunk.  Small reduction kernels finish both.
 // Every sum is taken in a fixed order (no floating-point atomics), so results repeat
