@@ -552,9 +552,11 @@ def main():
 
     projection = None
     if args.block:
-        # x_proj: x read once, B and C (bf16) and the step input (fp32) written per pathway
+        # x_proj: x read once; B and C (bf16), the step input (fp32) and u (bf16, for the
+        # scan) written per pathway
         M = w.batch * w.tokens
-        pb = M * w.channels * 2 + 2 * (2 * M * w.d_state * 2 + M * 4) + 2 * w.channels * (2 * w.d_state + 1) * 2
+        pb = (M * w.channels * 2 + 2 * (2 * M * w.d_state * 2 + M * 4 + M * w.channels * 2)
+              + 2 * w.channels * (2 * w.d_state + 1) * 2)
         pms = per_kernel["xproj"]
         projection = {"kernel": "xproj_kernel", "bound": "hbm", "ms_per_launch": pms, "algorithmic_bytes": pb,
                       "achieved_gbs": pb / (pms * 1e-3) / 1e9, "peak_gbs": pk["hbm_gbs"],

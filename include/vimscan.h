@@ -264,9 +264,12 @@ vim_status vim_scan_bidir_bwd_events(const void *u, const void *delta, const voi
  *   events  : NULL, or 5 CUDA events: start, after the projection, then those of
  *             vim_scan_bidir_events.
  *   workspace : vim_block_workspace_bytes(...) bytes, 256-byte aligned; it holds B, C
- *             (bf16) and s (fp32) of both pathways between the two kernels.
+ *             (bf16) and s (fp32) of both pathways between the two kernels, and with
+ *             the convolution front both pathways' u_k (bf16).
  * x_proj runs on the tensor cores with u_k rounded to bf16 and fp32 accumulation; B and
- * C are rounded to bf16, s stays fp32; Delta is never written to memory.  Only bf16 I/O
+ * C are rounded to bf16, s stays fp32; Delta is never written to memory.  With the
+ * convolution front the scan reads u_k as the projection kernel rounded and stored it
+ * (the front is formed once).  Only bf16 I/O
  * (VIM_F32 returns VIM_ERR_UNSUPPORTED), the first-order Bbar, and d_inner up to 2776
  * (one pathway's Wx, transposed, is held in one CTA's shared memory).
  */

@@ -15,10 +15,11 @@ namespace vimscan {
 namespace {
 
 struct BlockPlan {
-    size_t off_B, off_C, off_s, off_sum, total;
+    size_t off_B, off_C, off_s, off_u, off_sum, total;
 };
 
-BlockPlan block_plan(int batch, int L, int Di, int N) {
+// conv: the pathways' u (formed by the projection kernel) is kept for the scan
+BlockPlan block_plan(int batch, int L, int Di, int N, bool conv) {
     BlockPlan pl;
     const size_t M = (size_t)batch * L;
     size_t o = 0;
@@ -26,6 +27,7 @@ BlockPlan block_plan(int batch, int L, int Di, int N) {
     pl.off_B = take(2 * M * N * 2);
     pl.off_C = take(2 * M * N * 2);
     pl.off_s = take(2 * M * 4);
+    pl.off_u = take(conv ? 2 * M * Di * 2 : 0);
     pl.off_sum = take(summary_bytes(batch, L, Di, N));
     pl.total = o;
     return pl;
@@ -74,7 +76,7 @@ extern "C" {
 
 size_t vim_block_workspace_bytes(int batch, int L, int d_inner, int d_state) {
     if (batch <= 0 || L <= 0 || d_inner <= 0 || d_state <= 0) return 0;
-    return block_plan(batch, L, d_inner, d_state).total;
+    return block_plan(batch, L, d_inner, d_state, true).total;
 }
 
 vim_status vim_block_scan(const void *x, const float *conv_w, const float *conv_b, const void *Wx,
@@ -92,7 +94,8 @@ vim_status vim_block_scan(const void *x, const float *conv_w, const float *conv_
     if (!aligned16(x) || !aligned16(y) || (z && !aligned16(z)) || !al(Wx, 2) || !al(Wdt, 4) || !al(dt_bias, 4) ||
         !al(A, 4) || !al(D, 4) || !al(conv_w, 4) || !al(conv_b, 4))
         return VIM_ERR_INVALID_ARG;
-    const BlockPlan pl = block_plan(batch, L, d_inner, d_state);
+    const bool conv = conv_w != nullptr;
+    const BlockPlan pl = block_plan(batch, L, d_inner, d_state, conv);
     if (!workspace || workspace_bytes < pl.total || !al(workspace, kAlign)) return VIM_ERR_WORKSPACE;
     char *ws = static_cast<char *>(workspace);
     const int64_t M = (int64_t)batch * L;
@@ -101,14 +104,15 @@ vim_status vim_block_scan(const void *x, const float *conv_w, const float *conv_
     std::memset(&pa, 0, sizeof(pa));
     pa.x = x; pa.conv_w = conv_w; pa.conv_b = conv_b; pa.Wx = Wx;
     pa.Bo = ws + pl.off_B; pa.Co = ws + pl.off_C; pa.s = reinterpret_cast<float *>(ws + pl.off_s);
+    pa.uo = conv ? ws + pl.off_u : nullptr;
     pa.M = M; pa.L = L; pa.Di = d_inner;
 
     if (events && cudaEventRecord(events[0], stream) != cudaSuccess) return VIM_ERR_CUDA;
     switch (d_state) {
-        case 2: st = launch_proj<2>(pa, conv_w != nullptr, stream); break;
-        case 4: st = launch_proj<4>(pa, conv_w != nullptr, stream); break;
-        case 8: st = launch_proj<8>(pa, conv_w != nullptr, stream); break;
-        case 16: st = launch_proj<16>(pa, conv_w != nullptr, stream); break;
+        case 2: st = launch_proj<2>(pa, conv, stream); break;
+        case 4: st = launch_proj<4>(pa, conv, stream); break;
+        case 8: st = launch_proj<8>(pa, conv, stream); break;
+        case 16: st = launch_proj<16>(pa, conv, stream); break;
         default: return VIM_ERR_UNSUPPORTED;
     }
     if (st != VIM_OK) return st;
@@ -117,8 +121,11 @@ vim_status vim_block_scan(const void *x, const float *conv_w, const float *conv_
     const Plan sp = plan_for(batch, L, d_inner);
     PairArgs a;
     std::memset(&a, 0, sizeof(a));
-    a.u = x; a.z = z;
-    a.conv_w = conv_w; a.conv_b = conv_b;
+    // with the convolution front the scan reads each pathway's u as the projection
+    // stored it; without it both directions read x
+    a.u = conv ? static_cast<const void *>(ws + pl.off_u) : x;
+    a.u_dir_stride = conv ? M * d_inner : 0;
+    a.z = z;
     const __nv_bfloat16 *Bw = reinterpret_cast<const __nv_bfloat16 *>(ws + pl.off_B);
     const __nv_bfloat16 *Cw = reinterpret_cast<const __nv_bfloat16 *>(ws + pl.off_C);
     a.B[0] = Bw; a.B[1] = Bw + M * d_state;

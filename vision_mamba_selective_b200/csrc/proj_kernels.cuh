@@ -7,9 +7,10 @@
 //   P_k[m, :] = u_k[m, :] Wx[k],   u_k = silu(conv_k(x)) or x,
 //   B_k = P_k[:, 0:N],  C_k = P_k[:, N:2N],  s_k = P_k[:, 2N]
 // A CTA serves one pathway: it stages Wx[k] transposed once, then for each of its
-// 64-token tiles (rows of the flattened [batch*L] sequence) forms u_k one 64-channel
-// slice at a time in shared memory (bf16) and multiplies on the tensor cores with
-// mma.sync m16n8k16 (bf16 in, fp32 accumulate), one warp per 16 rows.  The
+// 128-token tiles (rows of the flattened [batch*L] sequence) forms u_k one 64-channel
+// slice at a time in shared memory (bf16), stores it for the scan when asked, and
+// multiplies on the tensor cores with mma.sync m16n8k16 (bf16 in, fp32 accumulate),
+// one warp per 16 rows.  The
 // product has only 2N + 1 <= 33 columns, so the kernel is bound by reading x, not by
 // the tensor pipe.
 #pragma once
@@ -24,6 +25,7 @@ struct ProjArgs {
     const void *Wx;                 // [2][Di][2N+1] bf16
     void *Bo, *Co;                  // [2][M][N] bf16
     float *s;                       // [2][M] fp32
+    void *uo;                       // [2][M][Di] bf16: each pathway's u as the scan reads it, or null
     int64_t M;
     int L, Di;
 };
@@ -190,6 +192,16 @@ __global__ void __launch_bounds__(kProjThreads) xproj_kernel(ProjArgs p) {
             }
         }
         __syncthreads();
+        if (p.uo) {
+            // the slice of u_k, 16 bytes at a time, for the scan (which then forms no front)
+            __nv_bfloat16 *uo = static_cast<__nv_bfloat16 *>(p.uo) + (size_t)dir * p.M * p.Di;
+            for (int li = tid; li < kProjRows * (kProjK / 8); li += kProjThreads) {
+                const int r = li / (kProjK / 8), c8 = (li % (kProjK / 8)) * 8;
+                const int m = m0 + r, dd = kc + c8;
+                if (m < M && dd < p.Di)
+                    *reinterpret_cast<uint4 *>(uo + (size_t)m * p.Di + dd) = *reinterpret_cast<const uint4 *>(&sU[r][c8]);
+            }
+        }
 #pragma unroll
         for (int ks = 0; ks < kProjK / 16; ++ks) {
             const int ra = warp * 16 + g, k0 = ks * 16 + tg * 2;

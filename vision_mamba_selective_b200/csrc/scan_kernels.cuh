@@ -211,6 +211,8 @@ __device__ __forceinline__ void load_row(const float *row, float2 (&v)[NP]) {
 // ----------------------------------------------------------------------------
 struct PairArgs {
     const void *u, *delta, *z;      // [batch, L, Di] by position
+    int64_t u_dir_stride;           // elements from the forward direction's u to the backward
+                                    // one's (0: both read the same u)
     const void *B[2], *C[2];        // per direction of the pair: [batch, L, N] by position
     const float *A;                 // [2][Di][N]: forward, backward
     const float *D;                 // [2][Di]
@@ -311,10 +313,10 @@ struct Stager {
 
     // u and delta of both tiles (with CONV: x and its halo rows instead of u)
     __device__ void issue(char *slot, int jf, int jb) const {
-        const T *gu = static_cast<const T *>(p.u);
         const T *gd = static_cast<const T *>(p.delta);
 #pragma unroll
         for (int dir = 0; dir < 2; ++dir) {
+            const T *gu = static_cast<const T *>(p.u) + (dir ? p.u_dir_stride : 0);
             const int j = dir ? jb : jf;
             const int rows = rows_of(j);
 #pragma unroll
