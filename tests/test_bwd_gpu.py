@@ -114,6 +114,35 @@ def test_bwd_small(vs, case):
     check_all(f"bwd_{case}", run(vs, x, gate), ref(x, gate), dtype)
 
 
+def offset_copy(t):
+    """A copy of t one element past the start of a device allocation, so that its address
+    is not a multiple of 8 bytes (bf16) or 16 bytes (fp32)."""
+    flat = torch.empty(t.numel() + 1, dtype=t.dtype, device="cuda")
+    v = flat[1:].view(t.shape)
+    v.copy_(t)
+    return v
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["fp32", "bf16"])
+def test_bwd_unaligned(vs, dtype):
+    """dout, z, B, C and the per-element outputs at addresses that rule out the kernels'
+    vector loads and stores (the entry point asks only for element alignment of these):
+    the element-wise paths give the same derivatives.  Three 32-token chunks, so the
+    summary kernels run too."""
+    batch, L, Di, N = 2, 70, 32, 16
+    x = inputs(batch, L, Di, N, dtype, seed=70)
+    c = lambda k: x[k].cuda()
+    u = c("u")
+    f32 = lambda *s: torch.zeros(s, dtype=torch.float32, device="cuda")
+    out = dict(du=offset_copy(torch.zeros_like(u)), ddelta=offset_copy(torch.zeros_like(u)),
+               dz=offset_copy(torch.zeros_like(u)), dB=f32(batch, L, N), dC=f32(batch, L, N), dA=f32(2, Di, N),
+               dD=f32(2, Di), ddelta_bias=f32(2, Di))
+    got = vs.vim_scan_bidir_bwd(u, c("delta"), offset_copy(c("z")), offset_copy(c("B")), offset_copy(c("C")),
+                                c("A"), c("D"), c("bias"), offset_copy(c("dout")), out=out)
+    torch.cuda.synchronize()
+    check_all(f"bwd_unaligned_{dtype}", got, ref(x), dtype)
+
+
 def test_bwd_deterministic(vs):
     x = inputs(2, 500, 64, 16, torch.float32, seed=8)
     a, b = run(vs, x), run(vs, x)

@@ -94,7 +94,9 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
         return VIM_ERR_CUDA;
     const dim3 gm(a.nblk, a.G, a.batch);
     if (a.G > 1) {
-        // staging overlaps the adjoint fold, which lets its dependents start early
+        // a programmatic dependent of the adjoint fold: its launch and the staging of
+        // the first CTAs overlap the fold's end; it waits for the fold before it reads
+        // the carries
         if (launch_dependent(bwd_main<T, N>, gm, dim3(BwdShape<N>::kThr), sm, stream, a) != cudaSuccess)
             return VIM_ERR_CUDA;
     } else {
