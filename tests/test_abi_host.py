@@ -172,6 +172,11 @@ def test_cross_bwd_and_block_reject(vs):
     assert blk(x=F + 8) == vs.VIM_ERR_INVALID_ARG
     assert blk(Di=3000) == vs.VIM_ERR_UNSUPPORTED             # Wx^T would not fit in shared memory
     assert blk(ws=None) == vs.VIM_ERR_WORKSPACE
+    # the workspace holds B, C (bf16), s (fp32) and, with the front, both pathways' u (bf16)
+    M, N, Di = 2 * 100, 16, 64
+    need = vs.vim_block_workspace_bytes(2, 100, Di, N)
+    assert need >= 2 * (2 * M * N * 2) + 2 * M * 4 + 2 * M * Di * 2
+    assert blk(wsb=need - 1) == vs.VIM_ERR_WORKSPACE          # with the front: one byte short
 
 
 def test_size_zero_is_a_noop(vs):
