@@ -249,6 +249,9 @@ def bwd_dout(w, seed):
     return torch.randn((w.batch, w.tokens, w.channels), generator=g).to(w.torch_dtype()).contiguous()
 
 
+CPU_SECONDS = 10.0   # host time the cpu_baseline leg spends on the oracle (about)
+
+
 def oracle_sample(w, target_s, conv=False, bwd=False, block=False):
     """A bounded sample of the workload for the oracle: its first batch items and
     first channels at the full sequence length, sized for about ``target_s`` seconds
@@ -564,11 +567,17 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        s, x, cores = oracle_sample(w, 5.0, conv=args.conv, bwd=args.bwd, block=args.block)
-        sec = run_oracle(s, x, cores, args.zoh)
-        cpu = {"value": s.tok_ch / sec, "unit": "tok*ch/s", "cores": cores, "kind": "oracle",
+        s, x, cores = oracle_sample(w, CPU_SECONDS, conv=args.conv, bwd=args.bwd, block=args.block)
+        # a sample that is the whole workload may finish in well under the target: run it
+        # again until the target is reached, and report the mean rate
+        sec, runs = 0.0, 0
+        while runs == 0 or sec < CPU_SECONDS:
+            sec += run_oracle(s, x, cores, args.zoh)
+            runs += 1
+        cpu = {"value": runs * s.tok_ch / sec, "unit": "tok*ch/s", "cores": cores, "kind": "oracle",
                "sample": f"{s.batch} of {w.batch} batch items x {s.channels} of {w.channels} channels "
-                         f"at the full {w.tokens} tokens ({s.tok_ch} token-channels), fp64, {sec:.2f} s"}
+                         f"at the full {w.tokens} tokens ({s.tok_ch} token-channels), {runs} run(s), "
+                         f"fp64, {sec:.2f} s"}
 
     if rank == 0:
         line = {
