@@ -59,9 +59,9 @@ class Oracle:
         lib.oracle_cross_order.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _I64]
         lib.oracle_conv_silu.argtypes = [_D, _D, _D, _D] + [ctypes.c_int] * 4
         lib.oracle_vim_bidir_conv.argtypes = [_D, _D, _D, _D, _D, _D, _D, ctypes.c_int64, _D, _D, _D, _D] + [ctypes.c_int] * 6
-        lib.oracle_s6_direction_bwd.argtypes = [_D] * 7 + [_I64] + [_D] * 8 + [ctypes.c_int] * 5
-        lib.oracle_vim_bidir_bwd.argtypes = [_D, _D, _D, _D, _D, ctypes.c_int64] + [_D] * 12 + [ctypes.c_int] * 5
-        lib.oracle_cross_scan4_bwd.argtypes = [_D] * 17 + [ctypes.c_int] * 6
+        lib.oracle_s6_direction_bwd.argtypes = [_D] * 7 + [_I64] + [_D] * 8 + [ctypes.c_int] * 6
+        lib.oracle_vim_bidir_bwd.argtypes = [_D, _D, _D, _D, _D, ctypes.c_int64] + [_D] * 12 + [ctypes.c_int] * 6
+        lib.oracle_cross_scan4_bwd.argtypes = [_D] * 17 + [ctypes.c_int] * 7
         lib.oracle_xproj.argtypes = [_D, _D, _D, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
@@ -125,8 +125,10 @@ class Oracle:
             raise ValueError("oracle_vim_bidir: bad sizes")
         return y
 
-    def vim_bidir_bwd(self, u, delta, z, B, C, A, D, bias, dout, *, bc_dir_stride=0, delta_is_raw=True):
-        """Derivatives of vim_bidir (first-order Bbar) for the loss sum(dout * y).
+    def vim_bidir_bwd(self, u, delta, z, B, C, A, D, bias, dout, *, bc_dir_stride=0, delta_is_raw=True,
+                      zoh=False):
+        """Derivatives of vim_bidir (first-order Bbar, or the exact hold with zoh) for
+        the loss sum(dout * y).
 
         Returns a dict of fp64 arrays: du, ddelta (w.r.t. the raw delta when
         delta_is_raw), dz (None without a gate), dB and dC shaped like B and C, dA
@@ -145,13 +147,14 @@ class Oracle:
                                            _p(A), _p(D), _p(bias), _p(dout), _p(out["du"]),
                                            _p(out["ddelta"]), _p(out["dz"]), _p(out["dB"]), _p(out["dC"]),
                                            _p(out["dA"]), _p(out["dD"]), _p(out["dbias"]),
-                                           batch, L, Di, N, int(bool(delta_is_raw)))
+                                           batch, L, Di, N, int(bool(delta_is_raw)), int(bool(zoh)))
         if rc:
             raise ValueError("oracle_vim_bidir_bwd: bad sizes")
         return out
 
-    def cross_scan4_bwd(self, u, delta, z, B, C, A, D, bias, dout, *, delta_is_raw=True):
-        """Derivatives of cross_scan4 (first-order Bbar) for the loss sum(dout * y).
+    def cross_scan4_bwd(self, u, delta, z, B, C, A, D, bias, dout, *, delta_is_raw=True, zoh=False):
+        """Derivatives of cross_scan4 (first-order Bbar, or the exact hold with zoh) for
+        the loss sum(dout * y).
 
         u, delta, z, dout: [batch, H, W, Ci]; B, C: [4, batch, H*W, N]; A [4, Ci, N];
         D, bias [4, Ci].  Returns a dict of fp64 arrays shaped like the inputs: du,
@@ -168,7 +171,7 @@ class Oracle:
         rc = self.lib.oracle_cross_scan4_bwd(_p(u), _p(delta), _p(z), _p(B), _p(C), _p(A), _p(D), _p(bias), _p(dout),
                                              _p(out["du"]), _p(out["ddelta"]), _p(out["dz"]), _p(out["dB"]),
                                              _p(out["dC"]), _p(out["dA"]), _p(out["dD"]), _p(out["dbias"]),
-                                             batch, H, W, Ci, N, int(bool(delta_is_raw)))
+                                             batch, H, W, Ci, N, int(bool(delta_is_raw)), int(bool(zoh)))
         if rc:
             raise ValueError("oracle_cross_scan4_bwd: bad sizes")
         return out

@@ -119,6 +119,38 @@ static double bbar(double dt, double An, double Bn, int zoh)
     return expm1(dt * An) / An * Bn;
 }
 
+/*
+ * Derivatives of one state's hold gain e(Delta, A_n) = Bbar_n / B_n (e = Delta for the
+ * first-order form; e = (exp(Delta A_n) - 1) / A_n for the exact hold, Delta at A_n = 0):
+ *   de/dDelta = 1, or exp(Delta A_n);
+ *   de/dA_n   = 0, or (z e^z - (e^z - 1)) / A_n^2 = Delta^2 S(z) with z = Delta A_n and
+ *               S(z) = sum_{k >= 1} k z^(k-1) / (k+1)!  (= 1/2 + z/3 + z^2/8 + ...),
+ * which follows from differentiating e = Delta sum_{k >= 0} z^k / (k+1)! term by term.
+ * S is summed as that series (18 terms, Horner) for |z| < 1/2, where the closed form
+ * loses digits to cancellation, and in closed form elsewhere; at A_n = 0 it is 1/2.
+ */
+static double hold_gain_ddt(double dt, double An, int zoh)
+{
+    return zoh ? exp(dt * An) : 1.0;
+}
+
+static double hold_gain_dA(double dt, double An, int zoh)
+{
+    if (!zoh) return 0.0;
+    double zz = dt * An;
+    if (fabs(zz) < 0.5) {
+        double c[19], f = 1.0;                 /* c[k] = k / (k+1)! */
+        for (int k = 1; k <= 18; ++k) {
+            f *= (double)(k + 1);
+            c[k] = (double)k / f;
+        }
+        double sum = c[18];
+        for (int k = 17; k >= 1; --k) sum = sum * zz + c[k];
+        return dt * dt * sum;
+    }
+    return (zz * exp(zz) - expm1(zz)) / (An * An);
+}
+
 int oracle_s6_direction(const double *u, const double *delta, const double *B, const double *C,
                         const double *A, const double *D, const double *bias,
                         const int64_t *order, double *y,
@@ -330,7 +362,8 @@ static double silu_grad(double z)
 }
 
 /*
- * Derivative of one S6 direction (oracle_s6_direction, first-order Bbar).
+ * Derivative of one S6 direction (oracle_s6_direction; the first-order Bbar, or the
+ * exact hold when zoh != 0).
  *   dy       : [batch, L, Di], the loss's derivative with respect to y
  *   du, ddelta : [batch, L, Di]   (ddelta is w.r.t. the raw delta when delta_is_raw,
  *                                  else w.r.t. Delta itself)
@@ -342,14 +375,17 @@ static double silu_grad(double z)
  *   dl/dAbar_n = g_n h_{t-1,n}  ->  dl/dDelta += that * Abar_n * A_n,
  *                                   dl/dA_n   += that * Abar_n * Delta_t,
  *   dl/dDelta += sum_n g_n B_tn u_t,  dl/dB_tn += g_n Delta_t u_t,
- * and g <- g * Abar is dl/dh_{t-1}.
+ * and g <- g * Abar is dl/dh_{t-1}.  With the exact hold, Bbar_n = e_n B_n with the
+ * gain e_n = (exp(Delta A_n) - 1) / A_n in place of Delta: Delta_t becomes e_n in
+ * dl/du and dl/dB, the Delta term gains the factor de_n/dDelta = exp(Delta A_n), and
+ * dl/dA_n gains g_n B_tn u_t de_n/dA_n (hold_gain_dA).
  */
 int oracle_s6_direction_bwd(const double *u, const double *delta, const double *B, const double *C,
                             const double *A, const double *D, const double *bias,
                             const int64_t *order, const double *dy,
                             double *du, double *ddelta, double *dB, double *dC,
                             double *dA, double *dD, double *dbias,
-                            int batch, int L, int Di, int N, int delta_is_raw)
+                            int batch, int L, int Di, int N, int delta_is_raw, int zoh)
 {
     if (batch < 0 || L < 0 || Di < 0 || N < 1 || N > ORACLE_MAX_STATE) return -1;
     int rc = 0;
@@ -380,7 +416,7 @@ int oracle_s6_direction_bwd(const double *u, const double *delta, const double *
                     double dt = delta_is_raw ? softplus(delta[ix] + bias[d]) : delta[ix];
                     dts[t] = dt;
                     for (int n = 0; n < N; ++n) {
-                        h[n] = exp(dt * Ad[n]) * h[n] + dt * Bt[n] * u[ix];
+                        h[n] = exp(dt * Ad[n]) * h[n] + bbar(dt, Ad[n], Bt[n], zoh) * u[ix];
                         hs[t * N + n] = h[n];
                     }
                 }
@@ -399,10 +435,12 @@ int oracle_s6_direction_bwd(const double *u, const double *delta, const double *
                         double Abar = exp(dt * Ad[n]);
                         double hprev = t > 0 ? hs[(t - 1) * N + n] : 0.0;
                         double dAbar = g[n] * hprev;
-                        dDelta += dAbar * Abar * Ad[n] + g[n] * Bt[n] * x;
+                        double gain = bbar(dt, Ad[n], 1.0, zoh);  /* Bbar_n / B_n       */
+                        dDelta += dAbar * Abar * Ad[n] + g[n] * Bt[n] * x * hold_gain_ddt(dt, Ad[n], zoh);
                         dA_loc[d * N + n] += dAbar * Abar * dt;
-                        dBt[n] += g[n] * dt * x;
-                        dx += g[n] * dt * Bt[n];
+                        if (zoh) dA_loc[d * N + n] += g[n] * Bt[n] * x * hold_gain_dA(dt, Ad[n], zoh);
+                        dBt[n] += g[n] * gain * x;
+                        dx += g[n] * gain * Bt[n];
                         g[n] *= Abar;                             /* dl/dh_{t-1} part   */
                     }
                     du[ix] += dx;
@@ -432,7 +470,8 @@ int oracle_s6_direction_bwd(const double *u, const double *delta, const double *
 }
 
 /*
- * Derivative of oracle_vim_bidir (first-order Bbar) for ell = sum dout * y.
+ * Derivative of oracle_vim_bidir (first-order Bbar, or the exact hold when zoh != 0)
+ * for ell = sum dout * y.
  *   dout : [batch, L, Di].  Outputs (overwritten):
  *   du, ddelta, dz : [batch, L, Di]  (dz untouched when z is NULL; ddelta w.r.t. the
  *                    raw delta when delta_is_raw)
@@ -447,7 +486,7 @@ int oracle_vim_bidir_bwd(const double *u, const double *delta, const double *z,
                          const double *A, const double *D, const double *bias, const double *dout,
                          double *du, double *ddelta, double *dz, double *dB, double *dC,
                          double *dA, double *dD, double *dbias,
-                         int batch, int L, int Di, int N, int delta_is_raw)
+                         int batch, int L, int Di, int N, int delta_is_raw, int zoh)
 {
     if (batch < 0 || L < 0 || Di < 0 || N < 1 || bc_dir_stride < 0) return -1;
     int64_t n_act = (int64_t)batch * L * Di, n_bc = (int64_t)batch * L * N;
@@ -465,7 +504,7 @@ int oracle_vim_bidir_bwd(const double *u, const double *delta, const double *z,
         double *ys = (double *)malloc((size_t)(n_act > 0 ? n_act : 1) * sizeof(double));
         if (!ys) { free(dy); free(order); return -1; }
         rc |= oracle_vim_bidir(u, delta, NULL, B, C, bc_dir_stride, A, D, bias, ys,
-                               batch, L, Di, N, delta_is_raw, 0);
+                               batch, L, Di, N, delta_is_raw, zoh);
         for (int64_t i = 0; i < n_act; ++i) {
             dz[i] = dout[i] * ys[i] * silu_grad(z[i]);
             dy[i] = dout[i] * silu(z[i]);
@@ -476,13 +515,13 @@ int oracle_vim_bidir_bwd(const double *u, const double *delta, const double *z,
     }
     for (int64_t t = 0; t < L; ++t) order[t] = t;
     rc |= oracle_s6_direction_bwd(u, delta, B, C, A, D, bias, order, dy, du, ddelta, dB, dC,
-                                  dA, dD, dbias, batch, L, Di, N, delta_is_raw);
+                                  dA, dD, dbias, batch, L, Di, N, delta_is_raw, zoh);
     for (int64_t t = 0; t < L; ++t) order[t] = L - 1 - t;
     rc |= oracle_s6_direction_bwd(u, delta, B + bc_dir_stride, C + bc_dir_stride,
                                   A + (int64_t)Di * N, D + Di, bias + Di, order, dy, du, ddelta,
                                   dB + bc_dir_stride, dC + bc_dir_stride,
                                   dA + (int64_t)Di * N, dD + Di, dbias + Di,
-                                  batch, L, Di, N, delta_is_raw);
+                                  batch, L, Di, N, delta_is_raw, zoh);
     free(dy); free(order);
     return rc ? -1 : 0;
 }
@@ -510,7 +549,8 @@ int oracle_xproj(const double *u, const double *Wx, double *P, int64_t M, int Di
 }
 
 /*
- * Derivative of oracle_cross_scan4 (first-order Bbar) for ell = sum dout * y, with
+ * Derivative of oracle_cross_scan4 (first-order Bbar, or the exact hold when zoh != 0)
+ * for ell = sum dout * y, with
  * y = (sum_k y_k) * silu(z): dl/dz = dout (sum_k y_k) silu'(z), and each of the four
  * CS-Traverse directions sees dl/dy_k = dout silu(z) at the grid positions it visits.
  *   dout : [batch, H*W, Ci].  Outputs (overwritten): du, ddelta, dz [batch, H*W, Ci]
@@ -522,7 +562,7 @@ int oracle_cross_scan4_bwd(const double *u, const double *delta, const double *z
                            const double *A, const double *D, const double *bias, const double *dout,
                            double *du, double *ddelta, double *dz, double *dB, double *dC,
                            double *dA, double *dD, double *dbias,
-                           int batch, int H, int W, int Ci, int N, int delta_is_raw)
+                           int batch, int H, int W, int Ci, int N, int delta_is_raw, int zoh)
 {
     if (H < 0 || W < 0 || batch < 0 || Ci < 0 || N < 1) return -1;
     int64_t L = (int64_t)H * W;
@@ -538,7 +578,7 @@ int oracle_cross_scan4_bwd(const double *u, const double *delta, const double *z
     if (z) {
         double *ys = (double *)malloc((size_t)(n_act > 0 ? n_act : 1) * sizeof(double));
         if (!ys) { free(dy); free(order); return -1; }
-        rc |= oracle_cross_scan4(u, delta, NULL, B, C, A, D, bias, ys, batch, H, W, Ci, N, delta_is_raw, 0);
+        rc |= oracle_cross_scan4(u, delta, NULL, B, C, A, D, bias, ys, batch, H, W, Ci, N, delta_is_raw, zoh);
         for (int64_t i = 0; i < n_act; ++i) {
             dz[i] = dout[i] * ys[i] * silu_grad(z[i]);
             dy[i] = dout[i] * silu(z[i]);
@@ -552,7 +592,7 @@ int oracle_cross_scan4_bwd(const double *u, const double *delta, const double *z
         rc |= oracle_s6_direction_bwd(u, delta, B + k * bc, C + k * bc, A + (int64_t)k * Ci * N,
                                       D + (int64_t)k * Ci, bias + (int64_t)k * Ci, order, dy, du, ddelta,
                                       dB + k * bc, dC + k * bc, dA + (int64_t)k * Ci * N, dD + (int64_t)k * Ci,
-                                      dbias + (int64_t)k * Ci, batch, (int)L, Ci, N, delta_is_raw);
+                                      dbias + (int64_t)k * Ci, batch, (int)L, Ci, N, delta_is_raw, zoh);
     }
     free(dy); free(order);
     return rc ? -1 : 0;

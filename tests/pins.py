@@ -500,11 +500,27 @@ def _bwd_case(rng, batch=1, L=5, Di=2, N=3, separate_bc=True):
     return c
 
 
-def _loss(orc, c, **over):
+def _loss(orc, c, zoh=False, **over):
     c = {**c, **over}
     y = orc.vim_bidir(c["u"], c["delta"], c["z"], c["B"], c["C"], c["A"], c["D"], c["bias"],
-                      bc_dir_stride=c["stride"], delta_is_raw=True)
+                      bc_dir_stride=c["stride"], delta_is_raw=True, zoh=zoh)
     return float(np.sum(c["dout"] * y))
+
+
+def _bwd_fd(orc, c, zoh):
+    g = orc.vim_bidir_bwd(c["u"], c["delta"], c["z"], c["B"], c["C"], c["A"], c["D"], c["bias"], c["dout"],
+                          bc_dir_stride=c["stride"], zoh=zoh)
+    for name, key in (("u", "du"), ("delta", "ddelta"), ("z", "dz"), ("B", "dB"), ("C", "dC"),
+                      ("A", "dA"), ("D", "dD"), ("bias", "dbias")):
+        arr, eps = c[name], 1e-6
+        fd = np.zeros_like(arr)
+        for i in np.ndindex(arr.shape):
+            up, dn = arr.copy(), arr.copy()
+            up[i] += eps
+            dn[i] -= eps
+            fd[i] = (_loss(orc, c, zoh, **{name: up}) - _loss(orc, c, zoh, **{name: dn})) / (2 * eps)
+        err = np.max(np.abs(fd - g[key])) / np.max(np.abs(fd))
+        assert err < 1e-7, (name, zoh, err)
 
 
 def pin_bwd_finite_differences(orc):
@@ -514,20 +530,19 @@ def pin_bwd_finite_differences(orc):
     via Zero-Order Hold (ZOH)", "The Selective State Space (S6) Mechanism", "2. The
     Bidirectional Mamba Block").  Step 1e-6 in fp64: truncation and rounding stay
     near 1e-9 of the gradient's size."""
-    c = _bwd_case(_rng(101))
-    g = orc.vim_bidir_bwd(c["u"], c["delta"], c["z"], c["B"], c["C"], c["A"], c["D"], c["bias"], c["dout"],
-                          bc_dir_stride=c["stride"])
-    for name, key in (("u", "du"), ("delta", "ddelta"), ("z", "dz"), ("B", "dB"), ("C", "dC"),
-                      ("A", "dA"), ("D", "dD"), ("bias", "dbias")):
-        arr, eps = c[name], 1e-6
-        fd = np.zeros_like(arr)
-        for i in np.ndindex(arr.shape):
-            up, dn = arr.copy(), arr.copy()
-            up[i] += eps
-            dn[i] -= eps
-            fd[i] = (_loss(orc, c, **{name: up}) - _loss(orc, c, **{name: dn})) / (2 * eps)
-        err = np.max(np.abs(fd - g[key])) / np.max(np.abs(fd))
-        assert err < 1e-7, (name, err)
+    _bwd_fd(orc, _bwd_case(_rng(101)), zoh=False)
+
+
+def pin_zoh_bwd_finite_differences(orc):
+    """The same check for the exact zero-order hold (section "Discretization via
+    Zero-Order Hold (ZOH)": Bbar_n = (exp(Delta A_n) - 1) / A_n B_n), with A spanning
+    small |Delta A_n| (the oracle's series for dBbar/dA), large ones (its closed form)
+    and one A_n = 0 (the limit Delta B_n, whose A-derivative is Delta^2 B_n / 2)."""
+    c = _bwd_case(_rng(131))
+    A = -np.exp(_rng(132).uniform(np.log(0.005), np.log(4.0), size=c["A"].shape))
+    A[0, 1, 2] = 0.0
+    c["A"] = A
+    _bwd_fd(orc, c, zoh=True)
 
 
 def pin_bwd_homogeneity(orc):
@@ -603,12 +618,8 @@ def pin_block_scan_composition(orc):
     np.testing.assert_allclose(y0, ref0, rtol=1e-11, atol=1e-11)
 
 
-def pin_cross_bwd_finite_differences(orc):
-    """Every derivative of the four-direction scan against central finite differences
-    of the forward oracle's loss sum(dout * y) on a 2 x 3 grid (H != W, so a transposed
-    traversal cannot pass), with per-direction B, C, A, D and bias (sections "1.
-    Cross-Scan Traversal" to "3. Cross-Merge Reversal")."""
-    rng = _rng(121)
+def _cross_bwd_fd(orc, seed, zoh):
+    rng = _rng(seed)
     b, H, W, c, N = 1, 2, 3, 2, 2
     x = dict(u=rng.normal(size=(b, H, W, c)), delta=rng.normal(size=(b, H, W, c)) * 0.8,
              z=rng.normal(size=(b, H, W, c)), B=rng.normal(size=(4, b, H * W, N)),
@@ -616,8 +627,9 @@ def pin_cross_bwd_finite_differences(orc):
              D=rng.normal(size=(4, c)), bias=rng.normal(size=(4, c)))
     dout = rng.normal(size=(b, H, W, c))
     loss = lambda **o: float(np.sum(dout * orc.cross_scan4(*[{**x, **o}[k] for k in
-                                                               ("u", "delta", "z", "B", "C", "A", "D", "bias")])))
-    g = orc.cross_scan4_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["bias"], dout)
+                                                               ("u", "delta", "z", "B", "C", "A", "D", "bias")],
+                                                             zoh=zoh)))
+    g = orc.cross_scan4_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["bias"], dout, zoh=zoh)
     for name, key in (("u", "du"), ("delta", "ddelta"), ("z", "dz"), ("B", "dB"), ("C", "dC"), ("A", "dA"),
                       ("D", "dD"), ("bias", "dbias")):
         arr, eps = x[name], 1e-6
@@ -628,7 +640,16 @@ def pin_cross_bwd_finite_differences(orc):
             dn[i] -= eps
             fd[i] = (loss(**{name: up}) - loss(**{name: dn})) / (2 * eps)
         err = np.max(np.abs(fd - g[key])) / np.max(np.abs(fd))
-        assert err < 1e-7, (name, err)
+        assert err < 1e-7, (name, zoh, err)
+
+
+def pin_cross_bwd_finite_differences(orc):
+    """Every derivative of the four-direction scan against central finite differences
+    of the forward oracle's loss sum(dout * y) on a 2 x 3 grid (H != W, so a transposed
+    traversal cannot pass), with per-direction B, C, A, D and bias (sections "1.
+    Cross-Scan Traversal" to "3. Cross-Merge Reversal"); first-order and exact hold."""
+    _cross_bwd_fd(orc, 121, zoh=False)
+    _cross_bwd_fd(orc, 122, zoh=True)
 
 
 ALL_PINS = [
@@ -650,6 +671,7 @@ ALL_PINS = [
     pin_zoh_fixed_point_and_limits,
     pin_zoh_reaches_every_entry,
     pin_bwd_finite_differences,
+    pin_zoh_bwd_finite_differences,
     pin_bwd_homogeneity,
     pin_xproj_is_matmul,
     pin_cross_bwd_finite_differences,

@@ -51,7 +51,7 @@ MUTANTS = {
     "bwd_adjoint_not_decayed": ("g[n] *= Abar;", "g[n] *= 1.0;"),
     "bwd_hprev_is_h": ("double hprev = t > 0 ? hs[(t - 1) * N + n] : 0.0;", "double hprev = hs[t * N + n];"),
     "bwd_dA_without_delta": ("dA_loc[d * N + n] += dAbar * Abar * dt;", "dA_loc[d * N + n] += dAbar * Abar;"),
-    "bwd_dB_without_u": ("dBt[n] += g[n] * dt * x;", "dBt[n] += g[n] * dt;"),
+    "bwd_dB_without_u": ("dBt[n] += g[n] * gain * x;", "dBt[n] += g[n] * gain;"),
     "bwd_softplus_grad_sign": ("return x > 20.0 ? 1.0 : 1.0 / (1.0 + exp(-x));",
                                "return x > 20.0 ? 1.0 : 1.0 / (1.0 + exp(x));"),
     "bwd_gate_grad_is_sigmoid": ("return s * (1.0 + z * (1.0 - s));", "return s;"),
@@ -64,6 +64,12 @@ MUTANTS = {
     "cross_bwd_same_order": ("rc |= oracle_cross_order(k, H, W, order);\n        rc |= oracle_s6_direction_bwd",
                              "rc |= oracle_cross_order(0, H, W, order);\n        rc |= oracle_s6_direction_bwd"),
     "zoh_sign": ("return expm1(dt * An) / An * Bn;", "return expm1(-dt * An) / An * Bn;"),
+    # the exact hold's derivative
+    "zoh_bwd_ddelta_first_order": ("g[n] * Bt[n] * x * hold_gain_ddt(dt, Ad[n], zoh)", "g[n] * Bt[n] * x * 1.0"),
+    "zoh_bwd_dA_hold_term_dropped": (
+        "if (zoh) dA_loc[d * N + n] += g[n] * Bt[n] * x * hold_gain_dA(dt, Ad[n], zoh);", ""),
+    "zoh_bwd_series_coefficient": ("c[k] = (double)k / f;", "c[k] = 1.0 / f;"),
+    "zoh_bwd_closed_form_sign": ("(zz * exp(zz) - expm1(zz))", "(zz * exp(zz) + expm1(zz))"),
 }
 
 
