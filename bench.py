@@ -227,7 +227,8 @@ def run_oracle(w, x, threads, zoh=False):
         oracle.vim_block_scan(x["u"], x["Wx"], x["Wdt"], x["A"], x["D"], x["dt_bias"], x["z"],
                               conv_w=x["conv_w"], conv_b=x["conv_b"])
     elif "dout" in x and w.kind == "vim":
-        oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], x["dout"])
+        oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], x["dout"],
+                             zoh=zoh)
     elif "dout" in x:
         oracle.cross_scan4_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], x["dout"])
     elif "conv_w" in x:
@@ -343,8 +344,8 @@ def main():
         raise SystemExit("--conv and --block apply to the Vim workloads only")
     if args.block and (args.conv or args.zoh or args.bwd or w.dtype != "bf16"):
         raise SystemExit("--block runs alone, on a bf16 workload")
-    if args.bwd and (args.conv or args.zoh):
-        raise SystemExit("--bwd covers the plain scan (no --conv, no --zoh)")
+    if args.bwd and (args.conv or (args.zoh and w.kind != "vim")):
+        raise SystemExit("--bwd covers the plain scan (no --conv), with --zoh on the Vim workloads")
     if args.impl == "reference":
         reference_arm(args, w)
         return
@@ -412,7 +413,8 @@ def main():
             return
         if args.bwd and w.kind == "vim":
             vs.vim_scan_bidir_bwd(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"],
-                                  params["delta_bias"], s["dout"], workspace=ws, out=s["out"], events=events)
+                                  params["delta_bias"], s["dout"], workspace=ws, out=s["out"], events=events,
+                                  zoh=args.zoh)
             return
         if args.bwd:
             vs.vmamba_cross_scan4_bwd(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"],

@@ -307,6 +307,24 @@ vim_status vim_scan_bidir_ex(const void *u, const float *conv_w, const float *co
                              int d_state, vim_dtype dt, unsigned flags, void *workspace,
                              size_t workspace_bytes, cudaStream_t stream, cudaEvent_t *events);
 
+/*
+ * vim_scan_bidir_bwd_events with options in `flags` (unknown bits return
+ * VIM_ERR_INVALID_ARG).  With VIM_FLAG_ZOH_EXACT it is the derivative of the scan with
+ * the exact hold, Bbar_n = e_n B_n, e_n = (exp(Delta A_n) - 1) / A_n: e_n takes Delta's
+ * place in du and dB; the Delta term has de_n/dDelta = exp(Delta A_n); dA_n gains
+ * g B_n u de_n/dA_n with de_n/dA_n = (Delta exp(Delta A_n) - e_n) / A_n (its series
+ * Delta^2 (1/2 + Delta A_n / 3 + ...) for small Delta A_n).  Other arguments, the
+ * workspace and the events as in vim_scan_bidir_bwd_events.
+ */
+vim_status vim_scan_bidir_bwd_ex(const void *u, const void *delta, const void *z,
+                                 const void *B, const void *C, int64_t bc_dir_stride,
+                                 const float *A, const float *D, const float *delta_bias,
+                                 const void *dout, void *du, void *ddelta, void *dz,
+                                 float *dB, float *dC, float *dA, float *dD, float *ddelta_bias,
+                                 int batch, int L, int d_inner, int d_state, vim_dtype dt,
+                                 unsigned flags, void *workspace, size_t workspace_bytes,
+                                 cudaStream_t stream, cudaEvent_t *events);
+
 /* vmamba_cross_scan4 with the options in `flags` and the events of
  * vmamba_cross_scan4_events when `events` is non-NULL. */
 vim_status vmamba_cross_scan4_ex(const void *u, const void *delta, const void *z,

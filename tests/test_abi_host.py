@@ -37,6 +37,7 @@ def test_header_declares_the_boundary():
                           "vim_scan_bidir_events", "vmamba_cross_scan4_events", "vim_scan_bidir_noalloc", "vim_scan_bidir_conv", "vim_scan_bidir_conv_events",
                           "vim_scan_bidir_ex", "vmamba_cross_scan4_ex",
                           "vim_scan_bidir_bwd", "vim_scan_bwd_workspace_bytes", "vim_scan_bidir_bwd_events",
+                          "vim_scan_bidir_bwd_ex",
                           "vim_block_scan", "vim_block_workspace_bytes",
                           "vmamba_cross_scan4_bwd", "vmamba_cross_scan4_bwd_workspace_bytes",
                           "vim_scan_workspace_bytes", "vim_status_string"}, names
@@ -119,6 +120,26 @@ def bwd(vs, **kw):
                                      a["bias"], a["dout"], a["du"], a["ddelta"], a["dz"], a["dB"], a["dC"],
                                      a["dA"], a["dD"], a["dbias"], a["batch"], a["L"], a["Di"], a["N"],
                                      a["dt"], a["ws"], a["ws_bytes"], None)
+
+
+def bwd_ex(vs, flags, **kw):
+    """vim_scan_bidir_bwd_ex on fake device addresses (each case fails a host check)."""
+    a = dict(u=FAKE, delta=FAKE, z=FAKE, B=FAKE, C=FAKE, stride=0, A=FAKE, D=FAKE, bias=FAKE, dout=FAKE,
+             du=FAKE, ddelta=FAKE, dz=FAKE, dB=FAKE, dC=FAKE, dA=FAKE, dD=FAKE, dbias=FAKE,
+             batch=2, L=100, Di=64, N=16, dt=vs.VIM_BF16, ws=FAKE, ws_bytes=1 << 40)
+    a.update(kw)
+    return vs.lib.vim_scan_bidir_bwd_ex(a["u"], a["delta"], a["z"], a["B"], a["C"], a["stride"], a["A"], a["D"],
+                                        a["bias"], a["dout"], a["du"], a["ddelta"], a["dz"], a["dB"], a["dC"],
+                                        a["dA"], a["dD"], a["dbias"], a["batch"], a["L"], a["Di"], a["N"],
+                                        a["dt"], flags, a["ws"], a["ws_bytes"], None, None)
+
+
+def test_bwd_ex_rejects(vs):
+    assert bwd_ex(vs, 2) == vs.VIM_ERR_INVALID_ARG                  # unknown flag bit
+    assert bwd_ex(vs, vs.VIM_FLAG_ZOH_EXACT | 4) == vs.VIM_ERR_INVALID_ARG
+    assert bwd_ex(vs, vs.VIM_FLAG_ZOH_EXACT, N=3) == vs.VIM_ERR_UNSUPPORTED
+    assert bwd_ex(vs, vs.VIM_FLAG_ZOH_EXACT, dz=None) == vs.VIM_ERR_INVALID_ARG
+    assert bwd_ex(vs, vs.VIM_FLAG_ZOH_EXACT, ws=None) == vs.VIM_ERR_WORKSPACE
 
 
 def test_bwd_rejects(vs):

@@ -167,6 +167,80 @@ def test_bwd_full_size(vs):
 
 
 # ---------------------------------------------------------------------------
+# the exact zero-order hold (vim_scan_bidir_bwd_ex with VIM_FLAG_ZOH_EXACT)
+# ---------------------------------------------------------------------------
+ZOH_CASES = [
+    # batch, L, Di, N, dtype, separate_bc, generic_A
+    (1, 5, 16, 16, torch.float32, False, False),
+    (2, 70, 32, 16, torch.float32, True, True),          # 3 chunks, general A
+    (1, 33, 16, 8, torch.float32, False, False),          # 2 chunks, the last 1 token
+    (2, 100, 24, 4, torch.float32, False, True),
+    (1, 300, 64, 16, torch.bfloat16, False, False),
+    (1, 97, 40, 2, torch.bfloat16, True, True),
+]
+
+
+def run_zoh(vs, x):
+    c = lambda k: x[k].cuda()
+    out = vs.vim_scan_bidir_bwd(c("u"), c("delta"), c("z"), c("B"), c("C"), c("A"), c("D"), c("bias"), c("dout"),
+                                bc_dir_stride=x["stride"], zoh=True)
+    torch.cuda.synchronize()
+    return out
+
+
+def ref_zoh(x):
+    return oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["bias"], x["dout"],
+                                bc_dir_stride=x["stride"], zoh=True)
+
+
+@pytest.mark.parametrize("case", ZOH_CASES, ids=lambda c: f"b{c[0]}_L{c[1]}_D{c[2]}_N{c[3]}_{str(c[4])[6:]}"
+                         f"{'_sepBC' if c[5] else ''}{'_genA' if c[6] else ''}")
+def test_bwd_zoh(vs, case):
+    """The exact hold's derivative against the oracle's (pinned by finite differences);
+    Delta A_n spans both sides of the kernels' series/closed-form switch at 1/2."""
+    batch, L, Di, N, dtype, sep, gen = case
+    x = inputs(batch, L, Di, N, dtype, seed=L * 7 + Di, separate_bc=sep, generic_A=gen)
+    check_all(f"bwd_zoh_{case}", run_zoh(vs, x), ref_zoh(x), dtype)
+
+
+def test_bwd_zoh_a_zero(vs):
+    """A_n = 0 for some states: the hold's gain is its limit Delta and its A-derivative
+    Delta^2 / 2."""
+    x = inputs(1, 50, 16, 16, torch.float32, seed=50, generic_A=True)
+    x["A"] = x["A"].clone()
+    x["A"][0, 3, :] = 0.0
+    x["A"][1, 5, 7] = 0.0
+    check_all("bwd_zoh_a_zero", run_zoh(vs, x), ref_zoh(x), torch.float32)
+
+
+def test_bwd_zoh_first_order_unchanged(vs):
+    """Without the flag the _ex entry point is the first-order derivative, bit for bit."""
+    x = inputs(2, 70, 32, 16, torch.float32, seed=71)
+    c = lambda k: x[k].cuda()
+    a = vs.vim_scan_bidir_bwd(c("u"), c("delta"), c("z"), c("B"), c("C"), c("A"), c("D"), c("bias"), c("dout"))
+    b = run(vs, x)
+    for k, _ in KEYS:
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_bwd_zoh_full_size(vs):
+    """The 1024 px Vim-Ti workload with the exact hold, against the oracle on every
+    output."""
+    w = wl.BY_NAME["vim_tiny_1024px_bf16"]
+    x = wl.make_inputs(w)
+    g = torch.Generator().manual_seed(778)
+    dout = torch.randn(x["u"].shape, generator=g).to(x["u"].dtype)
+    oracle.set_threads(max(1, len(os.sched_getaffinity(0))))
+    d = {k: v.cuda() for k, v in x.items()}
+    got = vs.vim_scan_bidir_bwd(d["u"], d["delta"], d["z"], d["B"], d["C"], d["A"], d["D"], d["delta_bias"],
+                                dout.cuda(), zoh=True)
+    torch.cuda.synchronize()
+    want = oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], dout,
+                                zoh=True)
+    check_all("bwd_zoh_full", got, want, torch.bfloat16, sum_tol=1e-3)
+
+
+# ---------------------------------------------------------------------------
 # the four-direction cross-scan
 # ---------------------------------------------------------------------------
 def cross_inputs(batch, H, W, Ch, N, dtype, seed, generic_A=False):

@@ -56,7 +56,9 @@ inline bool rec(cudaEvent_t *ev, int i, cudaStream_t stream) {
     return !ev || cudaEventRecord(ev[i], stream) == cudaSuccess;
 }
 
-template <typename T, int N>
+// ZOH: the exact hold's derivative (its own forward summaries and main kernel; the
+// adjoint summaries do not involve Bbar)
+template <typename T, int N, bool ZOH>
 vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], float *dC_out[2], float *dA,
                       float *dD, float *dbias, float *tmp, cudaStream_t stream, cudaEvent_t *ev) {
     if (!rec(ev, 0, stream)) return VIM_ERR_CUDA;
@@ -64,11 +66,11 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
         // h entering each chunk: the forward scan's own summary kernels
         const dim3 gf((a.Di + kDC - 1) / kDC, a.G, a.batch);
         const size_t sc = 2 * (size_t)Stage<T, N, false>::kSlotBytes;
-        auto carry = pair_carry<T, N, false, false, false>;
+        auto carry = pair_carry<T, N, false, false, ZOH>;
         if constexpr (bc_vectorizable<T, N>()) {
             // B and C rows as 16-byte vectors when every base allows it
             if (aligned16(fwd.B[0]) && aligned16(fwd.B[1]) && aligned16(fwd.C[0]) && aligned16(fwd.C[1]))
-                carry = pair_carry<T, N, true, false, false>;
+                carry = pair_carry<T, N, true, false, ZOH>;
         }
         if (cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sc) != cudaSuccess)
             return VIM_ERR_CUDA;
@@ -90,17 +92,17 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
     }
     if (!rec(ev, 1, stream)) return VIM_ERR_CUDA;
     constexpr size_t sm = BwdShape<N>::kSmemBytes;
-    if (cudaFuncSetAttribute(bwd_main<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
+    if (cudaFuncSetAttribute(bwd_main<T, N, ZOH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
         return VIM_ERR_CUDA;
     const dim3 gm(a.nblk, a.G, a.batch);
     if (a.G > 1) {
         // a programmatic dependent of the adjoint fold: its launch and the staging of
         // the first CTAs overlap the fold's end; it waits for the fold before it reads
         // the carries
-        if (launch_dependent(bwd_main<T, N>, gm, dim3(BwdShape<N>::kThr), sm, stream, a) != cudaSuccess)
+        if (launch_dependent(bwd_main<T, N, ZOH>, gm, dim3(BwdShape<N>::kThr), sm, stream, a) != cudaSuccess)
             return VIM_ERR_CUDA;
     } else {
-        bwd_main<T, N><<<gm, BwdShape<N>::kThr, sm, stream>>>(a);
+        bwd_main<T, N, ZOH><<<gm, BwdShape<N>::kThr, sm, stream>>>(a);
     }
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     if (!rec(ev, 2, stream)) return VIM_ERR_CUDA;
@@ -117,14 +119,14 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
     return rec(ev, 3, stream) ? VIM_OK : VIM_ERR_CUDA;
 }
 
-template <typename T>
+template <typename T, bool ZOH>
 vim_status launch_bwd_n(int N, const BwdArgs &a, const PairArgs &fwd, float *dB[2], float *dC[2], float *dA,
                         float *dD, float *dbias, float *tmp, cudaStream_t stream, cudaEvent_t *ev) {
     switch (N) {
-        case 2: return launch_bwd<T, 2>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
-        case 4: return launch_bwd<T, 4>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
-        case 8: return launch_bwd<T, 8>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
-        case 16: return launch_bwd<T, 16>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
+        case 2: return launch_bwd<T, 2, ZOH>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
+        case 4: return launch_bwd<T, 4, ZOH>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
+        case 8: return launch_bwd<T, 8, ZOH>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
+        case 16: return launch_bwd<T, 16, ZOH>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
         default: return VIM_ERR_UNSUPPORTED;
     }
 }
@@ -154,12 +156,14 @@ size_t vim_scan_bwd_workspace_bytes(int batch, int L, int d_inner, int d_state, 
     return bwd_plan(batch, L, d_inner, d_state, separate_bc).total;
 }
 
-vim_status vim_scan_bidir_bwd_events(const void *u, const void *delta, const void *z, const void *B,
-                                     const void *C, int64_t bc_dir_stride, const float *A, const float *D,
-                                     const float *delta_bias, const void *dout, void *du, void *ddelta, void *dz,
-                                     float *dB, float *dC, float *dA, float *dD, float *ddelta_bias, int batch,
-                                     int L, int d_inner, int d_state, vim_dtype dt, void *workspace,
-                                     size_t workspace_bytes, cudaStream_t stream, cudaEvent_t *events) {
+vim_status vim_scan_bidir_bwd_ex(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                                 int64_t bc_dir_stride, const float *A, const float *D, const float *delta_bias,
+                                 const void *dout, void *du, void *ddelta, void *dz, float *dB, float *dC,
+                                 float *dA, float *dD, float *ddelta_bias, int batch, int L, int d_inner,
+                                 int d_state, vim_dtype dt, unsigned flags, void *workspace, size_t workspace_bytes,
+                                 cudaStream_t stream, cudaEvent_t *events) {
+    if (flags & ~VIM_FLAG_ZOH_EXACT) return VIM_ERR_INVALID_ARG;
+    const bool zoh = (flags & VIM_FLAG_ZOH_EXACT) != 0;
     vim_status st = check_common(batch, L, d_inner, d_state, dt);
     if (st != VIM_OK) return st;
     if (bc_dir_stride < 0) return VIM_ERR_INVALID_ARG;
@@ -220,9 +224,23 @@ vim_status vim_scan_bidir_bwd_events(const void *u, const void *delta, const voi
 
     float *dBo[2] = {dB, dB + bc_dir_stride}, *dCo[2] = {dC, dC + bc_dir_stride};
     float *tmp = reinterpret_cast<float *>(ws + pl.off_tmp);
-    return dt == VIM_F32
-               ? launch_bwd_n<float>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream, events)
-               : launch_bwd_n<__nv_bfloat16>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream, events);
+    if (dt == VIM_F32)
+        return zoh ? launch_bwd_n<float, true>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream, events)
+                   : launch_bwd_n<float, false>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream, events);
+    return zoh ? launch_bwd_n<__nv_bfloat16, true>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream, events)
+               : launch_bwd_n<__nv_bfloat16, false>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream,
+                                                    events);
+}
+
+vim_status vim_scan_bidir_bwd_events(const void *u, const void *delta, const void *z, const void *B,
+                                     const void *C, int64_t bc_dir_stride, const float *A, const float *D,
+                                     const float *delta_bias, const void *dout, void *du, void *ddelta, void *dz,
+                                     float *dB, float *dC, float *dA, float *dD, float *ddelta_bias, int batch,
+                                     int L, int d_inner, int d_state, vim_dtype dt, void *workspace,
+                                     size_t workspace_bytes, cudaStream_t stream, cudaEvent_t *events) {
+    return vim_scan_bidir_bwd_ex(u, delta, z, B, C, bc_dir_stride, A, D, delta_bias, dout, du, ddelta, dz, dB, dC,
+                                 dA, dD, ddelta_bias, batch, L, d_inner, d_state, dt, 0u, workspace, workspace_bytes,
+                                 stream, events);
 }
 
 vim_status vim_scan_bidir_bwd(const void *u, const void *delta, const void *z, const void *B, const void *C,
@@ -324,8 +342,9 @@ vim_status vmamba_cross_scan4_bwd(const void *u, const void *delta, const void *
         float *tmp = reinterpret_cast<float *>(ws + pl.off_tmp);
         float *dAp = dA + (size_t)2 * pair * channels * d_state;
         float *dDp = dD + (size_t)2 * pair * channels, *dbp = ddelta_bias + (size_t)2 * pair * channels;
-        rc = dt == VIM_F32 ? launch_bwd_n<float>(d_state, a, f, dBo, dCo, dAp, dDp, dbp, tmp, stream, nullptr)
-                           : launch_bwd_n<__nv_bfloat16>(d_state, a, f, dBo, dCo, dAp, dDp, dbp, tmp, stream, nullptr);
+        rc = dt == VIM_F32
+                 ? launch_bwd_n<float, false>(d_state, a, f, dBo, dCo, dAp, dDp, dbp, tmp, stream, nullptr)
+                 : launch_bwd_n<__nv_bfloat16, false>(d_state, a, f, dBo, dCo, dAp, dDp, dbp, tmp, stream, nullptr);
     }
     return rc;
 }

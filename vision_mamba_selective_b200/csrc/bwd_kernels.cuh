@@ -1,8 +1,8 @@
 // bwd_kernels.cuh -- sm_100a kernels of the derivative of the Vim two-direction scan.
 //
 // The loss's derivative dout with respect to y = (y^f + y^b) * silu(z) is carried back
-// through the scan (first-order Bbar = Delta B), for every input: u, the raw delta,
-// z, B, C, A, D and the delta bias.  Per direction, with g_t the adjoint of h_t
+// through the scan (first-order Bbar = Delta B, or with ZOH the exact hold), for every
+// input: u, the raw delta, z, B, C, A, D and the delta bias.  Per direction, with g_t the adjoint of h_t
 // (g_t = C_t dy_t + Abar_(t+1) g_(t+1), dy = dout * silu(z)):
 //   dC_t += dy_t h_t                        dB_t += g_t Delta_t u_t
 //   du_t += D dy_t + Delta_t (g_t . B_t)    dD   += dy_t u_t
@@ -364,9 +364,47 @@ struct BwdThread {
     int tid, lane, q, cl, dir, wid, j0, d;
     bool valid;
     float2 A2[SH::NP], Araw[SH::NP];   // A of the thread's states, times log2(e) and as given
+    float2 invA[SH::NP];               // 1 / A_n (0 where A_n = 0), for the exact hold
     float Dk;
     size_t cbase;   // [b][c][dir][d]
 };
+
+// The exact hold's gain of one state, e = Bbar_n / B_n = (exp(z) - 1) / A_n with
+// z = Delta A_n, and its A-derivative, from z and Abar_n = exp(z) already formed:
+//   e       = Delta sum_{k>=0} z^k / (k+1)!            (Delta at A_n = 0)
+//   de/dA_n = (Delta Abar_n - e) / A_n = Delta^2 sum_{k>=1} k z^(k-1) / (k+1)!
+// (de/dDelta = Abar_n).  For |z| < 1/2 the series to z^7 (first omitted term below
+// 2e-8 of the sum), elsewhere the closed forms, which lose at most a few units of
+// rounding there.
+__device__ __forceinline__ float hold_gain(float dl, float z, float abar, float inv_a) {
+    if (fabsf(z) < 0.5f) {
+        float q = fmaf(z, 1.0f / 40320.0f, 1.0f / 5040.0f);
+        q = fmaf(z, q, 1.0f / 720.0f);
+        q = fmaf(z, q, 1.0f / 120.0f);
+        q = fmaf(z, q, 1.0f / 24.0f);
+        q = fmaf(z, q, 1.0f / 6.0f);
+        q = fmaf(z, q, 0.5f);
+        q = fmaf(z, q, 1.0f);
+        return dl * q;
+    }
+    return (abar - 1.0f) * inv_a;
+}
+__device__ __forceinline__ float hold_gain_dA(float dl, float z, float abar, float inv_a, float e) {
+    if (fabsf(z) < 0.5f) {
+        float q = fmaf(z, 1.0f / 45360.0f, 1.0f / 5760.0f);
+        q = fmaf(z, q, 1.0f / 840.0f);
+        q = fmaf(z, q, 1.0f / 144.0f);
+        q = fmaf(z, q, 1.0f / 30.0f);
+        q = fmaf(z, q, 1.0f / 8.0f);
+        q = fmaf(z, q, 1.0f / 3.0f);
+        q = fmaf(z, q, 0.5f);
+        return dl * dl * q;
+    }
+    return fmaf(dl, abar, -e) * inv_a;
+}
+__device__ __forceinline__ float2 hold_gain2(float dl, float2 z, float2 abar, float2 inv_a) {
+    return f2(hold_gain(dl, z.x, abar.x, inv_a.x), hold_gain(dl, z.y, abar.y, inv_a.y));
+}
 
 // h (or g) of the thread's states, from an fp32 row in global memory
 template <int NP>
@@ -413,7 +451,8 @@ __device__ __forceinline__ void channel_sum(const BwdThread<N> &th, float *red_w
 }
 
 // forward sweep of direction DIR: checkpoints, y^DIR (ungated) and the dC terms
-template <int N, int DIR>
+// (ZOH: the exact hold's Bbar in the state update)
+template <int N, int DIR, bool ZOH>
 __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
     using SH = BwdShape<N>;
     constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
@@ -440,7 +479,15 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
 #pragma unroll
             for (int k = 0; k < NP; ++k) {
                 const float2 e = mul2(dl2, th.A2[k]);
-                h[k] = fma2(f2(ex2(e.x), ex2(e.y)), h[k], mul2(du2, Bp[k]));
+                const float2 ab = f2(ex2(e.x), ex2(e.y));
+                float2 drive;
+                if constexpr (ZOH) {
+                    const float2 gn = hold_gain2(dl, mul2(dl2, th.Araw[k]), ab, th.invA[k]);
+                    drive = mul2(mul2(gn, Bp[k]), f2(tk.x, tk.x));
+                } else {
+                    drive = mul2(du2, Bp[k]);
+                }
+                h[k] = fma2(ab, h[k], drive);
                 yp = fma2(Cp[k], h[k], yp);
                 v[k] = mul2(dy2, h[k]);
             }
@@ -470,7 +517,7 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
 
 // adjoint sweep of direction DIR, segment by segment from the last: h re-run over
 // the segment from its checkpoint (keeping h and the decays), then g backwards
-template <int N, int DIR>
+template <int N, int DIR, bool ZOH>
 __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
     using SH = BwdShape<N>;
     constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
@@ -505,7 +552,14 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
             for (int k = 0; k < NP; ++k) {
                 const float2 e = mul2(dl2, th.A2[k]);
                 aa[m][k] = f2(ex2(e.x), ex2(e.y));
-                hh[m][k] = fma2(aa[m][k], m > 0 ? hh[m > 0 ? m - 1 : 0][k] : h0[k], mul2(du2, Bp[k]));
+                float2 drive;
+                if constexpr (ZOH) {
+                    const float2 gn = hold_gain2(dl, mul2(dl2, th.Araw[k]), aa[m][k], th.invA[k]);
+                    drive = mul2(mul2(gn, Bp[k]), f2(u, u));
+                } else {
+                    drive = mul2(du2, Bp[k]);
+                }
+                hh[m][k] = fma2(aa[m][k], m > 0 ? hh[m > 0 ? m - 1 : 0][k] : h0[k], drive);
             }
         }
 #pragma unroll
@@ -518,7 +572,7 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
             load_row<NP>(sm.B + (DIR * TC + r) * N + th.j0, Bp);
             load_row<NP>(sm.C + (DIR * TC + r) * N + th.j0, Cp);
             const float2 dl2 = f2(dl, dl), du2 = f2(du, du), dy2 = f2(tk.y, tk.y);
-            float2 sA = f2(0.f, 0.f), sB = f2(0.f, 0.f);
+            float2 sA = f2(0.f, 0.f), sB = f2(0.f, 0.f), sBa = f2(0.f, 0.f);
 #pragma unroll
             for (int k = 0; k < NP; ++k) {
                 g[k] = fma2(Cp[k], dy2, g[k]);                               // dl/dh_t
@@ -527,14 +581,35 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
                 const float2 w = mul2(ga, hp);
                 dA[k] = fma2(dl2, w, dA[k]);
                 sA = fma2(th.Araw[k], w, sA);
-                sB = fma2(g[k], Bp[k], sB);
-                v[k] = mul2(g[k], du2);
+                if constexpr (ZOH) {
+                    // Bbar_n = e_n B_n: du and dB take e_n for Delta, the Delta term
+                    // de_n/dDelta = Abar_n, and dA_n gains g B_n u de_n/dA_n
+                    const float2 zz = mul2(dl2, th.Araw[k]);
+                    const float2 gn = hold_gain2(dl, zz, aa[m][k], th.invA[k]);
+                    const float2 dg = f2(hold_gain_dA(dl, zz.x, aa[m][k].x, th.invA[k].x, gn.x),
+                                         hold_gain_dA(dl, zz.y, aa[m][k].y, th.invA[k].y, gn.y));
+                    const float2 gB = mul2(g[k], Bp[k]), uu = f2(tk.x, tk.x);
+                    sB = fma2(gB, gn, sB);
+                    sBa = fma2(gB, aa[m][k], sBa);
+                    dA[k] = fma2(mul2(gB, uu), dg, dA[k]);
+                    v[k] = mul2(mul2(g[k], gn), uu);
+                } else {
+                    sB = fma2(g[k], Bp[k], sB);
+                    v[k] = mul2(g[k], du2);
+                }
                 g[k] = ga;                                                   // dl/dh_(t-1) part
             }
             const float sAs = sA.x + sA.y, sBg = sB.x + sB.y;
             // this thread's share of du and d delta_raw, gathered over the Q lanes of
             // the channel: lane q = 0 ends with du, lane q = 1 with d delta_raw
-            float x0 = dl * sBg, x1 = fmaf(tk.x, sBg, sAs) * sgm;
+            float x0, x1;
+            if constexpr (ZOH) {
+                x0 = sBg;
+                x1 = fmaf(tk.x, sBa.x + sBa.y, sAs) * sgm;
+            } else {
+                x0 = dl * sBg;
+                x1 = fmaf(tk.x, sBg, sAs) * sgm;
+            }
             if constexpr (SH::BATCH) {
                 const int sl = kBwdSeg - 1 - m;
                 xq[2 * sl] = x0;
@@ -628,7 +703,7 @@ __device__ __forceinline__ void store_bc_part(const BwdArgs &p, const float *red
     }
 }
 
-template <typename T, int N>
+template <typename T, int N, bool ZOH>
 __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bwd_main(BwdArgs p) {
     using SH = BwdShape<N>;
     constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
@@ -733,6 +808,7 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
         const float2 a = th.valid ? f2(Ar[0], Ar[1]) : f2(0.f, 0.f);
         th.Araw[k] = a;
         th.A2[k] = f2(a.x * kLog2e, a.y * kLog2e);
+        th.invA[k] = f2(a.x != 0.0f ? 1.0f / a.x : 0.0f, a.y != 0.0f ? 1.0f / a.y : 0.0f);
     }
     th.Dk = th.valid ? p.D[(size_t)th.dir * p.Di + th.d] : 0.0f;
     th.cbase = (((size_t)b * p.G + c) * 2 + th.dir) * p.Di + th.d;
@@ -743,8 +819,8 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     // carries are read after the wait
     if (p.G > 1) cudaGridDependencySynchronize();
 
-    if (th.dir == 0) bwd_forward<N, 0>(p, sm, th);
-    else bwd_forward<N, 1>(p, sm, th);
+    if (th.dir == 0) bwd_forward<N, 0, ZOH>(p, sm, th);
+    else bwd_forward<N, 1, ZOH>(p, sm, th);
     __syncthreads();
     // dz = dout silu'(z) (sum of the directions' y), and the CTA's dC terms; the
     // cross-scan's first pair leaves its y for the second
@@ -773,8 +849,8 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     store_bc_part<N>(p, sm.red, p.dC_part, b, t0, tc, blk);
     __syncthreads();
 
-    if (th.dir == 0) bwd_adjoint<N, 0>(p, sm, th);
-    else bwd_adjoint<N, 1>(p, sm, th);
+    if (th.dir == 0) bwd_adjoint<N, 0, ZOH>(p, sm, th);
+    else bwd_adjoint<N, 1, ZOH>(p, sm, th);
     __syncthreads();
     for (int li = threadIdx.x; li < TC * (CH / kG); li += SH::kThr) {
         const int r = li / (CH / kG), c0 = (li % (CH / kG)) * kG, ch = d0 + c0;

@@ -54,6 +54,10 @@ lib.vim_scan_bidir_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp,
 lib.vim_scan_bidir_bwd.restype = _i
 lib.vim_scan_bidir_bwd_events.argtypes = lib.vim_scan_bidir_bwd.argtypes + [_vp]
 lib.vim_scan_bidir_bwd_events.restype = _i
+# the _bwd arguments with `flags` before the workspace, then the events
+lib.vim_scan_bidir_bwd_ex.argtypes = (lib.vim_scan_bidir_bwd.argtypes[:23] + [ctypes.c_uint]
+                                      + lib.vim_scan_bidir_bwd.argtypes[23:] + [_vp])
+lib.vim_scan_bidir_bwd_ex.restype = _i
 lib.vim_scan_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
 lib.vim_scan_bwd_workspace_bytes.restype = _sz
 lib.vim_block_scan.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
@@ -199,9 +203,10 @@ def vim_scan_bwd_workspace_bytes(batch, L, d_inner, d_state, separate_bc):
 
 
 def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stride=0, workspace=None,
-                       stream=None, out=None, events=None):
-    """Derivatives of vim_scan_bidir (first-order Bbar) for a loss whose derivative
-    with respect to y is ``dout``; see include/vimscan.h.
+                       stream=None, out=None, events=None, zoh=False):
+    """Derivatives of vim_scan_bidir (first-order Bbar, or with ``zoh`` the exact
+    zero-order hold) for a loss whose derivative with respect to y is ``dout``; see
+    include/vimscan.h.
 
     Returns a dict: du, ddelta (w.r.t. the raw delta), dz (None without z), in the
     input dtype; dB and dC (fp32, shaped like B and C); dA [2, d_inner, d_state], dD
@@ -221,8 +226,12 @@ def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stri
                dD=torch.empty((2, Di), dtype=torch.float32, device=dev),
                ddelta_bias=torch.empty((2, Di), dtype=torch.float32, device=dev))
     ws, ws_bytes = _workspace(vim_scan_bwd_workspace_bytes(batch, L, Di, N, bc_dir_stride > 0), workspace, dev)
-    fn = lib.vim_scan_bidir_bwd if events is None else lib.vim_scan_bidir_bwd_events
-    extra = () if events is None else (_events(events),)
+    if zoh:
+        fn = lib.vim_scan_bidir_bwd_ex
+        flags, extra = (VIM_FLAG_ZOH_EXACT,), (None if events is None else _events(events),)
+    else:
+        fn = lib.vim_scan_bidir_bwd if events is None else lib.vim_scan_bidir_bwd_events
+        flags, extra = (), (() if events is None else (_events(events),))
     st = fn(
         _ptr(u, name="u"), _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
         _ptr(B, dtype=u.dtype, name="B"), _ptr(C, dtype=u.dtype, name="C"), int(bc_dir_stride),
@@ -230,7 +239,7 @@ def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stri
         _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(dout, dtype=u.dtype, name="dout"),
         _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dz"]), _ptr(out["dB"]), _ptr(out["dC"]),
         _ptr(out["dA"]), _ptr(out["dD"]), _ptr(out["ddelta_bias"]),
-        batch, L, Di, N, dt, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream), *extra)
+        batch, L, Di, N, dt, *flags, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream), *extra)
     if st != VIM_OK:
         raise VimScanError(st, "vim_scan_bidir_bwd")
     return out
