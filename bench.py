@@ -230,7 +230,8 @@ def run_oracle(w, x, threads, zoh=False):
         oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], x["dout"],
                              zoh=zoh)
     elif "dout" in x:
-        oracle.cross_scan4_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], x["dout"])
+        oracle.cross_scan4_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], x["dout"],
+                               zoh=zoh)
     elif "conv_w" in x:
         oracle.vim_bidir_conv(x["u"], x["conv_w"], x["conv_b"], x["delta"], x["z"], x["B"], x["C"], x["A"],
                               x["D"], x["delta_bias"], zoh=zoh)
@@ -344,8 +345,8 @@ def main():
         raise SystemExit("--conv and --block apply to the Vim workloads only")
     if args.block and (args.conv or args.zoh or args.bwd or w.dtype != "bf16"):
         raise SystemExit("--block runs alone, on a bf16 workload")
-    if args.bwd and (args.conv or (args.zoh and w.kind != "vim")):
-        raise SystemExit("--bwd covers the plain scan (no --conv), with --zoh on the Vim workloads")
+    if args.bwd and args.conv:
+        raise SystemExit("--bwd covers the scan without the front (--zoh allowed)")
     if args.impl == "reference":
         reference_arm(args, w)
         return
@@ -418,7 +419,7 @@ def main():
             return
         if args.bwd:
             vs.vmamba_cross_scan4_bwd(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"],
-                                      params["delta_bias"], s["dout"], workspace=ws, out=s["out"])
+                                      params["delta_bias"], s["dout"], workspace=ws, out=s["out"], zoh=args.zoh)
             return
         if args.conv:
             # u holds x, the pathways' common input in front of the convolutions

@@ -325,6 +325,21 @@ vim_status vim_scan_bidir_bwd_ex(const void *u, const void *delta, const void *z
                                  unsigned flags, void *workspace, size_t workspace_bytes,
                                  cudaStream_t stream, cudaEvent_t *events);
 
+/*
+ * vmamba_cross_scan4_bwd with options in `flags` (unknown bits return
+ * VIM_ERR_INVALID_ARG): VIM_FLAG_ZOH_EXACT gives the derivative of the cross-scan with
+ * the exact hold, each direction's terms as in vim_scan_bidir_bwd_ex.  Other arguments
+ * and the workspace as in vmamba_cross_scan4_bwd.
+ */
+vim_status vmamba_cross_scan4_bwd_ex(const void *u, const void *delta, const void *z,
+                                     const void *B, const void *C,
+                                     const float *A, const float *D, const float *delta_bias,
+                                     const void *dout, void *du, void *ddelta, void *dz,
+                                     float *dB, float *dC, float *dA, float *dD, float *ddelta_bias,
+                                     int batch, int H, int W, int channels, int d_state, vim_dtype dt,
+                                     unsigned flags, void *workspace, size_t workspace_bytes,
+                                     cudaStream_t stream);
+
 /* vmamba_cross_scan4 with the options in `flags` and the events of
  * vmamba_cross_scan4_events when `events` is non-NULL. */
 vim_status vmamba_cross_scan4_ex(const void *u, const void *delta, const void *z,

@@ -40,6 +40,7 @@ def test_header_declares_the_boundary():
                           "vim_scan_bidir_bwd_ex",
                           "vim_block_scan", "vim_block_workspace_bytes",
                           "vmamba_cross_scan4_bwd", "vmamba_cross_scan4_bwd_workspace_bytes",
+                          "vmamba_cross_scan4_bwd_ex",
                           "vim_scan_workspace_bytes", "vim_status_string"}, names
 
 
@@ -180,6 +181,11 @@ def test_cross_bwd_and_block_reject(vs):
     assert xb(a23=None) == vs.VIM_ERR_WORKSPACE
     assert xb(a23=F + 16) == vs.VIM_ERR_WORKSPACE
     assert vs.lib.vmamba_cross_scan4_bwd_workspace_bytes(2, 8, 8, 64, 16) > 0
+    # the options entry: an unknown flag bit is refused; the exact hold's flag passes the
+    # flag check and stops at the missing workspace (no call here reaches a launch)
+    ex = lambda flags, ws: lib.vmamba_cross_scan4_bwd_ex(*(args[:23] + [flags, ws] + args[24:]))
+    assert ex(2, F) == vs.VIM_ERR_INVALID_ARG
+    assert ex(vs.VIM_FLAG_ZOH_EXACT, None) == vs.VIM_ERR_WORKSPACE
     # block scan: fp32 unsupported, half a convolution front, missing weights
     def blk(**kw):
         a = dict(x=F, cw=F, cb=F, Wx=F, Wdt=F, db=F, A=F, D=F, z=F, y=F, b=2, L=100, Di=64, N=16,

@@ -298,3 +298,28 @@ def test_cross_bwd_full_size(vs):
     torch.cuda.synchronize()
     want = oracle.cross_scan4_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], dout)
     check_all("cross_bwd_full", got, want, torch.bfloat16, sum_tol=1e-3)
+
+
+CROSS_ZOH_CASES = [
+    # batch, H, W, C, N, dtype, generic_A
+    (1, 3, 5, 16, 16, torch.float32, False),
+    (2, 5, 3, 24, 8, torch.float32, True),
+    (1, 7, 40, 64, 16, torch.float32, False),     # several 32-token chunks in both orders
+    (2, 16, 16, 64, 16, torch.bfloat16, False),
+]
+
+
+@pytest.mark.parametrize("case", CROSS_ZOH_CASES, ids=lambda c: f"b{c[0]}_{c[1]}x{c[2]}_C{c[3]}_N{c[4]}_"
+                         f"{str(c[5])[6:]}{'_genA' if c[6] else ''}")
+def test_cross_bwd_zoh(vs, case):
+    """The cross-scan's derivative with the exact hold (vmamba_cross_scan4_bwd_ex)
+    against the oracle's."""
+    batch, H, W, Ch, N, dtype, gen = case
+    x = cross_inputs(batch, H, W, Ch, N, dtype, seed=H * 19 + W, generic_A=gen)
+    c = lambda k: x[k].cuda()
+    got = vs.vmamba_cross_scan4_bwd(c("u"), c("delta"), c("z"), c("B"), c("C"), c("A"), c("D"), c("bias"),
+                                    c("dout"), zoh=True)
+    torch.cuda.synchronize()
+    want = oracle.cross_scan4_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["bias"], x["dout"],
+                                  zoh=True)
+    check_all(f"cross_bwd_zoh_{case}", got, want, dtype)

@@ -260,11 +260,14 @@ size_t vmamba_cross_scan4_bwd_workspace_bytes(int batch, int H, int W, int chann
     return bwd_plan(batch, L, channels, d_state, 1).total + 3 * round_up((size_t)batch * L * channels * 4);
 }
 
-vim_status vmamba_cross_scan4_bwd(const void *u, const void *delta, const void *z, const void *B, const void *C,
-                                  const float *A, const float *D, const float *delta_bias, const void *dout,
-                                  void *du, void *ddelta, void *dz, float *dB, float *dC, float *dA, float *dD,
-                                  float *ddelta_bias, int batch, int H, int W, int channels, int d_state,
-                                  vim_dtype dt, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+vim_status vmamba_cross_scan4_bwd_ex(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                                     const float *A, const float *D, const float *delta_bias, const void *dout,
+                                     void *du, void *ddelta, void *dz, float *dB, float *dC, float *dA, float *dD,
+                                     float *ddelta_bias, int batch, int H, int W, int channels, int d_state,
+                                     vim_dtype dt, unsigned flags, void *workspace, size_t workspace_bytes,
+                                     cudaStream_t stream) {
+    if (flags & ~VIM_FLAG_ZOH_EXACT) return VIM_ERR_INVALID_ARG;
+    const bool zoh = (flags & VIM_FLAG_ZOH_EXACT) != 0;
     if (H < 0 || W < 0) return VIM_ERR_INVALID_ARG;
     if ((int64_t)H * W > INT32_MAX) return VIM_ERR_UNSUPPORTED;
     const int L = H * W;
@@ -342,11 +345,25 @@ vim_status vmamba_cross_scan4_bwd(const void *u, const void *delta, const void *
         float *tmp = reinterpret_cast<float *>(ws + pl.off_tmp);
         float *dAp = dA + (size_t)2 * pair * channels * d_state;
         float *dDp = dD + (size_t)2 * pair * channels, *dbp = ddelta_bias + (size_t)2 * pair * channels;
-        rc = dt == VIM_F32
-                 ? launch_bwd_n<float, false>(d_state, a, f, dBo, dCo, dAp, dDp, dbp, tmp, stream, nullptr)
-                 : launch_bwd_n<__nv_bfloat16, false>(d_state, a, f, dBo, dCo, dAp, dDp, dbp, tmp, stream, nullptr);
+        if (dt == VIM_F32)
+            rc = zoh ? launch_bwd_n<float, true>(d_state, a, f, dBo, dCo, dAp, dDp, dbp, tmp, stream, nullptr)
+                     : launch_bwd_n<float, false>(d_state, a, f, dBo, dCo, dAp, dDp, dbp, tmp, stream, nullptr);
+        else
+            rc = zoh ? launch_bwd_n<__nv_bfloat16, true>(d_state, a, f, dBo, dCo, dAp, dDp, dbp, tmp, stream, nullptr)
+                     : launch_bwd_n<__nv_bfloat16, false>(d_state, a, f, dBo, dCo, dAp, dDp, dbp, tmp, stream,
+                                                          nullptr);
     }
     return rc;
+}
+
+vim_status vmamba_cross_scan4_bwd(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                                  const float *A, const float *D, const float *delta_bias, const void *dout,
+                                  void *du, void *ddelta, void *dz, float *dB, float *dC, float *dA, float *dD,
+                                  float *ddelta_bias, int batch, int H, int W, int channels, int d_state,
+                                  vim_dtype dt, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    return vmamba_cross_scan4_bwd_ex(u, delta, z, B, C, A, D, delta_bias, dout, du, ddelta, dz, dB, dC, dA, dD,
+                                     ddelta_bias, batch, H, W, channels, d_state, dt, 0u, workspace, workspace_bytes,
+                                     stream);
 }
 
 }  // extern "C"

@@ -66,6 +66,8 @@ lib.vim_block_scan.restype = _i
 lib.vim_block_workspace_bytes.argtypes = [_i, _i, _i, _i]
 lib.vim_block_workspace_bytes.restype = _sz
 lib.vmamba_cross_scan4_bwd.argtypes = [_vp] * 17 + [_i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
+lib.vmamba_cross_scan4_bwd_ex.argtypes = [_vp] * 17 + [_i, _i, _i, _i, _i, _i, ctypes.c_uint, _vp, _sz, _vp]
+lib.vmamba_cross_scan4_bwd_ex.restype = _i
 lib.vmamba_cross_scan4_bwd.restype = _i
 lib.vmamba_cross_scan4_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
 lib.vmamba_cross_scan4_bwd_workspace_bytes.restype = _sz
@@ -245,8 +247,10 @@ def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stri
     return out
 
 
-def vmamba_cross_scan4_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, workspace=None, stream=None, out=None):
-    """Derivatives of vmamba_cross_scan4 (first-order Bbar) for a loss whose derivative
+def vmamba_cross_scan4_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, workspace=None, stream=None, out=None,
+                           zoh=False):
+    """Derivatives of vmamba_cross_scan4 (first-order Bbar, or with ``zoh`` the exact
+    zero-order hold) for a loss whose derivative
     with respect to y is ``dout``; see include/vimscan.h.  Returns a dict: du, ddelta, dz
     (None without z) in the input dtype; dB, dC [4, batch, H*W, N], dA [4, C, N], dD and
     ddelta_bias [4, C] in fp32.  ``out`` may hold those tensors from an earlier call.
@@ -259,14 +263,16 @@ def vmamba_cross_scan4_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, workspa
         out = dict(du=torch.empty_like(u), ddelta=torch.empty_like(u), dz=torch.empty_like(u) if z is not None else None,
                    dB=f32(*B.shape), dC=f32(*C.shape), dA=f32(4, Ch, N), dD=f32(4, Ch), ddelta_bias=f32(4, Ch))
     ws, ws_bytes = _workspace(int(lib.vmamba_cross_scan4_bwd_workspace_bytes(batch, H, W, Ch, N)), workspace, dev)
-    st = lib.vmamba_cross_scan4_bwd(
+    fn = lib.vmamba_cross_scan4_bwd_ex if zoh else lib.vmamba_cross_scan4_bwd
+    flags = (VIM_FLAG_ZOH_EXACT,) if zoh else ()
+    st = fn(
         _ptr(u, name="u"), _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
         _ptr(B, dtype=u.dtype, name="B"), _ptr(C, dtype=u.dtype, name="C"),
         _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
         _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(dout, dtype=u.dtype, name="dout"),
         _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dz"]), _ptr(out["dB"]), _ptr(out["dC"]),
         _ptr(out["dA"]), _ptr(out["dD"]), _ptr(out["ddelta_bias"]),
-        batch, H, W, Ch, N, _dtype_code(u), None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
+        batch, H, W, Ch, N, _dtype_code(u), *flags, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
     if st != VIM_OK:
         raise VimScanError(st, "vmamba_cross_scan4_bwd")
     return out
