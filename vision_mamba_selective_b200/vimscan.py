@@ -1,7 +1,8 @@
 """Thin ctypes binding of libvimscan.so (declared in include/vimscan.h).
 
-Argument marshalling only: tensors are checked for device, dtype, shape and
-contiguity, turned into raw device pointers and handed to the C ABI together with
+Argument marshalling only: every tensor is checked for device (the current CUDA
+device), dtype, shape and contiguity before the library is called, then turned into
+raw device pointers and handed to the C ABI together with
 the current torch CUDA stream.  Every step of the scan runs in the library's sm_100a
 kernels; there is no fallback of any kind, and a missing library is an ImportError.
 """
@@ -117,6 +118,43 @@ def _ptr(t, *, dtype=None, name="tensor"):
     return t.data_ptr()
 
 
+def _check(where, ref, specs):
+    """Refuse, before the library is called, any tensor the kernels could not address
+    safely.
+
+    ``ref`` is the tensor that fixes the device; it must be the current CUDA device
+    (the stream the library launches on belongs to it).  ``specs`` holds
+    (name, tensor or None, rule) with rule either an exact shape tuple or
+    ("numel", n, last): at least n elements with last dimension ``last`` (buffers such
+    as B/C with a per-direction stride).  Raises TypeError or ValueError.
+    """
+    if not isinstance(ref, torch.Tensor) or not ref.is_cuda:
+        raise TypeError(f"{where}: inputs must be CUDA tensors")
+    cur = torch.cuda.current_device()
+    if ref.device.index != cur:
+        raise ValueError(f"{where}: tensors are on {ref.device} but the current device is cuda:{cur}")
+    for name, t, rule in specs:
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{where}: {name} must be a CUDA tensor")
+        if t.device != ref.device:
+            raise ValueError(f"{where}: {name} is on {t.device}, the other inputs on {ref.device}")
+        if rule and rule[0] == "numel":
+            _, n, last = rule
+            if t.numel() < n or t.dim() == 0 or t.shape[-1] != last:
+                raise ValueError(f"{where}: {name} has shape {tuple(t.shape)}; it needs at least {n} "
+                                 f"elements with last dimension {last}")
+        elif tuple(t.shape) != tuple(rule):
+            raise ValueError(f"{where}: {name} has shape {tuple(t.shape)}, expected {tuple(rule)}")
+
+
+def _bc_rule(batch, L, N, bc_dir_stride):
+    if bc_dir_stride < 0:
+        raise ValueError("bc_dir_stride must be >= 0")
+    return ("numel", int(bc_dir_stride) + batch * L * N, N)
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -148,6 +186,11 @@ def _bidir(name, u, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, y, bc_dir_
     batch, L, Di = u.shape
     N = B.shape[-1]
     dt = _dtype_code(u)
+    act = (batch, L, Di)
+    bc = _bc_rule(batch, L, N, bc_dir_stride)
+    _check(name, u, [("delta", delta, act), ("z", z, act), ("B", B, bc), ("C", C, bc), ("A", A, (2, Di, N)),
+                     ("D", D, (2, Di)), ("delta_bias", delta_bias, (2, Di)), ("y", y, act),
+                     ("conv_w", conv_w, (2, Di, 3)), ("conv_b", conv_b, (2, Di))])
     if y is None:
         y = torch.empty_like(u)
     ws, ws_bytes = _workspace(vim_scan_workspace_bytes(0, batch, L, 0, Di, N), workspace, u.device)
@@ -220,6 +263,17 @@ def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stri
     N = B.shape[-1]
     dt = _dtype_code(u)
     dev = u.device
+    act = (batch, L, Di)
+    bc = _bc_rule(batch, L, N, bc_dir_stride)
+    specs = [("delta", delta, act), ("z", z, act), ("B", B, bc), ("C", C, bc), ("A", A, (2, Di, N)),
+             ("D", D, (2, Di)), ("delta_bias", delta_bias, (2, Di)), ("dout", dout, act)]
+    if out is not None:
+        specs += [("out['du']", out["du"], act), ("out['ddelta']", out["ddelta"], act),
+                  ("out['dz']", out["dz"], act), ("out['dB']", out["dB"], bc), ("out['dC']", out["dC"], bc), ("out['dA']", out["dA"], (2, Di, N)),
+                  ("out['dD']", out["dD"], (2, Di)), ("out['ddelta_bias']", out["ddelta_bias"], (2, Di))]
+        if z is not None and out["dz"] is None:
+            raise ValueError("vim_scan_bidir_bwd: out['dz'] is needed when z is given")
+    _check("vim_scan_bidir_bwd", u, specs)
     out = out if out is not None else dict(du=torch.empty_like(u), ddelta=torch.empty_like(u),
                dz=torch.empty_like(u) if z is not None else None,
                dB=torch.zeros(B.shape, dtype=torch.float32, device=dev),
@@ -258,6 +312,18 @@ def vmamba_cross_scan4_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, workspa
     batch, H, W, Ch = u.shape
     N = B.shape[-1]
     dev = u.device
+    act = (batch, H, W, Ch)
+    bc = (4, batch, H * W, N)
+    specs = [("delta", delta, act), ("z", z, act), ("B", B, bc), ("C", C, bc), ("A", A, (4, Ch, N)),
+             ("D", D, (4, Ch)), ("delta_bias", delta_bias, (4, Ch)), ("dout", dout, act)]
+    if out is not None:
+        specs += [("out['du']", out["du"], act), ("out['ddelta']", out["ddelta"], act),
+                  ("out['dz']", out["dz"], act), ("out['dB']", out["dB"], bc), ("out['dC']", out["dC"], bc),
+                  ("out['dA']", out["dA"], (4, Ch, N)), ("out['dD']", out["dD"], (4, Ch)),
+                  ("out['ddelta_bias']", out["ddelta_bias"], (4, Ch))]
+        if z is not None and out["dz"] is None:
+            raise ValueError("vmamba_cross_scan4_bwd: out['dz'] is needed when z is given")
+    _check("vmamba_cross_scan4_bwd", u, specs)
     f32 = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
     if out is None:
         out = dict(du=torch.empty_like(u), ddelta=torch.empty_like(u), dz=torch.empty_like(u) if z is not None else None,
@@ -291,6 +357,10 @@ def vim_block_scan(x, Wx, Wdt, dt_bias, A, D, z, *, conv_w=None, conv_b=None, y=
     """
     batch, L, Di = x.shape
     N = A.shape[-1]
+    act = (batch, L, Di)
+    _check("vim_block_scan", x, [("Wx", Wx, (2, Di, 2 * N + 1)), ("Wdt", Wdt, (2, Di)), ("dt_bias", dt_bias, (2, Di)),
+                                  ("A", A, (2, Di, N)), ("D", D, (2, Di)), ("z", z, act), ("y", y, act),
+                                  ("conv_w", conv_w, (2, Di, 3)), ("conv_b", conv_b, (2, Di))])
     if y is None:
         y = torch.empty_like(x)
     ws, ws_bytes = _workspace(vim_block_workspace_bytes(batch, L, Di, N), workspace, x.device)
@@ -318,6 +388,11 @@ def vim_scan_bidir_noalloc(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_di
     batch, L, Di = u.shape
     N = B.shape[-1]
     dt = _dtype_code(u)
+    act = (batch, L, Di)
+    bc = _bc_rule(batch, L, N, bc_dir_stride)
+    _check("vim_scan_bidir_noalloc", u, [("delta", delta, act), ("z", z, act), ("B", B, bc), ("C", C, bc),
+                                          ("A", A, (2, Di, N)), ("D", D, (2, Di)),
+                                          ("delta_bias", delta_bias, (2, Di)), ("y", y, act)])
     if y is None:
         y = torch.empty_like(u)
     st = lib.vim_scan_bidir_noalloc(
@@ -342,6 +417,11 @@ def vmamba_cross_scan4(u, delta, z, B, C, A, D, delta_bias, *, y=None, workspace
     batch, H, W, Ch = u.shape
     N = B.shape[-1]
     dt = _dtype_code(u)
+    act = (batch, H, W, Ch)
+    bc = (4, batch, H * W, N)
+    _check("vmamba_cross_scan4", u, [("delta", delta, act), ("z", z, act), ("B", B, bc), ("C", C, bc),
+                                      ("A", A, (4, Ch, N)), ("D", D, (4, Ch)), ("delta_bias", delta_bias, (4, Ch)),
+                                      ("y", y, act)])
     if y is None:
         y = torch.empty_like(u)
     ws, ws_bytes = _workspace(vim_scan_workspace_bytes(1, batch, H, W, Ch, N), workspace, u.device)
@@ -367,8 +447,10 @@ def vmamba_cross_scan4(u, delta, z, B, C, A, D, delta_bias, *, y=None, workspace
 def cross_merge4(ys, z, H, W, *, y=None, stream=None):
     """CS-Merge alone: ys [4, batch, H*W, C] in scan order -> y [batch, H, W, C]."""
     _, batch, L, Ch = ys.shape
-    if L != H * W:
-        raise ValueError("ys.shape[2] must be H*W")
+    if ys.shape[0] != 4 or L != H * W:
+        raise ValueError("ys must be [4, batch, H*W, C]")
+    act = (batch, H, W, Ch)
+    _check("cross_merge4", ys, [("z", z, act), ("y", y, act)])
     dt = _dtype_code(ys)
     if y is None:
         y = torch.empty((batch, H, W, Ch), dtype=ys.dtype, device=ys.device)
