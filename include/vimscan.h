@@ -366,11 +366,14 @@ vim_status vmamba_cross_scan4_ex(const void *u, const void *delta, const void *z
  *     (sequences of up to 256 tokens need none).  Larger problems return
  *     VIM_ERR_WORKSPACE and launch nothing.
  *   - The first call on each device looks up the buffer's device address (with that
- *     device current) and remembers it; make that first call before any stream
- *     capture.  A failed lookup returns VIM_ERR_CUDA.
+ *     device current) and remembers it for the rest of the process; make that first
+ *     call before any stream capture.  A failed lookup returns VIM_ERR_CUDA.  The
+ *     remembered address belongs to the device's primary context as it was then: after
+ *     cudaDeviceReset (or anything else that destroys that context) this entry point
+ *     must not be called again in the same process.
  *   - All calls share the one buffer, and it keeps whatever the last call left in it.
- *     Nothing in it needs to start at zero: every value a call reads was written
- *     earlier by the same call.  Calls whose work overlaps on the GPU (two streams,
+ *     Nothing in it needs to start at zero: every value a call reads from it was
+ *     written earlier by the same call.  Calls whose work overlaps on the GPU (two streams,
  *     or two threads with the same device) race on the buffer and corrupt each
  *     other's results: serialise them.
  */
