@@ -85,7 +85,6 @@ template <typename T, int N, bool CONV>
 size_t carry_smem() {
     return 2 * (size_t)Stage<T, N, CONV>::kSlotBytes;
 }
-
 // Launch of a kernel that may start while the previous kernel on the stream drains
 // (programmatic dependent launch); the kernel itself waits, with
 // cudaGridDependencySynchronize, before it reads anything that kernel writes.

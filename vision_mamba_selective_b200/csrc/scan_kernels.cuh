@@ -28,6 +28,14 @@
 // For G > 1 the state entering each chunk comes from two small kernels: `pair_carry`
 // reduces every chunk to its end state from h = 0 plus its total Delta, and
 // `pair_combine` folds those summaries along each direction.
+//
+// State form (structured A, first-order Bbar; VIMSCAN_GF): the main kernel runs the
+// scaled state g = h / du, du = Delta u, instead of h (see main_tile): the decay chain
+// absorbs du_(t-1) / du_t and the drive is B itself, which removes one multiply per
+// state and token.  Units (bf16 I/O, first-order Bbar; VIMSCAN_L2U): Delta is kept as
+// L = Delta / ln 2, so softplus is log2(1 + 2^(x log2 e)) with no rescaling, the decay
+// base is 2^(A_0 L), and B is staged multiplied by ln 2; the chunk summaries leave
+// their Delta sums in natural units.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -64,6 +72,16 @@ constexpr int kCarryMinBlocks = VIMSCAN_CARRY_MIN_BLOCKS;
 constexpr int kCarryZohSub = VIMSCAN_CARRY_ZOH_KSUB;   // the same two with the exact hold
 constexpr int kCarryZohMinBlocks = VIMSCAN_CARRY_ZOH_MIN_BLOCKS;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.69314718055994531f;
+#ifndef VIMSCAN_GF
+#define VIMSCAN_GF 1
+#endif
+#ifndef VIMSCAN_L2U
+#define VIMSCAN_L2U 1
+#endif
+// bf16 first-order kernels may keep Delta in log2 units (L = Delta / ln 2)
+template <typename T, bool ZOH>
+__host__ __device__ constexpr bool lu_mode() { return VIMSCAN_L2U && sizeof(T) == 2 && !ZOH; }
 
 // ----------------------------------------------------------------------------
 // element types
@@ -185,6 +203,15 @@ __device__ __forceinline__ float zoh_gain(float dt, float An) {
 
 // silu(z) = z / (1 + exp(-z))
 __device__ __forceinline__ float silu(float z) { return z * rcp(1.0f + ex2(-z * kLog2e)); }
+
+// softplus in log2 units: log2(1 + 2^xl) for xl = x log2 e, and xl itself for x > 20
+__device__ __forceinline__ float softplus_l2(float xl) {
+    const float r = lg2(1.0f + ex2(xl));
+    return xl > 20.0f * kLog2e ? xl : r;
+}
+
+// |du| kept at or above 1e-20 for the scaled state g = h / du (see main_tile)
+__device__ __forceinline__ float clamp_du(float v) { return fabsf(v) < 1.0e-20f ? 1.0e-20f : v; }
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
@@ -389,8 +416,10 @@ struct Stager {
     }
 
     // With the exact zero-order hold, B is staged as B_n / (n + 1) (the kernels' form
-    // of Bbar divides by A_n = (n + 1) A_0; see main_tile).
+    // of Bbar divides by A_n = (n + 1) A_0; see main_tile); in log2 units as ln 2 B_n,
+    // so that (L u)(ln 2 B) = Delta u B.
     __device__ void store_bc(char *slot) const {
+        constexpr bool LU = lu_mode<T, ZOH>();
 #pragma unroll
         for (int k = 0; k < kBCPer; ++k) {
             const int i = threadIdx.x + k * kThreads;
@@ -407,12 +436,17 @@ struct Stager {
 #pragma unroll
                     for (int e = 0; e < V; ++e) f[e] *= __frcp_rn((float)(part * V + e + 1));
                 }
+                if (LU && which == 0) {
+#pragma unroll
+                    for (int e = 0; e < V; ++e) f[e] *= kLn2;
+                }
                 float4 *d4 = reinterpret_cast<float4 *>(dst + part * V);
 #pragma unroll
                 for (int q = 0; q < V / 4; ++q)
                     d4[q] = make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
             } else {
-                dst[part] = (ZOH && which == 0) ? pre_s[k] * __frcp_rn((float)(part + 1)) : pre_s[k];
+                dst[part] = (ZOH && which == 0) ? pre_s[k] * __frcp_rn((float)(part + 1))
+                            : (LU && which == 0) ? pre_s[k] * kLn2 : pre_s[k];
             }
         }
     }
@@ -424,7 +458,8 @@ struct Stager {
 template <int N>
 struct ChannelParams {
     const float *A;     // A[dir][d][:] (general-A path)
-    float A0;           // A[d][0] * log2(e)
+    float A0;           // A[d][0] times log2(e) (natural units) or 1 (log2 units)
+    float emul;         // the same factor for the general-A path
     float a0, inv_a0;   // A[d][0] and its reciprocal (0 when A[d][0] = 0)
     float D, bias;
     float cw_prev, cw_cur, cw_next, cbias;   // convolution front: taps on x[t-1], x[t], x[t+1]
@@ -432,9 +467,12 @@ struct ChannelParams {
     bool structured;    // A[d][n] == (n+1) A[d][0] for every n
     bool valid;
 
+    // LU: Delta in log2 units; the bias and dt_proj weight are then scaled by log2 e
+    template <bool LU = false>
     __device__ void load(const PairArgs &p, int dir, int d) {
         valid = d < p.Di;
         structured = true;
+        emul = LU ? 1.0f : kLog2e;
         A0 = D = bias = a0 = inv_a0 = 0.0f;
         cw_prev = cw_cur = cw_next = cbias = dtw = 0.0f;
         A = p.A;
@@ -448,15 +486,15 @@ struct ChannelParams {
             cw_next = dir ? w[0] : w[2];
             cbias = p.conv_b[(size_t)dir * p.Di + d];
         }
-        if (p.dt_w) dtw = p.dt_w[(size_t)dir * p.Di + d];
+        if (p.dt_w) dtw = p.dt_w[(size_t)dir * p.Di + d] * (LU ? kLog2e : 1.0f);
         A = p.A + ((size_t)dir * p.Di + d) * N;
         a0 = A[0];
 #pragma unroll
         for (int n = 0; n < N; ++n) structured = structured && (A[n] == (float)(n + 1) * a0);
-        A0 = a0 * kLog2e;
+        A0 = a0 * emul;
         inv_a0 = a0 != 0.0f ? 1.0f / a0 : 0.0f;
         D = p.D[(size_t)dir * p.Di + d];
-        bias = p.bias[(size_t)dir * p.Di + d];
+        bias = p.bias[(size_t)dir * p.Di + d] * (LU ? kLog2e : 1.0f);
     }
 };
 
@@ -482,11 +520,15 @@ __device__ __forceinline__ float u_of(const T *su, int r, int dl, const ChannelP
 // Delta of one staged row (rows past the tile end hold delta_raw = -1e4: Delta = 0).
 // In the step-input mode (DT) the row holds the token's x_proj step input s, and
 // delta_raw = s * dt_w[d] (dt_proj); rows past the data hold NaN and give Delta = 0.
-template <typename T, bool DT>
+// With LU the result is in log2 units (bias and dtw prescaled by log2 e).
+template <typename T, bool DT, bool LU = false>
 __device__ __forceinline__ float delta_at(const void *sd, int r, int dl, float bias, float dtw) {
     if constexpr (DT) {
         const float s = static_cast<const float *>(sd)[r];
-        return s == s ? softplus_io<T>(fmaf(s, dtw, bias)) : 0.0f;
+        if constexpr (LU) return s == s ? softplus_l2(fmaf(s, dtw, bias)) : 0.0f;
+        else return s == s ? softplus_io<T>(fmaf(s, dtw, bias)) : 0.0f;
+    } else if constexpr (LU) {
+        return softplus_l2(fmaf(to_f32(static_cast<const T *>(sd)[r * kDC + dl]), kLog2e, bias));
     } else {
         return softplus_io<T>(to_f32(static_cast<const T *>(sd)[r * kDC + dl]) + bias);
     }
@@ -505,6 +547,7 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
                                            int dl, const T *su, const void *sd, const float *sB) {
     constexpr int NP = N / 2;
     constexpr int kCarrySub = ZOH ? kCarryZohSub : vimscan::kCarrySub;
+    constexpr bool LU = lu_mode<T, ZOH>();
 #pragma unroll 1
     for (int sub = 0; sub < kTile / kCarrySub; ++sub) {
         // duv: Delta u (first-order Bbar); with the exact hold, the structured path
@@ -514,7 +557,7 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
 #pragma unroll
         for (int k = 0; k < kCarrySub; ++k) {
             const int r = walk_row<DESC>(sub * kCarrySub + k);
-            const float dt = delta_at<T, DT>(sd, r, dl, prm.bias, prm.dtw);
+            const float dt = delta_at<T, DT, LU>(sd, r, dl, prm.bias, prm.dtw);
             const float u = u_of<T, N, CONV>(su, r, dl, prm);
             if constexpr (!ZOH) {
                 duv[k] = dt * u;
@@ -568,7 +611,7 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
 #pragma unroll
                 for (int q = 0; q < NP; ++q) {
                     const float A0n = __ldg(prm.A + 2 * q), A1n = __ldg(prm.A + 2 * q + 1);
-                    float2 wq = f2(ex2(A0n * kLog2e * Sv[k]), ex2(A1n * kLog2e * Sv[k]));
+                    float2 wq = f2(ex2(A0n * prm.emul * Sv[k]), ex2(A1n * prm.emul * Sv[k]));
                     if constexpr (ZOH)   // gain per state, times n+1 against the staged B / (n+1)
                         wq = mul2(wq, f2(zoh_gain(qv[k], A0n) * (float)(2 * q + 1),
                                          zoh_gain(qv[k], A1n) * (float)(2 * q + 2)));
@@ -593,9 +636,10 @@ __global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMin
     const int nT = (tc + kTile - 1) / kTile;
     // the forward summary of the last chunk and the backward one of the first are unused
     const bool active = (dir == 0 ? (c < p.G - 1) : (c > 0)) && d < p.Di;
+    constexpr bool LU = lu_mode<T, ZOH>();
 
     ChannelParams<N> prm;
-    prm.load(p, dir, d);
+    prm.template load<LU>(p, dir, d);
     const bool fast = __all_sync(0xffffffffu, prm.structured);
 
     // the forward direction walks tiles nT-1 .. 0, the backward one 0 .. nT-1
@@ -641,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMin
         float2 *out = reinterpret_cast<float2 *>(p.hloc + base * N);
 #pragma unroll
         for (int k = 0; k < NP; ++k) out[k] = H[k];
-        p.ssum[base] = Ssum;
+        p.ssum[base] = LU ? Ssum * kLn2 : Ssum;   // natural units
     }
 }
 
@@ -651,8 +695,8 @@ __global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMin
 // One thread per (batch, direction, channel, state).  hloc[b][c][dir][d][n] is
 // replaced by the state entering chunk c in that direction's visiting order:
 // H_in(next) = exp(A_n * Ssum(c)) * H_in(c) + H_loc(c).  Loads run 16 chunks ahead.
-// The last chunk's summary in each direction was never formed: it is read and fed
-// into h after the last carry has been stored, which is harmless.  With fold_reverse
+// The last chunk's summary in each direction was never formed and is not read (the
+// state after the last chunk is not needed).  With fold_reverse
 // each direction is folded from its last chunk to its first (the adjoint of the
 // scan, whose summaries come from adj_carry).
 template <int N>
@@ -678,7 +722,8 @@ __global__ void __launch_bounds__(256) pair_combine(PairArgs p) {
         float loc[kAhead], P[kAhead];
 #pragma unroll
         for (int k = 0; k < kAhead; ++k) {
-            if (k < cnt) {
+            loc[k] = P[k] = 0.0f;
+            if (k < cnt && i0 + k < p.G - 1) {
                 loc[k] = hl[k * hs];
                 P[k] = ss[k * sstep];
             }
@@ -689,7 +734,7 @@ __global__ void __launch_bounds__(256) pair_combine(PairArgs p) {
         for (int k = 0; k < kAhead; ++k) {
             if (k < cnt) {
                 hl[k * hs] = h;                 // the state entering this chunk
-                h = fmaf(P[k], h, loc[k]);      // (unused after the last chunk)
+                h = fmaf(P[k], h, loc[k]);      // (zero after the last chunk, unused)
             }
         }
         hl += kAhead * hs;
@@ -720,11 +765,18 @@ __device__ __forceinline__ void add_f32(float (&acc)[V], const float *src) {
 // them.  Rows past the tile's end are no-op tokens.  The output of each token goes
 // to the chunk's fp32 partial buffer: stored on the tile's first visit, added on the
 // second (rows past the end only touch unread rows of the buffer).
+//
+// With structured A and the first-order Bbar, the scaled state g = h / du (du = Delta
+// u, |du| kept at or above 1e-20) can be run instead of h (VIMSCAN_GF):
+//     g_t = (Abar_t r_t) g_(t-1) + B_t,  r_t = du_(t-1) / du_t,  y_t = du_t C_t.g_t + D u_t,
+// which drops the drive multiply du B_n of every state; dprev carries du_(t-1).
 template <typename T, int N, bool FAST, bool DESC, bool CONV, bool ZOH, bool DT>
-__device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], const ChannelParams<N> &prm,
-                                          int dl, const T *su, const void *sd, const float *sB,
-                                          const float *sC, float *ypart) {
+__device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], float &dprev,
+                                          const ChannelParams<N> &prm, int dl, const T *su, const void *sd,
+                                          const float *sB, const float *sC, float *ypart) {
     constexpr int NP = N / 2;
+    constexpr bool LU = lu_mode<T, ZOH>();
+    constexpr bool GF = VIMSCAN_GF && FAST && !ZOH;
 #pragma unroll 1
     for (int sub = 0; sub < kTile / kSub; ++sub) {
         // qv: q = exp(Delta A_0) (structured A) or Delta (general A); duv: Delta u, or
@@ -733,7 +785,7 @@ __device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], const
 #pragma unroll
         for (int k = 0; k < kSub; ++k) {
             const int r = walk_row<DESC>(sub * kSub + k);
-            const float dt = delta_at<T, DT>(sd, r, dl, prm.bias, prm.dtw);
+            const float dt = delta_at<T, DT, LU>(sd, r, dl, prm.bias, prm.dtw);
             uv[k] = u_of<T, N, CONV>(su, r, dl, prm);
             qv[k] = FAST ? ex2(dt * prm.A0) : dt;
             if constexpr (ZOH && FAST)
@@ -753,6 +805,14 @@ __device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], const
             const float q = qv[k];
             float2 a = FAST ? f2(q, q * q) : f2(0.f, 0.f);
             const float2 step = FAST ? f2(a.y, a.y) : f2(0.f, 0.f);
+            float ysc = 1.0f;
+            if constexpr (GF) {
+                const float dv = clamp_du(duv[k]);
+                const float rr = dprev * rcp(dv);
+                dprev = dv;
+                a = mul2(a, f2(rr, rr));
+                ysc = dv;
+            }
             // exact hold, structured A: Bbar_n u = kappa u S_n B_n / (n+1) with
             // S_n = 1 + q + ... + q^n and B staged divided by n+1; KS = kappa u S for two
             // states at a time, KS_(n+2) = KS_n + kappa u (1+q) q^(n+1)
@@ -774,7 +834,11 @@ __device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], const
                 for (int e = 0; e < 2 && qq + e < NP; ++e) {
                     const int qi = qq + e;
                     float2 aq, drive;
-                    if constexpr (FAST) {
+                    if constexpr (GF) {
+                        aq = a;
+                        a = mul2(a, step);
+                        drive = Bp[e];
+                    } else if constexpr (FAST) {
                         aq = a;
                         a = mul2(a, step);
                         if constexpr (ZOH) {
@@ -785,7 +849,7 @@ __device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], const
                         }
                     } else {
                         const float A0n = __ldg(prm.A + 2 * qi), A1n = __ldg(prm.A + 2 * qi + 1);
-                        aq = f2(ex2(q * A0n * kLog2e), ex2(q * A1n * kLog2e));
+                        aq = f2(ex2(q * A0n * prm.emul), ex2(q * A1n * prm.emul));
                         if constexpr (ZOH)   // gain per state, times n+1 against the staged B / (n+1)
                             drive = mul2(mul2(f2(zoh_gain(q, A0n) * (float)(2 * qi + 1),
                                                  zoh_gain(q, A1n) * (float)(2 * qi + 2)),
@@ -800,7 +864,7 @@ __device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], const
                 }
             }
             const float2 ys = __fadd2_rn(y0, y1);
-            const float yv = fmaf(prm.D, uv[k], ys.x + ys.y);
+            const float yv = fmaf(ysc, ys.x + ys.y, prm.D * uv[k]);
             float *py = ypart + r * kDC;
             *py = second ? *py + yv : yv;
         }
@@ -922,7 +986,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
     const int nT = (tc + kTile - 1) / kTile;
 
     ChannelParams<N> prm;
-    prm.load(p, dir, d);
+    prm.template load<lu_mode<T, ZOH>()>(p, dir, d);
     const bool fast = __all_sync(0xffffffffu, prm.structured);
 
     Stager<T, N, VEC_BC, CONV, ZOH, DT> st(p, b, t0, tc, d0);
@@ -936,6 +1000,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
     float2 h[NP];
 #pragma unroll
     for (int k = 0; k < NP; ++k) h[k] = f2(0.f, 0.f);
+    float dprev = 1.0f;   // du before the chunk's first token (scaled state: g = h_in)
     if (p.G > 1) cudaGridDependencySynchronize();
     if (p.G > 1 && (dir == 0 ? c > 0 : c < p.G - 1) && prm.valid) {
         const size_t base = (((size_t)b * p.G + c) * 2 + dir) * p.Di + d;
@@ -969,11 +1034,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
             const float *sB = S::bc(cur, dir, 0), *sC = S::bc(cur, dir, 1);
             const bool second = twice > 0;
             if (dir == 0) {
-                if (fast) main_tile<T, N, true, false, CONV, ZOH, DT>(second, h, prm, dl, su, sd, sB, sC, ypart);
-                else main_tile<T, N, false, false, CONV, ZOH, DT>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                if (fast) main_tile<T, N, true, false, CONV, ZOH, DT>(second, h, dprev, prm, dl, su, sd, sB, sC, ypart);
+                else main_tile<T, N, false, false, CONV, ZOH, DT>(second, h, dprev, prm, dl, su, sd, sB, sC, ypart);
             } else {
-                if (fast) main_tile<T, N, true, true, CONV, ZOH, DT>(second, h, prm, dl, su, sd, sB, sC, ypart);
-                else main_tile<T, N, false, true, CONV, ZOH, DT>(second, h, prm, dl, su, sd, sB, sC, ypart);
+                if (fast) main_tile<T, N, true, true, CONV, ZOH, DT>(second, h, dprev, prm, dl, su, sd, sB, sC, ypart);
+                else main_tile<T, N, false, true, CONV, ZOH, DT>(second, h, dprev, prm, dl, su, sd, sB, sC, ypart);
             }
         }
         if (s + 1 < nT) {
