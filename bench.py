@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--workload", default="vim_tiny_1024px_bf16")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the forward timing of the other workloads (other_configs)")
     ap.add_argument("--conv", action="store_true",
                     help="Vim workloads: time the scan with the fused kernel-3 convolution + SiLU front")
     ap.add_argument("--zoh", action="store_true",
@@ -158,7 +160,7 @@ class ClockSampler:
         0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, index, period=0.002):
+    def __init__(self, index, period=0.0005):
         self.ok = False
         try:
             import pynvml
@@ -329,6 +331,80 @@ def reference_arm(args, w):
         "e2e": {"value": value, "unit": "tok*ch/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def time_forward(w, dev, steps, warmup=3):
+    """Device time of the plain forward scan of workload ``w`` (its own seeded inputs,
+    rotating copies larger than L2), with per-kernel times from the events entry
+    point.  Returns the numbers one line of ``other_configs`` reports."""
+    import torch
+
+    from vision_mamba_selective_b200 import vimscan as vs
+    from vision_mamba_selective_b200 import workloads as wl
+
+    host = wl.make_inputs(w)
+    keys = ["u", "delta", "z", "B", "C"]
+    set_bytes = sum(host[k].numel() * host[k].element_size() for k in keys) + wl.output_bytes(w)
+    nsets = max(2, math.ceil(2.2 * L2_BYTES / set_bytes))
+    params = {k: host[k].to(dev) for k in ("A", "D", "delta_bias")}
+    sets = []
+    for _ in range(nsets):
+        s = {k: host[k].to(dev) for k in keys}
+        s["y"] = torch.empty_like(s["u"])
+        sets.append(s)
+    which = 0 if w.kind == "vim" else 1
+    ws = torch.empty(max(1, vs.vim_scan_workspace_bytes(which, w.batch, w.L if w.kind == "vim" else w.H, w.W,
+                                                          w.channels, w.d_state)), dtype=torch.uint8, device=dev)
+    fn = vs.vim_scan_bidir if w.kind == "vim" else vs.vmamba_cross_scan4
+    pairs = 1 if w.kind == "vim" else 2
+
+    def step(i, events=None):
+        s = sets[i % nsets]
+        fn(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"], params["delta_bias"], y=s["y"],
+           workspace=ws, events=events)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(1 + 3 * pairs)] for _ in range(steps)]
+    for i in range(steps):
+        step(i, evs[i])
+    torch.cuda.synchronize()
+    names = ["pair_carry", "pair_combine", "pair_main"]
+    kernel_ms = {}
+    for p in range(pairs):
+        for k in range(3):
+            a = 1 + 3 * p + k
+            t = sum(evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(steps)) / steps
+            kernel_ms[f"{names[k]}[{p}]" if pairs > 1 else names[k]] = t
+    nbytes, ops = algorithmic(w)
+    pk = peaks()
+    peak_ops = SMS * FP32_LANES_PER_SM * pk["sm_max_mhz"] * 1e6
+    main_ms = sum(v for k, v in kernel_ms.items() if k.startswith("pair_main"))
+    return {"ms_per_step": ms, "tok_ch_per_s": w.tok_ch / (ms * 1e-3),
+            "hbm_frac_whole_step": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+            "fp32_frac_pair_main": ops / (main_ms * 1e-3) / peak_ops,
+            "fp32_frac_whole_step": ops / (ms * 1e-3) / peak_ops,
+            "kernel_ms": kernel_ms, "steps": steps, "io_dtype": w.dtype,
+            "shape": {"batch": w.batch, "tokens": w.tokens, "channels": w.channels, "d_state": w.d_state}}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 def workload_name(w, args):
@@ -544,10 +620,13 @@ def main():
     clocks = clk.summary()
     peak_ops = SMS * FP32_LANES_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e12
     achieved_ops = ops / (main_ms * 1e-3) / 1e12
+    traffic = None if (args.bwd or args.conv or args.zoh or args.block) else profiled_traffic(w)
     roofline = {
         "bound": "alu", "kernel": main_name, "achieved": achieved_ops, "peak": peak_ops,
         "unit": "Tops/s", "frac": achieved_ops / peak_ops,
-        "traffic": None if (args.bwd or args.conv or args.zoh or args.block) else profiled_traffic(w),
+        "traffic": traffic,
+        "traffic_source": ("ncu capture committed under profiles/ (same kernel source fingerprint), not "
+                           "measured in this run" if traffic is not None else None),
         "algorithmic_bytes": nbytes,
         "ops_per_launch": ops, "ms_per_launch": main_ms,
         "peak_basis": f"{SMS} SMs x {FP32_LANES_PER_SM} FP32 lanes x {pk['sm_max_mhz']:.0f} MHz",
@@ -568,6 +647,16 @@ def main():
                       "achieved_gbs": pb / (pms * 1e-3) / 1e9, "peak_gbs": pk["hbm_gbs"],
                       "frac": pb / (pms * 1e-3) / 1e9 / pk["hbm_gbs"]}
 
+    # ---- the other workloads of the target (forward scan only), timed the same way ---
+    others = None
+    if not (args.no_other_configs or args.bwd or args.conv or args.zoh or args.block):
+        others = {}
+        for ow in wl.WORKLOADS:
+            if ow.name == w.name:
+                continue
+            others[ow.name] = time_forward(ow, dev, steps=max(10, min(args.steps, 50)))
+            torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         s, x, cores = oracle_sample(w, CPU_SECONDS, conv=args.conv, bwd=args.bwd, block=args.block)
@@ -577,10 +666,21 @@ def main():
         while runs == 0 or sec < CPU_SECONDS:
             sec += run_oracle(s, x, cores, args.zoh)
             runs += 1
+        # the same oracle on one host thread, on a sample of about a quarter of the time
+        s1, x1, _ = oracle_sample(w, CPU_SECONDS / 4 / max(1, cores) * 1.0, conv=args.conv, bwd=args.bwd,
+                                  block=args.block)
+        sec1, runs1 = 0.0, 0
+        while runs1 == 0 or sec1 < CPU_SECONDS / 4:
+            sec1 += run_oracle(s1, x1, 1, args.zoh)
+            runs1 += 1
         cpu = {"value": runs * s.tok_ch / sec, "unit": "tok*ch/s", "cores": cores, "kind": "oracle",
+               "cpu_model": cpu_model(),
                "sample": f"{s.batch} of {w.batch} batch items x {s.channels} of {w.channels} channels "
                          f"at the full {w.tokens} tokens ({s.tok_ch} token-channels), {runs} run(s), "
-                         f"fp64, {sec:.2f} s"}
+                         f"fp64, {sec:.2f} s",
+               "single_thread": {"value": runs1 * s1.tok_ch / sec1, "unit": "tok*ch/s", "cores": 1,
+                                 "sample": f"{s1.batch} batch items x {s1.channels} channels at the full "
+                                           f"{w.tokens} tokens, {runs1} run(s), fp64, {sec1:.2f} s"}}
 
     if rank == 0:
         line = {
@@ -592,7 +692,9 @@ def main():
             "config": {"workload": workload_name(w, args), "batch_per_gpu": w.batch, "tokens": w.tokens,
                        "channels": w.channels, "d_state": w.d_state, "io_dtype": w.dtype,
                        "parallelism": f"replicas x{world} (batch shards, no collective)",
-                       "l2": f"{nsets} rotating input sets of {set_bytes / 1e6:.0f} MB (> 126 MB L2)"},
+                       "l2": f"{nsets} rotating input sets of {set_bytes / 1e6:.0f} MB each, "
+                             f"{nsets * set_bytes / 1e6:.0f} MB in all (L2: {L2_BYTES / 1e6:.0f} MB): each step "
+                             f"reads a set written {nsets - 1} steps earlier"},
             "hbm_gbs": roofline["hbm_gbs_whole_step"], "hbm_frac": roofline["hbm_frac_whole_step"],
             "kernel_ms": per_kernel,
             "roofline": roofline,
@@ -602,6 +704,7 @@ def main():
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
+            "other_configs": others,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
