@@ -9,11 +9,16 @@
 #include "bwd_kernels.cuh"
 #include "launch.cuh"
 
+#ifndef VIMSCAN_BWD_CLUSTER
+#define VIMSCAN_BWD_CLUSTER 1
+#endif
+
 namespace vimscan {
 namespace {
 
 struct BwdPlan {
     int G, nblk, nsets;
+    int cl, ncol;   // cluster size along the channel blocks, and the partials' columns
     size_t off_hloc, off_ssum, off_gloc, off_gsum, off_par, off_dBp, off_dCp, off_tmp, total;
 };
 
@@ -23,6 +28,12 @@ BwdPlan bwd_plan(int batch, int L, int Di, int N, int separate_bc) {
     const int ch = N >= 8 ? BwdShape<16>::CH : BwdShape<4>::CH;   // channels per bwd_main CTA
     pl.nblk = (Di + ch - 1) / ch;
     pl.nsets = separate_bc ? 2 : 1;
+    // channel blocks reduce their dB/dC terms in clusters of up to 8 (whole clusters of
+    // the grid; the chunk's 32 rows split evenly over the ranks)
+    pl.cl = 1;
+    for (int c = VIMSCAN_BWD_CLUSTER; c > 1; c /= 2)
+        if (pl.nblk % c == 0 && kBwdChunk % c == 0) { pl.cl = c; break; }
+    pl.ncol = pl.nblk / pl.cl;
     const size_t units = (size_t)batch * pl.G * 2 * Di;      // (b, chunk, dir, channel)
     const size_t cols = (size_t)2 * Di * (N + 2);        // [dA | dD | d delta_bias]
     size_t o = 0;
@@ -32,8 +43,8 @@ BwdPlan bwd_plan(int batch, int L, int Di, int N, int separate_bc) {
     pl.off_gloc = take(units * N * 4);
     pl.off_gsum = take(units * 4);
     pl.off_par = take(units * (N + 2) * 4);
-    pl.off_dBp = take((size_t)pl.nsets * batch * L * pl.nblk * N * 4);
-    pl.off_dCp = take((size_t)pl.nsets * batch * L * pl.nblk * N * 4);
+    pl.off_dBp = take((size_t)pl.nsets * batch * L * pl.ncol * N * 4);
+    pl.off_dCp = take((size_t)pl.nsets * batch * L * pl.ncol * N * 4);
     pl.off_tmp = take((size_t)kReduceParts * cols * 4);
     pl.total = o;
     return pl;
@@ -95,14 +106,33 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
     if (cudaFuncSetAttribute(bwd_main<T, N, ZOH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
         return VIM_ERR_CUDA;
     const dim3 gm(a.nblk, a.G, a.batch);
-    if (a.G > 1) {
-        // a programmatic dependent of the adjoint fold: its launch and the staging of
-        // the first CTAs overlap the fold's end; it waits for the fold before it reads
-        // the carries
-        if (launch_dependent(bwd_main<T, N, ZOH>, gm, dim3(BwdShape<N>::kThr), sm, stream, a) != cudaSuccess)
-            return VIM_ERR_CUDA;
-    } else {
-        bwd_main<T, N, ZOH><<<gm, BwdShape<N>::kThr, sm, stream>>>(a);
+    {
+        // with several chunks, a programmatic dependent of the adjoint fold: its launch
+        // and the staging of the first CTAs overlap the fold's end; it waits for the
+        // fold before it reads the carries.  Clusters of a.cl CTAs along the channel
+        // blocks reduce the dB/dC terms on chip.
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = gm;
+        cfg.blockDim = dim3(BwdShape<N>::kThr);
+        cfg.dynamicSmemBytes = sm;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[2];
+        int na = 0;
+        if (a.cl > 1) {
+            attr[na].id = cudaLaunchAttributeClusterDimension;
+            attr[na].val.clusterDim.x = (unsigned)a.cl;
+            attr[na].val.clusterDim.y = 1;
+            attr[na].val.clusterDim.z = 1;
+            ++na;
+        }
+        if (a.G > 1 && VIMSCAN_PDL) {
+            attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[na].val.programmaticStreamSerializationAllowed = 1;
+            ++na;
+        }
+        cfg.attrs = attr;
+        cfg.numAttrs = na;
+        if (cudaLaunchKernelEx(&cfg, bwd_main<T, N, ZOH>, a) != cudaSuccess) return VIM_ERR_CUDA;
     }
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     if (!rec(ev, 2, stream)) return VIM_ERR_CUDA;
@@ -110,8 +140,8 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
     const int rows = a.batch * a.L;
     for (int k = 0; k < sets; ++k) {
         const unsigned blocks = (unsigned)(((int64_t)rows * N + 255) / 256);
-        bwd_reduce_bc<N><<<blocks, 256, 0, stream>>>(a.dB_part[k], dB_out[k], rows, a.nblk);
-        bwd_reduce_bc<N><<<blocks, 256, 0, stream>>>(a.dC_part[k], dC_out[k], rows, a.nblk);
+        bwd_reduce_bc<N><<<blocks, 256, 0, stream>>>(a.dB_part[k], dB_out[k], rows, a.ncol);
+        bwd_reduce_bc<N><<<blocks, 256, 0, stream>>>(a.dC_part[k], dC_out[k], rows, a.ncol);
         if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     }
     const int prow = a.batch * a.G;
@@ -199,7 +229,7 @@ vim_status vim_scan_bidir_bwd_ex(const void *u, const void *delta, const void *z
     a.C[1] = static_cast<const char *>(C) + bc_dir_stride * (int64_t)es;
     a.A = A; a.D = D; a.bias = delta_bias;
     a.du = du; a.ddelta = ddelta; a.dz = dz;
-    const size_t set_elems = (size_t)batch * L * pl.nblk * d_state;
+    const size_t set_elems = (size_t)batch * L * pl.ncol * d_state;
     a.dB_part[0] = reinterpret_cast<float *>(ws + pl.off_dBp);
     a.dC_part[0] = reinterpret_cast<float *>(ws + pl.off_dCp);
     a.dB_part[1] = separate ? a.dB_part[0] + set_elems : a.dB_part[0];
@@ -208,7 +238,7 @@ vim_status vim_scan_bidir_bwd_ex(const void *u, const void *delta, const void *z
     a.hin = reinterpret_cast<const float *>(ws + pl.off_hloc);
     a.gloc = reinterpret_cast<float *>(ws + pl.off_gloc);
     a.gsum = reinterpret_cast<float *>(ws + pl.off_gsum);
-    a.batch = batch; a.L = L; a.Di = d_inner; a.G = pl.G; a.nblk = pl.nblk;
+    a.batch = batch; a.L = L; a.Di = d_inner; a.G = pl.G; a.nblk = pl.nblk; a.cl = pl.cl; a.ncol = pl.ncol;
     a.separate_bc = separate;
     set_vector_flags(a, dt, d_state);
 
@@ -298,7 +328,7 @@ vim_status vmamba_cross_scan4_bwd_ex(const void *u, const void *delta, const voi
     char *ws = static_cast<char *>(workspace);
     float *acc = reinterpret_cast<float *>(ws + pl.total);
     const size_t bc = (size_t)batch * L * d_state;               // elements per direction of B, C
-    const size_t set_elems = (size_t)batch * L * pl.nblk * d_state;
+    const size_t set_elems = (size_t)batch * L * pl.ncol * d_state;
 
     vim_status rc = VIM_OK;
     for (int pair = 0; pair < 2 && rc == VIM_OK; ++pair) {
@@ -321,7 +351,7 @@ vim_status vmamba_cross_scan4_bwd_ex(const void *u, const void *delta, const voi
         a.hin = reinterpret_cast<const float *>(ws + pl.off_hloc);
         a.gloc = reinterpret_cast<float *>(ws + pl.off_gloc);
         a.gsum = reinterpret_cast<float *>(ws + pl.off_gsum);
-        a.batch = batch; a.L = L; a.Di = channels; a.G = pl.G; a.nblk = pl.nblk;
+        a.batch = batch; a.L = L; a.Di = channels; a.G = pl.G; a.nblk = pl.nblk; a.cl = pl.cl; a.ncol = pl.ncol;
         a.separate_bc = 1;
         set_vector_flags(a, dt, d_state);
         a.order = pair; a.H = H; a.W = W;

@@ -30,6 +30,8 @@
 // bit for bit.
 #pragma once
 
+#include <cooperative_groups.h>
+
 #include "scan_kernels.cuh"
 
 namespace vimscan {
@@ -54,13 +56,15 @@ struct BwdArgs {
     const void *B[2], *C[2];            // per direction [batch, L, N]
     const float *A, *D, *bias;          // [2][Di][N], [2][Di], [2][Di]
     void *du, *ddelta, *dz;             // [batch, L, Di] (dz null when z is)
-    float *dB_part[2], *dC_part[2];     // [batch][L][nblk][N] per B/C set ([1] = [0] when shared)
+    float *dB_part[2], *dC_part[2];     // [batch][L][ncol][N] per B/C set ([1] = [0] when shared)
     float *par;                         // per-chunk sums over tokens, one row per (batch, chunk):
                                         // [dA: 2*Di*N | dD: 2*Di | d delta_bias: 2*Di]
     const float *hin;                   // [batch][G][2][Di][N] h entering each chunk (direction order)
     float *gloc;                        // [batch][G][2][Di][N] adjoint summaries, then adjoint entering
     float *gsum;                        // [batch][G][2][Di] chunk Delta sums
     int batch, L, Di, G, nblk;
+    int cl;                             // CTAs per thread-block cluster along the channel blocks (1: none)
+    int ncol;                           // columns of the dB/dC partials: nblk / cl
     int separate_bc;
     int vec_io;                         // u, delta, dout, z, du, d delta_raw, dz allow vector access
     int vec_bc;                         // B and C rows move as 16-byte vectors
@@ -673,14 +677,54 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
 }
 
 // The CTA's per-token sums over its channels of the dB (or dC) terms, from the
-// per-direction, per-warp slots, into part[set][b][t][blk][n]: the two directions
-// add into one set when B and C are shared.  Four states at a time.
+// per-direction, per-warp slots, into part[set][b][t][col][n]: the two directions
+// add into one set when B and C are shared.  Four states at a time.  In a cluster of
+// p.cl CTAs (consecutive channel blocks), the CTAs first wait for one another; then
+// CTA rank r sums rows r*TC/cl .. of every CTA's slots (read through distributed
+// shared memory, in rank order) into column blk / cl, and the CTAs wait again before
+// any of them reuses or leaves its slots.  The order of every sum is fixed.
 template <int N>
 __device__ __forceinline__ void store_bc_part(const BwdArgs &p, const float *red, float *const (&part)[2], int b,
                                               int t0, int tc, int blk) {
     using SH = BwdShape<N>;
     constexpr int TC = SH::TC, V = N % 4 == 0 ? 4 : 2;
     const int nsets = p.separate_bc ? 2 : 1;
+    if (p.cl > 1) {
+        namespace cg = cooperative_groups;
+        cg::cluster_group cluster = cg::this_cluster();
+        cluster.sync();
+        const int rank = (int)cluster.block_rank(), rows = TC / p.cl, r0 = rank * rows;
+        for (int li = threadIdx.x; li < nsets * rows * (N / V); li += SH::kThr) {
+            const int k = li / (rows * (N / V)), r = r0 + (li / (N / V)) % rows, n = (li % (N / V)) * V;
+            if (r >= tc) continue;
+            float acc[V];
+#pragma unroll
+            for (int e = 0; e < V; ++e) acc[e] = 0.0f;
+            for (int pr = 0; pr < p.cl; ++pr) {
+                const float *peer = cluster.map_shared_rank(red, pr);
+#pragma unroll
+                for (int dir = 0; dir < 2; ++dir) {
+                    if (p.separate_bc && dir != k) continue;
+#pragma unroll
+                    for (int w = 0; w < SH::WPD; ++w) {
+                        const float *src = peer + ((dir * SH::WPD + w) * TC + r) * N + n;
+                        if constexpr (V == 4) {
+                            const float4 v4 = *reinterpret_cast<const float4 *>(src);
+                            acc[0] += v4.x; acc[1] += v4.y; acc[2] += v4.z; acc[3] += v4.w;
+                        } else {
+                            const float2 v2 = *reinterpret_cast<const float2 *>(src);
+                            acc[0] += v2.x; acc[1] += v2.y;
+                        }
+                    }
+                }
+            }
+            float *dst = part[k] + (((size_t)b * p.L + bpos(p, t0 + r)) * p.ncol + blk / p.cl) * N + n;
+            if constexpr (V == 4) *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            else *reinterpret_cast<float2 *>(dst) = f2(acc[0], acc[1]);
+        }
+        cluster.sync();
+        return;
+    }
     for (int li = threadIdx.x; li < nsets * TC * (N / V); li += SH::kThr) {
         const int k = li / (TC * (N / V)), r = (li / (N / V)) % TC, n = (li % (N / V)) * V;
         if (r >= tc) continue;
@@ -697,7 +741,7 @@ __device__ __forceinline__ void store_bc_part(const BwdArgs &p, const float *red
                 for (int e = 0; e < V; ++e) acc[e] += src[e];
             }
         }
-        float *dst = part[k] + (((size_t)b * p.L + bpos(p, t0 + r)) * p.nblk + blk) * N + n;
+        float *dst = part[k] + (((size_t)b * p.L + bpos(p, t0 + r)) * p.ncol + blk) * N + n;
         if constexpr (V == 4) *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
         else *reinterpret_cast<float2 *>(dst) = f2(acc[0], acc[1]);
     }
@@ -880,7 +924,7 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     store_bc_part<N>(p, sm.red, p.dB_part, b, t0, tc, blk);
 }
 
-// dB / dC: sum of the per-CTA partials, [batch][L][nblk][N] -> [batch][L][N]
+// dB / dC: sum of the per-CTA (or per-cluster) partials, [batch][L][ncol][N] -> [batch][L][N]
 template <int N>
 __global__ void __launch_bounds__(256) bwd_reduce_bc(const float *part, float *out, int rows, int nblk) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // (row, n)
