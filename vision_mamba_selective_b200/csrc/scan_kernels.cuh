@@ -301,6 +301,7 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool va
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n));
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::); }
 
 // B and C rows can be moved as 16-byte vectors when a row is a whole number of them
@@ -542,83 +543,104 @@ __device__ __forceinline__ float delta_at(const void *sd, int r, int dl, float b
 // Delta summed over the tokens the direction visits after s inside the chunk.  With
 // A_n = (n+1) A_0 the weights are powers of w = exp(A_0 S_s), built by one multiply
 // per state.
+// The h-independent values of sub-batch `sub` of a summary walk (see carry_tile); S
+// enters as the Delta walked before the sub-batch, and the Delta after it is returned.
+template <typename T, int N, bool FAST, bool DESC, bool CONV, bool ZOH, bool DT, int KS>
+__device__ __forceinline__ float carry_form(int sub, float S, float (&Sv)[KS], float (&duv)[KS],
+                                            float (&qv)[ZOH ? KS : 1], const ChannelParams<N> &prm, int dl,
+                                            const T *su, const void *sd) {
+    constexpr int kCarrySub = KS;
+    constexpr bool LU = lu_mode<T, ZOH>();
+    // duv: Delta u (first-order Bbar); with the exact hold, the structured path
+    // keeps kappa u with kappa = expm1(Delta A_0) / A_0 and q = exp(Delta A_0), the
+    // general path u and Delta
+#pragma unroll
+    for (int k = 0; k < kCarrySub; ++k) {
+        const int r = walk_row<DESC>(sub * kCarrySub + k);
+        const float dt = delta_at<T, DT, LU>(sd, r, dl, prm.bias, prm.dtw);
+        const float u = u_of<T, N, CONV>(su, r, dl, prm);
+        if constexpr (!ZOH) {
+            duv[k] = dt * u;
+        } else if constexpr (FAST) {
+            const float q = ex2(dt * prm.A0);
+            const float em1 = expm1_acc(dt * prm.a0, q);
+            duv[k] = u * (prm.a0 != 0.0f ? em1 * prm.inv_a0 : dt);
+            qv[k] = q;
+        } else {
+            duv[k] = u;
+            qv[k] = dt;
+        }
+        Sv[k] = S;             // Delta of the tokens walked before this one
+        S += dt;
+    }
+    return S;
+}
+
+// The summary terms of the tokens of sub-batch `sub`, from their formed values.
+template <typename T, int N, bool FAST, bool DESC, bool CONV, bool ZOH, bool DT, int KS>
+__device__ __forceinline__ void carry_acc(int sub, const float (&Sv)[KS], const float (&duv)[KS],
+                                          const float (&qv)[ZOH ? KS : 1], float2 (&H)[N / 2],
+                                          const ChannelParams<N> &prm, const float *sB) {
+    constexpr int NP = N / 2;
+    constexpr int kCarrySub = KS;
+#pragma unroll
+    for (int k = 0; k < kCarrySub; ++k) {
+        const int r = walk_row<DESC>(sub * kCarrySub + k);
+        float2 Bv[NP];
+        load_row<NP>(sB + r * N, Bv);
+        if constexpr (FAST && !ZOH) {
+            const float w = ex2(prm.A0 * Sv[k]);
+            const float x0 = w * duv[k];
+            float2 x = f2(x0, x0 * w);
+            const float2 w2 = f2(w * w, w * w);
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                H[q] = fma2(x, Bv[q], H[q]);
+                x = mul2(x, w2);
+            }
+        } else if constexpr (FAST) {
+            // exact hold: state n gets w^(n+1) kappa u S_n B_n / (n+1) (B is staged
+            // divided by n+1), S_n = 1 + q + ... + q^n.  W_n = w^(n+1) kappa u S_n
+            // runs two states at a time: W_(n+2) = w^2 W_n + Q_n with
+            // Q_n = w^2 kappa u (1+q) (wq)^(n+1).
+            const float w = ex2(prm.A0 * Sv[k]);
+            const float q = qv[k], ku = duv[k];
+            const float c = ku * (1.0f + q);
+            const float ww = w * w, wq = w * q, wqwq = wq * wq;
+            float2 Wn = f2(ku * w, c * ww);
+            float2 Q = f2(ww * c * wq, ww * c * wqwq);
+            const float2 w2 = f2(ww, ww), wq2 = f2(wqwq, wqwq);
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                H[j] = fma2(Wn, Bv[j], H[j]);
+                Wn = fma2(w2, Wn, Q);
+                Q = mul2(Q, wq2);
+            }
+        } else {
+            const float2 du2 = f2(duv[k], duv[k]);
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                const float A0n = __ldg(prm.A + 2 * q), A1n = __ldg(prm.A + 2 * q + 1);
+                float2 wq = f2(ex2(A0n * prm.emul * Sv[k]), ex2(A1n * prm.emul * Sv[k]));
+                if constexpr (ZOH)   // gain per state, times n+1 against the staged B / (n+1)
+                    wq = mul2(wq, f2(zoh_gain(qv[k], A0n) * (float)(2 * q + 1),
+                                     zoh_gain(qv[k], A1n) * (float)(2 * q + 2)));
+                H[q] = fma2(mul2(wq, du2), Bv[q], H[q]);
+            }
+        }
+    }
+}
+
 template <typename T, int N, bool FAST, bool DESC, bool CONV, bool ZOH, bool DT>
 __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, const ChannelParams<N> &prm,
                                            int dl, const T *su, const void *sd, const float *sB) {
-    constexpr int NP = N / 2;
-    constexpr int kCarrySub = ZOH ? kCarryZohSub : vimscan::kCarrySub;
-    constexpr bool LU = lu_mode<T, ZOH>();
+    constexpr int KS = ZOH ? kCarryZohSub : vimscan::kCarrySub;
+    constexpr int kNSub = kTile / KS;
 #pragma unroll 1
-    for (int sub = 0; sub < kTile / kCarrySub; ++sub) {
-        // duv: Delta u (first-order Bbar); with the exact hold, the structured path
-        // keeps kappa u with kappa = expm1(Delta A_0) / A_0 and q = exp(Delta A_0), the
-        // general path u and Delta
-        float Sv[kCarrySub], duv[kCarrySub], qv[ZOH ? kCarrySub : 1];
-#pragma unroll
-        for (int k = 0; k < kCarrySub; ++k) {
-            const int r = walk_row<DESC>(sub * kCarrySub + k);
-            const float dt = delta_at<T, DT, LU>(sd, r, dl, prm.bias, prm.dtw);
-            const float u = u_of<T, N, CONV>(su, r, dl, prm);
-            if constexpr (!ZOH) {
-                duv[k] = dt * u;
-            } else if constexpr (FAST) {
-                const float q = ex2(dt * prm.A0);
-                const float em1 = expm1_acc(dt * prm.a0, q);
-                duv[k] = u * (prm.a0 != 0.0f ? em1 * prm.inv_a0 : dt);
-                qv[k] = q;
-            } else {
-                duv[k] = u;
-                qv[k] = dt;
-            }
-            Sv[k] = Ssum;          // Delta of the tokens walked before this one
-            Ssum += dt;
-        }
-#pragma unroll
-        for (int k = 0; k < kCarrySub; ++k) {
-            const int r = walk_row<DESC>(sub * kCarrySub + k);
-            float2 Bv[NP];
-            load_row<NP>(sB + r * N, Bv);
-            if constexpr (FAST && !ZOH) {
-                const float w = ex2(prm.A0 * Sv[k]);
-                const float x0 = w * duv[k];
-                float2 x = f2(x0, x0 * w);
-                const float2 w2 = f2(w * w, w * w);
-#pragma unroll
-                for (int q = 0; q < NP; ++q) {
-                    H[q] = fma2(x, Bv[q], H[q]);
-                    x = mul2(x, w2);
-                }
-            } else if constexpr (FAST) {
-                // exact hold: state n gets w^(n+1) kappa u S_n B_n / (n+1) (B is staged
-                // divided by n+1), S_n = 1 + q + ... + q^n.  W_n = w^(n+1) kappa u S_n
-                // runs two states at a time: W_(n+2) = w^2 W_n + Q_n with
-                // Q_n = w^2 kappa u (1+q) (wq)^(n+1).
-                const float w = ex2(prm.A0 * Sv[k]);
-                const float q = qv[k], ku = duv[k];
-                const float c = ku * (1.0f + q);
-                const float ww = w * w, wq = w * q, wqwq = wq * wq;
-                float2 Wn = f2(ku * w, c * ww);
-                float2 Q = f2(ww * c * wq, ww * c * wqwq);
-                const float2 w2 = f2(ww, ww), wq2 = f2(wqwq, wqwq);
-#pragma unroll
-                for (int j = 0; j < NP; ++j) {
-                    H[j] = fma2(Wn, Bv[j], H[j]);
-                    Wn = fma2(w2, Wn, Q);
-                    Q = mul2(Q, wq2);
-                }
-            } else {
-                const float2 du2 = f2(duv[k], duv[k]);
-#pragma unroll
-                for (int q = 0; q < NP; ++q) {
-                    const float A0n = __ldg(prm.A + 2 * q), A1n = __ldg(prm.A + 2 * q + 1);
-                    float2 wq = f2(ex2(A0n * prm.emul * Sv[k]), ex2(A1n * prm.emul * Sv[k]));
-                    if constexpr (ZOH)   // gain per state, times n+1 against the staged B / (n+1)
-                        wq = mul2(wq, f2(zoh_gain(qv[k], A0n) * (float)(2 * q + 1),
-                                         zoh_gain(qv[k], A1n) * (float)(2 * q + 2)));
-                    H[q] = fma2(mul2(wq, du2), Bv[q], H[q]);
-                }
-            }
-        }
+    for (int sub = 0; sub < kNSub; ++sub) {
+        float Sv[KS], duv[KS], qv[ZOH ? KS : 1];
+        Ssum = carry_form<T, N, FAST, DESC, CONV, ZOH, DT, KS>(sub, Ssum, Sv, duv, qv, prm, dl, su, sd);
+        carry_acc<T, N, FAST, DESC, CONV, ZOH, DT, KS>(sub, Sv, duv, qv, H, prm, sB);
     }
 }
 
@@ -770,104 +792,120 @@ __device__ __forceinline__ void add_f32(float (&acc)[V], const float *src) {
 // u, |du| kept at or above 1e-20) can be run instead of h (VIMSCAN_GF):
 //     g_t = (Abar_t r_t) g_(t-1) + B_t,  r_t = du_(t-1) / du_t,  y_t = du_t C_t.g_t + D u_t,
 // which drops the drive multiply du B_n of every state; dprev carries du_(t-1).
+// The h-independent values of kSub tokens of sub-batch `sub` (softplus Delta, the decay
+// base, Delta u), formed ahead of the recurrence that uses them.
+template <typename T, int N, bool FAST, bool DESC, bool CONV, bool ZOH, bool DT>
+__device__ __forceinline__ void main_form(int sub, float (&qv)[kSub], float (&duv)[kSub], float (&uv)[kSub],
+                                          const ChannelParams<N> &prm, int dl, const T *su, const void *sd) {
+    constexpr bool LU = lu_mode<T, ZOH>();
+#pragma unroll
+    for (int k = 0; k < kSub; ++k) {
+        const int r = walk_row<DESC>(sub * kSub + k);
+        const float dt = delta_at<T, DT, LU>(sd, r, dl, prm.bias, prm.dtw);
+        uv[k] = u_of<T, N, CONV>(su, r, dl, prm);
+        qv[k] = FAST ? ex2(dt * prm.A0) : dt;
+        if constexpr (ZOH && FAST)
+            duv[k] = uv[k] * (prm.a0 != 0.0f ? expm1_acc(dt * prm.a0, qv[k]) * prm.inv_a0 : dt);
+        else
+            duv[k] = dt * uv[k];
+    }
+}
+
+// The recurrence over the kSub tokens of sub-batch `sub`, from their formed values.
+template <typename T, int N, bool FAST, bool DESC, bool CONV, bool ZOH, bool DT>
+__device__ __forceinline__ void main_recur(int sub, const float (&qv)[kSub], const float (&duv)[kSub],
+                                           const float (&uv)[kSub], bool second, float2 (&h)[N / 2], float &dprev,
+                                           const ChannelParams<N> &prm, const float *sB, const float *sC,
+                                           float *ypart) {
+    constexpr int NP = N / 2;
+    constexpr bool GF = VIMSCAN_GF && FAST && !ZOH;
+#pragma unroll
+    for (int k = 0; k < kSub; ++k) {
+        const int r = walk_row<DESC>(sub * kSub + k);
+        const float4 *B4 = reinterpret_cast<const float4 *>(sB + r * N);
+        const float4 *C4 = reinterpret_cast<const float4 *>(sC + r * N);
+        const float2 du2 = f2(duv[k], duv[k]);
+        float2 y0 = f2(0.f, 0.f), y1 = f2(0.f, 0.f);
+        // decays a = (Abar_2q, Abar_2q+1): with A_n = (n+1) A_0 they are the powers
+        // q^(2q+1), q^(2q+2) of q = exp(Delta A_0), one multiply per state
+        const float q = qv[k];
+        float2 a = FAST ? f2(q, q * q) : f2(0.f, 0.f);
+        const float2 step = FAST ? f2(a.y, a.y) : f2(0.f, 0.f);
+        float ysc = 1.0f;
+        if constexpr (GF) {
+            const float dv = clamp_du(duv[k]);
+            const float rr = dprev * rcp(dv);
+            dprev = dv;
+            a = mul2(a, f2(rr, rr));
+            ysc = dv;
+        }
+        // exact hold, structured A: Bbar_n u = kappa u S_n B_n / (n+1) with
+        // S_n = 1 + q + ... + q^n and B staged divided by n+1; KS = kappa u S for two
+        // states at a time, KS_(n+2) = KS_n + kappa u (1+q) q^(n+1)
+        const float cz = (ZOH && FAST) ? duv[k] * (1.0f + q) : 0.0f;
+        float2 KS = f2(duv[k], cz);
+        const float2 cz2 = f2(cz, cz);
+#pragma unroll
+        for (int qq = 0; qq < NP; qq += 2) {
+            float2 Bp[2], Cp[2];
+            if constexpr (NP >= 2) {
+                const float4 b4 = B4[qq / 2], c4 = C4[qq / 2];
+                Bp[0] = f2(b4.x, b4.y); Bp[1] = f2(b4.z, b4.w);
+                Cp[0] = f2(c4.x, c4.y); Cp[1] = f2(c4.z, c4.w);
+            } else {
+                Bp[0] = *reinterpret_cast<const float2 *>(sB + r * N);
+                Cp[0] = *reinterpret_cast<const float2 *>(sC + r * N);
+            }
+#pragma unroll
+            for (int e = 0; e < 2 && qq + e < NP; ++e) {
+                const int qi = qq + e;
+                float2 aq, drive;
+                if constexpr (GF) {
+                    aq = a;
+                    a = mul2(a, step);
+                    drive = Bp[e];
+                } else if constexpr (FAST) {
+                    aq = a;
+                    a = mul2(a, step);
+                    if constexpr (ZOH) {
+                        drive = mul2(KS, Bp[e]);
+                        KS = fma2(aq, cz2, KS);
+                    } else {
+                        drive = mul2(du2, Bp[e]);
+                    }
+                } else {
+                    const float A0n = __ldg(prm.A + 2 * qi), A1n = __ldg(prm.A + 2 * qi + 1);
+                    aq = f2(ex2(q * A0n * prm.emul), ex2(q * A1n * prm.emul));
+                    if constexpr (ZOH)   // gain per state, times n+1 against the staged B / (n+1)
+                        drive = mul2(mul2(f2(zoh_gain(q, A0n) * (float)(2 * qi + 1),
+                                             zoh_gain(q, A1n) * (float)(2 * qi + 2)),
+                                          f2(uv[k], uv[k])),
+                                     Bp[e]);
+                    else
+                        drive = mul2(du2, Bp[e]);
+                }
+                h[qi] = fma2(aq, h[qi], drive);
+                if (qi & 1) y1 = fma2(Cp[e], h[qi], y1);
+                else y0 = fma2(Cp[e], h[qi], y0);
+            }
+        }
+        const float2 ys = __fadd2_rn(y0, y1);
+        const float yv = fmaf(ysc, ys.x + ys.y, prm.D * uv[k]);
+        float *py = ypart + r * kDC;
+        *py = second ? *py + yv : yv;
+    }
+}
+
 template <typename T, int N, bool FAST, bool DESC, bool CONV, bool ZOH, bool DT>
 __device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], float &dprev,
                                           const ChannelParams<N> &prm, int dl, const T *su, const void *sd,
                                           const float *sB, const float *sC, float *ypart) {
-    constexpr int NP = N / 2;
-    constexpr bool LU = lu_mode<T, ZOH>();
-    constexpr bool GF = VIMSCAN_GF && FAST && !ZOH;
+    constexpr int kNSub = kTile / kSub;
 #pragma unroll 1
-    for (int sub = 0; sub < kTile / kSub; ++sub) {
-        // qv: q = exp(Delta A_0) (structured A) or Delta (general A); duv: Delta u, or
-        // with the exact hold kappa u, kappa = expm1(Delta A_0) / A_0 (structured A)
+    for (int sub = 0; sub < kNSub; ++sub) {
         float qv[kSub], duv[kSub], uv[kSub];
-#pragma unroll
-        for (int k = 0; k < kSub; ++k) {
-            const int r = walk_row<DESC>(sub * kSub + k);
-            const float dt = delta_at<T, DT, LU>(sd, r, dl, prm.bias, prm.dtw);
-            uv[k] = u_of<T, N, CONV>(su, r, dl, prm);
-            qv[k] = FAST ? ex2(dt * prm.A0) : dt;
-            if constexpr (ZOH && FAST)
-                duv[k] = uv[k] * (prm.a0 != 0.0f ? expm1_acc(dt * prm.a0, qv[k]) * prm.inv_a0 : dt);
-            else
-                duv[k] = dt * uv[k];
-        }
-#pragma unroll
-        for (int k = 0; k < kSub; ++k) {
-            const int r = walk_row<DESC>(sub * kSub + k);
-            const float4 *B4 = reinterpret_cast<const float4 *>(sB + r * N);
-            const float4 *C4 = reinterpret_cast<const float4 *>(sC + r * N);
-            const float2 du2 = f2(duv[k], duv[k]);
-            float2 y0 = f2(0.f, 0.f), y1 = f2(0.f, 0.f);
-            // decays a = (Abar_2q, Abar_2q+1): with A_n = (n+1) A_0 they are the powers
-            // q^(2q+1), q^(2q+2) of q = exp(Delta A_0), one multiply per state
-            const float q = qv[k];
-            float2 a = FAST ? f2(q, q * q) : f2(0.f, 0.f);
-            const float2 step = FAST ? f2(a.y, a.y) : f2(0.f, 0.f);
-            float ysc = 1.0f;
-            if constexpr (GF) {
-                const float dv = clamp_du(duv[k]);
-                const float rr = dprev * rcp(dv);
-                dprev = dv;
-                a = mul2(a, f2(rr, rr));
-                ysc = dv;
-            }
-            // exact hold, structured A: Bbar_n u = kappa u S_n B_n / (n+1) with
-            // S_n = 1 + q + ... + q^n and B staged divided by n+1; KS = kappa u S for two
-            // states at a time, KS_(n+2) = KS_n + kappa u (1+q) q^(n+1)
-            const float cz = (ZOH && FAST) ? duv[k] * (1.0f + q) : 0.0f;
-            float2 KS = f2(duv[k], cz);
-            const float2 cz2 = f2(cz, cz);
-#pragma unroll
-            for (int qq = 0; qq < NP; qq += 2) {
-                float2 Bp[2], Cp[2];
-                if constexpr (NP >= 2) {
-                    const float4 b4 = B4[qq / 2], c4 = C4[qq / 2];
-                    Bp[0] = f2(b4.x, b4.y); Bp[1] = f2(b4.z, b4.w);
-                    Cp[0] = f2(c4.x, c4.y); Cp[1] = f2(c4.z, c4.w);
-                } else {
-                    Bp[0] = *reinterpret_cast<const float2 *>(sB + r * N);
-                    Cp[0] = *reinterpret_cast<const float2 *>(sC + r * N);
-                }
-#pragma unroll
-                for (int e = 0; e < 2 && qq + e < NP; ++e) {
-                    const int qi = qq + e;
-                    float2 aq, drive;
-                    if constexpr (GF) {
-                        aq = a;
-                        a = mul2(a, step);
-                        drive = Bp[e];
-                    } else if constexpr (FAST) {
-                        aq = a;
-                        a = mul2(a, step);
-                        if constexpr (ZOH) {
-                            drive = mul2(KS, Bp[e]);
-                            KS = fma2(aq, cz2, KS);
-                        } else {
-                            drive = mul2(du2, Bp[e]);
-                        }
-                    } else {
-                        const float A0n = __ldg(prm.A + 2 * qi), A1n = __ldg(prm.A + 2 * qi + 1);
-                        aq = f2(ex2(q * A0n * prm.emul), ex2(q * A1n * prm.emul));
-                        if constexpr (ZOH)   // gain per state, times n+1 against the staged B / (n+1)
-                            drive = mul2(mul2(f2(zoh_gain(q, A0n) * (float)(2 * qi + 1),
-                                                 zoh_gain(q, A1n) * (float)(2 * qi + 2)),
-                                              f2(uv[k], uv[k])),
-                                         Bp[e]);
-                        else
-                            drive = mul2(du2, Bp[e]);
-                    }
-                    h[qi] = fma2(aq, h[qi], drive);
-                    if (qi & 1) y1 = fma2(Cp[e], h[qi], y1);
-                    else y0 = fma2(Cp[e], h[qi], y0);
-                }
-            }
-            const float2 ys = __fadd2_rn(y0, y1);
-            const float yv = fmaf(ysc, ys.x + ys.y, prm.D * uv[k]);
-            float *py = ypart + r * kDC;
-            *py = second ? *py + yv : yv;
-        }
+        main_form<T, N, FAST, DESC, CONV, ZOH, DT>(sub, qv, duv, uv, prm, dl, su, sd);
+        main_recur<T, N, FAST, DESC, CONV, ZOH, DT>(sub, qv, duv, uv, second, h, dprev, prm, sB, sC, ypart);
     }
 }
 
