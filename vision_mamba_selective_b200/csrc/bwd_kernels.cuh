@@ -369,6 +369,9 @@ struct BwdThread {
     bool valid;
     float2 A2[SH::NP], Araw[SH::NP];   // A of the thread's states, times log2(e) and as given
     float2 invA[SH::NP];               // 1 / A_n (0 where A_n = 0), for the exact hold
+    float2 in1[SH::NP];                // 1 / (n + 1) of the thread's states
+    float a0, inv_a0;                  // A_0 of the channel and its reciprocal (0 when A_0 = 0)
+    bool structured;                   // A_n = (n + 1) A_0 for every state of the channel
     float Dk;
     size_t cbase;   // [b][c][dir][d]
 };
@@ -408,6 +411,73 @@ __device__ __forceinline__ float hold_gain_dA(float dl, float z, float abar, flo
 }
 __device__ __forceinline__ float2 hold_gain2(float dl, float2 z, float2 abar, float2 inv_a) {
     return f2(hold_gain(dl, z.x, abar.x, inv_a.x), hold_gain(dl, z.y, abar.y, inv_a.y));
+}
+
+// The exact hold's gains (and with DA their A-derivatives) of the thread's states when
+// A_n = (n + 1) A_0, from one evaluation per token instead of one per state.  With
+// z = Delta A_0, q = exp(z), z_n = (n + 1) z, E_n = expm1(z_n) and F_n = z_n exp(z_n) - E_n:
+//   e_n = E_n / ((n + 1) A_0),   de_n/dA_n = F_n / ((n + 1) A_0)^2,
+//   E_(n+1) = q E_n + E_0,       F_(n+1) = q F_n + z (E_(n+1) - z chi(z)),
+// (E_0 = expm1(z), the gain recurrence's constant term)
+// chi(z) = (phi(z) - 1) / z, phi(z) = expm1(z) / z.  Every step adds terms of one sign
+// (no cancellation).  E and F of the thread's first state come from series (|z| < 1/2)
+// or closed forms; at A_0 = 0 the limits Delta and Delta^2 / 2.
+template <int N, bool DA>
+__device__ __forceinline__ void hold_states(const BwdThread<N> &th, float dl, const float2 (&ab)[BwdShape<N>::NP],
+                                            float2 (&gn)[BwdShape<N>::NP], float2 (&dg)[BwdShape<N>::NP]) {
+    using SH = BwdShape<N>;
+    constexpr int NP = SH::NP, NT = SH::NT;
+    if (th.a0 == 0.0f) {
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+            gn[k] = f2(dl, dl);
+            if constexpr (DA) dg[k] = f2(0.5f * dl * dl, 0.5f * dl * dl);
+        }
+        return;
+    }
+    const float z = dl * th.a0;
+    const float q = ex2(z * kLog2e);
+    const float zj = (float)(th.j0 + 1) * z;   // the thread's first state; exp(zj) = ab[0].x
+    const float e0 = expm1_acc(z, q);
+    float E = expm1_acc(zj, ab[0].x);
+    float F = 0.0f, zc = 0.0f;
+    if constexpr (DA) {
+        // F at zj: zj^2 psi(zj), psi(x) = sum_k k x^(k-1) / (k+1)!, or zj exp(zj) - E
+        float ps = fmaf(zj, 1.0f / 45360.0f, 1.0f / 5760.0f);
+        ps = fmaf(zj, ps, 1.0f / 840.0f);
+        ps = fmaf(zj, ps, 1.0f / 144.0f);
+        ps = fmaf(zj, ps, 1.0f / 30.0f);
+        ps = fmaf(zj, ps, 1.0f / 8.0f);
+        ps = fmaf(zj, ps, 1.0f / 3.0f);
+        ps = fmaf(zj, ps, 0.5f);
+        F = fabsf(zj) < 0.5f ? zj * zj * ps : fmaf(zj, ab[0].x, -E);
+        // z chi(z) = phi(z) - 1 = sum_(k>=1) z^k / (k+1)!, or expm1(z) / z - 1
+        float ch = fmaf(z, 1.0f / 362880.0f, 1.0f / 40320.0f);
+        ch = fmaf(z, ch, 1.0f / 5040.0f);
+        ch = fmaf(z, ch, 1.0f / 720.0f);
+        ch = fmaf(z, ch, 1.0f / 120.0f);
+        ch = fmaf(z, ch, 1.0f / 24.0f);
+        ch = fmaf(z, ch, 1.0f / 6.0f);
+        ch = fmaf(z, ch, 0.5f);
+        zc = fabsf(z) < 0.5f ? z * ch : e0 / z - 1.0f;   // phi(z) - 1 = z chi(z)
+    }
+    float ev[NT], fv[NT];
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+        ev[i] = E;
+        if constexpr (DA) fv[i] = F;
+        if (i + 1 < NT) {
+            const float En = fmaf(q, E, e0);
+            if constexpr (DA) F = fmaf(q, F, z * (En - zc));
+            E = En;
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < NP; ++k) {
+        const float2 w = mul2(th.in1[k], f2(th.inv_a0, th.inv_a0));   // 1 / ((n + 1) A_0)
+        gn[k] = mul2(f2(ev[2 * k], ev[2 * k + 1]), w);
+        if constexpr (DA) dg[k] = mul2(mul2(f2(fv[2 * k], fv[2 * k + 1]), w), w);
+    }
 }
 
 // h (or g) of the thread's states, from an fp32 row in global memory
@@ -461,6 +531,7 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
     using SH = BwdShape<N>;
     constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
     float *red_w = sm.red + (DIR * SH::WPD + th.wid) * TC * N;
+    const bool fast = ZOH && __all_sync(0xffffffffu, th.structured);
     float2 h[NP];
 #pragma unroll
     for (int k = 0; k < NP; ++k) h[k] = f2(0.f, 0.f);
@@ -480,14 +551,27 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
             load_row<NP>(sm.C + (DIR * TC + r) * N + th.j0, Cp);
             const float2 dl2 = f2(dl, dl), du2 = f2(du, du), dy2 = f2(tk.y, tk.y);
             float2 yp = f2(th.q == 0 ? th.Dk * tk.x : 0.0f, 0.0f);
+            float2 abk[NP], gnk[NP];
 #pragma unroll
             for (int k = 0; k < NP; ++k) {
                 const float2 e = mul2(dl2, th.A2[k]);
-                const float2 ab = f2(ex2(e.x), ex2(e.y));
+                abk[k] = f2(ex2(e.x), ex2(e.y));
+            }
+            if constexpr (ZOH) {
+                if (fast) {
+                    float2 unused[NP];
+                    hold_states<N, false>(th, dl, abk, gnk, unused);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < NP; ++k) gnk[k] = hold_gain2(dl, mul2(dl2, th.Araw[k]), abk[k], th.invA[k]);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < NP; ++k) {
+                const float2 ab = abk[k];
                 float2 drive;
                 if constexpr (ZOH) {
-                    const float2 gn = hold_gain2(dl, mul2(dl2, th.Araw[k]), ab, th.invA[k]);
-                    drive = mul2(mul2(gn, Bp[k]), f2(tk.x, tk.x));
+                    drive = mul2(mul2(gnk[k], Bp[k]), f2(tk.x, tk.x));
                 } else {
                     drive = mul2(du2, Bp[k]);
                 }
@@ -528,6 +612,7 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
     // with Q > 1 lane q = 0 gathers du and lane q = 1 d delta_raw of the channel
     constexpr int kDdLane = Q > 1 ? 1 : 0;
     float *red_w = sm.red + (DIR * SH::WPD + th.wid) * TC * N;
+    const bool fast = ZOH && __all_sync(0xffffffffu, th.structured);
     float2 g[NP], dA[NP];
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
@@ -556,10 +641,22 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
             for (int k = 0; k < NP; ++k) {
                 const float2 e = mul2(dl2, th.A2[k]);
                 aa[m][k] = f2(ex2(e.x), ex2(e.y));
+            }
+            float2 gnk[NP];
+            if constexpr (ZOH) {
+                if (fast) {
+                    float2 unused[NP];
+                    hold_states<N, false>(th, dl, aa[m], gnk, unused);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < NP; ++k) gnk[k] = hold_gain2(dl, mul2(dl2, th.Araw[k]), aa[m][k], th.invA[k]);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < NP; ++k) {
                 float2 drive;
                 if constexpr (ZOH) {
-                    const float2 gn = hold_gain2(dl, mul2(dl2, th.Araw[k]), aa[m][k], th.invA[k]);
-                    drive = mul2(mul2(gn, Bp[k]), f2(u, u));
+                    drive = mul2(mul2(gnk[k], Bp[k]), f2(u, u));
                 } else {
                     drive = mul2(du2, Bp[k]);
                 }
@@ -577,6 +674,20 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
             load_row<NP>(sm.C + (DIR * TC + r) * N + th.j0, Cp);
             const float2 dl2 = f2(dl, dl), du2 = f2(du, du), dy2 = f2(tk.y, tk.y);
             float2 sA = f2(0.f, 0.f), sB = f2(0.f, 0.f), sBa = f2(0.f, 0.f);
+            float2 gnk[NP], dgk[NP];
+            if constexpr (ZOH) {
+                if (fast) {
+                    hold_states<N, true>(th, dl, aa[m], gnk, dgk);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < NP; ++k) {
+                        const float2 zz = mul2(dl2, th.Araw[k]);
+                        gnk[k] = hold_gain2(dl, zz, aa[m][k], th.invA[k]);
+                        dgk[k] = f2(hold_gain_dA(dl, zz.x, aa[m][k].x, th.invA[k].x, gnk[k].x),
+                                    hold_gain_dA(dl, zz.y, aa[m][k].y, th.invA[k].y, gnk[k].y));
+                    }
+                }
+            }
 #pragma unroll
             for (int k = 0; k < NP; ++k) {
                 g[k] = fma2(Cp[k], dy2, g[k]);                               // dl/dh_t
@@ -588,10 +699,7 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
                 if constexpr (ZOH) {
                     // Bbar_n = e_n B_n: du and dB take e_n for Delta, the Delta term
                     // de_n/dDelta = Abar_n, and dA_n gains g B_n u de_n/dA_n
-                    const float2 zz = mul2(dl2, th.Araw[k]);
-                    const float2 gn = hold_gain2(dl, zz, aa[m][k], th.invA[k]);
-                    const float2 dg = f2(hold_gain_dA(dl, zz.x, aa[m][k].x, th.invA[k].x, gn.x),
-                                         hold_gain_dA(dl, zz.y, aa[m][k].y, th.invA[k].y, gn.y));
+                    const float2 gn = gnk[k], dg = dgk[k];
                     const float2 gB = mul2(g[k], Bp[k]), uu = f2(tk.x, tk.x);
                     sB = fma2(gB, gn, sB);
                     sBa = fma2(gB, aa[m][k], sBa);
@@ -853,6 +961,15 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
         th.Araw[k] = a;
         th.A2[k] = f2(a.x * kLog2e, a.y * kLog2e);
         th.invA[k] = f2(a.x != 0.0f ? 1.0f / a.x : 0.0f, a.y != 0.0f ? 1.0f / a.y : 0.0f);
+        th.in1[k] = f2(1.0f / (float)(th.j0 + 2 * k + 1), 1.0f / (float)(th.j0 + 2 * k + 2));
+    }
+    {
+        const float *Ar = p.A + ((size_t)th.dir * p.Di + (th.valid ? th.d : 0)) * N;
+        th.a0 = th.valid ? Ar[0] : 0.0f;
+        th.inv_a0 = th.a0 != 0.0f ? 1.0f / th.a0 : 0.0f;
+        th.structured = true;
+#pragma unroll
+        for (int n = 0; n < N; ++n) th.structured = th.structured && (!th.valid || Ar[n] == (float)(n + 1) * th.a0);
     }
     th.Dk = th.valid ? p.D[(size_t)th.dir * p.Di + th.d] : 0.0f;
     th.cbase = (((size_t)b * p.G + c) * 2 + th.dir) * p.Di + th.d;
