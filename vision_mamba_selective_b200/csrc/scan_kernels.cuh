@@ -79,6 +79,9 @@ constexpr float kLn2 = 0.69314718055994531f;
 #ifndef VIMSCAN_L2U
 #define VIMSCAN_L2U 1
 #endif
+#ifndef VIMSCAN_COMBINE_AHEAD
+#define VIMSCAN_COMBINE_AHEAD 16   // chunk summaries pair_combine loads before it folds them
+#endif
 // bf16 first-order kernels may keep Delta in log2 units (L = Delta / ln 2)
 template <typename T, bool ZOH>
 __host__ __device__ constexpr bool lu_mode() { return VIMSCAN_L2U && sizeof(T) == 2 && !ZOH; }
@@ -723,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMin
 // scan, whose summaries come from adj_carry).
 template <int N>
 __global__ void __launch_bounds__(256) pair_combine(PairArgs p) {
-    constexpr int kAhead = 16;
+    constexpr int kAhead = VIMSCAN_COMBINE_AHEAD;
     // launched as a programmatic dependent of pair_carry: wait for its summaries
     cudaGridDependencySynchronize();
     const int idx = blockIdx.x * blockDim.x + threadIdx.x;   // (b, dir, d, n), n fastest
