@@ -369,8 +369,8 @@ struct BwdThread {
     bool valid;
     float2 A2[SH::NP], Araw[SH::NP];   // A of the thread's states, times log2(e) and as given
     float2 invA[SH::NP];               // 1 / A_n (0 where A_n = 0), for the exact hold
-    float2 in1[SH::NP];                // 1 / (n + 1) of the thread's states
-    float a0, inv_a0;                  // A_0 of the channel and its reciprocal (0 when A_0 = 0)
+    float2 w1[SH::NP];                 // 1 / ((n + 1) A_0) of the thread's states (0 when A_0 = 0)
+    float a0;                          // A_0 of the channel
     bool structured;                   // A_n = (n + 1) A_0 for every state of the channel
     float Dk;
     size_t cbase;   // [b][c][dir][d]
@@ -474,7 +474,7 @@ __device__ __forceinline__ void hold_states(const BwdThread<N> &th, float dl, co
     }
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
-        const float2 w = mul2(th.in1[k], f2(th.inv_a0, th.inv_a0));   // 1 / ((n + 1) A_0)
+        const float2 w = th.w1[k];
         gn[k] = mul2(f2(ev[2 * k], ev[2 * k + 1]), w);
         if constexpr (DA) dg[k] = mul2(mul2(f2(fv[2 * k], fv[2 * k + 1]), w), w);
     }
@@ -525,13 +525,13 @@ __device__ __forceinline__ void channel_sum(const BwdThread<N> &th, float *red_w
 }
 
 // forward sweep of direction DIR: checkpoints, y^DIR (ungated) and the dC terms
-// (ZOH: the exact hold's Bbar in the state update)
-template <int N, int DIR, bool ZOH>
+// (ZOH: the exact hold's Bbar in the state update; FAST: its gains from hold_states)
+template <int N, int DIR, bool ZOH, bool FAST>
 __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
     using SH = BwdShape<N>;
     constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
     float *red_w = sm.red + (DIR * SH::WPD + th.wid) * TC * N;
-    const bool fast = ZOH && __all_sync(0xffffffffu, th.structured);
+    constexpr bool fast = ZOH && FAST;
     float2 h[NP];
 #pragma unroll
     for (int k = 0; k < NP; ++k) h[k] = f2(0.f, 0.f);
@@ -558,7 +558,7 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
                 abk[k] = f2(ex2(e.x), ex2(e.y));
             }
             if constexpr (ZOH) {
-                if (fast) {
+                if constexpr (fast) {
                     float2 unused[NP];
                     hold_states<N, false>(th, dl, abk, gnk, unused);
                 } else {
@@ -605,14 +605,14 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
 
 // adjoint sweep of direction DIR, segment by segment from the last: h re-run over
 // the segment from its checkpoint (keeping h and the decays), then g backwards
-template <int N, int DIR, bool ZOH>
+template <int N, int DIR, bool ZOH, bool FAST>
 __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
     using SH = BwdShape<N>;
     constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
     // with Q > 1 lane q = 0 gathers du and lane q = 1 d delta_raw of the channel
     constexpr int kDdLane = Q > 1 ? 1 : 0;
     float *red_w = sm.red + (DIR * SH::WPD + th.wid) * TC * N;
-    const bool fast = ZOH && __all_sync(0xffffffffu, th.structured);
+    constexpr bool fast = ZOH && FAST;
     float2 g[NP], dA[NP];
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
@@ -644,7 +644,7 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
             }
             float2 gnk[NP];
             if constexpr (ZOH) {
-                if (fast) {
+                if constexpr (fast) {
                     float2 unused[NP];
                     hold_states<N, false>(th, dl, aa[m], gnk, unused);
                 } else {
@@ -676,7 +676,7 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
             float2 sA = f2(0.f, 0.f), sB = f2(0.f, 0.f), sBa = f2(0.f, 0.f);
             float2 gnk[NP], dgk[NP];
             if constexpr (ZOH) {
-                if (fast) {
+                if constexpr (fast) {
                     hold_states<N, true>(th, dl, aa[m], gnk, dgk);
                 } else {
 #pragma unroll
@@ -781,6 +781,18 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
         for (int k = 0; k < NP; ++k) pa[k] = dA[k];
         if (th.q == 0) pr[(size_t)2 * p.Di * N + col] = dD;
         if (th.q == kDdLane) pr[(size_t)2 * p.Di * (N + 1) + col] = dbias;
+    }
+}
+
+// one sweep of the thread's direction: forward (ADJ false) or adjoint
+template <int N, bool ZOH, bool FAST, bool ADJ>
+__device__ __forceinline__ void bwd_sweep(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
+    if constexpr (ADJ) {
+        if (th.dir == 0) bwd_adjoint<N, 0, ZOH, FAST>(p, sm, th);
+        else bwd_adjoint<N, 1, ZOH, FAST>(p, sm, th);
+    } else {
+        if (th.dir == 0) bwd_forward<N, 0, ZOH, FAST>(p, sm, th);
+        else bwd_forward<N, 1, ZOH, FAST>(p, sm, th);
     }
 }
 
@@ -961,12 +973,16 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
         th.Araw[k] = a;
         th.A2[k] = f2(a.x * kLog2e, a.y * kLog2e);
         th.invA[k] = f2(a.x != 0.0f ? 1.0f / a.x : 0.0f, a.y != 0.0f ? 1.0f / a.y : 0.0f);
-        th.in1[k] = f2(1.0f / (float)(th.j0 + 2 * k + 1), 1.0f / (float)(th.j0 + 2 * k + 2));
     }
     {
         const float *Ar = p.A + ((size_t)th.dir * p.Di + (th.valid ? th.d : 0)) * N;
         th.a0 = th.valid ? Ar[0] : 0.0f;
-        th.inv_a0 = th.a0 != 0.0f ? 1.0f / th.a0 : 0.0f;
+        const float inv_a0 = th.a0 != 0.0f ? 1.0f / th.a0 : 0.0f;
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+            const float2 in1 = f2(1.0f / (float)(th.j0 + 2 * k + 1), 1.0f / (float)(th.j0 + 2 * k + 2));
+            th.w1[k] = mul2(in1, f2(inv_a0, inv_a0));
+        }
         th.structured = true;
 #pragma unroll
         for (int n = 0; n < N; ++n) th.structured = th.structured && (!th.valid || Ar[n] == (float)(n + 1) * th.a0);
@@ -980,8 +996,12 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     // carries are read after the wait
     if (p.G > 1) cudaGridDependencySynchronize();
 
-    if (th.dir == 0) bwd_forward<N, 0, ZOH>(p, sm, th);
-    else bwd_forward<N, 1, ZOH>(p, sm, th);
+    // the exact hold's path is chosen once per warp: its structured-A code and the
+    // general code are separate copies of the sweeps, with no branch between them per
+    // token, and a warp fetches only the copy it runs
+    const bool fast = ZOH && __all_sync(0xffffffffu, th.structured);
+    if (fast) bwd_sweep<N, ZOH, ZOH, false>(p, sm, th);
+    else bwd_sweep<N, ZOH, false, false>(p, sm, th);
     __syncthreads();
     // dz = dout silu'(z) (sum of the directions' y), and the CTA's dC terms; the
     // cross-scan's first pair leaves its y for the second
@@ -1010,8 +1030,8 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     store_bc_part<N>(p, sm.red, p.dC_part, b, t0, tc, blk);
     __syncthreads();
 
-    if (th.dir == 0) bwd_adjoint<N, 0, ZOH>(p, sm, th);
-    else bwd_adjoint<N, 1, ZOH>(p, sm, th);
+    if (fast) bwd_sweep<N, ZOH, ZOH, true>(p, sm, th);
+    else bwd_sweep<N, ZOH, false, true>(p, sm, th);
     __syncthreads();
     for (int li = threadIdx.x; li < TC * (CH / kG); li += SH::kThr) {
         const int r = li / (CH / kG), c0 = (li % (CH / kG)) * kG, ch = d0 + c0;

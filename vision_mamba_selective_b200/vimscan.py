@@ -106,47 +106,59 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}: fp32 or bf16")
 
 
-def _ptr(t, *, dtype=None, name="tensor"):
-    if t is None:
-        return None
-    if not isinstance(t, torch.Tensor) or not t.is_cuda:
-        raise TypeError(f"{name} must be a CUDA tensor")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous")
-    if dtype is not None and t.dtype != dtype:
-        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
-    return t.data_ptr()
+def _ptrs(where, ref, specs):
+    """Check every tensor the kernels will address and return their data pointers, in
+    the order of ``specs`` (None for an absent tensor), before the library is called.
 
-
-def _check(where, ref, specs):
-    """Refuse, before the library is called, any tensor the kernels could not address
-    safely.
-
-    ``ref`` is the tensor that fixes the device; it must be the current CUDA device
-    (the stream the library launches on belongs to it).  ``specs`` holds
-    (name, tensor or None, rule) with rule either an exact shape tuple or
-    ("numel", n, last): at least n elements with last dimension ``last`` (buffers such
-    as B/C with a per-direction stride).  Raises TypeError or ValueError.
+    ``ref`` fixes the device; it must be the current CUDA device (the stream the library
+    launches on belongs to it).  ``specs`` holds (name, tensor or None, dtype or None,
+    rule) with rule either an exact shape tuple or ("numel", n, last): at least n
+    elements with last dimension ``last`` (buffers such as B/C with a per-direction
+    stride).  Every tensor must be contiguous.  Raises TypeError (not a CUDA tensor, a
+    wrong dtype) or ValueError (device, shape, layout).  One pass per tensor, integer
+    device indices and direct size comparisons: this runs on every call, so its cost
+    is part of a small problem's launch latency.
     """
     if not isinstance(ref, torch.Tensor) or not ref.is_cuda:
         raise TypeError(f"{where}: inputs must be CUDA tensors")
+    dev = ref.get_device()
     cur = torch.cuda.current_device()
-    if ref.device.index != cur:
+    if dev != cur:
         raise ValueError(f"{where}: tensors are on {ref.device} but the current device is cuda:{cur}")
-    for name, t, rule in specs:
+    out = []
+    for name, t, dtype, rule in specs:
         if t is None:
+            out.append(None)
             continue
-        if not isinstance(t, torch.Tensor) or not t.is_cuda:
-            raise TypeError(f"{where}: {name} must be a CUDA tensor")
-        if t.device != ref.device:
+        if not isinstance(t, torch.Tensor) or t.get_device() != dev:
+            if not isinstance(t, torch.Tensor) or not t.is_cuda:
+                raise TypeError(f"{where}: {name} must be a CUDA tensor")
             raise ValueError(f"{where}: {name} is on {t.device}, the other inputs on {ref.device}")
-        if rule and rule[0] == "numel":
+        if dtype is not None and t.dtype != dtype:
+            raise TypeError(f"{where}: {name} must be {dtype}, got {t.dtype}")
+        if rule[0] == "numel":
             _, n, last = rule
             if t.numel() < n or t.dim() == 0 or t.shape[-1] != last:
                 raise ValueError(f"{where}: {name} has shape {tuple(t.shape)}; it needs at least {n} "
                                  f"elements with last dimension {last}")
-        elif tuple(t.shape) != tuple(rule):
+        elif t.shape != rule:
             raise ValueError(f"{where}: {name} has shape {tuple(t.shape)}, expected {tuple(rule)}")
+        if not t.is_contiguous():
+            raise ValueError(f"{where}: {name} must be contiguous")
+        out.append(t.data_ptr())
+    return out
+
+
+def _out_specs(out, io, act, bc, a_shape, d_shape):
+    """The derivative outputs as _ptrs specs, in the library's argument order (none when
+    there is no output dict: the inputs were refused before it could be allocated)."""
+    if out is None:
+        return []
+    f32 = torch.float32
+    return [("out['du']", out["du"], io, act), ("out['ddelta']", out["ddelta"], io, act),
+            ("out['dz']", out["dz"], io, act), ("out['dB']", out["dB"], f32, bc), ("out['dC']", out["dC"], f32, bc),
+            ("out['dA']", out["dA"], f32, a_shape), ("out['dD']", out["dD"], f32, d_shape),
+            ("out['ddelta_bias']", out["ddelta_bias"], f32, d_shape)]
 
 
 def _bc_rule(batch, L, N, bc_dir_stride):
@@ -188,22 +200,18 @@ def _bidir(name, u, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, y, bc_dir_
     dt = _dtype_code(u)
     act = (batch, L, Di)
     bc = _bc_rule(batch, L, N, bc_dir_stride)
-    _check(name, u, [("delta", delta, act), ("z", z, act), ("B", B, bc), ("C", C, bc), ("A", A, (2, Di, N)),
-                     ("D", D, (2, Di)), ("delta_bias", delta_bias, (2, Di)), ("y", y, act),
-                     ("conv_w", conv_w, (2, Di, 3)), ("conv_b", conv_b, (2, Di))])
     if y is None:
         y = torch.empty_like(u)
-    ws, ws_bytes = _workspace(vim_scan_workspace_bytes(0, batch, L, 0, Di, N), workspace, u.device)
     conv = conv_w is not None or conv_b is not None
-    pre = (_ptr(u, name="x" if conv else "u"),)
-    if conv or zoh:
-        pre += (_ptr(conv_w, dtype=torch.float32, name="conv_w"), _ptr(conv_b, dtype=torch.float32, name="conv_b"))
-    args = pre + (
-        _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
-        _ptr(B, dtype=u.dtype, name="B"), _ptr(C, dtype=u.dtype, name="C"), int(bc_dir_stride),
-        _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
-        _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(y, dtype=u.dtype, name="y"),
-        batch, L, Di, N, dt)
+    f32, io = torch.float32, u.dtype
+    pu, pcw, pcb, pdelta, pz, pB, pC, pA, pD, pbias, py = _ptrs(name, u, [
+        ("x" if conv else "u", u, None, act), ("conv_w", conv_w, f32, (2, Di, 3)), ("conv_b", conv_b, f32, (2, Di)),
+        ("delta", delta, io, act), ("z", z, io, act), ("B", B, io, bc), ("C", C, io, bc),
+        ("A", A, f32, (2, Di, N)), ("D", D, f32, (2, Di)), ("delta_bias", delta_bias, f32, (2, Di)),
+        ("y", y, io, act)])
+    ws, ws_bytes = _workspace(vim_scan_workspace_bytes(0, batch, L, 0, Di, N), workspace, u.device)
+    pre = (pu, pcw, pcb) if conv or zoh else (pu,)
+    args = pre + (pdelta, pz, pB, pC, int(bc_dir_stride), pA, pD, pbias, py, batch, L, Di, N, dt)
     tail = (None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
     ev = None if events is None else _events(events)
     if zoh:
@@ -265,22 +273,22 @@ def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stri
     dev = u.device
     act = (batch, L, Di)
     bc = _bc_rule(batch, L, N, bc_dir_stride)
-    specs = [("delta", delta, act), ("z", z, act), ("B", B, bc), ("C", C, bc), ("A", A, (2, Di, N)),
-             ("D", D, (2, Di)), ("delta_bias", delta_bias, (2, Di)), ("dout", dout, act)]
     if out is not None:
-        specs += [("out['du']", out["du"], act), ("out['ddelta']", out["ddelta"], act),
-                  ("out['dz']", out["dz"], act), ("out['dB']", out["dB"], bc), ("out['dC']", out["dC"], bc), ("out['dA']", out["dA"], (2, Di, N)),
-                  ("out['dD']", out["dD"], (2, Di)), ("out['ddelta_bias']", out["ddelta_bias"], (2, Di))]
         if z is not None and out["dz"] is None:
             raise ValueError("vim_scan_bidir_bwd: out['dz'] is needed when z is given")
-    _check("vim_scan_bidir_bwd", u, specs)
-    out = out if out is not None else dict(du=torch.empty_like(u), ddelta=torch.empty_like(u),
-               dz=torch.empty_like(u) if z is not None else None,
-               dB=torch.zeros(B.shape, dtype=torch.float32, device=dev),
-               dC=torch.zeros(C.shape, dtype=torch.float32, device=dev),
-               dA=torch.empty((2, Di, N), dtype=torch.float32, device=dev),
-               dD=torch.empty((2, Di), dtype=torch.float32, device=dev),
-               ddelta_bias=torch.empty((2, Di), dtype=torch.float32, device=dev))
+    elif isinstance(u, torch.Tensor) and u.is_cuda:
+        out = dict(du=torch.empty_like(u), ddelta=torch.empty_like(u),
+                   dz=torch.empty_like(u) if z is not None else None,
+                   dB=torch.zeros(B.shape, dtype=torch.float32, device=dev),
+                   dC=torch.zeros(C.shape, dtype=torch.float32, device=dev),
+                   dA=torch.empty((2, Di, N), dtype=torch.float32, device=dev),
+                   dD=torch.empty((2, Di), dtype=torch.float32, device=dev),
+                   ddelta_bias=torch.empty((2, Di), dtype=torch.float32, device=dev))
+    f32, io = torch.float32, u.dtype
+    ptrs = _ptrs("vim_scan_bidir_bwd", u, [
+        ("u", u, None, act), ("delta", delta, io, act), ("z", z, io, act), ("B", B, io, bc), ("C", C, io, bc),
+        ("A", A, f32, (2, Di, N)), ("D", D, f32, (2, Di)), ("delta_bias", delta_bias, f32, (2, Di)),
+        ("dout", dout, io, act)] + _out_specs(out, io, act, bc, (2, Di, N), (2, Di)))
     ws, ws_bytes = _workspace(vim_scan_bwd_workspace_bytes(batch, L, Di, N, bc_dir_stride > 0), workspace, dev)
     if zoh:
         fn = lib.vim_scan_bidir_bwd_ex
@@ -289,12 +297,7 @@ def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stri
         fn = lib.vim_scan_bidir_bwd if events is None else lib.vim_scan_bidir_bwd_events
         flags, extra = (), (() if events is None else (_events(events),))
     st = fn(
-        _ptr(u, name="u"), _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
-        _ptr(B, dtype=u.dtype, name="B"), _ptr(C, dtype=u.dtype, name="C"), int(bc_dir_stride),
-        _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
-        _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(dout, dtype=u.dtype, name="dout"),
-        _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dz"]), _ptr(out["dB"]), _ptr(out["dC"]),
-        _ptr(out["dA"]), _ptr(out["dD"]), _ptr(out["ddelta_bias"]),
+        *ptrs[:5], int(bc_dir_stride), *ptrs[5:],
         batch, L, Di, N, dt, *flags, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream), *extra)
     if st != VIM_OK:
         raise VimScanError(st, "vim_scan_bidir_bwd")
@@ -314,30 +317,23 @@ def vmamba_cross_scan4_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, workspa
     dev = u.device
     act = (batch, H, W, Ch)
     bc = (4, batch, H * W, N)
-    specs = [("delta", delta, act), ("z", z, act), ("B", B, bc), ("C", C, bc), ("A", A, (4, Ch, N)),
-             ("D", D, (4, Ch)), ("delta_bias", delta_bias, (4, Ch)), ("dout", dout, act)]
     if out is not None:
-        specs += [("out['du']", out["du"], act), ("out['ddelta']", out["ddelta"], act),
-                  ("out['dz']", out["dz"], act), ("out['dB']", out["dB"], bc), ("out['dC']", out["dC"], bc),
-                  ("out['dA']", out["dA"], (4, Ch, N)), ("out['dD']", out["dD"], (4, Ch)),
-                  ("out['ddelta_bias']", out["ddelta_bias"], (4, Ch))]
         if z is not None and out["dz"] is None:
             raise ValueError("vmamba_cross_scan4_bwd: out['dz'] is needed when z is given")
-    _check("vmamba_cross_scan4_bwd", u, specs)
-    f32 = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
-    if out is None:
+    elif isinstance(u, torch.Tensor) and u.is_cuda:
+        e32 = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
         out = dict(du=torch.empty_like(u), ddelta=torch.empty_like(u), dz=torch.empty_like(u) if z is not None else None,
-                   dB=f32(*B.shape), dC=f32(*C.shape), dA=f32(4, Ch, N), dD=f32(4, Ch), ddelta_bias=f32(4, Ch))
+                   dB=e32(*B.shape), dC=e32(*C.shape), dA=e32(4, Ch, N), dD=e32(4, Ch), ddelta_bias=e32(4, Ch))
+    f32, io = torch.float32, u.dtype
+    ptrs = _ptrs("vmamba_cross_scan4_bwd", u, [
+        ("u", u, None, act), ("delta", delta, io, act), ("z", z, io, act), ("B", B, io, bc), ("C", C, io, bc),
+        ("A", A, f32, (4, Ch, N)), ("D", D, f32, (4, Ch)), ("delta_bias", delta_bias, f32, (4, Ch)),
+        ("dout", dout, io, act)] + _out_specs(out, io, act, bc, (4, Ch, N), (4, Ch)))
     ws, ws_bytes = _workspace(int(lib.vmamba_cross_scan4_bwd_workspace_bytes(batch, H, W, Ch, N)), workspace, dev)
     fn = lib.vmamba_cross_scan4_bwd_ex if zoh else lib.vmamba_cross_scan4_bwd
     flags = (VIM_FLAG_ZOH_EXACT,) if zoh else ()
     st = fn(
-        _ptr(u, name="u"), _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
-        _ptr(B, dtype=u.dtype, name="B"), _ptr(C, dtype=u.dtype, name="C"),
-        _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
-        _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(dout, dtype=u.dtype, name="dout"),
-        _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dz"]), _ptr(out["dB"]), _ptr(out["dC"]),
-        _ptr(out["dA"]), _ptr(out["dD"]), _ptr(out["ddelta_bias"]),
+        *ptrs,
         batch, H, W, Ch, N, _dtype_code(u), *flags, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
     if st != VIM_OK:
         raise VimScanError(st, "vmamba_cross_scan4_bwd")
@@ -358,18 +354,16 @@ def vim_block_scan(x, Wx, Wdt, dt_bias, A, D, z, *, conv_w=None, conv_b=None, y=
     batch, L, Di = x.shape
     N = A.shape[-1]
     act = (batch, L, Di)
-    _check("vim_block_scan", x, [("Wx", Wx, (2, Di, 2 * N + 1)), ("Wdt", Wdt, (2, Di)), ("dt_bias", dt_bias, (2, Di)),
-                                  ("A", A, (2, Di, N)), ("D", D, (2, Di)), ("z", z, act), ("y", y, act),
-                                  ("conv_w", conv_w, (2, Di, 3)), ("conv_b", conv_b, (2, Di))])
-    if y is None:
+    if y is None and isinstance(x, torch.Tensor) and x.is_cuda:
         y = torch.empty_like(x)
+    f32, io = torch.float32, x.dtype
+    ptrs = _ptrs("vim_block_scan", x, [
+        ("x", x, None, act), ("conv_w", conv_w, f32, (2, Di, 3)), ("conv_b", conv_b, f32, (2, Di)),
+        ("Wx", Wx, io, (2, Di, 2 * N + 1)), ("Wdt", Wdt, f32, (2, Di)), ("dt_bias", dt_bias, f32, (2, Di)),
+        ("A", A, f32, (2, Di, N)), ("D", D, f32, (2, Di)), ("z", z, io, act), ("y", y, io, act)])
     ws, ws_bytes = _workspace(vim_block_workspace_bytes(batch, L, Di, N), workspace, x.device)
     st = lib.vim_block_scan(
-        _ptr(x, name="x"), _ptr(conv_w, dtype=torch.float32, name="conv_w"),
-        _ptr(conv_b, dtype=torch.float32, name="conv_b"), _ptr(Wx, dtype=x.dtype, name="Wx"),
-        _ptr(Wdt, dtype=torch.float32, name="Wdt"), _ptr(dt_bias, dtype=torch.float32, name="dt_bias"),
-        _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
-        _ptr(z, dtype=x.dtype, name="z"), _ptr(y, dtype=x.dtype, name="y"),
+        *ptrs,
         batch, L, Di, N, _dtype_code(x), None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream),
         None if events is None else _events(events))
     if st != VIM_OK:
@@ -390,16 +384,15 @@ def vim_scan_bidir_noalloc(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_di
     dt = _dtype_code(u)
     act = (batch, L, Di)
     bc = _bc_rule(batch, L, N, bc_dir_stride)
-    _check("vim_scan_bidir_noalloc", u, [("delta", delta, act), ("z", z, act), ("B", B, bc), ("C", C, bc),
-                                          ("A", A, (2, Di, N)), ("D", D, (2, Di)),
-                                          ("delta_bias", delta_bias, (2, Di)), ("y", y, act)])
-    if y is None:
+    if y is None and isinstance(u, torch.Tensor) and u.is_cuda:
         y = torch.empty_like(u)
+    f32, io = torch.float32, u.dtype
+    ptrs = _ptrs("vim_scan_bidir_noalloc", u, [
+        ("u", u, None, act), ("delta", delta, io, act), ("z", z, io, act), ("B", B, io, bc), ("C", C, io, bc),
+        ("A", A, f32, (2, Di, N)), ("D", D, f32, (2, Di)), ("delta_bias", delta_bias, f32, (2, Di)),
+        ("y", y, io, act)])
     st = lib.vim_scan_bidir_noalloc(
-        _ptr(u, name="u"), _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
-        _ptr(B, dtype=u.dtype, name="B"), _ptr(C, dtype=u.dtype, name="C"), int(bc_dir_stride),
-        _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
-        _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(y, dtype=u.dtype, name="y"),
+        *ptrs[:5], int(bc_dir_stride), *ptrs[5:],
         batch, L, Di, N, dt, _stream(stream))
     if st != VIM_OK:
         raise VimScanError(st, "vim_scan_bidir_noalloc")
@@ -419,18 +412,14 @@ def vmamba_cross_scan4(u, delta, z, B, C, A, D, delta_bias, *, y=None, workspace
     dt = _dtype_code(u)
     act = (batch, H, W, Ch)
     bc = (4, batch, H * W, N)
-    _check("vmamba_cross_scan4", u, [("delta", delta, act), ("z", z, act), ("B", B, bc), ("C", C, bc),
-                                      ("A", A, (4, Ch, N)), ("D", D, (4, Ch)), ("delta_bias", delta_bias, (4, Ch)),
-                                      ("y", y, act)])
     if y is None:
         y = torch.empty_like(u)
+    f32, io = torch.float32, u.dtype
+    args = tuple(_ptrs("vmamba_cross_scan4", u, [
+        ("u", u, None, act), ("delta", delta, io, act), ("z", z, io, act), ("B", B, io, bc), ("C", C, io, bc),
+        ("A", A, f32, (4, Ch, N)), ("D", D, f32, (4, Ch)), ("delta_bias", delta_bias, f32, (4, Ch)),
+        ("y", y, io, act)])) + (batch, H, W, Ch, N, dt)
     ws, ws_bytes = _workspace(vim_scan_workspace_bytes(1, batch, H, W, Ch, N), workspace, u.device)
-    args = (
-        _ptr(u, name="u"), _ptr(delta, dtype=u.dtype, name="delta"), _ptr(z, dtype=u.dtype, name="z"),
-        _ptr(B, dtype=u.dtype, name="B"), _ptr(C, dtype=u.dtype, name="C"),
-        _ptr(A, dtype=torch.float32, name="A"), _ptr(D, dtype=torch.float32, name="D"),
-        _ptr(delta_bias, dtype=torch.float32, name="delta_bias"), _ptr(y, dtype=u.dtype, name="y"),
-        batch, H, W, Ch, N, dt)
     tail = (None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
     ev = None if events is None else _events(events)
     if zoh:
@@ -450,12 +439,12 @@ def cross_merge4(ys, z, H, W, *, y=None, stream=None):
     if ys.shape[0] != 4 or L != H * W:
         raise ValueError("ys must be [4, batch, H*W, C]")
     act = (batch, H, W, Ch)
-    _check("cross_merge4", ys, [("z", z, act), ("y", y, act)])
     dt = _dtype_code(ys)
-    if y is None:
+    if y is None and isinstance(ys, torch.Tensor) and ys.is_cuda:
         y = torch.empty((batch, H, W, Ch), dtype=ys.dtype, device=ys.device)
-    st = lib.cross_merge4(_ptr(ys, name="ys"), _ptr(z, dtype=ys.dtype, name="z"),
-                          _ptr(y, dtype=ys.dtype, name="y"), batch, H, W, Ch, dt, _stream(stream))
+    pys, pz, py = _ptrs("cross_merge4", ys, [("ys", ys, None, tuple(ys.shape)), ("z", z, ys.dtype, act),
+                                             ("y", y, ys.dtype, act)])
+    st = lib.cross_merge4(pys, pz, py, batch, H, W, Ch, dt, _stream(stream))
     if st != VIM_OK:
         raise VimScanError(st, "cross_merge4")
     return y
