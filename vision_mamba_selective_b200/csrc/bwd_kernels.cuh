@@ -47,6 +47,9 @@ constexpr int kReduceParts = 32;              // row groups of the first paramet
 #ifndef VIMSCAN_BWD_BATCH
 #define VIMSCAN_BWD_BATCH 1                      // reductions batched over each segment's tokens
 #endif
+#ifndef VIMSCAN_BWD_RTDIR
+#define VIMSCAN_BWD_RTDIR 1                      // one copy of the sweeps for both directions (bit 0:
+#endif                                           // exact hold, bit 1: first order)
 #ifndef VIMSCAN_BWD_MIN_WARPS
 #define VIMSCAN_BWD_MIN_WARPS 16                 // resident warps per SM the register budget targets
 #endif
@@ -422,11 +425,59 @@ __device__ __forceinline__ float2 hold_gain2(float dl, float2 z, float2 abar, fl
 // chi(z) = (phi(z) - 1) / z, phi(z) = expm1(z) / z.  Every step adds terms of one sign
 // (no cancellation).  E and F of the thread's first state come from series (|z| < 1/2)
 // or closed forms; at A_0 = 0 the limits Delta and Delta^2 / 2.
+//
+// q, E_0 and z chi(z) are the same for the Q lanes that share a channel.  hold_seg forms
+// them once per segment, token m by lane m mod Q of the channel, and hold_states takes
+// token m's by a shuffle from that lane (every lane of the warp takes part).
 template <int N, bool DA>
+struct HoldSeg {
+    static constexpr int K = kBwdSeg / BwdShape<N>::Q;   // tokens of the segment per lane
+    float q[K], e0[K], zc[DA ? K : 1];
+};
+template <int N, bool DA>
+__device__ __forceinline__ HoldSeg<N, DA> hold_seg(const BwdSmem<N> &sm, const BwdThread<N> &th, int DIR, int sg) {
+    using SH = BwdShape<N>;
+    static_assert(kBwdSeg % SH::Q == 0, "a segment's tokens split evenly over a channel's lanes");
+    HoldSeg<N, DA> s;
+#pragma unroll
+    for (int k = 0; k < HoldSeg<N, DA>::K; ++k) {
+        const int i = sg * kBwdSeg + th.q + k * SH::Q, r = DIR ? SH::TC - 1 - i : i;
+        const float dl = reinterpret_cast<const float *>(sm.dsg)[2 * ((DIR * SH::TC + r) * SH::CH + th.cl)];
+        const float z = dl * th.a0;
+        s.q[k] = ex2(z * kLog2e);
+        s.e0[k] = expm1_acc(z, s.q[k]);
+        if constexpr (DA) {
+            // z chi(z) = phi(z) - 1 = sum_(k>=1) z^k / (k+1)!, or expm1(z) / z - 1
+            float ch = fmaf(z, 1.0f / 362880.0f, 1.0f / 40320.0f);
+            ch = fmaf(z, ch, 1.0f / 5040.0f);
+            ch = fmaf(z, ch, 1.0f / 720.0f);
+            ch = fmaf(z, ch, 1.0f / 120.0f);
+            ch = fmaf(z, ch, 1.0f / 24.0f);
+            ch = fmaf(z, ch, 1.0f / 6.0f);
+            ch = fmaf(z, ch, 0.5f);
+            s.zc[k] = fabsf(z) < 0.5f ? z * ch : s.e0[k] / z - 1.0f;
+        }
+    }
+    return s;
+}
+template <int N>
+__device__ __forceinline__ float hold_take(const BwdThread<N> &th, const float (&v)[HoldSeg<N, false>::K], int m) {
+    constexpr int Q = BwdShape<N>::Q;
+    if constexpr (Q == 1) return v[m];
+    else return __shfl_sync(0xffffffffu, v[m / Q], (th.lane & ~(Q - 1)) | (m % Q));
+}
+
+template <int N, bool DA, bool SDA>
 __device__ __forceinline__ void hold_states(const BwdThread<N> &th, float dl, const float2 (&ab)[BwdShape<N>::NP],
+                                            const HoldSeg<N, SDA> &hs, int m,
                                             float2 (&gn)[BwdShape<N>::NP], float2 (&dg)[BwdShape<N>::NP]) {
     using SH = BwdShape<N>;
     constexpr int NP = SH::NP, NT = SH::NT;
+    static_assert(SDA || !DA, "the A-derivative needs the segment's z chi(z)");
+    const float q = hold_take<N>(th, hs.q, m);
+    const float e0 = hold_take<N>(th, hs.e0, m);
+    float zc = 0.0f;
+    if constexpr (DA) zc = hold_take<N>(th, hs.zc, m);
     if (th.a0 == 0.0f) {
 #pragma unroll
         for (int k = 0; k < NP; ++k) {
@@ -436,11 +487,9 @@ __device__ __forceinline__ void hold_states(const BwdThread<N> &th, float dl, co
         return;
     }
     const float z = dl * th.a0;
-    const float q = ex2(z * kLog2e);
     const float zj = (float)(th.j0 + 1) * z;   // the thread's first state; exp(zj) = ab[0].x
-    const float e0 = expm1_acc(z, q);
     float E = expm1_acc(zj, ab[0].x);
-    float F = 0.0f, zc = 0.0f;
+    float F = 0.0f;
     if constexpr (DA) {
         // F at zj: zj^2 psi(zj), psi(x) = sum_k k x^(k-1) / (k+1)!, or zj exp(zj) - E
         float ps = fmaf(zj, 1.0f / 45360.0f, 1.0f / 5760.0f);
@@ -451,15 +500,6 @@ __device__ __forceinline__ void hold_states(const BwdThread<N> &th, float dl, co
         ps = fmaf(zj, ps, 1.0f / 3.0f);
         ps = fmaf(zj, ps, 0.5f);
         F = fabsf(zj) < 0.5f ? zj * zj * ps : fmaf(zj, ab[0].x, -E);
-        // z chi(z) = phi(z) - 1 = sum_(k>=1) z^k / (k+1)!, or expm1(z) / z - 1
-        float ch = fmaf(z, 1.0f / 362880.0f, 1.0f / 40320.0f);
-        ch = fmaf(z, ch, 1.0f / 5040.0f);
-        ch = fmaf(z, ch, 1.0f / 720.0f);
-        ch = fmaf(z, ch, 1.0f / 120.0f);
-        ch = fmaf(z, ch, 1.0f / 24.0f);
-        ch = fmaf(z, ch, 1.0f / 6.0f);
-        ch = fmaf(z, ch, 0.5f);
-        zc = fabsf(z) < 0.5f ? z * ch : e0 / z - 1.0f;   // phi(z) - 1 = z chi(z)
     }
     float ev[NT], fv[NT];
 #pragma unroll
@@ -526,10 +566,11 @@ __device__ __forceinline__ void channel_sum(const BwdThread<N> &th, float *red_w
 
 // forward sweep of direction DIR: checkpoints, y^DIR (ungated) and the dC terms
 // (ZOH: the exact hold's Bbar in the state update; FAST: its gains from hold_states)
-template <int N, int DIR, bool ZOH, bool FAST>
+template <int N, int DIRT, bool ZOH, bool FAST>
 __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
     using SH = BwdShape<N>;
     constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
+    const int DIR = DIRT < 0 ? th.dir : DIRT;   // DIRT < 0: the direction at run time
     float *red_w = sm.red + (DIR * SH::WPD + th.wid) * TC * N;
     constexpr bool fast = ZOH && FAST;
     float2 h[NP];
@@ -539,6 +580,8 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
 #pragma unroll 1
     for (int sg = 0; sg < kBwdNSeg; ++sg) {
         store_ck<N>(sm, th.tid, sg, h);
+        [[maybe_unused]] HoldSeg<N, false> hs;
+        if constexpr (fast) hs = hold_seg<N, false>(sm, th, DIR, sg);
         float yv[kBwdSeg], vc[SH::BATCH ? kBwdSeg * SH::NT : 1];   // batched: y partials, dC terms
 #pragma unroll
         for (int m = 0; m < kBwdSeg; ++m) {
@@ -560,7 +603,7 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
             if constexpr (ZOH) {
                 if constexpr (fast) {
                     float2 unused[NP];
-                    hold_states<N, false>(th, dl, abk, gnk, unused);
+                    hold_states<N, false>(th, dl, abk, hs, m, gnk, unused);
                 } else {
 #pragma unroll
                     for (int k = 0; k < NP; ++k) gnk[k] = hold_gain2(dl, mul2(dl2, th.Araw[k]), abk[k], th.invA[k]);
@@ -605,10 +648,11 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
 
 // adjoint sweep of direction DIR, segment by segment from the last: h re-run over
 // the segment from its checkpoint (keeping h and the decays), then g backwards
-template <int N, int DIR, bool ZOH, bool FAST>
+template <int N, int DIRT, bool ZOH, bool FAST>
 __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
     using SH = BwdShape<N>;
     constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
+    const int DIR = DIRT < 0 ? th.dir : DIRT;   // DIRT < 0: the direction at run time
     // with Q > 1 lane q = 0 gathers du and lane q = 1 d delta_raw of the channel
     constexpr int kDdLane = Q > 1 ? 1 : 0;
     float *red_w = sm.red + (DIR * SH::WPD + th.wid) * TC * N;
@@ -625,6 +669,8 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
     for (int sg = kBwdNSeg - 1; sg >= 0; --sg) {
         float2 h0[NP];
         load_ck<N>(sm, th.tid, sg, h0);
+        [[maybe_unused]] HoldSeg<N, true> hs;
+        if constexpr (fast) hs = hold_seg<N, true>(sm, th, DIR, sg);
         float2 hh[kBwdSeg][NP], aa[kBwdSeg][NP];
         // batched: [slot][du, d delta_raw] partials and [slot][state] dB terms, slot = 3 - m
         float xq[SH::BATCH ? 2 * kBwdSeg : 1], vb[SH::BATCH ? kBwdSeg * SH::NT : 1];
@@ -646,7 +692,7 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
             if constexpr (ZOH) {
                 if constexpr (fast) {
                     float2 unused[NP];
-                    hold_states<N, false>(th, dl, aa[m], gnk, unused);
+                    hold_states<N, false>(th, dl, aa[m], hs, m, gnk, unused);
                 } else {
 #pragma unroll
                     for (int k = 0; k < NP; ++k) gnk[k] = hold_gain2(dl, mul2(dl2, th.Araw[k]), aa[m][k], th.invA[k]);
@@ -677,7 +723,7 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
             float2 gnk[NP], dgk[NP];
             if constexpr (ZOH) {
                 if constexpr (fast) {
-                    hold_states<N, true>(th, dl, aa[m], gnk, dgk);
+                    hold_states<N, true>(th, dl, aa[m], hs, m, gnk, dgk);
                 } else {
 #pragma unroll
                     for (int k = 0; k < NP; ++k) {
@@ -787,7 +833,10 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
 // one sweep of the thread's direction: forward (ADJ false) or adjoint
 template <int N, bool ZOH, bool FAST, bool ADJ>
 __device__ __forceinline__ void bwd_sweep(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
-    if constexpr (ADJ) {
+    if constexpr ((VIMSCAN_BWD_RTDIR >> (ZOH ? 0 : 1)) & 1) {
+        if constexpr (ADJ) bwd_adjoint<N, -1, ZOH, FAST>(p, sm, th);
+        else bwd_forward<N, -1, ZOH, FAST>(p, sm, th);
+    } else if constexpr (ADJ) {
         if (th.dir == 0) bwd_adjoint<N, 0, ZOH, FAST>(p, sm, th);
         else bwd_adjoint<N, 1, ZOH, FAST>(p, sm, th);
     } else {
