@@ -20,7 +20,8 @@
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous and
- *     row-major, 16-byte aligned.  The library allocates no device memory and keeps
+ *     row-major, 16-byte aligned (vim_scan_bidir_host takes its activations from
+ *     host memory; see there).  The library allocates no device memory and keeps
  *     no state between calls; scratch memory is the caller's workspace.
  *   - `dt` is the element type of u, delta, z, B, C, ys and y (fp32 or bf16).  A, D
  *     and delta_bias are always fp32.  Arithmetic is fp32 with the state h held in
@@ -383,6 +384,49 @@ vim_status vim_scan_bidir_noalloc(const void *u, const void *delta, const void *
                                   const float *A, const float *D, const float *delta_bias,
                                   void *y, int batch, int L, int d_inner, int d_state,
                                   vim_dtype dt, cudaStream_t stream);
+
+/*
+ * vim_scan_bidir for activations in HOST memory: the same operation, flags and
+ * parameters as vim_scan_bidir_ex without the convolution front, with u, delta, z,
+ * B, C read from the host and y written to the host.  The pages have no counterpart
+ * to this call; it is a packaging variant for callers whose activations live on the
+ * host, so that the transfers are part of the library's pipeline.
+ *
+ *   u, delta, z, B, C, y : HOST pointers, shaped as in vim_scan_bidir (z may be NULL;
+ *                 bc_dir_stride as there, counted in elements of the host B and C).
+ *                 Page-locked memory (cudaHostAlloc, cudaHostRegister) lets the copies
+ *                 run asynchronously and overlap; pageable memory gives the same result
+ *                 but the driver stages those copies and the call waits for them.
+ *   A, D, delta_bias : DEVICE pointers (the module's parameters stay resident).
+ *   slices      : the batch is cut into this many pieces (at most batch; >= 1).  Piece k
+ *                 goes to the device on `upload`, is scanned on `stream` and its y comes
+ *                 back on `download`, so that piece k+1's upload and piece k-1's
+ *                 download run while piece k is scanned.  Results do not depend on
+ *                 `slices` for sequences longer than 256 tokens; shorter ones may take
+ *                 a different chunking per piece and differ in rounding.
+ *   workspace   : DEVICE scratch of vim_scan_host_workspace_bytes(batch, L, d_inner,
+ *                 d_state, dt, slices, bc_dir_stride > 0) bytes, 256-byte aligned: two
+ *                 staging sets of one piece each, and the scan's summaries.
+ *   upload, download : streams for the copies (NULL: `stream` itself, and no overlap).
+ *                 Use two streams created with cudaStreamNonBlocking that nothing else
+ *                 uses during the call.
+ *
+ * Ordering: the copies start after the work queued on `stream` before the call, and
+ * `stream` reaches the end of the call when the last piece of y is on the host: wait
+ * on `stream` (an event or a synchronize) before reading y.  The host buffers must
+ * stay valid and unmodified until then.  The call creates and releases its own CUDA
+ * events and allocates no memory.  A failed check launches and copies nothing; a CUDA
+ * failure part-way (VIM_ERR_CUDA) may leave y partly written.
+ */
+vim_status vim_scan_bidir_host(const void *u, const void *delta, const void *z, const void *B,
+                               const void *C, int64_t bc_dir_stride, const float *A, const float *D,
+                               const float *delta_bias, void *y, int batch, int L, int d_inner,
+                               int d_state, vim_dtype dt, unsigned flags, int slices, void *workspace,
+                               size_t workspace_bytes, cudaStream_t stream, cudaStream_t upload,
+                               cudaStream_t download);
+/* Workspace bytes of vim_scan_bidir_host (0 for invalid arguments or an empty problem). */
+size_t vim_scan_host_workspace_bytes(int batch, int L, int d_inner, int d_state, vim_dtype dt, int slices,
+                                     int two_bc);
 
 /*
  * Workspace bytes the scan entry points need (0 when none).  which = 0 for

@@ -41,6 +41,7 @@ def test_header_declares_the_boundary():
                           "vim_block_scan", "vim_block_workspace_bytes",
                           "vmamba_cross_scan4_bwd", "vmamba_cross_scan4_bwd_workspace_bytes",
                           "vmamba_cross_scan4_bwd_ex",
+                          "vim_scan_bidir_host", "vim_scan_host_workspace_bytes",
                           "vim_scan_workspace_bytes", "vim_status_string"}, names
 
 
@@ -109,6 +110,47 @@ def test_bidir_rejects(vs):
     assert bidir(vs, L=4097, ws=None) == vs.VIM_ERR_WORKSPACE
     assert bidir(vs, L=4097, ws=FAKE, ws_bytes=16) == vs.VIM_ERR_WORKSPACE
     assert bidir(vs, L=4097, ws=FAKE + 16, ws_bytes=1 << 40) == vs.VIM_ERR_WORKSPACE
+
+
+def host(vs, **kw):
+    """vim_scan_bidir_host on fake addresses; every case below fails a host check (or is
+    an empty problem), before any CUDA call."""
+    a = dict(u=FAKE, delta=FAKE, z=FAKE, B=FAKE, C=FAKE, stride=0, A=FAKE, D=FAKE, bias=FAKE, y=FAKE,
+             batch=8, L=4097, Di=384, N=16, dt=vs.VIM_BF16, flags=0, slices=8, ws=FAKE, ws_bytes=1 << 40)
+    a.update(kw)
+    return vs.lib.vim_scan_bidir_host(a["u"], a["delta"], a["z"], a["B"], a["C"], a["stride"], a["A"], a["D"],
+                                      a["bias"], a["y"], a["batch"], a["L"], a["Di"], a["N"], a["dt"], a["flags"],
+                                      a["slices"], a["ws"], a["ws_bytes"], None, None, None)
+
+
+def test_host_entry_rejects(vs):
+    assert host(vs, u=None) == vs.VIM_ERR_INVALID_ARG
+    assert host(vs, y=None) == vs.VIM_ERR_INVALID_ARG
+    assert host(vs, A=None) == vs.VIM_ERR_INVALID_ARG
+    assert host(vs, D=FAKE + 2) == vs.VIM_ERR_INVALID_ARG             # parameters are fp32 on the device
+    assert host(vs, slices=0) == vs.VIM_ERR_INVALID_ARG
+    assert host(vs, stride=-1) == vs.VIM_ERR_INVALID_ARG
+    assert host(vs, flags=4) == vs.VIM_ERR_INVALID_ARG
+    assert host(vs, N=3) == vs.VIM_ERR_UNSUPPORTED
+    assert host(vs, Di=12) == vs.VIM_ERR_UNSUPPORTED
+    assert host(vs, ws=None) == vs.VIM_ERR_WORKSPACE
+    assert host(vs, ws_bytes=1024) == vs.VIM_ERR_WORKSPACE
+    assert host(vs, ws=FAKE + 16) == vs.VIM_ERR_WORKSPACE
+    assert host(vs, batch=0, ws=None) == vs.VIM_OK                    # empty: nothing to do
+    assert host(vs, L=0, u=None, ws=None) == vs.VIM_OK
+
+
+def test_host_workspace_bytes(vs):
+    f = vs.vim_scan_host_workspace_bytes
+    one = f(8, 4097, 384, 16, vs.VIM_BF16, 8, False)
+    act = 4097 * 384 * 2                                  # one batch item of u (bf16)
+    assert one % 256 == 0 and one >= 2 * (4 * act + 2 * 4097 * 16 * 2) + vs.vim_scan_workspace_bytes(0, 1, 4097, 0, 384, 16)
+    assert f(8, 4097, 384, 16, vs.VIM_BF16, 8, True) > one            # two copies of B and C
+    assert f(8, 4097, 384, 16, vs.VIM_BF16, 64, False) == one         # at most one piece per batch item
+    assert f(8, 4097, 384, 16, vs.VIM_BF16, 2, False) > one           # larger pieces
+    assert f(8, 4097, 384, 16, vs.VIM_BF16, 0, False) == 0
+    assert f(0, 4097, 384, 16, vs.VIM_BF16, 8, False) == 0
+    assert f(8, 4097, 384, 3, vs.VIM_BF16, 8, False) == 0
 
 
 def bwd(vs, **kw):

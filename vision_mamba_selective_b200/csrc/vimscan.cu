@@ -5,6 +5,7 @@
 // synchronises the stream.
 #include "vimscan.h"
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -291,6 +292,141 @@ vim_status vim_scan_bidir_noalloc(const void *u, const void *delta, const void *
     }
     return vim_scan_bidir(u, delta, z, B, C, bc_dir_stride, A, D, delta_bias, y, batch, L, d_inner,
                           d_state, dt, scratch, VIM_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+}  // extern "C"
+
+// ----------------------------------------------------------------------------
+// vim_scan_bidir over host activations (declared in vimscan.h)
+// ----------------------------------------------------------------------------
+namespace {
+
+// the batch cut into `slices` pieces of sb items (the last one may be shorter), and the
+// workspace: two staging sets (u, delta, z, y, B, C of one slice each) and the scan's
+// own summaries for the largest slice
+struct HostPlan {
+    int slices, sb;
+    size_t act, bc;        // elements of one slice's u (and delta, z, y) and of one B (or C) copy
+    size_t o_u, o_d, o_z, o_y, o_B, o_C, set_bytes, o_scan, scan_bytes, total;
+};
+
+HostPlan host_plan(int batch, int L, int Di, int N, vim_dtype dt, int slices, bool two_bc) {
+    HostPlan h;
+    std::memset(&h, 0, sizeof(h));
+    h.slices = std::max(1, std::min(slices, batch));
+    h.sb = (batch + h.slices - 1) / h.slices;
+    h.slices = (batch + h.sb - 1) / h.sb;
+    const size_t e = elem_size(dt);
+    h.act = (size_t)h.sb * L * Di;
+    h.bc = (size_t)h.sb * L * N;
+    size_t o = 0;
+    auto take = [&](size_t bytes) { const size_t at = o; o += round_up(bytes); return at; };
+    h.o_u = take(h.act * e);
+    h.o_d = take(h.act * e);
+    h.o_z = take(h.act * e);
+    h.o_y = take(h.act * e);
+    h.o_B = take(h.bc * e * (two_bc ? 2 : 1));
+    h.o_C = take(h.bc * e * (two_bc ? 2 : 1));
+    h.set_bytes = o;
+    h.o_scan = 2 * h.set_bytes;
+    const int last = batch - (h.slices - 1) * h.sb;
+    h.scan_bytes = std::max(summary_bytes(h.sb, L, Di, N), summary_bytes(last, L, Di, N));
+    h.total = h.o_scan + round_up(h.scan_bytes);
+    return h;
+}
+
+struct Events {
+    cudaEvent_t e[7] = {};   // entry, uploaded[2], scanned[2], downloaded[2]
+    bool ok = true;
+    Events() {
+        for (auto &x : e)
+            if (cudaEventCreateWithFlags(&x, cudaEventDisableTiming) != cudaSuccess) { x = nullptr; ok = false; }
+    }
+    ~Events() {   // pending records complete on their own; destroying them here is allowed
+        for (auto &x : e)
+            if (x) cudaEventDestroy(x);
+    }
+};
+
+}  // namespace
+
+extern "C" {
+
+size_t vim_scan_host_workspace_bytes(int batch, int L, int d_inner, int d_state, vim_dtype dt, int slices,
+                                     int two_bc) {
+    if (check_common(batch, L, d_inner, d_state, dt) != VIM_OK || slices < 1) return 0;
+    if (batch == 0 || L == 0 || d_inner == 0) return 0;
+    return host_plan(batch, L, d_inner, d_state, dt, slices, two_bc != 0).total;
+}
+
+vim_status vim_scan_bidir_host(const void *u, const void *delta, const void *z, const void *B,
+                               const void *C, int64_t bc_dir_stride, const float *A, const float *D,
+                               const float *delta_bias, void *y, int batch, int L, int d_inner,
+                               int d_state, vim_dtype dt, unsigned flags, int slices, void *workspace,
+                               size_t workspace_bytes, cudaStream_t stream, cudaStream_t upload,
+                               cudaStream_t download) {
+    vim_status st = check_common(batch, L, d_inner, d_state, dt);
+    if (st != VIM_OK) return st;
+    if (bc_dir_stride < 0 || slices < 1 || (flags & ~kKnownFlags)) return VIM_ERR_INVALID_ARG;
+    if (batch == 0 || L == 0 || d_inner == 0) return VIM_OK;
+    if (!u || !delta || !B || !C || !A || !D || !delta_bias || !y) return VIM_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(D) |
+         reinterpret_cast<uintptr_t>(delta_bias)) % 4)
+        return VIM_ERR_INVALID_ARG;
+    const bool two = bc_dir_stride > 0;
+    const HostPlan hp = host_plan(batch, L, d_inner, d_state, dt, slices, two);
+    if (!workspace || workspace_bytes < hp.total) return VIM_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return VIM_ERR_WORKSPACE;
+    if (!upload) upload = stream;
+    if (!download) download = stream;
+
+    Events ev;
+    if (!ev.ok) return VIM_ERR_CUDA;
+    cudaEvent_t entry = ev.e[0], *up = ev.e + 1, *sc = ev.e + 3, *dn = ev.e + 5;
+    const size_t e = elem_size(dt);
+    char *ws = static_cast<char *>(workspace);
+    const char *hu = static_cast<const char *>(u), *hd = static_cast<const char *>(delta),
+               *hz = static_cast<const char *>(z), *hB = static_cast<const char *>(B),
+               *hC = static_cast<const char *>(C);
+    char *hy = static_cast<char *>(y);
+    auto ok = [](cudaError_t r) { return r == cudaSuccess; };
+    // the copy streams start after everything queued on `stream` before this call
+    if (!ok(cudaEventRecord(entry, stream)) || !ok(cudaStreamWaitEvent(upload, entry, 0)) ||
+        !ok(cudaStreamWaitEvent(download, entry, 0)))
+        return VIM_ERR_CUDA;
+    for (int k = 0; k < hp.slices; ++k) {
+        const int set = k & 1, b0 = k * hp.sb, nb = std::min(hp.sb, batch - b0);
+        char *base = ws + set * hp.set_bytes;
+        const size_t act = (size_t)nb * L * d_inner * e, bc = (size_t)nb * L * d_state * e;
+        const size_t a0 = (size_t)b0 * L * d_inner * e, c0 = (size_t)b0 * L * d_state * e;
+        // slice k reuses the set of slice k - 2 once that slice's y has left the device
+        if (k >= 2 && !ok(cudaStreamWaitEvent(upload, dn[set], 0))) return VIM_ERR_CUDA;
+        bool good = ok(cudaMemcpyAsync(base + hp.o_u, hu + a0, act, cudaMemcpyHostToDevice, upload)) &&
+                    ok(cudaMemcpyAsync(base + hp.o_d, hd + a0, act, cudaMemcpyHostToDevice, upload)) &&
+                    (!z || ok(cudaMemcpyAsync(base + hp.o_z, hz + a0, act, cudaMemcpyHostToDevice, upload))) &&
+                    ok(cudaMemcpyAsync(base + hp.o_B, hB + c0, bc, cudaMemcpyHostToDevice, upload)) &&
+                    ok(cudaMemcpyAsync(base + hp.o_C, hC + c0, bc, cudaMemcpyHostToDevice, upload));
+        if (good && two) {
+            const size_t s0 = (size_t)bc_dir_stride * e;
+            good = ok(cudaMemcpyAsync(base + hp.o_B + bc, hB + s0 + c0, bc, cudaMemcpyHostToDevice, upload)) &&
+                   ok(cudaMemcpyAsync(base + hp.o_C + bc, hC + s0 + c0, bc, cudaMemcpyHostToDevice, upload));
+        }
+        if (!good || !ok(cudaEventRecord(up[set], upload)) || !ok(cudaStreamWaitEvent(stream, up[set], 0)))
+            return VIM_ERR_CUDA;
+        st = bidir_impl(base + hp.o_u, nullptr, nullptr, base + hp.o_d, z ? base + hp.o_z : nullptr,
+                        base + hp.o_B, base + hp.o_C, two ? (int64_t)nb * L * d_state : 0, A, D, delta_bias,
+                        base + hp.o_y, nb, L, d_inner, d_state, dt, flags, ws + hp.o_scan, hp.scan_bytes, stream,
+                        nullptr);
+        if (st != VIM_OK) return st;
+        if (!ok(cudaEventRecord(sc[set], stream)) || !ok(cudaStreamWaitEvent(download, sc[set], 0)) ||
+            !ok(cudaMemcpyAsync(hy + a0, base + hp.o_y, act, cudaMemcpyDeviceToHost, download)) ||
+            !ok(cudaEventRecord(dn[set], download)))
+            return VIM_ERR_CUDA;
+    }
+    // `stream` reaches the end of this call once the last slice's y is on the host
+    const int last = (hp.slices - 1) & 1;
+    if (!ok(cudaStreamWaitEvent(stream, dn[last], 0))) return VIM_ERR_CUDA;
+    return VIM_OK;
 }
 
 }  // extern "C"

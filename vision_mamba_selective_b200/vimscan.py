@@ -76,6 +76,11 @@ lib.vim_scan_bidir_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, 
                                        _i, _i, _i, _i, _i, _vp]
 lib.vim_scan_bidir_noalloc.restype = _i
 VIM_NOALLOC_SCRATCH_BYTES = 8 << 20
+lib.vim_scan_bidir_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
+                                    _i, _i, _i, _i, _i, _u, _i, _vp, _sz, _vp, _vp, _vp]
+lib.vim_scan_bidir_host.restype = _i
+lib.vim_scan_host_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+lib.vim_scan_host_workspace_bytes.restype = _sz
 lib.cross_merge4.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]
 lib.cross_merge4.restype = _i
 lib.vim_scan_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
@@ -447,4 +452,73 @@ def cross_merge4(ys, z, H, W, *, y=None, stream=None):
     st = lib.cross_merge4(pys, pz, py, batch, H, W, Ch, dt, _stream(stream))
     if st != VIM_OK:
         raise VimScanError(st, "cross_merge4")
+    return y
+
+
+def vim_scan_host_workspace_bytes(batch, L, d_inner, d_state, dtype_code, slices, two_bc):
+    return int(lib.vim_scan_host_workspace_bytes(batch, L, d_inner, d_state, dtype_code, slices, int(bool(two_bc))))
+
+
+_copy_streams = {}
+
+
+def _host_streams(device):
+    """Two non-blocking streams per device for the host entry's uploads and downloads."""
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    if idx not in _copy_streams:
+        _copy_streams[idx] = (torch.cuda.Stream(idx), torch.cuda.Stream(idx))
+    return _copy_streams[idx]
+
+
+def vim_scan_bidir_host(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride=0, slices=4,
+                        workspace=None, stream=None, upload=None, download=None, zoh=False):
+    """vim_scan_bidir for activations in host memory; see include/vimscan.h.
+
+    u, delta, z, B, C: CPU tensors shaped as for vim_scan_bidir (pinned memory lets the
+    copies overlap the scan); A, D, delta_bias: CUDA tensors on the current device.
+    Returns y, a CPU tensor (pinned when allocated here), complete once ``stream``
+    (default: the current stream) has reached the end of the call.
+    """
+    if not all(isinstance(t, torch.Tensor) for t in (u, delta, B, C)):
+        raise TypeError("vim_scan_bidir_host: u, delta, B and C must be tensors")
+    batch, L, Di = u.shape
+    N = B.shape[-1]
+    dt = _dtype_code(u)
+    act = (batch, L, Di)
+    bc = _bc_rule(batch, L, N, bc_dir_stride)
+    if y is None:
+        y = torch.empty(act, dtype=u.dtype, pin_memory=True)
+    for name, t, rule in (("u", u, act), ("delta", delta, act), ("z", z, act), ("B", B, bc), ("C", C, bc),
+                          ("y", y, act)):
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor) or t.device.type != "cpu":
+            raise TypeError(f"vim_scan_bidir_host: {name} must be a CPU tensor")
+        if t.dtype != u.dtype:
+            raise TypeError(f"vim_scan_bidir_host: {name} must be {u.dtype}, got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"vim_scan_bidir_host: {name} must be contiguous")
+        if rule[0] == "numel":
+            if t.numel() < rule[1] or t.dim() == 0 or t.shape[-1] != rule[2]:
+                raise ValueError(f"vim_scan_bidir_host: {name} has shape {tuple(t.shape)}; it needs at least "
+                                 f"{rule[1]} elements with last dimension {rule[2]}")
+        elif t.shape != rule:
+            raise ValueError(f"vim_scan_bidir_host: {name} has shape {tuple(t.shape)}, expected {rule}")
+    f32 = torch.float32
+    pA, pD, pbias = _ptrs("vim_scan_bidir_host", A, [("A", A, f32, (2, Di, N)), ("D", D, f32, (2, Di)),
+                                                     ("delta_bias", delta_bias, f32, (2, Di))])
+    dev = A.device
+    nbytes = vim_scan_host_workspace_bytes(batch, L, Di, N, dt, slices, bc_dir_stride > 0)
+    ws, ws_bytes = _workspace(nbytes, workspace, dev)
+    if upload is None or download is None:
+        up, down = _host_streams(dev)
+        upload = upload or up
+        download = download or down
+    st = lib.vim_scan_bidir_host(
+        u.data_ptr(), delta.data_ptr(), None if z is None else z.data_ptr(), B.data_ptr(), C.data_ptr(),
+        int(bc_dir_stride), pA, pD, pbias, y.data_ptr(), batch, L, Di, N, dt,
+        VIM_FLAG_ZOH_EXACT if zoh else 0, int(slices), None if ws is None else ws.data_ptr(), ws_bytes,
+        _stream(stream), upload.cuda_stream, download.cuda_stream)
+    if st != VIM_OK:
+        raise VimScanError(st, "vim_scan_bidir_host")
     return y
