@@ -316,24 +316,26 @@ constexpr bool bc_vectorizable() { return (N * sizeof(T)) % 16 == 0; }
 // converted to fp32, into the slot.
 // Rows past the end of the chunk and channels past d_inner are zero-filled, so that
 // they act as no-op tokens.
-template <typename T, int N, bool VEC_BC, bool CONV = false, bool ZOH = false, bool DT = false>
+template <typename T, int N, bool VEC_BC, bool CONV = false, bool ZOH = false, bool DT = false, int NTHR = kThreads>
 struct Stager {
     using S = Stage<T, N, CONV>;
     static constexpr int V = Vec<T>::n;                 // elements per 16-byte piece
     static constexpr int kRowPieces = kDC / V;          // pieces per u/delta row
-    static constexpr int kUVRep = kTile * kRowPieces / kThreads;   // pieces per thread per tensor
+    static constexpr int kUVRep = kTile * kRowPieces / NTHR;   // pieces per thread per tensor
     static constexpr int kBCRow = VEC_BC ? (int)(N * sizeof(T) / 16) : N;   // units per B/C row
     static constexpr int kBCUnits = 4 * kTile * kBCRow;
-    static constexpr int kBCPer = (kBCUnits + kThreads - 1) / kThreads;
-    static_assert(kTile * kRowPieces % kThreads == 0, "u/delta pieces must split evenly");
+    static constexpr int kBCPer = (kBCUnits + NTHR - 1) / NTHR;
+    static_assert(kTile * kRowPieces % NTHR == 0, "u/delta pieces must split evenly");
+    static_assert(NTHR >= kTile, "one thread per row of the step input");
 
     const PairArgs &p;
     const int b, t0, tc, d0;
+    const int tid;   // this thread's index among the NTHR staging threads
     uint4 pre_v[VEC_BC ? kBCPer : 1];
     float pre_s[VEC_BC ? 1 : kBCPer];
 
-    __device__ Stager(const PairArgs &pa, int b_, int t0_, int tc_, int d0_)
-        : p(pa), b(b_), t0(t0_), tc(tc_), d0(d0_) {}
+    __device__ Stager(const PairArgs &pa, int b_, int t0_, int tc_, int d0_, int tid_)
+        : p(pa), b(b_), t0(t0_), tc(tc_), d0(d0_), tid(tid_) {}
 
     __device__ int rows_of(int j) const { return min(kTile, tc - j * kTile); }
 
@@ -352,7 +354,7 @@ struct Stager {
             const int rows = rows_of(j);
 #pragma unroll
             for (int m = 0; m < kUVRep; ++m) {
-                const int li = threadIdx.x + m * kThreads;
+                const int li = tid + m * NTHR;
                 const int v = li % kRowPieces, r = li / kRowPieces;
                 const int ch = d0 + v * V;
                 const bool ok = r < rows && ch < p.Di;
@@ -371,8 +373,8 @@ struct Stager {
             if constexpr (DT) {
                 // the step input of each row (one value per token; the delta area holds
                 // them as floats), NaN past the data: delta_at turns it into Delta = 0
-                if (threadIdx.x < kTile) {
-                    const int r = threadIdx.x;
+                if (tid < kTile) {
+                    const int r = tid;
                     float v = __int_as_float(0x7fc00000);
                     if (r < rows) v = p.dt_in[(size_t)dir * p.batch * p.L + (size_t)b * p.L + position(p, t0 + j * kTile + r)];
                     reinterpret_cast<float *>(S::uv(slot, dir, 1))[r] = v;
@@ -381,7 +383,7 @@ struct Stager {
             if constexpr (CONV) {
                 // x rows -1 .. kTile of the tile (the convolution's neighbours), zero
                 // outside the sequence (the convolution's zero padding)
-                for (int li = threadIdx.x; li < S::kURows * kRowPieces; li += kThreads) {
+                for (int li = tid; li < S::kURows * kRowPieces; li += NTHR) {
                     const int v = li % kRowPieces, rr = li / kRowPieces;
                     const int ch = d0 + v * V;
                     const int t = t0 + j * kTile + rr - 1;
@@ -399,7 +401,7 @@ struct Stager {
     __device__ void load_bc(int jf, int jb) {
 #pragma unroll
         for (int k = 0; k < kBCPer; ++k) {
-            const int i = threadIdx.x + k * kThreads;
+            const int i = tid + k * NTHR;
             const int part = i % kBCRow;
             const int r = (i / kBCRow) % kTile;
             const int which = (i / (kBCRow * kTile)) % 2;
@@ -426,7 +428,7 @@ struct Stager {
         constexpr bool LU = lu_mode<T, ZOH>();
 #pragma unroll
         for (int k = 0; k < kBCPer; ++k) {
-            const int i = threadIdx.x + k * kThreads;
+            const int i = tid + k * NTHR;
             if (i >= kBCUnits) continue;
             const int part = i % kBCRow;
             const int r = (i / kBCRow) % kTile;
@@ -668,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMin
     const bool fast = __all_sync(0xffffffffu, prm.structured);
 
     // the forward direction walks tiles nT-1 .. 0, the backward one 0 .. nT-1
-    Stager<T, N, VEC_BC, CONV, ZOH, DT> st(p, b, t0, tc, d0);
+    Stager<T, N, VEC_BC, CONV, ZOH, DT> st(p, b, t0, tc, d0, threadIdx.x);
     st.issue(smem, nT - 1, 0);
     st.load_bc(nT - 1, 0);
     st.store_bc(smem);
@@ -919,16 +921,21 @@ __device__ __forceinline__ void main_tile(bool second, float2 (&h)[N / 2], float
 // second pair of the cross-scan), applies silu(z) and stores 16 or 32 bytes; the first
 // pair of the cross-scan stores its ungated fp32 sum instead.  z and partial_in are
 // loaded into registers at the start of the step, so their latency hides behind it.
-template <typename T, bool PIN>
+template <typename T, bool PIN, int NTHR = kThreads>
 struct Finisher {
     static constexpr int kG = 8;                                    // channels per vector
     static constexpr int kZ = kG * (int)sizeof(T) / 16;             // uint4 of z per vector
-    uint4 z[2][kZ];
-    float4 pin[2][PIN ? 2 : 1];
+    static constexpr int kItems = kTile * (kDC / kG);               // vectors per tile
+    static constexpr int kIPT = kItems / NTHR;                      // vectors per thread per tile
+    static_assert(kItems % NTHR == 0, "a tile's vectors split evenly over the finishing threads");
+    uint4 z[2][kIPT][kZ];
+    float4 pin[2][kIPT][PIN ? 2 : 1];
     int ntiles, tile[2];
+    int tid;   // this thread's index among the NTHR finishing threads
 
-    __device__ int row() const { return threadIdx.x / (kDC / kG); }
-    __device__ int group() const { return threadIdx.x % (kDC / kG); }
+    __device__ explicit Finisher(int tid_) : ntiles(0), tid(tid_) {}
+    __device__ int row(int m) const { return (tid + m * NTHR) / (kDC / kG); }
+    __device__ int group(int m) const { return (tid + m * NTHR) % (kDC / kG); }
 
     // the tiles completed by step s (none before the middle of the chunk)
     __device__ void plan(int s, int nT) {
@@ -941,23 +948,26 @@ struct Finisher {
 
     template <class ST>
     __device__ void prefetch(const ST &st, const PairArgs &p) {
-        const int r = row(), ch = st.d0 + group() * kG;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             if (i >= ntiles) break;
             const int j = tile[i];
-            if (r >= st.rows_of(j) || ch >= p.Di) continue;
-            const size_t off = st.row_off(j, r, ch);
-            if (p.z) {
-                const uint4 *zs = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.z) + off);
 #pragma unroll
-                for (int q = 0; q < kZ; ++q)
-                    if (sizeof(T) == 2 || ch + 4 * q < p.Di) z[i][q] = zs[q];
-            }
-            if constexpr (PIN) {
-                const float4 *ps = reinterpret_cast<const float4 *>(p.partial_in + off);
-                pin[i][0] = ps[0];
-                if (ch + 4 < p.Di) pin[i][1] = ps[1];
+            for (int m = 0; m < kIPT; ++m) {
+                const int r = row(m), ch = st.d0 + group(m) * kG;
+                if (r >= st.rows_of(j) || ch >= p.Di) continue;
+                const size_t off = st.row_off(j, r, ch);
+                if (p.z) {
+                    const uint4 *zs = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.z) + off);
+#pragma unroll
+                    for (int q = 0; q < kZ; ++q)
+                        if (sizeof(T) == 2 || ch + 4 * q < p.Di) z[i][m][q] = zs[q];
+                }
+                if constexpr (PIN) {
+                    const float4 *ps = reinterpret_cast<const float4 *>(p.partial_in + off);
+                    pin[i][m][0] = ps[0];
+                    if (ch + 4 < p.Di) pin[i][m][1] = ps[1];
+                }
             }
         }
     }
@@ -965,48 +975,52 @@ struct Finisher {
     template <class ST>
     __device__ void finish(const ST &st, const PairArgs &p, const float *ybuf,
                            const float *ymid) const {
-        const int r = row(), cl = group() * kG, ch = st.d0 + cl;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             if (i >= ntiles) break;
             const int j = tile[i];
-            if (r >= st.rows_of(j) || ch >= p.Di) continue;
-            float acc[kG];
-            add_f32<kG, false>(acc, ybuf + (size_t)(j * kTile + r) * kDC + cl);
-            if (ntiles == 1) add_f32<kG, true>(acc, ymid + r * kDC + cl);
-            if constexpr (PIN) {
-                acc[0] += pin[i][0].x; acc[1] += pin[i][0].y; acc[2] += pin[i][0].z; acc[3] += pin[i][0].w;
-                acc[4] += pin[i][1].x; acc[5] += pin[i][1].y; acc[6] += pin[i][1].z; acc[7] += pin[i][1].w;
-            }
-            const size_t off = st.row_off(j, r, ch);
-            const bool whole = ch + kG <= p.Di;   // fp32 channel counts may end half-way
-            if (p.partial_out) {
-                float4 *po = reinterpret_cast<float4 *>(p.partial_out + off);
-                po[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-                if (whole) po[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-                continue;
-            }
-            if (p.z) {
-                float zf[kG];
-                if constexpr (sizeof(T) == 2) {
-                    unpack16(z[i][0], zf);
-                } else {
-                    float a4[4], b4[4];
-                    unpack16(z[i][0], a4);
-                    unpack16(z[i][kZ - 1], b4);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) { zf[e] = a4[e]; zf[4 + e] = b4[e]; }
+            for (int m = 0; m < kIPT; ++m) {
+                const int r = row(m), cl = group(m) * kG, ch = st.d0 + cl;
+                if (r >= st.rows_of(j) || ch >= p.Di) continue;
+                float acc[kG];
+                add_f32<kG, false>(acc, ybuf + (size_t)(j * kTile + r) * kDC + cl);
+                if (ntiles == 1) add_f32<kG, true>(acc, ymid + r * kDC + cl);
+                if constexpr (PIN) {
+                    const float4 a = pin[i][m][0], b = pin[i][m][PIN ? 1 : 0];
+                    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+                    acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
                 }
+                const size_t off = st.row_off(j, r, ch);
+                const bool whole = ch + kG <= p.Di;   // fp32 channel counts may end half-way
+                if (p.partial_out) {
+                    float4 *po = reinterpret_cast<float4 *>(p.partial_out + off);
+                    po[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                    if (whole) po[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+                    continue;
+                }
+                if (p.z) {
+                    float zf[kG];
+                    if constexpr (sizeof(T) == 2) {
+                        unpack16(z[i][m][0], zf);
+                    } else {
+                        float a4[4], b4[4];
+                        unpack16(z[i][m][0], a4);
+                        unpack16(z[i][m][kZ - 1], b4);
 #pragma unroll
-                for (int e = 0; e < kG; ++e) acc[e] *= silu(zf[e]);
-            }
-            uint4 *yo = reinterpret_cast<uint4 *>(static_cast<T *>(p.y) + off);
-            if constexpr (sizeof(T) == 2) {
-                yo[0] = pack16(acc);
-            } else {
-                float a4[4] = {acc[0], acc[1], acc[2], acc[3]}, b4[4] = {acc[4], acc[5], acc[6], acc[7]};
-                yo[0] = pack16(a4);
-                if (whole) yo[1] = pack16(b4);
+                        for (int e = 0; e < 4; ++e) { zf[e] = a4[e]; zf[4 + e] = b4[e]; }
+                    }
+#pragma unroll
+                    for (int e = 0; e < kG; ++e) acc[e] *= silu(zf[e]);
+                }
+                uint4 *yo = reinterpret_cast<uint4 *>(static_cast<T *>(p.y) + off);
+                if constexpr (sizeof(T) == 2) {
+                    yo[0] = pack16(acc);
+                } else {
+                    float a4[4] = {acc[0], acc[1], acc[2], acc[3]}, b4[4] = {acc[4], acc[5], acc[6], acc[7]};
+                    yo[0] = pack16(a4);
+                    if (whole) yo[1] = pack16(b4);
+                }
             }
         }
     }
@@ -1030,7 +1044,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
     prm.template load<lu_mode<T, ZOH>()>(p, dir, d);
     const bool fast = __all_sync(0xffffffffu, prm.structured);
 
-    Stager<T, N, VEC_BC, CONV, ZOH, DT> st(p, b, t0, tc, d0);
+    Stager<T, N, VEC_BC, CONV, ZOH, DT> st(p, b, t0, tc, d0, threadIdx.x);
     st.issue(smem, 0, nT - 1);
     st.load_bc(0, nT - 1);
 
@@ -1054,7 +1068,27 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
     cp_async_wait_all();
     __syncthreads();
 
-    Finisher<T, PIN> fin;
+    Finisher<T, PIN> fin(threadIdx.x);
+    // one step of the recurrence warps: tile j = s (forward) or nT-1-s (backward) from
+    // the slot `cur`; the first visitor of a tile stores its partial, the second adds to
+    // it; when both come in the same step (the middle tile) the backward one writes to
+    // ymid instead
+    auto recur = [&](int s, char *cur) {
+        const int j = dir ? nT - 1 - s : s;
+        const int twice = 2 * s - (nT - 1);
+        float *ypart = (twice == 0 && dir == 1) ? ymid + dl : ybuf + (size_t)j * kTile * kDC + dl;
+        if (!prm.valid) return;
+        const T *su = S::uv(cur, dir, 0), *sd = S::uv(cur, dir, 1);
+        const float *sB = S::bc(cur, dir, 0), *sC = S::bc(cur, dir, 1);
+        const bool second = twice > 0;
+        if (dir == 0) {
+            if (fast) main_tile<T, N, true, false, CONV, ZOH, DT>(second, h, dprev, prm, dl, su, sd, sB, sC, ypart);
+            else main_tile<T, N, false, false, CONV, ZOH, DT>(second, h, dprev, prm, dl, su, sd, sB, sC, ypart);
+        } else {
+            if (fast) main_tile<T, N, true, true, CONV, ZOH, DT>(second, h, dprev, prm, dl, su, sd, sB, sC, ypart);
+            else main_tile<T, N, false, true, CONV, ZOH, DT>(second, h, dprev, prm, dl, su, sd, sB, sC, ypart);
+        }
+    };
     for (int s = 0; s < nT; ++s) {
         char *cur = smem + (s & 1) * kSlot;
         char *nxt = smem + ((s + 1) & 1) * kSlot;
@@ -1064,24 +1098,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
         }
         fin.plan(s, nT);
         fin.prefetch(st, p);
-        // the forward direction visits tile j at step j, the backward one at nT-1-j:
-        // the first visitor stores its partial, the second adds to it; when both come
-        // in the same step (the middle tile) the backward one writes to ymid instead
-        const int j = dir ? nT - 1 - s : s;
-        const int twice = 2 * s - (nT - 1);
-        float *ypart = (twice == 0 && dir == 1) ? ymid + dl : ybuf + (size_t)j * kTile * kDC + dl;
-        if (prm.valid) {
-            const T *su = S::uv(cur, dir, 0), *sd = S::uv(cur, dir, 1);
-            const float *sB = S::bc(cur, dir, 0), *sC = S::bc(cur, dir, 1);
-            const bool second = twice > 0;
-            if (dir == 0) {
-                if (fast) main_tile<T, N, true, false, CONV, ZOH, DT>(second, h, dprev, prm, dl, su, sd, sB, sC, ypart);
-                else main_tile<T, N, false, false, CONV, ZOH, DT>(second, h, dprev, prm, dl, su, sd, sB, sC, ypart);
-            } else {
-                if (fast) main_tile<T, N, true, true, CONV, ZOH, DT>(second, h, dprev, prm, dl, su, sd, sB, sC, ypart);
-                else main_tile<T, N, false, true, CONV, ZOH, DT>(second, h, dprev, prm, dl, su, sd, sB, sC, ypart);
-            }
-        }
+        recur(s, cur);
         if (s + 1 < nT) {
             st.store_bc(nxt);
             cp_async_wait_all();
