@@ -74,18 +74,21 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
                       float *dD, float *dbias, float *tmp, cudaStream_t stream, cudaEvent_t *ev) {
     if (!rec(ev, 0, stream)) return VIM_ERR_CUDA;
     if (a.G > 1) {
-        // h entering each chunk: the forward scan's own summary kernels
-        const dim3 gf((a.Di + kDC - 1) / kDC, a.G, a.batch);
+        // h entering each chunk: the forward scan's own summary kernels, each CTA walking
+        // kBwdCarrySpan consecutive chunks
+        PairArgs fc = fwd;
+        fc.carry_span = kBwdCarrySpan;
+        const dim3 gf((a.Di + kDC - 1) / kDC, (a.G + kBwdCarrySpan - 1) / kBwdCarrySpan, a.batch);
         const size_t sc = 2 * (size_t)Stage<T, N, false>::kSlotBytes;
-        auto carry = pair_carry<T, N, false, false, ZOH>;
+        auto carry = pair_carry<T, N, false, false, ZOH, false, true>;
         if constexpr (bc_vectorizable<T, N>()) {
             // B and C rows as 16-byte vectors when every base allows it
             if (aligned16(fwd.B[0]) && aligned16(fwd.B[1]) && aligned16(fwd.C[0]) && aligned16(fwd.C[1]))
-                carry = pair_carry<T, N, true, false, ZOH>;
+                carry = pair_carry<T, N, true, false, ZOH, false, true>;
         }
         if (cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sc) != cudaSuccess)
             return VIM_ERR_CUDA;
-        carry<<<gf, kThreads, sc, stream>>>(fwd);
+        carry<<<gf, kThreads, sc, stream>>>(fc);
         if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
         const int64_t units = (int64_t)a.batch * 2 * a.Di * N;
         const dim3 gc((unsigned)((units + 255) / 256));

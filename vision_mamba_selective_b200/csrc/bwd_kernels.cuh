@@ -40,6 +40,10 @@ constexpr int kBwdChunk = 32;                 // tokens per chunk
 constexpr int kBwdSeg = 4;                    // tokens between checkpoints of h
 constexpr int kBwdNSeg = kBwdChunk / kBwdSeg;
 constexpr int kAdjCh = 64;                    // channels per adj_carry CTA
+#ifndef VIMSCAN_BWD_CARRY_SPAN
+#define VIMSCAN_BWD_CARRY_SPAN 3
+#endif
+constexpr int kBwdCarrySpan = VIMSCAN_BWD_CARRY_SPAN;   // chunks per CTA of the forward summaries
 constexpr int kReduceParts = 32;              // row groups of the first parameter-reduction pass
 #ifndef VIMSCAN_BWD_NT
 #define VIMSCAN_BWD_NT 4                         // states per thread of bwd_main (4 or 8)

@@ -261,6 +261,7 @@ struct PairArgs {
     const float *dt_w;              // [2][Di] its dt_proj weights: delta_raw = dt_in * dt_w
     int zoh;                        // exact zero-order-hold Bbar instead of Delta B
     int fold_reverse;               // pair_combine folds each direction against its order
+    int carry_span;                 // consecutive chunks per pair_carry CTA (0 or 1: one)
 };
 
 // position visited at step t of the forward direction
@@ -650,19 +651,25 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
 }
 
 // (the exact hold needs more registers per thread, so fewer CTAs per SM)
-template <typename T, int N, bool VEC_BC, bool CONV, bool ZOH, bool DT = false>
+template <typename T, int N, bool VEC_BC, bool CONV, bool ZOH, bool DT = false, bool SPAN = false>
 __global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMinBlocks) pair_carry(PairArgs p) {
     using S = Stage<T, N, CONV>;
     constexpr int NP = N / 2;
     constexpr int kSlot = S::kSlotBytes;
     extern __shared__ __align__(16) char smem[];
 
-    const int b = blockIdx.z, c = blockIdx.y, d0 = blockIdx.x * kDC;
+    // With SPAN the CTA walks p.carry_span consecutive chunks (short chunks amortise the
+    // staging prologue this way) and writes each one's summary when its walk leaves it;
+    // without, one chunk
+    const int span = SPAN ? max(1, p.carry_span) : 1;
+    const int b = blockIdx.z, c0 = blockIdx.y * span, d0 = blockIdx.x * kDC;
     const int dir = threadIdx.x / kDC, dl = threadIdx.x % kDC, d = d0 + dl;
-    const int t0 = c * p.chunk, tc = min(p.chunk, p.L - t0);
+    const int t0 = c0 * p.chunk, tc = min(span * p.chunk, p.L - t0);
     const int nT = (tc + kTile - 1) / kTile;
+    const int tpc = p.chunk / kTile;   // tiles per chunk
     // the forward summary of the last chunk and the backward one of the first are unused
-    const bool active = (dir == 0 ? (c < p.G - 1) : (c > 0)) && d < p.Di;
+    auto is_active = [&](int cs) { return (dir == 0 ? (cs < p.G - 1) : (cs > 0)) && d < p.Di; };
+    bool active = is_active(c0);
     constexpr bool LU = lu_mode<T, ZOH>();
 
     ChannelParams<N> prm;
@@ -681,6 +688,13 @@ __global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMin
 #pragma unroll
     for (int k = 0; k < NP; ++k) H[k] = f2(0.f, 0.f);
     float Ssum = 0.0f;
+    auto write = [&](int cs) {
+        const size_t base = (((size_t)b * p.G + cs) * 2 + dir) * p.Di + d;
+        float2 *out = reinterpret_cast<float2 *>(p.hloc + base * N);
+#pragma unroll
+        for (int k = 0; k < NP; ++k) out[k] = H[k];
+        p.ssum[base] = LU ? Ssum * kLn2 : Ssum;   // natural units
+    };
 
     for (int s = 0; s < nT; ++s) {
         char *cur = smem + (s & 1) * kSlot;
@@ -689,6 +703,9 @@ __global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMin
             st.issue(nxt, nT - 2 - s, s + 1);
             st.load_bc(nT - 2 - s, s + 1);
         }
+        const int j = dir == 0 ? nT - 1 - s : s;   // the tile this step walks
+        const int cs = c0 + j / tpc;               // and its chunk
+        if constexpr (SPAN) active = is_active(cs);
         if (active) {
             const T *su = S::uv(cur, dir, 0), *sd = S::uv(cur, dir, 1);
             const float *sB = S::bc(cur, dir, 0);
@@ -700,20 +717,24 @@ __global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMin
                 else carry_tile<T, N, false, false, CONV, ZOH, DT>(H, Ssum, prm, dl, su, sd, sB);
             }
         }
+        if constexpr (SPAN) {
+            // the walk leaves chunk cs after this tile: its summary, then the next from zero
+            if (s < nT - 1 && (dir == 0 ? j - 1 : j + 1) / tpc != j / tpc) {
+                if (active) write(cs);
+#pragma unroll
+                for (int k = 0; k < NP; ++k) H[k] = f2(0.f, 0.f);
+                Ssum = 0.0f;
+            }
+        }
         if (s + 1 < nT) {
             st.store_bc(nxt);
             cp_async_wait_all();
         }
         __syncthreads();
     }
-
-    if (active) {
-        const size_t base = (((size_t)b * p.G + c) * 2 + dir) * p.Di + d;
-        float2 *out = reinterpret_cast<float2 *>(p.hloc + base * N);
-#pragma unroll
-        for (int k = 0; k < NP; ++k) out[k] = H[k];
-        p.ssum[base] = LU ? Ssum * kLn2 : Ssum;   // natural units
-    }
+    // the chunk the walk ends in (with SPAN: the first chunk forward, the last backward)
+    if constexpr (SPAN) active = is_active(dir == 0 ? c0 : c0 + (nT - 1) / tpc);
+    if (active) write(dir == 0 ? c0 : c0 + (nT - 1) / tpc);
 }
 
 // ----------------------------------------------------------------------------
