@@ -109,6 +109,12 @@ def test_bwd_small(vs, case):
     check_all(f"bwd_{case}", run(vs, x, gate), ref(x, gate), dtype)
 
 
+def test_bwd_long_carry_chains(vs):
+    # 17000 tokens are 532 chunks of 32, for both folds (the forward state and the adjoint)
+    x = inputs(1, 17000, 32, 16, torch.float32, seed=17)
+    check_all("bwd_long_L17000", run(vs, x), ref(x), torch.float32, sum_tol=SUM_TOL_FULL)
+
+
 def offset_copy(t):
     """A copy of t one element past the start of a device allocation, so that its address
     is not a multiple of 8 bytes (bf16) or 16 bytes (fp32)."""

@@ -102,6 +102,14 @@ def test_vim_small(vs, case):
     check(f"vim_{case}", run_vim(vs, x, gate), ref_vim(x, gate), dtype)
 
 
+@pytest.mark.parametrize("L", [12000, 50000], ids=["G125", "G521"])
+def test_vim_long_carry_chains(vs, L):
+    # long chains of chunk summaries: 125 and 521 chunks of 96 tokens, folded 16 loads at
+    # a time
+    x = vim_inputs(1, L, 64, 16, torch.float32, seed=L % 997)
+    check(f"vim_long_L{L}", run_vim(vs, x), ref_vim(x), torch.float32)
+
+
 def test_vim_softplus_cut_and_large_gate(vs):
     x = vim_inputs(2, 40, 64, 16, torch.float32, seed=5)
     x["delta"] = (x["delta"] * 0 + torch.linspace(-30, 30, 40)[None, :, None]).contiguous()
