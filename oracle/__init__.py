@@ -62,6 +62,7 @@ class Oracle:
         lib.oracle_s6_direction_bwd.argtypes = [_D] * 7 + [_I64] + [_D] * 8 + [ctypes.c_int] * 6
         lib.oracle_vim_bidir_bwd.argtypes = [_D, _D, _D, _D, _D, ctypes.c_int64] + [_D] * 12 + [ctypes.c_int] * 6
         lib.oracle_cross_scan4_bwd.argtypes = [_D] * 17 + [ctypes.c_int] * 7
+        lib.oracle_vim_bidir_conv_bwd.argtypes = [_D] * 7 + [ctypes.c_int64] + [_D] * 14 + [ctypes.c_int] * 6
         lib.oracle_xproj.argtypes = [_D, _D, _D, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
@@ -150,6 +151,33 @@ class Oracle:
                                            batch, L, Di, N, int(bool(delta_is_raw)), int(bool(zoh)))
         if rc:
             raise ValueError("oracle_vim_bidir_bwd: bad sizes")
+        return out
+
+    def vim_bidir_conv_bwd(self, x, conv_w, conv_b, delta, z, B, C, A, D, bias, dout, *, bc_dir_stride=0,
+                           delta_is_raw=True, zoh=False):
+        """Derivatives of vim_bidir_conv for the loss sum(dout * y).
+
+        Returns a dict of fp64 arrays: dx [batch, L, Di], dconv_w [2, Di, 3], dconv_b
+        [2, Di], and ddelta, dz (None without a gate), dB, dC, dA, dD, dbias as in
+        vim_bidir_bwd.
+        """
+        x, conv_w, conv_b, delta, z, B, C, A, D, bias, dout = map(
+            _f64, (x, conv_w, conv_b, delta, z, B, C, A, D, bias, dout))
+        batch, L, Di = x.shape
+        N = B.shape[-1]
+        if bias is None:
+            bias = np.zeros((2, Di))
+        out = dict(dx=np.zeros((batch, L, Di)), dconv_w=np.zeros((2, Di, 3)), dconv_b=np.zeros((2, Di)),
+                   ddelta=np.zeros((batch, L, Di)), dz=np.zeros((batch, L, Di)) if z is not None else None,
+                   dB=np.zeros(B.shape), dC=np.zeros(C.shape), dA=np.zeros((2, Di, N)),
+                   dD=np.zeros((2, Di)), dbias=np.zeros((2, Di)))
+        rc = self.lib.oracle_vim_bidir_conv_bwd(
+            _p(x), _p(conv_w), _p(conv_b), _p(delta), _p(z), _p(B), _p(C), int(bc_dir_stride), _p(A), _p(D),
+            _p(bias), _p(dout), _p(out["dx"]), _p(out["dconv_w"]), _p(out["dconv_b"]), _p(out["ddelta"]),
+            _p(out["dz"]), _p(out["dB"]), _p(out["dC"]), _p(out["dA"]), _p(out["dD"]), _p(out["dbias"]),
+            batch, L, Di, N, int(bool(delta_is_raw)), int(bool(zoh)))
+        if rc:
+            raise ValueError("oracle_vim_bidir_conv_bwd: bad sizes")
         return out
 
     def cross_scan4_bwd(self, u, delta, z, B, C, A, D, bias, dout, *, delta_is_raw=True, zoh=False):
@@ -339,6 +367,10 @@ def vim_block_scan(*a, **k):
 
 def vim_bidir_conv(*a, **k):
     return default().vim_bidir_conv(*a, **k)
+
+
+def vim_bidir_conv_bwd(*a, **k):
+    return default().vim_bidir_conv_bwd(*a, **k)
 
 
 def cross_merge4(*a, **k):

@@ -527,6 +527,98 @@ int oracle_vim_bidir_bwd(const double *u, const double *delta, const double *z,
 }
 
 /*
+ * Derivative of oracle_vim_bidir_conv (the scan with each pathway's convolution front)
+ * for ell = sum dout * y.  Outputs (overwritten):
+ *   dx : [batch, L, Di];  dconv_w [2][Di][3];  dconv_b [2][Di];
+ *   ddelta, dz, dB, dC, dA, dD, dbias : as in oracle_vim_bidir_bwd.
+ * The chain rule through u_k = silu(pre_k): each direction's dl/du_k comes from
+ * oracle_s6_direction_bwd on its own u_k; with dpre_k = dl/du_k * silu'(pre_k) and tap
+ * j of pathway k reading x[s_kj(t)] (s = t + j - 1 forward, t + 1 - j backward):
+ *   dl/dx[s_kj(t)] += w_k[j] dpre_k[t],  dl/dw_k[j] += dpre_k[t] x[s_kj(t)],
+ *   dl/dcb_k += dpre_k[t]   (taps that fall outside 0..L-1 read the zero padding).
+ */
+int oracle_vim_bidir_conv_bwd(const double *x, const double *conv_w, const double *conv_b,
+                              const double *delta, const double *z, const double *B, const double *C,
+                              int64_t bc_dir_stride, const double *A, const double *D, const double *bias,
+                              const double *dout, double *dx, double *dconv_w, double *dconv_b,
+                              double *ddelta, double *dz, double *dB, double *dC,
+                              double *dA, double *dD, double *dbias,
+                              int batch, int L, int Di, int N, int delta_is_raw, int zoh)
+{
+    if (batch < 0 || L < 0 || Di < 0 || N < 1 || bc_dir_stride < 0) return -1;
+    int64_t n_act = (int64_t)batch * L * Di, n_bc = (int64_t)batch * L * N;
+    int64_t n_bc_all = bc_dir_stride > 0 ? bc_dir_stride + n_bc : n_bc;
+    size_t na = (size_t)(n_act > 0 ? n_act : 1);
+    double *u[2], *du[2], *dy = (double *)malloc(na * sizeof(double));
+    int64_t *order = (int64_t *)malloc((size_t)(L > 0 ? L : 1) * sizeof(int64_t));
+    u[0] = (double *)calloc(na, sizeof(double)); u[1] = (double *)calloc(na, sizeof(double));
+    du[0] = (double *)calloc(na, sizeof(double)); du[1] = (double *)calloc(na, sizeof(double));
+    int rc = (!dy || !order || !u[0] || !u[1] || !du[0] || !du[1]) ? -1 : 0;
+    if (!rc) {
+        rc |= oracle_conv_silu(x, conv_w, conv_b, u[0], batch, L, Di, 0);
+        rc |= oracle_conv_silu(x, conv_w + (int64_t)Di * 3, conv_b + Di, u[1], batch, L, Di, 1);
+    }
+    if (!rc) {
+        for (int64_t i = 0; i < n_act; ++i) { dx[i] = 0.0; ddelta[i] = 0.0; }
+        for (int64_t i = 0; i < n_bc_all; ++i) { dB[i] = 0.0; dC[i] = 0.0; }
+        for (int64_t i = 0; i < 2 * (int64_t)Di * N; ++i) dA[i] = 0.0;
+        for (int64_t i = 0; i < 2 * (int64_t)Di; ++i) { dD[i] = 0.0; dbias[i] = 0.0; dconv_b[i] = 0.0; }
+        for (int64_t i = 0; i < 6 * (int64_t)Di; ++i) dconv_w[i] = 0.0;
+        if (z) {
+            double *ys = (double *)malloc(na * sizeof(double));
+            if (!ys) rc = -1;
+            else {
+                rc |= oracle_vim_bidir_conv(x, conv_w, conv_b, delta, NULL, B, C, bc_dir_stride, A, D, bias, ys,
+                                            batch, L, Di, N, delta_is_raw, zoh);
+                for (int64_t i = 0; i < n_act; ++i) {
+                    dz[i] = dout[i] * ys[i] * silu_grad(z[i]);
+                    dy[i] = dout[i] * silu(z[i]);
+                }
+                free(ys);
+            }
+        } else {
+            for (int64_t i = 0; i < n_act; ++i) dy[i] = dout[i];
+        }
+    }
+    if (!rc) {
+        for (int64_t t = 0; t < L; ++t) order[t] = t;
+        rc |= oracle_s6_direction_bwd(u[0], delta, B, C, A, D, bias, order, dy, du[0], ddelta, dB, dC,
+                                      dA, dD, dbias, batch, L, Di, N, delta_is_raw, zoh);
+        for (int64_t t = 0; t < L; ++t) order[t] = L - 1 - t;
+        rc |= oracle_s6_direction_bwd(u[1], delta, B + bc_dir_stride, C + bc_dir_stride,
+                                      A + (int64_t)Di * N, D + Di, bias + Di, order, dy, du[1], ddelta,
+                                      dB + bc_dir_stride, dC + bc_dir_stride,
+                                      dA + (int64_t)Di * N, dD + Di, dbias + Di,
+                                      batch, L, Di, N, delta_is_raw, zoh);
+    }
+    if (!rc) {
+        for (int k = 0; k < 2; ++k) {
+            const double *w = conv_w + (int64_t)k * Di * 3, *cb = conv_b + (int64_t)k * Di;
+            double *dw = dconv_w + (int64_t)k * Di * 3, *dcb = dconv_b + (int64_t)k * Di;
+            for (int64_t b = 0; b < batch; ++b)
+                for (int64_t t = 0; t < L; ++t)
+                    for (int64_t d = 0; d < Di; ++d) {
+                        double pre = cb[d];
+                        for (int j = 0; j < 3; ++j) {
+                            int64_t s = k ? t + 1 - j : t + j - 1;
+                            if (s >= 0 && s < L) pre += w[d * 3 + j] * x[(b * L + s) * Di + d];
+                        }
+                        double dpre = du[k][(b * L + t) * Di + d] * silu_grad(pre);
+                        dcb[d] += dpre;
+                        for (int j = 0; j < 3; ++j) {
+                            int64_t s = k ? t + 1 - j : t + j - 1;
+                            if (s < 0 || s >= L) continue;
+                            dx[(b * L + s) * Di + d] += w[d * 3 + j] * dpre;
+                            dw[d * 3 + j] += dpre * x[(b * L + s) * Di + d];
+                        }
+                    }
+        }
+    }
+    free(dy); free(order); free(u[0]); free(u[1]); free(du[0]); free(du[1]);
+    return rc ? -1 : 0;
+}
+
+/*
  * The input projections of the S6 module (page "Vision Mamba Guide", the PyTorch
  * SimpleSelectiveSSM under "The Selective State Space (S6) Mechanism": x_proj is a
  * linear map without bias from d_model to 2N + 1 columns, read as B (columns 0..N-1),

@@ -652,6 +652,71 @@ def pin_cross_bwd_finite_differences(orc):
     _cross_bwd_fd(orc, 122, zoh=True)
 
 
+def _conv_bwd_case(rng, batch=1, L=6, Di=2, N=3):
+    c = _bwd_case(rng, batch=batch, L=L, Di=Di, N=N, separate_bc=True)
+    c["x"] = c.pop("u")
+    c["conv_w"] = rng.normal(size=(2, Di, 3)) * 0.7
+    c["conv_b"] = rng.normal(size=(2, Di)) * 0.5
+    return c
+
+
+def _conv_loss(orc, c, zoh=False, **over):
+    c = {**c, **over}
+    y = orc.vim_bidir_conv(c["x"], c["conv_w"], c["conv_b"], c["delta"], c["z"], c["B"], c["C"], c["A"], c["D"],
+                           c["bias"], bc_dir_stride=c["stride"], delta_is_raw=True, zoh=zoh)
+    return float(np.sum(c["dout"] * y))
+
+
+def pin_conv_bwd_finite_differences(orc):
+    """Every derivative of the scan with its convolution front (x, both pathways'
+    taps and biases, raw delta, z, per-direction B and C, A, D, delta bias) against
+    central finite differences of the forward oracle's loss sum(dout * y) (section "2.
+    The Bidirectional Mamba Block": each pathway's "1D Conv -> SiLU" in front of its
+    SSM); first-order and exact hold.  Step 1e-6 in fp64."""
+    for seed, zoh in ((141, False), (142, True)):
+        c = _conv_bwd_case(_rng(seed))
+        g = orc.vim_bidir_conv_bwd(c["x"], c["conv_w"], c["conv_b"], c["delta"], c["z"], c["B"], c["C"], c["A"],
+                                   c["D"], c["bias"], c["dout"], bc_dir_stride=c["stride"], zoh=zoh)
+        for name, key in (("x", "dx"), ("conv_w", "dconv_w"), ("conv_b", "dconv_b"), ("delta", "ddelta"),
+                          ("z", "dz"), ("B", "dB"), ("C", "dC"), ("A", "dA"), ("D", "dD"), ("bias", "dbias")):
+            arr, eps = c[name], 1e-6
+            fd = np.zeros_like(arr)
+            for i in np.ndindex(arr.shape):
+                up, dn = arr.copy(), arr.copy()
+                up[i] += eps
+                dn[i] -= eps
+                fd[i] = (_conv_loss(orc, c, zoh, **{name: up}) - _conv_loss(orc, c, zoh, **{name: dn})) / (2 * eps)
+            err = np.max(np.abs(fd - g[key])) / np.max(np.abs(fd))
+            assert err < 1e-7, (name, zoh, err)
+
+
+def pin_conv_bwd_identity_taps(orc):
+    """With taps (0, 1, 0) and zero biases both pathways see u = silu(x), so the
+    front's derivative reduces to the plain scan's by the chain rule: dx = du silu'(x)
+    with du from the scan's derivative at u = silu(x); every other derivative equals
+    the scan's; summed over the two pathways, the bias derivatives are the token sums
+    of du silu'(x) and the middle taps' those of du silu'(x) x."""
+    rng = _rng(143)
+    c = _conv_bwd_case(rng, batch=2, L=9, Di=3, N=4)
+    c["conv_w"] = np.zeros((2, 3, 3))
+    c["conv_w"][:, :, 1] = 1.0
+    c["conv_b"] = np.zeros((2, 3))
+    x = c["x"]
+    u = x / (1 + np.exp(-x))
+    sg = 1 / (1 + np.exp(-x))
+    dsilu = sg * (1 + x * (1 - sg))
+    g = orc.vim_bidir_conv_bwd(x, c["conv_w"], c["conv_b"], c["delta"], c["z"], c["B"], c["C"], c["A"], c["D"],
+                               c["bias"], c["dout"], bc_dir_stride=c["stride"])
+    r = orc.vim_bidir_bwd(u, c["delta"], c["z"], c["B"], c["C"], c["A"], c["D"], c["bias"], c["dout"],
+                          bc_dir_stride=c["stride"])
+    np.testing.assert_allclose(g["dx"], r["du"] * dsilu, rtol=1e-11, atol=1e-13)
+    for k in ("ddelta", "dz", "dB", "dC", "dA", "dD", "dbias"):
+        np.testing.assert_allclose(g[k], r[k], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(g["dconv_b"].sum(axis=0), (r["du"] * dsilu).sum(axis=(0, 1)), rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(g["dconv_w"][:, :, 1].sum(axis=0), (r["du"] * dsilu * x).sum(axis=(0, 1)),
+                               rtol=1e-11, atol=1e-13)
+
+
 ALL_PINS = [
     pin_delta_zero,
     pin_constant_input_geometric,
@@ -676,4 +741,6 @@ ALL_PINS = [
     pin_xproj_is_matmul,
     pin_cross_bwd_finite_differences,
     pin_block_scan_composition,
+    pin_conv_bwd_finite_differences,
+    pin_conv_bwd_identity_taps,
 ]

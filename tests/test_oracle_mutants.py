@@ -70,6 +70,17 @@ MUTANTS = {
         "if (zoh) dA_loc[d * N + n] += g[n] * Bt[n] * x * hold_gain_dA(dt, Ad[n], zoh);", ""),
     "zoh_bwd_series_coefficient": ("c[k] = (double)k / f;", "c[k] = 1.0 / f;"),
     "zoh_bwd_closed_form_sign": ("(zz * exp(zz) - expm1(zz))", "(zz * exp(zz) + expm1(zz))"),
+    # the convolution front's derivative
+    "conv_bwd_no_silu_grad": ("double dpre = du[k][(b * L + t) * Di + d] * silu_grad(pre);",
+                              "double dpre = du[k][(b * L + t) * Di + d];"),
+    "conv_bwd_taps_not_reversed": ("int64_t s = k ? t + 1 - j : t + j - 1;", "int64_t s = t + j - 1;"),
+    "conv_bwd_dw_without_x": ("dw[d * 3 + j] += dpre * x[(b * L + s) * Di + d];", "dw[d * 3 + j] += dpre;"),
+    "conv_bwd_dx_tap_flipped": ("dx[(b * L + s) * Di + d] += w[d * 3 + j] * dpre;",
+                                "dx[(b * L + s) * Di + d] += w[d * 3 + 2 - j] * dpre;"),
+    "conv_bwd_shared_du": ("rc |= oracle_s6_direction_bwd(u[1], delta, B + bc_dir_stride, C + bc_dir_stride,\n"
+                           "                                      A + (int64_t)Di * N, D + Di, bias + Di, order, dy, du[1],",
+                           "rc |= oracle_s6_direction_bwd(u[1], delta, B + bc_dir_stride, C + bc_dir_stride,\n"
+                           "                                      A + (int64_t)Di * N, D + Di, bias + Di, order, dy, du[0],"),
 }
 
 
