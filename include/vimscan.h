@@ -386,6 +386,46 @@ vim_status vim_scan_bidir_noalloc(const void *u, const void *delta, const void *
                                   vim_dtype dt, cudaStream_t stream);
 
 /*
+ * Derivatives of vim_scan_bidir_conv (or, with VIM_FLAG_ZOH_EXACT in flags, of its
+ * exact-hold form) for a loss whose derivative with respect to y is dout: the scan's
+ * derivative carried through each pathway's convolution front (section "2. The
+ * Bidirectional Mamba Block": the pathways' "1D Conv -> SiLU" in front of their SSMs).
+ *
+ *   x, conv_w, conv_b, delta, z, B, C, bc_dir_stride, A, D, delta_bias, dt : as in
+ *                 vim_scan_bidir_conv (conv_w [2, d_inner, 3], conv_b [2, d_inner] fp32).
+ *   dout        : [batch, L, d_inner] (dt).
+ *   Outputs (overwritten): dx [batch, L, d_inner] (dt); dconv_w [2, d_inner, 3] and
+ *                 dconv_b [2, d_inner] fp32; ddelta (w.r.t. the raw delta), dz, dB, dC,
+ *                 dA, dD, ddelta_bias as in vim_scan_bidir_bwd (dz NULL exactly when z
+ *                 is).
+ *   workspace   : vim_scan_conv_bwd_workspace_bytes(batch, L, d_inner, d_state, dt,
+ *                 bc_dir_stride > 0) bytes, 256-byte aligned.  It holds, besides the
+ *                 scan derivative's scratch, both pathways' smoothed inputs u_k and
+ *                 their dl/du_k, in fp32.
+ *
+ * Every sum (over tokens for the taps, biases and parameters, over channels for dB
+ * and dC) is taken in a fixed order: results repeat bit for bit.  Errors as for
+ * vim_scan_bidir_bwd; size 0 writes zero parameter derivatives.
+ */
+vim_status vim_scan_bidir_conv_bwd_ex(const void *x, const float *conv_w, const float *conv_b, const void *delta,
+                                      const void *z, const void *B, const void *C, int64_t bc_dir_stride,
+                                      const float *A, const float *D, const float *delta_bias, const void *dout,
+                                      void *dx, float *dconv_w, float *dconv_b, void *ddelta, void *dz, float *dB,
+                                      float *dC, float *dA, float *dD, float *ddelta_bias, int batch, int L,
+                                      int d_inner, int d_state, vim_dtype dt, unsigned flags, void *workspace,
+                                      size_t workspace_bytes, cudaStream_t stream);
+/* vim_scan_bidir_conv_bwd_ex with flags 0 (the first-order Bbar). */
+vim_status vim_scan_bidir_conv_bwd(const void *x, const float *conv_w, const float *conv_b, const void *delta,
+                                   const void *z, const void *B, const void *C, int64_t bc_dir_stride,
+                                   const float *A, const float *D, const float *delta_bias, const void *dout,
+                                   void *dx, float *dconv_w, float *dconv_b, void *ddelta, void *dz, float *dB,
+                                   float *dC, float *dA, float *dD, float *ddelta_bias, int batch, int L,
+                                   int d_inner, int d_state, vim_dtype dt, void *workspace, size_t workspace_bytes,
+                                   cudaStream_t stream);
+/* Workspace bytes of vim_scan_bidir_conv_bwd (0 for invalid arguments or an empty problem). */
+size_t vim_scan_conv_bwd_workspace_bytes(int batch, int L, int d_inner, int d_state, vim_dtype dt, int separate_bc);
+
+/*
  * vim_scan_bidir for activations in HOST memory: the same operation, flags and
  * parameters as vim_scan_bidir_ex without the convolution front, with u, delta, z,
  * B, C read from the host and y written to the host.  The pages have no counterpart

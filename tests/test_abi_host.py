@@ -42,6 +42,7 @@ def test_header_declares_the_boundary():
                           "vmamba_cross_scan4_bwd", "vmamba_cross_scan4_bwd_workspace_bytes",
                           "vmamba_cross_scan4_bwd_ex",
                           "vim_scan_bidir_host", "vim_scan_host_workspace_bytes",
+                          "vim_scan_bidir_conv_bwd", "vim_scan_bidir_conv_bwd_ex", "vim_scan_conv_bwd_workspace_bytes",
                           "vim_scan_workspace_bytes", "vim_status_string"}, names
 
 
@@ -138,6 +139,39 @@ def test_host_entry_rejects(vs):
     assert host(vs, ws=FAKE + 16) == vs.VIM_ERR_WORKSPACE
     assert host(vs, batch=0, ws=None) == vs.VIM_OK                    # empty: nothing to do
     assert host(vs, L=0, u=None, ws=None) == vs.VIM_OK
+
+
+def conv_bwd(vs, **kw):
+    """vim_scan_bidir_conv_bwd_ex on fake device addresses; every case fails a host check."""
+    a = dict(x=FAKE, cw=FAKE, cb=FAKE, delta=FAKE, z=FAKE, B=FAKE, C=FAKE, stride=0, A=FAKE, D=FAKE, bias=FAKE,
+             dout=FAKE, dx=FAKE, dcw=FAKE, dcb=FAKE, ddelta=FAKE, dz=FAKE, dB=FAKE, dC=FAKE, dA=FAKE, dD=FAKE,
+             dbias=FAKE, batch=2, L=100, Di=64, N=16, dt=vs.VIM_BF16, flags=0, ws=FAKE, ws_bytes=1 << 40)
+    a.update(kw)
+    return vs.lib.vim_scan_bidir_conv_bwd_ex(
+        a["x"], a["cw"], a["cb"], a["delta"], a["z"], a["B"], a["C"], a["stride"], a["A"], a["D"], a["bias"],
+        a["dout"], a["dx"], a["dcw"], a["dcb"], a["ddelta"], a["dz"], a["dB"], a["dC"], a["dA"], a["dD"], a["dbias"],
+        a["batch"], a["L"], a["Di"], a["N"], a["dt"], a["flags"], a["ws"], a["ws_bytes"], None)
+
+
+def test_conv_bwd_rejects(vs):
+    assert conv_bwd(vs, x=None) == vs.VIM_ERR_INVALID_ARG
+    assert conv_bwd(vs, cw=None) == vs.VIM_ERR_INVALID_ARG
+    assert conv_bwd(vs, dcb=None) == vs.VIM_ERR_INVALID_ARG
+    assert conv_bwd(vs, dx=None) == vs.VIM_ERR_INVALID_ARG
+    assert conv_bwd(vs, z=None) == vs.VIM_ERR_INVALID_ARG                 # dz without z
+    assert conv_bwd(vs, cw=FAKE + 2) == vs.VIM_ERR_INVALID_ARG
+    assert conv_bwd(vs, x=FAKE + 8) == vs.VIM_ERR_INVALID_ARG             # not 16-byte aligned
+    assert conv_bwd(vs, flags=2) == vs.VIM_ERR_INVALID_ARG
+    assert conv_bwd(vs, stride=-1) == vs.VIM_ERR_INVALID_ARG
+    assert conv_bwd(vs, N=3) == vs.VIM_ERR_UNSUPPORTED
+    assert conv_bwd(vs, ws=None) == vs.VIM_ERR_WORKSPACE
+    assert conv_bwd(vs, ws_bytes=4096) == vs.VIM_ERR_WORKSPACE
+    assert conv_bwd(vs, ws=FAKE + 16) == vs.VIM_ERR_WORKSPACE
+    f = vs.vim_scan_conv_bwd_workspace_bytes
+    n = f(8, 4097, 384, 16, vs.VIM_BF16, False)
+    assert n % 256 == 0 and n > vs.vim_scan_bwd_workspace_bytes(8, 4097, 384, 16, False) + 4 * 8 * 4097 * 384 * 4
+    assert f(8, 4097, 384, 16, vs.VIM_BF16, True) > n
+    assert f(0, 4097, 384, 16, vs.VIM_BF16, False) == 0 and f(8, 4097, 384, 5, vs.VIM_BF16, False) == 0
 
 
 def test_host_workspace_bytes(vs):

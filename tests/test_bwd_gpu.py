@@ -324,3 +324,106 @@ def test_cross_bwd_zoh(vs, case):
     want = oracle.cross_scan4_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["bias"], x["dout"],
                                   zoh=True)
     check_all(f"cross_bwd_zoh_{case}", got, want, dtype)
+
+
+# ---------------------------------------------------------------------------
+# the scan with its convolution front (vim_scan_bidir_conv_bwd)
+# ---------------------------------------------------------------------------
+CONV_KEYS = [("dx", "dx"), ("ddelta", "ddelta"), ("dz", "dz"), ("dconv_w", "dconv_w"), ("dconv_b", "dconv_b"),
+             ("dB", "dB"), ("dC", "dC"), ("dA", "dA"), ("dD", "dD"), ("ddelta_bias", "dbias")]
+
+
+def conv_inputs(batch, L, Di, N, dtype, seed, separate_bc=False, generic_A=False):
+    x = inputs(batch, L, Di, N, dtype, seed, separate_bc=separate_bc, generic_A=generic_A)
+    x["x"] = x.pop("u")
+    g = torch.Generator().manual_seed(seed + 1)
+    k = 1.0 / np.sqrt(3.0)   # the kernel-3 depthwise convolution's default init bound
+    x["conv_w"] = ((torch.rand((2, Di, 3), generator=g) * 2 - 1) * k).contiguous()
+    x["conv_b"] = ((torch.rand((2, Di), generator=g) * 2 - 1) * k).contiguous()
+    return x
+
+
+def run_conv(vs, x, gate=True, zoh=False):
+    c = lambda k: x[k].cuda()
+    out = vs.vim_scan_bidir_conv_bwd(c("x"), c("conv_w"), c("conv_b"), c("delta"), c("z") if gate else None, c("B"),
+                                     c("C"), c("A"), c("D"), c("bias"), c("dout"), bc_dir_stride=x["stride"], zoh=zoh)
+    torch.cuda.synchronize()
+    return out
+
+
+def ref_conv(x, gate=True, zoh=False):
+    return oracle.vim_bidir_conv_bwd(x["x"], x["conv_w"], x["conv_b"], x["delta"], x["z"] if gate else None, x["B"],
+                                     x["C"], x["A"], x["D"], x["bias"], x["dout"], bc_dir_stride=x["stride"], zoh=zoh)
+
+
+def check_conv(name, got, want, dtype, sum_tol=SUM_TOL):
+    """dx, d delta_raw, dz: both gates; the sums (the taps' and biases' over tokens,
+    dB, dC over channels, dA, dD, d delta_bias): normwise within sum_tol."""
+    for k_got, k_ref in CONV_KEYS:
+        if want[k_ref] is None:
+            assert got[k_got] is None
+            continue
+        if k_got in ("dx", "ddelta", "dz"):
+            gates.gate(f"{name}:{k_got}", got[k_got], want[k_ref], dtype)
+        else:
+            gates.gate(f"{name}:{k_got}", got[k_got], want[k_ref], dtype, norm_tol=sum_tol, elementwise=False)
+
+
+CONV_CASES = [
+    # batch, L, Di, N, dtype, separate_bc, generic_A, gate, zoh
+    (1, 1, 16, 16, torch.float32, False, False, True, False),
+    (1, 5, 16, 4, torch.float32, True, False, True, False),
+    (2, 33, 64, 16, torch.float32, True, False, True, False),     # 2 chunks, the last 1 token
+    (1, 100, 40, 8, torch.float32, False, True, False, False),    # 2 runs of the front's walk
+    (2, 197, 64, 16, torch.bfloat16, False, False, True, False),
+    (1, 300, 72, 16, torch.bfloat16, True, False, True, False),
+    (1, 1000, 64, 16, torch.float32, False, False, True, False),
+    (2, 70, 32, 16, torch.float32, True, True, True, True),        # exact hold, general A
+    (1, 300, 64, 16, torch.bfloat16, False, False, True, True),
+]
+
+
+@pytest.mark.parametrize("case", CONV_CASES, ids=lambda c: f"b{c[0]}_L{c[1]}_D{c[2]}_N{c[3]}_{str(c[4])[6:]}"
+                         f"{'_sepBC' if c[5] else ''}{'_genA' if c[6] else ''}{'' if c[7] else '_nogate'}"
+                         f"{'_zoh' if c[8] else ''}")
+def test_conv_bwd(vs, case):
+    batch, L, Di, N, dtype, sep, gen, gate, zoh = case
+    x = conv_inputs(batch, L, Di, N, dtype, seed=L * 5 + Di, separate_bc=sep, generic_A=gen)
+    check_conv(f"conv_bwd_{case}", run_conv(vs, x, gate, zoh), ref_conv(x, gate, zoh), dtype)
+
+
+def test_conv_bwd_identity_taps_is_the_scan_derivative(vs):
+    # taps (0, 1, 0), zero biases: every derivative but dx and the front's own equals the
+    # scan derivative at u = silu(x), and dx = du silu'(x)
+    x = conv_inputs(2, 300, 64, 16, torch.float32, seed=9)
+    x["conv_w"].zero_()
+    x["conv_w"][:, :, 1] = 1.0
+    x["conv_b"].zero_()
+    got = run_conv(vs, x)
+    u = torch.nn.functional.silu(x["x"])
+    c = lambda t: t.cuda()
+    plain = vs.vim_scan_bidir_bwd(c(u), c(x["delta"]), c(x["z"]), c(x["B"]), c(x["C"]), c(x["A"]), c(x["D"]),
+                                  c(x["bias"]), c(x["dout"]))
+    torch.cuda.synchronize()
+    s = torch.sigmoid(x["x"].double())
+    dsilu = (s * (1 + x["x"].double() * (1 - s))).cuda()
+    gates.gate("conv_identity:dx", got["dx"], plain["du"].double() * dsilu, torch.float32)
+    for k in ("ddelta", "dz"):
+        gates.gate(f"conv_identity:{k}", got[k], plain[k], torch.float32)
+    for k in ("dB", "dC", "dA", "dD", "ddelta_bias"):
+        gates.gate(f"conv_identity:{k}", got[k], plain[k], torch.float32, norm_tol=SUM_TOL, elementwise=False)
+
+
+def test_conv_bwd_larger(vs):
+    """4097 tokens (129 chunks, 65 runs of the front's walk) at bf16, batch 2, against
+    the oracle."""
+    x = conv_inputs(2, 4097, 128, 16, torch.bfloat16, seed=31)
+    oracle.set_threads(max(1, len(os.sched_getaffinity(0))))
+    check_conv("conv_bwd_4097", run_conv(vs, x), ref_conv(x), torch.bfloat16, sum_tol=SUM_TOL_FULL)
+
+
+def test_conv_bwd_deterministic(vs):
+    x = conv_inputs(2, 500, 64, 16, torch.float32, seed=12)
+    a, b = run_conv(vs, x), run_conv(vs, x)
+    for k, _ in CONV_KEYS:
+        assert torch.equal(a[k], b[k]), k

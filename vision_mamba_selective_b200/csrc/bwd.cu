@@ -69,7 +69,7 @@ inline bool rec(cudaEvent_t *ev, int i, cudaStream_t stream) {
 
 // ZOH: the exact hold's derivative (its own forward summaries and main kernel; the
 // adjoint summaries do not involve Bbar)
-template <typename T, int N, bool ZOH>
+template <typename T, int N, bool ZOH, bool U2 = false>
 vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], float *dC_out[2], float *dA,
                       float *dD, float *dbias, float *tmp, cudaStream_t stream, cudaEvent_t *ev) {
     if (!rec(ev, 0, stream)) return VIM_ERR_CUDA;
@@ -79,12 +79,14 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
         PairArgs fc = fwd;
         fc.carry_span = kBwdCarrySpan;
         const dim3 gf((a.Di + kDC - 1) / kDC, (a.G + kBwdCarrySpan - 1) / kBwdCarrySpan, a.batch);
-        const size_t sc = 2 * (size_t)Stage<T, N, false>::kSlotBytes;
-        auto carry = pair_carry<T, N, false, false, ZOH, false, true>;
+        // (U2: the pathways' inputs formed from x by the convolution fronts, as in the
+        // scan with its front)
+        const size_t sc = 2 * (size_t)Stage<T, N, U2>::kSlotBytes;
+        auto carry = pair_carry<T, N, false, U2, ZOH, false, true>;
         if constexpr (bc_vectorizable<T, N>()) {
             // B and C rows as 16-byte vectors when every base allows it
             if (aligned16(fwd.B[0]) && aligned16(fwd.B[1]) && aligned16(fwd.C[0]) && aligned16(fwd.C[1]))
-                carry = pair_carry<T, N, true, false, ZOH, false, true>;
+                carry = pair_carry<T, N, true, U2, ZOH, false, true>;
         }
         if (cudaFuncSetAttribute(carry, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sc) != cudaSuccess)
             return VIM_ERR_CUDA;
@@ -106,7 +108,8 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
     }
     if (!rec(ev, 1, stream)) return VIM_ERR_CUDA;
     constexpr size_t sm = BwdShape<N>::kSmemBytes;
-    if (cudaFuncSetAttribute(bwd_main<T, N, ZOH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
+    if (cudaFuncSetAttribute(bwd_main<T, N, ZOH, U2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
+        cudaSuccess)
         return VIM_ERR_CUDA;
     const dim3 gm(a.nblk, a.G, a.batch);
     {
@@ -135,7 +138,7 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
         }
         cfg.attrs = attr;
         cfg.numAttrs = na;
-        if (cudaLaunchKernelEx(&cfg, bwd_main<T, N, ZOH>, a) != cudaSuccess) return VIM_ERR_CUDA;
+        if (cudaLaunchKernelEx(&cfg, bwd_main<T, N, ZOH, U2>, a) != cudaSuccess) return VIM_ERR_CUDA;
     }
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     if (!rec(ev, 2, stream)) return VIM_ERR_CUDA;
@@ -152,14 +155,14 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
     return rec(ev, 3, stream) ? VIM_OK : VIM_ERR_CUDA;
 }
 
-template <typename T, bool ZOH>
+template <typename T, bool ZOH, bool U2 = false>
 vim_status launch_bwd_n(int N, const BwdArgs &a, const PairArgs &fwd, float *dB[2], float *dC[2], float *dA,
                         float *dD, float *dbias, float *tmp, cudaStream_t stream, cudaEvent_t *ev) {
     switch (N) {
-        case 2: return launch_bwd<T, 2, ZOH>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
-        case 4: return launch_bwd<T, 4, ZOH>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
-        case 8: return launch_bwd<T, 8, ZOH>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
-        case 16: return launch_bwd<T, 16, ZOH>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
+        case 2: return launch_bwd<T, 2, ZOH, U2>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
+        case 4: return launch_bwd<T, 4, ZOH, U2>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
+        case 8: return launch_bwd<T, 8, ZOH, U2>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
+        case 16: return launch_bwd<T, 16, ZOH, U2>(a, fwd, dB, dC, dA, dD, dbias, tmp, stream, ev);
         default: return VIM_ERR_UNSUPPORTED;
     }
 }
@@ -285,6 +288,186 @@ vim_status vim_scan_bidir_bwd(const void *u, const void *delta, const void *z, c
     return vim_scan_bidir_bwd_events(u, delta, z, B, C, bc_dir_stride, A, D, delta_bias, dout, du, ddelta, dz,
                                      dB, dC, dA, dD, ddelta_bias, batch, L, d_inner, d_state, dt, workspace,
                                      workspace_bytes, stream, nullptr);
+}
+
+}  // extern "C"
+
+// ----------------------------------------------------------------------------
+// the derivative of the scan with its convolution front
+// ----------------------------------------------------------------------------
+namespace vimscan {
+namespace {
+
+// the derivative's own workspace, then both pathways' u (element type) and dl/du
+// (fp32), and the fronts' partial sums with their reduction buffer
+struct ConvBwdPlan {
+    BwdPlan pl;
+    int runs;
+    size_t off_u2, off_du2, off_part, off_ptmp, total;
+};
+
+ConvBwdPlan conv_bwd_plan(int batch, int L, int Di, int N, vim_dtype dt, int separate_bc) {
+    ConvBwdPlan c;
+    c.pl = bwd_plan(batch, L, Di, N, separate_bc);
+    size_t o = round_up(c.pl.total);
+    auto take = [&](size_t bytes) { const size_t at = o; o += round_up(bytes); return at; };
+    const size_t act = (size_t)batch * L * Di;
+    c.runs = (L + kFrontRows - 1) / kFrontRows;
+    c.off_u2 = take(2 * act * 4);
+    c.off_du2 = take(2 * act * 4);
+    c.off_part = take((size_t)batch * c.runs * 8 * Di * 4);
+    c.off_ptmp = take((size_t)kReduceParts * 8 * Di * 4);
+    c.total = o;
+    return c;
+}
+
+template <typename T>
+vim_status launch_fronts_bwd(const T *x, const float *conv_w, const float *conv_b, const float *du2, T *dx,
+                             float *part, float *ptmp, float *dconv_w, float *dconv_b, int batch, int L, int Di,
+                             int runs, int vec, cudaStream_t stream) {
+    const int64_t items = (int64_t)batch * runs * (Di / 4);
+    conv_front_bwd<T><<<(unsigned)((items + 255) / 256), 256, 0, stream>>>(x, conv_w, conv_b, du2, dx, part, batch,
+                                                                            L, Di, vec);
+    if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+    // rows of [dw: 6 Di | dcb: 2 Di] summed in a fixed order
+    const int cols = 8 * Di;
+    bwd_reduce_cols1<<<dim3((cols + 255) / 256, kReduceParts), 256, 0, stream>>>(part, ptmp, batch * runs, cols);
+    if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+    bwd_reduce_cols2<<<(cols + 255) / 256, 256, 0, stream>>>(ptmp, dconv_w, dconv_b, dconv_b + Di, 6 * Di, Di);
+    return cudaGetLastError() == cudaSuccess ? VIM_OK : VIM_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace vimscan
+
+extern "C" {
+
+size_t vim_scan_conv_bwd_workspace_bytes(int batch, int L, int d_inner, int d_state, vim_dtype dt, int separate_bc) {
+    if (check_common(batch, L, d_inner, d_state, dt) != VIM_OK) return 0;
+    if (batch <= 0 || L <= 0 || d_inner <= 0) return 0;
+    return conv_bwd_plan(batch, L, d_inner, d_state, dt, separate_bc).total;
+}
+
+vim_status vim_scan_bidir_conv_bwd_ex(const void *x, const float *conv_w, const float *conv_b, const void *delta,
+                                      const void *z, const void *B, const void *C, int64_t bc_dir_stride,
+                                      const float *A, const float *D, const float *delta_bias, const void *dout,
+                                      void *dx, float *dconv_w, float *dconv_b, void *ddelta, void *dz, float *dB,
+                                      float *dC, float *dA, float *dD, float *ddelta_bias, int batch, int L,
+                                      int d_inner, int d_state, vim_dtype dt, unsigned flags, void *workspace,
+                                      size_t workspace_bytes, cudaStream_t stream) {
+    if (flags & ~VIM_FLAG_ZOH_EXACT) return VIM_ERR_INVALID_ARG;
+    const bool zoh = (flags & VIM_FLAG_ZOH_EXACT) != 0;
+    vim_status st = check_common(batch, L, d_inner, d_state, dt);
+    if (st != VIM_OK) return st;
+    if (bc_dir_stride < 0) return VIM_ERR_INVALID_ARG;
+    if ((z == nullptr) != (dz == nullptr)) return VIM_ERR_INVALID_ARG;
+    if (!A || !D || !delta_bias || !dA || !dD || !ddelta_bias || !conv_w || !conv_b || !dconv_w || !dconv_b)
+        return VIM_ERR_INVALID_ARG;
+    if (!aligned_to(A, 4) || !aligned_to(D, 4) || !aligned_to(delta_bias, 4) || !aligned_to(dA, 4) ||
+        !aligned_to(dD, 4) || !aligned_to(ddelta_bias, 4) || !aligned_to(conv_w, 4) || !aligned_to(conv_b, 4) ||
+        !aligned_to(dconv_w, 4) || !aligned_to(dconv_b, 4))
+        return VIM_ERR_INVALID_ARG;
+    const size_t es = elem_size(dt);
+    if (batch == 0 || L == 0 || d_inner == 0) {
+        // no tokens: the parameter derivatives are zero
+        if (cudaMemsetAsync(dA, 0, sizeof(float) * 2 * (size_t)d_inner * d_state, stream) != cudaSuccess ||
+            cudaMemsetAsync(dD, 0, sizeof(float) * 2 * (size_t)d_inner, stream) != cudaSuccess ||
+            cudaMemsetAsync(ddelta_bias, 0, sizeof(float) * 2 * (size_t)d_inner, stream) != cudaSuccess ||
+            cudaMemsetAsync(dconv_w, 0, sizeof(float) * 6 * (size_t)d_inner, stream) != cudaSuccess ||
+            cudaMemsetAsync(dconv_b, 0, sizeof(float) * 2 * (size_t)d_inner, stream) != cudaSuccess)
+            return VIM_ERR_CUDA;
+        return VIM_OK;
+    }
+    if (!x || !delta || !B || !C || !dout || !dx || !ddelta || !dB || !dC) return VIM_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(delta) || !aligned_to(B, es) || !aligned_to(C, es) || !aligned_to(dout, es) ||
+        !aligned_to(dx, es) || !aligned_to(ddelta, es) || (z && !aligned_to(z, es)) || (dz && !aligned_to(dz, es)) ||
+        !aligned_to(dB, 4) || !aligned_to(dC, 4))
+        return VIM_ERR_INVALID_ARG;
+    const int separate = bc_dir_stride > 0 ? 1 : 0;
+    const ConvBwdPlan cp = conv_bwd_plan(batch, L, d_inner, d_state, dt, separate);
+    const BwdPlan &pl = cp.pl;
+    if (!workspace || workspace_bytes < cp.total || !aligned_to(workspace, kAlign)) return VIM_ERR_WORKSPACE;
+    char *ws = static_cast<char *>(workspace);
+    float *u2 = reinterpret_cast<float *>(ws + cp.off_u2);
+    float *du2 = reinterpret_cast<float *>(ws + cp.off_du2);
+    const int64_t act = (int64_t)batch * L * d_inner;
+    const int vec = aligned_to(x, dt == VIM_F32 ? 16 : 8) && aligned_to(dx, dt == VIM_F32 ? 16 : 8) ? 1 : 0;
+
+    // both pathways' smoothed inputs
+    {
+        const int64_t items = act / 4;
+        const unsigned blocks = (unsigned)std::min<int64_t>((items + 255) / 256, 148 * 16);
+        if (dt == VIM_F32)
+            conv_front_fwd<float><<<blocks, 256, 0, stream>>>(static_cast<const float *>(x), conv_w, conv_b, u2,
+                                                               batch, L, d_inner, vec);
+        else
+            conv_front_fwd<__nv_bfloat16><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(x), conv_w,
+                                                                       conv_b, u2, batch, L, d_inner, vec);
+        if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+    }
+
+    BwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.u = u2; a.u_dir_stride = act; a.du2 = du2;
+    a.delta = delta; a.z = z; a.dout = dout;
+    a.B[0] = B; a.C[0] = C;
+    a.B[1] = static_cast<const char *>(B) + bc_dir_stride * (int64_t)es;
+    a.C[1] = static_cast<const char *>(C) + bc_dir_stride * (int64_t)es;
+    a.A = A; a.D = D; a.bias = delta_bias;
+    a.ddelta = ddelta; a.dz = dz;
+    const size_t set_elems = (size_t)batch * L * pl.ncol * d_state;
+    a.dB_part[0] = reinterpret_cast<float *>(ws + pl.off_dBp);
+    a.dC_part[0] = reinterpret_cast<float *>(ws + pl.off_dCp);
+    a.dB_part[1] = separate ? a.dB_part[0] + set_elems : a.dB_part[0];
+    a.dC_part[1] = separate ? a.dC_part[0] + set_elems : a.dC_part[0];
+    a.par = reinterpret_cast<float *>(ws + pl.off_par);
+    a.hin = reinterpret_cast<const float *>(ws + pl.off_hloc);
+    a.gloc = reinterpret_cast<float *>(ws + pl.off_gloc);
+    a.gsum = reinterpret_cast<float *>(ws + pl.off_gsum);
+    a.batch = batch; a.L = L; a.Di = d_inner; a.G = pl.G; a.nblk = pl.nblk; a.cl = pl.cl; a.ncol = pl.ncol;
+    a.separate_bc = separate;
+    set_vector_flags(a, dt, d_state);
+
+    PairArgs f;
+    std::memset(&f, 0, sizeof(f));
+    f.u = x; f.conv_w = conv_w; f.conv_b = conv_b; f.delta = delta;
+    f.B[0] = a.B[0]; f.B[1] = a.B[1]; f.C[0] = a.C[0]; f.C[1] = a.C[1];
+    f.A = A; f.D = D; f.bias = delta_bias;
+    f.hloc = reinterpret_cast<float *>(ws + pl.off_hloc);
+    f.ssum = reinterpret_cast<float *>(ws + pl.off_ssum);
+    f.batch = batch; f.L = L; f.Di = d_inner; f.H = 1; f.W = L; f.order = 0;
+    f.chunk = kBwdChunk; f.G = pl.G;
+
+    float *dBo[2] = {dB, dB + bc_dir_stride}, *dCo[2] = {dC, dC + bc_dir_stride};
+    float *tmp = reinterpret_cast<float *>(ws + pl.off_tmp);
+    float *part = reinterpret_cast<float *>(ws + cp.off_part), *ptmp = reinterpret_cast<float *>(ws + cp.off_ptmp);
+    if (dt == VIM_F32) {
+        st = zoh ? launch_bwd_n<float, true, true>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream, nullptr)
+                 : launch_bwd_n<float, false, true>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream, nullptr);
+        if (st != VIM_OK) return st;
+        return launch_fronts_bwd<float>(static_cast<const float *>(x), conv_w, conv_b, du2, static_cast<float *>(dx),
+                                        part, ptmp, dconv_w, dconv_b, batch, L, d_inner, cp.runs, vec, stream);
+    }
+    st = zoh ? launch_bwd_n<__nv_bfloat16, true, true>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream,
+                                                       nullptr)
+             : launch_bwd_n<__nv_bfloat16, false, true>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream,
+                                                        nullptr);
+    if (st != VIM_OK) return st;
+    return launch_fronts_bwd<__nv_bfloat16>(static_cast<const __nv_bfloat16 *>(x), conv_w, conv_b, du2,
+                                            static_cast<__nv_bfloat16 *>(dx), part, ptmp, dconv_w, dconv_b, batch, L,
+                                            d_inner, cp.runs, vec, stream);
+}
+
+vim_status vim_scan_bidir_conv_bwd(const void *x, const float *conv_w, const float *conv_b, const void *delta,
+                                   const void *z, const void *B, const void *C, int64_t bc_dir_stride,
+                                   const float *A, const float *D, const float *delta_bias, const void *dout,
+                                   void *dx, float *dconv_w, float *dconv_b, void *ddelta, void *dz, float *dB,
+                                   float *dC, float *dA, float *dD, float *ddelta_bias, int batch, int L,
+                                   int d_inner, int d_state, vim_dtype dt, void *workspace, size_t workspace_bytes,
+                                   cudaStream_t stream) {
+    return vim_scan_bidir_conv_bwd_ex(x, conv_w, conv_b, delta, z, B, C, bc_dir_stride, A, D, delta_bias, dout, dx,
+                                      dconv_w, dconv_b, ddelta, dz, dB, dC, dA, dD, ddelta_bias, batch, L, d_inner,
+                                      d_state, dt, 0u, workspace, workspace_bytes, stream);
 }
 
 size_t vmamba_cross_scan4_bwd_workspace_bytes(int batch, int H, int W, int channels, int d_state) {

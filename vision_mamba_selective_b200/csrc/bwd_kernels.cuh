@@ -80,6 +80,9 @@ struct BwdArgs {
     int stage;                          // 0: one pair (Vim), final outputs; 1: first pair of the
                                         // cross-scan, fp32 partials to acc_*; 2: second pair, adds them
     float *acc_y, *acc_du, *acc_dd;     // [batch, L, Di] fp32 by position (stages 1 and 2)
+    int64_t u_dir_stride;               // with per-direction inputs (bwd_main's U2; u is then fp32):
+                                        // elements from the forward direction's u to the backward one's
+    float *du2;                         // with U2: [2][batch, L, Di] fp32 dl/du_k per direction
 };
 
 namespace {
@@ -570,7 +573,15 @@ __device__ __forceinline__ void channel_sum(const BwdThread<N> &th, float *red_w
 
 // forward sweep of direction DIR: checkpoints, y^DIR (ungated) and the dC terms
 // (ZOH: the exact hold's Bbar in the state update; FAST: its gains from hold_states)
-template <int N, int DIRT, bool ZOH, bool FAST>
+// u of token row r for direction DIR: the shared u, or with U2 the backward
+// direction's own (staged in the dz-factor area, which U2 does not use)
+template <int N, bool U2>
+__device__ __forceinline__ float u_of_dir(const BwdSmem<N> &sm, int DIR, int r, int cl, float shared_u) {
+    if constexpr (U2) return DIR ? sm.dzf[r * BwdShape<N>::CH + cl] : shared_u;
+    else return shared_u;
+}
+
+template <int N, int DIRT, bool ZOH, bool FAST, bool U2>
 __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
     using SH = BwdShape<N>;
     constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
@@ -590,7 +601,8 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
 #pragma unroll
         for (int m = 0; m < kBwdSeg; ++m) {
             const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
-            const float2 tk = sm.tok[r * CH + th.cl];   // u, dy
+            const float2 tk0 = sm.tok[r * CH + th.cl];   // u, dy
+            const float2 tk = f2(u_of_dir<N, U2>(sm, DIR, r, th.cl, tk0.x), tk0.y);
             const float dl = reinterpret_cast<const float *>(sm.dsg)[2 * ((DIR * TC + r) * CH + th.cl)];
             const float du = dl * tk.x;
             float2 Bp[NP], Cp[NP], v[NP];
@@ -652,7 +664,7 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
 
 // adjoint sweep of direction DIR, segment by segment from the last: h re-run over
 // the segment from its checkpoint (keeping h and the decays), then g backwards
-template <int N, int DIRT, bool ZOH, bool FAST>
+template <int N, int DIRT, bool ZOH, bool FAST, bool U2>
 __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
     using SH = BwdShape<N>;
     constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
@@ -681,7 +693,7 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
 #pragma unroll
         for (int m = 0; m < kBwdSeg; ++m) {
             const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
-            const float u = reinterpret_cast<const float *>(sm.tok)[2 * (r * CH + th.cl)];
+            const float u = u_of_dir<N, U2>(sm, DIR, r, th.cl, reinterpret_cast<const float *>(sm.tok)[2 * (r * CH + th.cl)]);
             const float dl = reinterpret_cast<const float *>(sm.dsg)[2 * ((DIR * TC + r) * CH + th.cl)];
             const float du = dl * u;
             float2 Bp[NP];
@@ -716,7 +728,8 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
 #pragma unroll
         for (int m = kBwdSeg - 1; m >= 0; --m) {
             const int i = sg * kBwdSeg + m, r = DIR ? TC - 1 - i : i;
-            const float2 tk = sm.tok[r * CH + th.cl];                   // u, dy
+            const float2 tk0 = sm.tok[r * CH + th.cl];                  // u, dy
+            const float2 tk = f2(u_of_dir<N, U2>(sm, DIR, r, th.cl, tk0.x), tk0.y);
             const float2 ds = sm.dsg[(DIR * TC + r) * CH + th.cl];      // Delta, sigmoid
             const float dl = ds.x, sgm = ds.y, du = dl * tk.x;
             float2 Bp[NP], Cp[NP], v[NP];
@@ -804,7 +817,8 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
             // du and d delta_raw of one token of the segment per lane of the channel
             const int ox = reduce_scatter<2 * kBwdSeg, 1, Q>(xq, th.lane);
             const int ix = sg * kBwdSeg + kBwdSeg - 1 - ox / 2, rx = DIR ? TC - 1 - ix : ix;
-            const float2 tk = sm.tok[rx * CH + th.cl];   // u, dy
+            const float2 tk0 = sm.tok[rx * CH + th.cl];   // u, dy
+            const float2 tk = f2(u_of_dir<N, U2>(sm, DIR, rx, th.cl, tk0.x), tk0.y);
             sm.yb[(DIR * TC + rx) * CH + th.cl] = fmaf(th.Dk, tk.y, xq[0]);
             sm.dd[(DIR * TC + rx) * CH + th.cl] = xq[1];
             dD = fmaf(tk.y, tk.x, dD);
@@ -835,17 +849,17 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
 }
 
 // one sweep of the thread's direction: forward (ADJ false) or adjoint
-template <int N, bool ZOH, bool FAST, bool ADJ>
+template <int N, bool ZOH, bool FAST, bool ADJ, bool U2>
 __device__ __forceinline__ void bwd_sweep(const BwdArgs &p, const BwdSmem<N> &sm, const BwdThread<N> &th) {
     if constexpr ((VIMSCAN_BWD_RTDIR >> (ZOH ? 0 : 1)) & 1) {
-        if constexpr (ADJ) bwd_adjoint<N, -1, ZOH, FAST>(p, sm, th);
-        else bwd_forward<N, -1, ZOH, FAST>(p, sm, th);
+        if constexpr (ADJ) bwd_adjoint<N, -1, ZOH, FAST, U2>(p, sm, th);
+        else bwd_forward<N, -1, ZOH, FAST, U2>(p, sm, th);
     } else if constexpr (ADJ) {
-        if (th.dir == 0) bwd_adjoint<N, 0, ZOH, FAST>(p, sm, th);
-        else bwd_adjoint<N, 1, ZOH, FAST>(p, sm, th);
+        if (th.dir == 0) bwd_adjoint<N, 0, ZOH, FAST, U2>(p, sm, th);
+        else bwd_adjoint<N, 1, ZOH, FAST, U2>(p, sm, th);
     } else {
-        if (th.dir == 0) bwd_forward<N, 0, ZOH, FAST>(p, sm, th);
-        else bwd_forward<N, 1, ZOH, FAST>(p, sm, th);
+        if (th.dir == 0) bwd_forward<N, 0, ZOH, FAST, U2>(p, sm, th);
+        else bwd_forward<N, 1, ZOH, FAST, U2>(p, sm, th);
     }
 }
 
@@ -920,7 +934,9 @@ __device__ __forceinline__ void store_bc_part(const BwdArgs &p, const float *red
     }
 }
 
-template <typename T, int N, bool ZOH>
+// U2: each direction scans its own u, fp32 (the backward one's at p.u +
+// p.u_dir_stride), and dl/du leaves per direction in p.du2 (fp32); the Vim pair only.
+template <typename T, int N, bool ZOH, bool U2 = false>
 __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bwd_main(BwdArgs p) {
     using SH = BwdShape<N>;
     constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
@@ -942,7 +958,8 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
         for (int k = 0; k < kG; ++k) { u[k] = 0.0f; dr[k] = 0.0f; e[k] = 0.0f; zf[k] = 0.0f; }
         if (ok) {
             const size_t i = ((size_t)b * p.L + bpos(p, t0 + r)) * p.Di + ch;
-            load4<T>(p.u, i, vio, u);
+            if constexpr (U2) load4<float>(p.u, i, true, u);   // fp32 pathway inputs
+            else load4<T>(p.u, i, vio, u);
             load4<T>(p.delta, i, vio, dr);
             load4<T>(p.dout, i, vio, e);
             if (p.z) {
@@ -954,6 +971,8 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
                     e[k] *= silu(zz[k]);
                 }
             }
+            // U2: the dz-factor area holds the backward direction's u (dz re-reads its factor)
+            if constexpr (U2) load4<float>(static_cast<const float *>(p.u) + p.u_dir_stride, i, true, zf);
         }
         float ds0[2 * kG], ds1[2 * kG];
 #pragma unroll
@@ -1053,8 +1072,8 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     // general code are separate copies of the sweeps, with no branch between them per
     // token, and a warp fetches only the copy it runs
     const bool fast = ZOH && __all_sync(0xffffffffu, th.structured);
-    if (fast) bwd_sweep<N, ZOH, ZOH, false>(p, sm, th);
-    else bwd_sweep<N, ZOH, false, false>(p, sm, th);
+    if (fast) bwd_sweep<N, ZOH, ZOH, false, U2>(p, sm, th);
+    else bwd_sweep<N, ZOH, false, false, U2>(p, sm, th);
     __syncthreads();
     // dz = dout silu'(z) (sum of the directions' y), and the CTA's dC terms; the
     // cross-scan's first pair leaves its y for the second
@@ -1073,7 +1092,16 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
                         const float4 a = *reinterpret_cast<const float4 *>(p.acc_y + i);
                         y[0] += a.x; y[1] += a.y; y[2] += a.z; y[3] += a.w;
                     }
-                    const float4 f = *reinterpret_cast<const float4 *>(sm.dzf + r * CH + c0);
+                    float4 f;
+                    if constexpr (U2) {   // the factor dout silu'(z), formed again from its inputs
+                        float e[kG], zz[kG];
+                        load4<T>(p.dout, i, vio, e);
+                        load4<T>(p.z, i, vio, zz);
+                        f = make_float4(e[0] * silu_grad(zz[0]), e[1] * silu_grad(zz[1]), e[2] * silu_grad(zz[2]),
+                                        e[3] * silu_grad(zz[3]));
+                    } else {
+                        f = *reinterpret_cast<const float4 *>(sm.dzf + r * CH + c0);
+                    }
                     y[0] *= f.x; y[1] *= f.y; y[2] *= f.z; y[3] *= f.w;
                     store4<T>(p.dz, i, vio, y);
                 }
@@ -1083,8 +1111,8 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     store_bc_part<N>(p, sm.red, p.dC_part, b, t0, tc, blk);
     __syncthreads();
 
-    if (fast) bwd_sweep<N, ZOH, ZOH, true>(p, sm, th);
-    else bwd_sweep<N, ZOH, false, true>(p, sm, th);
+    if (fast) bwd_sweep<N, ZOH, ZOH, true, U2>(p, sm, th);
+    else bwd_sweep<N, ZOH, false, true, U2>(p, sm, th);
     __syncthreads();
     for (int li = threadIdx.x; li < TC * (CH / kG); li += SH::kThr) {
         const int r = li / (CH / kG), c0 = (li % (CH / kG)) * kG, ch = d0 + c0;
@@ -1096,7 +1124,11 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
             const float4 b1 = *reinterpret_cast<const float4 *>(sm.dd + (TC + r) * CH + c0);
             float du[kG] = {a0.x + a1.x, a0.y + a1.y, a0.z + a1.z, a0.w + a1.w};
             float dd[kG] = {b0.x + b1.x, b0.y + b1.y, b0.z + b1.z, b0.w + b1.w};
-            if (p.stage == 1) {
+            if constexpr (U2) {   // dl/du per direction; d delta_raw summed as usual
+                *reinterpret_cast<float4 *>(p.du2 + i) = a0;
+                *reinterpret_cast<float4 *>(p.du2 + (size_t)p.batch * p.L * p.Di + i) = a1;
+                store4<T>(p.ddelta, i, vio, dd);
+            } else if (p.stage == 1) {
                 *reinterpret_cast<float4 *>(p.acc_du + i) = make_float4(du[0], du[1], du[2], du[3]);
                 *reinterpret_cast<float4 *>(p.acc_dd + i) = make_float4(dd[0], dd[1], dd[2], dd[3]);
             } else {
@@ -1112,6 +1144,149 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
         }
     }
     store_bc_part<N>(p, sm.red, p.dB_part, b, t0, tc, blk);
+}
+
+// ----------------------------------------------------------------------------
+// the pathways' convolution fronts and their derivative (vim_scan_bidir_conv_bwd)
+// ----------------------------------------------------------------------------
+// pre_k[t] = cb_k + w_k[0] x[s_k0] + w_k[1] x[t] + w_k[2] x[s_k2], with the forward
+// pathway's taps on x[t-1], x[t], x[t+1] and the backward one's on x[t+1], x[t], x[t-1]
+// (x = 0 outside the sequence); u_k = silu(pre_k).
+template <int K>
+__device__ __forceinline__ float conv_pre(const float *w, float cb, float xm, float x0, float xp) {
+    return K == 0 ? fmaf(w[0], xm, fmaf(w[1], x0, fmaf(w[2], xp, cb))) : fmaf(w[0], xp, fmaf(w[1], x0, fmaf(w[2], xm, cb)));
+}
+
+// u2[k] = u_k for both pathways, [2][batch, L, Di] fp32; one thread per (b, t, four
+// channels)
+template <typename T>
+__global__ void __launch_bounds__(256) conv_front_fwd(const T *x, const float *conv_w, const float *conv_b,
+                                                      float *u2, int batch, int L, int Di, int vec) {
+    const int q4 = Di / 4;
+    const int64_t items = (int64_t)batch * L * q4, plane = (int64_t)batch * L * Di;
+    for (int64_t it = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; it < items;
+         it += (int64_t)gridDim.x * blockDim.x) {
+        const int d = (int)(it % q4) * 4;
+        const int64_t bt = it / q4;
+        const int t = (int)(bt % L);
+        const size_t i = (size_t)bt * Di + d;
+        float xm[4] = {0.f, 0.f, 0.f, 0.f}, x0[4], xp[4] = {0.f, 0.f, 0.f, 0.f};
+        load4<T>(x, i, vec != 0, x0);
+        if (t > 0) load4<T>(x, i - Di, vec != 0, xm);
+        if (t + 1 < L) load4<T>(x, i + Di, vec != 0, xp);
+        float uf[4], ub[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            uf[e] = silu(conv_pre<0>(conv_w + (size_t)(d + e) * 3, conv_b[d + e], xm[e], x0[e], xp[e]));
+            ub[e] = silu(conv_pre<1>(conv_w + (size_t)(Di + d + e) * 3, conv_b[Di + d + e], xm[e], x0[e], xp[e]));
+        }
+        *reinterpret_cast<float4 *>(u2 + i) = make_float4(uf[0], uf[1], uf[2], uf[3]);
+        *reinterpret_cast<float4 *>(u2 + plane + i) = make_float4(ub[0], ub[1], ub[2], ub[3]);
+    }
+}
+
+// Derivative of the fronts from dl/du_k (du2, fp32): with dpre_k = dl/du_k silu'(pre_k),
+//   dl/dx[t]  = w_f[0] dpre_f[t+1] + w_f[1] dpre_f[t] + w_f[2] dpre_f[t-1]
+//             + w_b[0] dpre_b[t-1] + w_b[1] dpre_b[t] + w_b[2] dpre_b[t+1],
+//   dl/dw_k[j] = sum_t dpre_k[t] x[s_kj(t)],   dl/dcb_k = sum_t dpre_k[t].
+// One thread per (b, run of kFrontRows tokens, four channels) walks its tokens with a
+// window of x and dpre one token either side; it writes dx and one row of partial sums
+// part[b * runs + run][8 Di] = [dw: (k * Di + d) * 3 + j | dcb: 6 Di + k * Di + d].
+constexpr int kFrontRows = 64;
+template <typename T>
+__global__ void __launch_bounds__(256) conv_front_bwd(const T *x, const float *conv_w, const float *conv_b,
+                                                      const float *du2, T *dx, float *part, int batch, int L, int Di,
+                                                      int vec) {
+    const int q4 = Di / 4, runs = (L + kFrontRows - 1) / kFrontRows;
+    const int64_t items = (int64_t)batch * runs * q4, plane = (int64_t)batch * L * Di;
+    const int64_t it = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (it >= items) return;
+    const int d = (int)(it % q4) * 4;
+    const int run = (int)((it / q4) % runs), b = (int)(it / ((int64_t)q4 * runs));
+    const int r0 = run * kFrontRows, r1 = min(L, r0 + kFrontRows);
+    const size_t base = (size_t)b * L * Di + d;   // element of (b, t = 0, d)
+    float w[2][4][3], cb[2][4];
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            cb[k][e] = conv_b[k * Di + d + e];
+#pragma unroll
+            for (int j = 0; j < 3; ++j) w[k][e][j] = conv_w[((size_t)k * Di + d + e) * 3 + j];
+        }
+    auto xrow = [&](int t, float (&v)[4]) {
+        if (t >= 0 && t < L) load4<T>(x, base + (size_t)t * Di, vec != 0, v);
+        else v[0] = v[1] = v[2] = v[3] = 0.0f;
+    };
+    // dpre of both pathways at token t from x[t-1], x[t], x[t+1]; zero outside the sequence
+    auto dpre_at = [&](int t, const float (&xm)[4], const float (&x0)[4], const float (&xp)[4], float (&o)[2][4]) {
+        if (t < 0 || t >= L) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[0][e] = o[1][e] = 0.0f;
+            return;
+        }
+        const float4 gf = *reinterpret_cast<const float4 *>(du2 + base + (size_t)t * Di);
+        const float4 gb = *reinterpret_cast<const float4 *>(du2 + plane + base + (size_t)t * Di);
+        const float df[4] = {gf.x, gf.y, gf.z, gf.w}, db[4] = {gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            o[0][e] = df[e] * silu_grad(conv_pre<0>(w[0][e], cb[0][e], xm[e], x0[e], xp[e]));
+            o[1][e] = db[e] * silu_grad(conv_pre<1>(w[1][e], cb[1][e], xm[e], x0[e], xp[e]));
+        }
+    };
+    float xa[4], xb[4], xc[4], xd[4];   // x[t-1], x[t], x[t+1], x[t+2]
+    float pm[2][4], p0[2][4], pp[2][4];   // dpre at t-1, t, t+1
+    {
+        float xz[4];
+        xrow(r0 - 2, xz);
+        xrow(r0 - 1, xa);
+        xrow(r0, xb);
+        xrow(r0 + 1, xc);
+        dpre_at(r0 - 1, xz, xa, xb, pm);
+        dpre_at(r0, xa, xb, xc, p0);
+    }
+    float dw[2][4][3], dcb[2][4];
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            dcb[k][e] = 0.0f;
+            dw[k][e][0] = dw[k][e][1] = dw[k][e][2] = 0.0f;
+        }
+    for (int t = r0; t < r1; ++t) {
+        xrow(t + 2, xd);
+        dpre_at(t + 1, xb, xc, xd, pp);
+        float g[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            g[e] = w[0][e][0] * pp[0][e] + w[0][e][1] * p0[0][e] + w[0][e][2] * pm[0][e] +
+                   w[1][e][0] * pm[1][e] + w[1][e][1] * p0[1][e] + w[1][e][2] * pp[1][e];
+            dcb[0][e] += p0[0][e];
+            dcb[1][e] += p0[1][e];
+            dw[0][e][0] = fmaf(p0[0][e], xa[e], dw[0][e][0]);   // forward taps: x[t-1], x[t], x[t+1]
+            dw[0][e][1] = fmaf(p0[0][e], xb[e], dw[0][e][1]);
+            dw[0][e][2] = fmaf(p0[0][e], xc[e], dw[0][e][2]);
+            dw[1][e][0] = fmaf(p0[1][e], xc[e], dw[1][e][0]);   // backward taps: x[t+1], x[t], x[t-1]
+            dw[1][e][1] = fmaf(p0[1][e], xb[e], dw[1][e][1]);
+            dw[1][e][2] = fmaf(p0[1][e], xa[e], dw[1][e][2]);
+        }
+        store4<T>(dx, base + (size_t)t * Di, vec != 0, g);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            xa[e] = xb[e]; xb[e] = xc[e]; xc[e] = xd[e];
+            pm[0][e] = p0[0][e]; pm[1][e] = p0[1][e];
+            p0[0][e] = pp[0][e]; p0[1][e] = pp[1][e];
+        }
+    }
+    float *row = part + ((size_t)b * runs + run) * (8 * (size_t)Di);
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+#pragma unroll
+            for (int j = 0; j < 3; ++j) row[((size_t)k * Di + d + e) * 3 + j] = dw[k][e][j];
+            row[6 * (size_t)Di + k * Di + d + e] = dcb[k][e];
+        }
 }
 
 // dB / dC: sum of the per-CTA (or per-cluster) partials, [batch][L][ncol][N] -> [batch][L][N]

@@ -76,6 +76,15 @@ lib.vim_scan_bidir_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, 
                                        _i, _i, _i, _i, _i, _vp]
 lib.vim_scan_bidir_noalloc.restype = _i
 VIM_NOALLOC_SCRATCH_BYTES = 8 << 20
+lib.vim_scan_bidir_conv_bwd_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
+                                           _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                           _i, _i, _i, _i, _i, _u, _vp, _sz, _vp]
+lib.vim_scan_bidir_conv_bwd_ex.restype = _i
+lib.vim_scan_bidir_conv_bwd.argtypes = (lib.vim_scan_bidir_conv_bwd_ex.argtypes[:27]
+                                        + lib.vim_scan_bidir_conv_bwd_ex.argtypes[28:])
+lib.vim_scan_bidir_conv_bwd.restype = _i
+lib.vim_scan_conv_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
+lib.vim_scan_conv_bwd_workspace_bytes.restype = _sz
 lib.vim_scan_bidir_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
                                     _i, _i, _i, _i, _i, _u, _i, _vp, _sz, _vp, _vp, _vp]
 lib.vim_scan_bidir_host.restype = _i
@@ -306,6 +315,59 @@ def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stri
         batch, L, Di, N, dt, *flags, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream), *extra)
     if st != VIM_OK:
         raise VimScanError(st, "vim_scan_bidir_bwd")
+    return out
+
+
+def vim_scan_conv_bwd_workspace_bytes(batch, L, d_inner, d_state, dtype_code, separate_bc):
+    return int(lib.vim_scan_conv_bwd_workspace_bytes(batch, L, d_inner, d_state, dtype_code, int(bool(separate_bc))))
+
+
+def vim_scan_bidir_conv_bwd(x, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stride=0,
+                            workspace=None, stream=None, out=None, zoh=False):
+    """Derivatives of vim_scan_bidir_conv (first-order Bbar, or with ``zoh`` the exact
+    hold) for a loss whose derivative with respect to y is ``dout``; see
+    include/vimscan.h.
+
+    Returns a dict: dx, ddelta (w.r.t. the raw delta), dz (None without z) in the input
+    dtype; dconv_w [2, d_inner, 3] and dconv_b [2, d_inner] fp32; dB, dC (fp32, shaped
+    like B and C), dA [2, d_inner, d_state], dD and ddelta_bias [2, d_inner] fp32.
+    ``out`` may hold those tensors from an earlier call to be written again.
+    """
+    batch, L, Di = x.shape
+    N = B.shape[-1]
+    dt = _dtype_code(x)
+    dev = x.device
+    act = (batch, L, Di)
+    bc = _bc_rule(batch, L, N, bc_dir_stride)
+    if out is not None:
+        if z is not None and out["dz"] is None:
+            raise ValueError("vim_scan_bidir_conv_bwd: out['dz'] is needed when z is given")
+    elif isinstance(x, torch.Tensor) and x.is_cuda:
+        e32 = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
+        out = dict(dx=torch.empty_like(x), ddelta=torch.empty_like(x), dz=torch.empty_like(x) if z is not None else None,
+                   dconv_w=e32(2, Di, 3), dconv_b=e32(2, Di),
+                   dB=torch.zeros(B.shape, dtype=torch.float32, device=dev),
+                   dC=torch.zeros(C.shape, dtype=torch.float32, device=dev),
+                   dA=e32(2, Di, N), dD=e32(2, Di), ddelta_bias=e32(2, Di))
+    f32, io = torch.float32, x.dtype
+    specs = [("x", x, None, act), ("conv_w", conv_w, f32, (2, Di, 3)), ("conv_b", conv_b, f32, (2, Di)),
+             ("delta", delta, io, act), ("z", z, io, act), ("B", B, io, bc), ("C", C, io, bc),
+             ("A", A, f32, (2, Di, N)), ("D", D, f32, (2, Di)), ("delta_bias", delta_bias, f32, (2, Di)),
+             ("dout", dout, io, act)]
+    if out is not None:
+        specs += [("out['dx']", out["dx"], io, act), ("out['dconv_w']", out["dconv_w"], f32, (2, Di, 3)),
+                  ("out['dconv_b']", out["dconv_b"], f32, (2, Di)), ("out['ddelta']", out["ddelta"], io, act),
+                  ("out['dz']", out["dz"], io, act), ("out['dB']", out["dB"], f32, bc),
+                  ("out['dC']", out["dC"], f32, bc), ("out['dA']", out["dA"], f32, (2, Di, N)),
+                  ("out['dD']", out["dD"], f32, (2, Di)), ("out['ddelta_bias']", out["ddelta_bias"], f32, (2, Di))]
+    ptrs = _ptrs("vim_scan_bidir_conv_bwd", x, specs)
+    ws, ws_bytes = _workspace(vim_scan_conv_bwd_workspace_bytes(batch, L, Di, N, dt, bc_dir_stride > 0), workspace,
+                              dev)
+    st = lib.vim_scan_bidir_conv_bwd_ex(
+        *ptrs[:7], int(bc_dir_stride), *ptrs[7:], batch, L, Di, N, dt, VIM_FLAG_ZOH_EXACT if zoh else 0,
+        None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
+    if st != VIM_OK:
+        raise VimScanError(st, "vim_scan_bidir_conv_bwd")
     return out
 
 
