@@ -230,6 +230,9 @@ def run_oracle(w, x, threads, zoh=False):
     if "Wx" in x:
         oracle.vim_block_scan(x["u"], x["Wx"], x["Wdt"], x["A"], x["D"], x["dt_bias"], x["z"],
                               conv_w=x["conv_w"], conv_b=x["conv_b"])
+    elif "dout" in x and "conv_w" in x:
+        oracle.vim_bidir_conv_bwd(x["u"], x["conv_w"], x["conv_b"], x["delta"], x["z"], x["B"], x["C"], x["A"],
+                                  x["D"], x["delta_bias"], x["dout"], zoh=zoh)
     elif "dout" in x and w.kind == "vim":
         oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["delta_bias"], x["dout"],
                              zoh=zoh)
@@ -423,8 +426,8 @@ def main():
         raise SystemExit("--conv and --block apply to the Vim workloads only")
     if args.block and (args.conv or args.zoh or args.bwd or w.dtype != "bf16"):
         raise SystemExit("--block runs alone, on a bf16 workload")
-    if args.bwd and args.conv:
-        raise SystemExit("--bwd covers the scan without the front (--zoh allowed)")
+    if args.bwd and args.conv and w.kind != "vim":
+        raise SystemExit("--bwd --conv applies to the Vim workloads only")
     if args.impl == "reference":
         reference_arm(args, w)
         return
@@ -463,6 +466,10 @@ def main():
             s["out"] = dict(du=torch.empty_like(s["u"]), ddelta=torch.empty_like(s["u"]), dz=torch.empty_like(s["u"]),
                             dB=f32(*s["B"].shape), dC=f32(*s["C"].shape), dA=f32(w.directions, w.channels, w.d_state),
                             dD=f32(w.directions, w.channels), ddelta_bias=f32(w.directions, w.channels))
+            if args.conv:   # x's derivative in place of u's, and the fronts' parameters
+                s["out"]["dx"] = s["out"].pop("du")
+                s["out"]["dconv_w"] = f32(2, w.channels, 3)
+                s["out"]["dconv_b"] = f32(2, w.channels)
         sets.append(s)
     if w.kind == "vim":
         ws_bytes = vs.vim_scan_workspace_bytes(0, w.batch, w.L, 0, w.channels, w.d_state)
@@ -470,6 +477,9 @@ def main():
         ws_bytes = vs.vim_scan_workspace_bytes(1, w.batch, w.H, w.W, w.channels, w.d_state)
     if args.bwd and w.kind == "vim":
         ws_bytes = vs.vim_scan_bwd_workspace_bytes(w.batch, w.L, w.channels, w.d_state, False)
+        if args.conv:
+            ws_bytes = vs.vim_scan_conv_bwd_workspace_bytes(w.batch, w.L, w.channels, w.d_state,
+                                                            vs.VIM_F32 if w.dtype == "f32" else vs.VIM_BF16, False)
     elif args.bwd:
         ws_bytes = int(vs.lib.vmamba_cross_scan4_bwd_workspace_bytes(w.batch, w.H, w.W, w.channels, w.d_state))
     if args.block:
@@ -489,6 +499,12 @@ def main():
             vs.vim_block_scan(s["u"], params["Wx"], params["Wdt"], params["dt_bias"], params["A"], params["D"],
                               s["z"], conv_w=params["conv_w"], conv_b=params["conv_b"], y=s["y"], workspace=ws,
                               events=events)
+            return
+        if args.bwd and args.conv:
+            # u holds x; the derivative through the pathways' convolution fronts
+            vs.vim_scan_bidir_conv_bwd(s["u"], params["conv_w"], params["conv_b"], s["delta"], s["z"], s["B"], s["C"],
+                                       params["A"], params["D"], params["delta_bias"], s["dout"], workspace=ws,
+                                       out=s["out"], zoh=args.zoh)
             return
         if args.bwd and w.kind == "vim":
             vs.vim_scan_bidir_bwd(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"],
@@ -536,8 +552,10 @@ def main():
     kernels_per_pair = 3
     pairs = 1 if w.kind == "vim" else 2
     nev = 4 if args.bwd else (5 if args.block else 1 + kernels_per_pair * pairs)
-    if args.bwd and w.kind != "vim":
-        nev = 2       # the cross-scan derivative has no per-phase events: the whole call is timed
+    whole_call = args.bwd and (w.kind != "vim" or args.conv)
+    if whole_call:
+        nev = 2       # the cross-scan's and the front's derivatives have no per-phase events:
+                      # the whole call is timed
     prof_steps = min(args.steps, 200)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(prof_steps)]
     for i in range(prof_steps):
@@ -549,7 +567,7 @@ def main():
             t = [evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(prof_steps)]
             per_kernel[name] = sum(t) / len(t)
         launches_per_step = 1 + (3 if w.tokens > 256 else 1)
-    elif args.bwd and w.kind != "vim":
+    elif whole_call:
         t = []
         for i in range(prof_steps):
             e0, e1 = evs[i]
@@ -558,10 +576,17 @@ def main():
             e1.record()
         torch.cuda.synchronize()
         t = [evs[i][0].elapsed_time(evs[i][1]) for i in range(prof_steps)]
-        per_kernel["vmamba_cross_scan4_bwd"] = sum(t) / len(t)
-        # per pair: pair_carry, pair_combine, adj_carry, pair_combine, bwd_main, four dB/dC
-        # reductions, one two-pass column sum
-        launches_per_step = 2 * ((4 if w.tokens > 32 else 0) + 1 + 4 + 2)
+        if args.conv:
+            per_kernel["vim_scan_bidir_conv_bwd"] = sum(t) / len(t)
+            # the fronts' forward kernel, pair_carry, pair_combine, adj_carry, pair_combine,
+            # bwd_main, two dB/dC reductions, two column sums for the parameters, the
+            # fronts' derivative and two column sums for their taps and biases
+            launches_per_step = 1 + (4 if w.tokens > 32 else 0) + 1 + 2 + 2 + 1 + 2
+        else:
+            per_kernel["vmamba_cross_scan4_bwd"] = sum(t) / len(t)
+            # per pair: pair_carry, pair_combine, adj_carry, pair_combine, bwd_main, four
+            # dB/dC reductions, one two-pass column sum
+            launches_per_step = 2 * ((4 if w.tokens > 32 else 0) + 1 + 4 + 2)
     elif args.bwd:
         for a, name in enumerate(["summaries", "bwd_main", "reductions"], start=1):
             t = [evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(prof_steps)]
@@ -582,7 +607,7 @@ def main():
     # ---- end to end: pinned host inputs -> device -> scan -> host result ---------
     pinned = {k: host[k].pin_memory() for k in act_keys}
     if args.bwd:
-        res_dev = [sets[0]["out"][k] for k in ("du", "ddelta", "dz", "dB", "dC")]
+        res_dev = [sets[0]["out"][k] for k in ("dx" if args.conv else "du", "ddelta", "dz", "dB", "dC")]
     else:
         res_dev = [sets[0]["y"]]
     res_host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in res_dev]
@@ -634,8 +659,8 @@ def main():
     pk = peaks()
     nbytes, ops = algorithmic_bwd(w) if args.bwd else algorithmic(w, args.conv)
     main_name = "bwd_main" if args.bwd else "pair_main"
-    if args.bwd and w.kind != "vim":
-        main_name = "vmamba_cross_scan4_bwd"     # the whole call (all its kernels)
+    if whole_call:
+        main_name = "vim_scan_bidir_conv_bwd" if args.conv else "vmamba_cross_scan4_bwd"   # the whole call
     main_ms = sum(v for k, v in per_kernel.items() if k.startswith(main_name))
     clocks = clk.summary()
     peak_ops = SMS * FP32_LANES_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e12
