@@ -1192,7 +1192,10 @@ __global__ void __launch_bounds__(256) conv_front_fwd(const T *x, const float *c
 // One thread per (b, run of kFrontRows tokens, four channels) walks its tokens with a
 // window of x and dpre one token either side; it writes dx and one row of partial sums
 // part[b * runs + run][8 Di] = [dw: (k * Di + d) * 3 + j | dcb: 6 Di + k * Di + d].
-constexpr int kFrontRows = 64;
+#ifndef VIMSCAN_FRONT_ROWS
+#define VIMSCAN_FRONT_ROWS 64
+#endif
+constexpr int kFrontRows = VIMSCAN_FRONT_ROWS;   // tokens one thread of conv_front_bwd walks
 template <typename T>
 __global__ void __launch_bounds__(256) conv_front_bwd(const T *x, const float *conv_w, const float *conv_b,
                                                       const float *du2, T *dx, float *part, int batch, int L, int Di,
