@@ -63,6 +63,7 @@ class Oracle:
         lib.oracle_vim_bidir_bwd.argtypes = [_D, _D, _D, _D, _D, ctypes.c_int64] + [_D] * 12 + [ctypes.c_int] * 6
         lib.oracle_cross_scan4_bwd.argtypes = [_D] * 17 + [ctypes.c_int] * 7
         lib.oracle_vim_bidir_conv_bwd.argtypes = [_D] * 7 + [ctypes.c_int64] + [_D] * 14 + [ctypes.c_int] * 6
+        lib.oracle_vim_block_scan_bwd.argtypes = [_D] * 19 + [ctypes.c_int] * 4
         lib.oracle_xproj.argtypes = [_D, _D, _D, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
@@ -244,6 +245,29 @@ class Oracle:
             y *= z / (1.0 + np.exp(-z))
         return y
 
+    def vim_block_scan_bwd(self, x, Wx, Wdt, A, D, bias, z, dout, *, conv_w=None, conv_b=None):
+        """Derivatives of vim_block_scan (first-order Bbar) for the loss sum(dout * y).
+
+        Returns a dict of fp64 arrays: dx [batch, L, Di], dz (None without a gate), dWx
+        [2, Di, 2N+1], dWdt, dbias, dD [2, Di], dA [2, Di, N], and with the convolution
+        front dconv_w [2, Di, 3], dconv_b [2, Di] (else None).
+        """
+        x, Wx, Wdt, A, D, bias, z, dout, conv_w, conv_b = map(_f64, (x, Wx, Wdt, A, D, bias, z, dout, conv_w, conv_b))
+        batch, L, Di = x.shape
+        N = A.shape[-1]
+        conv = conv_w is not None
+        out = dict(dx=np.zeros((batch, L, Di)), dz=np.zeros((batch, L, Di)) if z is not None else None,
+                   dWx=np.zeros((2, Di, 2 * N + 1)), dWdt=np.zeros((2, Di)), dbias=np.zeros((2, Di)),
+                   dD=np.zeros((2, Di)), dA=np.zeros((2, Di, N)),
+                   dconv_w=np.zeros((2, Di, 3)) if conv else None, dconv_b=np.zeros((2, Di)) if conv else None)
+        rc = self.lib.oracle_vim_block_scan_bwd(
+            _p(x), _p(conv_w), _p(conv_b), _p(Wx), _p(Wdt), _p(A), _p(D), _p(bias), _p(z), _p(dout), _p(out["dx"]),
+            _p(out["dz"]), _p(out["dWx"]), _p(out["dWdt"]), _p(out["dbias"]), _p(out["dD"]), _p(out["dA"]),
+            _p(out["dconv_w"]), _p(out["dconv_b"]), batch, L, Di, N)
+        if rc:
+            raise ValueError("oracle_vim_block_scan_bwd: bad sizes")
+        return out
+
     def conv_silu(self, x, w, cb, *, reversed=False):
         """silu of the kernel-3 depthwise convolution (zero padding 1) in front of a
         pathway; reversed=True for the backward pathway (taps x[t+1], x[t], x[t-1]).
@@ -371,6 +395,10 @@ def vim_bidir_conv(*a, **k):
 
 def vim_bidir_conv_bwd(*a, **k):
     return default().vim_bidir_conv_bwd(*a, **k)
+
+
+def vim_block_scan_bwd(*a, **k):
+    return default().vim_block_scan_bwd(*a, **k)
 
 
 def cross_merge4(*a, **k):

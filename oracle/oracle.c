@@ -641,6 +641,138 @@ int oracle_xproj(const double *u, const double *Wx, double *P, int64_t M, int Di
 }
 
 /*
+ * Derivative of the Vim block scan with its projections (the composition the Python
+ * side's vim_block_scan evaluates: per pathway k, u_k = silu(conv_k(x)) (conv_w given)
+ * or x, P_k = u_k Wx[k], B_k = P_k[:, 0:N], C_k = P_k[:, N:2N], s_k = P_k[:, 2N],
+ * delta_raw_k[t, d] = s_k[t] Wdt[k][d], y = (S6_f + S6_b) silu(z)), first-order Bbar, for
+ * ell = sum dout * y.  By the chain rule through each step:
+ *   dl/dP_k = [dl/dB_k | dl/dC_k | dl/ds_k],  dl/ds_k[t] = sum_d dl/ddelta_raw_k[t, d] Wdt[k][d],
+ *   dl/dWdt[k][d] = sum_t dl/ddelta_raw_k[t, d] s_k[t],
+ *   dl/du_k += dl/dP_k Wx[k]^T,  dl/dWx[k] = u_k^T dl/dP_k,
+ * and then through the convolution front as in oracle_vim_bidir_conv_bwd (without it,
+ * dl/dx = dl/du_f + dl/du_b).
+ *   x, z, dout : [batch, L, Di] (z may be NULL);  Wx [2][Di][2N+1];  Wdt, bias, D [2][Di];
+ *   A [2][Di][N];  conv_w [2][Di][3], conv_b [2][Di] or both NULL.
+ *   Outputs (overwritten): dx [batch, L, Di]; dz (untouched when z is NULL); dWx
+ *   [2][Di][2N+1]; dWdt, dbias, dD [2][Di]; dA [2][Di][N]; dconv_w, dconv_b (when
+ *   conv_w is given).
+ */
+int oracle_vim_block_scan_bwd(const double *x, const double *conv_w, const double *conv_b, const double *Wx,
+                              const double *Wdt, const double *A, const double *D, const double *bias,
+                              const double *z, const double *dout, double *dx, double *dz, double *dWx,
+                              double *dWdt, double *dbias, double *dD, double *dA, double *dconv_w,
+                              double *dconv_b, int batch, int L, int Di, int N)
+{
+    if (batch < 0 || L < 0 || Di < 0 || N < 1 || (!conv_w != !conv_b)) return -1;
+    const int NO = 2 * N + 1;
+    const int64_t M = (int64_t)batch * L, n_act = M * Di;
+    size_t na = (size_t)(n_act > 0 ? n_act : 1), nm = (size_t)(M > 0 ? M : 1);
+    double *u[2], *du[2], *P[2], *Bk[2], *Ck[2], *dr[2], *ddr[2], *dB[2], *dC[2];
+    double *dy = (double *)malloc(na * sizeof(double)), *ys = (double *)calloc(na, sizeof(double));
+    int64_t *order = (int64_t *)malloc((size_t)(L > 0 ? L : 1) * sizeof(int64_t));
+    int rc = (!dy || !ys || !order) ? -1 : 0;
+    for (int k = 0; k < 2; ++k) {
+        u[k] = (double *)calloc(na, sizeof(double)); du[k] = (double *)calloc(na, sizeof(double));
+        P[k] = (double *)calloc(nm * NO, sizeof(double));
+        Bk[k] = (double *)calloc(nm * N, sizeof(double)); Ck[k] = (double *)calloc(nm * N, sizeof(double));
+        dr[k] = (double *)calloc(na, sizeof(double)); ddr[k] = (double *)calloc(na, sizeof(double));
+        dB[k] = (double *)calloc(nm * N, sizeof(double)); dC[k] = (double *)calloc(nm * N, sizeof(double));
+        if (!u[k] || !du[k] || !P[k] || !Bk[k] || !Ck[k] || !dr[k] || !ddr[k] || !dB[k] || !dC[k]) rc = -1;
+    }
+    /* the forward steps of each pathway */
+    for (int k = 0; k < 2 && !rc; ++k) {
+        if (conv_w) rc |= oracle_conv_silu(x, conv_w + (int64_t)k * Di * 3, conv_b + (int64_t)k * Di, u[k],
+                                           batch, L, Di, k);
+        else for (int64_t i = 0; i < n_act; ++i) u[k][i] = x[i];
+        rc |= oracle_xproj(u[k], Wx + (int64_t)k * Di * NO, P[k], M, Di, NO);
+        for (int64_t m = 0; m < M; ++m) {
+            for (int n = 0; n < N; ++n) {
+                Bk[k][m * N + n] = P[k][m * NO + n];
+                Ck[k][m * N + n] = P[k][m * NO + N + n];
+            }
+            for (int64_t d = 0; d < Di; ++d) dr[k][m * Di + d] = P[k][m * NO + 2 * N] * Wdt[(int64_t)k * Di + d];
+        }
+        for (int64_t t = 0; t < L; ++t) order[t] = k ? L - 1 - t : t;
+        rc |= oracle_s6_direction(u[k], dr[k], Bk[k], Ck[k], A + (int64_t)k * Di * N, D + (int64_t)k * Di,
+                                  bias + (int64_t)k * Di, order, ys, batch, L, Di, N, 1, k, 0);
+    }
+    if (!rc) {
+        for (int64_t i = 0; i < n_act; ++i) {
+            if (z) { dz[i] = dout[i] * ys[i] * silu_grad(z[i]); dy[i] = dout[i] * silu(z[i]); }
+            else dy[i] = dout[i];
+            dx[i] = 0.0;
+        }
+        for (int64_t i = 0; i < 2 * (int64_t)Di * N; ++i) dA[i] = 0.0;
+        for (int64_t i = 0; i < 2 * (int64_t)Di; ++i) { dD[i] = 0.0; dbias[i] = 0.0; dWdt[i] = 0.0; }
+        for (int64_t i = 0; i < 2 * (int64_t)Di * NO; ++i) dWx[i] = 0.0;
+        if (conv_w) {
+            for (int64_t i = 0; i < 6 * (int64_t)Di; ++i) dconv_w[i] = 0.0;
+            for (int64_t i = 0; i < 2 * (int64_t)Di; ++i) dconv_b[i] = 0.0;
+        }
+    }
+    /* the scan's derivative per pathway, then the projections' */
+    for (int k = 0; k < 2 && !rc; ++k) {
+        for (int64_t t = 0; t < L; ++t) order[t] = k ? L - 1 - t : t;
+        rc |= oracle_s6_direction_bwd(u[k], dr[k], Bk[k], Ck[k], A + (int64_t)k * Di * N, D + (int64_t)k * Di,
+                                      bias + (int64_t)k * Di, order, dy, du[k], ddr[k], dB[k], dC[k],
+                                      dA + (int64_t)k * Di * N, dD + (int64_t)k * Di, dbias + (int64_t)k * Di,
+                                      batch, L, Di, N, 1, 0);
+        const double *W = Wx + (int64_t)k * Di * NO, *wdt = Wdt + (int64_t)k * Di;
+        double *dW = dWx + (int64_t)k * Di * NO, *dwdt = dWdt + (int64_t)k * Di;
+        for (int64_t m = 0; m < M && !rc; ++m) {
+            double dP[2 * ORACLE_MAX_STATE + 1];
+            double s = P[k][m * NO + 2 * N], ds = 0.0;
+            for (int64_t d = 0; d < Di; ++d) {
+                ds += ddr[k][m * Di + d] * wdt[d];
+                dwdt[d] += ddr[k][m * Di + d] * s;
+            }
+            for (int n = 0; n < N; ++n) { dP[n] = dB[k][m * N + n]; dP[N + n] = dC[k][m * N + n]; }
+            dP[2 * N] = ds;
+            for (int64_t d = 0; d < Di; ++d) {
+                double acc = 0.0;
+                for (int j = 0; j < NO; ++j) {
+                    acc += dP[j] * W[d * NO + j];
+                    dW[d * NO + j] += u[k][m * Di + d] * dP[j];
+                }
+                du[k][m * Di + d] += acc;
+            }
+        }
+    }
+    /* through the convolution front (or the identity) to x */
+    if (!rc && conv_w) {
+        for (int k = 0; k < 2; ++k) {
+            const double *w = conv_w + (int64_t)k * Di * 3, *cb = conv_b + (int64_t)k * Di;
+            double *dw = dconv_w + (int64_t)k * Di * 3, *dcb = dconv_b + (int64_t)k * Di;
+            for (int64_t b = 0; b < batch; ++b)
+                for (int64_t t = 0; t < L; ++t)
+                    for (int64_t d = 0; d < Di; ++d) {
+                        double pre = cb[d];
+                        for (int j = 0; j < 3; ++j) {
+                            int64_t sx = k ? t + 1 - j : t + j - 1;
+                            if (sx >= 0 && sx < L) pre += w[d * 3 + j] * x[(b * L + sx) * Di + d];
+                        }
+                        double dpre = du[k][(b * L + t) * Di + d] * silu_grad(pre);
+                        dcb[d] += dpre;
+                        for (int j = 0; j < 3; ++j) {
+                            int64_t sx = k ? t + 1 - j : t + j - 1;
+                            if (sx < 0 || sx >= L) continue;
+                            dx[(b * L + sx) * Di + d] += w[d * 3 + j] * dpre;
+                            dw[d * 3 + j] += dpre * x[(b * L + sx) * Di + d];
+                        }
+                    }
+        }
+    } else if (!rc) {
+        for (int64_t i = 0; i < n_act; ++i) dx[i] = du[0][i] + du[1][i];
+    }
+    free(dy); free(ys); free(order);
+    for (int k = 0; k < 2; ++k) {
+        free(u[k]); free(du[k]); free(P[k]); free(Bk[k]); free(Ck[k]); free(dr[k]); free(ddr[k]); free(dB[k]);
+        free(dC[k]);
+    }
+    return rc ? -1 : 0;
+}
+
+/*
  * Derivative of oracle_cross_scan4 (first-order Bbar, or the exact hold when zoh != 0)
  * for ell = sum dout * y, with
  * y = (sum_k y_k) * silu(z): dl/dz = dout (sum_k y_k) silu'(z), and each of the four

@@ -717,6 +717,45 @@ def pin_conv_bwd_identity_taps(orc):
                                rtol=1e-11, atol=1e-13)
 
 
+def pin_block_bwd_finite_differences(orc):
+    """Every derivative of the block scan with its projections (x, both pathways'
+    taps and biases, x_proj's Wx, dt_proj's Wdt and bias, A, D, z) against central
+    finite differences of the forward oracle's loss sum(dout * y) (page "Vision Mamba
+    Guide": the SSM module derives B, C and Delta from its input by x_proj and dt_proj,
+    section "The Selective State Space (S6) Mechanism"; the pathways' "1D Conv -> SiLU",
+    section "2. The Bidirectional Mamba Block"), with and without the convolution front."""
+    for seed, conv in ((151, True), (152, False)):
+        rng = _rng(seed)
+        b, L, Di, N = 1, 5, 3, 2
+        c = dict(x=rng.normal(size=(b, L, Di)), Wx=rng.normal(size=(2, Di, 2 * N + 1)) * 0.6,
+                 Wdt=rng.normal(size=(2, Di)) * 0.8, A=-rng.uniform(0.2, 2.0, size=(2, Di, N)),
+                 D=rng.normal(size=(2, Di)), bias=rng.normal(size=(2, Di)) * 0.5, z=rng.normal(size=(b, L, Di)),
+                 conv_w=rng.normal(size=(2, Di, 3)) * 0.7 if conv else None,
+                 conv_b=rng.normal(size=(2, Di)) * 0.5 if conv else None)
+        dout = rng.normal(size=(b, L, Di))
+
+        def loss(**over):
+            d = {**c, **over}
+            y = orc.vim_block_scan(d["x"], d["Wx"], d["Wdt"], d["A"], d["D"], d["bias"], d["z"],
+                                   conv_w=d["conv_w"], conv_b=d["conv_b"])
+            return float(np.sum(dout * y))
+
+        g = orc.vim_block_scan_bwd(c["x"], c["Wx"], c["Wdt"], c["A"], c["D"], c["bias"], c["z"], dout,
+                                   conv_w=c["conv_w"], conv_b=c["conv_b"])
+        names = [("x", "dx"), ("Wx", "dWx"), ("Wdt", "dWdt"), ("bias", "dbias"), ("A", "dA"), ("D", "dD"),
+                 ("z", "dz")] + ([("conv_w", "dconv_w"), ("conv_b", "dconv_b")] if conv else [])
+        for name, key in names:
+            arr, eps = c[name], 1e-6
+            fd = np.zeros_like(arr)
+            for i in np.ndindex(arr.shape):
+                up, dn = arr.copy(), arr.copy()
+                up[i] += eps
+                dn[i] -= eps
+                fd[i] = (loss(**{name: up}) - loss(**{name: dn})) / (2 * eps)
+            err = np.max(np.abs(fd - g[key])) / np.max(np.abs(fd))
+            assert err < 1e-7, (name, conv, err)
+
+
 ALL_PINS = [
     pin_delta_zero,
     pin_constant_input_geometric,
@@ -743,4 +782,5 @@ ALL_PINS = [
     pin_block_scan_composition,
     pin_conv_bwd_finite_differences,
     pin_conv_bwd_identity_taps,
+    pin_block_bwd_finite_differences,
 ]

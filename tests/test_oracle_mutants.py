@@ -77,6 +77,12 @@ MUTANTS = {
     "conv_bwd_dw_without_x": ("dw[d * 3 + j] += dpre * x[(b * L + s) * Di + d];", "dw[d * 3 + j] += dpre;"),
     "conv_bwd_dx_tap_flipped": ("dx[(b * L + s) * Di + d] += w[d * 3 + j] * dpre;",
                                 "dx[(b * L + s) * Di + d] += w[d * 3 + 2 - j] * dpre;"),
+    # the projections' derivative
+    "block_bwd_ds_without_wdt": ("ds += ddr[k][m * Di + d] * wdt[d];", "ds += ddr[k][m * Di + d];"),
+    "block_bwd_dwx_transposed": ("dW[d * NO + j] += u[k][m * Di + d] * dP[j];",
+                                 "dW[d * NO + j] += u[k][m * Di + d] * dP[NO - 1 - j];"),
+    "block_bwd_du_misses_projection": ("                du[k][m * Di + d] += acc;", "                du[k][m * Di + d] += 0.0 * acc;"),
+    "block_bwd_dwdt_without_s": ("dwdt[d] += ddr[k][m * Di + d] * s;", "dwdt[d] += ddr[k][m * Di + d];"),
     "conv_bwd_shared_du": ("rc |= oracle_s6_direction_bwd(u[1], delta, B + bc_dir_stride, C + bc_dir_stride,\n"
                            "                                      A + (int64_t)Di * N, D + Di, bias + Di, order, dy, du[1],",
                            "rc |= oracle_s6_direction_bwd(u[1], delta, B + bc_dir_stride, C + bc_dir_stride,\n"
