@@ -282,6 +282,31 @@ vim_status vim_block_scan(const void *x, const float *conv_w, const float *conv_
 size_t vim_block_workspace_bytes(int batch, int L, int d_inner, int d_state);
 
 /*
+ * Derivatives of vim_block_scan (first-order Bbar) for a loss whose derivative with
+ * respect to y is dout: the scan's derivative per pathway, carried back through dt_proj
+ * and x_proj (P_k = u_k Wx[k], delta_raw_k = s_k Wdt[k]) and the convolution fronts.
+ *
+ *   x, conv_w, conv_b, Wx, Wdt, dt_bias, A, D, z : as in vim_block_scan (bf16 x, z, Wx).
+ *   dout      : [batch, L, d_inner] bf16.
+ *   Outputs (overwritten): dx [batch, L, d_inner] bf16; dz (NULL exactly when z is);
+ *             dWx [2, d_inner, 2*d_state + 1], dWdt and ddt_bias [2, d_inner], dA [2,
+ *             d_inner, d_state], dD [2, d_inner] fp32; dconv_w [2, d_inner, 3] and
+ *             dconv_b [2, d_inner] fp32 exactly when conv_w and conv_b are given.
+ *   workspace : vim_block_bwd_workspace_bytes(batch, L, d_inner, d_state) bytes,
+ *             256-byte aligned.
+ * The projections are formed again as the forward call forms them (B, C rounded to
+ * bf16, s in fp32); the pathways' inputs u_k are formed in fp32 for the derivative.
+ * Every sum is taken in a fixed order.  Only bf16 I/O (VIM_ERR_UNSUPPORTED else) and
+ * the d_inner limit of vim_block_scan.  Size 0 writes zero parameter derivatives.
+ */
+vim_status vim_block_scan_bwd(const void *x, const float *conv_w, const float *conv_b, const void *Wx,
+                              const float *Wdt, const float *dt_bias, const float *A, const float *D, const void *z,
+                              const void *dout, void *dx, float *dconv_w, float *dconv_b, float *dWx, float *dWdt,
+                              float *ddt_bias, float *dA, float *dD, void *dz, int batch, int L, int d_inner,
+                              int d_state, vim_dtype dt, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+size_t vim_block_bwd_workspace_bytes(int batch, int L, int d_inner, int d_state);
+
+/*
  * Options of the _ex entry points, or-ed into `flags` (unknown bits return
  * VIM_ERR_INVALID_ARG).
  *

@@ -43,6 +43,7 @@ def test_header_declares_the_boundary():
                           "vmamba_cross_scan4_bwd_ex",
                           "vim_scan_bidir_host", "vim_scan_host_workspace_bytes",
                           "vim_scan_bidir_conv_bwd", "vim_scan_bidir_conv_bwd_ex", "vim_scan_conv_bwd_workspace_bytes",
+                          "vim_block_scan_bwd", "vim_block_bwd_workspace_bytes",
                           "vim_scan_workspace_bytes", "vim_status_string"}, names
 
 
@@ -172,6 +173,33 @@ def test_conv_bwd_rejects(vs):
     assert n % 256 == 0 and n > vs.vim_scan_bwd_workspace_bytes(8, 4097, 384, 16, False) + 4 * 8 * 4097 * 384 * 4
     assert f(8, 4097, 384, 16, vs.VIM_BF16, True) > n
     assert f(0, 4097, 384, 16, vs.VIM_BF16, False) == 0 and f(8, 4097, 384, 5, vs.VIM_BF16, False) == 0
+
+
+def test_block_bwd_rejects(vs):
+    f = vs.lib.vim_block_scan_bwd
+
+    def call(**kw):
+        a = dict(x=FAKE, cw=FAKE, cb=FAKE, Wx=FAKE, Wdt=FAKE, bias=FAKE, A=FAKE, D=FAKE, z=FAKE, dout=FAKE, dx=FAKE,
+                 dcw=FAKE, dcb=FAKE, dWx=FAKE, dWdt=FAKE, dbias=FAKE, dA=FAKE, dD=FAKE, dz=FAKE, batch=2, L=100, Di=64,
+                 N=16, dt=vs.VIM_BF16, ws=FAKE, ws_bytes=1 << 40)
+        a.update(kw)
+        return f(a["x"], a["cw"], a["cb"], a["Wx"], a["Wdt"], a["bias"], a["A"], a["D"], a["z"], a["dout"], a["dx"],
+                 a["dcw"], a["dcb"], a["dWx"], a["dWdt"], a["dbias"], a["dA"], a["dD"], a["dz"], a["batch"], a["L"],
+                 a["Di"], a["N"], a["dt"], a["ws"], a["ws_bytes"], None)
+
+    assert call(dt=vs.VIM_F32) == vs.VIM_ERR_UNSUPPORTED
+    assert call(cw=None) == vs.VIM_ERR_INVALID_ARG                      # one of the front's two
+    assert call(dcb=None) == vs.VIM_ERR_INVALID_ARG                     # front given, its derivative not
+    assert call(z=None) == vs.VIM_ERR_INVALID_ARG                       # dz without z
+    assert call(Wx=FAKE + 1) == vs.VIM_ERR_INVALID_ARG
+    assert call(x=FAKE + 8) == vs.VIM_ERR_INVALID_ARG
+    assert call(dWx=None) == vs.VIM_ERR_INVALID_ARG
+    assert call(N=3) == vs.VIM_ERR_UNSUPPORTED
+    assert call(ws=None) == vs.VIM_ERR_WORKSPACE
+    assert call(ws_bytes=1024) == vs.VIM_ERR_WORKSPACE
+    n = vs.vim_block_bwd_workspace_bytes(8, 4097, 384, 16)
+    assert n % 256 == 0 and n > vs.vim_scan_bwd_workspace_bytes(8, 4097, 384, 16, True)
+    assert vs.vim_block_bwd_workspace_bytes(0, 4097, 384, 16) == 0
 
 
 def test_host_workspace_bytes(vs):

@@ -99,3 +99,100 @@ def test_block_full_size(vs):
     p = block_inputs(w.batch, w.L, w.channels, w.d_state, seed=4097, conv=True)
     oracle.set_threads(max(1, len(os.sched_getaffinity(0))))
     gates.gate("block_full_vim_tiny_1024px_bf16", run(vs, p), ref(p), torch.bfloat16, norm_tol=TOL, elementwise=False)
+
+
+# ---------------------------------------------------------------------------
+# the derivative (vim_block_scan_bwd)
+# ---------------------------------------------------------------------------
+BWD_KEYS = ["dx", "dz", "dWx", "dWdt", "ddt_bias", "dA", "dD", "dconv_w", "dconv_b"]
+REF_KEY = {"ddt_bias": "dbias"}
+
+
+def run_bwd(vs, p, dout, gate=True):
+    c = lambda t: None if t is None else t.cuda()
+    out = vs.vim_block_scan_bwd(c(p["x"]), c(p["Wx"]), c(p["Wdt"]), c(p["bias"]), c(p["A"]), c(p["D"]),
+                                c(p["z"]) if gate else None, c(dout), conv_w=c(p["cw"]), conv_b=c(p["cb"]))
+    torch.cuda.synchronize()
+    return out
+
+
+def ref_bwd(p, dout, gate=True):
+    return oracle.vim_block_scan_bwd(p["x"], p["Wx"], p["Wdt"], p["A"], p["D"], p["bias"], p["z"] if gate else None,
+                                     dout, conv_w=p["cw"], conv_b=p["cb"])
+
+
+BWD_CASES = [
+    # batch, L, Di, N, conv, gate
+    (1, 5, 16, 16, True, True),
+    (2, 33, 64, 16, True, True),        # 2 chunks of the derivative, the last 1 token
+    (1, 197, 72, 8, True, True),        # partial channel slices
+    (2, 100, 64, 4, False, True),       # no convolution front
+    (1, 300, 128, 16, True, False),
+    (3, 65, 64, 16, True, True),        # projection tiles across batch boundaries
+    (1, 700, 64, 2, False, False),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=lambda c: f"b{c[0]}_L{c[1]}_D{c[2]}_N{c[3]}"
+                         f"{'_conv' if c[4] else ''}{'' if c[5] else '_nogate'}")
+def test_block_bwd(vs, case):
+    """Every derivative against the oracle's, normwise within the bf16 tolerance: the
+    kernel takes B and C rounded to bf16 (as the forward call does); the oracle exactly."""
+    batch, L, Di, N, conv, gate = case
+    p = block_inputs(batch, L, Di, N, seed=L * 3 + Di, conv=conv)
+    g = torch.Generator().manual_seed(L + 1)
+    dout = torch.randn((batch, L, Di), generator=g).to(torch.bfloat16)
+    got, want = run_bwd(vs, p, dout, gate), ref_bwd(p, dout, gate)
+    for k in BWD_KEYS:
+        w = want[REF_KEY.get(k, k)]
+        if w is None:
+            assert got[k] is None, k
+            continue
+        gates.gate(f"block_bwd_{case}:{k}", got[k], w, torch.bfloat16, norm_tol=TOL, elementwise=False)
+
+
+def test_block_bwd_deterministic(vs):
+    p = block_inputs(2, 300, 64, 16, seed=4, conv=True)
+    dout = torch.randn((2, 300, 64), generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    a, b = run_bwd(vs, p, dout), run_bwd(vs, p, dout)
+    for k in BWD_KEYS:
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_block_bwd_larger(vs):
+    """4097 tokens, batch 2, d_inner 128 with the convolution front, against the oracle."""
+    p = block_inputs(2, 4097, 128, 16, seed=44, conv=True)
+    dout = torch.randn((2, 4097, 128), generator=torch.Generator().manual_seed(45)).to(torch.bfloat16)
+    oracle.set_threads(max(1, len(os.sched_getaffinity(0))))
+    got, want = run_bwd(vs, p, dout), ref_bwd(p, dout)
+    for k in BWD_KEYS:
+        gates.gate(f"block_bwd_4097:{k}", got[k], want[REF_KEY.get(k, k)], torch.bfloat16, norm_tol=TOL,
+                   elementwise=False)
+
+
+def test_block_bwd_exact_projection(vs):
+    """Inputs whose projections are exact in bf16 (no convolution front; x in {0, +-1/2},
+    Wx with at most four entries of +-1/8 per column), so the kernel's B and C equal the
+    oracle's and every fp32 derivative must agree to fp32 accuracy: this isolates the
+    chain through dt_proj and x_proj from the bf16 rounding the other cases allow for."""
+    batch, L, Di, N = 2, 200, 64, 16
+    g = torch.Generator().manual_seed(61)
+    p = block_inputs(batch, L, Di, N, seed=61, conv=False)
+    p["x"] = (torch.randint(-1, 2, (batch, L, Di), generator=g).float() * 0.5).to(torch.bfloat16)
+    Wx = torch.zeros(2, Di, 2 * N + 1)
+    for k in range(2):
+        for j in range(2 * N + 1):
+            rows = torch.randperm(Di, generator=g)[:4]
+            Wx[k, rows, j] = (torch.randint(0, 2, (4,), generator=g).float() * 2 - 1) * 0.125
+    p["Wx"] = Wx.to(torch.bfloat16).contiguous()
+    dout = torch.randn((batch, L, Di), generator=g).to(torch.bfloat16)
+    got, want = run_bwd(vs, p, dout), ref_bwd(p, dout)
+    for k in BWD_KEYS:
+        w = want[REF_KEY.get(k, k)]
+        if w is None:
+            assert got[k] is None, k
+            continue
+        if k in ("dx", "dz"):   # bf16 outputs, rounded once
+            gates.gate(f"block_bwd_exact:{k}", got[k], w, torch.bfloat16)
+        else:
+            gates.gate(f"block_bwd_exact:{k}", got[k], w, torch.float32, norm_tol=5e-5, elementwise=False)

@@ -83,6 +83,9 @@ struct BwdArgs {
     int64_t u_dir_stride;               // with per-direction inputs (bwd_main's U2; u is then fp32):
                                         // elements from the forward direction's u to the backward one's
     float *du2;                         // with U2: [2][batch, L, Di] fp32 dl/du_k per direction
+    const float *dt_in;                 // with DT: [2][batch*L] step input per direction and position;
+    const float *dt_w;                  // [2][Di] dt_proj weights: delta_raw_k = dt_in_k * dt_w_k
+    float *dd2;                         // with DT: [2][batch, L, Di] fp32 dl/ddelta_raw_k per direction
 };
 
 namespace {
@@ -156,10 +159,12 @@ __device__ __forceinline__ float silu_grad(float z) {
 // visited up to and including s.  One thread per (channel, direction), all N states;
 // with A_n = (n+1) A_0 (checked per warp) the weights are powers of one exp.
 // ----------------------------------------------------------------------------
-template <typename T, int N>
+// DT: delta_raw of direction k is dt_in_k[t] * dt_w_k[d] (the projections' step input)
+template <typename T, int N, bool DT = false>
 __global__ void __launch_bounds__(2 * kAdjCh) adj_carry(BwdArgs p) {
-    __shared__ __align__(16) float sDr[kBwdChunk][kAdjCh], sDy[kBwdChunk][kAdjCh];
+    __shared__ __align__(16) float sDr[DT ? 1 : kBwdChunk][kAdjCh], sDy[kBwdChunk][kAdjCh];
     __shared__ __align__(16) float sC[2][kBwdChunk][N];
+    __shared__ float sS[2][DT ? kBwdChunk : 1];
     const int b = blockIdx.z, c = blockIdx.y, d0 = blockIdx.x * kAdjCh;
     const int t0 = c * kBwdChunk, tc = min(kBwdChunk, p.L - t0);
     // four channels per item (d_inner is a multiple of 4)
@@ -168,7 +173,7 @@ __global__ void __launch_bounds__(2 * kAdjCh) adj_carry(BwdArgs p) {
         float dr[4] = {0.0f, 0.0f, 0.0f, 0.0f}, e[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         if (r < tc && ch < p.Di) {
             const size_t i = ((size_t)b * p.L + bpos(p, t0 + r)) * p.Di + ch;
-            load4<T>(p.delta, i, p.vec_io, dr);
+            if constexpr (!DT) load4<T>(p.delta, i, p.vec_io, dr);
             load4<T>(p.dout, i, p.vec_io, e);
             if (p.z) {
                 float zz[4];
@@ -177,8 +182,14 @@ __global__ void __launch_bounds__(2 * kAdjCh) adj_carry(BwdArgs p) {
                 for (int k = 0; k < 4; ++k) e[k] *= silu(zz[k]);
             }
         }
-        *reinterpret_cast<float4 *>(&sDr[r][c0]) = make_float4(dr[0], dr[1], dr[2], dr[3]);
+        if constexpr (!DT) *reinterpret_cast<float4 *>(&sDr[r][c0]) = make_float4(dr[0], dr[1], dr[2], dr[3]);
         *reinterpret_cast<float4 *>(&sDy[r][c0]) = make_float4(e[0], e[1], e[2], e[3]);
+    }
+    if constexpr (DT) {
+        for (int li = threadIdx.x; li < 2 * kBwdChunk; li += 2 * kAdjCh) {
+            const int k = li / kBwdChunk, r = li % kBwdChunk;
+            sS[k][r] = r < tc ? p.dt_in[(size_t)k * p.batch * p.L + (size_t)b * p.L + bpos(p, t0 + r)] : 0.0f;
+        }
     }
     bool c_done = false;
     if constexpr ((N * sizeof(T)) % 16 == 0) {
@@ -220,6 +231,7 @@ __global__ void __launch_bounds__(2 * kAdjCh) adj_carry(BwdArgs p) {
     if (!valid) return;
     const float A0 = Ad[0] * kLog2e;
     const float bias = p.bias[(size_t)dir * p.Di + d];
+    const float wdt = DT ? p.dt_w[(size_t)dir * p.Di + d] : 0.0f;
     float2 G[NP];
 #pragma unroll
     for (int k = 0; k < NP; ++k) G[k] = f2(0.f, 0.f);
@@ -230,7 +242,7 @@ __global__ void __launch_bounds__(2 * kAdjCh) adj_carry(BwdArgs p) {
     for (int i = 0; i < kBwdChunk; ++i) {
         const bool ok = i < tc;
         const int r = ok ? (dir ? tc - 1 - i : i) : 0;
-        S += ok ? softplus_io<T>(sDr[r][dl] + bias) : 0.0f;
+        S += ok ? softplus_io<T>((DT ? sS[dir][r] * wdt : sDr[DT ? 0 : r][dl]) + bias) : 0.0f;
         const float e = ok ? sDy[r][dl] : 0.0f;
         float2 Cv[NP];
         load_row<NP>(&sC[dir][r][0], Cv);
@@ -936,7 +948,9 @@ __device__ __forceinline__ void store_bc_part(const BwdArgs &p, const float *red
 
 // U2: each direction scans its own u, fp32 (the backward one's at p.u +
 // p.u_dir_stride), and dl/du leaves per direction in p.du2 (fp32); the Vim pair only.
-template <typename T, int N, bool ZOH, bool U2 = false>
+// DT: delta_raw of direction k is p.dt_in_k[t] * p.dt_w_k[d], and dl/ddelta_raw leaves
+// per direction in p.dd2 (fp32) instead of summed into p.ddelta.
+template <typename T, int N, bool ZOH, bool U2 = false, bool DT = false>
 __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bwd_main(BwdArgs p) {
     using SH = BwdShape<N>;
     constexpr int NP = SH::NP, Q = SH::Q, CH = SH::CH, TC = SH::TC;
@@ -960,7 +974,7 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
             const size_t i = ((size_t)b * p.L + bpos(p, t0 + r)) * p.Di + ch;
             if constexpr (U2) load4<float>(p.u, i, true, u);   // fp32 pathway inputs
             else load4<T>(p.u, i, vio, u);
-            load4<T>(p.delta, i, vio, dr);
+            if constexpr (!DT) load4<T>(p.delta, i, vio, dr);
             load4<T>(p.dout, i, vio, e);
             if (p.z) {
                 float zz[kG];
@@ -975,11 +989,20 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
             if constexpr (U2) load4<float>(static_cast<const float *>(p.u) + p.u_dir_stride, i, true, zf);
         }
         float ds0[2 * kG], ds1[2 * kG];
+        float sdt0 = 0.0f, sdt1 = 0.0f;   // DT: the two directions' step inputs of this token
+        if constexpr (DT) {
+            if (ok) {
+                const size_t m = (size_t)b * p.L + bpos(p, t0 + r);
+                sdt0 = p.dt_in[m];
+                sdt1 = p.dt_in[(size_t)p.batch * p.L + m];
+            }
+        }
 #pragma unroll
         for (int k = 0; k < kG; ++k) {
             float dl0 = 0.0f, dl1 = 0.0f, sg0 = 0.0f, sg1 = 0.0f;
             if (ok) {
-                const float x0 = dr[k] + p.bias[ch + k], x1 = dr[k] + p.bias[p.Di + ch + k];
+                const float r0 = DT ? sdt0 * p.dt_w[ch + k] : dr[k], r1 = DT ? sdt1 * p.dt_w[p.Di + ch + k] : dr[k];
+                const float x0 = r0 + p.bias[ch + k], x1 = r1 + p.bias[p.Di + ch + k];
                 dl0 = softplus_io<T>(x0); sg0 = softplus_grad(x0);
                 dl1 = softplus_io<T>(x1); sg1 = softplus_grad(x1);
             }
@@ -1124,10 +1147,20 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
             const float4 b1 = *reinterpret_cast<const float4 *>(sm.dd + (TC + r) * CH + c0);
             float du[kG] = {a0.x + a1.x, a0.y + a1.y, a0.z + a1.z, a0.w + a1.w};
             float dd[kG] = {b0.x + b1.x, b0.y + b1.y, b0.z + b1.z, b0.w + b1.w};
-            if constexpr (U2) {   // dl/du per direction; d delta_raw summed as usual
-                *reinterpret_cast<float4 *>(p.du2 + i) = a0;
-                *reinterpret_cast<float4 *>(p.du2 + (size_t)p.batch * p.L * p.Di + i) = a1;
-                store4<T>(p.ddelta, i, vio, dd);
+            if constexpr (U2 || DT) {   // per direction where the mode asks, else summed as usual
+                const size_t plane = (size_t)p.batch * p.L * p.Di;
+                if constexpr (U2) {
+                    *reinterpret_cast<float4 *>(p.du2 + i) = a0;
+                    *reinterpret_cast<float4 *>(p.du2 + plane + i) = a1;
+                } else {
+                    store4<T>(p.du, i, vio, du);
+                }
+                if constexpr (DT) {
+                    *reinterpret_cast<float4 *>(p.dd2 + i) = b0;
+                    *reinterpret_cast<float4 *>(p.dd2 + plane + i) = b1;
+                } else {
+                    store4<T>(p.ddelta, i, vio, dd);
+                }
             } else if (p.stage == 1) {
                 *reinterpret_cast<float4 *>(p.acc_du + i) = make_float4(du[0], du[1], du[2], du[3]);
                 *reinterpret_cast<float4 *>(p.acc_dd + i) = make_float4(dd[0], dd[1], dd[2], dd[3]);

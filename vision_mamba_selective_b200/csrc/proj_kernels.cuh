@@ -15,6 +15,9 @@
 // the tensor pipe.
 #pragma once
 
+#include <algorithm>
+#include <atomic>
+
 #include "scan_kernels.cuh"
 
 namespace vimscan {
@@ -239,6 +242,41 @@ __global__ void __launch_bounds__(kProjThreads) xproj_kernel(ProjArgs p) {
         // sU and this step's sX buffer are rewritten two steps on: the barrier at the
         // top of the next step orders the reads above before those writes
     }
+}
+
+// ----------------------------------------------------------------------------
+// launch of the projection kernel (host side)
+// ----------------------------------------------------------------------------
+template <int N, bool CONV>
+vim_status launch_proj_c(const ProjArgs &pa, cudaStream_t stream) {
+    const size_t sm = ProjShape<N>::smem_bytes(pa.Di);
+    auto kernel = xproj_kernel<N, CONV>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
+        return VIM_ERR_CUDA;
+    // resident CTAs per SM for this variant and d_inner, looked up once (per device: the
+    // first device's answer serves every B200 of a node)
+    static std::atomic<int> cached_sms{0}, cached_per_sm{0}, cached_di{-1};
+    int sms = cached_sms.load(), per_sm = cached_per_sm.load();
+    if (sms == 0 || cached_di.load() != pa.Di) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kProjThreads, sm) != cudaSuccess)
+            return VIM_ERR_CUDA;
+        cached_sms.store(sms);
+        cached_per_sm.store(per_sm);
+        cached_di.store(pa.Di);
+    }
+    // each pathway's tiles spread over about half the resident CTAs; Wx is staged once per CTA
+    const int64_t tiles = (pa.M + kProjRows - 1) / kProjRows;
+    const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(tiles, (int64_t)sms * std::max(per_sm, 1) / 2));
+    kernel<<<dim3(2, (unsigned)ctas), kProjThreads, sm, stream>>>(pa);
+    return cudaGetLastError() == cudaSuccess ? VIM_OK : VIM_ERR_CUDA;
+}
+
+template <int N>
+vim_status launch_proj(const ProjArgs &pa, bool conv, cudaStream_t stream) {
+    return conv ? launch_proj_c<N, true>(pa, stream) : launch_proj_c<N, false>(pa, stream);
 }
 
 }  // namespace

@@ -85,6 +85,10 @@ lib.vim_scan_bidir_conv_bwd.argtypes = (lib.vim_scan_bidir_conv_bwd_ex.argtypes[
 lib.vim_scan_bidir_conv_bwd.restype = _i
 lib.vim_scan_conv_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
 lib.vim_scan_conv_bwd_workspace_bytes.restype = _sz
+lib.vim_block_scan_bwd.argtypes = [_vp] * 19 + [_i, _i, _i, _i, _i, _vp, _sz, _vp]
+lib.vim_block_scan_bwd.restype = _i
+lib.vim_block_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i]
+lib.vim_block_bwd_workspace_bytes.restype = _sz
 lib.vim_scan_bidir_host.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp,
                                     _i, _i, _i, _i, _i, _u, _i, _vp, _sz, _vp, _vp, _vp]
 lib.vim_scan_bidir_host.restype = _i
@@ -436,6 +440,53 @@ def vim_block_scan(x, Wx, Wdt, dt_bias, A, D, z, *, conv_w=None, conv_b=None, y=
     if st != VIM_OK:
         raise VimScanError(st, "vim_block_scan")
     return y
+
+
+def vim_block_bwd_workspace_bytes(batch, L, d_inner, d_state):
+    return int(lib.vim_block_bwd_workspace_bytes(batch, L, d_inner, d_state))
+
+
+def vim_block_scan_bwd(x, Wx, Wdt, dt_bias, A, D, z, dout, *, conv_w=None, conv_b=None, workspace=None, stream=None,
+                       out=None):
+    """Derivatives of vim_block_scan for a loss whose derivative with respect to y is
+    ``dout``; see include/vimscan.h.  bf16 x, z, dout, Wx.
+
+    Returns a dict: dx, dz (None without z) in bf16; dWx [2, d_inner, 2N+1], dWdt,
+    ddt_bias, dD [2, d_inner], dA [2, d_inner, N] fp32; dconv_w [2, d_inner, 3] and
+    dconv_b [2, d_inner] fp32 with the convolution front (else None).  ``out`` may hold
+    those tensors from an earlier call.
+    """
+    batch, L, Di = x.shape
+    N = A.shape[-1]
+    NO = 2 * N + 1
+    dev = x.device
+    act = (batch, L, Di)
+    conv = conv_w is not None
+    if out is not None:
+        if (z is not None) != (out["dz"] is not None) or conv != (out["dconv_w"] is not None):
+            raise ValueError("vim_block_scan_bwd: out['dz'] and out['dconv_w'] must match z and conv_w")
+    elif isinstance(x, torch.Tensor) and x.is_cuda:
+        e32 = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
+        out = dict(dx=torch.empty_like(x), dz=torch.empty_like(x) if z is not None else None, dWx=e32(2, Di, NO),
+                   dWdt=e32(2, Di), ddt_bias=e32(2, Di), dA=e32(2, Di, N), dD=e32(2, Di),
+                   dconv_w=e32(2, Di, 3) if conv else None, dconv_b=e32(2, Di) if conv else None)
+    f32, io = torch.float32, x.dtype
+    specs = [("x", x, None, act), ("conv_w", conv_w, f32, (2, Di, 3)), ("conv_b", conv_b, f32, (2, Di)),
+             ("Wx", Wx, io, (2, Di, NO)), ("Wdt", Wdt, f32, (2, Di)), ("dt_bias", dt_bias, f32, (2, Di)),
+             ("A", A, f32, (2, Di, N)), ("D", D, f32, (2, Di)), ("z", z, io, act), ("dout", dout, io, act)]
+    if out is not None:
+        specs += [("out['dx']", out["dx"], io, act), ("out['dconv_w']", out["dconv_w"], f32, (2, Di, 3)),
+                  ("out['dconv_b']", out["dconv_b"], f32, (2, Di)), ("out['dWx']", out["dWx"], f32, (2, Di, NO)),
+                  ("out['dWdt']", out["dWdt"], f32, (2, Di)), ("out['ddt_bias']", out["ddt_bias"], f32, (2, Di)),
+                  ("out['dA']", out["dA"], f32, (2, Di, N)), ("out['dD']", out["dD"], f32, (2, Di)),
+                  ("out['dz']", out["dz"], io, act)]
+    ptrs = _ptrs("vim_block_scan_bwd", x, specs)
+    ws, ws_bytes = _workspace(vim_block_bwd_workspace_bytes(batch, L, Di, N), workspace, dev)
+    st = lib.vim_block_scan_bwd(*ptrs, batch, L, Di, N, _dtype_code(x), None if ws is None else ws.data_ptr(),
+                                ws_bytes, _stream(stream))
+    if st != VIM_OK:
+        raise VimScanError(st, "vim_block_scan_bwd")
+    return out
 
 
 def vim_scan_bidir_noalloc(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride=0, stream=None):
