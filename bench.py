@@ -227,7 +227,10 @@ def run_oracle(w, x, threads, zoh=False):
 
     oracle.set_threads(threads)
     t = time.perf_counter()
-    if "Wx" in x:
+    if "Wx" in x and "dout" in x:
+        oracle.vim_block_scan_bwd(x["u"], x["Wx"], x["Wdt"], x["A"], x["D"], x["dt_bias"], x["z"], x["dout"],
+                                  conv_w=x["conv_w"], conv_b=x["conv_b"])
+    elif "Wx" in x:
         oracle.vim_block_scan(x["u"], x["Wx"], x["Wdt"], x["A"], x["D"], x["dt_bias"], x["z"],
                               conv_w=x["conv_w"], conv_b=x["conv_b"])
     elif "dout" in x and "conv_w" in x:
@@ -424,8 +427,8 @@ def main():
     w = wl.BY_NAME[args.workload]
     if (args.conv or args.block) and w.kind != "vim":
         raise SystemExit("--conv and --block apply to the Vim workloads only")
-    if args.block and (args.conv or args.zoh or args.bwd or w.dtype != "bf16"):
-        raise SystemExit("--block runs alone, on a bf16 workload")
+    if args.block and (args.conv or args.zoh or w.dtype != "bf16"):
+        raise SystemExit("--block runs alone (or with --bwd), on a bf16 workload")
     if args.bwd and args.conv and w.kind != "vim":
         raise SystemExit("--bwd --conv applies to the Vim workloads only")
     if args.impl == "reference":
@@ -470,6 +473,11 @@ def main():
                 s["out"]["dx"] = s["out"].pop("du")
                 s["out"]["dconv_w"] = f32(2, w.channels, 3)
                 s["out"]["dconv_b"] = f32(2, w.channels)
+            if args.block:  # the block's parameters: projections, fronts, A, D
+                s["out"] = dict(dx=torch.empty_like(s["u"]), dz=torch.empty_like(s["u"]),
+                                dWx=f32(2, w.channels, 2 * w.d_state + 1), dWdt=f32(2, w.channels),
+                                ddt_bias=f32(2, w.channels), dA=f32(2, w.channels, w.d_state), dD=f32(2, w.channels),
+                                dconv_w=f32(2, w.channels, 3), dconv_b=f32(2, w.channels))
         sets.append(s)
     if w.kind == "vim":
         ws_bytes = vs.vim_scan_workspace_bytes(0, w.batch, w.L, 0, w.channels, w.d_state)
@@ -484,6 +492,8 @@ def main():
         ws_bytes = int(vs.lib.vmamba_cross_scan4_bwd_workspace_bytes(w.batch, w.H, w.W, w.channels, w.d_state))
     if args.block:
         ws_bytes = vs.vim_block_workspace_bytes(w.batch, w.L, w.channels, w.d_state)
+        if args.bwd:
+            ws_bytes = vs.vim_block_bwd_workspace_bytes(w.batch, w.L, w.channels, w.d_state)
         blk = block_params(w, w.seed + 3)
         params.update({k: v.to(dev) for k, v in blk.items()})
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
@@ -494,6 +504,11 @@ def main():
 
     def step(i, events=None):
         s = sets[i % nsets]
+        if args.block and args.bwd:
+            vs.vim_block_scan_bwd(s["u"], params["Wx"], params["Wdt"], params["dt_bias"], params["A"], params["D"],
+                                  s["z"], s["dout"], conv_w=params["conv_w"], conv_b=params["conv_b"], workspace=ws,
+                                  out=s["out"])
+            return
         if args.block:
             # u holds x, the block's input; B, C and delta come from the projections
             vs.vim_block_scan(s["u"], params["Wx"], params["Wdt"], params["dt_bias"], params["A"], params["D"],
@@ -552,7 +567,7 @@ def main():
     kernels_per_pair = 3
     pairs = 1 if w.kind == "vim" else 2
     nev = 4 if args.bwd else (5 if args.block else 1 + kernels_per_pair * pairs)
-    whole_call = args.bwd and (w.kind != "vim" or args.conv)
+    whole_call = args.bwd and (w.kind != "vim" or args.conv or args.block)
     if whole_call:
         nev = 2       # the cross-scan's and the front's derivatives have no per-phase events:
                       # the whole call is timed
@@ -562,7 +577,7 @@ def main():
         step(i, events=evs[i])
     torch.cuda.synchronize()
     per_kernel = {}
-    if args.block:
+    if args.block and not args.bwd:
         for a, name in enumerate(["xproj", "pair_carry", "pair_combine", "pair_main"], start=1):
             t = [evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(prof_steps)]
             per_kernel[name] = sum(t) / len(t)
@@ -576,7 +591,14 @@ def main():
             e1.record()
         torch.cuda.synchronize()
         t = [evs[i][0].elapsed_time(evs[i][1]) for i in range(prof_steps)]
-        if args.conv:
+        if args.block:
+            per_kernel["vim_block_scan_bwd"] = sum(t) / len(t)
+            # the projection, the fronts, pair_carry, pair_combine, adj_carry, pair_combine,
+            # bwd_main, four dB/dC reductions, two column sums for the parameters; dl/ds,
+            # two for dWdt, dl/du and dWx partials, two for dWx; the fronts' derivative and
+            # two column sums
+            launches_per_step = 2 + (4 if w.tokens > 32 else 0) + 1 + 4 + 2 + 1 + 2 + 1 + 2 + 1 + 2
+        elif args.conv:
             per_kernel["vim_scan_bidir_conv_bwd"] = sum(t) / len(t)
             # the fronts' forward kernel, pair_carry, pair_combine, adj_carry, pair_combine,
             # bwd_main, two dB/dC reductions, two column sums for the parameters, the
@@ -607,7 +629,8 @@ def main():
     # ---- end to end: pinned host inputs -> device -> scan -> host result ---------
     pinned = {k: host[k].pin_memory() for k in act_keys}
     if args.bwd:
-        res_dev = [sets[0]["out"][k] for k in ("dx" if args.conv else "du", "ddelta", "dz", "dB", "dC")]
+        keys = ("dx", "dz", "dWx") if args.block else ("dx" if args.conv else "du", "ddelta", "dz", "dB", "dC")
+        res_dev = [sets[0]["out"][k] for k in keys]
     else:
         res_dev = [sets[0]["y"]]
     res_host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in res_dev]
@@ -660,7 +683,8 @@ def main():
     nbytes, ops = algorithmic_bwd(w) if args.bwd else algorithmic(w, args.conv)
     main_name = "bwd_main" if args.bwd else "pair_main"
     if whole_call:
-        main_name = "vim_scan_bidir_conv_bwd" if args.conv else "vmamba_cross_scan4_bwd"   # the whole call
+        main_name = ("vim_block_scan_bwd" if args.block else "vim_scan_bidir_conv_bwd" if args.conv
+                     else "vmamba_cross_scan4_bwd")   # the whole call
     main_ms = sum(v for k, v in per_kernel.items() if k.startswith(main_name))
     clocks = clk.summary()
     peak_ops = SMS * FP32_LANES_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e12
@@ -681,7 +705,7 @@ def main():
     }
 
     projection = None
-    if args.block:
+    if args.block and not args.bwd:
         # x_proj: x read once; B and C (bf16), the step input (fp32) and u (bf16, for the
         # scan) written per pathway
         M = w.batch * w.tokens

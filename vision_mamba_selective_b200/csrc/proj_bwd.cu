@@ -54,14 +54,15 @@ __global__ void __launch_bounds__(256) proj_bwd_ds(const float *dd2, const float
     for (int j = lane; j < NO; j += 32) out[j] = j < N ? dB2[bc + j] : j < 2 * N ? dC2[bc + j - N] : acc;
 }
 
-// dl/dWdt partials: tmp[part][k * Di + d] = sum over part's rows m of dd2_k[m, d] s_k[m]
+// dl/dWdt partials: part[p][k * Di + d] = sum over rows m of part p (kWdtRows each) of
+// dd2_k[m, d] s_k[m]; the column kernels then sum the parts in a fixed order
+constexpr int kWdtRows = 64;
 __global__ void __launch_bounds__(256) proj_bwd_dwdt(const float *dd2, const float *s2, float *tmp, int64_t M,
                                                      int Di) {
     const int col = blockIdx.x * blockDim.x + threadIdx.x, part = blockIdx.y;
     if (col >= 2 * Di) return;
     const int k = col / Di, d = col % Di;
-    const int64_t per = (M + kReduceParts - 1) / kReduceParts;
-    const int64_t m0 = part * per, m1 = m0 + per < M ? m0 + per : M;
+    const int64_t m0 = (int64_t)part * kWdtRows, m1 = m0 + kWdtRows < M ? m0 + kWdtRows : M;
     const float *src = dd2 + (size_t)k * M * Di + d, *s = s2 + (size_t)k * M;
     float a0 = 0.0f, a1 = 0.0f;
     int64_t m = m0;
@@ -81,37 +82,64 @@ template <int N>
 __global__ void __launch_bounds__(kPbCh) proj_bwd_du_dwx(const float *dP, const __nv_bfloat16 *Wx, const float *u2,
                                                          float *du2, float *part, int64_t M, int Di) {
     constexpr int NO = 2 * N + 1;
-    __shared__ float sP[kPbRows][NO];
+    constexpr int NQ = (NO + 3) / 4;   // float4 per staged row (the row padded with zeros)
+    __shared__ __align__(16) float4 sP[kPbRows][NQ];
     const int k = blockIdx.z, tile = blockIdx.y, d = blockIdx.x * kPbCh + threadIdx.x;
     const int64_t m0 = (int64_t)tile * kPbRows;
     const int rows = (int)(M - m0 < kPbRows ? M - m0 : kPbRows);
     const float *src = dP + ((size_t)k * M + m0) * NO;
-    for (int i = threadIdx.x; i < rows * NO; i += kPbCh) sP[i / NO][i % NO] = src[i];
+    float *sp = reinterpret_cast<float *>(sP);
+    for (int i = threadIdx.x; i < kPbRows * NQ * 4; i += kPbCh) {
+        const int r = i / (NQ * 4), j = i % (NQ * 4);
+        sp[i] = (r < rows && j < NO) ? src[(size_t)r * NO + j] : 0.0f;
+    }
     __syncthreads();
     if (d >= Di) return;
-    float w[NO], acc[NO];
+    float2 w[2 * NQ], acc[2 * NQ];   // columns (2q, 2q+1), zero past NO
 #pragma unroll
-    for (int j = 0; j < NO; ++j) {
-        w[j] = __bfloat162float(Wx[((size_t)k * Di + d) * NO + j]);
-        acc[j] = 0.0f;
+    for (int q = 0; q < 2 * NQ; ++q) {
+        const int j0 = 2 * q, j1 = 2 * q + 1;
+        const __nv_bfloat16 *wr = Wx + ((size_t)k * Di + d) * NO;
+        w[q] = f2(j0 < NO ? __bfloat162float(wr[j0]) : 0.0f, j1 < NO ? __bfloat162float(wr[j1]) : 0.0f);
+        acc[q] = f2(0.0f, 0.0f);
     }
     const size_t plane = (size_t)M * Di;
     const float *u = u2 + (size_t)k * plane + (size_t)m0 * Di + d;
     float *g = du2 + (size_t)k * plane + (size_t)m0 * Di + d;
-    for (int r = 0; r < rows; ++r) {
-        const float ur = u[(size_t)r * Di];
-        float s = 0.0f;
+    // kPbAhead tokens at a time: their u and dl/du loads are in flight together
+    constexpr int kPbAhead = 8;
+    for (int r0 = 0; r0 < rows; r0 += kPbAhead) {
+        float uv[kPbAhead], gv[kPbAhead];
 #pragma unroll
-        for (int j = 0; j < NO; ++j) {
-            const float p = sP[r][j];
-            s = fmaf(p, w[j], s);
-            acc[j] = fmaf(ur, p, acc[j]);
+        for (int e = 0; e < kPbAhead; ++e) {
+            const bool ok = r0 + e < rows;
+            uv[e] = ok ? u[(size_t)(r0 + e) * Di] : 0.0f;
+            gv[e] = ok ? g[(size_t)(r0 + e) * Di] : 0.0f;
         }
-        g[(size_t)r * Di] += s;
+#pragma unroll
+        for (int e = 0; e < kPbAhead; ++e) {
+            const int r = r0 + e;
+            if (r >= rows) break;
+            const float2 ur2 = f2(uv[e], uv[e]);
+            float2 s = f2(0.0f, 0.0f);
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                const float4 p = sP[r][q];
+                const float2 pa = f2(p.x, p.y), pb = f2(p.z, p.w);
+                s = fma2(pa, w[2 * q], s);
+                s = fma2(pb, w[2 * q + 1], s);
+                acc[2 * q] = fma2(ur2, pa, acc[2 * q]);
+                acc[2 * q + 1] = fma2(ur2, pb, acc[2 * q + 1]);
+            }
+            g[(size_t)r * Di] = gv[e] + (s.x + s.y);
+        }
     }
     float *o = part + (size_t)tile * 2 * Di * NO + ((size_t)k * Di + d) * NO;
 #pragma unroll
-    for (int j = 0; j < NO; ++j) o[j] = acc[j];
+    for (int q = 0; q < 2 * NQ; ++q) {
+        if (2 * q < NO) o[2 * q] = acc[q].x;
+        if (2 * q + 1 < NO) o[2 * q + 1] = acc[q].y;
+    }
 }
 
 // dx = dl/du_f + dl/du_b (the block without convolution fronts)
@@ -144,7 +172,7 @@ BlockBwdPlan block_bwd_plan(int batch, int L, int Di, int N) {
     c.off_dB = take(2 * M * N * 4);
     c.off_dC = take(2 * M * N * 4);
     c.off_dP = take(2 * M * NO * 4);
-    c.off_wtmp = take((size_t)kReduceParts * 2 * Di * 4);
+    c.off_wtmp = take(((M + 63) / 64 + kReduceParts) * 2 * Di * 4);   // the parts, then the column pass
     c.off_xpart = take((size_t)c.tiles * 2 * Di * NO * 4);
     c.off_xtmp = take((size_t)kReduceParts * 2 * Di * NO * 4);
     c.off_part = take((size_t)batch * c.runs * 8 * Di * 4);
@@ -233,9 +261,13 @@ vim_status block_bwd_n(const void *x, const float *conv_w, const float *conv_b, 
     proj_bwd_ds<<<(unsigned)((2 * M * 32 + 255) / 256), 256, 0, stream>>>(dd2, Wdt, dB2, dC2, dP, M, Di, N);
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     float *wtmp = reinterpret_cast<float *>(ws + cp.off_wtmp);
-    proj_bwd_dwdt<<<dim3((2 * Di + 255) / 256, kReduceParts), 256, 0, stream>>>(dd2, s2, wtmp, M, Di);
+    const int wparts = (int)((M + kWdtRows - 1) / kWdtRows);
+    float *wtmp2 = wtmp + (size_t)wparts * 2 * Di;
+    proj_bwd_dwdt<<<dim3((2 * Di + 255) / 256, wparts), 256, 0, stream>>>(dd2, s2, wtmp, M, Di);
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
-    bwd_reduce_cols2<<<(2 * Di + 255) / 256, 256, 0, stream>>>(wtmp, dWdt, nullptr, nullptr, 2 * Di, 0);
+    bwd_reduce_cols1<<<dim3((2 * Di + 255) / 256, kReduceParts), 256, 0, stream>>>(wtmp, wtmp2, wparts, 2 * Di);
+    if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+    bwd_reduce_cols2<<<(2 * Di + 255) / 256, 256, 0, stream>>>(wtmp2, dWdt, nullptr, nullptr, 2 * Di, 0);
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     float *xpart = reinterpret_cast<float *>(ws + cp.off_xpart), *xtmp = reinterpret_cast<float *>(ws + cp.off_xtmp);
     proj_bwd_du_dwx<N><<<dim3((Di + kPbCh - 1) / kPbCh, cp.tiles, 2), kPbCh, 0, stream>>>(
