@@ -374,7 +374,8 @@ CONV_CASES = [
     (1, 1, 16, 16, torch.float32, False, False, True, False),
     (1, 5, 16, 4, torch.float32, True, False, True, False),
     (2, 33, 64, 16, torch.float32, True, False, True, False),     # 2 chunks, the last 1 token
-    (1, 100, 40, 8, torch.float32, False, True, False, False),    # 2 runs of the front's walk
+    (1, 100, 40, 8, torch.float32, False, True, False, False),    # 2 front tiles, a partial channel tile
+    (2, 128, 48, 16, torch.float32, False, False, True, False),   # 2 whole front tiles, half a channel tile
     (2, 197, 64, 16, torch.bfloat16, False, False, True, False),
     (1, 300, 72, 16, torch.bfloat16, True, False, True, False),
     (1, 1000, 64, 16, torch.float32, False, False, True, False),

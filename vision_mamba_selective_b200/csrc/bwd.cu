@@ -176,17 +176,11 @@ vim_status vim_scan_bidir_conv_bwd_ex(const void *x, const float *conv_w, const 
     const int vec = aligned_to(x, dt == VIM_F32 ? 16 : 8) && aligned_to(dx, dt == VIM_F32 ? 16 : 8) ? 1 : 0;
 
     // both pathways' smoothed inputs
-    {
-        const int64_t items = act / 4;
-        const unsigned blocks = (unsigned)std::min<int64_t>((items + 255) / 256, 148 * 16);
-        if (dt == VIM_F32)
-            conv_front_fwd<float><<<blocks, 256, 0, stream>>>(static_cast<const float *>(x), conv_w, conv_b, u2,
-                                                               batch, L, d_inner, vec);
-        else
-            conv_front_fwd<__nv_bfloat16><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(x), conv_w,
-                                                                       conv_b, u2, batch, L, d_inner, vec);
-        if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
-    }
+    st = dt == VIM_F32 ? launch_front_fwd<float>(static_cast<const float *>(x), conv_w, conv_b, u2, batch, L,
+                                                 d_inner, vec, stream)
+                       : launch_front_fwd<__nv_bfloat16>(static_cast<const __nv_bfloat16 *>(x), conv_w, conv_b, u2,
+                                                         batch, L, d_inner, vec, stream);
+    if (st != VIM_OK) return st;
 
     BwdArgs a;
     std::memset(&a, 0, sizeof(a));

@@ -57,6 +57,9 @@ constexpr int kReduceParts = 32;              // row groups of the first paramet
 #ifndef VIMSCAN_BWD_MIN_WARPS
 #define VIMSCAN_BWD_MIN_WARPS 16                 // resident warps per SM the register budget targets
 #endif
+#ifndef VIMSCAN_BWD_CHAIN
+#define VIMSCAN_BWD_CHAIN 1                      // structured A: decays as powers of exp(Delta A_0)
+#endif                                           // (bit 0: exact hold, bit 1: first order)
 
 struct BwdArgs {
     const void *u, *delta, *z, *dout;   // [batch, L, Di]
@@ -487,13 +490,12 @@ __device__ __forceinline__ float hold_take(const BwdThread<N> &th, const float (
 }
 
 template <int N, bool DA, bool SDA>
-__device__ __forceinline__ void hold_states(const BwdThread<N> &th, float dl, const float2 (&ab)[BwdShape<N>::NP],
-                                            const HoldSeg<N, SDA> &hs, int m,
+__device__ __forceinline__ void hold_states(const BwdThread<N> &th, float dl, float q,
+                                            const float2 (&ab)[BwdShape<N>::NP], const HoldSeg<N, SDA> &hs, int m,
                                             float2 (&gn)[BwdShape<N>::NP], float2 (&dg)[BwdShape<N>::NP]) {
     using SH = BwdShape<N>;
     constexpr int NP = SH::NP, NT = SH::NT;
     static_assert(SDA || !DA, "the A-derivative needs the segment's z chi(z)");
-    const float q = hold_take<N>(th, hs.q, m);
     const float e0 = hold_take<N>(th, hs.e0, m);
     float zc = 0.0f;
     if constexpr (DA) zc = hold_take<N>(th, hs.zc, m);
@@ -536,6 +538,50 @@ __device__ __forceinline__ void hold_states(const BwdThread<N> &th, float dl, co
         const float2 w = th.w1[k];
         gn[k] = mul2(f2(ev[2 * k], ev[2 * k + 1]), w);
         if constexpr (DA) dg[k] = mul2(mul2(f2(fv[2 * k], fv[2 * k + 1]), w), w);
+    }
+}
+
+// q = exp(Delta A_0) of a segment's tokens for the first-order structured-A decays,
+// formed as hold_seg forms it: token m by lane m mod Q of the channel, taken by the
+// others with hold_take.
+template <int N>
+struct QSeg {
+    float q[HoldSeg<N, false>::K];
+};
+template <int N>
+__device__ __forceinline__ QSeg<N> q_seg(const BwdSmem<N> &sm, const BwdThread<N> &th, int DIR, int sg) {
+    using SH = BwdShape<N>;
+    QSeg<N> s;
+#pragma unroll
+    for (int k = 0; k < HoldSeg<N, false>::K; ++k) {
+        const int i = sg * kBwdSeg + th.q + k * SH::Q, r = DIR ? SH::TC - 1 - i : i;
+        const float dl = reinterpret_cast<const float *>(sm.dsg)[2 * ((DIR * SH::TC + r) * SH::CH + th.cl)];
+        s.q[k] = ex2(dl * th.a0 * kLog2e);
+    }
+    return s;
+}
+
+// Abar_n = exp(Delta A_n) of the thread's states at one token.  With structured A
+// (A_n = (n + 1) A_0 for the channel, CHAIN) the first state's exp(Delta A_j0) and then
+// powers of q = exp(Delta A_0): one exp2 and one multiply per state pair instead of one
+// exp2 per state.  Otherwise one exp2 per state.
+template <int N, bool CHAIN>
+__device__ __forceinline__ void state_decays(const BwdThread<N> &th, float dl, float q,
+                                             float2 (&ab)[BwdShape<N>::NP]) {
+    constexpr int NP = BwdShape<N>::NP;
+    if constexpr (CHAIN) {
+        const float b0 = ex2(dl * th.A2[0].x);
+        ab[0] = f2(b0, b0 * q);
+        const float q2 = q * q;
+#pragma unroll
+        for (int k = 1; k < NP; ++k) ab[k] = mul2(ab[k - 1], f2(q2, q2));
+    } else {
+        const float2 dl2 = f2(dl, dl);
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+            const float2 e = mul2(dl2, th.A2[k]);
+            ab[k] = f2(ex2(e.x), ex2(e.y));
+        }
     }
 }
 
@@ -584,7 +630,8 @@ __device__ __forceinline__ void channel_sum(const BwdThread<N> &th, float *red_w
 }
 
 // forward sweep of direction DIR: checkpoints, y^DIR (ungated) and the dC terms
-// (ZOH: the exact hold's Bbar in the state update; FAST: its gains from hold_states)
+// (ZOH: the exact hold's Bbar in the state update; FAST: structured A, the decays from
+// state_decays' power chain and the exact hold's gains from hold_states)
 // u of token row r for direction DIR: the shared u, or with U2 the backward
 // direction's own (staged in the dz-factor area, which U2 does not use)
 template <int N, bool U2>
@@ -600,6 +647,7 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
     const int DIR = DIRT < 0 ? th.dir : DIRT;   // DIRT < 0: the direction at run time
     float *red_w = sm.red + (DIR * SH::WPD + th.wid) * TC * N;
     constexpr bool fast = ZOH && FAST;
+    constexpr bool chain = FAST && ((VIMSCAN_BWD_CHAIN >> (ZOH ? 0 : 1)) & 1);
     float2 h[NP];
 #pragma unroll
     for (int k = 0; k < NP; ++k) h[k] = f2(0.f, 0.f);
@@ -608,7 +656,9 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
     for (int sg = 0; sg < kBwdNSeg; ++sg) {
         store_ck<N>(sm, th.tid, sg, h);
         [[maybe_unused]] HoldSeg<N, false> hs;
+        [[maybe_unused]] QSeg<N> qs;
         if constexpr (fast) hs = hold_seg<N, false>(sm, th, DIR, sg);
+        else if constexpr (chain) qs = q_seg<N>(sm, th, DIR, sg);
         float yv[kBwdSeg], vc[SH::BATCH ? kBwdSeg * SH::NT : 1];   // batched: y partials, dC terms
 #pragma unroll
         for (int m = 0; m < kBwdSeg; ++m) {
@@ -623,15 +673,14 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
             const float2 dl2 = f2(dl, dl), du2 = f2(du, du), dy2 = f2(tk.y, tk.y);
             float2 yp = f2(th.q == 0 ? th.Dk * tk.x : 0.0f, 0.0f);
             float2 abk[NP], gnk[NP];
-#pragma unroll
-            for (int k = 0; k < NP; ++k) {
-                const float2 e = mul2(dl2, th.A2[k]);
-                abk[k] = f2(ex2(e.x), ex2(e.y));
-            }
+            float qm = 0.0f;
+            if constexpr (fast) qm = hold_take<N>(th, hs.q, m);
+            else if constexpr (chain) qm = hold_take<N>(th, qs.q, m);
+            state_decays<N, chain>(th, dl, qm, abk);
             if constexpr (ZOH) {
                 if constexpr (fast) {
                     float2 unused[NP];
-                    hold_states<N, false>(th, dl, abk, hs, m, gnk, unused);
+                    hold_states<N, false>(th, dl, qm, abk, hs, m, gnk, unused);
                 } else {
 #pragma unroll
                     for (int k = 0; k < NP; ++k) gnk[k] = hold_gain2(dl, mul2(dl2, th.Araw[k]), abk[k], th.invA[k]);
@@ -685,6 +734,7 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
     constexpr int kDdLane = Q > 1 ? 1 : 0;
     float *red_w = sm.red + (DIR * SH::WPD + th.wid) * TC * N;
     constexpr bool fast = ZOH && FAST;
+    constexpr bool chain = FAST && ((VIMSCAN_BWD_CHAIN >> (ZOH ? 0 : 1)) & 1);
     float2 g[NP], dA[NP];
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
@@ -698,8 +748,11 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
         float2 h0[NP];
         load_ck<N>(sm, th.tid, sg, h0);
         [[maybe_unused]] HoldSeg<N, true> hs;
+        [[maybe_unused]] QSeg<N> qs;
         if constexpr (fast) hs = hold_seg<N, true>(sm, th, DIR, sg);
+        else if constexpr (chain) qs = q_seg<N>(sm, th, DIR, sg);
         float2 hh[kBwdSeg][NP], aa[kBwdSeg][NP];
+        [[maybe_unused]] float qv[kBwdSeg];   // the exact hold's q of each token, for its second use
         // batched: [slot][du, d delta_raw] partials and [slot][state] dB terms, slot = 3 - m
         float xq[SH::BATCH ? 2 * kBwdSeg : 1], vb[SH::BATCH ? kBwdSeg * SH::NT : 1];
 #pragma unroll
@@ -711,16 +764,16 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
             float2 Bp[NP];
             load_row<NP>(sm.B + (DIR * TC + r) * N + th.j0, Bp);
             const float2 dl2 = f2(dl, dl), du2 = f2(du, du);
-#pragma unroll
-            for (int k = 0; k < NP; ++k) {
-                const float2 e = mul2(dl2, th.A2[k]);
-                aa[m][k] = f2(ex2(e.x), ex2(e.y));
-            }
+            float qm = 0.0f;
+            if constexpr (fast) qm = hold_take<N>(th, hs.q, m);
+            else if constexpr (chain) qm = hold_take<N>(th, qs.q, m);
+            if constexpr (fast) qv[m] = qm;
+            state_decays<N, chain>(th, dl, qm, aa[m]);
             float2 gnk[NP];
             if constexpr (ZOH) {
                 if constexpr (fast) {
                     float2 unused[NP];
-                    hold_states<N, false>(th, dl, aa[m], hs, m, gnk, unused);
+                    hold_states<N, false>(th, dl, qm, aa[m], hs, m, gnk, unused);
                 } else {
 #pragma unroll
                     for (int k = 0; k < NP; ++k) gnk[k] = hold_gain2(dl, mul2(dl2, th.Araw[k]), aa[m][k], th.invA[k]);
@@ -752,7 +805,7 @@ __device__ __forceinline__ void bwd_adjoint(const BwdArgs &p, const BwdSmem<N> &
             float2 gnk[NP], dgk[NP];
             if constexpr (ZOH) {
                 if constexpr (fast) {
-                    hold_states<N, true>(th, dl, aa[m], hs, m, gnk, dgk);
+                    hold_states<N, true>(th, dl, qv[m], aa[m], hs, m, gnk, dgk);
                 } else {
 #pragma unroll
                     for (int k = 0; k < NP; ++k) {
@@ -1091,11 +1144,13 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     // carries are read after the wait
     if (p.G > 1) cudaGridDependencySynchronize();
 
-    // the exact hold's path is chosen once per warp: its structured-A code and the
-    // general code are separate copies of the sweeps, with no branch between them per
-    // token, and a warp fetches only the copy it runs
-    const bool fast = ZOH && __all_sync(0xffffffffu, th.structured);
-    if (fast) bwd_sweep<N, ZOH, ZOH, false, U2>(p, sm, th);
+    // the path is chosen once per warp: the structured-A code (decays as powers of
+    // exp(Delta A_0), and the exact hold's gains from hold_states) and the general code
+    // are separate copies of the sweeps, with no branch between them per token, and a
+    // warp fetches only the copy it runs
+    constexpr bool kTwo = ZOH || ((VIMSCAN_BWD_CHAIN >> 1) & 1);   // a structured-A copy exists
+    const bool fast = kTwo && __all_sync(0xffffffffu, th.structured);
+    if (fast) bwd_sweep<N, ZOH, kTwo, false, U2>(p, sm, th);
     else bwd_sweep<N, ZOH, false, false, U2>(p, sm, th);
     __syncthreads();
     // dz = dout silu'(z) (sum of the directions' y), and the CTA's dC terms; the
@@ -1134,7 +1189,7 @@ __global__ void __launch_bounds__(BwdShape<N>::kThr, BwdShape<N>::kMinBlocks) bw
     store_bc_part<N>(p, sm.red, p.dC_part, b, t0, tc, blk);
     __syncthreads();
 
-    if (fast) bwd_sweep<N, ZOH, ZOH, true, U2>(p, sm, th);
+    if (fast) bwd_sweep<N, ZOH, kTwo, true, U2>(p, sm, th);
     else bwd_sweep<N, ZOH, false, true, U2>(p, sm, th);
     __syncthreads();
     for (int li = threadIdx.x; li < TC * (CH / kG); li += SH::kThr) {
@@ -1190,31 +1245,68 @@ __device__ __forceinline__ float conv_pre(const float *w, float cb, float xm, fl
     return K == 0 ? fmaf(w[0], xm, fmaf(w[1], x0, fmaf(w[2], xp, cb))) : fmaf(w[0], xp, fmaf(w[1], x0, fmaf(w[2], xm, cb)));
 }
 
-// u2[k] = u_k for both pathways, [2][batch, L, Di] fp32; one thread per (b, t, four
-// channels)
+#ifndef VIMSCAN_FRONT_ROWS
+#define VIMSCAN_FRONT_ROWS 64
+#endif
+// The front kernels work on tiles of kFrontRows tokens x kFrontCh channels of one batch
+// item, one CTA of 256 threads each (grid x: batch item and run of tokens, grid y:
+// channel tile).  The tile's x rows, with a halo, are staged in shared memory by
+// coalesced vector loads; then every thread owns one channel and a set of rows.
+constexpr int kFrontRows = VIMSCAN_FRONT_ROWS;   // tokens per tile (one row of partial sums each)
+constexpr int kFrontCh = 32;                     // channels per tile
+constexpr int kFrontThr = 256;
+constexpr int kFrontGroups = kFrontThr / kFrontCh;   // row groups of a tile
+static_assert(kFrontRows % kFrontGroups == 0, "a tile's rows split evenly over its row groups");
+
+// x rows tfirst .. tfirst + nrows - 1 of channels c0 .. c0 + kFrontCh - 1 of batch item b
+// into xs[nrows][kFrontCh] (fp32; 0 outside the sequence and past Di, a multiple of 4)
 template <typename T>
-__global__ void __launch_bounds__(256) conv_front_fwd(const T *x, const float *conv_w, const float *conv_b,
-                                                      float *u2, int batch, int L, int Di, int vec) {
-    const int q4 = Di / 4;
-    const int64_t items = (int64_t)batch * L * q4, plane = (int64_t)batch * L * Di;
-    for (int64_t it = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; it < items;
-         it += (int64_t)gridDim.x * blockDim.x) {
-        const int d = (int)(it % q4) * 4;
-        const int64_t bt = it / q4;
-        const int t = (int)(bt % L);
-        const size_t i = (size_t)bt * Di + d;
-        float xm[4] = {0.f, 0.f, 0.f, 0.f}, x0[4], xp[4] = {0.f, 0.f, 0.f, 0.f};
-        load4<T>(x, i, vec != 0, x0);
-        if (t > 0) load4<T>(x, i - Di, vec != 0, xm);
-        if (t + 1 < L) load4<T>(x, i + Di, vec != 0, xp);
-        float uf[4], ub[4];
+__device__ __forceinline__ void front_stage(const T *x, float *xs, int nrows, int tfirst, int c0, int b, int L,
+                                            int Di, int vec) {
+    constexpr int V = kFrontCh / 4;
+    for (int li = threadIdx.x; li < nrows * V; li += kFrontThr) {
+        const int r = li / V, cg = (li % V) * 4, t = tfirst + r, ch = c0 + cg;
+        float v[4] = {0.f, 0.f, 0.f, 0.f};
+        if (t >= 0 && t < L && ch < Di) load4<T>(x, ((size_t)b * L + t) * Di + ch, vec != 0, v);
+        *reinterpret_cast<float4 *>(xs + r * kFrontCh + cg) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+}
+
+// u2[k] = u_k for both pathways, [2][batch, L, Di] fp32.  Each thread walks kFrontRows /
+// kFrontGroups consecutive rows of its channel with x[t-1], x[t], x[t+1] from the staged
+// rows; a warp stores 32 consecutive channels of a row.
+template <typename T>
+__global__ void __launch_bounds__(kFrontThr) conv_front_fwd(const T *x, const float *conv_w, const float *conv_b,
+                                                            float *u2, int batch, int L, int Di, int vec) {
+    constexpr int TR = kFrontRows, CC = kFrontCh, RPT = TR / kFrontGroups;
+    __shared__ __align__(16) float xs[(TR + 2) * CC];   // rows t0 - 1 .. t0 + TR
+    const int runs = (L + TR - 1) / TR;
+    const int b = blockIdx.x / runs, t0 = (blockIdx.x % runs) * TR, c0 = blockIdx.y * CC;
+    front_stage<T>(x, xs, TR + 2, t0 - 1, c0, b, L, Di, vec);
+    __syncthreads();
+    const int c = threadIdx.x % CC, g = threadIdx.x / CC, d = c0 + c;
+    if (d >= Di) return;   // no barrier follows
+    float wf[3], wb[3];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            uf[e] = silu(conv_pre<0>(conv_w + (size_t)(d + e) * 3, conv_b[d + e], xm[e], x0[e], xp[e]));
-            ub[e] = silu(conv_pre<1>(conv_w + (size_t)(Di + d + e) * 3, conv_b[Di + d + e], xm[e], x0[e], xp[e]));
+    for (int j = 0; j < 3; ++j) {
+        wf[j] = conv_w[(size_t)d * 3 + j];
+        wb[j] = conv_w[((size_t)Di + d) * 3 + j];
+    }
+    const float bf = conv_b[d], bb = conv_b[Di + d];
+    const int64_t plane = (int64_t)batch * L * Di;
+    const int rb = g * RPT;   // first row of the thread; xs row s holds token t0 - 1 + s
+    float xm = xs[rb * CC + c], x0 = xs[(rb + 1) * CC + c];
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+        const int t = t0 + rb + k;
+        const float xp = xs[(rb + k + 2) * CC + c];
+        if (t < L) {
+            const size_t i = ((size_t)b * L + t) * Di + d;
+            u2[i] = silu(conv_pre<0>(wf, bf, xm, x0, xp));
+            u2[plane + i] = silu(conv_pre<1>(wb, bb, xm, x0, xp));
         }
-        *reinterpret_cast<float4 *>(u2 + i) = make_float4(uf[0], uf[1], uf[2], uf[3]);
-        *reinterpret_cast<float4 *>(u2 + plane + i) = make_float4(ub[0], ub[1], ub[2], ub[3]);
+        xm = x0;
+        x0 = xp;
     }
 }
 
@@ -1222,107 +1314,92 @@ __global__ void __launch_bounds__(256) conv_front_fwd(const T *x, const float *c
 //   dl/dx[t]  = w_f[0] dpre_f[t+1] + w_f[1] dpre_f[t] + w_f[2] dpre_f[t-1]
 //             + w_b[0] dpre_b[t-1] + w_b[1] dpre_b[t] + w_b[2] dpre_b[t+1],
 //   dl/dw_k[j] = sum_t dpre_k[t] x[s_kj(t)],   dl/dcb_k = sum_t dpre_k[t].
-// One thread per (b, run of kFrontRows tokens, four channels) walks its tokens with a
-// window of x and dpre one token either side; it writes dx and one row of partial sums
-// part[b * runs + run][8 Di] = [dw: (k * Di + d) * 3 + j | dcb: 6 Di + k * Di + d].
-#ifndef VIMSCAN_FRONT_ROWS
-#define VIMSCAN_FRONT_ROWS 64
-#endif
-constexpr int kFrontRows = VIMSCAN_FRONT_ROWS;   // tokens one thread of conv_front_bwd walks
+// Per tile: x rows with two halo rows each side staged; dpre of both pathways for the
+// tile's rows and one either side, into shared memory (each thread a channel and every
+// kFrontGroups-th row, so the du2 loads of a thread are independent); then per thread a
+// channel and kFrontRows / kFrontGroups consecutive rows: dx and the eight tap and bias
+// sums, summed over the row groups in order into the tile's slice of one row of partial
+// sums part[b * runs + run][8 Di] = [dw: (k * Di + d) * 3 + j | dcb: 6 Di + k * Di + d].
 template <typename T>
-__global__ void __launch_bounds__(256) conv_front_bwd(const T *x, const float *conv_w, const float *conv_b,
-                                                      const float *du2, T *dx, float *part, int batch, int L, int Di,
-                                                      int vec) {
-    const int q4 = Di / 4, runs = (L + kFrontRows - 1) / kFrontRows;
-    const int64_t items = (int64_t)batch * runs * q4, plane = (int64_t)batch * L * Di;
-    const int64_t it = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (it >= items) return;
-    const int d = (int)(it % q4) * 4;
-    const int run = (int)((it / q4) % runs), b = (int)(it / ((int64_t)q4 * runs));
-    const int r0 = run * kFrontRows, r1 = min(L, r0 + kFrontRows);
-    const size_t base = (size_t)b * L * Di + d;   // element of (b, t = 0, d)
-    float w[2][4][3], cb[2][4];
+__global__ void __launch_bounds__(kFrontThr) conv_front_bwd(const T *x, const float *conv_w, const float *conv_b,
+                                                            const float *du2, T *dx, float *part, int batch, int L,
+                                                            int Di, int vec) {
+    constexpr int TR = kFrontRows, CC = kFrontCh, G = kFrontGroups, RPT = TR / G;
+    static_assert(G == 8, "one row group per partial sum in the final pass");
+    __shared__ __align__(16) float xs[(TR + 4) * CC];      // x rows t0 - 2 .. t0 + TR + 1
+    __shared__ __align__(16) float dp[2 * (TR + 2) * CC];  // dpre_k rows t0 - 1 .. t0 + TR
+    const int runs = (L + TR - 1) / TR;
+    const int b = blockIdx.x / runs, run = blockIdx.x % runs, t0 = run * TR, c0 = blockIdx.y * CC;
+    front_stage<T>(x, xs, TR + 4, t0 - 2, c0, b, L, Di, vec);
+    __syncthreads();
+    const int c = threadIdx.x % CC, g = threadIdx.x / CC, d = c0 + c;
+    const bool dv = d < Di;
+    float w[2][3], cb[2];
 #pragma unroll
-    for (int k = 0; k < 2; ++k)
+    for (int k = 0; k < 2; ++k) {
+        cb[k] = dv ? conv_b[k * Di + d] : 0.0f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            cb[k][e] = conv_b[k * Di + d + e];
-#pragma unroll
-            for (int j = 0; j < 3; ++j) w[k][e][j] = conv_w[((size_t)k * Di + d + e) * 3 + j];
-        }
-    auto xrow = [&](int t, float (&v)[4]) {
-        if (t >= 0 && t < L) load4<T>(x, base + (size_t)t * Di, vec != 0, v);
-        else v[0] = v[1] = v[2] = v[3] = 0.0f;
-    };
-    // dpre of both pathways at token t from x[t-1], x[t], x[t+1]; zero outside the sequence
-    auto dpre_at = [&](int t, const float (&xm)[4], const float (&x0)[4], const float (&xp)[4], float (&o)[2][4]) {
-        if (t < 0 || t >= L) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) o[0][e] = o[1][e] = 0.0f;
-            return;
-        }
-        const float4 gf = *reinterpret_cast<const float4 *>(du2 + base + (size_t)t * Di);
-        const float4 gb = *reinterpret_cast<const float4 *>(du2 + plane + base + (size_t)t * Di);
-        const float df[4] = {gf.x, gf.y, gf.z, gf.w}, db[4] = {gb.x, gb.y, gb.z, gb.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            o[0][e] = df[e] * silu_grad(conv_pre<0>(w[0][e], cb[0][e], xm[e], x0[e], xp[e]));
-            o[1][e] = db[e] * silu_grad(conv_pre<1>(w[1][e], cb[1][e], xm[e], x0[e], xp[e]));
-        }
-    };
-    float xa[4], xb[4], xc[4], xd[4];   // x[t-1], x[t], x[t+1], x[t+2]
-    float pm[2][4], p0[2][4], pp[2][4];   // dpre at t-1, t, t+1
-    {
-        float xz[4];
-        xrow(r0 - 2, xz);
-        xrow(r0 - 1, xa);
-        xrow(r0, xb);
-        xrow(r0 + 1, xc);
-        dpre_at(r0 - 1, xz, xa, xb, pm);
-        dpre_at(r0, xa, xb, xc, p0);
+        for (int j = 0; j < 3; ++j) w[k][j] = dv ? conv_w[((size_t)k * Di + d) * 3 + j] : 0.0f;
     }
-    float dw[2][4][3], dcb[2][4];
+    const int64_t plane = (int64_t)batch * L * Di;
+    // dpre row r <-> token t0 - 1 + r, whose x[t-1], x[t], x[t+1] are xs rows r, r+1, r+2
 #pragma unroll
-    for (int k = 0; k < 2; ++k)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            dcb[k][e] = 0.0f;
-            dw[k][e][0] = dw[k][e][1] = dw[k][e][2] = 0.0f;
+    for (int k = 0; k < (TR + 2 + G - 1) / G; ++k) {
+        const int r = g + k * G, t = t0 - 1 + r;
+        if (r >= TR + 2) break;
+        float pf = 0.0f, pb = 0.0f;
+        if (dv && t >= 0 && t < L) {
+            const size_t i = ((size_t)b * L + t) * Di + d;
+            const float xm = xs[r * CC + c], x0 = xs[(r + 1) * CC + c], xp = xs[(r + 2) * CC + c];
+            pf = du2[i] * silu_grad(conv_pre<0>(w[0], cb[0], xm, x0, xp));
+            pb = du2[plane + i] * silu_grad(conv_pre<1>(w[1], cb[1], xm, x0, xp));
         }
-    for (int t = r0; t < r1; ++t) {
-        xrow(t + 2, xd);
-        dpre_at(t + 1, xb, xc, xd, pp);
-        float g[4];
+        dp[r * CC + c] = pf;
+        dp[(TR + 2 + r) * CC + c] = pb;
+    }
+    __syncthreads();
+    const float *df = dp, *db = dp + (TR + 2) * CC;
+    float sum[8];   // dw_f[0..2], dw_b[0..2], dcb_f, dcb_b
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            g[e] = w[0][e][0] * pp[0][e] + w[0][e][1] * p0[0][e] + w[0][e][2] * pm[0][e] +
-                   w[1][e][0] * pm[1][e] + w[1][e][1] * p0[1][e] + w[1][e][2] * pp[1][e];
-            dcb[0][e] += p0[0][e];
-            dcb[1][e] += p0[1][e];
-            dw[0][e][0] = fmaf(p0[0][e], xa[e], dw[0][e][0]);   // forward taps: x[t-1], x[t], x[t+1]
-            dw[0][e][1] = fmaf(p0[0][e], xb[e], dw[0][e][1]);
-            dw[0][e][2] = fmaf(p0[0][e], xc[e], dw[0][e][2]);
-            dw[1][e][0] = fmaf(p0[1][e], xc[e], dw[1][e][0]);   // backward taps: x[t+1], x[t], x[t-1]
-            dw[1][e][1] = fmaf(p0[1][e], xb[e], dw[1][e][1]);
-            dw[1][e][2] = fmaf(p0[1][e], xa[e], dw[1][e][2]);
-        }
-        store4<T>(dx, base + (size_t)t * Di, vec != 0, g);
+    for (int e = 0; e < 8; ++e) sum[e] = 0.0f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            xa[e] = xb[e]; xb[e] = xc[e]; xc[e] = xd[e];
-            pm[0][e] = p0[0][e]; pm[1][e] = p0[1][e];
-            p0[0][e] = pp[0][e]; p0[1][e] = pp[1][e];
+    for (int k = 0; k < RPT; ++k) {
+        const int r = g * RPT + k, t = t0 + r;   // dpre rows r, r+1, r+2 = t-1, t, t+1; xs rows r+1..r+3
+        if (dv && t < L) {
+            const float fm = df[r * CC + c], f0 = df[(r + 1) * CC + c], fp = df[(r + 2) * CC + c];
+            const float bm = db[r * CC + c], b0 = db[(r + 1) * CC + c], bp = db[(r + 2) * CC + c];
+            float gx = w[0][0] * fp;
+            gx = fmaf(w[0][1], f0, gx);
+            gx = fmaf(w[0][2], fm, gx);
+            gx = fmaf(w[1][0], bm, gx);
+            gx = fmaf(w[1][1], b0, gx);
+            gx = fmaf(w[1][2], bp, gx);
+            dx[((size_t)b * L + t) * Di + d] = from_f32<T>(gx);
+            const float xa = xs[(r + 1) * CC + c], xb = xs[(r + 2) * CC + c], xc = xs[(r + 3) * CC + c];
+            sum[0] = fmaf(f0, xa, sum[0]);   // forward taps: x[t-1], x[t], x[t+1]
+            sum[1] = fmaf(f0, xb, sum[1]);
+            sum[2] = fmaf(f0, xc, sum[2]);
+            sum[3] = fmaf(b0, xc, sum[3]);   // backward taps: x[t+1], x[t], x[t-1]
+            sum[4] = fmaf(b0, xb, sum[4]);
+            sum[5] = fmaf(b0, xa, sum[5]);
+            sum[6] += f0;
+            sum[7] += b0;
         }
     }
-    float *row = part + ((size_t)b * runs + run) * (8 * (size_t)Di);
+    __syncthreads();   // dp is reused for the row groups' sums
+    float *red = dp;   // [8 sums][G][CC]
 #pragma unroll
-    for (int k = 0; k < 2; ++k)
+    for (int e = 0; e < 8; ++e) red[(e * G + g) * CC + c] = sum[e];
+    __syncthreads();
+    if (dv) {
+        const int e = g;   // this thread sums partial e of its channel over the row groups
+        float acc = 0.0f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-#pragma unroll
-            for (int j = 0; j < 3; ++j) row[((size_t)k * Di + d + e) * 3 + j] = dw[k][e][j];
-            row[6 * (size_t)Di + k * Di + d + e] = dcb[k][e];
-        }
+        for (int q = 0; q < G; ++q) acc += red[(e * G + q) * CC + c];
+        float *row = part + ((size_t)b * runs + run) * (8 * (size_t)Di);
+        if (e < 6) row[((size_t)(e / 3) * Di + d) * 3 + e % 3] = acc;
+        else row[6 * (size_t)Di + (size_t)(e - 6) * Di + d] = acc;
+    }
 }
 
 // dB / dC: sum of the per-CTA (or per-cluster) partials, [batch][L][ncol][N] -> [batch][L][N]

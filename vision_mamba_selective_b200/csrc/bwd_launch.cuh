@@ -211,13 +211,26 @@ ConvBwdPlan conv_bwd_plan(int batch, int L, int Di, int N, vim_dtype dt, int sep
     return c;
 }
 
+// grid of the front kernels: (batch item, run of kFrontRows tokens) x channel tiles
+inline dim3 front_grid(int batch, int L, int Di) {
+    return dim3((unsigned)((int64_t)batch * ((L + kFrontRows - 1) / kFrontRows)),
+                (unsigned)((Di + kFrontCh - 1) / kFrontCh));
+}
+
+// both pathways' smoothed inputs u_k = silu(conv_k(x)) into u2 [2][batch, L, Di] fp32
+template <typename T>
+vim_status launch_front_fwd(const T *x, const float *conv_w, const float *conv_b, float *u2, int batch, int L, int Di,
+                            int vec, cudaStream_t stream) {
+    conv_front_fwd<T><<<front_grid(batch, L, Di), kFrontThr, 0, stream>>>(x, conv_w, conv_b, u2, batch, L, Di, vec);
+    return cudaGetLastError() == cudaSuccess ? VIM_OK : VIM_ERR_CUDA;
+}
+
 template <typename T>
 vim_status launch_fronts_bwd(const T *x, const float *conv_w, const float *conv_b, const float *du2, T *dx,
                              float *part, float *ptmp, float *dconv_w, float *dconv_b, int batch, int L, int Di,
                              int runs, int vec, cudaStream_t stream) {
-    const int64_t items = (int64_t)batch * runs * (Di / 4);
-    conv_front_bwd<T><<<(unsigned)((items + 255) / 256), 256, 0, stream>>>(x, conv_w, conv_b, du2, dx, part, batch,
-                                                                            L, Di, vec);
+    conv_front_bwd<T><<<front_grid(batch, L, Di), kFrontThr, 0, stream>>>(x, conv_w, conv_b, du2, dx, part, batch, L,
+                                                                           Di, vec);
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     // rows of [dw: 6 Di | dcb: 2 Di] summed in a fixed order
     const int cols = 8 * Di;

@@ -207,12 +207,13 @@ vim_status block_bwd_n(const void *x, const float *conv_w, const float *conv_b, 
     pa.M = M; pa.L = L; pa.Di = Di;
     vim_status st = launch_proj<N>(pa, conv, stream);
     if (st != VIM_OK) return st;
-    const unsigned ublocks = (unsigned)std::min<int64_t>((act / 4 + 255) / 256, grid_stride);
-    if (conv)
-        conv_front_fwd<__nv_bfloat16><<<ublocks, 256, 0, stream>>>(xb, conv_w, conv_b, u2, batch, L, Di, 1);
-    else
+    if (conv) {
+        st = launch_front_fwd<__nv_bfloat16>(xb, conv_w, conv_b, u2, batch, L, Di, 1, stream);
+        if (st != VIM_OK) return st;
+    } else {
         block_u_copy<<<(unsigned)std::min<int64_t>((act + 255) / 256, grid_stride), 256, 0, stream>>>(xb, u2, act);
-    if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+        if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+    }
 
     // ---- the scan's derivative, per direction ----------------------------------------
     const __nv_bfloat16 *Bw = reinterpret_cast<const __nv_bfloat16 *>(ws + cp.off_B);
