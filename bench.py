@@ -76,21 +76,27 @@ def peaks():
         return dict(hbm_gbs=6650.0, sm_max_mhz=1965.0, source="fallback")
 
 
-def profiled_traffic(w):
-    """DRAM bytes per launch of pair_main from the committed ncu summary of this workload,
+def profiled_traffic(w, bwd=False, zoh=False):
+    """DRAM bytes per launch of the dominant kernel (pair_main; bwd_main for the derivative,
+    with or without the exact hold) from the committed ncu summary of this workload and mode,
     or None when there is none or the kernel source changed since it was captured."""
     import hashlib
     import re
 
-    path = os.path.join(ROOT, "profiles", f"ncu_scan_kernels_{w.name}.md")
-    src = os.path.join(ROOT, "vision_mamba_selective_b200", "csrc", "scan_kernels.cuh")
+    if bwd:
+        name = f"ncu_bwd_main_zoh_{w.name}.md" if zoh else f"ncu_bwd_kernels_{w.name}.md"
+        source, kernel = "bwd_kernels.cuh", "bwd_main"
+    else:
+        name, source, kernel = f"ncu_scan_kernels_{w.name}.md", "scan_kernels.cuh", "pair_main"
+    path = os.path.join(ROOT, "profiles", name)
+    src = os.path.join(ROOT, "vision_mamba_selective_b200", "csrc", source)
     try:
         text = open(path).read()
         fp = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     except OSError:
         return None
-    m = re.search(r"traffic_bytes_per_launch pair_main: (\d+)", text)
-    f = re.search(r"kernel source fingerprint \(sha256 of scan_kernels.cuh, first 16 hex\): ([0-9a-f]+)", text)
+    m = re.search(rf"traffic_bytes_per_launch {kernel}: (\d+)", text)
+    f = re.search(rf"kernel source fingerprint \(sha256 of {re.escape(source)}, first 16 hex\): ([0-9a-f]+)", text)
     if not m or not f or f.group(1) != fp:
         return None
     return int(m.group(1))
@@ -689,7 +695,12 @@ def main():
     clocks = clk.summary()
     peak_ops = SMS * FP32_LANES_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e12
     achieved_ops = ops / (main_ms * 1e-3) / 1e12
-    traffic = None if (args.bwd or args.conv or args.zoh or args.block) else profiled_traffic(w)
+    if whole_call or args.block or args.conv:
+        traffic = None
+    elif args.bwd:
+        traffic = profiled_traffic(w, bwd=True, zoh=args.zoh)
+    else:
+        traffic = None if args.zoh else profiled_traffic(w)
     roofline = {
         "bound": "alu", "kernel": main_name, "achieved": achieved_ops, "peak": peak_ops,
         "unit": "Tops/s", "frac": achieved_ops / peak_ops,
