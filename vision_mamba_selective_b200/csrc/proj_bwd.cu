@@ -35,43 +35,79 @@ __global__ void __launch_bounds__(256) block_u_copy(const __nv_bfloat16 *x, floa
     }
 }
 
-// dl/ds_k[m] (one warp per (k, m): a dot over the channels) and the row dP_k[m, :]
-__global__ void __launch_bounds__(256) proj_bwd_ds(const float *dd2, const float *Wdt, const float *dB2,
-                                                   const float *dC2, float *dP, int64_t M, int Di, int N) {
-    const int NO = 2 * N + 1;
-    const int64_t w = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) / 32;
-    const int lane = threadIdx.x % 32;
-    if (w >= 2 * M) return;   // whole warps: 256 threads per CTA
-    const int k = (int)(w / M);
-    const int64_t m = w % M;
-    const float *row = dd2 + (size_t)w * Di, *wdt = Wdt + (size_t)k * Di;
-    float acc = 0.0f;
-    for (int d = lane; d < Di; d += 32) acc = fmaf(row[d], wdt[d], acc);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    float *out = dP + (size_t)w * NO;
-    const size_t bc = ((size_t)k * M + m) * N;
-    for (int j = lane; j < NO; j += 32) out[j] = j < N ? dB2[bc + j] : j < 2 * N ? dC2[bc + j - N] : acc;
-}
-
-// dl/dWdt partials: part[p][k * Di + d] = sum over rows m of part p (kWdtRows each) of
-// dd2_k[m, d] s_k[m]; the column kernels then sum the parts in a fixed order
+// Back through dt_proj, per pathway k and tile of kWdtRows tokens (one CTA of 256
+// threads; warp w takes rows 8w .. 8w+7 of the tile, lane l channels l, l + 32, ...):
+//   dl/ds_k[m] = sum_d dd2_k[m, d] Wdt_k[d]      (the row dP_k[m, :] = [dl/dB_k | dl/dC_k | dl/ds_k]),
+//   part[tile][k * Di + d] = sum over the tile's rows of dd2_k[m, d] s_k[m]   (dl/dWdt partials).
+// dd2 is read once, four 32-channel steps of the warp's 8 rows in flight per lane; each
+// warp's column sums go to its row of red[8][Di] in shared memory (dynamic, 32 Di bytes),
+// which the CTA adds in warp order after one barrier; the column kernels sum the tiles.
 constexpr int kWdtRows = 64;
-__global__ void __launch_bounds__(256) proj_bwd_dwdt(const float *dd2, const float *s2, float *tmp, int64_t M,
-                                                     int Di) {
-    const int col = blockIdx.x * blockDim.x + threadIdx.x, part = blockIdx.y;
-    if (col >= 2 * Di) return;
-    const int k = col / Di, d = col % Di;
-    const int64_t m0 = (int64_t)part * kWdtRows, m1 = m0 + kWdtRows < M ? m0 + kWdtRows : M;
-    const float *src = dd2 + (size_t)k * M * Di + d, *s = s2 + (size_t)k * M;
-    float a0 = 0.0f, a1 = 0.0f;
-    int64_t m = m0;
-    for (; m + 2 <= m1; m += 2) {
-        a0 = fmaf(src[(size_t)m * Di], s[m], a0);
-        a1 = fmaf(src[(size_t)(m + 1) * Di], s[m + 1], a1);
+#ifndef VIMSCAN_DT_STEPS
+#define VIMSCAN_DT_STEPS 2
+#endif
+constexpr int kDtSteps = VIMSCAN_DT_STEPS;   // 32-channel steps of a lane's loads in flight
+#ifndef VIMSCAN_DT_MINB
+#define VIMSCAN_DT_MINB 3     // resident CTAs per SM the register budget targets
+#endif
+__global__ void __launch_bounds__(256, VIMSCAN_DT_MINB) proj_bwd_dt(const float *dd2, const float *Wdt, const float *s2,
+                                                   const float *dB2, const float *dC2, float *dP, float *tmp,
+                                                   int64_t M, int Di, int N) {
+    constexpr int RW = kWdtRows / 8;   // rows per warp
+    extern __shared__ float red[];     // [8][Di]
+    const int k = blockIdx.y, warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t m0 = (int64_t)blockIdx.x * kWdtRows + warp * RW;   // the warp's first row
+    const float *src = dd2 + ((size_t)k * M) * Di, *wdt = Wdt + (size_t)k * Di, *sk = s2 + (size_t)k * M;
+    float sv[RW], rs[RW];
+#pragma unroll
+    for (int r = 0; r < RW; ++r) {
+        sv[r] = m0 + r < M ? sk[m0 + r] : 0.0f;
+        rs[r] = 0.0f;
     }
-    if (m < m1) a0 = fmaf(src[(size_t)m * Di], s[m], a0);
-    tmp[(size_t)part * 2 * Di + col] = a0 + a1;
+    for (int c0 = 0; c0 < Di; c0 += 32 * kDtSteps) {
+        float v[kDtSteps][RW];
+#pragma unroll
+        for (int e = 0; e < kDtSteps; ++e)
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                const int d = c0 + 32 * e + lane;
+                v[e][r] = (m0 + r < M && d < Di) ? src[(size_t)(m0 + r) * Di + d] : 0.0f;
+            }
+#pragma unroll
+        for (int e = 0; e < kDtSteps; ++e) {
+            const int d = c0 + 32 * e + lane;
+            if (d < Di) {
+                const float wd = wdt[d];
+                float cs = 0.0f;
+#pragma unroll
+                for (int r = 0; r < RW; ++r) {
+                    rs[r] = fmaf(v[e][r], wd, rs[r]);
+                    cs = fmaf(v[e][r], sv[r], cs);
+                }
+                red[warp * Di + d] = cs;
+            }
+        }
+    }
+    __syncthreads();
+    for (int d = threadIdx.x; d < Di; d += 256) {
+        float a = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) a += red[q * Di + d];
+        tmp[(size_t)blockIdx.x * 2 * Di + (size_t)k * Di + d] = a;
+    }
+    const int NO = 2 * N + 1;
+#pragma unroll
+    for (int r = 0; r < RW; ++r) {
+        float a = rs[r];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        const int64_t m = m0 + r;
+        if (m < M) {
+            const size_t row = (size_t)k * M + m;
+            float *out = dP + row * NO;
+            for (int j = lane; j < NO; j += 32) out[j] = j < N ? dB2[row * N + j] : j < 2 * N ? dC2[row * N + j - N] : a;
+        }
+    }
 }
 
 // dl/du_k += dP_k Wx_k^T, and dl/dWx_k partial sums over a tile of kPbRows tokens:
@@ -259,12 +295,14 @@ vim_status block_bwd_n(const void *x, const float *conv_w, const float *conv_b, 
     if (st != VIM_OK) return st;
 
     // ---- back through dt_proj and x_proj ------------------------------------------------
-    proj_bwd_ds<<<(unsigned)((2 * M * 32 + 255) / 256), 256, 0, stream>>>(dd2, Wdt, dB2, dC2, dP, M, Di, N);
-    if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     float *wtmp = reinterpret_cast<float *>(ws + cp.off_wtmp);
     const int wparts = (int)((M + kWdtRows - 1) / kWdtRows);
     float *wtmp2 = wtmp + (size_t)wparts * 2 * Di;
-    proj_bwd_dwdt<<<dim3((2 * Di + 255) / 256, wparts), 256, 0, stream>>>(dd2, s2, wtmp, M, Di);
+    const size_t dt_smem = (size_t)8 * Di * sizeof(float);
+    if (dt_smem > 48 * 1024 &&
+        cudaFuncSetAttribute(proj_bwd_dt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dt_smem) != cudaSuccess)
+        return VIM_ERR_CUDA;
+    proj_bwd_dt<<<dim3(wparts, 2), 256, dt_smem, stream>>>(dd2, Wdt, s2, dB2, dC2, dP, wtmp, M, Di, N);
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
     bwd_reduce_cols1<<<dim3((2 * Di + 255) / 256, kReduceParts), 256, 0, stream>>>(wtmp, wtmp2, wparts, 2 * Di);
     if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
