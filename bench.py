@@ -76,10 +76,11 @@ def peaks():
         return dict(hbm_gbs=6650.0, sm_max_mhz=1965.0, source="fallback")
 
 
-def profiled_traffic(w, bwd=False, zoh=False):
-    """DRAM bytes per launch of the dominant kernel (pair_main; bwd_main for the derivative,
-    with or without the exact hold) from the committed ncu summary of this workload and mode,
-    or None when there is none or the kernel source changed since it was captured."""
+def profiled_traffic(w, bwd=False, zoh=False, conv=False):
+    """DRAM bytes per launch of the dominant kernel (pair_main, with the fused front or the
+    exact hold or neither; bwd_main for the derivative, with or without the exact hold) from
+    the committed ncu summary of this workload and mode, or None when there is none or the
+    kernel source changed since it was captured."""
     import hashlib
     import re
 
@@ -87,7 +88,10 @@ def profiled_traffic(w, bwd=False, zoh=False):
         name = f"ncu_bwd_main_zoh_{w.name}.md" if zoh else f"ncu_bwd_kernels_{w.name}.md"
         source, kernel = "bwd_kernels.cuh", "bwd_main"
     else:
-        name, source, kernel = f"ncu_scan_kernels_{w.name}.md", "scan_kernels.cuh", "pair_main"
+        if conv and zoh:
+            return None
+        mode = "conv_" if conv else "zoh_" if zoh else ""
+        name, source, kernel = f"ncu_scan_kernels_{mode}{w.name}.md", "scan_kernels.cuh", "pair_main"
     path = os.path.join(ROOT, "profiles", name)
     src = os.path.join(ROOT, "vision_mamba_selective_b200", "csrc", source)
     try:
@@ -695,12 +699,12 @@ def main():
     clocks = clk.summary()
     peak_ops = SMS * FP32_LANES_PER_SM * pk["sm_max_mhz"] * 1e6 / 1e12
     achieved_ops = ops / (main_ms * 1e-3) / 1e12
-    if whole_call or args.block or args.conv:
+    if whole_call or args.block:
         traffic = None
     elif args.bwd:
         traffic = profiled_traffic(w, bwd=True, zoh=args.zoh)
     else:
-        traffic = None if args.zoh else profiled_traffic(w)
+        traffic = profiled_traffic(w, zoh=args.zoh, conv=args.conv)
     roofline = {
         "bound": "alu", "kernel": main_name, "achieved": achieved_ops, "peak": peak_ops,
         "unit": "Tops/s", "frac": achieved_ops / peak_ops,

@@ -48,8 +48,14 @@ def test_profiled_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
     (tmp_path / "profiles" / f"ncu_bwd_kernels_{w.name}.md").write_text(
         "traffic_bytes_per_launch adj_carry: 7\ntraffic_bytes_per_launch bwd_main: 456\n\nkernel source "
         f"fingerprint (sha256 of bwd_kernels.cuh, first 16 hex): {fp['bwd_kernels.cuh']}\n")
+    (tmp_path / "profiles" / f"ncu_scan_kernels_conv_{w.name}.md").write_text(
+        "traffic_bytes_per_launch pair_main: 321\n\nkernel source fingerprint (sha256 of scan_kernels.cuh, "
+        f"first 16 hex): {fp['scan_kernels.cuh']}\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.profiled_traffic(w) == 123
+    assert bench.profiled_traffic(w, conv=True) == 321
+    assert bench.profiled_traffic(w, zoh=True) is None                # no capture of that mode
+    assert bench.profiled_traffic(w, zoh=True, conv=True) is None
     assert bench.profiled_traffic(w, bwd=True) == 456
     assert bench.profiled_traffic(w, bwd=True, zoh=True) is None   # no capture of that mode
     assert bench.profiled_traffic(workloads.WORKLOADS[0]) is None   # nor of that workload

@@ -39,9 +39,10 @@ __global__ void __launch_bounds__(256) block_u_copy(const __nv_bfloat16 *x, floa
 // threads; warp w takes rows 8w .. 8w+7 of the tile, lane l channels l, l + 32, ...):
 //   dl/ds_k[m] = sum_d dd2_k[m, d] Wdt_k[d]      (the row dP_k[m, :] = [dl/dB_k | dl/dC_k | dl/ds_k]),
 //   part[tile][k * Di + d] = sum over the tile's rows of dd2_k[m, d] s_k[m]   (dl/dWdt partials).
-// dd2 is read once, four 32-channel steps of the warp's 8 rows in flight per lane; each
-// warp's column sums go to its row of red[8][Di] in shared memory (dynamic, 32 Di bytes),
-// which the CTA adds in warp order after one barrier; the column kernels sum the tiles.
+// dd2 is read once, kDtSteps 32-channel steps of the warp's 8 rows in flight per lane (16
+// loads); each warp's column sums go to its row of red[8][Di] in shared memory (dynamic,
+// 32 Di bytes), which the CTA adds in warp order after one barrier; the column kernels sum
+// the tiles.
 constexpr int kWdtRows = 64;
 #ifndef VIMSCAN_DT_STEPS
 #define VIMSCAN_DT_STEPS 2
@@ -50,9 +51,9 @@ constexpr int kDtSteps = VIMSCAN_DT_STEPS;   // 32-channel steps of a lane's loa
 #ifndef VIMSCAN_DT_MINB
 #define VIMSCAN_DT_MINB 3     // resident CTAs per SM the register budget targets
 #endif
-__global__ void __launch_bounds__(256, VIMSCAN_DT_MINB) proj_bwd_dt(const float *dd2, const float *Wdt, const float *s2,
-                                                   const float *dB2, const float *dC2, float *dP, float *tmp,
-                                                   int64_t M, int Di, int N) {
+__global__ void __launch_bounds__(256, VIMSCAN_DT_MINB)
+    proj_bwd_dt(const float *dd2, const float *Wdt, const float *s2, const float *dB2, const float *dC2, float *dP,
+                float *tmp, int64_t M, int Di, int N) {
     constexpr int RW = kWdtRows / 8;   // rows per warp
     extern __shared__ float red[];     // [8][Di]
     const int k = blockIdx.y, warp = threadIdx.x / 32, lane = threadIdx.x % 32;
