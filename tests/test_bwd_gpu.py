@@ -269,6 +269,7 @@ CROSS_CASES = [
     (1, 7, 40, 64, 16, torch.float32, False, True),     # 280 tokens: several 32-token chunks
     (1, 40, 7, 32, 4, torch.float32, True, False),
     (2, 16, 16, 64, 16, torch.bfloat16, False, True),
+    (1, 127, 3, 32, 16, torch.float32, False, True),    # tall grid: chunks span column ends at odd H
 ]
 
 

@@ -260,6 +260,8 @@ CROSS_CASES = [
     (1, 7, 40, 64, 16, torch.float32, False, True),     # 280 tokens: several chunks
     (1, 40, 7, 64, 4, torch.float32, True, True),
     (2, 32, 48, 72, 16, torch.bfloat16, False, True),
+    (1, 127, 3, 64, 16, torch.float32, False, True),    # tall: a tile spans column ends at odd H
+    (1, 2, 300, 64, 16, torch.float32, False, True),    # H = 2: every other token starts a column
 ]
 
 

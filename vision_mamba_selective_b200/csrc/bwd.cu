@@ -316,7 +316,7 @@ vim_status vmamba_cross_scan4_bwd_ex(const void *u, const void *delta, const voi
         a.batch = batch; a.L = L; a.Di = channels; a.G = pl.G; a.nblk = pl.nblk; a.cl = pl.cl; a.ncol = pl.ncol;
         a.separate_bc = 1;
         set_vector_flags(a, dt, d_state);
-        a.order = pair; a.H = H; a.W = W;
+        a.order = pair; a.H = H; a.W = W; a.hdiv = div_inv((unsigned)H);
         a.stage = pair + 1;                  // the row pair leaves partials, the column pair finishes
         a.acc_y = acc;
         a.acc_du = reinterpret_cast<float *>(ws + pl.total + acc_bytes);
@@ -329,7 +329,7 @@ vim_status vmamba_cross_scan4_bwd_ex(const void *u, const void *delta, const voi
         f.A = a.A; f.D = a.D; f.bias = a.bias;
         f.hloc = reinterpret_cast<float *>(ws + pl.off_hloc);
         f.ssum = reinterpret_cast<float *>(ws + pl.off_ssum);
-        f.batch = batch; f.L = L; f.Di = channels; f.H = H; f.W = W; f.order = pair;
+        f.batch = batch; f.L = L; f.Di = channels; f.H = H; f.W = W; f.order = pair; f.hdiv = div_inv((unsigned)H);
         f.chunk = kBwdChunk; f.G = pl.G;
 
         float *dBo[2] = {dB + (2 * pair) * bc, dB + (2 * pair + 1) * bc};

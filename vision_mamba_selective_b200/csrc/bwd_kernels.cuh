@@ -80,6 +80,7 @@ struct BwdArgs {
     int vec_bc;                         // B and C rows move as 16-byte vectors
     int order, H, W;                    // visiting order of the pair (0: position = step;
                                         // 1: column-major on H x W, the cross-scan's second pair)
+    DivInv hdiv;                        // division by H (order 1)
     int stage;                          // 0: one pair (Vim), final outputs; 1: first pair of the
                                         // cross-scan, fp32 partials to acc_*; 2: second pair, adds them
     float *acc_y, *acc_du, *acc_dd;     // [batch, L, Di] fp32 by position (stages 1 and 2)
@@ -96,7 +97,7 @@ namespace {
 // grid position visited at step t of the pair's forward direction
 __device__ __forceinline__ int bpos(const BwdArgs &p, int t) {
     if (p.order == 0) return t;
-    const int h = t % p.H, w = t / p.H;
+    const int w = (int)div_by((unsigned)t, p.hdiv), h = t - w * p.H;
     return h * p.W + w;
 }
 

@@ -237,6 +237,33 @@ __device__ __forceinline__ void load_row(const float *row, float2 (&v)[NP]) {
 }
 
 // ----------------------------------------------------------------------------
+// division by the grid height H, which the column-major order needs for every row it
+// stages: the method of Granlund and Montgomery, "Division by Invariant Integers using
+// Multiplication" (PLDI 1994), Figure 4.1, for 32-bit unsigned n and 1 <= d < 2^32:
+//   l = ceil(log2 d),  m = floor(2^32 (2^l - d) / d) + 1,  s1 = min(l, 1),  s2 = max(l - 1, 0),
+//   t = high 32 bits of m n,  n / d = (t + ((n - t) >> s1)) >> s2.
+// The host forms (m, s1, s2) once per call; the kernels then divide in four instructions
+// instead of a full integer division per row.
+// ----------------------------------------------------------------------------
+struct DivInv {
+    unsigned m;
+    int s1, s2;
+};
+inline DivInv div_inv(unsigned d) {
+    int l = 0;
+    while (l < 32 && (1ull << l) < d) ++l;   // ceil(log2 d)
+    DivInv v;
+    v.m = (unsigned)((((1ull << l) - d) << 32) / d + 1);
+    v.s1 = l < 1 ? l : 1;
+    v.s2 = l > 1 ? l - 1 : 0;
+    return v;
+}
+__device__ __forceinline__ unsigned div_by(unsigned n, const DivInv &v) {
+    const unsigned t = __umulhi(v.m, n);
+    return (t + ((n - t) >> v.s1)) >> v.s2;
+}
+
+// ----------------------------------------------------------------------------
 // arguments
 // ----------------------------------------------------------------------------
 struct PairArgs {
@@ -256,6 +283,7 @@ struct PairArgs {
     float *ssum;                    // [batch][G][2][Di]    chunk Delta sums
     int batch, L, Di, H, W;
     int order;                      // 0: position = step; 1: column-major on H x W
+    DivInv hdiv;                    // division by H (order 1)
     int chunk, G;                   // tokens per chunk (multiple of kTile), chunks
     const float *dt_in;             // [2][batch*L] step input per direction and position, or null
     const float *dt_w;              // [2][Di] its dt_proj weights: delta_raw = dt_in * dt_w
@@ -267,7 +295,7 @@ struct PairArgs {
 // position visited at step t of the forward direction
 __device__ __forceinline__ int position(const PairArgs &p, int t) {
     if (p.order == 0) return t;
-    const int h = t % p.H, w = t / p.H;
+    const int w = (int)div_by((unsigned)t, p.hdiv), h = t - w * p.H;
     return h * p.W + w;
 }
 

@@ -191,6 +191,7 @@ vim_status vmamba_cross_scan4_ex(const void *u, const void *delta, const void *z
         a.bias = delta_bias + (size_t)2 * pair * channels;
         a.batch = batch; a.L = L; a.Di = channels; a.H = H; a.W = W;
         a.order = pair;               // pair 0: scans 1/2 (rows), pair 1: scans 3/4 (columns)
+        a.hdiv = div_inv((unsigned)H);
         a.chunk = pl.chunk; a.G = pl.G;
         a.zoh = (flags & VIM_FLAG_ZOH_EXACT) ? 1 : 0;
         if (pl.G > 1) {
