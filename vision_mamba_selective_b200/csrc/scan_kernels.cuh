@@ -258,8 +258,12 @@ inline DivInv div_inv(unsigned d) {
     v.s2 = l > 1 ? l - 1 : 0;
     return v;
 }
-__device__ __forceinline__ unsigned div_by(unsigned n, const DivInv &v) {
+__host__ __device__ __forceinline__ unsigned div_by(unsigned n, const DivInv &v) {
+#ifdef __CUDA_ARCH__
     const unsigned t = __umulhi(v.m, n);
+#else
+    const unsigned t = (unsigned)(((unsigned long long)v.m * n) >> 32);
+#endif
     return (t + ((n - t) >> v.s1)) >> v.s2;
 }
 
