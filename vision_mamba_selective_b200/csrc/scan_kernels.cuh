@@ -56,6 +56,9 @@ constexpr int kTile = 16;            // tokens per staged tile
 #ifndef VIMSCAN_CARRY_KSUB
 #define VIMSCAN_CARRY_KSUB 8
 #endif
+#ifndef VIMSCAN_CARRY_DT_MIN_BLOCKS
+#define VIMSCAN_CARRY_DT_MIN_BLOCKS 5   // the step-input carry spills at the register budget of 6
+#endif
 #ifndef VIMSCAN_CARRY_MIN_BLOCKS
 #define VIMSCAN_CARRY_MIN_BLOCKS 6
 #endif
@@ -69,6 +72,7 @@ constexpr int kSub = VIMSCAN_KSUB;   // tokens whose independent work is formed 
 constexpr int kMinBlocks = VIMSCAN_MIN_BLOCKS;   // resident CTAs per SM the register budget targets
 constexpr int kCarrySub = VIMSCAN_CARRY_KSUB;          // the same for the chunk-summary kernel
 constexpr int kCarryMinBlocks = VIMSCAN_CARRY_MIN_BLOCKS;
+constexpr int kCarryDtMinBlocks = VIMSCAN_CARRY_DT_MIN_BLOCKS;
 constexpr int kCarryZohSub = VIMSCAN_CARRY_ZOH_KSUB;   // the same two with the exact hold
 constexpr int kCarryZohMinBlocks = VIMSCAN_CARRY_ZOH_MIN_BLOCKS;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -684,7 +688,8 @@ __device__ __forceinline__ void carry_tile(float2 (&H)[N / 2], float &Ssum, cons
 
 // (the exact hold needs more registers per thread, so fewer CTAs per SM)
 template <typename T, int N, bool VEC_BC, bool CONV, bool ZOH, bool DT = false, bool SPAN = false>
-__global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : kCarryMinBlocks) pair_carry(PairArgs p) {
+__global__ void __launch_bounds__(kThreads, ZOH ? kCarryZohMinBlocks : DT ? kCarryDtMinBlocks : kCarryMinBlocks)
+    pair_carry(PairArgs p) {
     using S = Stage<T, N, CONV>;
     constexpr int NP = N / 2;
     constexpr int kSlot = S::kSlotBytes;
