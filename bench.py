@@ -61,6 +61,11 @@ def parse():
                     help="Vim workloads: time vim_block_scan (x_proj + dt_proj + the convolution front + scan)")
     ap.add_argument("--bwd", action="store_true",
                     help="Vim workloads: time the scan's derivative (vim_scan_bidir_bwd) instead")
+    ap.add_argument("--ckpt", action="store_true",
+                    help="Vim workloads: the forward scan keeps the derivative's chunk states "
+                         "(vim_scan_bidir_ckpt); with --bwd, time the derivative that takes them "
+                         "(vim_scan_bidir_bwd_ckpt; the states are the forward pass's outputs, formed "
+                         "before the timed region)")
     ap.add_argument("--e2e-slices", type=int, default=4,
                     help="pieces of the batch in the end-to-end figure's host-memory entry point")
     return ap.parse_args()
@@ -425,9 +430,17 @@ def cpu_model():
     return None
 
 
+def vs_ckpt_shape(w):
+    """Shape of the forward pass's checkpoints for a Vim workload."""
+    from vision_mamba_selective_b200 import vimscan as vs
+
+    return vs.ckpt_shape(w.batch, w.L, w.channels, w.d_state)
+
+
 def workload_name(w, args):
     return (w.name + ("+conv_front" if args.conv else "") + ("+zoh_exact" if args.zoh else "")
-            + ("+derivative" if args.bwd else "") + ("+projections+conv_front" if args.block else ""))
+            + ("+derivative" if args.bwd else "") + ("+projections+conv_front" if args.block else "")
+            + ("+checkpoints" if args.ckpt else ""))
 
 
 def main():
@@ -441,6 +454,8 @@ def main():
         raise SystemExit("--block runs alone (or with --bwd), on a bf16 workload")
     if args.bwd and args.conv and w.kind != "vim":
         raise SystemExit("--bwd --conv applies to the Vim workloads only")
+    if args.ckpt and (w.kind != "vim" or args.conv or args.block):
+        raise SystemExit("--ckpt applies to the Vim scan without front or projections")
     if args.impl == "reference":
         reference_arm(args, w)
         return
@@ -467,6 +482,7 @@ def main():
         host["dout"] = bwd_dout(w, replicas.rank_seed(w.seed + 2, rank)).reshape(host["u"].shape).contiguous()
         act_keys.append("dout")
         out_bytes = 3 * w.tok_ch * el + 2 * w.batch * w.tokens * w.d_state * 4 * (1 if w.kind == "vim" else 4)
+    ck_shape = vs_ckpt_shape(w) if args.ckpt else None
     set_bytes = sum(host[k].numel() * host[k].element_size() for k in act_keys) + out_bytes
     nsets = max(2, math.ceil(2.2 * L2_BYTES / set_bytes))
     params = {k: host[k].to(dev) for k in ("A", "D", "delta_bias")}
@@ -474,6 +490,8 @@ def main():
     for _ in range(nsets):
         s = {k: host[k].to(dev) for k in act_keys}
         s["y"] = torch.empty_like(s["u"])
+        if args.ckpt:
+            s["ck"] = torch.empty(ck_shape, dtype=torch.float32, device=dev)
         if args.bwd:
             f32 = lambda *shape: torch.empty(shape, dtype=torch.float32, device=dev)
             s["out"] = dict(du=torch.empty_like(s["u"]), ddelta=torch.empty_like(s["u"]), dz=torch.empty_like(s["u"]),
@@ -534,7 +552,7 @@ def main():
         if args.bwd and w.kind == "vim":
             vs.vim_scan_bidir_bwd(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"],
                                   params["delta_bias"], s["dout"], workspace=ws, out=s["out"], events=events,
-                                  zoh=args.zoh)
+                                  zoh=args.zoh, ckpt=s["ck"] if args.ckpt else None)
             return
         if args.bwd:
             vs.vmamba_cross_scan4_bwd(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"],
@@ -546,8 +564,23 @@ def main():
                                    s["C"], params["A"], params["D"], params["delta_bias"], y=s["y"],
                                    workspace=ws, events=events, zoh=args.zoh)
             return
+        if args.ckpt:
+            fn(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"], params["delta_bias"],
+               y=s["y"], workspace=fws, events=events, zoh=args.zoh, ckpt=s["ck"])
+            return
         fn(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"], params["delta_bias"],
            y=s["y"], workspace=ws, events=events, zoh=args.zoh)
+
+    if args.ckpt:
+        # the forward scan's workspace, and with --bwd the states each input set's forward
+        # pass leaves (inputs of the derivative, formed before any timing)
+        fws = torch.empty(max(vs.vim_scan_workspace_bytes(0, w.batch, w.L, 0, w.channels, w.d_state), 1),
+                          dtype=torch.uint8, device=dev)
+        if args.bwd:
+            for s in sets:
+                fn(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"], params["delta_bias"],
+                   y=s["y"], workspace=fws, zoh=args.zoh, ckpt=s["ck"])
+            torch.cuda.synchronize()
 
     barrier = replicas.barrier
 
@@ -623,9 +656,10 @@ def main():
         for a, name in enumerate(["summaries", "bwd_main", "reductions"], start=1):
             t = [evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(prof_steps)]
             per_kernel[name] = sum(t) / len(t)
-        # pair_carry, pair_combine, adj_carry, pair_combine (more than one chunk of
-        # 32 tokens), bwd_main, two dB/dC reductions, one two-pass column sum
-        launches_per_step = (4 if w.tokens > 32 else 0) + 1 + 2 + 2
+        # pair_carry, pair_combine (not with the forward's checkpoints), adj_carry,
+        # pair_combine (more than one chunk of 32 tokens), bwd_main, two dB/dC reductions,
+        # one two-pass column sum
+        launches_per_step = ((2 if args.ckpt else 4) if w.tokens > 32 else 0) + 1 + 2 + 2
     else:
         names = ["pair_carry", "pair_combine", "pair_main"]
         for p in range(pairs):
@@ -637,6 +671,9 @@ def main():
         launches_per_step = pairs * (3 if w.tokens > 256 else 1)
 
     # ---- end to end: pinned host inputs -> device -> scan -> host result ---------
+    if args.ckpt and args.bwd:
+        host["ck"] = sets[0]["ck"].cpu()
+        act_keys.append("ck")
     pinned = {k: host[k].pin_memory() for k in act_keys}
     if args.bwd:
         keys = ("dx", "dz", "dWx") if args.block else ("dx" if args.conv else "du", "ddelta", "dz", "dB", "dC")
@@ -653,7 +690,7 @@ def main():
 
     # the Vim forward scan has a host-memory entry point, which pipelines the copies of
     # batch pieces with their scans; the other modes copy everything, run, copy back
-    host_entry = w.kind == "vim" and not (args.bwd or args.block or args.conv)
+    host_entry = w.kind == "vim" and not (args.bwd or args.block or args.conv or args.ckpt)
     if host_entry:
         slices = max(1, min(args.e2e_slices, w.batch))
         hws = torch.empty(max(vs.vim_scan_host_workspace_bytes(w.batch, w.L, w.channels, w.d_state,
@@ -691,6 +728,8 @@ def main():
     # ---- roofline of the dominant kernel -----------------------------------------
     pk = peaks()
     nbytes, ops = algorithmic_bwd(w) if args.bwd else algorithmic(w, args.conv)
+    if args.ckpt:   # the checkpoints: written by the forward pass, read by the derivative
+        nbytes += math.prod(vs_ckpt_shape(w)) * 4
     main_name = "bwd_main" if args.bwd else "pair_main"
     if whole_call:
         main_name = ("vim_block_scan_bwd" if args.block else "vim_scan_bidir_conv_bwd" if args.conv
@@ -703,6 +742,8 @@ def main():
         traffic = None
     elif args.bwd:
         traffic = profiled_traffic(w, bwd=True, zoh=args.zoh)
+    elif args.ckpt:
+        traffic = None   # no capture of the forward kernel writing checkpoints
     else:
         traffic = profiled_traffic(w, zoh=args.zoh, conv=args.conv)
     roofline = {

@@ -494,6 +494,42 @@ size_t vim_scan_host_workspace_bytes(int batch, int L, int d_inner, int d_state,
                                      int two_bc);
 
 /*
+ * Training pair: the forward scan that also keeps the states its derivative needs, and
+ * the derivative that takes them.  Reverse mode needs h entering every 32-token chunk
+ * of the derivative in each direction ("Vision Mamba Guide", "Discretization via
+ * Zero-Order Hold (ZOH)": the recurrence h_t = Abar_t h_(t-1) + Bbar_t u_t, run by the
+ * forward pass anyway).  vim_scan_bidir_bwd forms them with a summary pass and a fold of
+ * its own; after vim_scan_bidir_ckpt the forward pass has written them as it went.
+ *
+ * vim_scan_bidir_ckpt: vim_scan_bidir_ex without the convolution front (same arguments,
+ * same y, same workspace), and
+ *   ckpt  : DEVICE, fp32 [batch][ceil(L / 32)][2][d_state][d_inner] (state-major, so that
+ *           the forward kernels write whole lines), vim_scan_ckpt_bytes bytes, 8-byte
+ *           aligned, written whole: entry [b][c][k] is the state of direction k (0 forward,
+ *           1 backward) entering 32-token chunk c in that direction's visiting order (zeros
+ *           for the chunk each direction visits first).
+ * vim_scan_bidir_bwd_ckpt: vim_scan_bidir_bwd_ex (same arguments, outputs and workspace)
+ *   with ckpt as written by vim_scan_bidir_ckpt on the same u, delta, B, C, A,
+ *   delta_bias and flags.  The results equal vim_scan_bidir_bwd_ex's up to rounding (the
+ *   states come from the forward kernels' arithmetic instead of the derivative's
+ *   summaries).  Checkpoints from other inputs give a wrong derivative, not an error.
+ * Both return VIM_ERR_INVALID_ARG for a NULL or misaligned ckpt on a non-empty problem.
+ */
+vim_status vim_scan_bidir_ckpt(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                               int64_t bc_dir_stride, const float *A, const float *D, const float *delta_bias,
+                               void *y, float *ckpt, int batch, int L, int d_inner, int d_state, vim_dtype dt,
+                               unsigned flags, void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                               cudaEvent_t *events);
+vim_status vim_scan_bidir_bwd_ckpt(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                                   int64_t bc_dir_stride, const float *A, const float *D, const float *delta_bias,
+                                   const float *ckpt, const void *dout, void *du, void *ddelta, void *dz, float *dB,
+                                   float *dC, float *dA, float *dD, float *ddelta_bias, int batch, int L,
+                                   int d_inner, int d_state, vim_dtype dt, unsigned flags, void *workspace,
+                                   size_t workspace_bytes, cudaStream_t stream, cudaEvent_t *events);
+/* Bytes of the checkpoints (0 for invalid arguments or an empty problem). */
+size_t vim_scan_ckpt_bytes(int batch, int L, int d_inner, int d_state);
+
+/*
  * Workspace bytes the scan entry points need (0 when none).  which = 0 for
  * vim_scan_bidir (L_or_H = L, W ignored), 1 for vmamba_cross_scan4 (L_or_H = H).
  * Returns 0 for invalid arguments as well; the entry point then reports them.

@@ -44,6 +44,7 @@ def test_header_declares_the_boundary():
                           "vim_scan_bidir_host", "vim_scan_host_workspace_bytes",
                           "vim_scan_bidir_conv_bwd", "vim_scan_bidir_conv_bwd_ex", "vim_scan_conv_bwd_workspace_bytes",
                           "vim_block_scan_bwd", "vim_block_bwd_workspace_bytes",
+                          "vim_scan_bidir_ckpt", "vim_scan_bidir_bwd_ckpt", "vim_scan_ckpt_bytes",
                           "vim_scan_workspace_bytes", "vim_status_string"}, names
 
 
@@ -237,6 +238,48 @@ def bwd_ex(vs, flags, **kw):
                                         a["bias"], a["dout"], a["du"], a["ddelta"], a["dz"], a["dB"], a["dC"],
                                         a["dA"], a["dD"], a["dbias"], a["batch"], a["L"], a["Di"], a["N"],
                                         a["dt"], flags, a["ws"], a["ws_bytes"], None, None)
+
+
+def bwd_ckpt(vs, flags, **kw):
+    """vim_scan_bidir_bwd_ckpt on fake device addresses (each case fails a host check)."""
+    a = dict(u=FAKE, delta=FAKE, z=FAKE, B=FAKE, C=FAKE, stride=0, A=FAKE, D=FAKE, bias=FAKE, ckpt=FAKE,
+             dout=FAKE, du=FAKE, ddelta=FAKE, dz=FAKE, dB=FAKE, dC=FAKE, dA=FAKE, dD=FAKE, dbias=FAKE,
+             batch=2, L=100, Di=64, N=16, dt=vs.VIM_BF16, ws=FAKE, ws_bytes=1 << 40)
+    a.update(kw)
+    return vs.lib.vim_scan_bidir_bwd_ckpt(a["u"], a["delta"], a["z"], a["B"], a["C"], a["stride"], a["A"],
+                                          a["D"], a["bias"], a["ckpt"], a["dout"], a["du"], a["ddelta"], a["dz"],
+                                          a["dB"], a["dC"], a["dA"], a["dD"], a["dbias"], a["batch"], a["L"],
+                                          a["Di"], a["N"], a["dt"], flags, a["ws"], a["ws_bytes"], None, None)
+
+
+def fwd_ckpt(vs, flags, **kw):
+    """vim_scan_bidir_ckpt on fake device addresses (each case fails a host check)."""
+    a = dict(u=FAKE, delta=FAKE, z=FAKE, B=FAKE, C=FAKE, stride=0, A=FAKE, D=FAKE, bias=FAKE, y=FAKE, ckpt=FAKE,
+             batch=2, L=100, Di=64, N=16, dt=vs.VIM_BF16, ws=FAKE, ws_bytes=1 << 40)
+    a.update(kw)
+    return vs.lib.vim_scan_bidir_ckpt(a["u"], a["delta"], a["z"], a["B"], a["C"], a["stride"], a["A"], a["D"],
+                                      a["bias"], a["y"], a["ckpt"], a["batch"], a["L"], a["Di"], a["N"], a["dt"],
+                                      flags, a["ws"], a["ws_bytes"], None, None)
+
+
+def test_ckpt_pair_rejects(vs):
+    # the checkpoints are required, 8-byte aligned; the rest is checked as without them
+    assert fwd_ckpt(vs, 0, ckpt=None) == vs.VIM_ERR_INVALID_ARG
+    assert fwd_ckpt(vs, 0, ckpt=FAKE + 4) == vs.VIM_ERR_INVALID_ARG
+    assert fwd_ckpt(vs, 2) == vs.VIM_ERR_INVALID_ARG                  # unknown flag bit
+    assert fwd_ckpt(vs, 0, N=3) == vs.VIM_ERR_UNSUPPORTED
+    assert fwd_ckpt(vs, vs.VIM_FLAG_ZOH_EXACT, ws=None) == vs.VIM_ERR_WORKSPACE
+    assert bwd_ckpt(vs, 0, ckpt=None) == vs.VIM_ERR_INVALID_ARG
+    assert bwd_ckpt(vs, 0, ckpt=FAKE + 4) == vs.VIM_ERR_INVALID_ARG
+    assert bwd_ckpt(vs, 2) == vs.VIM_ERR_INVALID_ARG
+    assert bwd_ckpt(vs, 0, dz=None) == vs.VIM_ERR_INVALID_ARG
+    assert bwd_ckpt(vs, vs.VIM_FLAG_ZOH_EXACT, ws=None) == vs.VIM_ERR_WORKSPACE
+    # [batch][ceil(L / 32)][2][d_state][d_inner] fp32
+    assert vs.lib.vim_scan_ckpt_bytes(2, 100, 64, 16) == 2 * 4 * 2 * 64 * 16 * 4
+    assert vs.lib.vim_scan_ckpt_bytes(8, 4097, 384, 16) == 8 * 129 * 2 * 384 * 16 * 4
+    assert vs.lib.vim_scan_ckpt_bytes(0, 100, 64, 16) == 0
+    assert vs.lib.vim_scan_ckpt_bytes(2, 100, 64, 3) == 0
+    assert vs.ckpt_shape(2, 100, 64, 16) == (2, 4, 2, 16, 64)
 
 
 def test_bwd_ex_rejects(vs):

@@ -429,3 +429,72 @@ def test_conv_bwd_deterministic(vs):
     a, b = run_conv(vs, x), run_conv(vs, x)
     for k, _ in CONV_KEYS:
         assert torch.equal(a[k], b[k]), k
+
+
+# the training pair: the forward scan keeping the derivative's chunk states
+# (vim_scan_bidir(ckpt=...)) and the derivative that takes them
+CKPT_CASES = [
+    # batch, L, Di, N, dtype, separate_bc, generic_A, gate, zoh
+    (1, 1, 16, 16, torch.float32, False, False, True, False),
+    (2, 31, 16, 4, torch.float32, True, False, True, False),       # one partial chunk
+    (1, 64, 64, 16, torch.float32, False, True, True, False),      # two whole chunks
+    (2, 100, 40, 8, torch.float32, False, False, False, False),    # the forward's 32-token chunks
+    (1, 240, 72, 16, torch.bfloat16, False, False, True, False),   # the forward's single chunk (L <= 256)
+    (1, 300, 64, 16, torch.float32, True, False, True, False),     # 96-token chunks, a ragged last one
+    (2, 1000, 64, 16, torch.bfloat16, False, False, True, False),
+    (1, 333, 64, 16, torch.float32, False, True, True, True),      # exact hold, general A
+    (1, 500, 64, 16, torch.bfloat16, False, False, True, True),
+]
+
+
+def ckpt_pair(vs, x, gate=True, zoh=False):
+    c = lambda k: x[k].cuda()
+    batch, L, Di = x["u"].shape
+    N = x["B"].shape[-1]
+    ck = torch.full(vs.ckpt_shape(batch, L, Di, N), float("nan"), device="cuda")
+    y = vs.vim_scan_bidir(c("u"), c("delta"), c("z") if gate else None, c("B"), c("C"), c("A"), c("D"), c("bias"),
+                          bc_dir_stride=x["stride"], zoh=zoh, ckpt=ck)
+    y_plain = vs.vim_scan_bidir(c("u"), c("delta"), c("z") if gate else None, c("B"), c("C"), c("A"), c("D"),
+                                c("bias"), bc_dir_stride=x["stride"], zoh=zoh)
+    got = vs.vim_scan_bidir_bwd(c("u"), c("delta"), c("z") if gate else None, c("B"), c("C"), c("A"), c("D"),
+                                c("bias"), c("dout"), bc_dir_stride=x["stride"], zoh=zoh, ckpt=ck)
+    torch.cuda.synchronize()
+    return y, y_plain, ck, got
+
+
+@pytest.mark.parametrize("case", CKPT_CASES, ids=lambda c: f"b{c[0]}_L{c[1]}_D{c[2]}_N{c[3]}_{str(c[4])[6:]}"
+                         f"{'_sepBC' if c[5] else ''}{'_genA' if c[6] else ''}{'' if c[7] else '_nogate'}"
+                         f"{'_zoh' if c[8] else ''}")
+def test_ckpt_pair(vs, case):
+    batch, L, Di, N, dtype, sep, gen, gate, zoh = case
+    x = inputs(batch, L, Di, N, dtype, seed=L * 11 + Di, separate_bc=sep, generic_A=gen)
+    y, y_plain, ck, got = ckpt_pair(vs, x, gate, zoh)
+    # keeping the states changes nothing in y; every entry is written, and the chunk each
+    # direction visits first starts from zero
+    assert torch.equal(y, y_plain)
+    assert torch.isfinite(ck).all()
+    assert (ck[:, 0, 0] == 0).all() and (ck[:, -1, 1] == 0).all()
+    want = oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"] if gate else None, x["B"], x["C"], x["A"], x["D"],
+                                x["bias"], x["dout"], bc_dir_stride=x["stride"], zoh=zoh)
+    check_all(f"bwd_ckpt_{case}", got, want, dtype)
+
+
+def test_ckpt_pair_full_size(vs):
+    """The 1024 px Vim-Ti workload: the derivative from the forward's states against the
+    oracle, and against the derivative that forms its own."""
+    w = wl.BY_NAME["vim_tiny_1024px_bf16"]
+    x = wl.make_inputs(w)
+    g = torch.Generator().manual_seed(779)
+    x["dout"] = torch.randn(x["u"].shape, generator=g).to(x["u"].dtype)
+    x["bias"], x["stride"] = x["delta_bias"], 0
+    oracle.set_threads(max(1, len(os.sched_getaffinity(0))))
+    y, y_plain, ck, got = ckpt_pair(vs, x)
+    assert torch.equal(y, y_plain)
+    c = lambda k: x[k].cuda()
+    own = vs.vim_scan_bidir_bwd(c("u"), c("delta"), c("z"), c("B"), c("C"), c("A"), c("D"), c("bias"), c("dout"))
+    torch.cuda.synchronize()
+    for k in ("dA", "dD", "ddelta_bias", "dB", "dC"):
+        gates.gate(f"bwd_ckpt_vs_own:{k}", got[k], own[k].double(), torch.float32, norm_tol=SUM_TOL_FULL,
+                   elementwise=False)
+    want = oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["bias"], x["dout"])
+    check_all("bwd_ckpt_full", got, want, torch.bfloat16, sum_tol=SUM_TOL_FULL)

@@ -18,12 +18,18 @@ size_t vim_scan_bwd_workspace_bytes(int batch, int L, int d_inner, int d_state, 
     return bwd_plan(batch, L, d_inner, d_state, separate_bc).total;
 }
 
-vim_status vim_scan_bidir_bwd_ex(const void *u, const void *delta, const void *z, const void *B, const void *C,
-                                 int64_t bc_dir_stride, const float *A, const float *D, const float *delta_bias,
-                                 const void *dout, void *du, void *ddelta, void *dz, float *dB, float *dC,
-                                 float *dA, float *dD, float *ddelta_bias, int batch, int L, int d_inner,
-                                 int d_state, vim_dtype dt, unsigned flags, void *workspace, size_t workspace_bytes,
-                                 cudaStream_t stream, cudaEvent_t *events) {
+}  // extern "C"
+
+namespace {
+
+// the derivative of vim_scan_bidir; ckpt, or null: the forward pass's checkpoints
+// (vim_scan_bidir_ckpt), which replace the derivative's own forward summaries
+vim_status bidir_bwd_impl(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                          int64_t bc_dir_stride, const float *A, const float *D, const float *delta_bias,
+                          const void *dout, void *du, void *ddelta, void *dz, float *dB, float *dC, float *dA,
+                          float *dD, float *ddelta_bias, int batch, int L, int d_inner, int d_state, vim_dtype dt,
+                          unsigned flags, void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                          cudaEvent_t *events, const float *ckpt) {
     if (flags & ~VIM_FLAG_ZOH_EXACT) return VIM_ERR_INVALID_ARG;
     const bool zoh = (flags & VIM_FLAG_ZOH_EXACT) != 0;
     vim_status st = check_common(batch, L, d_inner, d_state, dt);
@@ -67,12 +73,14 @@ vim_status vim_scan_bidir_bwd_ex(const void *u, const void *delta, const void *z
     a.dB_part[1] = separate ? a.dB_part[0] + set_elems : a.dB_part[0];
     a.dC_part[1] = separate ? a.dC_part[0] + set_elems : a.dC_part[0];
     a.par = reinterpret_cast<float *>(ws + pl.off_par);
-    a.hin = reinterpret_cast<const float *>(ws + pl.off_hloc);
+    a.hin = ckpt ? ckpt : reinterpret_cast<const float *>(ws + pl.off_hloc);
+    a.hin_given = ckpt ? 1 : 0;
     a.gloc = reinterpret_cast<float *>(ws + pl.off_gloc);
     a.gsum = reinterpret_cast<float *>(ws + pl.off_gsum);
     a.batch = batch; a.L = L; a.Di = d_inner; a.G = pl.G; a.nblk = pl.nblk; a.cl = pl.cl; a.ncol = pl.ncol;
     a.separate_bc = separate;
     set_vector_flags(a, dt, d_state);
+    static_assert(kCkTokens == kBwdChunk, "the forward pass's checkpoints are the derivative's chunk starts");
 
     PairArgs f;
     std::memset(&f, 0, sizeof(f));
@@ -92,6 +100,33 @@ vim_status vim_scan_bidir_bwd_ex(const void *u, const void *delta, const void *z
     return zoh ? launch_bwd_n<__nv_bfloat16, true>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream, events)
                : launch_bwd_n<__nv_bfloat16, false>(d_state, a, f, dBo, dCo, dA, dD, ddelta_bias, tmp, stream,
                                                     events);
+}
+
+}  // namespace
+
+extern "C" {
+
+vim_status vim_scan_bidir_bwd_ex(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                                 int64_t bc_dir_stride, const float *A, const float *D, const float *delta_bias,
+                                 const void *dout, void *du, void *ddelta, void *dz, float *dB, float *dC,
+                                 float *dA, float *dD, float *ddelta_bias, int batch, int L, int d_inner,
+                                 int d_state, vim_dtype dt, unsigned flags, void *workspace, size_t workspace_bytes,
+                                 cudaStream_t stream, cudaEvent_t *events) {
+    return bidir_bwd_impl(u, delta, z, B, C, bc_dir_stride, A, D, delta_bias, dout, du, ddelta, dz, dB, dC, dA, dD,
+                          ddelta_bias, batch, L, d_inner, d_state, dt, flags, workspace, workspace_bytes, stream,
+                          events, nullptr);
+}
+
+vim_status vim_scan_bidir_bwd_ckpt(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                                   int64_t bc_dir_stride, const float *A, const float *D, const float *delta_bias,
+                                   const float *ckpt, const void *dout, void *du, void *ddelta, void *dz, float *dB,
+                                   float *dC, float *dA, float *dD, float *ddelta_bias, int batch, int L,
+                                   int d_inner, int d_state, vim_dtype dt, unsigned flags, void *workspace,
+                                   size_t workspace_bytes, cudaStream_t stream, cudaEvent_t *events) {
+    if (batch > 0 && L > 0 && d_inner > 0 && (!ckpt || !aligned_to(ckpt, 8))) return VIM_ERR_INVALID_ARG;
+    return bidir_bwd_impl(u, delta, z, B, C, bc_dir_stride, A, D, delta_bias, dout, du, ddelta, dz, dB, dC, dA, dD,
+                          ddelta_bias, batch, L, d_inner, d_state, dt, flags, workspace, workspace_bytes, stream,
+                          events, ckpt);
 }
 
 vim_status vim_scan_bidir_bwd_events(const void *u, const void *delta, const void *z, const void *B,

@@ -90,6 +90,8 @@ struct BwdArgs {
     const float *dt_in;                 // with DT: [2][batch*L] step input per direction and position;
     const float *dt_w;                  // [2][Di] dt_proj weights: delta_raw_k = dt_in_k * dt_w_k
     float *dd2;                         // with DT: [2][batch, L, Di] fp32 dl/ddelta_raw_k per direction
+    int hin_given;                      // hin holds the forward pass's checkpoints, state-major
+                                        // [batch][G][2][N][Di]: no forward summaries
 };
 
 namespace {
@@ -652,7 +654,16 @@ __device__ __forceinline__ void bwd_forward(const BwdArgs &p, const BwdSmem<N> &
     float2 h[NP];
 #pragma unroll
     for (int k = 0; k < NP; ++k) h[k] = f2(0.f, 0.f);
-    if (p.G > 1 && th.valid) load_pairs<NP>(p.hin + th.cbase * N + th.j0, h);
+    if (p.G > 1 && th.valid) {
+        if (p.hin_given) {   // the forward pass's checkpoints: [unit][N][Di], unit = cbase / Di
+            const float *row = p.hin + (th.cbase / p.Di) * N * p.Di + th.d;
+#pragma unroll
+            for (int k = 0; k < NP; ++k)
+                h[k] = f2(row[(size_t)(th.j0 + 2 * k) * p.Di], row[(size_t)(th.j0 + 2 * k + 1) * p.Di]);
+        } else {
+            load_pairs<NP>(p.hin + th.cbase * N + th.j0, h);
+        }
+    }
 #pragma unroll 1
     for (int sg = 0; sg < kBwdNSeg; ++sg) {
         store_ck<N>(sm, th.tid, sg, h);

@@ -78,9 +78,9 @@ template <typename T, int N, bool ZOH, bool U2 = false, bool DT = false, bool FR
 vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], float *dC_out[2], float *dA,
                       float *dD, float *dbias, float *tmp, cudaStream_t stream, cudaEvent_t *ev) {
     if (!rec(ev, 0, stream)) return VIM_ERR_CUDA;
-    if (a.G > 1) {
+    if (a.G > 1 && !a.hin_given) {
         // h entering each chunk: the forward scan's own summary kernels, each CTA walking
-        // kBwdCarrySpan consecutive chunks
+        // kBwdCarrySpan consecutive chunks (skipped when the forward pass left them)
         PairArgs fc = fwd;
         fc.carry_span = kBwdCarrySpan;
         const dim3 gf((a.Di + kDC - 1) / kDC, (a.G + kBwdCarrySpan - 1) / kBwdCarrySpan, a.batch);
@@ -101,6 +101,10 @@ vim_status launch_bwd(const BwdArgs &a, const PairArgs &fwd, float *dB_out[2], f
         const dim3 gc((unsigned)((units + 255) / 256));
         pair_combine<N><<<gc, 256, 0, stream>>>(fwd);
         if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;
+    }
+    if (a.G > 1) {
+        const int64_t units = (int64_t)a.batch * 2 * a.Di * N;
+        const dim3 gc((unsigned)((units + 255) / 256));
         // adjoint entering each chunk from the side its direction visits later
         adj_carry<T, N, DT><<<dim3((a.Di + kAdjCh - 1) / kAdjCh, a.G, a.batch), 2 * kAdjCh, 0, stream>>>(a);
         if (cudaGetLastError() != cudaSuccess) return VIM_ERR_CUDA;

@@ -298,7 +298,11 @@ struct PairArgs {
     int zoh;                        // exact zero-order-hold Bbar instead of Delta B
     int fold_reverse;               // pair_combine folds each direction against its order
     int carry_span;                 // consecutive chunks per pair_carry CTA (0 or 1: one)
+    float *hck;                     // or null: the state entering every kCkTokens-token segment,
+                                    // [batch][ceil(L/kCkTokens)][2][N][Di] fp32, in each direction's
+                                    // visiting order (the Vim scan without front or step input)
 };
+constexpr int kCkTokens = 32;       // tokens per checkpoint segment (the derivative's chunk)
 
 // position visited at step t of the forward direction
 __device__ __forceinline__ int position(const PairArgs &p, int t) {
@@ -1136,6 +1140,23 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
         const int twice = 2 * s - (nT - 1);
         float *ypart = (twice == 0 && dir == 1) ? ymid + dl : ybuf + (size_t)j * kTile * kDC + dl;
         if (!prm.valid) return;
+        if constexpr (!CONV && !DT && !PIN) {
+            // the state entering a checkpoint segment: chunks start at multiples of
+            // kCkTokens, so a segment is two tiles; the forward direction enters it at its
+            // even tile, the backward one at its odd tile (or the chunk's last tile).  In
+            // the scaled form the state is dprev g.
+            static_assert(kCkTokens == 2 * kTile, "a checkpoint segment is two tiles");
+            if (p.hck && (dir == 0 ? (j & 1) == 0 : ((j & 1) == 1 || j == nT - 1))) {
+                // state-major rows: a warp's 32 channels of one state are 128 contiguous bytes
+                const int seg = (t0 + j * kTile) / kCkTokens, nseg = (p.L + kCkTokens - 1) / kCkTokens;
+                float *o = p.hck + (((size_t)b * nseg + seg) * 2 + dir) * N * p.Di + d;
+#pragma unroll
+                for (int k = 0; k < NP; ++k) {
+                    o[(size_t)(2 * k) * p.Di] = h[k].x * dprev;
+                    o[(size_t)(2 * k + 1) * p.Di] = h[k].y * dprev;
+                }
+            }
+        }
         const T *su = S::uv(cur, dir, 0), *sd = S::uv(cur, dir, 1);
         const float *sB = S::bc(cur, dir, 0), *sC = S::bc(cur, dir, 1);
         const bool second = twice > 0;

@@ -46,12 +46,13 @@ size_t vim_scan_workspace_bytes(int which, int batch, int L_or_H, int W, int cha
 namespace {
 constexpr unsigned kKnownFlags = VIM_FLAG_ZOH_EXACT;
 
-// vim_scan_bidir with an optional convolution front (conv_w/conv_b non-null: u holds x)
+// vim_scan_bidir with an optional convolution front (conv_w/conv_b non-null: u holds x), and
+// optionally the states entering every checkpoint segment (ckpt, the scan without front)
 vim_status bidir_impl(const void *u, const float *conv_w, const float *conv_b, const void *delta,
                       const void *z, const void *B, const void *C, int64_t bc_dir_stride, const float *A,
                       const float *D, const float *delta_bias, void *y, int batch, int L, int d_inner,
                       int d_state, vim_dtype dt, unsigned flags, void *workspace, size_t workspace_bytes,
-                      cudaStream_t stream, cudaEvent_t *events) {
+                      cudaStream_t stream, cudaEvent_t *events, float *ckpt = nullptr) {
     vim_status st = check_common(batch, L, d_inner, d_state, dt);
     if (st != VIM_OK) return st;
     if (bc_dir_stride < 0 || (flags & ~kKnownFlags)) return VIM_ERR_INVALID_ARG;
@@ -67,6 +68,7 @@ vim_status bidir_impl(const void *u, const float *conv_w, const float *conv_b, c
     if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(D) |
          reinterpret_cast<uintptr_t>(delta_bias)) % 4)
         return VIM_ERR_INVALID_ARG;
+    if (ckpt && (conv_w || reinterpret_cast<uintptr_t>(ckpt) % 8)) return VIM_ERR_INVALID_ARG;
     const size_t need = summary_bytes(batch, L, d_inner, d_state);
     if (need > 0) {
         if (!workspace || workspace_bytes < need) return VIM_ERR_WORKSPACE;
@@ -86,6 +88,7 @@ vim_status bidir_impl(const void *u, const float *conv_w, const float *conv_b, c
     a.batch = batch; a.L = L; a.Di = d_inner; a.H = 1; a.W = L; a.order = 0;
     a.chunk = pl.chunk; a.G = pl.G;
     a.zoh = (flags & VIM_FLAG_ZOH_EXACT) ? 1 : 0;
+    a.hck = ckpt;
     if (pl.G > 1) {
         const size_t units = (size_t)batch * pl.G * 2 * d_inner;
         a.hloc = static_cast<float *>(workspace);
@@ -115,6 +118,21 @@ vim_status vim_scan_bidir_ex(const void *u, const float *conv_w, const float *co
                              size_t workspace_bytes, cudaStream_t stream, cudaEvent_t *events) {
     return bidir_impl(u, conv_w, conv_b, delta, z, B, C, bc_dir_stride, A, D, delta_bias, y, batch, L,
                       d_inner, d_state, dt, flags, workspace, workspace_bytes, stream, events);
+}
+
+size_t vim_scan_ckpt_bytes(int batch, int L, int d_inner, int d_state) {
+    if (batch <= 0 || L <= 0 || d_inner <= 0 || !supported_state(d_state)) return 0;
+    return (size_t)batch * ((L + kCkTokens - 1) / kCkTokens) * 2 * d_inner * d_state * sizeof(float);
+}
+
+vim_status vim_scan_bidir_ckpt(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                               int64_t bc_dir_stride, const float *A, const float *D, const float *delta_bias,
+                               void *y, float *ckpt, int batch, int L, int d_inner, int d_state, vim_dtype dt,
+                               unsigned flags, void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                               cudaEvent_t *events) {
+    if (batch > 0 && L > 0 && d_inner > 0 && !ckpt) return VIM_ERR_INVALID_ARG;
+    return bidir_impl(u, nullptr, nullptr, delta, z, B, C, bc_dir_stride, A, D, delta_bias, y, batch, L, d_inner,
+                      d_state, dt, flags, workspace, workspace_bytes, stream, events, ckpt);
 }
 
 vim_status vim_scan_bidir_conv_events(const void *x, const float *conv_w, const float *conv_b,

@@ -59,6 +59,16 @@ lib.vim_scan_bidir_bwd_events.restype = _i
 lib.vim_scan_bidir_bwd_ex.argtypes = (lib.vim_scan_bidir_bwd.argtypes[:23] + [ctypes.c_uint]
                                       + lib.vim_scan_bidir_bwd.argtypes[23:] + [_vp])
 lib.vim_scan_bidir_bwd_ex.restype = _i
+# the training pair: the forward scan keeping the derivative's chunk states, and the
+# derivative that takes them
+lib.vim_scan_bidir_ckpt.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp,
+                                    _i, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp]
+lib.vim_scan_bidir_ckpt.restype = _i
+lib.vim_scan_bidir_bwd_ckpt.argtypes = (lib.vim_scan_bidir_bwd_ex.argtypes[:9] + [_vp]
+                                        + lib.vim_scan_bidir_bwd_ex.argtypes[9:])
+lib.vim_scan_bidir_bwd_ckpt.restype = _i
+lib.vim_scan_ckpt_bytes.argtypes = [_i, _i, _i, _i]
+lib.vim_scan_ckpt_bytes.restype = _sz
 lib.vim_scan_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
 lib.vim_scan_bwd_workspace_bytes.restype = _sz
 lib.vim_block_scan.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
@@ -212,7 +222,7 @@ def _events(events):
 
 
 def _bidir(name, u, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, y, bc_dir_stride, workspace, stream,
-           events, zoh):
+           events, zoh, ckpt=None):
     batch, L, Di = u.shape
     N = B.shape[-1]
     dt = _dtype_code(u)
@@ -228,6 +238,15 @@ def _bidir(name, u, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, y, bc_dir_
         ("A", A, f32, (2, Di, N)), ("D", D, f32, (2, Di)), ("delta_bias", delta_bias, f32, (2, Di)),
         ("y", y, io, act)])
     ws, ws_bytes = _workspace(vim_scan_workspace_bytes(0, batch, L, 0, Di, N), workspace, u.device)
+    if ckpt is not None:
+        (pk,) = _ptrs(name, u, [("ckpt", ckpt, f32, ckpt_shape(batch, L, Di, N))])
+        st = lib.vim_scan_bidir_ckpt(pu, pdelta, pz, pB, pC, int(bc_dir_stride), pA, pD, pbias, py, pk, batch, L,
+                                     Di, N, dt, VIM_FLAG_ZOH_EXACT if zoh else 0,
+                                     None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream),
+                                     None if events is None else _events(events))
+        if st != VIM_OK:
+            raise VimScanError(st, name)
+        return y
     pre = (pu, pcw, pcb) if conv or zoh else (pu,)
     args = pre + (pdelta, pz, pB, pC, int(bc_dir_stride), pA, pD, pbias, py, batch, L, Di, N, dt)
     tail = (None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
@@ -244,17 +263,25 @@ def _bidir(name, u, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, y, bc_dir_
     return y
 
 
+def ckpt_shape(batch, L, d_inner, d_state):
+    """Shape of the checkpoints vim_scan_bidir(ckpt=...) writes and
+    vim_scan_bidir_bwd(ckpt=...) reads: [batch, ceil(L / 32), 2, d_state, d_inner]."""
+    return (batch, (L + 31) // 32, 2, d_state, d_inner)
+
+
 def vim_scan_bidir(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride=0,
-                   workspace=None, stream=None, events=None, zoh=False):
+                   workspace=None, stream=None, events=None, zoh=False, ckpt=None):
     """Vim bidirectional selective scan, (y^f + y^b) * silu(z); see include/vimscan.h.
 
     u, delta, z: [batch, L, d_inner]; B, C: [batch, L, d_state] (or a larger buffer
     whose backward copy starts ``bc_dir_stride`` elements in); A: [2, d_inner,
     d_state] fp32; D, delta_bias: [2, d_inner] fp32.  Returns y [batch, L, d_inner].
-    zoh=True takes the exact zero-order-hold Bbar (VIM_FLAG_ZOH_EXACT).
+    zoh=True takes the exact zero-order-hold Bbar (VIM_FLAG_ZOH_EXACT).  ``ckpt``, an
+    fp32 tensor of ckpt_shape(...), receives the states the derivative needs
+    (vim_scan_bidir_ckpt) for vim_scan_bidir_bwd(ckpt=...).
     """
     return _bidir("vim_scan_bidir", u, None, None, delta, z, B, C, A, D, delta_bias, y, bc_dir_stride,
-                  workspace, stream, events, zoh)
+                  workspace, stream, events, zoh, ckpt)
 
 
 def vim_scan_bidir_conv(x, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride=0,
@@ -274,7 +301,7 @@ def vim_scan_bwd_workspace_bytes(batch, L, d_inner, d_state, separate_bc):
 
 
 def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stride=0, workspace=None,
-                       stream=None, out=None, events=None, zoh=False):
+                       stream=None, out=None, events=None, zoh=False, ckpt=None):
     """Derivatives of vim_scan_bidir (first-order Bbar, or with ``zoh`` the exact
     zero-order hold) for a loss whose derivative with respect to y is ``dout``; see
     include/vimscan.h.
@@ -283,7 +310,9 @@ def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stri
     input dtype; dB and dC (fp32, shaped like B and C); dA [2, d_inner, d_state], dD
     and ddelta_bias [2, d_inner] (fp32).  ``out`` may hold those tensors from an
     earlier call to be written again; ``events`` 4 CUDA events (see
-    vim_scan_bidir_bwd_events).
+    vim_scan_bidir_bwd_events).  ``ckpt``: the checkpoints vim_scan_bidir(ckpt=...) wrote
+    for the same inputs (vim_scan_bidir_bwd_ckpt), which replace the derivative's own
+    forward summaries.
     """
     batch, L, Di = u.shape
     N = B.shape[-1]
@@ -308,6 +337,15 @@ def vim_scan_bidir_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stri
         ("A", A, f32, (2, Di, N)), ("D", D, f32, (2, Di)), ("delta_bias", delta_bias, f32, (2, Di)),
         ("dout", dout, io, act)] + _out_specs(out, io, act, bc, (2, Di, N), (2, Di)))
     ws, ws_bytes = _workspace(vim_scan_bwd_workspace_bytes(batch, L, Di, N, bc_dir_stride > 0), workspace, dev)
+    if ckpt is not None:
+        (pk,) = _ptrs("vim_scan_bidir_bwd", u, [("ckpt", ckpt, f32, ckpt_shape(batch, L, Di, N))])
+        st = lib.vim_scan_bidir_bwd_ckpt(
+            *ptrs[:5], int(bc_dir_stride), *ptrs[5:8], pk, *ptrs[8:], batch, L, Di, N, dt,
+            VIM_FLAG_ZOH_EXACT if zoh else 0, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream),
+            None if events is None else _events(events))
+        if st != VIM_OK:
+            raise VimScanError(st, "vim_scan_bidir_bwd")
+        return out
     if zoh:
         fn = lib.vim_scan_bidir_bwd_ex
         flags, extra = (VIM_FLAG_ZOH_EXACT,), (None if events is None else _events(events),)
