@@ -454,8 +454,8 @@ def main():
         raise SystemExit("--block runs alone (or with --bwd), on a bf16 workload")
     if args.bwd and args.conv and w.kind != "vim":
         raise SystemExit("--bwd --conv applies to the Vim workloads only")
-    if args.ckpt and (w.kind != "vim" or args.conv or args.block):
-        raise SystemExit("--ckpt applies to the Vim scan without front or projections")
+    if args.ckpt and (w.kind != "vim" or args.block):
+        raise SystemExit("--ckpt applies to the Vim scan (with or without its front), not the block")
     if args.impl == "reference":
         reference_arm(args, w)
         return
@@ -547,7 +547,7 @@ def main():
             # u holds x; the derivative through the pathways' convolution fronts
             vs.vim_scan_bidir_conv_bwd(s["u"], params["conv_w"], params["conv_b"], s["delta"], s["z"], s["B"], s["C"],
                                        params["A"], params["D"], params["delta_bias"], s["dout"], workspace=ws,
-                                       out=s["out"], zoh=args.zoh)
+                                       out=s["out"], zoh=args.zoh, ckpt=s["ck"] if args.ckpt else None)
             return
         if args.bwd and w.kind == "vim":
             vs.vim_scan_bidir_bwd(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"],
@@ -562,7 +562,8 @@ def main():
             # u holds x, the pathways' common input in front of the convolutions
             vs.vim_scan_bidir_conv(s["u"], params["conv_w"], params["conv_b"], s["delta"], s["z"], s["B"],
                                    s["C"], params["A"], params["D"], params["delta_bias"], y=s["y"],
-                                   workspace=ws, events=events, zoh=args.zoh)
+                                   workspace=fws if args.ckpt else ws, events=events, zoh=args.zoh,
+                                   ckpt=s["ck"] if args.ckpt else None)
             return
         if args.ckpt:
             fn(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"], params["delta_bias"],
@@ -578,8 +579,13 @@ def main():
                           dtype=torch.uint8, device=dev)
         if args.bwd:
             for s in sets:
-                fn(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"], params["delta_bias"],
-                   y=s["y"], workspace=fws, zoh=args.zoh, ckpt=s["ck"])
+                if args.conv:
+                    vs.vim_scan_bidir_conv(s["u"], params["conv_w"], params["conv_b"], s["delta"], s["z"], s["B"],
+                                           s["C"], params["A"], params["D"], params["delta_bias"], y=s["y"],
+                                           workspace=fws, zoh=args.zoh, ckpt=s["ck"])
+                else:
+                    fn(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"], params["delta_bias"],
+                       y=s["y"], workspace=fws, zoh=args.zoh, ckpt=s["ck"])
             torch.cuda.synchronize()
 
     barrier = replicas.barrier
@@ -646,7 +652,7 @@ def main():
             # the fronts' forward kernel, pair_carry, pair_combine, adj_carry, pair_combine,
             # bwd_main, two dB/dC reductions, two column sums for the parameters, the
             # fronts' derivative and two column sums for their taps and biases
-            launches_per_step = 1 + (4 if w.tokens > 32 else 0) + 1 + 2 + 2 + 1 + 2
+            launches_per_step = 1 + ((2 if args.ckpt else 4) if w.tokens > 32 else 0) + 1 + 2 + 2 + 1 + 2
         else:
             per_kernel["vmamba_cross_scan4_bwd"] = sum(t) / len(t)
             # per pair: pair_carry, pair_combine, adj_carry, pair_combine, bwd_main, four

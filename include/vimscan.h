@@ -513,7 +513,11 @@ size_t vim_scan_host_workspace_bytes(int batch, int L, int d_inner, int d_state,
  *   delta_bias and flags.  The results equal vim_scan_bidir_bwd_ex's up to rounding (the
  *   states come from the forward kernels' arithmetic instead of the derivative's
  *   summaries).  Checkpoints from other inputs give a wrong derivative, not an error.
- * Both return VIM_ERR_INVALID_ARG for a NULL or misaligned ckpt on a non-empty problem.
+ * vim_scan_bidir_conv_ckpt / vim_scan_bidir_conv_bwd_ckpt: the same pair for the scan with
+ *   the pathways' convolution front (the arguments of vim_scan_bidir_conv / _ex and of
+ *   vim_scan_bidir_conv_bwd_ex, with ckpt as above: the states of the recurrence on each
+ *   pathway's u_k = silu(conv_k(x))).
+ * All return VIM_ERR_INVALID_ARG for a NULL or misaligned ckpt on a non-empty problem.
  */
 vim_status vim_scan_bidir_ckpt(const void *u, const void *delta, const void *z, const void *B, const void *C,
                                int64_t bc_dir_stride, const float *A, const float *D, const float *delta_bias,
@@ -526,6 +530,19 @@ vim_status vim_scan_bidir_bwd_ckpt(const void *u, const void *delta, const void 
                                    float *dC, float *dA, float *dD, float *ddelta_bias, int batch, int L,
                                    int d_inner, int d_state, vim_dtype dt, unsigned flags, void *workspace,
                                    size_t workspace_bytes, cudaStream_t stream, cudaEvent_t *events);
+vim_status vim_scan_bidir_conv_ckpt(const void *x, const float *conv_w, const float *conv_b, const void *delta,
+                                    const void *z, const void *B, const void *C, int64_t bc_dir_stride,
+                                    const float *A, const float *D, const float *delta_bias, void *y, float *ckpt,
+                                    int batch, int L, int d_inner, int d_state, vim_dtype dt, unsigned flags,
+                                    void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                                    cudaEvent_t *events);
+vim_status vim_scan_bidir_conv_bwd_ckpt(const void *x, const float *conv_w, const float *conv_b, const void *delta,
+                                        const void *z, const void *B, const void *C, int64_t bc_dir_stride,
+                                        const float *A, const float *D, const float *delta_bias, const float *ckpt,
+                                        const void *dout, void *dx, float *dconv_w, float *dconv_b, void *ddelta,
+                                        void *dz, float *dB, float *dC, float *dA, float *dD, float *ddelta_bias,
+                                        int batch, int L, int d_inner, int d_state, vim_dtype dt, unsigned flags,
+                                        void *workspace, size_t workspace_bytes, cudaStream_t stream);
 /* Bytes of the checkpoints (0 for invalid arguments or an empty problem). */
 size_t vim_scan_ckpt_bytes(int batch, int L, int d_inner, int d_state);
 

@@ -45,6 +45,7 @@ def test_header_declares_the_boundary():
                           "vim_scan_bidir_conv_bwd", "vim_scan_bidir_conv_bwd_ex", "vim_scan_conv_bwd_workspace_bytes",
                           "vim_block_scan_bwd", "vim_block_bwd_workspace_bytes",
                           "vim_scan_bidir_ckpt", "vim_scan_bidir_bwd_ckpt", "vim_scan_ckpt_bytes",
+                          "vim_scan_bidir_conv_ckpt", "vim_scan_bidir_conv_bwd_ckpt",
                           "vim_scan_workspace_bytes", "vim_status_string"}, names
 
 
@@ -280,6 +281,22 @@ def test_ckpt_pair_rejects(vs):
     assert vs.lib.vim_scan_ckpt_bytes(0, 100, 64, 16) == 0
     assert vs.lib.vim_scan_ckpt_bytes(2, 100, 64, 3) == 0
     assert vs.ckpt_shape(2, 100, 64, 16) == (2, 4, 2, 16, 64)
+
+
+def test_conv_ckpt_pair_rejects(vs):
+    lib, F = vs.lib, FAKE
+    fwd = lambda ckpt=F, cw=F, ws=F: lib.vim_scan_bidir_conv_ckpt(F, cw, F, F, F, F, F, 0, F, F, F, F, ckpt, 2, 100,
+                                                                   64, 16, vs.VIM_BF16, 0, ws, 1 << 40, None, None)
+    assert fwd(ckpt=None) == vs.VIM_ERR_INVALID_ARG
+    assert fwd(cw=None) == vs.VIM_ERR_INVALID_ARG          # the front is required
+    assert fwd(ckpt=F + 4) == vs.VIM_ERR_INVALID_ARG
+    assert fwd(ws=None) == vs.VIM_ERR_WORKSPACE
+    bwd = lambda ckpt=F, ws=F: lib.vim_scan_bidir_conv_bwd_ckpt(F, F, F, F, F, F, F, 0, F, F, F, ckpt, F, F, F, F, F,
+                                                                F, F, F, F, F, F, 2, 100, 64, 16, vs.VIM_BF16, 0,
+                                                                ws, 1 << 40, None)
+    assert bwd(ckpt=None) == vs.VIM_ERR_INVALID_ARG
+    assert bwd(ckpt=F + 4) == vs.VIM_ERR_INVALID_ARG
+    assert bwd(ws=None) == vs.VIM_ERR_WORKSPACE
 
 
 def test_bwd_ex_rejects(vs):

@@ -498,3 +498,33 @@ def test_ckpt_pair_full_size(vs):
                    elementwise=False)
     want = oracle.vim_bidir_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["bias"], x["dout"])
     check_all("bwd_ckpt_full", got, want, torch.bfloat16, sum_tol=SUM_TOL_FULL)
+
+
+# the training pair with the convolution front
+CONV_CKPT_CASES = [
+    # batch, L, Di, N, dtype, gate, zoh
+    (1, 5, 16, 4, torch.float32, True, False),
+    (2, 100, 40, 8, torch.float32, False, False),   # the forward's 32-token chunks
+    (1, 300, 72, 16, torch.bfloat16, True, False),  # 96-token chunks, a ragged last one
+    (1, 333, 64, 16, torch.float32, True, True),     # exact hold
+]
+
+
+@pytest.mark.parametrize("case", CONV_CKPT_CASES, ids=lambda c: f"b{c[0]}_L{c[1]}_D{c[2]}_N{c[3]}_"
+                         f"{str(c[4])[6:]}{'' if c[5] else '_nogate'}{'_zoh' if c[6] else ''}")
+def test_conv_ckpt_pair(vs, case):
+    batch, L, Di, N, dtype, gate, zoh = case
+    x = conv_inputs(batch, L, Di, N, dtype, seed=L * 13 + Di)
+    c = lambda k: x[k].cuda()
+    ck = torch.full(vs.ckpt_shape(batch, L, Di, N), float("nan"), device="cuda")
+    zz = c("z") if gate else None
+    y = vs.vim_scan_bidir_conv(c("x"), c("conv_w"), c("conv_b"), c("delta"), zz, c("B"), c("C"), c("A"), c("D"),
+                               c("bias"), zoh=zoh, ckpt=ck)
+    y_plain = vs.vim_scan_bidir_conv(c("x"), c("conv_w"), c("conv_b"), c("delta"), zz, c("B"), c("C"), c("A"),
+                                     c("D"), c("bias"), zoh=zoh)
+    got = vs.vim_scan_bidir_conv_bwd(c("x"), c("conv_w"), c("conv_b"), c("delta"), zz, c("B"), c("C"), c("A"),
+                                     c("D"), c("bias"), c("dout"), zoh=zoh, ckpt=ck)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_plain)
+    assert torch.isfinite(ck).all() and (ck[:, 0, 0] == 0).all() and (ck[:, -1, 1] == 0).all()
+    check_conv(f"conv_bwd_ckpt_{case}", got, ref_conv(x, gate, zoh), dtype)

@@ -165,13 +165,18 @@ size_t vim_scan_conv_bwd_workspace_bytes(int batch, int L, int d_inner, int d_st
     return conv_bwd_plan(batch, L, d_inner, d_state, dt, separate_bc).total;
 }
 
-vim_status vim_scan_bidir_conv_bwd_ex(const void *x, const float *conv_w, const float *conv_b, const void *delta,
-                                      const void *z, const void *B, const void *C, int64_t bc_dir_stride,
-                                      const float *A, const float *D, const float *delta_bias, const void *dout,
-                                      void *dx, float *dconv_w, float *dconv_b, void *ddelta, void *dz, float *dB,
-                                      float *dC, float *dA, float *dD, float *ddelta_bias, int batch, int L,
-                                      int d_inner, int d_state, vim_dtype dt, unsigned flags, void *workspace,
-                                      size_t workspace_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// the derivative of vim_scan_bidir_conv; ckpt, or null: the forward pass's checkpoints
+// (vim_scan_bidir_conv_ckpt), which replace the derivative's own forward summaries
+vim_status conv_bwd_impl(const void *x, const float *conv_w, const float *conv_b, const void *delta, const void *z,
+                         const void *B, const void *C, int64_t bc_dir_stride, const float *A, const float *D,
+                         const float *delta_bias, const void *dout, void *dx, float *dconv_w, float *dconv_b,
+                         void *ddelta, void *dz, float *dB, float *dC, float *dA, float *dD, float *ddelta_bias,
+                         int batch, int L, int d_inner, int d_state, vim_dtype dt, unsigned flags, void *workspace,
+                         size_t workspace_bytes, cudaStream_t stream, const float *ckpt) {
     if (flags & ~VIM_FLAG_ZOH_EXACT) return VIM_ERR_INVALID_ARG;
     const bool zoh = (flags & VIM_FLAG_ZOH_EXACT) != 0;
     vim_status st = check_common(batch, L, d_inner, d_state, dt);
@@ -232,7 +237,8 @@ vim_status vim_scan_bidir_conv_bwd_ex(const void *x, const float *conv_w, const 
     a.dB_part[1] = separate ? a.dB_part[0] + set_elems : a.dB_part[0];
     a.dC_part[1] = separate ? a.dC_part[0] + set_elems : a.dC_part[0];
     a.par = reinterpret_cast<float *>(ws + pl.off_par);
-    a.hin = reinterpret_cast<const float *>(ws + pl.off_hloc);
+    a.hin = ckpt ? ckpt : reinterpret_cast<const float *>(ws + pl.off_hloc);
+    a.hin_given = ckpt ? 1 : 0;
     a.gloc = reinterpret_cast<float *>(ws + pl.off_gloc);
     a.gsum = reinterpret_cast<float *>(ws + pl.off_gsum);
     a.batch = batch; a.L = L; a.Di = d_inner; a.G = pl.G; a.nblk = pl.nblk; a.cl = pl.cl; a.ncol = pl.ncol;
@@ -267,6 +273,35 @@ vim_status vim_scan_bidir_conv_bwd_ex(const void *x, const float *conv_w, const 
     return launch_fronts_bwd<__nv_bfloat16>(static_cast<const __nv_bfloat16 *>(x), conv_w, conv_b, du2,
                                             static_cast<__nv_bfloat16 *>(dx), part, ptmp, dconv_w, dconv_b, batch, L,
                                             d_inner, cp.runs, vec, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+vim_status vim_scan_bidir_conv_bwd_ex(const void *x, const float *conv_w, const float *conv_b, const void *delta,
+                                      const void *z, const void *B, const void *C, int64_t bc_dir_stride,
+                                      const float *A, const float *D, const float *delta_bias, const void *dout,
+                                      void *dx, float *dconv_w, float *dconv_b, void *ddelta, void *dz, float *dB,
+                                      float *dC, float *dA, float *dD, float *ddelta_bias, int batch, int L,
+                                      int d_inner, int d_state, vim_dtype dt, unsigned flags, void *workspace,
+                                      size_t workspace_bytes, cudaStream_t stream) {
+    return conv_bwd_impl(x, conv_w, conv_b, delta, z, B, C, bc_dir_stride, A, D, delta_bias, dout, dx, dconv_w,
+                         dconv_b, ddelta, dz, dB, dC, dA, dD, ddelta_bias, batch, L, d_inner, d_state, dt, flags,
+                         workspace, workspace_bytes, stream, nullptr);
+}
+
+vim_status vim_scan_bidir_conv_bwd_ckpt(const void *x, const float *conv_w, const float *conv_b, const void *delta,
+                                        const void *z, const void *B, const void *C, int64_t bc_dir_stride,
+                                        const float *A, const float *D, const float *delta_bias, const float *ckpt,
+                                        const void *dout, void *dx, float *dconv_w, float *dconv_b, void *ddelta,
+                                        void *dz, float *dB, float *dC, float *dA, float *dD, float *ddelta_bias,
+                                        int batch, int L, int d_inner, int d_state, vim_dtype dt, unsigned flags,
+                                        void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (batch > 0 && L > 0 && d_inner > 0 && (!ckpt || !aligned_to(ckpt, 8))) return VIM_ERR_INVALID_ARG;
+    return conv_bwd_impl(x, conv_w, conv_b, delta, z, B, C, bc_dir_stride, A, D, delta_bias, dout, dx, dconv_w,
+                         dconv_b, ddelta, dz, dB, dC, dA, dD, ddelta_bias, batch, L, d_inner, d_state, dt, flags,
+                         workspace, workspace_bytes, stream, ckpt);
 }
 
 vim_status vim_scan_bidir_conv_bwd(const void *x, const float *conv_w, const float *conv_b, const void *delta,

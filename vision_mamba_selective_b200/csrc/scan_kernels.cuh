@@ -300,7 +300,7 @@ struct PairArgs {
     int carry_span;                 // consecutive chunks per pair_carry CTA (0 or 1: one)
     float *hck;                     // or null: the state entering every kCkTokens-token segment,
                                     // [batch][ceil(L/kCkTokens)][2][N][Di] fp32, in each direction's
-                                    // visiting order (the Vim scan without front or step input)
+                                    // visiting order (the Vim scan, with or without its front)
 };
 constexpr int kCkTokens = 32;       // tokens per checkpoint segment (the derivative's chunk)
 
@@ -1140,7 +1140,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
         const int twice = 2 * s - (nT - 1);
         float *ypart = (twice == 0 && dir == 1) ? ymid + dl : ybuf + (size_t)j * kTile * kDC + dl;
         if (!prm.valid) return;
-        if constexpr (!CONV && !DT && !PIN) {
+        if constexpr (!DT && !PIN) {
             // the state entering a checkpoint segment: chunks start at multiples of
             // kCkTokens, so a segment is two tiles; the forward direction enters it at its
             // even tile, the backward one at its odd tile (or the chunk's last tile).  In

@@ -47,7 +47,7 @@ namespace {
 constexpr unsigned kKnownFlags = VIM_FLAG_ZOH_EXACT;
 
 // vim_scan_bidir with an optional convolution front (conv_w/conv_b non-null: u holds x), and
-// optionally the states entering every checkpoint segment (ckpt, the scan without front)
+// optionally the states entering every checkpoint segment (ckpt)
 vim_status bidir_impl(const void *u, const float *conv_w, const float *conv_b, const void *delta,
                       const void *z, const void *B, const void *C, int64_t bc_dir_stride, const float *A,
                       const float *D, const float *delta_bias, void *y, int batch, int L, int d_inner,
@@ -68,7 +68,7 @@ vim_status bidir_impl(const void *u, const float *conv_w, const float *conv_b, c
     if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(D) |
          reinterpret_cast<uintptr_t>(delta_bias)) % 4)
         return VIM_ERR_INVALID_ARG;
-    if (ckpt && (conv_w || reinterpret_cast<uintptr_t>(ckpt) % 8)) return VIM_ERR_INVALID_ARG;
+    if (ckpt && reinterpret_cast<uintptr_t>(ckpt) % 8) return VIM_ERR_INVALID_ARG;
     const size_t need = summary_bytes(batch, L, d_inner, d_state);
     if (need > 0) {
         if (!workspace || workspace_bytes < need) return VIM_ERR_WORKSPACE;
@@ -132,6 +132,17 @@ vim_status vim_scan_bidir_ckpt(const void *u, const void *delta, const void *z, 
                                cudaEvent_t *events) {
     if (batch > 0 && L > 0 && d_inner > 0 && !ckpt) return VIM_ERR_INVALID_ARG;
     return bidir_impl(u, nullptr, nullptr, delta, z, B, C, bc_dir_stride, A, D, delta_bias, y, batch, L, d_inner,
+                      d_state, dt, flags, workspace, workspace_bytes, stream, events, ckpt);
+}
+
+vim_status vim_scan_bidir_conv_ckpt(const void *x, const float *conv_w, const float *conv_b, const void *delta,
+                                    const void *z, const void *B, const void *C, int64_t bc_dir_stride,
+                                    const float *A, const float *D, const float *delta_bias, void *y, float *ckpt,
+                                    int batch, int L, int d_inner, int d_state, vim_dtype dt, unsigned flags,
+                                    void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                                    cudaEvent_t *events) {
+    if (batch > 0 && L > 0 && d_inner > 0 && (!ckpt || !conv_w || !conv_b)) return VIM_ERR_INVALID_ARG;
+    return bidir_impl(x, conv_w, conv_b, delta, z, B, C, bc_dir_stride, A, D, delta_bias, y, batch, L, d_inner,
                       d_state, dt, flags, workspace, workspace_bytes, stream, events, ckpt);
 }
 

@@ -93,6 +93,13 @@ lib.vim_scan_bidir_conv_bwd_ex.restype = _i
 lib.vim_scan_bidir_conv_bwd.argtypes = (lib.vim_scan_bidir_conv_bwd_ex.argtypes[:27]
                                         + lib.vim_scan_bidir_conv_bwd_ex.argtypes[28:])
 lib.vim_scan_bidir_conv_bwd.restype = _i
+# the training pair with the convolution front
+lib.vim_scan_bidir_conv_ckpt.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp,
+                                         _i, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp]
+lib.vim_scan_bidir_conv_ckpt.restype = _i
+lib.vim_scan_bidir_conv_bwd_ckpt.argtypes = (lib.vim_scan_bidir_conv_bwd_ex.argtypes[:11] + [_vp]
+                                             + lib.vim_scan_bidir_conv_bwd_ex.argtypes[11:])
+lib.vim_scan_bidir_conv_bwd_ckpt.restype = _i
 lib.vim_scan_conv_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
 lib.vim_scan_conv_bwd_workspace_bytes.restype = _sz
 lib.vim_block_scan_bwd.argtypes = [_vp] * 19 + [_i, _i, _i, _i, _i, _vp, _sz, _vp]
@@ -240,10 +247,13 @@ def _bidir(name, u, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, y, bc_dir_
     ws, ws_bytes = _workspace(vim_scan_workspace_bytes(0, batch, L, 0, Di, N), workspace, u.device)
     if ckpt is not None:
         (pk,) = _ptrs(name, u, [("ckpt", ckpt, f32, ckpt_shape(batch, L, Di, N))])
-        st = lib.vim_scan_bidir_ckpt(pu, pdelta, pz, pB, pC, int(bc_dir_stride), pA, pD, pbias, py, pk, batch, L,
-                                     Di, N, dt, VIM_FLAG_ZOH_EXACT if zoh else 0,
-                                     None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream),
-                                     None if events is None else _events(events))
+        tail = (batch, L, Di, N, dt, VIM_FLAG_ZOH_EXACT if zoh else 0, None if ws is None else ws.data_ptr(),
+                ws_bytes, _stream(stream), None if events is None else _events(events))
+        if conv:
+            st = lib.vim_scan_bidir_conv_ckpt(pu, pcw, pcb, pdelta, pz, pB, pC, int(bc_dir_stride), pA, pD, pbias,
+                                              py, pk, *tail)
+        else:
+            st = lib.vim_scan_bidir_ckpt(pu, pdelta, pz, pB, pC, int(bc_dir_stride), pA, pD, pbias, py, pk, *tail)
         if st != VIM_OK:
             raise VimScanError(st, name)
         return y
@@ -285,15 +295,16 @@ def vim_scan_bidir(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride
 
 
 def vim_scan_bidir_conv(x, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, *, y=None, bc_dir_stride=0,
-                        workspace=None, stream=None, events=None, zoh=False):
+                        workspace=None, stream=None, events=None, zoh=False, ckpt=None):
     """vim_scan_bidir with the pathways' kernel-3 convolution + SiLU front fused in.
 
     x, delta, z: [batch, L, d_inner]; conv_w: [2, d_inner, 3] fp32; conv_b: [2, d_inner]
     fp32; the rest as in vim_scan_bidir.  Returns y [batch, L, d_inner].  A missing
-    half of the front (conv_w or conv_b None) is rejected by the library.
+    half of the front (conv_w or conv_b None) is rejected by the library.  ``ckpt`` as in
+    vim_scan_bidir (vim_scan_bidir_conv_ckpt), for vim_scan_bidir_conv_bwd(ckpt=...).
     """
     return _bidir("vim_scan_bidir_conv", x, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, y,
-                  bc_dir_stride, workspace, stream, events, zoh)
+                  bc_dir_stride, workspace, stream, events, zoh, ckpt)
 
 
 def vim_scan_bwd_workspace_bytes(batch, L, d_inner, d_state, separate_bc):
@@ -365,7 +376,7 @@ def vim_scan_conv_bwd_workspace_bytes(batch, L, d_inner, d_state, dtype_code, se
 
 
 def vim_scan_bidir_conv_bwd(x, conv_w, conv_b, delta, z, B, C, A, D, delta_bias, dout, *, bc_dir_stride=0,
-                            workspace=None, stream=None, out=None, zoh=False):
+                            workspace=None, stream=None, out=None, zoh=False, ckpt=None):
     """Derivatives of vim_scan_bidir_conv (first-order Bbar, or with ``zoh`` the exact
     hold) for a loss whose derivative with respect to y is ``dout``; see
     include/vimscan.h.
@@ -373,7 +384,9 @@ def vim_scan_bidir_conv_bwd(x, conv_w, conv_b, delta, z, B, C, A, D, delta_bias,
     Returns a dict: dx, ddelta (w.r.t. the raw delta), dz (None without z) in the input
     dtype; dconv_w [2, d_inner, 3] and dconv_b [2, d_inner] fp32; dB, dC (fp32, shaped
     like B and C), dA [2, d_inner, d_state], dD and ddelta_bias [2, d_inner] fp32.
-    ``out`` may hold those tensors from an earlier call to be written again.
+    ``out`` may hold those tensors from an earlier call to be written again.  ``ckpt``: the
+    checkpoints vim_scan_bidir_conv(ckpt=...) wrote for the same inputs
+    (vim_scan_bidir_conv_bwd_ckpt).
     """
     batch, L, Di = x.shape
     N = B.shape[-1]
@@ -405,9 +418,15 @@ def vim_scan_bidir_conv_bwd(x, conv_w, conv_b, delta, z, B, C, A, D, delta_bias,
     ptrs = _ptrs("vim_scan_bidir_conv_bwd", x, specs)
     ws, ws_bytes = _workspace(vim_scan_conv_bwd_workspace_bytes(batch, L, Di, N, dt, bc_dir_stride > 0), workspace,
                               dev)
-    st = lib.vim_scan_bidir_conv_bwd_ex(
-        *ptrs[:7], int(bc_dir_stride), *ptrs[7:], batch, L, Di, N, dt, VIM_FLAG_ZOH_EXACT if zoh else 0,
-        None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
+    if ckpt is not None:
+        (pk,) = _ptrs("vim_scan_bidir_conv_bwd", x, [("ckpt", ckpt, f32, ckpt_shape(batch, L, Di, N))])
+        st = lib.vim_scan_bidir_conv_bwd_ckpt(
+            *ptrs[:7], int(bc_dir_stride), *ptrs[7:10], pk, *ptrs[10:], batch, L, Di, N, dt,
+            VIM_FLAG_ZOH_EXACT if zoh else 0, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
+    else:
+        st = lib.vim_scan_bidir_conv_bwd_ex(
+            *ptrs[:7], int(bc_dir_stride), *ptrs[7:], batch, L, Di, N, dt, VIM_FLAG_ZOH_EXACT if zoh else 0,
+            None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
     if st != VIM_OK:
         raise VimScanError(st, "vim_scan_bidir_conv_bwd")
     return out
