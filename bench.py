@@ -431,10 +431,12 @@ def cpu_model():
 
 
 def vs_ckpt_shape(w):
-    """Shape of the forward pass's checkpoints for a Vim workload."""
+    """Shape of the forward pass's checkpoints for a workload."""
     from vision_mamba_selective_b200 import vimscan as vs
 
-    return vs.ckpt_shape(w.batch, w.L, w.channels, w.d_state)
+    if w.kind == "vim":
+        return vs.ckpt_shape(w.batch, w.L, w.channels, w.d_state)
+    return vs.cross_ckpt_shape(w.batch, w.H, w.W, w.channels, w.d_state)
 
 
 def workload_name(w, args):
@@ -454,8 +456,8 @@ def main():
         raise SystemExit("--block runs alone (or with --bwd), on a bf16 workload")
     if args.bwd and args.conv and w.kind != "vim":
         raise SystemExit("--bwd --conv applies to the Vim workloads only")
-    if args.ckpt and (w.kind != "vim" or args.block):
-        raise SystemExit("--ckpt applies to the Vim scan (with or without its front), not the block")
+    if args.ckpt and args.block:
+        raise SystemExit("--ckpt applies to the scans (Vim with or without its front, the cross-scan), not the block")
     if args.impl == "reference":
         reference_arm(args, w)
         return
@@ -556,7 +558,8 @@ def main():
             return
         if args.bwd:
             vs.vmamba_cross_scan4_bwd(s["u"], s["delta"], s["z"], s["B"], s["C"], params["A"], params["D"],
-                                      params["delta_bias"], s["dout"], workspace=ws, out=s["out"], zoh=args.zoh)
+                                      params["delta_bias"], s["dout"], workspace=ws, out=s["out"], zoh=args.zoh,
+                                      ckpt=s["ck"] if args.ckpt else None)
             return
         if args.conv:
             # u holds x, the pathways' common input in front of the convolutions
@@ -575,8 +578,9 @@ def main():
     if args.ckpt:
         # the forward scan's workspace, and with --bwd the states each input set's forward
         # pass leaves (inputs of the derivative, formed before any timing)
-        fws = torch.empty(max(vs.vim_scan_workspace_bytes(0, w.batch, w.L, 0, w.channels, w.d_state), 1),
-                          dtype=torch.uint8, device=dev)
+        fws_bytes = (vs.vim_scan_workspace_bytes(0, w.batch, w.L, 0, w.channels, w.d_state) if w.kind == "vim"
+                     else vs.vim_scan_workspace_bytes(1, w.batch, w.H, w.W, w.channels, w.d_state))
+        fws = torch.empty(max(fws_bytes, 1), dtype=torch.uint8, device=dev)
         if args.bwd:
             for s in sets:
                 if args.conv:
@@ -657,7 +661,7 @@ def main():
             per_kernel["vmamba_cross_scan4_bwd"] = sum(t) / len(t)
             # per pair: pair_carry, pair_combine, adj_carry, pair_combine, bwd_main, four
             # dB/dC reductions, one two-pass column sum
-            launches_per_step = 2 * ((4 if w.tokens > 32 else 0) + 1 + 4 + 2)
+            launches_per_step = 2 * (((2 if args.ckpt else 4) if w.tokens > 32 else 0) + 1 + 4 + 2)
     elif args.bwd:
         for a, name in enumerate(["summaries", "bwd_main", "reductions"], start=1):
             t = [evs[i][a - 1].elapsed_time(evs[i][a]) for i in range(prof_steps)]

@@ -517,6 +517,10 @@ size_t vim_scan_host_workspace_bytes(int batch, int L, int d_inner, int d_state,
  *   the pathways' convolution front (the arguments of vim_scan_bidir_conv / _ex and of
  *   vim_scan_bidir_conv_bwd_ex, with ckpt as above: the states of the recurrence on each
  *   pathway's u_k = silu(conv_k(x))).
+ * vmamba_cross_scan4_ckpt / vmamba_cross_scan4_bwd_ckpt: the pair for the cross-scan (the
+ *   arguments of vmamba_cross_scan4_ex and vmamba_cross_scan4_bwd_ex), ckpt fp32
+ *   [2][batch][ceil(H W / 32)][2][d_state][channels], vmamba_cross_ckpt_bytes bytes: per pair
+ *   of scans (rows, then columns) the states above over that pair's steps.
  * All return VIM_ERR_INVALID_ARG for a NULL or misaligned ckpt on a non-empty problem.
  */
 vim_status vim_scan_bidir_ckpt(const void *u, const void *delta, const void *z, const void *B, const void *C,
@@ -543,8 +547,20 @@ vim_status vim_scan_bidir_conv_bwd_ckpt(const void *x, const float *conv_w, cons
                                         void *dz, float *dB, float *dC, float *dA, float *dD, float *ddelta_bias,
                                         int batch, int L, int d_inner, int d_state, vim_dtype dt, unsigned flags,
                                         void *workspace, size_t workspace_bytes, cudaStream_t stream);
+vim_status vmamba_cross_scan4_ckpt(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                                   const float *A, const float *D, const float *delta_bias, void *y, float *ckpt,
+                                   int batch, int H, int W, int channels, int d_state, vim_dtype dt, unsigned flags,
+                                   void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                                   cudaEvent_t *events);
+vim_status vmamba_cross_scan4_bwd_ckpt(const void *u, const void *delta, const void *z, const void *B,
+                                       const void *C, const float *A, const float *D, const float *delta_bias,
+                                       const float *ckpt, const void *dout, void *du, void *ddelta, void *dz,
+                                       float *dB, float *dC, float *dA, float *dD, float *ddelta_bias, int batch,
+                                       int H, int W, int channels, int d_state, vim_dtype dt, unsigned flags,
+                                       void *workspace, size_t workspace_bytes, cudaStream_t stream);
 /* Bytes of the checkpoints (0 for invalid arguments or an empty problem). */
 size_t vim_scan_ckpt_bytes(int batch, int L, int d_inner, int d_state);
+size_t vmamba_cross_ckpt_bytes(int batch, int H, int W, int channels, int d_state);
 
 /*
  * Workspace bytes the scan entry points need (0 when none).  which = 0 for

@@ -46,6 +46,7 @@ def test_header_declares_the_boundary():
                           "vim_block_scan_bwd", "vim_block_bwd_workspace_bytes",
                           "vim_scan_bidir_ckpt", "vim_scan_bidir_bwd_ckpt", "vim_scan_ckpt_bytes",
                           "vim_scan_bidir_conv_ckpt", "vim_scan_bidir_conv_bwd_ckpt",
+                          "vmamba_cross_scan4_ckpt", "vmamba_cross_scan4_bwd_ckpt", "vmamba_cross_ckpt_bytes",
                           "vim_scan_workspace_bytes", "vim_status_string"}, names
 
 
@@ -297,6 +298,23 @@ def test_conv_ckpt_pair_rejects(vs):
     assert bwd(ckpt=None) == vs.VIM_ERR_INVALID_ARG
     assert bwd(ckpt=F + 4) == vs.VIM_ERR_INVALID_ARG
     assert bwd(ws=None) == vs.VIM_ERR_WORKSPACE
+
+
+def test_cross_ckpt_pair_rejects(vs):
+    lib, F = vs.lib, FAKE
+    fwd = lambda ckpt=F, ws=F: lib.vmamba_cross_scan4_ckpt(F, F, F, F, F, F, F, F, F, ckpt, 2, 8, 8, 64, 16,
+                                                            vs.VIM_BF16, 0, ws, 1 << 40, None, None)
+    assert fwd(ckpt=None) == vs.VIM_ERR_INVALID_ARG
+    assert fwd(ckpt=F + 4) == vs.VIM_ERR_INVALID_ARG
+    assert fwd(ws=None) == vs.VIM_ERR_WORKSPACE
+    bwd = lambda ckpt=F, ws=F: lib.vmamba_cross_scan4_bwd_ckpt(F, F, F, F, F, F, F, F, ckpt, F, F, F, F, F, F, F, F,
+                                                                F, 2, 8, 8, 64, 16, vs.VIM_BF16, 0, ws, 1 << 40, None)
+    assert bwd(ckpt=None) == vs.VIM_ERR_INVALID_ARG
+    assert bwd(ckpt=F + 4) == vs.VIM_ERR_INVALID_ARG
+    assert bwd(ws=None) == vs.VIM_ERR_WORKSPACE
+    assert lib.vmamba_cross_ckpt_bytes(2, 8, 8, 64, 16) == 2 * 2 * 2 * 2 * 16 * 64 * 4
+    assert lib.vmamba_cross_ckpt_bytes(0, 8, 8, 64, 16) == 0
+    assert vs.cross_ckpt_shape(2, 8, 8, 64, 16) == (2, 2, 2, 2, 16, 64)
 
 
 def test_bwd_ex_rejects(vs):

@@ -528,3 +528,33 @@ def test_conv_ckpt_pair(vs, case):
     assert torch.equal(y, y_plain)
     assert torch.isfinite(ck).all() and (ck[:, 0, 0] == 0).all() and (ck[:, -1, 1] == 0).all()
     check_conv(f"conv_bwd_ckpt_{case}", got, ref_conv(x, gate, zoh), dtype)
+
+
+# the training pair of the cross-scan
+CROSS_CKPT_CASES = [
+    # batch, H, W, C, N, dtype, generic_A, zoh
+    (1, 3, 5, 16, 16, torch.float32, False, False),
+    (1, 7, 40, 64, 16, torch.float32, True, False),    # several chunks, tiles across column ends
+    (2, 16, 16, 64, 16, torch.bfloat16, False, False),
+    (1, 20, 17, 32, 8, torch.float32, False, True),    # exact hold
+]
+
+
+@pytest.mark.parametrize("case", CROSS_CKPT_CASES, ids=lambda c: f"b{c[0]}_{c[1]}x{c[2]}_C{c[3]}_N{c[4]}_"
+                         f"{str(c[5])[6:]}{'_genA' if c[6] else ''}{'_zoh' if c[7] else ''}")
+def test_cross_ckpt_pair(vs, case):
+    batch, H, W, Ch, N, dtype, gen, zoh = case
+    x = cross_inputs(batch, H, W, Ch, N, dtype, seed=H * 19 + W, generic_A=gen)
+    c = lambda k: x[k].cuda()
+    ck = torch.full(vs.cross_ckpt_shape(batch, H, W, Ch, N), float("nan"), device="cuda")
+    y = vs.vmamba_cross_scan4(c("u"), c("delta"), c("z"), c("B"), c("C"), c("A"), c("D"), c("bias"), zoh=zoh,
+                              ckpt=ck)
+    y_plain = vs.vmamba_cross_scan4(c("u"), c("delta"), c("z"), c("B"), c("C"), c("A"), c("D"), c("bias"), zoh=zoh)
+    got = vs.vmamba_cross_scan4_bwd(c("u"), c("delta"), c("z"), c("B"), c("C"), c("A"), c("D"), c("bias"),
+                                    c("dout"), zoh=zoh, ckpt=ck)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_plain)
+    assert torch.isfinite(ck).all() and (ck[:, :, 0, 0] == 0).all() and (ck[:, :, -1, 1] == 0).all()
+    want = oracle.cross_scan4_bwd(x["u"], x["delta"], x["z"], x["B"], x["C"], x["A"], x["D"], x["bias"], x["dout"],
+                                  zoh=zoh)
+    check_all(f"cross_bwd_ckpt_{case}", got, want, dtype)

@@ -322,12 +322,18 @@ size_t vmamba_cross_scan4_bwd_workspace_bytes(int batch, int H, int W, int chann
     return bwd_plan(batch, L, channels, d_state, 1).total + 3 * round_up((size_t)batch * L * channels * 4);
 }
 
-vim_status vmamba_cross_scan4_bwd_ex(const void *u, const void *delta, const void *z, const void *B, const void *C,
-                                     const float *A, const float *D, const float *delta_bias, const void *dout,
-                                     void *du, void *ddelta, void *dz, float *dB, float *dC, float *dA, float *dD,
-                                     float *ddelta_bias, int batch, int H, int W, int channels, int d_state,
-                                     vim_dtype dt, unsigned flags, void *workspace, size_t workspace_bytes,
-                                     cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// the derivative of vmamba_cross_scan4; ckpt, or null: the forward pass's checkpoints
+// (vmamba_cross_scan4_ckpt, [2 pairs][batch][ceil(L/32)][2][N][C]), which replace each
+// pair's own forward summaries
+vim_status cross_bwd_impl(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                          const float *A, const float *D, const float *delta_bias, const void *dout, void *du,
+                          void *ddelta, void *dz, float *dB, float *dC, float *dA, float *dD, float *ddelta_bias,
+                          int batch, int H, int W, int channels, int d_state, vim_dtype dt, unsigned flags,
+                          void *workspace, size_t workspace_bytes, cudaStream_t stream, const float *ckpt) {
     if (flags & ~VIM_FLAG_ZOH_EXACT) return VIM_ERR_INVALID_ARG;
     const bool zoh = (flags & VIM_FLAG_ZOH_EXACT) != 0;
     if (H < 0 || W < 0) return VIM_ERR_INVALID_ARG;
@@ -380,7 +386,9 @@ vim_status vmamba_cross_scan4_bwd_ex(const void *u, const void *delta, const voi
         a.dB_part[1] = a.dB_part[0] + set_elems;
         a.dC_part[1] = a.dC_part[0] + set_elems;
         a.par = reinterpret_cast<float *>(ws + pl.off_par);
-        a.hin = reinterpret_cast<const float *>(ws + pl.off_hloc);
+        a.hin = ckpt ? ckpt + (size_t)pair * batch * pl.G * 2 * d_state * channels
+                     : reinterpret_cast<const float *>(ws + pl.off_hloc);
+        a.hin_given = ckpt ? 1 : 0;
         a.gloc = reinterpret_cast<float *>(ws + pl.off_gloc);
         a.gsum = reinterpret_cast<float *>(ws + pl.off_gsum);
         a.batch = batch; a.L = L; a.Di = channels; a.G = pl.G; a.nblk = pl.nblk; a.cl = pl.cl; a.ncol = pl.ncol;
@@ -416,6 +424,31 @@ vim_status vmamba_cross_scan4_bwd_ex(const void *u, const void *delta, const voi
                                                           nullptr);
     }
     return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+vim_status vmamba_cross_scan4_bwd_ex(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                                     const float *A, const float *D, const float *delta_bias, const void *dout,
+                                     void *du, void *ddelta, void *dz, float *dB, float *dC, float *dA, float *dD,
+                                     float *ddelta_bias, int batch, int H, int W, int channels, int d_state,
+                                     vim_dtype dt, unsigned flags, void *workspace, size_t workspace_bytes,
+                                     cudaStream_t stream) {
+    return cross_bwd_impl(u, delta, z, B, C, A, D, delta_bias, dout, du, ddelta, dz, dB, dC, dA, dD, ddelta_bias,
+                          batch, H, W, channels, d_state, dt, flags, workspace, workspace_bytes, stream, nullptr);
+}
+
+vim_status vmamba_cross_scan4_bwd_ckpt(const void *u, const void *delta, const void *z, const void *B,
+                                       const void *C, const float *A, const float *D, const float *delta_bias,
+                                       const float *ckpt, const void *dout, void *du, void *ddelta, void *dz,
+                                       float *dB, float *dC, float *dA, float *dD, float *ddelta_bias, int batch,
+                                       int H, int W, int channels, int d_state, vim_dtype dt, unsigned flags,
+                                       void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (batch > 0 && H > 0 && W > 0 && channels > 0 && (!ckpt || !aligned_to(ckpt, 8))) return VIM_ERR_INVALID_ARG;
+    return cross_bwd_impl(u, delta, z, B, C, A, D, delta_bias, dout, du, ddelta, dz, dB, dC, dA, dD, ddelta_bias,
+                          batch, H, W, channels, d_state, dt, flags, workspace, workspace_bytes, stream, ckpt);
 }
 
 vim_status vmamba_cross_scan4_bwd(const void *u, const void *delta, const void *z, const void *B, const void *C,

@@ -300,7 +300,8 @@ struct PairArgs {
     int carry_span;                 // consecutive chunks per pair_carry CTA (0 or 1: one)
     float *hck;                     // or null: the state entering every kCkTokens-token segment,
                                     // [batch][ceil(L/kCkTokens)][2][N][Di] fp32, in each direction's
-                                    // visiting order (the Vim scan, with or without its front)
+                                    // visiting order (the Vim scan, with or without its front, and
+                                    // each pair of the cross-scan, over the pair's steps)
 };
 constexpr int kCkTokens = 32;       // tokens per checkpoint segment (the derivative's chunk)
 
@@ -1140,7 +1141,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) pair_main(PairArgs p) {
         const int twice = 2 * s - (nT - 1);
         float *ypart = (twice == 0 && dir == 1) ? ymid + dl : ybuf + (size_t)j * kTile * kDC + dl;
         if (!prm.valid) return;
-        if constexpr (!DT && !PIN) {
+        if constexpr (!DT) {
             // the state entering a checkpoint segment: chunks start at multiples of
             // kCkTokens, so a segment is two tiles; the forward direction enters it at its
             // even tile, the backward one at its odd tile (or the chunk's last tile).  In

@@ -177,12 +177,18 @@ vim_status vim_scan_bidir(const void *u, const void *delta, const void *z, const
                                  d_inner, d_state, dt, workspace, workspace_bytes, stream, nullptr);
 }
 
-vim_status vmamba_cross_scan4_ex(const void *u, const void *delta, const void *z, const void *B,
-                                 const void *C, const float *A, const float *D, const float *delta_bias,
-                                 void *y, int batch, int H, int W, int channels, int d_state, vim_dtype dt,
-                                 unsigned flags, void *workspace, size_t workspace_bytes,
-                                 cudaStream_t stream, cudaEvent_t *events) {
+}  // extern "C"
+
+namespace {
+
+// vmamba_cross_scan4, and optionally each pair's states entering every checkpoint segment
+// (ckpt: [2 pairs][batch][ceil(L/32)][2][N][C], over the pair's steps)
+vim_status cross_impl(const void *u, const void *delta, const void *z, const void *B, const void *C, const float *A,
+                      const float *D, const float *delta_bias, void *y, int batch, int H, int W, int channels,
+                      int d_state, vim_dtype dt, unsigned flags, void *workspace, size_t workspace_bytes,
+                      cudaStream_t stream, cudaEvent_t *events, float *ckpt) {
     if (H < 0 || W < 0 || (flags & ~kKnownFlags)) return VIM_ERR_INVALID_ARG;
+    if (ckpt && reinterpret_cast<uintptr_t>(ckpt) % 8) return VIM_ERR_INVALID_ARG;
     if ((int64_t)H * W > INT32_MAX) return VIM_ERR_UNSUPPORTED;
     const int L = H * W;
     vim_status st = check_common(batch, L, channels, d_state, dt);
@@ -221,6 +227,8 @@ vim_status vmamba_cross_scan4_ex(const void *u, const void *delta, const void *z
         a.batch = batch; a.L = L; a.Di = channels; a.H = H; a.W = W;
         a.order = pair;               // pair 0: scans 1/2 (rows), pair 1: scans 3/4 (columns)
         a.hdiv = div_inv((unsigned)H);
+        if (ckpt)
+            a.hck = ckpt + (size_t)pair * batch * ((L + kCkTokens - 1) / kCkTokens) * 2 * d_state * channels;
         a.chunk = pl.chunk; a.G = pl.G;
         a.zoh = (flags & VIM_FLAG_ZOH_EXACT) ? 1 : 0;
         if (pl.G > 1) {
@@ -238,6 +246,34 @@ vim_status vmamba_cross_scan4_ex(const void *u, const void *delta, const void *z
         rc = launch_pair(a, d_state, dt, stream, events ? events + 1 + 3 * pair : nullptr);
     }
     return rc;
+}
+}  // namespace
+
+extern "C" {
+
+vim_status vmamba_cross_scan4_ex(const void *u, const void *delta, const void *z, const void *B,
+                                 const void *C, const float *A, const float *D, const float *delta_bias,
+                                 void *y, int batch, int H, int W, int channels, int d_state, vim_dtype dt,
+                                 unsigned flags, void *workspace, size_t workspace_bytes,
+                                 cudaStream_t stream, cudaEvent_t *events) {
+    return cross_impl(u, delta, z, B, C, A, D, delta_bias, y, batch, H, W, channels, d_state, dt, flags, workspace,
+                      workspace_bytes, stream, events, nullptr);
+}
+
+vim_status vmamba_cross_scan4_ckpt(const void *u, const void *delta, const void *z, const void *B, const void *C,
+                                   const float *A, const float *D, const float *delta_bias, void *y, float *ckpt,
+                                   int batch, int H, int W, int channels, int d_state, vim_dtype dt, unsigned flags,
+                                   void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                                   cudaEvent_t *events) {
+    if (batch > 0 && H > 0 && W > 0 && channels > 0 && !ckpt) return VIM_ERR_INVALID_ARG;
+    return cross_impl(u, delta, z, B, C, A, D, delta_bias, y, batch, H, W, channels, d_state, dt, flags, workspace,
+                      workspace_bytes, stream, events, ckpt);
+}
+
+size_t vmamba_cross_ckpt_bytes(int batch, int H, int W, int channels, int d_state) {
+    if (batch <= 0 || H <= 0 || W <= 0 || channels <= 0 || !supported_state(d_state)) return 0;
+    if ((int64_t)H * W > INT32_MAX) return 0;
+    return 2 * vim_scan_ckpt_bytes(batch, H * W, channels, d_state);
 }
 
 vim_status vmamba_cross_scan4_events(const void *u, const void *delta, const void *z,

@@ -100,6 +100,13 @@ lib.vim_scan_bidir_conv_ckpt.restype = _i
 lib.vim_scan_bidir_conv_bwd_ckpt.argtypes = (lib.vim_scan_bidir_conv_bwd_ex.argtypes[:11] + [_vp]
                                              + lib.vim_scan_bidir_conv_bwd_ex.argtypes[11:])
 lib.vim_scan_bidir_conv_bwd_ckpt.restype = _i
+# the training pair of the cross-scan
+lib.vmamba_cross_scan4_ckpt.argtypes = [_vp] * 10 + [_i, _i, _i, _i, _i, _i, _u, _vp, _sz, _vp, _vp]
+lib.vmamba_cross_scan4_ckpt.restype = _i
+lib.vmamba_cross_scan4_bwd_ckpt.argtypes = [_vp] * 18 + [_i, _i, _i, _i, _i, _i, _u, _vp, _sz, _vp]
+lib.vmamba_cross_scan4_bwd_ckpt.restype = _i
+lib.vmamba_cross_ckpt_bytes.argtypes = [_i, _i, _i, _i, _i]
+lib.vmamba_cross_ckpt_bytes.restype = _sz
 lib.vim_scan_conv_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
 lib.vim_scan_conv_bwd_workspace_bytes.restype = _sz
 lib.vim_block_scan_bwd.argtypes = [_vp] * 19 + [_i, _i, _i, _i, _i, _vp, _sz, _vp]
@@ -433,12 +440,14 @@ def vim_scan_bidir_conv_bwd(x, conv_w, conv_b, delta, z, B, C, A, D, delta_bias,
 
 
 def vmamba_cross_scan4_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, workspace=None, stream=None, out=None,
-                           zoh=False):
+                           zoh=False, ckpt=None):
     """Derivatives of vmamba_cross_scan4 (first-order Bbar, or with ``zoh`` the exact
     zero-order hold) for a loss whose derivative
     with respect to y is ``dout``; see include/vimscan.h.  Returns a dict: du, ddelta, dz
     (None without z) in the input dtype; dB, dC [4, batch, H*W, N], dA [4, C, N], dD and
     ddelta_bias [4, C] in fp32.  ``out`` may hold those tensors from an earlier call.
+    ``ckpt``: the checkpoints vmamba_cross_scan4(ckpt=...) wrote for the same inputs
+    (vmamba_cross_scan4_bwd_ckpt).
     """
     batch, H, W, Ch = u.shape
     N = B.shape[-1]
@@ -458,11 +467,18 @@ def vmamba_cross_scan4_bwd(u, delta, z, B, C, A, D, delta_bias, dout, *, workspa
         ("A", A, f32, (4, Ch, N)), ("D", D, f32, (4, Ch)), ("delta_bias", delta_bias, f32, (4, Ch)),
         ("dout", dout, io, act)] + _out_specs(out, io, act, bc, (4, Ch, N), (4, Ch)))
     ws, ws_bytes = _workspace(int(lib.vmamba_cross_scan4_bwd_workspace_bytes(batch, H, W, Ch, N)), workspace, dev)
-    fn = lib.vmamba_cross_scan4_bwd_ex if zoh else lib.vmamba_cross_scan4_bwd
-    flags = (VIM_FLAG_ZOH_EXACT,) if zoh else ()
-    st = fn(
-        *ptrs,
-        batch, H, W, Ch, N, _dtype_code(u), *flags, None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
+    if ckpt is not None:
+        (pk,) = _ptrs("vmamba_cross_scan4_bwd", u, [("ckpt", ckpt, f32, cross_ckpt_shape(batch, H, W, Ch, N))])
+        st = lib.vmamba_cross_scan4_bwd_ckpt(
+            *ptrs[:8], pk, *ptrs[8:], batch, H, W, Ch, N, _dtype_code(u), VIM_FLAG_ZOH_EXACT if zoh else 0,
+            None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
+    else:
+        fn = lib.vmamba_cross_scan4_bwd_ex if zoh else lib.vmamba_cross_scan4_bwd
+        flags = (VIM_FLAG_ZOH_EXACT,) if zoh else ()
+        st = fn(
+            *ptrs,
+            batch, H, W, Ch, N, _dtype_code(u), *flags, None if ws is None else ws.data_ptr(), ws_bytes,
+            _stream(stream))
     if st != VIM_OK:
         raise VimScanError(st, "vmamba_cross_scan4_bwd")
     return out
@@ -574,13 +590,21 @@ def vim_scan_bidir_noalloc(u, delta, z, B, C, A, D, delta_bias, *, y=None, bc_di
     return y
 
 
+def cross_ckpt_shape(batch, H, W, channels, d_state):
+    """Shape of the cross-scan's checkpoints (vmamba_cross_scan4(ckpt=...),
+    vmamba_cross_scan4_bwd(ckpt=...)): [2 pairs, batch, ceil(H*W / 32), 2, d_state, C]."""
+    return (2,) + ckpt_shape(batch, H * W, channels, d_state)
+
+
 def vmamba_cross_scan4(u, delta, z, B, C, A, D, delta_bias, *, y=None, workspace=None, stream=None,
-                       events=None, zoh=False):
+                       events=None, zoh=False, ckpt=None):
     """VMamba four-direction cross-scan with CS-Merge; see include/vimscan.h.
 
     u, delta, z: [batch, H, W, C]; B, C: [4, batch, H*W, d_state] by grid position;
     A: [4, C, d_state] fp32; D, delta_bias: [4, C] fp32.  Returns y [batch, H, W, C].
-    zoh=True takes the exact zero-order-hold Bbar (VIM_FLAG_ZOH_EXACT).
+    zoh=True takes the exact zero-order-hold Bbar (VIM_FLAG_ZOH_EXACT).  ``ckpt``, an fp32
+    tensor of cross_ckpt_shape(...), receives the states vmamba_cross_scan4_bwd(ckpt=...)
+    takes (vmamba_cross_scan4_ckpt).
     """
     batch, H, W, Ch = u.shape
     N = B.shape[-1]
@@ -597,7 +621,10 @@ def vmamba_cross_scan4(u, delta, z, B, C, A, D, delta_bias, *, y=None, workspace
     ws, ws_bytes = _workspace(vim_scan_workspace_bytes(1, batch, H, W, Ch, N), workspace, u.device)
     tail = (None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream))
     ev = None if events is None else _events(events)
-    if zoh:
+    if ckpt is not None:
+        (pk,) = _ptrs("vmamba_cross_scan4", u, [("ckpt", ckpt, f32, cross_ckpt_shape(batch, H, W, Ch, N))])
+        st = lib.vmamba_cross_scan4_ckpt(*args[:9], pk, *args[9:], VIM_FLAG_ZOH_EXACT if zoh else 0, *tail, ev)
+    elif zoh:
         st = lib.vmamba_cross_scan4_ex(*args, VIM_FLAG_ZOH_EXACT, *tail, ev)
     elif ev is None:
         st = lib.vmamba_cross_scan4(*args, *tail)
