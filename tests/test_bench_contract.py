@@ -62,3 +62,12 @@ def test_profiled_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
     (csrc / "bwd_kernels.cuh").write_bytes(b"// bwd v2\n")
     assert bench.profiled_traffic(w, bwd=True) is None             # the source changed since
     assert bench.profiled_traffic(w) == 123
+
+
+def test_mode_combinations_are_checked_before_any_gpu_work():
+    # modes that do not combine are refused with a message, on the host, before CUDA
+    for args, msg in ((["--block", "--ckpt"], "--ckpt applies"), (["--block", "--zoh"], "--block runs alone"),
+                      (["--workload", "vmamba_64x64_bf16", "--conv"], "--conv and --block apply")):
+        r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], capture_output=True, text=True,
+                           cwd=ROOT, timeout=120)
+        assert r.returncode != 0 and msg in r.stderr, (args, r.stderr[-300:])
