@@ -85,6 +85,35 @@ def test_block_small(vs, case):
     gates.gate(f"block_{case}", run(vs, p, gate), ref(p, gate), torch.bfloat16, norm_tol=TOL, elementwise=False)
 
 
+# Sequence ends at every offset within the projection's 16-row groups: the front's
+# outer taps meet the zero padding at t = 0 and t = L - 1, so those rows (and rows past
+# the data) are formed with masks, all other groups without.  (L 49: a group ends just
+# before the last row; L 48: a group ends on it; L 17: both ends in one group; L 100 with
+# no front: the unmasked copy of u.)
+EDGE_CASES = [
+    (2, 49, 64, 16, True),
+    (1, 48, 64, 16, True),
+    (3, 17, 64, 16, True),
+    (2, 161, 128, 16, True),
+    (1, 100, 64, 16, False),
+]
+
+
+@pytest.mark.parametrize("case", EDGE_CASES, ids=lambda c: f"b{c[0]}_L{c[1]}_D{c[2]}_N{c[3]}"
+                         f"{'_conv' if c[4] else ''}")
+def test_block_sequence_ends_per_token(vs, case):
+    """Each token's error against the oracle, normwise over its channels with the floor
+    sqrt(d_inner) rms(y): a token whose front took a wrong neighbour differs by O(1)
+    there, which the gate over the whole output could dilute."""
+    batch, L, Di, N, conv = case
+    p = block_inputs(batch, L, Di, N, seed=7 * L + Di, conv=conv)
+    y, r = gates.as_np(run(vs, p)), gates.as_np(ref(p))
+    floor = np.sqrt(Di) * np.sqrt(np.mean(r * r))
+    err = np.linalg.norm(y - r, axis=-1) / np.maximum(np.linalg.norm(r, axis=-1), floor)
+    worst = np.unravel_index(np.argmax(err), err.shape)
+    assert err.max() <= TOL, f"token (b, t) = {worst}: error {err.max():.3e} > {TOL:.0e}"
+
+
 def test_block_rejects_fp32(vs):
     p = block_inputs(1, 10, 16, 16, seed=1, conv=False)
     with pytest.raises(vs.VimScanError):

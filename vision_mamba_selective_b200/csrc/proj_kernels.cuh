@@ -17,6 +17,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <type_traits>
 
 #include "scan_kernels.cuh"
 
@@ -157,43 +158,57 @@ __global__ void __launch_bounds__(kProjThreads) xproj_kernel(ProjArgs p) {
             cbv = f2(p.conv_b[(size_t)dir * p.Di + d], p.conv_b[(size_t)dir * p.Di + d + 1]);
         }
         const int r0 = rg * 16;
-        int t = (m0 + r0) % p.L;                  // position of row r0 in its sequence
+        const int t = (m0 + r0) % p.L;            // position of row r0 in its sequence
         auto xrow = [&](int r) {                  // x of tile row r (-1 .. 64), channels d, d+1
             return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(xs + (r + 1) * LDU + 2 * cp));
         };
-        // sliding window over the rows, kept in registers (one shared-memory load per row)
-        float2 xm = CONV ? xrow(r0 - 1) : f2(0.f, 0.f), x0 = xrow(r0);
-#pragma unroll 4
-        for (int r = 0; r < 16; ++r) {
-            const int m = m0 + r0 + r;
-            float2 u = x0;
-            float2 xp = f2(0.f, 0.f);
-            if (CONV) {
-                xp = xrow(r0 + r + 1);
-                // neighbours outside the sequence are the convolution's zero padding
-                const float2 mm = t > 0 ? wm : f2(0.f, 0.f), mp = t < p.L - 1 ? wp : f2(0.f, 0.f);
-                const float2 v = fma2(mm, xm, fma2(wc, x0, fma2(mp, xp, cbv)));
+        // sliding window over the rows, kept in registers (one shared-memory load per row).
+        // MASK: the group reaches a sequence end (where the convolution's outer taps meet
+        // its zero padding) or the data's end, or the pair lies past d_inner; the other
+        // groups run without the per-row selects
+        auto form_rows = [&](auto mask) {
+            constexpr bool MASK = decltype(mask)::value;
+            int tt = t;
+            float2 xm = CONV ? xrow(r0 - 1) : f2(0.f, 0.f), x0 = xrow(r0);
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float2 u = x0;
+                float2 xp = f2(0.f, 0.f);
+                if (CONV) {
+                    xp = xrow(r0 + r + 1);
+                    float2 mm = wm, mp = wp;
+                    if constexpr (MASK) {   // neighbours outside the sequence are the zero padding
+                        if (tt == 0) mm = f2(0.f, 0.f);
+                        if (tt == p.L - 1) mp = f2(0.f, 0.f);
+                    }
+                    const float2 v = fma2(mm, xm, fma2(wc, x0, fma2(mp, xp, cbv)));
 #if VIMSCAN_PROJ_TANH
-                // silu(v) = v (1 + tanh(v/2)) / 2 with the MUFU tanh (relative error near
-                // 2^-11, below the bf16 rounding that u takes next)
-                const float2 hv = mul2(v, f2(0.5f, 0.5f));
-                u = fma2(hv, f2(tanh_approx(hv.x), tanh_approx(hv.y)), hv);
+                    // silu(v) = v (1 + tanh(v/2)) / 2 with the MUFU tanh (relative error near
+                    // 2^-11, below the bf16 rounding that u takes next)
+                    const float2 hv = mul2(v, f2(0.5f, 0.5f));
+                    u = fma2(hv, f2(tanh_approx(hv.x), tanh_approx(hv.y)), hv);
 #else
-                const float2 e = mul2(v, f2(-kLog2e, -kLog2e));
-                const float2 den = f2(1.0f + ex2(e.x), 1.0f + ex2(e.y));
-                u = mul2(v, f2(rcp(den.x), rcp(den.y)));          // silu(v) = v / (1 + e^-v)
+                    const float2 e = mul2(v, f2(-kLog2e, -kLog2e));
+                    const float2 den = f2(1.0f + ex2(e.x), 1.0f + ex2(e.y));
+                    u = mul2(v, f2(rcp(den.x), rcp(den.y)));          // silu(v) = v / (1 + e^-v)
 #endif
+                }
+                if constexpr (MASK) {
+                    if (m0 + r0 + r >= M || !dvalid) u = f2(0.f, 0.f);
+                    tt = tt + 1 == p.L ? 0 : tt + 1;
+                }
+                *reinterpret_cast<__nv_bfloat162 *>(&sU[r0 + r][2 * cp]) = __floats2bfloat162_rn(u.x, u.y);
+                if (CONV) {
+                    xm = x0;
+                    x0 = xp;
+                } else if (r + 1 < 16) {
+                    x0 = xrow(r0 + r + 1);
+                }
             }
-            if (m >= M || !dvalid) u = f2(0.f, 0.f);
-            *reinterpret_cast<__nv_bfloat162 *>(&sU[r0 + r][2 * cp]) = __floats2bfloat162_rn(u.x, u.y);
-            t = t + 1 == p.L ? 0 : t + 1;
-            if (CONV) {
-                xm = x0;
-                x0 = xp;
-            } else if (r + 1 < 16) {
-                x0 = xrow(r0 + r + 1);
-            }
-        }
+        };
+        // rows t .. t+15 of one sequence, none at its first or last position, all below M
+        if (dvalid && t > 0 && t + 16 < p.L && m0 + r0 + 16 <= M) form_rows(std::false_type{});
+        else form_rows(std::true_type{});
         __syncthreads();
         if (p.uo) {
             // the slice of u_k, 16 bytes at a time, for the scan (which then forms no front)
