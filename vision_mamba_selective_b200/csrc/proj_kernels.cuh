@@ -125,8 +125,26 @@ __global__ void __launch_bounds__(kProjThreads) xproj_kernel(ProjArgs p) {
         sW[(NO + li / p.Di) * LDW + li % p.Di] = __float2bfloat16_rn(0.0f);
 
     const int cp = lane, rg = warp;          // channel pair and row group of the u pass
+    // the pair's taps on x[t-1], x[t], x[t+1] and bias for the slice of step `st`, as
+    // (channel d, channel d+1); the backward pathway convolves the reversed sequence,
+    // which swaps the outer taps.  Loaded one step ahead, beside that step's x rows.
+    struct Taps { float2 wm, wc, wp, cb; };
+    auto taps_of = [&](int st) {
+        Taps tp{f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f), f2(0.f, 0.f)};
+        const int d = (st % nslice) * kProjK + 2 * cp;
+        if (CONV && d < p.Di) {
+            const float *wa = p.conv_w + ((size_t)dir * p.Di + d) * 3;
+            tp.wm = dir ? f2(wa[2], wa[5]) : f2(wa[0], wa[3]);
+            tp.wc = f2(wa[1], wa[4]);
+            tp.wp = dir ? f2(wa[0], wa[3]) : f2(wa[2], wa[5]);
+            tp.cb = f2(p.conv_b[(size_t)dir * p.Di + d], p.conv_b[(size_t)dir * p.Di + d + 1]);
+        }
+        return tp;
+    };
+    Taps next_taps = taps_of(0);
     float acc[NT8][4];
     for (int st = 0; st < nsteps; ++st) {
+        const Taps taps = next_taps;
         const int tile = blockIdx.y + (st / nslice) * gridDim.y, kc = (st % nslice) * kProjK;
         const int m0 = tile * kProjRows;
         if (kc == 0) {
@@ -137,6 +155,7 @@ __global__ void __launch_bounds__(kProjThreads) xproj_kernel(ProjArgs p) {
         }
         if (st + 1 < nsteps) {
             issue(st + 1, (st + 1) & 1);
+            next_taps = taps_of(st + 1);
             asm volatile("cp.async.wait_group 1;\n" ::);
         } else {
             cp_async_wait_all();
@@ -147,16 +166,7 @@ __global__ void __launch_bounds__(kProjThreads) xproj_kernel(ProjArgs p) {
         const __nv_bfloat16 *xs = sX + (st & 1) * XROWS * LDU;
         const int d = kc + 2 * cp;
         const bool dvalid = d < p.Di;            // d_inner is a multiple of 8: pairs are whole
-        // the pair's taps on x[t-1], x[t], x[t+1] and bias, as (channel d, channel d+1);
-        // the backward pathway convolves the reversed sequence, which swaps the outer taps
-        float2 wm = f2(0.f, 0.f), wc = f2(0.f, 0.f), wp = f2(0.f, 0.f), cbv = f2(0.f, 0.f);
-        if (CONV && dvalid) {
-            const float *wa = p.conv_w + ((size_t)dir * p.Di + d) * 3;
-            wm = dir ? f2(wa[2], wa[5]) : f2(wa[0], wa[3]);
-            wc = f2(wa[1], wa[4]);
-            wp = dir ? f2(wa[0], wa[3]) : f2(wa[2], wa[5]);
-            cbv = f2(p.conv_b[(size_t)dir * p.Di + d], p.conv_b[(size_t)dir * p.Di + d + 1]);
-        }
+        const float2 wm = taps.wm, wc = taps.wc, wp = taps.wp, cbv = taps.cb;
         const int r0 = rg * 16;
         const int t = (m0 + r0) % p.L;            // position of row r0 in its sequence
         auto xrow = [&](int r) {                  // x of tile row r (-1 .. 64), channels d, d+1
