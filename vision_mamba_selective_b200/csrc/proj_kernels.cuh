@@ -73,7 +73,7 @@ template <int N> struct ProjShape {
     }
 };
 
-// One CTA per pathway and group of 64-token tiles.  Wx[k] is staged once, transposed
+// One CTA per pathway and group of kProjRows-token tiles.  Wx[k] is staged once, transposed
 // ([output column][channel]).  The (tile, 64-channel slice) steps form one pipeline:
 // cp.async brings the next step's x rows (the tile plus one neighbour row on each side)
 // while the current step forms u -- thread (pair p, group q) takes channels 2p, 2p+1 of
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kProjThreads) xproj_kernel(ProjArgs p) {
     const int mytiles = blockIdx.y < ntiles ? (ntiles - 1 - blockIdx.y) / gridDim.y + 1 : 0;
     const int nsteps = mytiles * nslice;
 
-    // x rows m0-1 .. m0+64, channels kc .. kc+63 of step `st` into buffer `buf`; rows
+    // x rows m0-1 .. m0+kProjRows, channels kc .. kc+63 of step `st` into buffer `buf`; rows
     // outside 0..M-1 and channels past d_inner are zero-filled
     auto issue = [&](int st, int buf) {
         const int tile = blockIdx.y + (st / nslice) * gridDim.y, kc = (st % nslice) * kProjK;
@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kProjThreads) xproj_kernel(ProjArgs p) {
         const float2 wm = taps.wm, wc = taps.wc, wp = taps.wp, cbv = taps.cb;
         const int r0 = rg * 16;
         const int t = (m0 + r0) % p.L;            // position of row r0 in its sequence
-        auto xrow = [&](int r) {                  // x of tile row r (-1 .. 64), channels d, d+1
+        auto xrow = [&](int r) {                  // x of tile row r (-1 .. kProjRows), channels d, d+1
             return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(xs + (r + 1) * LDU + 2 * cp));
         };
         // sliding window over the rows, kept in registers (one shared-memory load per row).
