@@ -39,6 +39,9 @@ MUTANTS = {
     "conv_backward_taps_forward": ("int64_t s = reversed ? t + 1 - k : t + k - 1;",
                                    "int64_t s = t + k - 1;"),
     "conv_bias_dropped": ("double acc = cb[d];", "double acc = 0.0;"),
+    "conv_padding_crosses_sequences": ("if (s >= 0 && s < L) acc += w[d * 3 + k] * x[(b * L + s) * Di + d];",
+                                       "if (b * L + s >= 0 && b * L + s < batch * L)\n"
+                                       "                        acc += w[d * 3 + k] * x[(b * L + s) * Di + d];"),
     "conv_no_silu": ("u[(b * L + t) * Di + d] = silu(acc);", "u[(b * L + t) * Di + d] = acc;"),
     "conv_backward_uses_forward_weights": ("oracle_conv_silu(x, conv_w + (int64_t)Di * 3, conv_b + Di, ub",
                                            "oracle_conv_silu(x, conv_w, conv_b, ub"),
